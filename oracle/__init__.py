@@ -1,0 +1,215 @@
+"""fp64 CPU oracle for linear attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline /
+reference arm may import this package.  The CUDA library never does, and this
+package never imports the CUDA library: the two share nothing but the seeded
+input generators in ``synth``.
+
+The arithmetic lives in ``la_oracle.c`` (plain C, double precision); this module
+compiles it with gcc on first use (``build()``) and marshals numpy arrays.
+Every array is [B, H, T, D] float64, C-contiguous.
+
+Definitions (see the header of ``la_oracle.c`` for the derivations):
+  * ``bidir_fwd``  -- "Flash Bi-directional Linear Attention" README, intro:
+    non-causal linear attention with phi = elu + 1 and the norm term,
+    o_t = phi(q_t) S / (phi(q_t) . z + eps).
+  * ``simple_fwd`` -- same README, "Update" list (simple_la): identity phi,
+    no norm term.
+  * ``retention_fwd`` -- "flash-linear-attention" README, "Benchmarks" (RetNet)
+    and "Different forms of linear attention" (FusedRecurrent): causal, per-head
+    scalar decay, o_t = sum_{s<=t} gamma^(t-s) (q_t . k_s) v_s.
+  * the ``*_bwd`` functions are the hand-derived gradients of those forwards.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "la_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_default = None
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile la_oracle.c into liboracle.so (plain gcc, -O2, no fast-math, no FMA contraction)."""
+    stale = (not os.path.exists(out)) or os.path.getmtime(out) < os.path.getmtime(src)
+    if force or stale:
+        tmp = out + ".tmp%d" % os.getpid()
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+               "-ffp-contract=off", "-o", tmp, src, "-lm", "-lpthread"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, out)
+    return out
+
+
+def _bind(lib):
+    P = ctypes.c_void_p
+    L = ctypes.c_long
+    Dbl = ctypes.c_double
+    I = ctypes.c_int
+    lib.oracle_bidir_fwd.argtypes = [P, P, P, P, P, L, L, L, L, Dbl, I]
+    lib.oracle_simple_fwd.argtypes = [P, P, P, P, P, L, L, L, L, I]
+    lib.oracle_bidir_bwd.argtypes = [P, P, P, P, P, P, P, L, L, L, L, Dbl, I]
+    lib.oracle_simple_bwd.argtypes = [P, P, P, P, P, P, P, L, L, L, L, I]
+    lib.oracle_retention_fwd.argtypes = [P, P, P, P, P, L, L, L, L, I]
+    lib.oracle_retention_bwd.argtypes = [P, P, P, P, P, P, P, P, L, L, L, L, I]
+    for name in ("oracle_bidir_fwd", "oracle_simple_fwd", "oracle_bidir_bwd",
+                 "oracle_simple_bwd", "oracle_retention_fwd", "oracle_retention_bwd"):
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _default
+    with _lock:
+        if _default is None:
+            build()
+            _default = _bind(ctypes.CDLL(_LIB))
+    return _default
+
+
+def default_threads() -> int:
+    return os.cpu_count() or 1
+
+
+def _f64(a) -> np.ndarray:
+    """Widen to a C-contiguous float64 numpy array (exact for f16/bf16/f32)."""
+    if hasattr(a, "detach"):  # torch tensor (CPU); widen through float64 exactly
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _shape4(q):
+    if q.ndim != 4:
+        raise ValueError("expected a [B, H, T, D] array, got shape %r" % (q.shape,))
+    return q.shape
+
+
+def _check(rc, name):
+    if rc != 0:
+        raise RuntimeError("%s failed (rc=%d)" % (name, rc))
+
+
+class Oracle:
+    """The oracle's functions, bound to one compiled library (the default one, or a
+    variant compiled from an edited copy of la_oracle.c by the oracle's own tests)."""
+
+    def __init__(self, lib=None):
+        self._lib = lib if lib is not None else _load()
+
+    def bidir_fwd(self, q, k, v, eps: float = 1e-6, nthreads: int | None = None, want_state: bool = False):
+        """o = phi(q) S / (phi(q) . z + eps);  returns o (and state [B,H,D,D+1] if asked)."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, H, T, D = _shape4(q)
+        o = np.empty_like(q)
+        st = np.empty((B, H, D, D + 1)) if want_state else None
+        rc = self._lib.oracle_bidir_fwd(_p(q), _p(k), _p(v), _p(o), _p(st) if st is not None else None,
+                                      B, H, T, D, float(eps), nthreads or default_threads())
+        _check(rc, "oracle_bidir_fwd")
+        return (o, st) if want_state else o
+
+    def simple_fwd(self, q, k, v, nthreads: int | None = None, want_state: bool = False):
+        """o = q (k^T v): identity feature map, no norm term."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, H, T, D = _shape4(q)
+        o = np.empty_like(q)
+        st = np.empty((B, H, D, D + 1)) if want_state else None
+        rc = self._lib.oracle_simple_fwd(_p(q), _p(k), _p(v), _p(o), _p(st) if st is not None else None,
+                                       B, H, T, D, nthreads or default_threads())
+        _check(rc, "oracle_simple_fwd")
+        return (o, st) if want_state else o
+
+    def bidir_bwd(self, q, k, v, dout, eps: float = 1e-6, nthreads: int | None = None):
+        """Gradients (dq, dk, dv) of sum(o * dout) for bidir_fwd."""
+        q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(dout)
+        B, H, T, D = _shape4(q)
+        dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+        rc = self._lib.oracle_bidir_bwd(_p(q), _p(k), _p(v), _p(g), _p(dq), _p(dk), _p(dv),
+                                      B, H, T, D, float(eps), nthreads or default_threads())
+        _check(rc, "oracle_bidir_bwd")
+        return dq, dk, dv
+
+    def simple_bwd(self, q, k, v, dout, nthreads: int | None = None):
+        """Gradients (dq, dk, dv) of sum(o * dout) for simple_fwd."""
+        q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(dout)
+        B, H, T, D = _shape4(q)
+        dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+        rc = self._lib.oracle_simple_bwd(_p(q), _p(k), _p(v), _p(g), _p(dq), _p(dk), _p(dv),
+                                       B, H, T, D, nthreads or default_threads())
+        _check(rc, "oracle_simple_bwd")
+        return dq, dk, dv
+
+    def retention_fwd(self, q, k, v, gamma, nthreads: int | None = None):
+        """o_t = sum_{s<=t} gamma_h^(t-s) (q_t . k_s) v_s, recurrent form; gamma is [H]."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, H, T, D = _shape4(q)
+        gm = _f64(gamma).reshape(-1)
+        if gm.shape[0] != H:
+            raise ValueError("gamma must have H=%d entries" % H)
+        o = np.empty_like(q)
+        rc = self._lib.oracle_retention_fwd(_p(q), _p(k), _p(v), _p(gm), _p(o), B, H, T, D,
+                                          nthreads or default_threads())
+        _check(rc, "oracle_retention_fwd")
+        return o
+
+    def retention_bwd(self, q, k, v, dout, gamma, nthreads: int | None = None):
+        """Gradients (dq, dk, dv) of sum(o * dout) for retention_fwd."""
+        q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(dout)
+        B, H, T, D = _shape4(q)
+        gm = _f64(gamma).reshape(-1)
+        if gm.shape[0] != H:
+            raise ValueError("gamma must have H=%d entries" % H)
+        dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+        rc = self._lib.oracle_retention_bwd(_p(q), _p(k), _p(v), _p(g), _p(gm), _p(dq), _p(dk), _p(dv),
+                                          B, H, T, D, nthreads or default_threads())
+        _check(rc, "oracle_retention_bwd")
+        return dq, dk, dv
+
+
+_inst = None
+
+
+def _instance() -> Oracle:
+    global _inst
+    if _inst is None:
+        _inst = Oracle()
+    return _inst
+
+
+def load_variant(path: str) -> Oracle:
+    """Bind an Oracle to another compiled copy of la_oracle.c (used by the oracle's tests)."""
+    return Oracle(_bind(ctypes.CDLL(path)))
+
+
+def bidir_fwd(*a, **kw):
+    return _instance().bidir_fwd(*a, **kw)
+
+
+def simple_fwd(*a, **kw):
+    return _instance().simple_fwd(*a, **kw)
+
+
+def bidir_bwd(*a, **kw):
+    return _instance().bidir_bwd(*a, **kw)
+
+
+def simple_bwd(*a, **kw):
+    return _instance().simple_bwd(*a, **kw)
+
+
+def retention_fwd(*a, **kw):
+    return _instance().retention_fwd(*a, **kw)
+
+
+def retention_bwd(*a, **kw):
+    return _instance().retention_bwd(*a, **kw)

@@ -1,0 +1,355 @@
+/*
+ * la_oracle.c -- plain, slow, fp64 CPU oracle for linear attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline / reference arm use it.  It shares no code, header, table or
+ * helper with the CUDA library; it sees the same (already rounded) input
+ * values, widened exactly to double.
+ *
+ * Sources (web pages on the subject):
+ *  - "Flash Bi-directional Linear Attention" README (fla-org), intro and
+ *    "Update" list: bidirectional (non-causal) linear attention `linear_attn`
+ *    with a norm term, and `simple_la`, the same without the norm term.
+ *  - "flash-linear-attention" README (sustcsonglin), "Benchmarks" (RetNet,
+ *    i.e. retention) and "Different forms of linear attention"
+ *    (Parallel / FusedRecurrent / FusedChunk / ParallelChunk).
+ *
+ * The pages name the operations but print no formulas; the definitions used
+ * here are the plain readings (every one is listed in the design notes):
+ *
+ *   phi(x)  = elu(x) + 1  = x + 1 (x > 0),  exp(x) (x <= 0)
+ *   bidir:   S = sum_s phi(k_s)^T v_s (D x D),  z = sum_s phi(k_s) (D)
+ *            o_t = phi(q_t) S / (phi(q_t) . z + eps)
+ *   simple:  o_t = q_t (sum_s k_s^T v_s)            (identity phi, no norm)
+ *   retention (causal, per-head scalar decay gamma_h):
+ *            o_t = sum_{s<=t} gamma^(t-s) (q_t . k_s) v_s
+ *            computed in the recurrent ("FusedRecurrent") form
+ *            S_t = gamma S_{t-1} + k_t^T v_t,  o_t = q_t S_t.
+ *
+ * The backward formulas are derived by hand from those definitions (chain
+ * rule, written out next to each function).  Every function works on one
+ * (b,h) head at a time; heads are independent and are spread over
+ * `nthreads` POSIX threads with a fixed head->thread assignment, so the
+ * result does not depend on the thread count.
+ *
+ * Layout: every tensor is contiguous [B, H, T, D] (row-major, D fastest).
+ * The optional bidir/simple `state` output is [B, H, D, D+1]: row i holds
+ * S[i][0..D-1] followed by z[i] (z = 0 for simple).
+ *
+ * Return value: 0 on success, -1 on a bad argument or out of memory.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------- phi -- */
+
+/* elu(x) + 1 with elu's alpha = 1.  For x <= 0, elu(x) + 1 = exp(x) - 1 + 1
+ * = exp(x); writing exp(x) directly avoids a cancellation. */
+static double phi(double x) { return x > 0.0 ? x + 1.0 : exp(x); }
+
+/* d/dx (elu(x) + 1): 1 for x > 0, exp(x) for x <= 0 (continuous at 0). */
+static double dphi(double x) { return x > 0.0 ? 1.0 : exp(x); }
+
+/* ------------------------------------------------------- head threading -- */
+
+typedef struct {
+    const double *q, *k, *v, *g;   /* g = upstream gradient dO (bwd only) */
+    double *o, *state, *dq, *dk, *dv;
+    const double *gamma;           /* [H] (retention only) */
+    long B, H, T, D;
+    double eps;
+    int use_phi, use_norm;
+    int status;
+} job_t;
+
+typedef void (*head_fn)(job_t *job, long bh, double *scratch);
+
+typedef struct {
+    job_t *job;
+    head_fn fn;
+    long first, stride, nheads;
+    size_t scratch_doubles;
+    int failed;
+} worker_t;
+
+static void *worker_main(void *arg) {
+    worker_t *w = (worker_t *)arg;
+    double *scratch = (double *)malloc(w->scratch_doubles * sizeof(double));
+    if (!scratch) { w->failed = 1; return NULL; }
+    for (long bh = w->first; bh < w->nheads; bh += w->stride) w->fn(w->job, bh, scratch);
+    free(scratch);
+    return NULL;
+}
+
+/* Run fn over all B*H heads on nthreads threads (head bh -> thread bh % n). */
+static int for_each_head(job_t *job, head_fn fn, size_t scratch_doubles, int nthreads) {
+    long nheads = job->B * job->H;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > nheads) nthreads = (int)(nheads > 0 ? nheads : 1);
+    worker_t *ws = (worker_t *)calloc((size_t)nthreads, sizeof(worker_t));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!ws || !th) { free(ws); free(th); return -1; }
+    int rc = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        ws[i].job = job; ws[i].fn = fn; ws[i].first = i; ws[i].stride = nthreads;
+        ws[i].nheads = nheads; ws[i].scratch_doubles = scratch_doubles; ws[i].failed = 0;
+    }
+    int started = 0;
+    for (int i = 1; i < nthreads; ++i) {
+        if (pthread_create(&th[i], NULL, worker_main, &ws[i]) != 0) { ws[i].failed = 2; continue; }
+        ++started;
+    }
+    worker_main(&ws[0]);
+    for (int i = 1; i < nthreads; ++i)
+        if (ws[i].failed != 2) pthread_join(th[i], NULL);
+    for (int i = 0; i < nthreads; ++i) {
+        if (ws[i].failed == 2) worker_main(&ws[i]);   /* thread could not start: run inline */
+        if (ws[i].failed == 1) rc = -1;
+    }
+    (void)started;
+    free(ws); free(th);
+    return rc;
+}
+
+static int check_dims(long B, long H, long T, long D) {
+    return (B >= 1 && H >= 1 && T >= 0 && D >= 1) ? 0 : -1;
+}
+
+/* ------------------------------------------- bidir / simple: forward ---- */
+
+/* One head of the state form:
+ *   S[i][j] = sum_s f(k_s)[i] v_s[j],   z[i] = sum_s f(k_s)[i]
+ *   u_t[j]  = sum_i f(q_t)[i] S[i][j],  n_t = f(q_t) . z + eps
+ *   o_t     = u_t / n_t        (norm on)      or   o_t = u_t  (norm off)
+ * with f = phi (bidir) or the identity (simple). */
+static void state_fwd_head(job_t *jb, long bh, double *scratch) {
+    const long T = jb->T, D = jb->D;
+    const double *q = jb->q + bh * T * D, *k = jb->k + bh * T * D, *v = jb->v + bh * T * D;
+    double *o = jb->o + bh * T * D;
+    double *S = scratch;            /* D*D */
+    double *z = S + D * D;          /* D */
+    double *fq = z + D;             /* D */
+    memset(S, 0, (size_t)(D * D + D) * sizeof(double));
+    for (long s = 0; s < T; ++s) {
+        for (long i = 0; i < D; ++i) {
+            double fk = jb->use_phi ? phi(k[s * D + i]) : k[s * D + i];
+            z[i] += fk;
+            for (long j = 0; j < D; ++j) S[i * D + j] += fk * v[s * D + j];
+        }
+    }
+    for (long t = 0; t < T; ++t) {
+        double n = jb->eps;
+        for (long i = 0; i < D; ++i) {
+            fq[i] = jb->use_phi ? phi(q[t * D + i]) : q[t * D + i];
+            n += fq[i] * z[i];
+        }
+        for (long j = 0; j < D; ++j) {
+            double u = 0.0;
+            for (long i = 0; i < D; ++i) u += fq[i] * S[i * D + j];
+            o[t * D + j] = jb->use_norm ? u / n : u;
+        }
+    }
+    if (jb->state) {
+        double *st = jb->state + bh * D * (D + 1);
+        for (long i = 0; i < D; ++i) {
+            for (long j = 0; j < D; ++j) st[i * (D + 1) + j] = S[i * D + j];
+            st[i * (D + 1) + D] = jb->use_norm ? z[i] : 0.0;
+        }
+    }
+}
+
+/* ------------------------------------------ bidir / simple: backward ---- */
+
+/* One head.  With g_t = dL/do_t and the forward quantities above:
+ *   norm on:   dL/du_t = g_t / n_t,
+ *              dL/dn_t = -(g_t . u_t) / n_t^2 = -(g_t . o_t) / n_t
+ *              dfq_t   = (g_t S^T - (g_t . o_t) z) / n_t
+ *              dS      = sum_t f(q_t)^T (g_t / n_t)
+ *              dz      = -sum_t f(q_t) (g_t . o_t) / n_t
+ *   norm off:  dfq_t = g_t S^T,  dS = sum_t q_t^T g_t,  dz = 0
+ *   then       dfk_s = v_s dS^T + dz       (dfk_s[i] = sum_j dS[i][j] v_s[j] + dz[i])
+ *              dv_s  = f(k_s) dS           (dv_s[j]  = sum_i f(k_s)[i] dS[i][j])
+ *   and        dq = dfq * f'(q),  dk = dfk * f'(k)   (f' = dphi or 1). */
+static void state_bwd_head(job_t *jb, long bh, double *scratch) {
+    const long T = jb->T, D = jb->D;
+    const long off = bh * T * D;
+    const double *q = jb->q + off, *k = jb->k + off, *v = jb->v + off, *g = jb->g + off;
+    double *dq = jb->dq + off, *dk = jb->dk + off, *dv = jb->dv + off;
+    double *S = scratch, *z = S + D * D, *dS = z + D, *dz = dS + D * D, *fq = dz + D, *u = fq + D;
+    memset(S, 0, (size_t)(2 * D * D + 2 * D) * sizeof(double));
+    /* recompute S, z */
+    for (long s = 0; s < T; ++s) {
+        for (long i = 0; i < D; ++i) {
+            double fk = jb->use_phi ? phi(k[s * D + i]) : k[s * D + i];
+            z[i] += fk;
+            for (long j = 0; j < D; ++j) S[i * D + j] += fk * v[s * D + j];
+        }
+    }
+    /* query side: dq, and accumulate dS, dz */
+    for (long t = 0; t < T; ++t) {
+        double n = jb->eps;
+        for (long i = 0; i < D; ++i) {
+            fq[i] = jb->use_phi ? phi(q[t * D + i]) : q[t * D + i];
+            n += fq[i] * z[i];
+        }
+        double go = 0.0;   /* g_t . o_t */
+        for (long j = 0; j < D; ++j) {
+            double uj = 0.0;
+            for (long i = 0; i < D; ++i) uj += fq[i] * S[i * D + j];
+            u[j] = uj;
+            double oj = jb->use_norm ? uj / n : uj;
+            go += g[t * D + j] * oj;
+        }
+        for (long i = 0; i < D; ++i) {
+            double gs = 0.0;   /* (g_t S^T)[i] = sum_j g_t[j] S[i][j] */
+            for (long j = 0; j < D; ++j) gs += g[t * D + j] * S[i * D + j];
+            double dfq = jb->use_norm ? (gs - go * z[i]) / n : gs;
+            double fp = jb->use_phi ? dphi(q[t * D + i]) : 1.0;
+            dq[t * D + i] = dfq * fp;
+            for (long j = 0; j < D; ++j)
+                dS[i * D + j] += fq[i] * (jb->use_norm ? g[t * D + j] / n : g[t * D + j]);
+            if (jb->use_norm) dz[i] -= fq[i] * go / n;
+        }
+    }
+    /* key/value side */
+    for (long s = 0; s < T; ++s) {
+        for (long i = 0; i < D; ++i) {
+            double a = dz[i];
+            for (long j = 0; j < D; ++j) a += dS[i * D + j] * v[s * D + j];
+            double fp = jb->use_phi ? dphi(k[s * D + i]) : 1.0;
+            dk[s * D + i] = a * fp;
+        }
+        for (long j = 0; j < D; ++j) {
+            double a = 0.0;
+            for (long i = 0; i < D; ++i) {
+                double fk = jb->use_phi ? phi(k[s * D + i]) : k[s * D + i];
+                a += fk * dS[i * D + j];
+            }
+            dv[s * D + j] = a;
+        }
+    }
+}
+
+int oracle_bidir_fwd(const double *q, const double *k, const double *v, double *o, double *state,
+                     long B, long H, long T, long D, double eps, int nthreads) {
+    if (check_dims(B, H, T, D) || !q || !k || !v || !o) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.o = o; jb.state = state;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D; jb.eps = eps; jb.use_phi = 1; jb.use_norm = 1;
+    return for_each_head(&jb, state_fwd_head, (size_t)(D * D + 2 * D), nthreads);
+}
+
+int oracle_simple_fwd(const double *q, const double *k, const double *v, double *o, double *state,
+                      long B, long H, long T, long D, int nthreads) {
+    if (check_dims(B, H, T, D) || !q || !k || !v || !o) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.o = o; jb.state = state;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D; jb.eps = 0.0; jb.use_phi = 0; jb.use_norm = 0;
+    return for_each_head(&jb, state_fwd_head, (size_t)(D * D + 2 * D), nthreads);
+}
+
+int oracle_bidir_bwd(const double *q, const double *k, const double *v, const double *dout,
+                     double *dq, double *dk, double *dv,
+                     long B, long H, long T, long D, double eps, int nthreads) {
+    if (check_dims(B, H, T, D) || !q || !k || !v || !dout || !dq || !dk || !dv) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.g = dout; jb.dq = dq; jb.dk = dk; jb.dv = dv;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D; jb.eps = eps; jb.use_phi = 1; jb.use_norm = 1;
+    return for_each_head(&jb, state_bwd_head, (size_t)(2 * D * D + 4 * D), nthreads);
+}
+
+int oracle_simple_bwd(const double *q, const double *k, const double *v, const double *dout,
+                      double *dq, double *dk, double *dv,
+                      long B, long H, long T, long D, int nthreads) {
+    if (check_dims(B, H, T, D) || !q || !k || !v || !dout || !dq || !dk || !dv) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.g = dout; jb.dq = dq; jb.dk = dk; jb.dv = dv;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D; jb.eps = 0.0; jb.use_phi = 0; jb.use_norm = 0;
+    return for_each_head(&jb, state_bwd_head, (size_t)(2 * D * D + 4 * D), nthreads);
+}
+
+/* ------------------------------------------------ retention (recurrent) -- */
+
+/* Forward, one head, the recurrent form:
+ *   S_t = gamma S_{t-1} + k_t^T v_t   (S_{-1} = 0),   o_t = q_t S_t. */
+static void retention_fwd_head(job_t *jb, long bh, double *scratch) {
+    const long T = jb->T, D = jb->D;
+    const double gamma = jb->gamma[bh % jb->H];
+    const long off = bh * T * D;
+    const double *q = jb->q + off, *k = jb->k + off, *v = jb->v + off;
+    double *o = jb->o + off;
+    double *S = scratch;
+    memset(S, 0, (size_t)(D * D) * sizeof(double));
+    for (long t = 0; t < T; ++t) {
+        for (long i = 0; i < D; ++i)
+            for (long j = 0; j < D; ++j)
+                S[i * D + j] = gamma * S[i * D + j] + k[t * D + i] * v[t * D + j];
+        for (long j = 0; j < D; ++j) {
+            double a = 0.0;
+            for (long i = 0; i < D; ++i) a += q[t * D + i] * S[i * D + j];
+            o[t * D + j] = a;
+        }
+    }
+}
+
+/* Backward, one head.
+ *   dq_t[i] = sum_j S_t[i][j] g_t[j]                        (forward sweep)
+ *   R_t     = gamma R_{t+1} + q_t^T g_t   (R_T = 0)          (reverse sweep)
+ *             i.e. R_s = sum_{t>=s} gamma^(t-s) q_t^T g_t
+ *   dk_s[i] = sum_j R_s[i][j] v_s[j],   dv_s[j] = sum_i k_s[i] R_s[i][j]. */
+static void retention_bwd_head(job_t *jb, long bh, double *scratch) {
+    const long T = jb->T, D = jb->D;
+    const double gamma = jb->gamma[bh % jb->H];
+    const long off = bh * T * D;
+    const double *q = jb->q + off, *k = jb->k + off, *v = jb->v + off, *g = jb->g + off;
+    double *dq = jb->dq + off, *dk = jb->dk + off, *dv = jb->dv + off;
+    double *S = scratch, *R = S + D * D;
+    memset(S, 0, (size_t)(2 * D * D) * sizeof(double));
+    for (long t = 0; t < T; ++t) {
+        for (long i = 0; i < D; ++i)
+            for (long j = 0; j < D; ++j)
+                S[i * D + j] = gamma * S[i * D + j] + k[t * D + i] * v[t * D + j];
+        for (long i = 0; i < D; ++i) {
+            double a = 0.0;
+            for (long j = 0; j < D; ++j) a += S[i * D + j] * g[t * D + j];
+            dq[t * D + i] = a;
+        }
+    }
+    for (long s = T - 1; s >= 0; --s) {
+        for (long i = 0; i < D; ++i)
+            for (long j = 0; j < D; ++j)
+                R[i * D + j] = gamma * R[i * D + j] + q[s * D + i] * g[s * D + j];
+        for (long i = 0; i < D; ++i) {
+            double a = 0.0;
+            for (long j = 0; j < D; ++j) a += R[i * D + j] * v[s * D + j];
+            dk[s * D + i] = a;
+        }
+        for (long j = 0; j < D; ++j) {
+            double a = 0.0;
+            for (long i = 0; i < D; ++i) a += k[s * D + i] * R[i * D + j];
+            dv[s * D + j] = a;
+        }
+    }
+}
+
+int oracle_retention_fwd(const double *q, const double *k, const double *v, const double *gamma,
+                         double *o, long B, long H, long T, long D, int nthreads) {
+    if (check_dims(B, H, T, D) || !q || !k || !v || !gamma || !o) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.gamma = gamma; jb.o = o;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D;
+    return for_each_head(&jb, retention_fwd_head, (size_t)(D * D), nthreads);
+}
+
+int oracle_retention_bwd(const double *q, const double *k, const double *v, const double *dout,
+                         const double *gamma, double *dq, double *dk, double *dv,
+                         long B, long H, long T, long D, int nthreads) {
+    if (check_dims(B, H, T, D) || !q || !k || !v || !dout || !gamma || !dq || !dk || !dv) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.g = dout; jb.gamma = gamma; jb.dq = dq; jb.dk = dk; jb.dv = dv;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D;
+    return for_each_head(&jb, retention_bwd_head, (size_t)(2 * D * D), nthreads);
+}

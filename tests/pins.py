@@ -1,0 +1,302 @@
+"""Pins for the fp64 oracle: checks against facts that do not come from the oracle itself.
+
+Each check takes an ``oracle.Oracle`` instance and raises AssertionError on a
+mismatch, so the same checks run against the real oracle (test_oracle_pins.py)
+and against deliberately broken copies of it (test_oracle_mutations.py, which
+shows that a dropped term, a wrong sign, index or transposed operand fails at
+least one of them).
+
+The facts used:
+  * hand-worked examples (tests/golden/hand_examples.json);
+  * brute force on tiny inputs in the pairwise ("Parallel", O(T^2)) form, a
+    different computation from the oracle's state / recurrent forms;
+  * closed forms: all-zero q,k (phi = 1 -> plain mean), inputs whose feature
+    values are 0.5 / 1 / 2 (weighted mean), V = 1 with eps = 0 (output 1),
+    gamma = 1 (prefix sums), gamma -> 0 (diagonal only);
+  * invariances: permutation of tokens, linearity in V, per-head independence,
+    thread-count independence;
+  * gradients: central finite differences of the oracle's forward, and torch
+    autograd through an independently written pairwise form in float64.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "hand_examples.json")
+
+
+def _close(a, b, rtol=1e-12, atol=1e-12, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    if a.shape != b.shape:
+        raise AssertionError("%s: shape %r vs %r" % (what, a.shape, b.shape))
+    err = np.abs(a - b)
+    lim = atol + rtol * np.abs(b)
+    if not np.all(err <= lim):
+        i = int(np.argmax(err - lim))
+        raise AssertionError("%s: max excess at flat index %d: got %r want %r" % (
+            what, i, a.reshape(-1)[i], b.reshape(-1)[i]))
+
+
+def _feature(x):
+    """phi = elu + 1, written independently of the oracle (numpy)."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+
+
+def _rand(shape, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal(shape) * scale
+
+
+def _as4(a):
+    a = np.asarray(a, dtype=np.float64)
+    return a.reshape(1, 1, *a.shape)
+
+
+def _parse(x):
+    if isinstance(x, list):
+        return [_parse(e) for e in x]
+    if isinstance(x, str):
+        return {"-ln2": -math.log(2.0), "ln2": math.log(2.0)}[x]
+    return float(x)
+
+
+# ------------------------------------------------------------------ golden --
+
+def check_golden(orc):
+    cases = json.load(open(GOLDEN))["cases"]
+    for c in cases:
+        q, k, v = (_as4(_parse(c[n])) for n in ("q", "k", "v"))
+        if c["op"] == "bidir":
+            o = orc.bidir_fwd(q, k, v, eps=c["eps"])
+        elif c["op"] == "simple":
+            o = orc.simple_fwd(q, k, v)
+        else:
+            o = orc.retention_fwd(q, k, v, np.array([c["gamma"]]))
+        _close(o[0, 0], _parse(c["o"]), what=c["name"] + " o")
+        if "do" in c:
+            g = _as4(_parse(c["do"]))
+            if c["op"] == "bidir":
+                grads = orc.bidir_bwd(q, k, v, g, eps=c["eps"])
+            elif c["op"] == "simple":
+                grads = orc.simple_bwd(q, k, v, g)
+            else:
+                grads = orc.retention_bwd(q, k, v, g, np.array([c["gamma"]]))
+            for name, got in zip(("dq", "dk", "dv"), grads):
+                _close(got[0, 0], _parse(c[name]), what=c["name"] + " " + name)
+
+
+# ------------------------------------------------------------- brute force --
+
+def brute_bidir(q, k, v, eps):
+    """Pairwise form: o_t = sum_s a_ts v_s / (sum_s a_ts + eps), a_ts = phi(q_t).phi(k_s)."""
+    a = np.einsum("bhti,bhsi->bhts", _feature(q), _feature(k))
+    return np.einsum("bhts,bhsj->bhtj", a, v) / (a.sum(-1, keepdims=True) + eps)
+
+
+def brute_simple(q, k, v):
+    a = np.einsum("bhti,bhsi->bhts", q, k)
+    return np.einsum("bhts,bhsj->bhtj", a, v)
+
+
+def brute_retention(q, k, v, gamma):
+    """Pairwise causal form with an explicit decay matrix gamma^(t-s) [t >= s]."""
+    B, H, T, D = q.shape
+    t = np.arange(T)
+    diff = t[:, None] - t[None, :]
+    out = np.empty_like(q)
+    for h in range(H):
+        m = np.where(diff >= 0, np.power(float(gamma[h]), np.maximum(diff, 0).astype(np.float64)), 0.0)
+        a = np.einsum("bti,bsi->bts", q[:, h], k[:, h]) * m
+        out[:, h] = np.einsum("bts,bsj->btj", a, v[:, h])
+    return out
+
+
+def check_brute(orc):
+    B, H, T, D = 2, 3, 13, 5
+    q, k, v = _rand((B, H, T, D), 1), _rand((B, H, T, D), 2), _rand((B, H, T, D), 3)
+    _close(orc.bidir_fwd(q, k, v, eps=1e-3), brute_bidir(q, k, v, 1e-3), rtol=1e-11, atol=1e-13,
+           what="bidir vs pairwise")
+    _close(orc.simple_fwd(q, k, v), brute_simple(q, k, v), rtol=1e-11, atol=1e-12,
+           what="simple vs pairwise")
+    gam = np.array([0.5, 0.9, 0.999])
+    _close(orc.retention_fwd(q, k, v, gam), brute_retention(q, k, v, gam), rtol=1e-11, atol=1e-12,
+           what="retention vs pairwise")
+
+
+# ------------------------------------------------------------ closed forms --
+
+def check_closed_forms(orc):
+    T, D = 11, 4
+    v = _rand((1, 1, T, D), 7)
+    # all-zero q, k: phi = 1 everywhere, every weight equal -> o_t = D sum_s v_s / (T D + eps)
+    z = np.zeros((1, 1, T, D))
+    eps = 0.3
+    want = np.broadcast_to(v.sum(2, keepdims=True) * D / (T * D + eps), v.shape)
+    _close(orc.bidir_fwd(z, z, v, eps=eps), want, what="phi(0)=1 mean")
+    # per-token feature values 0.5 / 1 / 2 (k = -ln2 / 0 / 1), q = 0, eps = 0 -> weighted mean
+    kv = np.array([-math.log(2.0), 0.0, 1.0])[np.arange(T) % 3]
+    w = np.array([0.5, 1.0, 2.0])[np.arange(T) % 3]
+    k = np.broadcast_to(kv[None, None, :, None], (1, 1, T, D)).copy()
+    want = np.broadcast_to((w[:, None] * v[0, 0]).sum(0) / w.sum(), (1, 1, T, D))
+    _close(orc.bidir_fwd(z, k, v, eps=0.0), want, what="weighted mean (phi = 0.5/1/2)")
+    # V = 1 and eps = 0: every output is exactly 1 (numerator and denominator coincide)
+    q, k = _rand((2, 2, T, D), 8), _rand((2, 2, T, D), 9)
+    _close(orc.bidir_fwd(q, k, np.ones((2, 2, T, D)), eps=0.0), np.ones((2, 2, T, D)),
+           rtol=1e-14, atol=1e-14, what="V=1 identity")
+    # V = 1 with eps > 0 stays strictly below 1
+    o = orc.bidir_fwd(q, k, np.ones((2, 2, T, D)), eps=0.5)
+    if not np.all(o < 1.0):
+        raise AssertionError("V=1 with eps>0 must give o < 1")
+    # simple_la with q = e_a, k = e_b one-hot rows: o_t = sum_{s: k_s = e_a} v_s
+    qs = np.zeros((1, 1, T, D)); qs[..., 0] = 1.0
+    ks = np.zeros((1, 1, T, D)); ks[0, 0, ::2, 0] = 1.0; ks[0, 0, 1::2, 1] = 1.0
+    want = np.broadcast_to(v[0, 0, ::2].sum(0), (1, 1, T, D))
+    _close(orc.simple_fwd(qs, ks, v), want, what="simple one-hot selection")
+    # retention, gamma = 1: o_t = q_t (sum_{s<=t} k_s^T v_s)  (prefix sums)
+    q, k = _rand((1, 1, T, D), 10), _rand((1, 1, T, D), 11)
+    pref = np.cumsum(np.einsum("ti,tj->tij", k[0, 0], v[0, 0]), axis=0)
+    want = np.einsum("ti,tij->tj", q[0, 0], pref)[None, None]
+    _close(orc.retention_fwd(q, k, v, np.array([1.0])), want, rtol=1e-12, atol=1e-12, what="gamma=1 prefix")
+    # retention, gamma -> 0: only the diagonal survives, o_t = (q_t . k_t) v_t
+    want = ((q * k).sum(-1, keepdims=True) * v)
+    _close(orc.retention_fwd(q, k, v, np.array([1e-30])), want, rtol=1e-12, atol=1e-12, what="gamma=0 diagonal")
+    # T = 1: bidir o = v (a / (a + eps)) with a = phi(q).phi(k)
+    q1, k1, v1 = _rand((1, 1, 1, D), 12), _rand((1, 1, 1, D), 13), _rand((1, 1, 1, D), 14)
+    a = float((_feature(q1) * _feature(k1)).sum())
+    _close(orc.bidir_fwd(q1, k1, v1, eps=0.1), v1 * a / (a + 0.1), what="T=1")
+
+
+# -------------------------------------------------------------- invariances --
+
+def check_invariances(orc):
+    B, H, T, D = 1, 2, 17, 6
+    q, k, v = _rand((B, H, T, D), 20), _rand((B, H, T, D), 21), _rand((B, H, T, D), 22)
+    perm = np.random.default_rng(23).permutation(T)
+    o = orc.bidir_fwd(q, k, v, eps=1e-6)
+    _close(orc.bidir_fwd(q[:, :, perm], k, v, eps=1e-6), o[:, :, perm], rtol=1e-13, atol=1e-14,
+           what="permute queries")
+    _close(orc.bidir_fwd(q, k[:, :, perm], v[:, :, perm], eps=1e-6), o, rtol=1e-12, atol=1e-14,
+           what="permute keys/values jointly")
+    v2 = _rand((B, H, T, D), 24)
+    for fn in (lambda vv: orc.bidir_fwd(q, k, vv, eps=1e-6), lambda vv: orc.simple_fwd(q, k, vv),
+               lambda vv: orc.retention_fwd(q, k, vv, np.array([0.8, 0.95]))):
+        _close(fn(v + 2.0 * v2), fn(v) + 2.0 * fn(v2), rtol=1e-10, atol=1e-11, what="linear in V")
+    # per-head independence and indexing: each head equals a single-head call on its slice
+    B, H = 2, 3
+    q, k, v = _rand((B, H, 9, 4), 25), _rand((B, H, 9, 4), 26), _rand((B, H, 9, 4), 27)
+    g = _rand((B, H, 9, 4), 28)
+    gam = np.array([0.3, 0.7, 0.95])
+    full = [orc.bidir_fwd(q, k, v, eps=1e-2), orc.retention_fwd(q, k, v, gam)]
+    fullg = [orc.bidir_bwd(q, k, v, g, eps=1e-2), orc.retention_bwd(q, k, v, g, gam)]
+    for b in range(B):
+        for h in range(H):
+            s = (slice(b, b + 1), slice(h, h + 1))
+            _close(full[0][s], orc.bidir_fwd(q[s], k[s], v[s], eps=1e-2), rtol=0, atol=0, what="head slice bidir")
+            _close(full[1][s], orc.retention_fwd(q[s], k[s], v[s], gam[h:h + 1]), rtol=0, atol=0,
+                   what="head slice retention")
+            for a_full, a_one in zip(fullg[1], orc.retention_bwd(q[s], k[s], v[s], g[s], gam[h:h + 1])):
+                _close(a_full[s], a_one, rtol=0, atol=0, what="head slice retention bwd")
+    # thread count does not change a single bit
+    _close(orc.bidir_bwd(q, k, v, g, eps=1e-2, nthreads=1)[1], fullg[0][1], rtol=0, atol=0, what="threads")
+    # stored state = (sum_s phi(k_s)^T v_s | sum_s phi(k_s))
+    o, st = orc.bidir_fwd(q, k, v, eps=1e-2, want_state=True)
+    fk = _feature(k)
+    _close(st[..., :-1], np.einsum("bhsi,bhsj->bhij", fk, v), rtol=1e-12, atol=1e-12, what="state S")
+    _close(st[..., -1], fk.sum(2), rtol=1e-12, atol=1e-12, what="state z")
+    o, st = orc.simple_fwd(q, k, v, want_state=True)
+    _close(st[..., :-1], np.einsum("bhsi,bhsj->bhij", k, v), rtol=1e-12, atol=1e-12, what="simple state S")
+    _close(st[..., -1], np.zeros_like(st[..., -1]), rtol=0, atol=0, what="simple state z")
+
+
+# --------------------------------------------------------------- gradients --
+
+def _fd_grads(fwd, q, k, v, g, h=1e-6):
+    """Central finite differences of L = sum(fwd(q,k,v) * g) with respect to q, k, v."""
+    out = []
+    for idx in range(3):
+        args = [q.copy(), k.copy(), v.copy()]
+        grad = np.zeros_like(args[idx])
+        it = np.nditer(args[idx], flags=["multi_index"])
+        for _ in it:
+            mi = it.multi_index
+            base = args[idx][mi]
+            args[idx][mi] = base + h
+            lp = float((fwd(*args) * g).sum())
+            args[idx][mi] = base - h
+            lm = float((fwd(*args) * g).sum())
+            args[idx][mi] = base
+            grad[mi] = (lp - lm) / (2 * h)
+        out.append(grad)
+    return out
+
+
+def _keep_off_zero(x, margin=1e-2):
+    """Move entries away from 0, where phi' has a kink, so central differences are smooth."""
+    return np.where(np.abs(x) < margin, np.sign(x + 1e-30) * margin + x, x)
+
+
+def check_fd_gradients(orc):
+    B, H, T, D = 1, 2, 6, 3
+    q = _keep_off_zero(_rand((B, H, T, D), 30))
+    k = _keep_off_zero(_rand((B, H, T, D), 31))
+    v, g = _rand((B, H, T, D), 32), _rand((B, H, T, D), 33)
+    gam = np.array([0.6, 0.9])
+    cases = [
+        ("bidir", lambda a, b, c: orc.bidir_fwd(a, b, c, eps=0.05), orc.bidir_bwd(q, k, v, g, eps=0.05)),
+        ("simple", lambda a, b, c: orc.simple_fwd(a, b, c), orc.simple_bwd(q, k, v, g)),
+        ("retention", lambda a, b, c: orc.retention_fwd(a, b, c, gam), orc.retention_bwd(q, k, v, g, gam)),
+    ]
+    for name, fwd, grads in cases:
+        fd = _fd_grads(fwd, q, k, v, g)
+        for n, a, b in zip(("dq", "dk", "dv"), grads, fd):
+            _close(a, b, rtol=1e-6, atol=1e-7, what="%s %s vs finite differences" % (name, n))
+
+
+def _torch_pairwise(op, q, k, v, eps=0.0, gamma=None):
+    """Independent float64 torch forms used only through autograd."""
+    if op in ("bidir",):
+        fq = torch.where(q > 0, q + 1.0, torch.exp(torch.clamp(q, max=0.0)))
+        fk = torch.where(k > 0, k + 1.0, torch.exp(torch.clamp(k, max=0.0)))
+        a = fq @ fk.transpose(-1, -2)
+        return (a @ v) / (a.sum(-1, keepdim=True) + eps)
+    if op == "simple":
+        return (q @ k.transpose(-1, -2)) @ v
+    T = q.shape[-2]
+    t = torch.arange(T, dtype=torch.float64)
+    diff = t[:, None] - t[None, :]
+    outs = []
+    for h in range(q.shape[1]):
+        m = torch.where(diff >= 0, torch.pow(torch.tensor(float(gamma[h]), dtype=torch.float64),
+                                             torch.clamp(diff, min=0.0)), torch.zeros(()))
+        a = (q[:, h] @ k[:, h].transpose(-1, -2)) * m
+        outs.append(a @ v[:, h])
+    return torch.stack(outs, 1)
+
+
+def check_autograd(orc):
+    B, H, T, D = 2, 2, 9, 4
+    q, k, v, g = (_rand((B, H, T, D), s) for s in (40, 41, 42, 43))
+    gam = np.array([0.7, 0.97])
+    for op in ("bidir", "simple", "retention"):
+        tq, tk, tv = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (q, k, v))
+        out = _torch_pairwise(op, tq, tk, tv, eps=0.02, gamma=gam)
+        (out * torch.tensor(g)).sum().backward()
+        if op == "bidir":
+            got = orc.bidir_bwd(q, k, v, g, eps=0.02)
+        elif op == "simple":
+            got = orc.simple_bwd(q, k, v, g)
+        else:
+            got = orc.retention_bwd(q, k, v, g, gam)
+        for n, a, b in zip(("dq", "dk", "dv"), got, (tq.grad, tk.grad, tv.grad)):
+            _close(a, b.numpy(), rtol=1e-10, atol=1e-11, what="%s %s vs autograd" % (op, n))
+
+
+ALL_CHECKS = (check_golden, check_brute, check_closed_forms, check_invariances,
+              check_fd_gradients, check_autograd)

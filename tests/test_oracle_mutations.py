@@ -1,0 +1,65 @@
+"""The oracle's pins catch plausible mistakes: each case plants one mistake in a copy
+of la_oracle.c (on the CPU), compiles it, and requires at least one pin to fail."""
+import os
+
+import pytest
+
+import oracle
+from tests import pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "la_oracle.c")
+
+# (name, text to find, replacement, which occurrence (0-based))
+MUTATIONS = [
+    ("phi_drops_plus_one", "x > 0.0 ? x + 1.0 : exp(x); }", "x > 0.0 ? x : exp(x); }", 0),
+    ("phi_prime_constant", "x > 0.0 ? 1.0 : exp(x); }", "x > 0.0 ? 1.0 : 1.0; }", 0),
+    ("fwd_drops_eps", "double n = jb->eps;", "double n = 0.0;", 0),
+    ("bwd_drops_eps", "double n = jb->eps;", "double n = 0.0;", 1),
+    ("fwd_state_transposed", "u += fq[i] * S[i * D + j];", "u += fq[i] * S[j * D + i];", 0),
+    ("fwd_z_dropped", "z[i] += fk;", "z[i] += 1.0;", 0),
+    ("bwd_dz_sign", "dz[i] -= fq[i] * go / n;", "dz[i] += fq[i] * go / n;", 0),
+    ("bwd_dq_drops_norm_term", "(gs - go * z[i]) / n", "gs / n", 0),
+    ("bwd_dq_wrong_state_index", "gs += g[t * D + j] * S[i * D + j];", "gs += g[t * D + j] * S[j * D + i];", 0),
+    ("bwd_dv_transposed", "a += fk * dS[i * D + j];", "a += fk * dS[j * D + i];", 0),
+    ("bwd_dk_drops_dz", "double a = dz[i];", "double a = 0.0;", 0),
+    ("bwd_dk_uses_phi_not_dphi", "double fp = jb->use_phi ? dphi(k[s * D + i]) : 1.0;",
+     "double fp = jb->use_phi ? phi(k[s * D + i]) : 1.0;", 0),
+    ("bwd_dq_no_dphi", "double fp = jb->use_phi ? dphi(q[t * D + i]) : 1.0;", "double fp = 1.0;", 0),
+    ("ret_fwd_no_decay", "S[i * D + j] = gamma * S[i * D + j] + k[t * D + i] * v[t * D + j];",
+     "S[i * D + j] = S[i * D + j] + k[t * D + i] * v[t * D + j];", 0),
+    ("ret_fwd_output_before_update_index", "a += q[t * D + i] * S[i * D + j];", "a += q[t * D + i] * S[j * D + i];", 0),
+    ("ret_bwd_reverse_no_decay", "R[i * D + j] = gamma * R[i * D + j] + q[s * D + i] * g[s * D + j];",
+     "R[i * D + j] = R[i * D + j] + q[s * D + i] * g[s * D + j];", 0),
+    ("ret_bwd_dq_transposed", "a += S[i * D + j] * g[t * D + j];", "a += S[j * D + i] * g[t * D + j];", 0),
+    ("ret_bwd_dv_transposed", "a += k[s * D + i] * R[i * D + j];", "a += k[s * D + i] * R[j * D + i];", 0),
+    ("ret_fwd_gamma_head_index", "const double gamma = jb->gamma[bh % jb->H];", "const double gamma = jb->gamma[0];", 0),
+    ("ret_bwd_gamma_head_index", "const double gamma = jb->gamma[bh % jb->H];", "const double gamma = jb->gamma[0];", 1),
+    ("head_offset_dropped", "const long off = bh * T * D;", "const long off = 0;", 0),
+]
+
+
+def _mutate(text, find, repl, occurrence):
+    pos = -1
+    for _ in range(occurrence + 1):
+        pos = text.find(find, pos + 1)
+        if pos < 0:
+            raise ValueError("mutation target not found: %r (occurrence %d)" % (find, occurrence))
+    return text[:pos] + repl + text[pos + len(find):]
+
+
+@pytest.mark.parametrize("name,find,repl,occ", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_mutation(tmp_path, name, find, repl, occ):
+    text = open(SRC).read()
+    mutated = _mutate(text, find, repl, occ)
+    assert mutated != text
+    src = tmp_path / "mut.c"
+    src.write_text(mutated)
+    lib = oracle.build(force=True, src=str(src), out=str(tmp_path / "libmut.so"))
+    orc = oracle.load_variant(lib)
+    failures = []
+    for check in pins.ALL_CHECKS:
+        try:
+            check(orc)
+        except (AssertionError, FloatingPointError) as e:
+            failures.append((check.__name__, str(e)[:80]))
+    assert failures, "mutation %s was not caught by any pin" % name
