@@ -1,0 +1,414 @@
+"""Benchmark: bidirectional linear attention forward + backward on B200, one JSON line.
+
+A step is one forward (la_bidir_fwd, which also stores the fp32 state) plus one
+backward (la_bidir_bwd, consuming that state) over one batch of the workload,
+inputs resident in HBM.  The default workload is B=8 H=16 T=4096 D=64, fp16
+storage with fp32 accumulation, phi = elu+1, eps = 1e-6, Q,K,V ~ 0.5 N(0,1),
+dO ~ N(0,1) (seed 0 + rank).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--T T] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch of the
+same shape (independent heads, no collective on the data path: weak scaling);
+the timed region is bracketed by barriers and the reported time is the max
+over ranks.  ``--impl reference`` times the fp64 CPU oracle on the host cores
+instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "linear-attn fwd+bwd tokens/s and % of HBM roofline, B8 H16 D64 T=4K-16K"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+# The pages' own A800 Triton timings for B8-H16-D64 (ms): T -> (fwd, bwd).  Context only.
+PAGE_TIMINGS_MS = {128: (0.049152, 0.651264), 256: (0.056320, 0.625664), 512: (0.058368, 0.630784),
+                   1024: (0.090112, 0.719872), 2048: (0.151552, 0.702464), 4096: (0.276480, 1.324032),
+                   8192: (0.521216, 2.556928), 16384: (0.980992, 5.022208)}
+
+# Algorithmic HBM bytes of each kernel per launch, in units of one [B,H,T,D] tensor of the
+# storage dtype: the tensors it must read or write (state and partials are not counted).
+KERNEL_TENSORS = {
+    "simt_state_partial": 2, "simt_output": 2, "simt_bwd_q": 3, "simt_bwd_k": 4,
+    "tc_state_reduce": 2, "tc_output": 2, "tc_bwd_q": 3, "tc_bwd_kv": 4,
+}
+
+
+# ------------------------------------------------------------------ ranks --
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def init_dist(world, local_rank, backend="nccl", timeout_s=120):
+    import datetime
+    import torch.distributed as dist
+    if world <= 1:
+        return None
+    if backend == "nccl":
+        torch.cuda.set_device(local_rank)
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return dist
+
+
+def max_over_ranks(value: float, dist, device=None) -> float:
+    """Largest value over all ranks (the device timing rule for multi-GPU numbers)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank: float, world: int, seconds: float) -> float:
+    """Whole-job throughput: units processed by all ranks / the slowest rank's time."""
+    return units_per_rank * world / seconds
+
+
+# ---------------------------------------------------------------- helpers --
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "linear_attention_attn_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, T: int):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    e = rec.get(kernel)
+    if not e or e.get("source_sha") != source_hash():
+        return None
+    return float(e["dram_bytes_per_launch"]) * (T / float(e["T"]))
+
+
+def gpu_selector(dev) -> str:
+    """nvidia-smi -i argument naming this CUDA device (its UUID; the CUDA ordinal may differ from
+    nvidia-smi's index when CUDA_VISIBLE_DEVICES is set)."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev.index or 0)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: str):
+        self.gpu = gpu
+        self.proc = None
+        self.path = os.path.join("/tmp", "la_clocks_%d.csv" % os.getpid())
+
+    def start(self):
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, flag in zip(names, parts[5:9]):
+                if flag.lower() == "active":
+                    reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------- oracle arm --
+
+def oracle_step_sample(w, inp, budget_s: float, threads: int):
+    """Time the fp64 oracle on a bounded sample of the workload: n (b,h) heads at a prefix of
+    T tokens, sized to take about budget_s.  Returns (tokens/s, seconds, sample text, threads used)."""
+    import oracle
+    BH = w.B * w.H
+    q = inp["q"].reshape(BH, w.T, w.D)
+    k = inp["k"].reshape(BH, w.T, w.D)
+    v = inp["v"].reshape(BH, w.T, w.D)
+    g = inp["do"].reshape(BH, w.T, w.D)
+    # calibrate the per-token cost on one head, single thread (untimed)
+    tc = min(w.T, 512)
+    t0 = time.perf_counter()
+    oracle.bidir_fwd(q[:1, None, :tc], k[:1, None, :tc], v[:1, None, :tc], eps=w.eps, nthreads=1)
+    oracle.bidir_bwd(q[:1, None, :tc], k[:1, None, :tc], v[:1, None, :tc], g[:1, None, :tc], eps=w.eps, nthreads=1)
+    per_token = (time.perf_counter() - t0) / tc
+    budget_tokens = max(1.0, budget_s / per_token) * threads
+    n = int(max(1, min(BH, budget_tokens // w.T)))
+    Ts = w.T if n > 1 or budget_tokens >= w.T else int(max(64, min(w.T, budget_tokens)))
+    used = min(threads, n)
+    sl = slice(0, n)
+    t0 = time.perf_counter()
+    oracle.bidir_fwd(q[sl, None, :Ts].reshape(1, n, Ts, w.D), k[sl, None, :Ts].reshape(1, n, Ts, w.D),
+                     v[sl, None, :Ts].reshape(1, n, Ts, w.D), eps=w.eps, nthreads=used)
+    oracle.bidir_bwd(q[sl, None, :Ts].reshape(1, n, Ts, w.D), k[sl, None, :Ts].reshape(1, n, Ts, w.D),
+                     v[sl, None, :Ts].reshape(1, n, Ts, w.D), g[sl, None, :Ts].reshape(1, n, Ts, w.D),
+                     eps=w.eps, nthreads=used)
+    dt = time.perf_counter() - t0
+    tokens = n * Ts / float(w.H)          # token = one position of one batch row, all H heads
+    sample = "%d of %d (b,h) heads x %d of %d tokens, fp64 fwd+bwd, %d threads" % (n, BH, Ts, w.T, used)
+    return tokens / dt, dt, sample, used
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    inp = synth.make_inputs(w, seed=0)
+    cores = host_cores()
+    budget = max(0.02, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_step_sample(w, inp, budget, cores)
+    rates, secs, sample, used = [], 0.0, "", cores
+    for _ in range(args.steps):
+        r, dt, sample, used = oracle_step_sample(w, inp, budget, cores)
+        rates.append(r)
+        secs += dt
+    value = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------- ours --
+
+def config_of(w, args):
+    step_bytes = 11 * w.B * w.H * w.T * w.D * 2
+    return {"workload": "bidirectional linear attention fwd+bwd, fp16 storage / fp32 accumulate, "
+                        "B=%d H=%d T=%d D=%d, phi=elu+1, eps=%g, Q,K,V ~ 0.5 N(0,1), dO ~ N(0,1)"
+                        % (w.B, w.H, w.T, w.D, w.eps),
+            "B": w.B, "H": w.H, "T": w.T, "D": w.D, "global_batch": w.B * max(1, args.gpus), "seq_len": w.T,
+            "parallelism": "dp%d (independent batches, no collective)" % max(1, args.gpus),
+            "l2": "inputs larger than L2: %.0f MB of algorithmic traffic per step vs 126 MB L2, no flush"
+                  % (step_bytes / 1e6)}
+
+
+def run_ours(args, w):
+    import linear_attention_attn_b200 as la
+    rank, world, local = dist_env()
+    dist = init_dist(world, local)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    host = synth.make_inputs(w, seed=rank)
+    q, k, v, g = (host[n].to(dev) for n in ("q", "k", "v", "do"))
+    B, H, T, D = w.B, w.H, w.T, w.D
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    state = torch.empty((B, H, D, D + 1), dtype=torch.float32, device=dev)
+    ws_bytes = max(la.la_workspace_size("bidir_fwd", B, H, T, D, q.dtype),
+                   la.la_workspace_size("bidir_bwd", B, H, T, D, q.dtype))
+    ws = torch.empty(max(256, ws_bytes), dtype=torch.uint8, device=dev)
+
+    def step():
+        la.la_bidir_fwd(q, k, v, o, state, eps=w.eps, workspace=ws)
+        la.la_bidir_bwd(q, k, v, g, dq, dk, dv, state, eps=w.eps, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    # ---- timed region: K steps, device events, barriers on both sides
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(gpu_selector(dev))
+    sampler.start()
+    la.la_prof_enable(True)
+    la.la_prof_collect()              # drop anything recorded before
+    launches0 = la.la_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = la.la_launch_count() - launches0
+    la.la_prof_enable(False)
+    per_kernel = la.la_prof_collect()
+    if dist is not None:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(ms, dist, dev)
+    seconds = ms / 1e3
+    tokens_per_rank = B * T * args.steps
+    value = aggregate_throughput(tokens_per_rank, world, seconds)
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    e2e = None
+    hq, hk, hv, hg = (host[n].pin_memory() for n in ("q", "k", "v", "do"))
+    ho, hdq, hdk, hdv = (torch.empty_like(hq).pin_memory() for _ in range(4))
+    k_e2e = max(3, min(args.steps, 20))
+    for it in range(2 + k_e2e):
+        if it == 2:
+            if dist is not None:
+                dist.barrier()
+            torch.cuda.synchronize(dev)
+            x0 = torch.cuda.Event(enable_timing=True)
+            x0.record(stream)
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        g.copy_(hg, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+        hdq.copy_(dq, non_blocking=True)
+        hdk.copy_(dk, non_blocking=True)
+        hdv.copy_(dv, non_blocking=True)
+    x1 = torch.cuda.Event(enable_timing=True)
+    x1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1), dist, dev)
+    tensor_bytes = B * H * T * D * q.element_size()
+    e2e = {"value": aggregate_throughput(B * T * k_e2e, world, e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": 4 * tensor_bytes, "d2h_bytes_per_step": 4 * tensor_bytes,
+           "steps": k_e2e, "note": "pinned host inputs copied in and o, dq, dk, dv copied out every step"}
+
+    # ---- roofline of the dominant kernel (rank 0's per-kernel events)
+    roof = None
+    if per_kernel:
+        name, n_launch, tot_ms = max(per_kernel, key=lambda r: r[2])
+        peak, peak_kind = measured_peaks()
+        if name in KERNEL_TENSORS and n_launch > 0:
+            alg_bytes = KERNEL_TENSORS[name] * tensor_bytes
+            avg_s = tot_ms / n_launch / 1e3
+            achieved = alg_bytes / avg_s / 1e9
+            traffic = ncu_traffic(name, T)
+            roof = {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "peak_source": peak_kind, "traffic": traffic,
+                    "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_ms": tot_ms / n_launch,
+                    "share_of_step": tot_ms / max(1e-9, sum(r[2] for r in per_kernel))}
+    step_bytes = 11 * tensor_bytes
+    peak, peak_kind = measured_peaks()
+    step_roof = {"bytes_per_step": step_bytes, "achieved_gbs": step_bytes / (seconds / args.steps) / 1e9,
+                 "frac": step_bytes / (seconds / args.steps) / 1e9 / peak, "peak": peak, "peak_source": peak_kind}
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cores = host_cores()
+        r, dt, sample, used = oracle_step_sample(w, host, 15.0, cores)
+        cpu = {"value": r, "unit": UNIT, "cores": used, "kind": "oracle", "sample": sample, "seconds": dt}
+
+    vs = None
+    if T in PAGE_TIMINGS_MS and (B, H, D) == (8, 16, 64):
+        page_rate = B * T / (sum(PAGE_TIMINGS_MS[T]) / 1e3)
+        vs = value / page_rate
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": vs, "dtype": "f16", "data": "synthetic", "config": config_of(w, args),
+        "roofline": roof, "step_roofline": step_roof, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches, "clocks": clocks,
+        "kernels": [{"name": n, "launches": c, "total_ms": t} for n, c, t in per_kernel],
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--T", type=int, default=4096)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = synth.WORKLOADS["bidir_f16"].with_T(args.T)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,165 @@
+/*
+ * la.h -- C ABI of the B200 (sm_100a) linear-attention library (libla_b200.so).
+ *
+ * Three operations, forward and backward, on one GPU:
+ *
+ *  la_bidir_*   bidirectional (non-causal) linear attention with the feature
+ *               map phi = elu + 1 and the norm term:
+ *                   S = sum_s phi(k_s)^T v_s,  z = sum_s phi(k_s),
+ *                   o_t = phi(q_t) S / (phi(q_t) . z + eps).
+ *               Source: "Flash Bi-directional Linear Attention" README
+ *               (fla-org), intro ("bi-directional linear attention for
+ *               non-causal modeling") and "Benchmarks" (B8-H16-D64).
+ *  la_simple_*  simple_la: the same without the norm term and with the
+ *               identity feature map, o_t = q_t (sum_s k_s^T v_s).
+ *               Source: same README, "Update" (2024-12-28: simple_la, a
+ *               simple form of linear_attn without the norm term).
+ *  la_chunk_decay_*  causal linear attention with a per-head scalar decay
+ *               (retention), computed chunk by chunk:
+ *                   o_t = sum_{s<=t} gamma_h^(t-s) (q_t . k_s) v_s.
+ *               Source: "flash-linear-attention" README (sustcsonglin),
+ *               "Benchmarks" (RetNet, B8-H32-D128) and "Different forms of
+ *               linear attention" (FusedChunk / ParallelChunk).
+ *
+ * Common conventions
+ *  - Every tensor argument is a DEVICE pointer to a contiguous [B, H, T, D]
+ *    row-major array (D fastest) of `dtype`, 16-byte aligned.  Outputs have
+ *    the inputs' dtype.  Accumulation is fp32 throughout.
+ *  - D must be 64 or 128; B, H >= 1 with B * H <= 65535; T >= 0 (T = 0 is a
+ *    no-op that still zeroes `state`).  B * H * T * D must be < 2^31.
+ *  - Scaling (e.g. D^-1/2 on q) is the caller's: gradients are with respect
+ *    to the tensors passed.
+ *  - The caller owns all memory.  `workspace` is device scratch of at least
+ *    la_workspace_size(op, B, H, T, D, dtype) bytes, 256-byte aligned; its
+ *    contents on entry do not matter and are clobbered.  The library
+ *    allocates no device memory.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *    asynchronous: they enqueue kernels on `stream` and return; no host
+ *    synchronisation.  Results are bitwise deterministic for a given
+ *    (B, H, T, D, dtype): split reductions are combined in a fixed order.
+ *  - Two calls may run concurrently on different streams only with
+ *    different workspaces.
+ *  - Errors: arguments are validated before any CUDA call, and an invalid
+ *    call enqueues nothing.  LA_ERR_CUDA means a launch or runtime call
+ *    failed; la_last_error() gives the text (per calling thread).
+ */
+#ifndef LA_B200_H
+#define LA_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { LA_F32 = 0, LA_F16 = 1, LA_BF16 = 2 } la_dtype;
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, eps < 0, decay not in (0, 1] */
+    LA_ERR_UNSUPPORTED = 2,   /* D not in {64, 128}, unknown dtype, too many heads for decay */
+    LA_ERR_ALIGNMENT = 3,     /* a tensor or workspace pointer is not suitably aligned */
+    LA_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than la_workspace_size() */
+    LA_ERR_CUDA = 5           /* a CUDA runtime call or kernel launch failed */
+} la_status;
+
+typedef enum {
+    LA_OP_BIDIR_FWD = 0,
+    LA_OP_BIDIR_BWD = 1,
+    LA_OP_SIMPLE_FWD = 2,
+    LA_OP_SIMPLE_BWD = 3,
+    LA_OP_CHUNK_DECAY_FWD = 4,
+    LA_OP_CHUNK_DECAY_BWD = 5
+} la_op;
+
+/* Largest H accepted by la_chunk_decay_* (the decays travel as kernel arguments). */
+#define LA_MAX_DECAY_HEADS 512
+
+/* Bytes of device workspace the call `op` needs for this shape (0 if none).
+ * Depends only on its arguments.  Returns 0 for invalid arguments too. */
+size_t la_workspace_size(la_op op, int B, int H, int T, int D, la_dtype dtype);
+
+/* Bidirectional linear attention, forward.
+ *  q, k, v  in  [B,H,T,D] dtype
+ *  o        out [B,H,T,D] dtype:  o_t = phi(q_t) S / (phi(q_t) . z + eps)
+ *  state    out [B,H,D,D+1] fp32, or NULL: row i = (S[i][0..D-1], z[i]).
+ *           Pass it to la_bidir_bwd to skip recomputing S and z.
+ *  eps      >= 0, added to the denominator only.                           */
+la_status la_bidir_fwd(const void *q, const void *k, const void *v, void *o, float *state,
+                       int B, int H, int T, int D, la_dtype dtype, float eps,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bidirectional linear attention, backward.
+ *  dout     in  [B,H,T,D]: gradient of the loss with respect to o
+ *  state    in  [B,H,D,D+1] fp32 from la_bidir_fwd with the same q,k,v, or
+ *           NULL to recompute it
+ *  dq,dk,dv out [B,H,T,D] dtype: gradients with respect to q, k, v.
+ * With n_t = phi(q_t).z + eps and o_t as in the forward:
+ *  dS = sum_t phi(q_t)^T dout_t / n_t,   dz = -sum_t phi(q_t) (dout_t . o_t) / n_t
+ *  dq_t = (dout_t S^T - (dout_t . o_t) z) / n_t * phi'(q_t)
+ *  dk_s = (v_s dS^T + dz) * phi'(k_s),   dv_s = phi(k_s) dS                    */
+la_status la_bidir_bwd(const void *q, const void *k, const void *v, const void *dout,
+                       const float *state, void *dq, void *dk, void *dv,
+                       int B, int H, int T, int D, la_dtype dtype, float eps,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* simple_la forward: o_t = q_t S with S = sum_s k_s^T v_s.
+ *  state    out [B,H,D,D+1] fp32 or NULL (column D is written as 0).         */
+la_status la_simple_fwd(const void *q, const void *k, const void *v, void *o, float *state,
+                        int B, int H, int T, int D, la_dtype dtype,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* simple_la backward: dq_t = dout_t S^T, dS = sum_t q_t^T dout_t,
+ *  dk_s = v_s dS^T, dv_s = k_s dS.   state as for la_bidir_bwd (or NULL).    */
+la_status la_simple_bwd(const void *q, const void *k, const void *v, const void *dout,
+                        const float *state, void *dq, void *dk, void *dv,
+                        int B, int H, int T, int D, la_dtype dtype,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* Causal linear attention with per-head decay (retention), forward.
+ *  decay    HOST pointer to H floats, gamma_h in (0, 1]; read during the call.
+ *  o        out: o_t = sum_{s<=t} gamma_h^(t-s) (q_t . k_s) v_s               */
+la_status la_chunk_decay_fwd(const void *q, const void *k, const void *v, void *o,
+                             const float *decay,
+                             int B, int H, int T, int D, la_dtype dtype,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/* Retention backward.  With R_s = sum_{t>=s} gamma^(t-s) q_t^T dout_t and
+ * S_t = sum_{s<=t} gamma^(t-s) k_s^T v_s:
+ *  dq_t = dout_t S_t^T,  dk_s = v_s R_s^T,  dv_s = k_s R_s.                   */
+la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const void *dout,
+                             const float *decay, void *dq, void *dk, void *dv,
+                             int B, int H, int T, int D, la_dtype dtype,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/* Static text for a status code. */
+const char *la_status_string(la_status status);
+
+/* Text of the last error raised on the calling thread ("" if none). */
+const char *la_last_error(void);
+
+/* ---- instrumentation (off by default; host-side only) ------------------- */
+
+/* Count of kernels this library has launched in this process. */
+long long la_launch_count(void);
+
+/* When enabled, every kernel launch is bracketed by two CUDA events recorded
+ * on its stream.  Returns the previous setting. */
+int la_prof_enable(int enabled);
+
+/* Per-kernel totals since the last collect, for kernels launched while
+ * profiling was on.  Synchronises on the recorded events.  Fills up to
+ * `max_records` entries (name is a static string) and returns the number of
+ * distinct kernels seen (may exceed max_records), or -1 on a CUDA error. */
+typedef struct {
+    const char *name;
+    long long launches;
+    double total_ms;
+} la_prof_record;
+int la_prof_collect(la_prof_record *records, int max_records);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_B200_H */

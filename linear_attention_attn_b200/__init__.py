@@ -1,0 +1,243 @@
+"""Python binding of libla_b200.so: B200 (sm_100a) linear attention, forward and backward.
+
+Argument marshalling only: each function checks the tensors, takes their device
+pointers and calls the C entry point of the same name (``include/la.h``).  All
+arithmetic runs in the library's CUDA kernels; there is no CPU or PyTorch
+fallback -- importing this package fails if the compiled library is missing.
+
+Tensors are torch CUDA tensors, contiguous [B, H, T, D], dtype float32, float16
+or bfloat16, 16-byte aligned.  ``state`` tensors are float32 [B, H, D, D+1].
+When ``workspace`` is omitted, a torch uint8 buffer of la_workspace_size()
+bytes is allocated (torch's allocator is the only allocator involved).  When
+``stream`` is omitted the current torch stream is used.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libla_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("libla_b200.so is not built: run `python -m linear_attention_attn_b200.build` "
+                      "(or __graft_entry__.build()) first")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+LA_F32, LA_F16, LA_BF16 = 0, 1, 2
+OPS = {"bidir_fwd": 0, "bidir_bwd": 1, "simple_fwd": 2, "simple_bwd": 3,
+       "chunk_decay_fwd": 4, "chunk_decay_bwd": 5}
+STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_ALIGNMENT",
+          4: "LA_ERR_WORKSPACE", 5: "LA_ERR_CUDA"}
+MAX_DECAY_HEADS = 512
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_Z = ctypes.c_size_t
+
+
+class _ProfRecord(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_longlong), ("total_ms", ctypes.c_double)]
+
+
+_lib.la_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I]
+_lib.la_workspace_size.restype = _Z
+_lib.la_bidir_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
+_lib.la_simple_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
+_lib.la_bidir_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
+_lib.la_simple_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
+_lib.la_chunk_decay_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
+_lib.la_chunk_decay_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
+for _n in ("la_bidir_fwd", "la_simple_fwd", "la_bidir_bwd", "la_simple_bwd", "la_chunk_decay_fwd",
+           "la_chunk_decay_bwd"):
+    getattr(_lib, _n).restype = _I
+_lib.la_status_string.argtypes = [_I]
+_lib.la_status_string.restype = ctypes.c_char_p
+_lib.la_last_error.argtypes = []
+_lib.la_last_error.restype = ctypes.c_char_p
+_lib.la_launch_count.argtypes = []
+_lib.la_launch_count.restype = ctypes.c_longlong
+_lib.la_prof_enable.argtypes = [_I]
+_lib.la_prof_enable.restype = _I
+_lib.la_prof_collect.argtypes = [ctypes.POINTER(_ProfRecord), _I]
+_lib.la_prof_collect.restype = _I
+
+
+class LAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.la_last_error().decode(errors="replace")
+        super().__init__("%s: %s: %s" % (where, STATUS.get(status, status), msg))
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise LAError(rc, where)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    codes = {torch.float32: LA_F32, torch.float16: LA_F16, torch.bfloat16: LA_BF16}
+    if t.dtype not in codes:
+        raise TypeError("unsupported dtype %s" % t.dtype)
+    return codes[t.dtype]
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _shape(q, *others):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, T, D] tensors, got %r" % (tuple(q.shape),))
+    for o in others:
+        if o is None:
+            continue
+        if tuple(o.shape) != tuple(q.shape) or o.dtype != q.dtype or o.device != q.device:
+            raise ValueError("all tensors must share shape, dtype and device")
+    for o in (q,) + others:
+        if o is not None and (not o.is_cuda or not o.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    return tuple(int(x) for x in q.shape)
+
+
+def _stream(stream, dev):
+    import torch
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _state_check(state, B, H, D, dev):
+    import torch
+    if state is None:
+        return
+    if (tuple(state.shape) != (B, H, D, D + 1) or state.dtype != torch.float32 or not state.is_cuda
+            or not state.is_contiguous() or state.device != dev):
+        raise ValueError("state must be a contiguous float32 CUDA tensor [B, H, D, D+1] on the inputs' device")
+
+
+def la_workspace_size(op, B: int, H: int, T: int, D: int, dtype) -> int:
+    """Bytes of workspace the op needs (op is a name from OPS or its code; dtype a torch dtype or code)."""
+    import torch
+    code = OPS[op] if isinstance(op, str) else int(op)
+    if isinstance(dtype, torch.dtype):
+        dtype = {torch.float32: LA_F32, torch.float16: LA_F16, torch.bfloat16: LA_BF16}[dtype]
+    return int(_lib.la_workspace_size(code, B, H, T, D, int(dtype)))
+
+
+def _workspace(op, shape, dt, workspace, dev, stream):
+    import torch
+    need = _lib.la_workspace_size(OPS[op], *shape, dt)
+    if workspace is not None:
+        return ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size(), workspace
+    if need == 0:
+        return None, 0, None
+    buf = torch.empty(need + 256, dtype=torch.uint8, device=dev)
+    if isinstance(stream, torch.cuda.Stream):
+        buf.record_stream(stream)   # the kernels run on `stream`, not torch's current one
+    off = (-buf.data_ptr()) % 256
+    buf = buf[off:off + need]
+    return ctypes.c_void_p(buf.data_ptr()), need, buf
+
+
+def la_bidir_fwd(q, k, v, o, state=None, eps: float = 1e-6, workspace=None, stream=None):
+    """o <- phi(q) S / (phi(q) . z + eps); optionally state <- (S | z). See include/la.h."""
+    B, H, T, D = _shape(q, k, v, o)
+    _state_check(state, B, H, D, q.device)
+    dt = _dtype_code(q)
+    wp, wn, _keep = _workspace("bidir_fwd", (B, H, T, D), dt, workspace, q.device, stream)
+    _check(_lib.la_bidir_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), B, H, T, D, dt, float(eps),
+                             wp, wn, _stream(stream, q.device)), "la_bidir_fwd")
+
+
+def la_simple_fwd(q, k, v, o, state=None, workspace=None, stream=None):
+    """o <- q (k^T v). See include/la.h."""
+    B, H, T, D = _shape(q, k, v, o)
+    _state_check(state, B, H, D, q.device)
+    dt = _dtype_code(q)
+    wp, wn, _keep = _workspace("simple_fwd", (B, H, T, D), dt, workspace, q.device, stream)
+    _check(_lib.la_simple_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), B, H, T, D, dt,
+                              wp, wn, _stream(stream, q.device)), "la_simple_fwd")
+
+
+def la_bidir_bwd(q, k, v, dout, dq, dk, dv, state=None, eps: float = 1e-6, workspace=None, stream=None):
+    """dq, dk, dv <- gradients of sum(o * dout) for la_bidir_fwd. See include/la.h."""
+    B, H, T, D = _shape(q, k, v, dout, dq, dk, dv)
+    _state_check(state, B, H, D, q.device)
+    dt = _dtype_code(q)
+    wp, wn, _keep = _workspace("bidir_bwd", (B, H, T, D), dt, workspace, q.device, stream)
+    _check(_lib.la_bidir_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(state), _ptr(dq), _ptr(dk), _ptr(dv),
+                             B, H, T, D, dt, float(eps), wp, wn, _stream(stream, q.device)), "la_bidir_bwd")
+
+
+def la_simple_bwd(q, k, v, dout, dq, dk, dv, state=None, workspace=None, stream=None):
+    """dq, dk, dv <- gradients of sum(o * dout) for la_simple_fwd. See include/la.h."""
+    B, H, T, D = _shape(q, k, v, dout, dq, dk, dv)
+    _state_check(state, B, H, D, q.device)
+    dt = _dtype_code(q)
+    wp, wn, _keep = _workspace("simple_bwd", (B, H, T, D), dt, workspace, q.device, stream)
+    _check(_lib.la_simple_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(state), _ptr(dq), _ptr(dk), _ptr(dv),
+                              B, H, T, D, dt, wp, wn, _stream(stream, q.device)), "la_simple_bwd")
+
+
+def _decay(decay, H):
+    vals = [float(x) for x in (decay.tolist() if hasattr(decay, "tolist") else decay)]
+    if len(vals) != H:
+        raise ValueError("decay must have H=%d entries" % H)
+    return (ctypes.c_float * H)(*vals)
+
+
+def la_chunk_decay_fwd(q, k, v, o, decay, workspace=None, stream=None):
+    """o_t <- sum_{s<=t} decay[h]^(t-s) (q_t . k_s) v_s; decay is a length-H host sequence."""
+    B, H, T, D = _shape(q, k, v, o)
+    dt = _dtype_code(q)
+    dec = _decay(decay, H)
+    wp, wn, _keep = _workspace("chunk_decay_fwd", (B, H, T, D), dt, workspace, q.device, stream)
+    _check(_lib.la_chunk_decay_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.cast(dec, _P), B, H, T, D, dt,
+                                   wp, wn, _stream(stream, q.device)), "la_chunk_decay_fwd")
+
+
+def la_chunk_decay_bwd(q, k, v, dout, decay, dq, dk, dv, workspace=None, stream=None):
+    """dq, dk, dv <- gradients of sum(o * dout) for la_chunk_decay_fwd."""
+    B, H, T, D = _shape(q, k, v, dout, dq, dk, dv)
+    dt = _dtype_code(q)
+    dec = _decay(decay, H)
+    wp, wn, _keep = _workspace("chunk_decay_bwd", (B, H, T, D), dt, workspace, q.device, stream)
+    _check(_lib.la_chunk_decay_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), ctypes.cast(dec, _P), _ptr(dq),
+                                   _ptr(dk), _ptr(dv), B, H, T, D, dt, wp, wn, _stream(stream, q.device)),
+           "la_chunk_decay_bwd")
+
+
+def la_status_string(status: int) -> str:
+    return _lib.la_status_string(int(status)).decode()
+
+
+def la_last_error() -> str:
+    return _lib.la_last_error().decode(errors="replace")
+
+
+def la_launch_count() -> int:
+    return int(_lib.la_launch_count())
+
+
+def la_prof_enable(enabled: bool) -> bool:
+    return bool(_lib.la_prof_enable(1 if enabled else 0))
+
+
+def la_prof_collect(max_records: int = 64):
+    """[(kernel name, launches, total ms)] for launches made while profiling was on."""
+    recs = (_ProfRecord * max_records)()
+    n = _lib.la_prof_collect(recs, max_records)
+    if n < 0:
+        raise RuntimeError("la_prof_collect failed: " + la_last_error())
+    return [(recs[i].name.decode(), int(recs[i].launches), float(recs[i].total_ms)) for i in range(min(n, max_records))]
+
+
+def raw_lib():
+    """The ctypes handle of libla_b200.so (for callers passing raw pointers)."""
+    return _lib

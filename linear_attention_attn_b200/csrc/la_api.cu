@@ -1,0 +1,348 @@
+// la_api.cu -- the C entry points: argument validation, workspace layout,
+// path selection, launch accounting and the optional per-kernel timing.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "la_internal.cuh"
+#include "la_tc.cuh"
+
+namespace la {
+
+// ---------------------------------------------------------------- errors --
+
+static thread_local std::string g_last_error;
+
+void set_error(const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+}
+
+la_status cuda_fail(cudaError_t e, const char *what) {
+    set_error("%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+    return LA_ERR_CUDA;
+}
+
+static la_status fail(la_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+// ------------------------------------------------- launches and profiling --
+
+static std::atomic<long long> g_launches{0};
+static std::atomic<int> g_prof_on{0};
+
+struct ProfEntry {
+    const char *name;
+    cudaEvent_t start, stop;
+};
+static std::mutex g_prof_mu;
+static std::vector<ProfEntry> g_prof;            // recorded, not yet collected
+static std::vector<cudaEvent_t> g_event_pool;     // reusable events
+static thread_local const char *t_pending_name = nullptr;
+static thread_local cudaEvent_t t_pending_start = nullptr;
+
+static cudaEvent_t take_event() {
+    {
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        if (!g_event_pool.empty()) {
+            cudaEvent_t e = g_event_pool.back();
+            g_event_pool.pop_back();
+            return e;
+        }
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+void prof_before(const char *name, cudaStream_t s) {
+    t_pending_name = nullptr;
+    if (!g_prof_on.load(std::memory_order_relaxed)) return;
+    cudaEvent_t e = take_event();
+    if (!e) return;
+    cudaEventRecord(e, s);
+    t_pending_name = name;
+    t_pending_start = e;
+}
+
+void prof_after(cudaStream_t s) {
+    if (!t_pending_name) return;
+    cudaEvent_t e = take_event();
+    if (!e) return;
+    cudaEventRecord(e, s);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof.push_back({t_pending_name, t_pending_start, e});
+    t_pending_name = nullptr;
+}
+
+// ----------------------------------------------------- shapes / workspace --
+
+int state_splits(const Shape &s, int rows_per_unit) {
+    // Aim at about two CTAs per SM of a 148-SM part, never fewer rows per split
+    // than one unit, never more than 64 splits.
+    const long long target = 296;
+    long long want = (target + s.BH() - 1) / s.BH();
+    long long max_units = (s.T + rows_per_unit - 1) / rows_per_unit;
+    if (want > max_units) want = max_units;
+    if (want > 64) want = 64;
+    if (want < 1) want = 1;
+    return (int)want;
+}
+
+size_t state_bytes(const Shape &s, long long copies) {
+    size_t b = (size_t)s.BH() * (size_t)copies * (size_t)s.D * (size_t)(s.D + 1) * sizeof(float);
+    return (b + 255) & ~(size_t)255;
+}
+
+static bool path_tc(const Shape &s, la_dtype dt) { return tc::supports(s, dt); }
+
+static la_status validate(const Shape &s, la_dtype dt) {
+    if (s.B < 1 || s.H < 1 || s.T < 0) return fail(LA_ERR_INVALID_ARG, "B, H must be >= 1 and T >= 0");
+    if (dt != LA_F32 && dt != LA_F16 && dt != LA_BF16) return fail(LA_ERR_UNSUPPORTED, "unknown dtype %d", (int)dt);
+    if (s.D != 64 && s.D != 128) return fail(LA_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", s.D);
+    if ((double)s.B * s.H * s.T * s.D >= 2147483648.0)
+        return fail(LA_ERR_UNSUPPORTED, "tensor too large (B*H*T*D must be < 2^31)");
+    if (s.BH() > 65535) return fail(LA_ERR_UNSUPPORTED, "B*H must be <= 65535");
+    return LA_OK;
+}
+
+static la_status check_ptr(const void *p, const char *name) {
+    if (!p) return fail(LA_ERR_INVALID_ARG, "%s is NULL", name);
+    if (((uintptr_t)p) & 15) return fail(LA_ERR_ALIGNMENT, "%s is not 16-byte aligned", name);
+    return LA_OK;
+}
+
+static size_t ws_size(la_op op, const Shape &s, la_dtype dt) {
+    if (path_tc(s, dt)) return tc::workspace_size(op, s, dt);
+    return simt::workspace_size(op, s);
+}
+
+static la_status check_ws(la_op op, const Shape &s, la_dtype dt, void *ws, size_t ws_bytes) {
+    const size_t need = ws_size(op, s, dt);
+    if (need == 0) return LA_OK;
+    if (!ws) return fail(LA_ERR_WORKSPACE, "workspace is NULL but %zu bytes are needed", need);
+    if (((uintptr_t)ws) & 255) return fail(LA_ERR_ALIGNMENT, "workspace is not 256-byte aligned");
+    if (ws_bytes < need) return fail(LA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", ws_bytes, need);
+    return LA_OK;
+}
+
+#define LA_TRY(x)                     \
+    do {                              \
+        la_status _rc = (x);          \
+        if (_rc != LA_OK) return _rc; \
+    } while (0)
+
+// Common front half of the bidir / simple entry points.
+static la_status state_fwd_entry(bool bidir, const void *q, const void *k, const void *v, void *o, float *state,
+                                 int B, int H, int T, int D, la_dtype dt, float eps, void *ws, size_t ws_bytes,
+                                 void *stream) {
+    const Shape s{B, H, T, D};
+    const la_op op = bidir ? LA_OP_BIDIR_FWD : LA_OP_SIMPLE_FWD;
+    LA_TRY(validate(s, dt));
+    if (!(eps >= 0.f)) return fail(LA_ERR_INVALID_ARG, "eps must be >= 0");
+    LA_TRY(check_ptr(q, "q"));
+    LA_TRY(check_ptr(k, "k"));
+    LA_TRY(check_ptr(v, "v"));
+    LA_TRY(check_ptr(o, "o"));
+    if (state && (((uintptr_t)state) & 15)) return fail(LA_ERR_ALIGNMENT, "state is not 16-byte aligned");
+    LA_TRY(check_ws(op, s, dt, ws, ws_bytes));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (T == 0) {
+        if (state) {
+            cudaError_t e = cudaMemsetAsync(state, 0, (size_t)s.BH() * D * (D + 1) * sizeof(float), st);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(state)");
+        }
+        return LA_OK;
+    }
+    if (path_tc(s, dt)) return tc::state_fwd(bidir, q, k, v, o, state, s, dt, eps, ws, st);
+    return simt::state_fwd(bidir, q, k, v, o, state, s, dt, eps, ws, st);
+}
+
+static la_status state_bwd_entry(bool bidir, const void *q, const void *k, const void *v, const void *g,
+                                 const float *state, void *dq, void *dk, void *dv, int B, int H, int T, int D,
+                                 la_dtype dt, float eps, void *ws, size_t ws_bytes, void *stream) {
+    const Shape s{B, H, T, D};
+    const la_op op = bidir ? LA_OP_BIDIR_BWD : LA_OP_SIMPLE_BWD;
+    LA_TRY(validate(s, dt));
+    if (!(eps >= 0.f)) return fail(LA_ERR_INVALID_ARG, "eps must be >= 0");
+    LA_TRY(check_ptr(q, "q"));
+    LA_TRY(check_ptr(k, "k"));
+    LA_TRY(check_ptr(v, "v"));
+    LA_TRY(check_ptr(g, "dout"));
+    LA_TRY(check_ptr(dq, "dq"));
+    LA_TRY(check_ptr(dk, "dk"));
+    LA_TRY(check_ptr(dv, "dv"));
+    if (state && (((uintptr_t)state) & 15)) return fail(LA_ERR_ALIGNMENT, "state is not 16-byte aligned");
+    LA_TRY(check_ws(op, s, dt, ws, ws_bytes));
+    if (T == 0) return LA_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (path_tc(s, dt)) return tc::state_bwd(bidir, q, k, v, g, state, dq, dk, dv, s, dt, eps, ws, st);
+    return simt::state_bwd(bidir, q, k, v, g, state, dq, dk, dv, s, dt, eps, ws, st);
+}
+
+static la_status decay_args(const float *decay, int H, DecayArgs *out) {
+    if (!decay) return fail(LA_ERR_INVALID_ARG, "decay is NULL");
+    if (H > LA_MAX_DECAY_HEADS) return fail(LA_ERR_UNSUPPORTED, "H=%d exceeds %d for the decay op", H, LA_MAX_DECAY_HEADS);
+    memset(out, 0, sizeof *out);
+    for (int h = 0; h < H; ++h) {
+        const float g = decay[h];
+        if (!(g > 0.f && g <= 1.f)) return fail(LA_ERR_INVALID_ARG, "decay[%d]=%g is not in (0, 1]", h, (double)g);
+        out->gamma[h] = g;
+    }
+    return LA_OK;
+}
+
+}  // namespace la
+
+using namespace la;
+
+extern "C" {
+
+size_t la_workspace_size(la_op op, int B, int H, int T, int D, la_dtype dtype) {
+    const Shape s{B, H, T, D};
+    if (s.B < 1 || s.H < 1 || s.T < 0 || (s.D != 64 && s.D != 128)) return 0;
+    if (dtype != LA_F32 && dtype != LA_F16 && dtype != LA_BF16) return 0;
+    if ((int)op < 0 || (int)op > 5) return 0;
+    return ws_size(op, s, dtype);
+}
+
+la_status la_bidir_fwd(const void *q, const void *k, const void *v, void *o, float *state, int B, int H, int T,
+                       int D, la_dtype dtype, float eps, void *workspace, size_t workspace_bytes, void *stream) {
+    return state_fwd_entry(true, q, k, v, o, state, B, H, T, D, dtype, eps, workspace, workspace_bytes, stream);
+}
+
+la_status la_simple_fwd(const void *q, const void *k, const void *v, void *o, float *state, int B, int H, int T,
+                        int D, la_dtype dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    return state_fwd_entry(false, q, k, v, o, state, B, H, T, D, dtype, 0.f, workspace, workspace_bytes, stream);
+}
+
+la_status la_bidir_bwd(const void *q, const void *k, const void *v, const void *dout, const float *state, void *dq,
+                       void *dk, void *dv, int B, int H, int T, int D, la_dtype dtype, float eps, void *workspace,
+                       size_t workspace_bytes, void *stream) {
+    return state_bwd_entry(true, q, k, v, dout, state, dq, dk, dv, B, H, T, D, dtype, eps, workspace,
+                           workspace_bytes, stream);
+}
+
+la_status la_simple_bwd(const void *q, const void *k, const void *v, const void *dout, const float *state, void *dq,
+                        void *dk, void *dv, int B, int H, int T, int D, la_dtype dtype, void *workspace,
+                        size_t workspace_bytes, void *stream) {
+    return state_bwd_entry(false, q, k, v, dout, state, dq, dk, dv, B, H, T, D, dtype, 0.f, workspace,
+                           workspace_bytes, stream);
+}
+
+la_status la_chunk_decay_fwd(const void *q, const void *k, const void *v, void *o, const float *decay, int B, int H,
+                             int T, int D, la_dtype dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    const Shape s{B, H, T, D};
+    LA_TRY(validate(s, dtype));
+    LA_TRY(check_ptr(q, "q"));
+    LA_TRY(check_ptr(k, "k"));
+    LA_TRY(check_ptr(v, "v"));
+    LA_TRY(check_ptr(o, "o"));
+    DecayArgs dec;
+    LA_TRY(decay_args(decay, H, &dec));
+    LA_TRY(check_ws(LA_OP_CHUNK_DECAY_FWD, s, dtype, workspace, workspace_bytes));
+    if (T == 0) return LA_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (path_tc(s, dtype)) return tc::decay_fwd(q, k, v, o, dec, s, dtype, workspace, st);
+    return simt::decay_fwd(q, k, v, o, dec, s, dtype, st);
+}
+
+la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const void *dout, const float *decay,
+                             void *dq, void *dk, void *dv, int B, int H, int T, int D, la_dtype dtype,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    const Shape s{B, H, T, D};
+    LA_TRY(validate(s, dtype));
+    LA_TRY(check_ptr(q, "q"));
+    LA_TRY(check_ptr(k, "k"));
+    LA_TRY(check_ptr(v, "v"));
+    LA_TRY(check_ptr(dout, "dout"));
+    LA_TRY(check_ptr(dq, "dq"));
+    LA_TRY(check_ptr(dk, "dk"));
+    LA_TRY(check_ptr(dv, "dv"));
+    DecayArgs dec;
+    LA_TRY(decay_args(decay, H, &dec));
+    LA_TRY(check_ws(LA_OP_CHUNK_DECAY_BWD, s, dtype, workspace, workspace_bytes));
+    if (T == 0) return LA_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (path_tc(s, dtype)) return tc::decay_bwd(q, k, v, dout, dec, dq, dk, dv, s, dtype, workspace, st);
+    return simt::decay_bwd(q, k, v, dout, dec, dq, dk, dv, s, dtype, st);
+}
+
+const char *la_status_string(la_status status) {
+    switch (status) {
+    case LA_OK: return "LA_OK";
+    case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG";
+    case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED";
+    case LA_ERR_ALIGNMENT: return "LA_ERR_ALIGNMENT";
+    case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE";
+    case LA_ERR_CUDA: return "LA_ERR_CUDA";
+    }
+    return "LA_ERR_UNKNOWN";
+}
+
+const char *la_last_error(void) { return g_last_error.c_str(); }
+
+long long la_launch_count(void) { return g_launches.load(); }
+
+int la_prof_enable(int enabled) { return g_prof_on.exchange(enabled ? 1 : 0); }
+
+int la_prof_collect(la_prof_record *records, int max_records) {
+    std::vector<ProfEntry> entries;
+    {
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        entries.swap(g_prof);
+    }
+    struct Agg {
+        const char *name;
+        long long n;
+        double ms;
+    };
+    std::vector<Agg> agg;
+    int rc = 0;
+    for (const ProfEntry &e : entries) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(e.stop) != cudaSuccess || cudaEventElapsedTime(&ms, e.start, e.stop) != cudaSuccess) {
+            rc = -1;
+        }
+        size_t i = 0;
+        for (; i < agg.size(); ++i)
+            if (strcmp(agg[i].name, e.name) == 0) break;
+        if (i == agg.size()) agg.push_back({e.name, 0, 0.0});
+        agg[i].n += 1;
+        agg[i].ms += ms;
+    }
+    {
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        for (const ProfEntry &e : entries) {
+            g_event_pool.push_back(e.start);
+            g_event_pool.push_back(e.stop);
+        }
+    }
+    if (rc) return -1;
+    for (size_t i = 0; i < agg.size() && (int)i < max_records; ++i) {
+        records[i].name = agg[i].name;
+        records[i].launches = agg[i].n;
+        records[i].total_ms = agg[i].ms;
+    }
+    return (int)agg.size();
+}
+
+}  // extern "C"

@@ -1,0 +1,97 @@
+// la_internal.cuh -- shared declarations of the library's CUDA sources (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/la.h"
+
+namespace la {
+
+// ---------------------------------------------------------------- errors --
+void set_error(const char *fmt, ...);
+la_status cuda_fail(cudaError_t e, const char *what);
+
+// ------------------------------------------------------------- launching --
+// Every kernel goes through launch(): it counts launches and, when profiling
+// is on, brackets the launch with two events on its stream.
+void prof_before(const char *name, cudaStream_t s);
+void prof_after(cudaStream_t s);
+void count_launch();
+
+template <typename Kernel, typename... Args>
+la_status launch(const char *name, Kernel kernel, dim3 grid, dim3 block, size_t smem,
+                 cudaStream_t stream, Args... args) {
+    if (grid.x == 0 || grid.y == 0 || grid.z == 0) return LA_OK;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, name);
+    }
+    prof_before(name, stream);
+    kernel<<<grid, block, smem, stream>>>(args...);
+    cudaError_t e = cudaGetLastError();
+    prof_after(stream);
+    count_launch();
+    if (e != cudaSuccess) return cuda_fail(e, name);
+    return LA_OK;
+}
+
+// ---------------------------------------------------------- element I/O --
+template <typename T> struct io;
+template <> struct io<float> {
+    static __device__ __forceinline__ float ld(const float *p) { return __ldg(p); }
+    static __device__ __forceinline__ void st(float *p, float x) { *p = x; }
+};
+template <> struct io<__half> {
+    static __device__ __forceinline__ float ld(const __half *p) { return __half2float(__ldg(p)); }
+    static __device__ __forceinline__ void st(__half *p, float x) { *p = __float2half_rn(x); }
+};
+template <> struct io<__nv_bfloat16> {
+    static __device__ __forceinline__ float ld(const __nv_bfloat16 *p) { return __bfloat162float(__ldg(p)); }
+    static __device__ __forceinline__ void st(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+};
+
+// Feature map of bidirectional linear attention: elu(x) + 1, i.e. x + 1 for
+// x > 0 and exp(x) for x <= 0, and its derivative (1, resp. exp(x)).
+__device__ __forceinline__ float feature(float x) { return x > 0.f ? x + 1.f : expf(x); }
+__device__ __forceinline__ float feature_grad(float x) { return x > 0.f ? 1.f : expf(x); }
+
+// Per-head decays of the chunked causal op travel by value.
+struct DecayArgs {
+    float gamma[LA_MAX_DECAY_HEADS];
+};
+
+// ------------------------------------------------------ shape / workspace --
+struct Shape {
+    int B, H, T, D;
+    long long BH() const { return (long long)B * H; }
+};
+
+// Split count of the T-reductions: a function of (B, H, T) only, so results
+// are deterministic for a shape whatever GPU runs them.
+int state_splits(const Shape &s, int rows_per_unit);
+
+// Bytes of one [BH, D, D+1] fp32 state block, rounded up to 256.
+size_t state_bytes(const Shape &s, long long copies);
+
+// ------------------------------------------------------------ SIMT path --
+// Plain CUDA-core kernels (fp32 FMA).  They implement every op for every
+// dtype; the fp16/bf16 ops at D in {64,128} normally run on the tensor-core
+// path instead.
+namespace simt {
+size_t workspace_size(la_op op, const Shape &s);
+la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, void *o, float *state,
+                    const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
+la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, const void *g,
+                    const float *state, void *dq, void *dk, void *dv, const Shape &s, la_dtype dt,
+                    float eps, void *ws, cudaStream_t st);
+la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec,
+                    const Shape &s, la_dtype dt, cudaStream_t st);
+la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec,
+                    void *dq, void *dk, void *dv, const Shape &s, la_dtype dt, cudaStream_t st);
+}  // namespace simt
+
+}  // namespace la

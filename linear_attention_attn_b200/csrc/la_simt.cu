@@ -1,0 +1,604 @@
+// la_simt.cu -- CUDA-core (fp32 FMA) kernels for every op and dtype.
+//
+// This is the straightforward path: every contraction is a loop of fp32
+// FMAs over shared-memory tiles.  It carries fp32 inputs (where the tensor
+// cores would round operands) and is the reference GPU implementation that
+// the tensor-core kernels are checked against besides the CPU oracle.
+//
+// Bidirectional / simple_la ("Flash Bi-directional Linear Attention" README,
+// intro and "Update": linear_attn with and without the norm term):
+//   state_partial  per (b,h, T-split): S_part = sum phi(k)^T v, z_part = sum phi(k)
+//   combine        fixed-order sum of the splits          -> state [BH, D, D+1]
+//   output         o_t = phi(q_t) S / (phi(q_t).z + eps)
+//   bwd_q          dq and the per-split partials of dS, dz
+//   bwd_k          dk = (v dS^T + dz) phi'(k),  dv = phi(k) dS
+// Retention ("flash-linear-attention" README, "Benchmarks" and "Different
+// forms of linear attention", FusedRecurrent): one CTA per (b,h) walks T
+// with the D x D state held in registers, one state column (or row) per
+// thread.
+#include "la_internal.cuh"
+
+namespace la {
+namespace simt {
+
+constexpr int kTile = 32;      // rows per shared-memory tile
+constexpr int kRetTile = 16;   // rows per tile in the recurrent (retention) kernels
+constexpr int kThreads = 256;
+
+// ------------------------------------------------------------ reductions --
+
+// Partial S (and z for bidir) over rows [split*rps, min(T, (split+1)*rps)) of
+// head blockIdx.y.  Thread (ti, tj) owns the R x R block S[ti*R.., tj*R..].
+template <typename T, int D, bool BIDIR>
+__global__ void __launch_bounds__(kThreads)
+state_partial(const T *__restrict__ k, const T *__restrict__ v, float *__restrict__ part,
+              int T_len, int nsplit, int rps) {
+    constexpr int R = D / 16;
+    __shared__ float ks[kTile][D];
+    __shared__ float vs[kTile][D];
+    const int split = blockIdx.x, bh = blockIdx.y;
+    const long long base = (long long)bh * T_len * D;
+    const int t0 = split * rps;
+    const int t1 = min(T_len, t0 + rps);
+    const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
+    float acc[R][R];
+    float zacc[R];
+#pragma unroll
+    for (int x = 0; x < R; ++x) {
+        zacc[x] = 0.f;
+#pragma unroll
+        for (int y = 0; y < R; ++y) acc[x][y] = 0.f;
+    }
+    for (int ts = t0; ts < t1; ts += kTile) {
+        for (int e = threadIdx.x; e < kTile * D; e += kThreads) {
+            const int r = e / D, c = e % D, t = ts + r;
+            float kk = 0.f, vv = 0.f;
+            if (t < t1) {
+                kk = io<T>::ld(k + base + (long long)t * D + c);
+                if (BIDIR) kk = feature(kk);
+                vv = io<T>::ld(v + base + (long long)t * D + c);
+            }
+            ks[r][c] = kk;
+            vs[r][c] = vv;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int r = 0; r < kTile; ++r) {
+            float a[R], b[R];
+#pragma unroll
+            for (int x = 0; x < R; ++x) {
+                a[x] = ks[r][ti * R + x];
+                b[x] = vs[r][tj * R + x];
+            }
+#pragma unroll
+            for (int x = 0; x < R; ++x) {
+                if (BIDIR) zacc[x] += a[x];
+#pragma unroll
+                for (int y = 0; y < R; ++y) acc[x][y] = fmaf(a[x], b[y], acc[x][y]);
+            }
+        }
+        __syncthreads();
+    }
+    float *out = part + ((long long)bh * nsplit + split) * D * (D + 1);
+#pragma unroll
+    for (int x = 0; x < R; ++x) {
+#pragma unroll
+        for (int y = 0; y < R; ++y) out[(ti * R + x) * (D + 1) + tj * R + y] = acc[x][y];
+        if (tj == 0) out[(ti * R + x) * (D + 1) + D] = BIDIR ? zacc[x] : 0.f;
+    }
+}
+
+// out[bh][e] = sum_{s=0..nsplit-1} part[bh][s][e], always in that order.
+__global__ void __launch_bounds__(kThreads)
+combine(const float *__restrict__ part, float *__restrict__ out, int nsplit, int n) {
+    const long long bh = blockIdx.x;
+    for (int e = threadIdx.x; e < n; e += kThreads) {
+        float s = 0.f;
+        for (int sp = 0; sp < nsplit; ++sp) s += part[(bh * nsplit + sp) * n + e];
+        out[bh * n + e] = s;
+    }
+}
+
+// --------------------------------------------------------------- outputs --
+
+// o_t = f(q_t) S / (f(q_t).z + eps)  (bidir)  or  q_t S  (simple).
+// 32 rows per CTA, 8 threads per row, thread cg owns columns cg + 8c.
+template <typename T, int D, bool BIDIR>
+__global__ void __launch_bounds__(kThreads)
+output(const T *__restrict__ q, const float *__restrict__ state, T *__restrict__ o, int T_len, float eps) {
+    constexpr int TPR = kThreads / kTile;
+    constexpr int CPT = D / TPR;
+    constexpr int LD = D + 1;
+    extern __shared__ float sm[];
+    float *S = sm;              // D x D
+    float *z = S + D * D;       // D
+    float *qs = z + D;          // kTile x LD
+    const int bh = blockIdx.y;
+    const int row0 = blockIdx.x * kTile;
+    const long long base = (long long)bh * T_len * D;
+    const float *st = state + (long long)bh * D * (D + 1);
+    for (int e = threadIdx.x; e < D * D; e += kThreads) S[e] = st[(e / D) * (D + 1) + e % D];
+    for (int e = threadIdx.x; e < D; e += kThreads) z[e] = st[e * (D + 1) + D];
+    for (int e = threadIdx.x; e < kTile * D; e += kThreads) {
+        const int r = e / D, c = e % D, t = row0 + r;
+        float x = t < T_len ? io<T>::ld(q + base + (long long)t * D + c) : 0.f;
+        qs[r * LD + c] = (BIDIR && t < T_len) ? feature(x) : x;
+    }
+    __syncthreads();
+    const int r = threadIdx.x / TPR, cg = threadIdx.x % TPR, t = row0 + r;
+    float acc[CPT];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) acc[c] = 0.f;
+    float n = eps;
+    for (int i = 0; i < D; ++i) {
+        const float qi = qs[r * LD + i];
+        if (BIDIR) n = fmaf(qi, z[i], n);
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) acc[c] = fmaf(qi, S[i * D + cg + TPR * c], acc[c]);
+    }
+    if (t < T_len) {
+#pragma unroll
+        for (int c = 0; c < CPT; ++c)
+            io<T>::st(o + base + (long long)t * D + cg + TPR * c, BIDIR ? acc[c] / n : acc[c]);
+    }
+}
+
+// ------------------------------------------------------------- backward ---
+
+// Query side of the backward pass over rows [split*rps, ...) of one head:
+// writes dq and the split's partial (dS | dz) into part.
+template <typename T, int D, bool BIDIR>
+__global__ void __launch_bounds__(kThreads)
+bwd_q(const T *__restrict__ q, const T *__restrict__ g, const float *__restrict__ state,
+      T *__restrict__ dq, float *__restrict__ part, int T_len, int nsplit, int rps, float eps) {
+    constexpr int TPR = kThreads / kTile;
+    constexpr int CPT = D / TPR;
+    constexpr int LD = D + 1;
+    constexpr int R = D / 16;
+    extern __shared__ float sm[];
+    float *S = sm;                 // D x LD
+    float *z = S + D * LD;         // D
+    float *qraw = z + D;           // kTile x LD
+    float *qf = qraw + kTile * LD; // kTile x LD   (feature of q, 0 on padded rows)
+    float *gs = qf + kTile * LD;   // kTile x LD   (g, then g / n)
+    float *wr = gs + kTile * LD;   // kTile        (-(g.o)/n)
+    const int split = blockIdx.x, bh = blockIdx.y;
+    const long long base = (long long)bh * T_len * D;
+    const int t0 = split * rps;
+    const int t1 = min(T_len, t0 + rps);
+    const float *st = state + (long long)bh * D * (D + 1);
+    for (int e = threadIdx.x; e < D * D; e += kThreads) S[(e / D) * LD + e % D] = st[(e / D) * (D + 1) + e % D];
+    for (int e = threadIdx.x; e < D; e += kThreads) z[e] = BIDIR ? st[e * (D + 1) + D] : 0.f;
+    const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
+    float acc[R][R];
+    float zacc[R];
+#pragma unroll
+    for (int x = 0; x < R; ++x) {
+        zacc[x] = 0.f;
+#pragma unroll
+        for (int y = 0; y < R; ++y) acc[x][y] = 0.f;
+    }
+    const int r = threadIdx.x / TPR, cg = threadIdx.x % TPR;
+    for (int ts = t0; ts < t1; ts += kTile) {
+        __syncthreads();
+        for (int e = threadIdx.x; e < kTile * D; e += kThreads) {
+            const int rr = e / D, c = e % D, t = ts + rr;
+            float x = 0.f, gg = 0.f;
+            if (t < t1) {
+                x = io<T>::ld(q + base + (long long)t * D + c);
+                gg = io<T>::ld(g + base + (long long)t * D + c);
+            }
+            qraw[rr * LD + c] = x;
+            qf[rr * LD + c] = (BIDIR && t < t1) ? feature(x) : x;
+            gs[rr * LD + c] = gg;
+        }
+        __syncthreads();
+        // Phase A: per-row outputs.
+        const int t = ts + r;
+        float n = eps;
+        float gdot = 0.f;
+        if (BIDIR) {
+            float u[CPT];
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) u[c] = 0.f;
+            for (int i = 0; i < D; ++i) {
+                const float qi = qf[r * LD + i];
+                n = fmaf(qi, z[i], n);
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) u[c] = fmaf(qi, S[i * LD + cg + TPR * c], u[c]);
+            }
+            if (t >= t1) n = 1.f;  // padded row: keep 0/0 out of the tile (its g is 0)
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) gdot = fmaf(gs[r * LD + cg + TPR * c], u[c] / n, gdot);
+#pragma unroll
+            for (int m = 1; m < TPR; m <<= 1) gdot += __shfl_xor_sync(0xffffffffu, gdot, m);
+        }
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+            const int i = cg + TPR * c;
+            float a = 0.f;
+            for (int j = 0; j < D; ++j) a = fmaf(gs[r * LD + j], S[i * LD + j], a);
+            if (BIDIR) a = (a - gdot * z[i]) / n * feature_grad(qraw[r * LD + i]);
+            if (t < t1) io<T>::st(dq + base + (long long)t * D + i, a);
+        }
+        __syncthreads();
+        if (BIDIR) {
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) gs[r * LD + cg + TPR * c] /= n;
+            if (cg == 0) wr[r] = t < t1 ? -gdot / n : 0.f;
+        }
+        __syncthreads();
+        // Phase B: dS += f(q)^T (g/n), dz += f(q)^T w.
+#pragma unroll 4
+        for (int rr = 0; rr < kTile; ++rr) {
+            float a[R], b[R];
+#pragma unroll
+            for (int x = 0; x < R; ++x) {
+                a[x] = qf[rr * LD + ti * R + x];
+                b[x] = gs[rr * LD + tj * R + x];
+            }
+            const float w = BIDIR ? wr[rr] : 0.f;
+#pragma unroll
+            for (int x = 0; x < R; ++x) {
+                if (BIDIR) zacc[x] = fmaf(a[x], w, zacc[x]);
+#pragma unroll
+                for (int y = 0; y < R; ++y) acc[x][y] = fmaf(a[x], b[y], acc[x][y]);
+            }
+        }
+    }
+    float *out = part + ((long long)bh * nsplit + split) * D * (D + 1);
+#pragma unroll
+    for (int x = 0; x < R; ++x) {
+#pragma unroll
+        for (int y = 0; y < R; ++y) out[(ti * R + x) * (D + 1) + tj * R + y] = acc[x][y];
+        if (tj == 0) out[(ti * R + x) * (D + 1) + D] = zacc[x];
+    }
+}
+
+// Key/value side: dk = (v dS^T + dz) f'(k),  dv = f(k) dS.
+template <typename T, int D, bool BIDIR>
+__global__ void __launch_bounds__(kThreads)
+bwd_k(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ dstate,
+      T *__restrict__ dk, T *__restrict__ dv, int T_len) {
+    constexpr int TPR = kThreads / kTile;
+    constexpr int CPT = D / TPR;
+    constexpr int LD = D + 1;
+    extern __shared__ float sm[];
+    float *dS = sm;                // D x LD
+    float *dz = dS + D * LD;       // D
+    float *kraw = dz + D;          // kTile x LD
+    float *kf = kraw + kTile * LD; // kTile x LD
+    float *vs = kf + kTile * LD;   // kTile x LD
+    const int bh = blockIdx.y;
+    const int row0 = blockIdx.x * kTile;
+    const long long base = (long long)bh * T_len * D;
+    const float *st = dstate + (long long)bh * D * (D + 1);
+    for (int e = threadIdx.x; e < D * D; e += kThreads) dS[(e / D) * LD + e % D] = st[(e / D) * (D + 1) + e % D];
+    for (int e = threadIdx.x; e < D; e += kThreads) dz[e] = BIDIR ? st[e * (D + 1) + D] : 0.f;
+    for (int e = threadIdx.x; e < kTile * D; e += kThreads) {
+        const int r = e / D, c = e % D, t = row0 + r;
+        float x = 0.f, y = 0.f;
+        if (t < T_len) {
+            x = io<T>::ld(k + base + (long long)t * D + c);
+            y = io<T>::ld(v + base + (long long)t * D + c);
+        }
+        kraw[r * LD + c] = x;
+        kf[r * LD + c] = BIDIR ? feature(x) : x;
+        vs[r * LD + c] = y;
+    }
+    __syncthreads();
+    const int r = threadIdx.x / TPR, cg = threadIdx.x % TPR, t = row0 + r;
+    if (t >= T_len) return;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int i = cg + TPR * c;
+        float a = dz[i];
+        for (int j = 0; j < D; ++j) a = fmaf(dS[i * LD + j], vs[r * LD + j], a);
+        if (BIDIR) a *= feature_grad(kraw[r * LD + i]);
+        io<T>::st(dk + base + (long long)t * D + i, a);
+    }
+    float acc[CPT];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) acc[c] = 0.f;
+    for (int i = 0; i < D; ++i) {
+        const float ki = kf[r * LD + i];
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) acc[c] = fmaf(ki, dS[i * LD + cg + TPR * c], acc[c]);
+    }
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) io<T>::st(dv + base + (long long)t * D + cg + TPR * c, acc[c]);
+}
+
+// ------------------------------------------------------------ retention ---
+
+// Loads rows [ts, ts+kRetTile) of up to four [T, D] tensors of one head into
+// fp32 shared tiles (zero past T).
+template <typename T, int D, int N>
+__device__ __forceinline__ void load_rows(const T *const (&src)[N], float (*dst)[kRetTile][D], long long base,
+                                          int ts, int T_len, int nthreads) {
+    for (int e = threadIdx.x; e < kRetTile * D; e += nthreads) {
+        const int r = e / D, c = e % D, t = ts + r;
+#pragma unroll
+        for (int m = 0; m < N; ++m)
+            dst[m][r][c] = t < T_len ? io<T>::ld(src[m] + base + (long long)t * D + c) : 0.f;
+    }
+}
+
+// Forward recurrence, thread j holds column j of S:
+//   S_t = gamma S_{t-1} + k_t^T v_t,   o_t[j] = sum_i q_t[i] S_t[i][j].
+template <typename T, int D>
+__global__ void __launch_bounds__(D)
+ret_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, T *__restrict__ o,
+        DecayArgs dec, int T_len, int H) {
+    __shared__ float tiles[3][kRetTile][D];
+    const int bh = blockIdx.x;
+    const float gamma = dec.gamma[bh % H];
+    const long long base = (long long)bh * T_len * D;
+    const int j = threadIdx.x;
+    float S[D];
+#pragma unroll
+    for (int i = 0; i < D; ++i) S[i] = 0.f;
+    const T *const src[3] = {q, k, v};
+    for (int ts = 0; ts < T_len; ts += kRetTile) {
+        __syncthreads();
+        load_rows<T, D, 3>(src, tiles, base, ts, T_len, D);
+        __syncthreads();
+        const int nr = min(kRetTile, T_len - ts);
+        for (int r = 0; r < nr; ++r) {
+            const float vj = tiles[2][r][j];
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < D; ++i) {
+                S[i] = fmaf(gamma, S[i], tiles[1][r][i] * vj);
+                acc = fmaf(tiles[0][r][i], S[i], acc);
+            }
+            io<T>::st(o + base + (long long)(ts + r) * D + j, acc);
+        }
+    }
+}
+
+// Backward, forward sweep, thread i holds row i of S: dq_t[i] = sum_j S_t[i][j] g_t[j].
+template <typename T, int D>
+__global__ void __launch_bounds__(D)
+ret_bwd_dq(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g, T *__restrict__ dq,
+           DecayArgs dec, int T_len, int H) {
+    __shared__ float tiles[3][kRetTile][D];
+    const int bh = blockIdx.x;
+    const float gamma = dec.gamma[bh % H];
+    const long long base = (long long)bh * T_len * D;
+    const int i = threadIdx.x;
+    float S[D];
+#pragma unroll
+    for (int j = 0; j < D; ++j) S[j] = 0.f;
+    const T *const src[3] = {k, v, g};
+    for (int ts = 0; ts < T_len; ts += kRetTile) {
+        __syncthreads();
+        load_rows<T, D, 3>(src, tiles, base, ts, T_len, D);
+        __syncthreads();
+        const int nr = min(kRetTile, T_len - ts);
+        for (int r = 0; r < nr; ++r) {
+            const float ki = tiles[0][r][i];
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < D; ++j) {
+                S[j] = fmaf(gamma, S[j], ki * tiles[1][r][j]);
+                acc = fmaf(S[j], tiles[2][r][j], acc);
+            }
+            io<T>::st(dq + base + (long long)(ts + r) * D + i, acc);
+        }
+    }
+}
+
+// Backward, reverse sweep over R_s = gamma R_{s+1} + q_s^T g_s.  Threads
+// 0..D-1 hold row i of R (dk_s[i] = sum_j R[i][j] v_s[j]); threads D..2D-1
+// hold column j of R (dv_s[j] = sum_i k_s[i] R[i][j]).
+template <typename T, int D>
+__global__ void __launch_bounds__(2 * D)
+ret_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+             const T *__restrict__ g, T *__restrict__ dk, T *__restrict__ dv, DecayArgs dec, int T_len, int H) {
+    __shared__ float tiles[4][kRetTile][D];
+    const int bh = blockIdx.x;
+    const float gamma = dec.gamma[bh % H];
+    const long long base = (long long)bh * T_len * D;
+    const bool row_side = threadIdx.x < D;
+    const int idx = row_side ? threadIdx.x : threadIdx.x - D;
+    float Rr[D];
+#pragma unroll
+    for (int m = 0; m < D; ++m) Rr[m] = 0.f;
+    const T *const src[4] = {q, k, v, g};
+    const int ntiles = (T_len + kRetTile - 1) / kRetTile;
+    for (int tile = ntiles - 1; tile >= 0; --tile) {
+        const int ts = tile * kRetTile;
+        __syncthreads();
+        load_rows<T, D, 4>(src, tiles, base, ts, T_len, 2 * D);
+        __syncthreads();
+        const int nr = min(kRetTile, T_len - ts);
+        for (int r = nr - 1; r >= 0; --r) {
+            float acc = 0.f;
+            if (row_side) {
+                const float qi = tiles[0][r][idx];
+#pragma unroll
+                for (int j = 0; j < D; ++j) {
+                    Rr[j] = fmaf(gamma, Rr[j], qi * tiles[3][r][j]);
+                    acc = fmaf(Rr[j], tiles[2][r][j], acc);
+                }
+                io<T>::st(dk + base + (long long)(ts + r) * D + idx, acc);
+            } else {
+                const float gj = tiles[3][r][idx];
+#pragma unroll
+                for (int i = 0; i < D; ++i) {
+                    Rr[i] = fmaf(gamma, Rr[i], tiles[0][r][i] * gj);
+                    acc = fmaf(tiles[1][r][i], Rr[i], acc);
+                }
+                io<T>::st(dv + base + (long long)(ts + r) * D + idx, acc);
+            }
+        }
+    }
+}
+
+// -------------------------------------------------------------- drivers ---
+
+namespace {
+
+int simt_splits(const Shape &s) { return state_splits(s, kTile); }
+
+template <typename T, int D>
+la_status state_fwd_t(bool bidir, const T *q, const T *k, const T *v, T *o, float *state, const Shape &s,
+                      float eps, void *ws, cudaStream_t st) {
+    const int nsplit = simt_splits(s);
+    const int rps = (s.T + nsplit - 1) / nsplit;
+    float *part = (float *)ws;
+    float *stt = state ? state : (float *)((char *)ws + state_bytes(s, nsplit));
+    const dim3 g1(nsplit, (unsigned)s.BH());
+    la_status rc = bidir ? launch("simt_state_partial", state_partial<T, D, true>, g1, dim3(kThreads), 0, st, k, v,
+                                  part, s.T, nsplit, rps)
+                         : launch("simt_state_partial", state_partial<T, D, false>, g1, dim3(kThreads), 0, st, k, v,
+                                  part, s.T, nsplit, rps);
+    if (rc) return rc;
+    rc = launch("simt_combine", combine, dim3((unsigned)s.BH()), dim3(kThreads), 0, st, (const float *)part, stt,
+                nsplit, D * (D + 1));
+    if (rc) return rc;
+    const size_t smem = (size_t)(D * D + D + kTile * (D + 1)) * sizeof(float);
+    const dim3 g2((s.T + kTile - 1) / kTile, (unsigned)s.BH());
+    return bidir ? launch("simt_output", output<T, D, true>, g2, dim3(kThreads), smem, st, q, (const float *)stt, o,
+                          s.T, eps)
+                 : launch("simt_output", output<T, D, false>, g2, dim3(kThreads), smem, st, q, (const float *)stt, o,
+                          s.T, eps);
+}
+
+template <typename T, int D>
+la_status state_bwd_t(bool bidir, const T *q, const T *k, const T *v, const T *g, const float *state, T *dq,
+                      T *dk, T *dv, const Shape &s, float eps, void *ws, cudaStream_t st) {
+    const int nsplit = simt_splits(s);
+    const int rps = (s.T + nsplit - 1) / nsplit;
+    char *w = (char *)ws;
+    float *part = (float *)w;
+    float *stt = (float *)(w + state_bytes(s, nsplit));
+    float *dstate = (float *)(w + state_bytes(s, nsplit) + state_bytes(s, 1));
+    la_status rc;
+    const dim3 g1(nsplit, (unsigned)s.BH());
+    if (!state) {
+        rc = bidir ? launch("simt_state_partial", state_partial<T, D, true>, g1, dim3(kThreads), 0, st, k, v, part,
+                            s.T, nsplit, rps)
+                   : launch("simt_state_partial", state_partial<T, D, false>, g1, dim3(kThreads), 0, st, k, v, part,
+                            s.T, nsplit, rps);
+        if (rc) return rc;
+        rc = launch("simt_combine", combine, dim3((unsigned)s.BH()), dim3(kThreads), 0, st, (const float *)part, stt,
+                    nsplit, D * (D + 1));
+        if (rc) return rc;
+        state = stt;
+    }
+    const size_t smemq = (size_t)(D * (D + 1) + D + 3 * kTile * (D + 1) + kTile) * sizeof(float);
+    rc = bidir ? launch("simt_bwd_q", bwd_q<T, D, true>, g1, dim3(kThreads), smemq, st, q, g, state, dq, part, s.T,
+                        nsplit, rps, eps)
+               : launch("simt_bwd_q", bwd_q<T, D, false>, g1, dim3(kThreads), smemq, st, q, g, state, dq, part, s.T,
+                        nsplit, rps, eps);
+    if (rc) return rc;
+    rc = launch("simt_combine", combine, dim3((unsigned)s.BH()), dim3(kThreads), 0, st, (const float *)part, dstate,
+                nsplit, D * (D + 1));
+    if (rc) return rc;
+    const size_t smemk = (size_t)(D * (D + 1) + D + 3 * kTile * (D + 1)) * sizeof(float);
+    const dim3 g2((s.T + kTile - 1) / kTile, (unsigned)s.BH());
+    return bidir ? launch("simt_bwd_k", bwd_k<T, D, true>, g2, dim3(kThreads), smemk, st, k, v,
+                          (const float *)dstate, dk, dv, s.T)
+                 : launch("simt_bwd_k", bwd_k<T, D, false>, g2, dim3(kThreads), smemk, st, k, v,
+                          (const float *)dstate, dk, dv, s.T);
+}
+
+template <typename T>
+la_status state_fwd_d(bool bidir, const void *q, const void *k, const void *v, void *o, float *state, const Shape &s,
+                      float eps, void *ws, cudaStream_t st) {
+    if (s.D == 64)
+        return state_fwd_t<T, 64>(bidir, (const T *)q, (const T *)k, (const T *)v, (T *)o, state, s, eps, ws, st);
+    return state_fwd_t<T, 128>(bidir, (const T *)q, (const T *)k, (const T *)v, (T *)o, state, s, eps, ws, st);
+}
+
+template <typename T>
+la_status state_bwd_d(bool bidir, const void *q, const void *k, const void *v, const void *g, const float *state,
+                      void *dq, void *dk, void *dv, const Shape &s, float eps, void *ws, cudaStream_t st) {
+    if (s.D == 64)
+        return state_bwd_t<T, 64>(bidir, (const T *)q, (const T *)k, (const T *)v, (const T *)g, state, (T *)dq,
+                                  (T *)dk, (T *)dv, s, eps, ws, st);
+    return state_bwd_t<T, 128>(bidir, (const T *)q, (const T *)k, (const T *)v, (const T *)g, state, (T *)dq,
+                               (T *)dk, (T *)dv, s, eps, ws, st);
+}
+
+template <typename T, int D>
+la_status decay_fwd_t(const T *q, const T *k, const T *v, T *o, const DecayArgs &dec, const Shape &s,
+                      cudaStream_t st) {
+    return launch("simt_ret_fwd", ret_fwd<T, D>, dim3((unsigned)s.BH()), dim3(D), 0, st, q, k, v, o, dec, s.T, s.H);
+}
+
+template <typename T, int D>
+la_status decay_bwd_t(const T *q, const T *k, const T *v, const T *g, const DecayArgs &dec, T *dq, T *dk, T *dv,
+                      const Shape &s, cudaStream_t st) {
+    la_status rc = launch("simt_ret_bwd_dq", ret_bwd_dq<T, D>, dim3((unsigned)s.BH()), dim3(D), 0, st, k, v, g, dq,
+                          dec, s.T, s.H);
+    if (rc) return rc;
+    return launch("simt_ret_bwd_dkdv", ret_bwd_dkdv<T, D>, dim3((unsigned)s.BH()), dim3(2 * D), 0, st, q, k, v, g,
+                  dk, dv, dec, s.T, s.H);
+}
+
+}  // namespace
+
+size_t workspace_size(la_op op, const Shape &s) {
+    switch (op) {
+    case LA_OP_BIDIR_FWD:
+    case LA_OP_SIMPLE_FWD:
+        return state_bytes(s, simt_splits(s)) + state_bytes(s, 1);
+    case LA_OP_BIDIR_BWD:
+    case LA_OP_SIMPLE_BWD:
+        return state_bytes(s, simt_splits(s)) + 2 * state_bytes(s, 1);
+    default:
+        return 0;
+    }
+}
+
+la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, void *o, float *state, const Shape &s,
+                    la_dtype dt, float eps, void *ws, cudaStream_t st) {
+    switch (dt) {
+    case LA_F32: return state_fwd_d<float>(bidir, q, k, v, o, state, s, eps, ws, st);
+    case LA_F16: return state_fwd_d<__half>(bidir, q, k, v, o, state, s, eps, ws, st);
+    default: return state_fwd_d<__nv_bfloat16>(bidir, q, k, v, o, state, s, eps, ws, st);
+    }
+}
+
+la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, const void *g, const float *state,
+                    void *dq, void *dk, void *dv, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st) {
+    switch (dt) {
+    case LA_F32: return state_bwd_d<float>(bidir, q, k, v, g, state, dq, dk, dv, s, eps, ws, st);
+    case LA_F16: return state_bwd_d<__half>(bidir, q, k, v, g, state, dq, dk, dv, s, eps, ws, st);
+    default: return state_bwd_d<__nv_bfloat16>(bidir, q, k, v, g, state, dq, dk, dv, s, eps, ws, st);
+    }
+}
+
+la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, const Shape &s,
+                    la_dtype dt, cudaStream_t st) {
+#define LA_RET_FWD(TY)                                                                                     \
+    return s.D == 64 ? decay_fwd_t<TY, 64>((const TY *)q, (const TY *)k, (const TY *)v, (TY *)o, dec, s, st) \
+                     : decay_fwd_t<TY, 128>((const TY *)q, (const TY *)k, (const TY *)v, (TY *)o, dec, s, st)
+    switch (dt) {
+    case LA_F32: LA_RET_FWD(float);
+    case LA_F16: LA_RET_FWD(__half);
+    default: LA_RET_FWD(__nv_bfloat16);
+    }
+#undef LA_RET_FWD
+}
+
+la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec, void *dq,
+                    void *dk, void *dv, const Shape &s, la_dtype dt, cudaStream_t st) {
+#define LA_RET_BWD(TY)                                                                                          \
+    return s.D == 64 ? decay_bwd_t<TY, 64>((const TY *)q, (const TY *)k, (const TY *)v, (const TY *)g, dec,       \
+                                           (TY *)dq, (TY *)dk, (TY *)dv, s, st)                                  \
+                     : decay_bwd_t<TY, 128>((const TY *)q, (const TY *)k, (const TY *)v, (const TY *)g, dec,      \
+                                            (TY *)dq, (TY *)dk, (TY *)dv, s, st)
+    switch (dt) {
+    case LA_F32: LA_RET_BWD(float);
+    case LA_F16: LA_RET_BWD(__half);
+    default: LA_RET_BWD(__nv_bfloat16);
+    }
+#undef LA_RET_BWD
+}
+
+}  // namespace simt
+}  // namespace la

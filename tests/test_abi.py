@@ -1,0 +1,101 @@
+"""The C ABI without a GPU: the library builds, loads and exports every declared
+entry point; arguments are validated before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "la.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tests.conftest import load_build_module
+    return ctypes.CDLL(load_build_module().build())
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(la_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_api():
+    names = declared_functions()
+    for n in ("la_bidir_fwd", "la_bidir_bwd", "la_simple_fwd", "la_simple_bwd", "la_chunk_decay_fwd",
+              "la_chunk_decay_bwd", "la_workspace_size", "la_status_string", "la_last_error"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, "not exported: %s" % missing
+
+
+def _binding():
+    import linear_attention_attn_b200 as la
+    return la
+
+
+def test_binding_names_match_abi():
+    la = _binding()
+    for n in declared_functions():
+        if n == "la_prof_collect" or n == "la_prof_enable" or n.startswith("la_"):
+            assert hasattr(la, n), "binding lacks %s" % n
+
+
+def test_workspace_size_is_deterministic():
+    la = _binding()
+    a = la.la_workspace_size("bidir_bwd", 8, 16, 4096, 64, la.LA_F16)
+    b = la.la_workspace_size("bidir_bwd", 8, 16, 4096, 64, la.LA_F16)
+    assert a == b and a > 0 and a % 256 == 0
+    assert la.la_workspace_size("bidir_fwd", 8, 16, 4096, 65, la.LA_F16) == 0
+    assert la.la_workspace_size("bidir_fwd", 0, 16, 4096, 64, la.LA_F16) == 0
+
+
+def _call_fwd(lib, q=0x1000, k=0x1000, v=0x1000, o=0x1000, B=1, H=1, T=16, D=64, dt=1, eps=1e-6,
+              ws=0x100000, wsb=1 << 30):
+    P = ctypes.c_void_p
+    f = lib.la_bidir_fwd
+    f.restype = ctypes.c_int
+    return f(P(q), P(k), P(v), P(o), P(0), B, H, T, D, dt, ctypes.c_float(eps), P(ws), ctypes.c_size_t(wsb), P(0))
+
+
+def test_validation_codes(lib):
+    # status codes as in include/la.h; none of these reach a CUDA call
+    assert _call_fwd(lib, D=65) == 2            # LA_ERR_UNSUPPORTED
+    assert _call_fwd(lib, dt=7) == 2
+    assert _call_fwd(lib, q=0) == 1             # LA_ERR_INVALID_ARG
+    assert _call_fwd(lib, B=0) == 1
+    assert _call_fwd(lib, T=-1) == 1
+    assert _call_fwd(lib, eps=-1.0) == 1
+    assert _call_fwd(lib, eps=float("nan")) == 1
+    assert _call_fwd(lib, k=0x1001) == 3        # LA_ERR_ALIGNMENT
+    assert _call_fwd(lib, ws=0) == 4            # LA_ERR_WORKSPACE
+    assert _call_fwd(lib, wsb=16) == 4
+    assert _call_fwd(lib, ws=0x100010) == 3     # workspace must be 256-byte aligned
+    lib.la_last_error.restype = ctypes.c_char_p
+    assert b"workspace" in lib.la_last_error()
+
+
+def test_decay_validation(lib):
+    P = ctypes.c_void_p
+    f = lib.la_chunk_decay_fwd
+    f.restype = ctypes.c_int
+    bad = (ctypes.c_float * 2)(0.5, 1.5)
+    assert f(P(0x1000), P(0x1000), P(0x1000), P(0x1000), ctypes.cast(bad, P), 1, 2, 16, 64, 2, P(0x100000),
+             ctypes.c_size_t(1 << 30), P(0)) == 1
+    assert f(P(0x1000), P(0x1000), P(0x1000), P(0x1000), P(0), 1, 2, 16, 64, 2, P(0x100000),
+             ctypes.c_size_t(1 << 30), P(0)) == 1
+    many = (ctypes.c_float * 600)(*([0.5] * 600))
+    assert f(P(0x1000), P(0x1000), P(0x1000), P(0x1000), ctypes.cast(many, P), 1, 600, 16, 64, 2, P(0x100000),
+             ctypes.c_size_t(1 << 30), P(0)) == 2
+
+
+def test_status_strings(lib):
+    lib.la_status_string.restype = ctypes.c_char_p
+    assert lib.la_status_string(0) == b"LA_OK"
+    assert lib.la_status_string(5) == b"LA_ERR_CUDA"
