@@ -112,9 +112,12 @@ size_t state_bytes(const Shape &s, long long copies) {
     return (b + 255) & ~(size_t)255;
 }
 
+static thread_local bool t_allow_null = false;   // set while validating a T == 0 call
+
 static bool path_tc(const Shape &s, la_dtype dt) { return tc::supports(s, dt); }
 
 static la_status validate(const Shape &s, la_dtype dt) {
+    t_allow_null = (s.T == 0);
     if (s.B < 1 || s.H < 1 || s.T < 0) return fail(LA_ERR_INVALID_ARG, "B, H must be >= 1 and T >= 0");
     if (dt != LA_F32 && dt != LA_F16 && dt != LA_BF16) return fail(LA_ERR_UNSUPPORTED, "unknown dtype %d", (int)dt);
     if (s.D != 64 && s.D != 128) return fail(LA_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", s.D);
@@ -125,6 +128,7 @@ static la_status validate(const Shape &s, la_dtype dt) {
 }
 
 static la_status check_ptr(const void *p, const char *name) {
+    if (!p && t_allow_null) return LA_OK;
     if (!p) return fail(LA_ERR_INVALID_ARG, "%s is NULL", name);
     if (((uintptr_t)p) & 15) return fail(LA_ERR_ALIGNMENT, "%s is not 16-byte aligned", name);
     return LA_OK;
