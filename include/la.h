@@ -89,6 +89,28 @@ la_status la_bidir_fwd(const void *q, const void *k, const void *v, void *o, flo
                        int B, int H, int T, int D, la_dtype dtype, float eps,
                        void *workspace, size_t workspace_bytes, void *stream);
 
+/* Size of the scratch array built into the library for la_bidir_fwd_static (32 MiB). */
+#define LA_STATIC_SCRATCH_BYTES (32u << 20)
+
+/* la_bidir_fwd without a workspace argument, for callers that cannot allocate
+ * device memory: code inside a host framework that owns the CUDA allocator and
+ * only hands out the tensors it manages, plugins in a serving process, or
+ * runtimes that may not call cudaMalloc after start-up.  (The pages describe no
+ * such entry point; it has no counterpart there.)
+ *  Arguments and results are those of la_bidir_fwd.  The scratch comes from a
+ *  LA_STATIC_SCRATCH_BYTES device array inside the library, which every GPU that
+ *  loads the library holds until the process exits.  This call allocates
+ *  nothing.
+ *  - Shapes whose la_workspace_size(LA_OP_BIDIR_FWD, ...) exceeds
+ *    LA_STATIC_SCRATCH_BYTES return LA_ERR_WORKSPACE (see la_last_error()).
+ *  - The first call on each device looks up the array's device address on that
+ *    device (the current one); make that first call before any stream capture.
+ *  - All calls share the array and it keeps the last call's contents; calls
+ *    that overlap on the GPU (unordered streams or host threads) race on it.
+ *    Nothing needs clearing between calls.                                    */
+la_status la_bidir_fwd_static(const void *q, const void *k, const void *v, void *o, float *state,
+                              int B, int H, int T, int D, la_dtype dtype, float eps, void *stream);
+
 /* Bidirectional linear attention, backward.
  *  dout     in  [B,H,T,D]: gradient of the loss with respect to o
  *  state    in  [B,H,D,D+1] fp32 from la_bidir_fwd with the same q,k,v, or

@@ -53,6 +53,8 @@ _lib.la_chunk_decay_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, 
 for _n in ("la_bidir_fwd", "la_simple_fwd", "la_bidir_bwd", "la_simple_bwd", "la_chunk_decay_fwd",
            "la_chunk_decay_bwd"):
     getattr(_lib, _n).restype = _I
+_lib.la_bidir_fwd_static.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
+_lib.la_bidir_fwd_static.restype = _I
 _lib.la_status_string.argtypes = [_I]
 _lib.la_status_string.restype = ctypes.c_char_p
 _lib.la_last_error.argtypes = []
@@ -153,6 +155,20 @@ def la_bidir_fwd(q, k, v, o, state=None, eps: float = 1e-6, workspace=None, stre
     wp, wn, _keep = _workspace("bidir_fwd", (B, H, T, D), dt, workspace, q.device, stream)
     _check(_lib.la_bidir_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), B, H, T, D, dt, float(eps),
                              wp, wn, _stream(stream, q.device)), "la_bidir_fwd")
+
+
+def la_bidir_fwd_static(q, k, v, o, state=None, eps: float = 1e-6, stream=None):
+    """la_bidir_fwd for callers that cannot allocate device memory: the scratch is a fixed
+    LA_STATIC_SCRATCH_BYTES array inside the library (shared by all calls; calls that
+    overlap on the GPU race).  No workspace is allocated here either."""
+    B, H, T, D = _shape(q, k, v, o)
+    _state_check(state, B, H, D, q.device)
+    dt = _dtype_code(q)
+    _check(_lib.la_bidir_fwd_static(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), B, H, T, D, dt, float(eps),
+                                    _stream(stream, q.device)), "la_bidir_fwd_static")
+
+
+STATIC_SCRATCH_BYTES = 32 << 20
 
 
 def la_simple_fwd(q, k, v, o, state=None, workspace=None, stream=None):
