@@ -286,6 +286,12 @@ def run_ours(args, w):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
+    if args.profile_only:
+        for _ in range(args.steps):
+            step()
+        torch.cuda.synchronize(dev)
+        la.la_device_check()
+        return 0
 
     # ---- timed region: K steps, device events, barriers on both sides
     if dist is not None:
@@ -401,6 +407,9 @@ def main(argv=None):
     ap.add_argument("--T", type=int, default=4096)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-only", action="store_true",
+                    help="run the warm-up and timed steps only (no e2e, CPU baseline or clock sampling): "
+                         "the command profiled under ncu")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

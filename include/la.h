@@ -60,7 +60,8 @@ typedef enum {
     LA_ERR_UNSUPPORTED = 2,   /* D not in {64, 128}, unknown dtype, too many heads for decay */
     LA_ERR_ALIGNMENT = 3,     /* a tensor or workspace pointer is not suitably aligned */
     LA_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than la_workspace_size() */
-    LA_ERR_CUDA = 5           /* a CUDA runtime call or kernel launch failed */
+    LA_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
+    LA_ERR_TIMEOUT = 6        /* a kernel gave up waiting on the GPU (see la_device_check) */
 } la_status;
 
 typedef enum {
@@ -153,6 +154,14 @@ la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const 
                              const float *decay, void *dq, void *dk, void *dv,
                              int B, int H, int T, int D, la_dtype dtype,
                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* Reports, and clears, the fault word of this library's tensor-core kernels on
+ * the current device.  Every wait inside those kernels is bounded (2 s); a wait
+ * that runs out makes the kernel wind down early (its outputs are then invalid)
+ * and sets the word.  Call it once the work of interest has completed (after a
+ * stream or device synchronisation).  Returns LA_OK, LA_ERR_TIMEOUT, or
+ * LA_ERR_CUDA if the word could not be read. */
+la_status la_device_check(void);
 
 /* Static text for a status code. */
 const char *la_status_string(la_status status);

@@ -29,7 +29,7 @@ LA_F32, LA_F16, LA_BF16 = 0, 1, 2
 OPS = {"bidir_fwd": 0, "bidir_bwd": 1, "simple_fwd": 2, "simple_bwd": 3,
        "chunk_decay_fwd": 4, "chunk_decay_bwd": 5}
 STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_ALIGNMENT",
-          4: "LA_ERR_WORKSPACE", 5: "LA_ERR_CUDA"}
+          4: "LA_ERR_WORKSPACE", 5: "LA_ERR_CUDA", 6: "LA_ERR_TIMEOUT"}
 MAX_DECAY_HEADS = 512
 
 _P = ctypes.c_void_p
@@ -59,6 +59,8 @@ _lib.la_status_string.argtypes = [_I]
 _lib.la_status_string.restype = ctypes.c_char_p
 _lib.la_last_error.argtypes = []
 _lib.la_last_error.restype = ctypes.c_char_p
+_lib.la_device_check.argtypes = []
+_lib.la_device_check.restype = _I
 _lib.la_launch_count.argtypes = []
 _lib.la_launch_count.restype = ctypes.c_longlong
 _lib.la_prof_enable.argtypes = [_I]
@@ -235,6 +237,11 @@ def la_status_string(status: int) -> str:
 
 def la_last_error() -> str:
     return _lib.la_last_error().decode(errors="replace")
+
+
+def la_device_check() -> None:
+    """Raise LAError if a tensor-core kernel gave up waiting since the last check."""
+    _check(_lib.la_device_check(), "la_device_check")
 
 
 def la_launch_count() -> int:

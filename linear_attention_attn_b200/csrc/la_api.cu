@@ -114,7 +114,7 @@ size_t state_bytes(const Shape &s, long long copies) {
 
 static thread_local bool t_allow_null = false;   // set while validating a T == 0 call
 
-static bool path_tc(const Shape &s, la_dtype dt) { return tc::supports(s, dt); }
+static bool path_tc(la_op op, const Shape &s, la_dtype dt) { return tc::supports(op, s, dt); }
 
 static la_status validate(const Shape &s, la_dtype dt) {
     t_allow_null = (s.T == 0);
@@ -135,7 +135,7 @@ static la_status check_ptr(const void *p, const char *name) {
 }
 
 static size_t ws_size(la_op op, const Shape &s, la_dtype dt) {
-    if (path_tc(s, dt)) return tc::workspace_size(op, s, dt);
+    if (path_tc(op, s, dt)) return tc::workspace_size(op, s, dt);
     return simt::workspace_size(op, s);
 }
 
@@ -176,7 +176,7 @@ static la_status state_fwd_entry(bool bidir, const void *q, const void *k, const
         }
         return LA_OK;
     }
-    if (path_tc(s, dt)) return tc::state_fwd(bidir, q, k, v, o, state, s, dt, eps, ws, st);
+    if (path_tc(op, s, dt)) return tc::state_fwd(bidir, q, k, v, o, state, s, dt, eps, ws, st);
     return simt::state_fwd(bidir, q, k, v, o, state, s, dt, eps, ws, st);
 }
 
@@ -198,7 +198,7 @@ static la_status state_bwd_entry(bool bidir, const void *q, const void *k, const
     LA_TRY(check_ws(op, s, dt, ws, ws_bytes));
     if (T == 0) return LA_OK;
     cudaStream_t st = (cudaStream_t)stream;
-    if (path_tc(s, dt)) return tc::state_bwd(bidir, q, k, v, g, state, dq, dk, dv, s, dt, eps, ws, st);
+    if (path_tc(op, s, dt)) return tc::state_bwd(bidir, q, k, v, g, state, dq, dk, dv, s, dt, eps, ws, st);
     return simt::state_bwd(bidir, q, k, v, g, state, dq, dk, dv, s, dt, eps, ws, st);
 }
 
@@ -265,7 +265,7 @@ la_status la_chunk_decay_fwd(const void *q, const void *k, const void *v, void *
     LA_TRY(check_ws(LA_OP_CHUNK_DECAY_FWD, s, dtype, workspace, workspace_bytes));
     if (T == 0) return LA_OK;
     cudaStream_t st = (cudaStream_t)stream;
-    if (path_tc(s, dtype)) return tc::decay_fwd(q, k, v, o, dec, s, dtype, workspace, st);
+    if (path_tc(LA_OP_CHUNK_DECAY_FWD, s, dtype)) return tc::decay_fwd(q, k, v, o, dec, s, dtype, workspace, st);
     return simt::decay_fwd(q, k, v, o, dec, s, dtype, st);
 }
 
@@ -286,7 +286,7 @@ la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const 
     LA_TRY(check_ws(LA_OP_CHUNK_DECAY_BWD, s, dtype, workspace, workspace_bytes));
     if (T == 0) return LA_OK;
     cudaStream_t st = (cudaStream_t)stream;
-    if (path_tc(s, dtype)) return tc::decay_bwd(q, k, v, dout, dec, dq, dk, dv, s, dtype, workspace, st);
+    if (path_tc(LA_OP_CHUNK_DECAY_BWD, s, dtype)) return tc::decay_bwd(q, k, v, dout, dec, dq, dk, dv, s, dtype, workspace, st);
     return simt::decay_bwd(q, k, v, dout, dec, dq, dk, dv, s, dtype, st);
 }
 
@@ -298,11 +298,19 @@ const char *la_status_string(la_status status) {
     case LA_ERR_ALIGNMENT: return "LA_ERR_ALIGNMENT";
     case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE";
     case LA_ERR_CUDA: return "LA_ERR_CUDA";
+    case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT";
     }
     return "LA_ERR_UNKNOWN";
 }
 
 const char *la_last_error(void) { return g_last_error.c_str(); }
+
+la_status la_device_check(void) {
+    const unsigned int f = tc::read_and_clear_fault();
+    if (f == 0xFFFFFFFFu) return fail(LA_ERR_CUDA, "could not read the device fault word");
+    if (f) return fail(LA_ERR_TIMEOUT, "a tensor-core kernel wait ran out (fault bits 0x%08x)", f);
+    return LA_OK;
+}
 
 long long la_launch_count(void) { return g_launches.load(); }
 

@@ -1,19 +1,30 @@
-// la_tc.cu -- tensor-core path dispatch.
+// la_tc.cu -- which ops and shapes the tensor-core path covers, and its workspace.
 #include "la_tc.cuh"
 
 namespace la {
 namespace tc {
 
-bool supports(const Shape &, la_dtype) { return false; }
-size_t workspace_size(la_op, const Shape &, la_dtype) { return 0; }
-la_status state_fwd(bool, const void *, const void *, const void *, void *, float *, const Shape &, la_dtype, float,
-                    void *, cudaStream_t) {
-    return LA_ERR_UNSUPPORTED;
+bool supports(la_op op, const Shape &s, la_dtype dt) {
+    if (dt != LA_F16 && dt != LA_BF16) return false;
+    switch (op) {
+    case LA_OP_BIDIR_FWD:
+    case LA_OP_BIDIR_BWD:
+    case LA_OP_SIMPLE_FWD:
+    case LA_OP_SIMPLE_BWD: return s.D == 64;
+    default: return false;
+    }
 }
-la_status state_bwd(bool, const void *, const void *, const void *, const void *, const float *, void *, void *,
-                    void *, const Shape &, la_dtype, float, void *, cudaStream_t) {
-    return LA_ERR_UNSUPPORTED;
+
+size_t workspace_size(la_op op, const Shape &s, la_dtype) {
+    switch (op) {
+    case LA_OP_BIDIR_FWD:
+    case LA_OP_BIDIR_BWD:
+    case LA_OP_SIMPLE_FWD:
+    case LA_OP_SIMPLE_BWD: return state_workspace_size(op, s);
+    default: return 0;
+    }
 }
+
 la_status decay_fwd(const void *, const void *, const void *, void *, const DecayArgs &, const Shape &, la_dtype,
                     void *, cudaStream_t) {
     return LA_ERR_UNSUPPORTED;

@@ -1,0 +1,219 @@
+// la_tc_common.cuh -- pieces shared by the tensor-core kernels: the persistent tile
+// partition, the 16-bit element helpers, the feature-map transform of a swizzled
+// tile, state gathering and operand building.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "la_internal.cuh"
+#include "la_tc_ptx.cuh"
+
+namespace la {
+namespace tc {
+
+constexpr int kGrid = 148;          // persistent CTAs; fixed so partial-slot layout depends on the shape only
+constexpr int kRows = 128;          // rows of q/k/v per tile (the UMMA M of the row-wise products)
+constexpr int kThreads = 192;       // warp 0: TMA producer, warp 1: UMMA issuer + TMEM, warps 2..5: workers
+constexpr int kWorkers = 128;
+constexpr int kTileBytes = kRows * 128;   // 128 rows x 64 16-bit elements, 128-byte swizzled
+constexpr int kStateElems = 64 * 65;      // one fp32 [64][65] state block: S | z
+
+// ------------------------------------------------------------- partition --
+// Tiles of all heads, head-major (x = h * nt + j), split into G contiguous
+// ranges with G = min(kGrid, N): CTA c takes [start(c), start(c+1)), never
+// empty.  The CTAs touching head h are first_cta(h) .. last_cta(h); CTA c writes
+// its partial of head h into slot c - first_cta(h), so a head's slots are
+// 0 .. last_cta(h) - first_cta(h), all written.
+struct Partition {
+    long long N;
+    int nt;
+    int G;
+    __host__ __device__ long long start(int c) const { return (long long)c * N / G; }
+    __host__ __device__ int cta_of(long long x) const { return (int)(((x + 1) * G - 1) / N); }
+    __host__ __device__ int first_cta(int h) const { return cta_of((long long)h * nt); }
+    __host__ __device__ int last_cta(int h) const { return cta_of((long long)h * nt + nt - 1); }
+};
+
+__host__ __device__ inline int grid_for(long long N) { return N < kGrid ? (int)N : kGrid; }
+
+// Upper bound of last_cta(h) - first_cta(h) + 1 over heads (G <= kGrid CTAs over BH heads).
+__host__ __device__ inline int max_slots(int BH) { return (kGrid + BH - 1) / BH + 1; }
+
+// ------------------------------------------------------------ 16-bit I/O --
+template <bool BF16> struct h2;
+template <> struct h2<false> {
+    static __device__ __forceinline__ float2 to_f2(uint32_t u) {
+        __half2 h = *reinterpret_cast<__half2 *>(&u);
+        return __half22float2(h);
+    }
+    static __device__ __forceinline__ uint32_t from_f2(float a, float b) {
+        __half2 h = __floats2half2_rn(a, b);
+        return *reinterpret_cast<uint32_t *>(&h);
+    }
+    static __device__ __forceinline__ uint16_t one() { return 0x3C00u; }
+};
+template <> struct h2<true> {
+    static __device__ __forceinline__ float2 to_f2(uint32_t u) {
+        __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162 *>(&u);
+        return __bfloat1622float2(h);
+    }
+    static __device__ __forceinline__ uint32_t from_f2(float a, float b) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<uint32_t *>(&h);
+    }
+    static __device__ __forceinline__ uint16_t one() { return 0x3F80u; }
+};
+
+__device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+
+// Feature map elu+1 applied in place to row `row` of a 128-byte-swizzled tile
+// (the row's 8 chunks are visited in an order that spreads banks); rows that
+// lie past the sequence end are zeroed when `zero` is set.
+template <bool BF16>
+__device__ __forceinline__ void phi_row_inplace(uint8_t *tile, int row, bool zero) {
+    uint8_t *p = tile + row * 128;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        uint4 *c = reinterpret_cast<uint4 *>(p + ((it ^ (row & 7)) << 4));
+        uint4 u = *c;
+        if (zero) {
+            u = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+            uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float2 f = h2<BF16>::to_f2(w[k]);
+                w[k] = h2<BF16>::from_f2(phi_f(f.x), phi_f(f.y));
+            }
+            u = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        *c = u;
+    }
+}
+
+// Feature map with a two-term result: hi = round(phi(x)) replaces x in place,
+// lo = round(phi(x) - hi) goes to the same position of `lo_tile`.
+template <bool BF16>
+__device__ __forceinline__ void phi_row_split(uint8_t *tile, uint8_t *lo_tile, int row) {
+    uint8_t *p = tile + row * 128;
+    uint8_t *q = lo_tile + row * 128;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        const int off = (it ^ (row & 7)) << 4;
+        uint4 u = *reinterpret_cast<uint4 *>(p + off);
+        uint32_t w[4] = {u.x, u.y, u.z, u.w}, l[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float2 f = h2<BF16>::to_f2(w[k]);
+            const float a = phi_f(f.x), b = phi_f(f.y);
+            w[k] = h2<BF16>::from_f2(a, b);
+            const float2 hv = h2<BF16>::to_f2(w[k]);
+            l[k] = h2<BF16>::from_f2(a - hv.x, b - hv.y);
+        }
+        *reinterpret_cast<uint4 *>(p + off) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4 *>(q + off) = make_uint4(l[0], l[1], l[2], l[3]);
+    }
+}
+
+// Reads the 64 elements of row `row` of a swizzled 16-bit tile into fp32.
+template <bool BF16>
+__device__ __forceinline__ void load_row(const uint8_t *tile, int row, float (&out)[64]) {
+    const uint8_t *p = tile + row * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint4 u = *reinterpret_cast<const uint4 *>(p + ((c ^ (row & 7)) << 4));
+        float2 a = h2<BF16>::to_f2(u.x), b = h2<BF16>::to_f2(u.y), d = h2<BF16>::to_f2(u.z),
+               e = h2<BF16>::to_f2(u.w);
+        out[c * 8 + 0] = a.x; out[c * 8 + 1] = a.y; out[c * 8 + 2] = b.x; out[c * 8 + 3] = b.y;
+        out[c * 8 + 4] = d.x; out[c * 8 + 5] = d.y; out[c * 8 + 6] = e.x; out[c * 8 + 7] = e.y;
+    }
+}
+
+// Writes 64 fp32 values as row `row` of a swizzled 16-bit tile (round to nearest even).
+template <bool BF16>
+__device__ __forceinline__ void store_row(uint8_t *tile, int row, const float (&v)[64]) {
+    uint8_t *p = tile + row * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint4 u;
+        u.x = h2<BF16>::from_f2(v[c * 8 + 0], v[c * 8 + 1]);
+        u.y = h2<BF16>::from_f2(v[c * 8 + 2], v[c * 8 + 3]);
+        u.z = h2<BF16>::from_f2(v[c * 8 + 4], v[c * 8 + 5]);
+        u.w = h2<BF16>::from_f2(v[c * 8 + 6], v[c * 8 + 7]);
+        *reinterpret_cast<uint4 *>(p + ((c ^ (row & 7)) << 4)) = u;
+    }
+}
+
+// 64 fp32 accumulator columns [col, col+64) of this warp's TMEM lanes.
+__device__ __forceinline__ void tmem_row64(uint32_t taddr, float (&v)[64]) {
+    float a[16], b[16], c[16], d[16];
+    tmem_ld16(taddr + 0, a);
+    tmem_ld16(taddr + 16, b);
+    tmem_ld16(taddr + 32, c);
+    tmem_ld16(taddr + 48, d);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        v[i] = a[i];
+        v[16 + i] = b[i];
+        v[32 + i] = c[i];
+        v[48 + i] = d[i];
+    }
+}
+
+// ------------------------------------------------------------- state I/O --
+// stage[e] = sum over s in [0, nslots) of src[s * kStateElems + e], in slot order
+// (a fixed order: the result does not depend on which CTA finished first).
+// Returns this thread's max |stage[e]| over the elements it summed.
+__device__ __forceinline__ float gather_state(const float *__restrict__ src, int nslots, float *stage, int tid) {
+    float m = 0.f;
+    for (int e = tid; e < kStateElems; e += kWorkers) {
+        float acc = 0.f;
+        for (int s = 0; s < nslots; ++s) acc += src[(long long)s * kStateElems + e];
+        stage[e] = acc;
+        m = fmaxf(m, fabsf(acc));
+    }
+    return m;
+}
+
+// Max over the 128 worker threads (named barrier 2); `red` is 4 floats of smem.
+__device__ __forceinline__ float workers_max(float m, float *red, int tid) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) red[tid >> 5] = m;
+    named_bar(2, kWorkers);
+    m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    named_bar(2, kWorkers);
+    return m;
+}
+
+// Power-of-two scale that puts max |x| = m in [2^13, 2^14) for fp16 operands
+// (range and subnormal safety); bf16 shares fp32's range and needs none.
+template <bool BF16>
+__device__ __forceinline__ float operand_scale(float m) {
+    if (BF16 || !(m > 0.f) || !isfinite(m)) return 1.f;
+    int e;
+    frexpf(m, &e);                        // m = f * 2^e, f in [0.5, 1)
+    e = 14 - e;
+    e = e < -100 ? -100 : (e > 100 ? 100 : e);
+    return ldexpf(1.f, e);
+}
+
+// One row of a K-major 128-byte-swizzled 16-bit operand from 64 fp32 values
+// scaled by sc: hi = round(x), lo = round(x - hi) (lo only with NOPS == 2).
+template <bool BF16, int NOPS>
+__device__ __forceinline__ void operand_row(uint8_t *op0, uint8_t *op1, int row, const float (&x)[64]) {
+    float hi[64];
+    store_row<BF16>(op0, row, x);
+    if (NOPS == 2) {
+        load_row<BF16>(op0, row, hi);
+        float lo[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) lo[i] = x[i] - hi[i];
+        store_row<BF16>(op1, row, lo);
+    }
+}
+
+}  // namespace tc
+}  // namespace la

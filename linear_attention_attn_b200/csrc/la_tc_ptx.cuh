@@ -51,6 +51,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // CTA's abort flag and the module's fault word, and the kernel winds down.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// abort_flag may be null: the wait then ignores aborts and ends only on
+// completion or on the time limit (used to drain copies and UMMAs in flight).
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                             unsigned int *fault_word, unsigned int code) {
     const uint64_t t0 = globaltimer_ns();
@@ -58,10 +60,10 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volat
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
+        if (abort_flag && *abort_flag) return false;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            atomicOr(fault_word, code);
+            if (abort_flag) *abort_flag = 1;
+            atomicOr(fault_word, code | 0x80000000u);
             return false;
         }
     }

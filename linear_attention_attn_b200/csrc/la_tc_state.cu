@@ -1,0 +1,1258 @@
+// la_tc_state.cu -- tensor-core kernels of bidirectional linear attention and simple_la
+// (fp16 / bf16 storage, D = 64, fp32 accumulation in TMEM).
+//
+// "Flash Bi-directional Linear Attention" README (intro; "Update": simple_la is
+// linear_attn without the norm term).  Forward, with f = elu+1 (bidir) or the
+// identity (simple):
+//   state_reduce:  S = sum_t f(k_t)^T v_t, z = sum_t f(k_t)     (per CTA partial, fp32)
+//   output:        o_t = f(q_t) S / (f(q_t).z + eps)  (bidir)  |  q_t S  (simple)
+// Backward (hand-derived; see include/la.h):
+//   bwd_q:   n_t, o_t recomputed; dq_t = (g_t S^T - (g_t.o_t) z)/n_t * f'(q_t);
+//            partial dS = sum_t f(q_t)^T g_t/n_t, dz = -sum_t f(q_t)(g_t.o_t)/n_t
+//   bwd_kv:  dk_s = (v_s dS^T + dz) * f'(k_s),  dv_s = f(k_s) dS
+//
+// Every kernel is persistent: kGrid CTAs split the head-major list of 128-row
+// tiles into contiguous ranges (Partition).  Warp 0 streams q/k/v/dO tiles with
+// TMA into a ring of 128-byte-swizzled stages; warp 1 issues tcgen05 UMMAs
+// (fp32 accumulators in TMEM); warps 2..5 apply the feature map in place, run
+// the epilogues (TMEM -> registers -> swizzled staging -> TMA store) and build
+// the per-head state operand.  A reduction's per-CTA partial goes to slot
+// (cta - first_cta(head)) of the workspace; its consumer sums the slots in slot
+// order, so results are deterministic.
+//
+// The D x D state operand of the row-wise products is stored K-major with the
+// state's column index as the row: row n holds S[0..63][n], row 64 holds z.
+// Read K-major it is [S | z]^T (for f(q)[S | z]); read MN-major (its first 64
+// rows) it is S (for g S^T).  fp16 operands carry a power-of-two scale chosen
+// per head (range); bf16 operands are split hi + lo (precision).
+#include "la_tc.cuh"
+#include "la_tc_common.cuh"
+
+#include <cudaTypedefs.h>
+#include <mutex>
+
+namespace la {
+namespace tc {
+
+// Fault word of the tensor-core kernels (a wait ran out): read by la_device_check().
+__device__ unsigned int g_tc_fault = 0;
+
+namespace {
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+#ifndef LA_TRY
+#define LA_TRY(x)                     \
+    do {                              \
+        la_status _rc = (x);          \
+        if (_rc != LA_OK) return _rc; \
+    } while (0)
+#endif
+
+// Waits used by every role; codes identify the barrier in the fault word.
+#define LA_WAIT(bar, par, code) mbar_wait((bar), (par), s_abort, &g_tc_fault, (code))
+
+// ============================================================ state_reduce ==
+// Partial (S | z) of every (CTA, head) segment.  UMMA M = 64 (the state row i),
+// N = 64 (+16 with the ones block that yields z), K = 128 tile rows:
+//   A = f(K)^T read MN-major from the k tile, B = [V | 1] read MN-major.
+template <bool BIDIR, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    float *__restrict__ part, int T, int BH, int nt, int maxslots) {
+    constexpr bool KLO = BIDIR && BF16;      // bf16: f(k) = hi + lo, both multiplied in
+    constexpr int NST = KLO ? 3 : 4;
+    constexpr int N = BIDIR ? 80 : 64;
+    constexpr uint32_t IDESC = idesc_f16(64, N, BF16, true, true);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *sK = smem;
+    uint8_t *sV = sK + NST * kTileBytes;
+    uint8_t *sOnes = sV + NST * kTileBytes;
+    uint8_t *sKlo = sOnes + kTileBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sKlo + (KLO ? NST * kTileBytes : 0));
+    uint64_t *xf = full + NST;
+    uint64_t *empty = xf + NST;
+    uint64_t *accfull = empty + NST;   // [2]
+    uint64_t *accfree = accfull + 2;   // [2]
+    uint64_t *drain = accfree + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Partition P{(long long)BH * nt, nt, grid_for((long long)BH * nt)};
+    const int cta = blockIdx.x;
+    const long long x0 = P.start(cta), x1 = P.start(cta + 1);
+    if (x0 >= x1) return;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&xf[s], 4);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&accfull[a], 1);
+            mbar_init(&accfree[a], 4);
+        }
+        mbar_init(drain, 1);
+        *s_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch(&tmK);
+        tma_prefetch(&tmV);
+    }
+    if (BIDIR && warp >= 2) {
+        // ones block: column 0 (state column 64) = 1 for every tile row, zeros elsewhere
+        const int r = threadIdx.x - 64;
+        uint8_t *p = sOnes + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(p + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint16_t *>(sOnes + sw128_offset(r, 0)) = h2<BF16>::one();
+        fence_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            long long issued = 0;
+            for (long long x = x0; x < x1; ++x) {
+                const int h = (int)(x / nt), j = (int)(x % nt);
+                if (!LA_WAIT(&empty[s], ph ^ 1, 0x1u)) break;
+                mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
+                tma_load_3d(sK + s * kTileBytes, &tmK, &full[s], 0, j * kRows, h);
+                tma_load_3d(sV + s * kTileBytes, &tmV, &full[s], 0, j * kRows, h);
+                ++issued;
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+            // on an abort, let the loads in flight land before the CTA's smem goes away
+            if (*s_abort) {
+                for (long long i = issued - 1; i >= 0 && i >= issued - NST; --i)
+                    mbar_wait_slow(smem_u32(&full[i % NST]), (uint32_t)((i / NST) & 1), nullptr, &g_tc_fault, 0x200u);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int s = 0, a = 0;
+            uint32_t ph = 0, aph = 0;
+            bool seg_start = true;
+            for (long long x = x0; x < x1; ++x) {
+                const long long h = x / nt;
+                const bool seg_end = (x + 1 == x1) || ((x + 1) / nt != h);
+                if (seg_start) {
+                    if (!LA_WAIT(&accfree[a], aph ^ 1, 0x2u)) break;
+                }
+                if (!LA_WAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)a * 128u;
+                const uint32_t aK = smem_u32(sK + s * kTileBytes), aV = smem_u32(sV + s * kTileBytes);
+                const uint32_t lbo = BIDIR ? (smem_u32(sOnes) - aV) : (uint32_t)kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kRows / 16; ++kk) {
+                    const uint64_t ad = sdesc_sw128(aK + kk * 2048, kTileBytes, 1024);
+                    const uint64_t bd = sdesc_sw128(aV + kk * 2048, lbo, 1024);
+                    umma_f16_ss(d, ad, bd, IDESC, (seg_start && kk == 0) ? 0u : 1u);
+                    if (KLO)
+                        umma_f16_ss(d, sdesc_sw128(smem_u32(sKlo + s * kTileBytes) + kk * 2048, kTileBytes, 1024), bd,
+                                    IDESC, 1u);
+                }
+                umma_commit(&empty[s]);
+                if (seg_end) {
+                    umma_commit(&accfull[a]);
+                    a ^= 1;
+                    if (a == 0) aph ^= 1;
+                }
+                seg_start = seg_end;
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+            umma_commit(drain);
+            mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+        }
+    } else {
+        const int sub = warp & 3;                 // TMEM subpartition of this warp
+        const int row = sub * 32 + lane;          // tile row this thread transforms
+        int s = 0, a = 0;
+        uint32_t ph = 0, aph = 0;
+        for (long long x = x0; x < x1; ++x) {
+            const int h = (int)(x / nt), j = (int)(x % nt);
+            const bool seg_end = (x + 1 == x1) || ((x + 1) / nt != h);
+            if (BIDIR) {
+                const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
+                if (!got) break;
+                if (KLO) {
+                    if (j * kRows + row >= T) {
+                        phi_row_inplace<BF16>(sK + s * kTileBytes, row, true);
+                        phi_row_inplace<BF16>(sKlo + s * kTileBytes, row, true);
+                    } else {
+                        phi_row_split<BF16>(sK + s * kTileBytes, sKlo + s * kTileBytes, row);
+                    }
+                } else {
+                    phi_row_inplace<BF16>(sK + s * kTileBytes, row, j * kRows + row >= T);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xf[s]);
+            }
+            if (++s == NST) { s = 0; ph ^= 1; }
+            if (seg_end) {
+                const bool got = __all_sync(0xffffffffu, LA_WAIT(&accfull[a], aph, 0x10u));
+                if (!got) break;
+                tc_fence_after();
+                // M = 64 accumulator: state row i = 16*sub + l sits in TMEM lane 32*sub + l (l < 16)
+                const uint32_t base = tmem + (uint32_t)a * 128u + ((uint32_t)(32 * sub) << 16);
+                float v[64];
+                tmem_row64(base, v);
+                float zz = 0.f;
+                if (BIDIR) {
+                    float t16[16];
+                    tmem_ld16(base + 64, t16);
+                    tmem_ld_wait();
+                    zz = t16[0];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accfree[a]);
+                if (lane < 16) {
+                    const int i = 16 * sub + lane;
+                    const int slot = cta - P.first_cta(h);
+                    float *dst = part + (((long long)h * maxslots + slot) * 64 + i) * 65;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) dst[c] = v[c];
+                    dst[64] = zz;
+                }
+                a ^= 1;
+                if (a == 0) aph ^= 1;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ================================================================= output ==
+// o = f(q) [S | z] / n per tile: UMMA M = 128 rows, N = 80 (64 + z + pad) or 64,
+// K = 64, A = f(Q) tile K-major, B = state operand K-major (hi [+ lo]).
+template <bool BIDIR, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+              const float *__restrict__ src, int src_per_head, int src_single, float *__restrict__ state_out, int T,
+              int BH, int nt, float eps) {
+    constexpr int NST = 4;
+    constexpr int OST = 2;
+    constexpr int NOPS = BF16 ? 2 : 1;
+    constexpr int N = BIDIR ? 80 : 64;
+    constexpr int OPB = 80 * 128;                 // operand bytes (80 rows)
+    constexpr uint32_t IDESC = idesc_f16(128, N, BF16, false, false);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *sQ = smem;
+    uint8_t *sO = sQ + NST * kTileBytes;
+    uint8_t *sOp = sO + OST * kTileBytes;          // NOPS x OPB (1024-aligned: OPB = 10 x 1024)
+    float *stage = reinterpret_cast<float *>(sOp + 2 * OPB);
+    float *red = stage + kStateElems;
+    uint64_t *full = reinterpret_cast<uint64_t *>(red + 8);
+    uint64_t *xf = full + NST;
+    uint64_t *empty = xf + NST;
+    uint64_t *accfull = empty + NST;
+    uint64_t *accempty = accfull + 2;
+    uint64_t *opready = accempty + 2;
+    uint64_t *drain = opready + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
+    float *s_scale = reinterpret_cast<float *>(s_abort + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Partition P{(long long)BH * nt, nt, grid_for((long long)BH * nt)};
+    const int cta = blockIdx.x;
+    const long long x0 = P.start(cta), x1 = P.start(cta + 1);
+    if (x0 >= x1) return;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&xf[s], 4);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&accfull[a], 1);
+            mbar_init(&accempty[a], 4);
+        }
+        mbar_init(opready, 1);
+        mbar_init(drain, 1);
+        *s_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch(&tmQ);
+        tma_prefetch(&tmO);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            long long issued = 0;
+            for (long long x = x0; x < x1; ++x) {
+                const int h = (int)(x / nt), j = (int)(x % nt);
+                if (!LA_WAIT(&empty[s], ph ^ 1, 0x1u)) break;
+                mbar_arrive_expect_tx(&full[s], kTileBytes);
+                tma_load_3d(sQ + s * kTileBytes, &tmQ, &full[s], 0, j * kRows, h);
+                ++issued;
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+            if (*s_abort) {
+                for (long long i = issued - 1; i >= 0 && i >= issued - NST; --i)
+                    mbar_wait_slow(smem_u32(&full[i % NST]), (uint32_t)((i / NST) & 1), nullptr, &g_tc_fault, 0x200u);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int s = 0, a = 0;
+            uint32_t ph = 0, aph = 0, oph = 0;
+            long long prev_h = -1;
+            for (long long x = x0; x < x1; ++x) {
+                const long long h = x / nt;
+                if (h != prev_h) {
+                    if (!LA_WAIT(opready, oph, 0x20u)) break;
+                    oph ^= 1;
+                    prev_h = h;
+                }
+                if (!LA_WAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
+                if (!LA_WAIT(&accempty[a], aph ^ 1, 0x2u)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)a * 128u;
+                const uint32_t aQ = smem_u32(sQ + s * kTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                    for (int op = 0; op < NOPS; ++op) {
+                        const uint64_t ad = sdesc_sw128(aQ + kk * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(smem_u32(sOp + op * OPB) + kk * 32, 16, 1024);
+                        umma_f16_ss(d, ad, bd, IDESC, (kk | op) ? 1u : 0u);
+                    }
+                }
+                umma_commit(&empty[s]);
+                umma_commit(&accfull[a]);
+                a ^= 1;
+                if (a == 0) aph ^= 1;
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+            umma_commit(drain);
+            mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+        }
+    } else {
+        // Workers.  Every named barrier below is reached by all 128 workers whatever
+        // happens to the mbarrier waits (a failed wait only skips the work), so an
+        // abort cannot leave a worker stuck at a barrier.
+        const int tid = threadIdx.x - 64;          // 0..127
+        const int sub = warp & 3;
+        const int row = sub * 32 + lane;
+        int s = 0, a = 0, ob = 0;
+        uint32_t ph = 0, aph = 0;
+        long long prev_h = -1;
+        bool live = true;
+        auto epilogue = [&](long long xe, int ae, uint32_t aphe) {
+            const int h = (int)(xe / nt), j = (int)(xe % nt);
+            bool got = live && LA_WAIT(&accfull[ae], aphe, 0x10u);
+            got = __all_sync(0xffffffffu, got);
+            live = live && got;
+            float v[64];
+            float nz = 0.f;
+            if (got) {
+                tc_fence_after();
+                const uint32_t base = tmem + (uint32_t)ae * 128u + ((uint32_t)(32 * sub) << 16);
+                tmem_row64(base, v);
+                if (BIDIR) {
+                    float t16[16];
+                    tmem_ld16(base + 64, t16);
+                    tmem_ld_wait();
+                    nz = t16[0];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[ae]);
+                const float sc = *s_scale;
+                const float inv = BIDIR ? 1.f / (nz + eps * sc) : 1.f / sc;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) v[c] *= inv;
+            }
+            if (tid == 0) tma_store_wait_read<OST - 1>();
+            named_bar(1, kWorkers);
+            if (got) store_row<BF16>(sO + ob * kTileBytes, row, v);
+            fence_async_smem();
+            named_bar(1, kWorkers);
+            if (tid == 0 && live) {
+                tma_store_3d(&tmO, sO + ob * kTileBytes, 0, j * kRows, h);
+                tma_store_commit();
+            }
+            if (++ob == OST) ob = 0;
+        };
+        int a_prev = 0;
+        uint32_t aph_prev = 0;
+        for (long long x = x0; x < x1; ++x) {
+            const long long h = x / nt;
+            if (BIDIR) {
+                bool got = live && LA_WAIT(&full[s], ph, 0x8u);
+                got = __all_sync(0xffffffffu, got);
+                live = live && got;
+                if (got) {
+                    phi_row_inplace<BF16>(sQ + s * kTileBytes, row, false);
+                    fence_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0 && got) mbar_arrive(&xf[s]);
+            }
+            if (++s == NST) { s = 0; ph ^= 1; }
+            if (x > x0) epilogue(x - 1, a_prev, aph_prev);
+            if (h != prev_h) {
+                // the previous head's UMMAs are complete: its last epilogue waited on them
+                const float *srch = src + h * (long long)src_per_head;
+                const int ns = src_single ? 1 : (P.last_cta((int)h) - P.first_cta((int)h) + 1);
+                float m = gather_state(srch, ns, stage, tid);
+                named_bar(1, kWorkers);
+                if (state_out && (x % nt) == 0) {
+                    float *dst = state_out + h * (long long)kStateElems;
+                    for (int e = tid; e < kStateElems; e += kWorkers) dst[e] = stage[e];
+                }
+                if (!BF16) m = workers_max(m, red, tid);
+                const float sc = operand_scale<BF16>(m);
+                if (tid < 80) {
+                    float xv[64];
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        xv[i] = tid < 64 ? stage[i * 65 + tid] * sc
+                                         : ((BIDIR && tid == 64) ? stage[i * 65 + 64] * sc : 0.f);
+                    operand_row<BF16, NOPS>(sOp, sOp + OPB, tid, xv);
+                }
+                if (tid == 0) *s_scale = sc;
+                fence_async_smem();
+                named_bar(1, kWorkers);
+                if (tid == 0) mbar_arrive(opready);
+                prev_h = h;
+            }
+            a_prev = a;
+            aph_prev = aph;
+            a ^= 1;
+            if (a == 0) aph ^= 1;
+        }
+        epilogue(x1 - 1, a_prev, aph_prev);
+        if (tid == 0) tma_store_wait_all<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+
+// ================================================================== bwd_q ==
+// Per tile: MMA1 [u | q.z] = f(Q) [S | z] (M=128, N=80), MMA2 g S^T (M=128, N=64,
+// B = the state operand read MN-major); the workers form n, o, g.o, dq and write
+// g/n (in place over the dO tile) and w = -(g.o)/n (column 0 of a zero block);
+// MMA3 accumulates [dS | dz] += f(Q)^T [g/n | w] (M=64, N=80, both MN-major).
+// bf16 bidir also keeps lo = round(f(q) - hi) of the feature map (one more tile per
+// stage): MMA1 then adds f(Q)_lo S_hi, and f'(q) = min(hi + lo, 1).
+template <bool BIDIR, bool BF16>
+struct BwdQLayout {
+    static constexpr bool QLO = BIDIR && BF16;
+    static constexpr int NST = QLO ? 2 : 3, OST = 2, OPB = 80 * 128;
+    static constexpr int qoff = 0;
+    static constexpr int goff = qoff + NST * kTileBytes;
+    static constexpr int woff = goff + NST * kTileBytes;
+    static constexpr int qloff = woff + (BIDIR ? NST * kTileBytes : 0);
+    static constexpr int dqoff = qloff + (QLO ? NST * kTileBytes : 0);
+    static constexpr int opoff = dqoff + OST * kTileBytes;
+    static constexpr int stageoff = opoff + 2 * OPB;
+    static constexpr int zsoff = stageoff + kStateElems * 4;
+    static constexpr int redoff = zsoff + 64 * 4;
+    static constexpr int baroff = redoff + 32;
+    static constexpr int nbars = 4 * NST + 4 + 4;
+    static constexpr int misc = baroff + nbars * 8;
+    static constexpr int bytes = misc + 32 + 1024;
+};
+
+template <bool BIDIR, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
+             const __grid_constant__ CUtensorMap tmDQ, const float *__restrict__ src, int src_per_head,
+             int src_single, float *__restrict__ dpart, int T, int BH, int nt, int maxslots, float eps) {
+    using L = BwdQLayout<BIDIR, BF16>;
+    constexpr int NST = L::NST, OST = L::OST, OPB = L::OPB;
+    constexpr bool QLO = L::QLO;
+    constexpr int NOPS = BF16 ? 2 : 1;
+    constexpr int N1 = 80;
+    constexpr int N3 = BIDIR ? 80 : 64;
+    constexpr uint32_t IDESC1 = idesc_f16(128, N1, BF16, false, false);
+    constexpr uint32_t IDESC2 = idesc_f16(128, 64, BF16, false, true);
+    constexpr uint32_t IDESC3 = idesc_f16(64, N3, BF16, true, true);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *sQ = smem + L::qoff;
+    uint8_t *sG = smem + L::goff;
+    uint8_t *sW = smem + L::woff;
+    uint8_t *sQlo = smem + L::qloff;
+    uint8_t *sDQ = smem + L::dqoff;
+    uint8_t *sOp = smem + L::opoff;
+    float *stage = reinterpret_cast<float *>(smem + L::stageoff);
+    float *zs = reinterpret_cast<float *>(smem + L::zsoff);
+    float *red = reinterpret_cast<float *>(smem + L::redoff);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::baroff);
+    uint64_t *xf = full + NST;
+    uint64_t *gnready = xf + NST;
+    uint64_t *empty = gnready + NST;
+    uint64_t *acc12full = empty + NST;   // [2]
+    uint64_t *acc12empty = acc12full + 2;
+    uint64_t *accSfull = acc12empty + 2;
+    uint64_t *accSfree = accSfull + 1;
+    uint64_t *opready = accSfree + 1;
+    uint64_t *drain = opready + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc);
+    int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Partition P{(long long)BH * nt, nt, grid_for((long long)BH * nt)};
+    const int cta = blockIdx.x;
+    const long long x0 = P.start(cta), x1 = P.start(cta + 1);
+    if (x0 >= x1) return;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&xf[s], 4);
+            mbar_init(&gnready[s], 4);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc12full[b], 1);
+            mbar_init(&acc12empty[b], 4);
+        }
+        mbar_init(accSfull, 1);
+        mbar_init(accSfree, 4);
+        mbar_init(opready, 1);
+        mbar_init(drain, 1);
+        *s_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch(&tmQ);
+        tma_prefetch(&tmG);
+        tma_prefetch(&tmDQ);
+    }
+    if (BIDIR && warp >= 2) {
+        const int r = threadIdx.x - 64;
+        for (int st = 0; st < NST; ++st) {
+            uint8_t *p = sW + st * kTileBytes + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(p + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    constexpr uint32_t kAccS = 176;    // columns 176..255: the M=64 [dS | dz] accumulator
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            long long issued = 0;
+            for (long long x = x0; x < x1; ++x) {
+                const int h = (int)(x / nt), j = (int)(x % nt);
+                if (!LA_WAIT(&empty[s], ph ^ 1, 0x1u)) break;
+                mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
+                tma_load_3d(sQ + s * kTileBytes, &tmQ, &full[s], 0, j * kRows, h);
+                tma_load_3d(sG + s * kTileBytes, &tmG, &full[s], 0, j * kRows, h);
+                ++issued;
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+            if (*s_abort) {
+                for (long long i = issued - 1; i >= 0 && i >= issued - NST; --i)
+                    mbar_wait_slow(smem_u32(&full[i % NST]), (uint32_t)((i / NST) & 1), nullptr, &g_tc_fault, 0x200u);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int s = 0, b = 0;
+            uint32_t ph = 0, bph = 0, oph = 0;
+            long long prev_h = -1;
+            long long seg = 0;                     // segments started (for the accS free parity)
+            bool dead = false;
+            // MMA3 of tile xe (stage se, phase phe)
+            auto issue3 = [&](long long xe, int se, uint32_t phe) {
+                const bool seg_start = (xe == x0) || (xe % nt == 0);
+                const bool seg_end = (xe + 1 == x1) || ((xe + 1) % nt == 0);
+                if (seg_start) {
+                    if (!LA_WAIT(accSfree, (uint32_t)((seg & 1) ^ 1), 0x40u)) { dead = true; return; }
+                    ++seg;
+                }
+                if (!LA_WAIT(&gnready[se], phe, 0x80u)) { dead = true; return; }
+                tc_fence_after();
+                const uint32_t aQ = smem_u32(sQ + se * kTileBytes), aG = smem_u32(sG + se * kTileBytes);
+                const uint32_t lbo = BIDIR ? smem_u32(sW + se * kTileBytes) - aG : (uint32_t)kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kRows / 16; ++kk) {
+                    const uint64_t ad = sdesc_sw128(aQ + kk * 2048, kTileBytes, 1024);
+                    const uint64_t bd = sdesc_sw128(aG + kk * 2048, lbo, 1024);
+                    umma_f16_ss(tmem + kAccS, ad, bd, IDESC3, (seg_start && kk == 0) ? 0u : 1u);
+                }
+                umma_commit(&empty[se]);
+                if (seg_end) umma_commit(accSfull);
+            };
+            long long xp = -1;
+            int sp = 0;
+            uint32_t php = 0;
+            for (long long x = x0; x < x1 && !dead; ++x) {
+                const long long h = x / nt;
+                if (h != prev_h) {
+                    if (!LA_WAIT(opready, oph, 0x20u)) break;
+                    oph ^= 1;
+                    prev_h = h;
+                }
+                if (!LA_WAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
+                if (!LA_WAIT(&acc12empty[b], bph ^ 1, 0x2u)) break;
+                tc_fence_after();
+                const uint32_t d1 = tmem + (uint32_t)b * 256u, d2 = d1 + 96u;
+                const uint32_t aQ = smem_u32(sQ + s * kTileBytes), aG = smem_u32(sG + s * kTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                    for (int op = 0; op < NOPS; ++op) {
+                        const uint32_t aO = smem_u32(sOp + op * OPB);
+                        if (BIDIR)
+                            umma_f16_ss(d1, sdesc_sw128(aQ + kk * 32, 16, 1024), sdesc_sw128(aO + kk * 32, 16, 1024),
+                                        IDESC1, (kk | op) ? 1u : 0u);
+                        umma_f16_ss(d2, sdesc_sw128(aG + kk * 32, 16, 1024), sdesc_sw128(aO + kk * 2048, OPB, 1024),
+                                    IDESC2, (kk | op) ? 1u : 0u);
+                    }
+                    if (QLO)
+                        umma_f16_ss(d1, sdesc_sw128(smem_u32(sQlo + s * kTileBytes) + kk * 32, 16, 1024),
+                                    sdesc_sw128(smem_u32(sOp) + kk * 32, 16, 1024), IDESC1, 1u);
+                }
+                umma_commit(&acc12full[b]);
+                b ^= 1;
+                if (b == 0) bph ^= 1;
+                if (xp >= 0) issue3(xp, sp, php);
+                xp = x;
+                sp = s;
+                php = ph;
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+            if (xp >= 0 && !dead && !*s_abort) issue3(xp, sp, php);
+            umma_commit(drain);
+            mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+        }
+    } else {
+        // Workers (every named barrier is reached by all 128 whatever the waits return).
+        const int tid = threadIdx.x - 64;
+        const int sub = warp & 3;
+        const int row = sub * 32 + lane;
+        int s = 0, b = 0, ob = 0;
+        uint32_t ph = 0, bph = 0;
+        long long prev_h = -1;
+        uint32_t sfull_ph = 0;
+        bool live = true;
+        float cur_sc = 1.f, cur_scn = 1.f;
+
+        auto epilogue = [&](long long xe, int se, uint32_t phe, int be, uint32_t bphe) {
+            const int h = (int)(xe / nt), j = (int)(xe % nt);
+            bool got = live && LA_WAIT(&acc12full[be], bphe, 0x10u);
+            got = __all_sync(0xffffffffu, got);
+            live = live && got;
+            const uint32_t lanes = (uint32_t)(32 * sub) << 16;
+            const uint32_t d1 = tmem + (uint32_t)be * 256u + lanes, d2 = d1 + 96u;
+            uint8_t *tq = sQ + se * kTileBytes, *tg = sG + se * kTileBytes;
+            uint8_t *dqrow = sDQ + ob * kTileBytes;
+            float gdot = 0.f, inv = 1.f;
+            float dq[64];
+            if (got) {
+                tc_fence_after();
+                if (BIDIR) {
+                    float u[64], g[64];
+                    tmem_row64(d1, u);
+                    float t16[16];
+                    tmem_ld16(d1 + 64, t16);
+                    tmem_ld_wait();
+                    inv = 1.f / (t16[0] + eps * cur_sc);
+                    load_row<BF16>(tg, row, g);
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) gdot = fmaf(g[c], u[c] * inv, gdot);
+                    const float gsc = inv * cur_sc * cur_scn;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) g[c] *= gsc;
+                    store_row<BF16>(tg, row, g);    // g/n (scaled) replaces dO in place: MMA2 is done
+                    const float w = -gdot * gsc;
+                    if (BF16) {
+                        __nv_bfloat16 wv = __float2bfloat16_rn(w);
+                        *reinterpret_cast<__nv_bfloat16 *>(sW + se * kTileBytes + sw128_offset(row, 0)) = wv;
+                    } else {
+                        __half wv = __float2half_rn(w);
+                        *reinterpret_cast<__half *>(sW + se * kTileBytes + sw128_offset(row, 0)) = wv;
+                    }
+                }
+                tmem_row64(d2, dq);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc12empty[be]);
+                if (BIDIR) {
+                    float qf[64];
+                    load_row<BF16>(tq, row, qf);
+                    if (QLO) {
+                        float ql[64];
+                        load_row<BF16>(sQlo + se * kTileBytes, row, ql);
+#pragma unroll
+                        for (int c = 0; c < 64; ++c) qf[c] += ql[c];
+                    }
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) dq[c] = (dq[c] - gdot * zs[c]) * inv * fminf(qf[c], 1.f);
+                } else {
+                    const float isc = 1.f / cur_sc;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) dq[c] *= isc;
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&gnready[se]);
+            }
+            if (tid == 0) tma_store_wait_read<OST - 1>();
+            named_bar(1, kWorkers);
+            if (got) store_row<BF16>(dqrow, row, dq);
+            fence_async_smem();
+            named_bar(1, kWorkers);
+            if (tid == 0 && live) {
+                tma_store_3d(&tmDQ, dqrow, 0, j * kRows, h);
+                tma_store_commit();
+            }
+            if (++ob == OST) ob = 0;
+        };
+        // [dS | dz] partial of the segment of head hs that just ended
+        auto read_accS = [&](int hs, float scn) {
+            bool got = live && LA_WAIT(accSfull, sfull_ph, 0x100u);
+            got = __all_sync(0xffffffffu, got);
+            live = live && got;
+            sfull_ph ^= 1;
+            if (!got) return;
+            tc_fence_after();
+            const uint32_t base = tmem + kAccS + ((uint32_t)(32 * sub) << 16);
+            float v[64];
+            tmem_row64(base, v);
+            float zz = 0.f;
+            if (BIDIR) {
+                float t16[16];
+                tmem_ld16(base + 64, t16);
+                tmem_ld_wait();
+                zz = t16[0];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(accSfree);
+            if (lane < 16) {
+                const int i = 16 * sub + lane;
+                const int slot = cta - P.first_cta(hs);
+                float *dst = dpart + (((long long)hs * maxslots + slot) * 64 + i) * 65;
+                const float is = 1.f / scn;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) dst[c] = v[c] * is;
+                dst[64] = zz * is;
+            }
+        };
+
+        int s_prev = 0, b_prev = 0;
+        uint32_t ph_prev = 0, bph_prev = 0;
+        for (long long x = x0; x < x1; ++x) {
+            const long long h = x / nt;
+            if (BIDIR) {
+                bool got = live && LA_WAIT(&full[s], ph, 0x8u);
+                got = __all_sync(0xffffffffu, got);
+                live = live && got;
+                if (got) {
+                    if (QLO)
+                        phi_row_split<BF16>(sQ + s * kTileBytes, sQlo + s * kTileBytes, row);
+                    else
+                        phi_row_inplace<BF16>(sQ + s * kTileBytes, row, false);
+                    fence_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0 && got) mbar_arrive(&xf[s]);
+            }
+            if (x > x0) epilogue(x - 1, s_prev, ph_prev, b_prev, bph_prev);
+            const float prev_scn = cur_scn;
+            if (h != prev_h) {
+                const float *srch = src + h * (long long)src_per_head;
+                const int ns = src_single ? 1 : (P.last_cta((int)h) - P.first_cta((int)h) + 1);
+                float m = gather_state(srch, ns, stage, tid);
+                named_bar(1, kWorkers);
+                if (!BF16) m = workers_max(m, red, tid);
+                const float sc = operand_scale<BF16>(m);
+                float zsum = 0.f;
+                for (int i = 0; i < 64; ++i) zsum += fabsf(stage[i * 65 + 64]);
+                float scn = 1.f;
+                if (BIDIR && zsum > 0.f && isfinite(zsum)) {
+                    int e;
+                    frexpf(zsum, &e);
+                    e = e < -100 ? -100 : (e > 100 ? 100 : e);
+                    scn = ldexpf(1.f, e - 1);
+                }
+                if (tid < 80) {
+                    float xv[64];
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        xv[i] = tid < 64 ? stage[i * 65 + tid] * sc
+                                         : ((BIDIR && tid == 64) ? stage[i * 65 + 64] * sc : 0.f);
+                    operand_row<BF16, NOPS>(sOp, sOp + OPB, tid, xv);
+                }
+                if (tid < 64) zs[tid] = stage[tid * 65 + 64] * sc;
+                fence_async_smem();
+                named_bar(1, kWorkers);
+                cur_sc = sc;
+                cur_scn = scn;
+                if (tid == 0) mbar_arrive(opready);
+                if (x > x0) read_accS((int)((x - 1) / nt), prev_scn);   // the previous head's segment ended
+                prev_h = h;
+            }
+            s_prev = s;
+            ph_prev = ph;
+            b_prev = b;
+            bph_prev = bph;
+            if (++s == NST) { s = 0; ph ^= 1; }
+            b ^= 1;
+            if (b == 0) bph ^= 1;
+        }
+        epilogue(x1 - 1, s_prev, ph_prev, b_prev, bph_prev);
+        read_accS((int)((x1 - 1) / nt), cur_scn);
+        if (tid == 0) tma_store_wait_all<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ================================================================= bwd_kv ==
+// Per tile: MMA_a  v dS^T (A = V tile, B = dS operand K-major),
+//           MMA_b  f(K) dS (A = f(K) tile, B = dS operand read MN-major);
+// dk = (v dS^T + dz) f'(k), dv = f(k) dS.  The dS operand rows are dS's rows.
+struct BwdKvLayout {
+    static constexpr int NST = 3, OST = 2, OPB = 64 * 128;
+    static constexpr int koff = 0;
+    static constexpr int voff = koff + NST * kTileBytes;
+    static constexpr int dkoff = voff + NST * kTileBytes;
+    static constexpr int dvoff = dkoff + OST * kTileBytes;
+    static constexpr int opoff = dvoff + OST * kTileBytes;
+    static constexpr int stageoff = opoff + 2 * OPB;
+    static constexpr int dzoff = stageoff + kStateElems * 4;
+    static constexpr int redoff = dzoff + 64 * 4;
+    static constexpr int baroff = redoff + 32;
+    static constexpr int nbars = 3 * NST + 4 + 2;
+    static constexpr int misc = baroff + nbars * 8;
+    static constexpr int bytes = misc + 32 + 1024;
+};
+
+template <bool BIDIR, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+              const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
+              const float *__restrict__ dpart, int T, int BH, int nt, int maxslots) {
+    using L = BwdKvLayout;
+    constexpr int NST = L::NST, OST = L::OST, OPB = L::OPB;
+    constexpr int NOPS = BF16 ? 2 : 1;
+    constexpr uint32_t IDESC_A = idesc_f16(128, 64, BF16, false, false);
+    constexpr uint32_t IDESC_B = idesc_f16(128, 64, BF16, false, true);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *sK = smem + L::koff;
+    uint8_t *sV = smem + L::voff;
+    uint8_t *sDK = smem + L::dkoff;
+    uint8_t *sDV = smem + L::dvoff;
+    uint8_t *sOp = smem + L::opoff;
+    float *stage = reinterpret_cast<float *>(smem + L::stageoff);
+    float *dz = reinterpret_cast<float *>(smem + L::dzoff);
+    float *red = reinterpret_cast<float *>(smem + L::redoff);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::baroff);
+    uint64_t *xf = full + NST;
+    uint64_t *empty = xf + NST;
+    uint64_t *accfull = empty + NST;
+    uint64_t *accempty = accfull + 2;
+    uint64_t *opready = accempty + 2;
+    uint64_t *drain = opready + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc);
+    int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Partition P{(long long)BH * nt, nt, grid_for((long long)BH * nt)};
+    const int cta = blockIdx.x;
+    const long long x0 = P.start(cta), x1 = P.start(cta + 1);
+    if (x0 >= x1) return;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&xf[s], 4);
+            mbar_init(&empty[s], BIDIR ? 5 : 1);   // UMMA commit (+ the 4 worker warps that read f(k) for f'(k))
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accfull[b], 1);
+            mbar_init(&accempty[b], 4);
+        }
+        mbar_init(opready, 1);
+        mbar_init(drain, 1);
+        *s_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch(&tmK);
+        tma_prefetch(&tmV);
+        tma_prefetch(&tmDK);
+        tma_prefetch(&tmDV);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            long long issued = 0;
+            for (long long x = x0; x < x1; ++x) {
+                const int h = (int)(x / nt), j = (int)(x % nt);
+                if (!LA_WAIT(&empty[s], ph ^ 1, 0x1u)) break;
+                mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
+                tma_load_3d(sK + s * kTileBytes, &tmK, &full[s], 0, j * kRows, h);
+                tma_load_3d(sV + s * kTileBytes, &tmV, &full[s], 0, j * kRows, h);
+                ++issued;
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+            if (*s_abort) {
+                for (long long i = issued - 1; i >= 0 && i >= issued - NST; --i)
+                    mbar_wait_slow(smem_u32(&full[i % NST]), (uint32_t)((i / NST) & 1), nullptr, &g_tc_fault, 0x200u);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int s = 0, b = 0;
+            uint32_t ph = 0, bph = 0, oph = 0;
+            long long prev_h = -1;
+            for (long long x = x0; x < x1; ++x) {
+                const long long h = x / nt;
+                if (h != prev_h) {
+                    if (!LA_WAIT(opready, oph, 0x20u)) break;
+                    oph ^= 1;
+                    prev_h = h;
+                }
+                if (!LA_WAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
+                if (!LA_WAIT(&accempty[b], bph ^ 1, 0x2u)) break;
+                tc_fence_after();
+                const uint32_t da = tmem + (uint32_t)b * 128u, db = da + 64u;
+                const uint32_t aK = smem_u32(sK + s * kTileBytes), aV = smem_u32(sV + s * kTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                    for (int op = 0; op < NOPS; ++op) {
+                        const uint32_t aO = smem_u32(sOp + op * OPB);
+                        umma_f16_ss(da, sdesc_sw128(aV + kk * 32, 16, 1024), sdesc_sw128(aO + kk * 32, 16, 1024),
+                                    IDESC_A, (kk | op) ? 1u : 0u);
+                        umma_f16_ss(db, sdesc_sw128(aK + kk * 32, 16, 1024), sdesc_sw128(aO + kk * 2048, OPB, 1024),
+                                    IDESC_B, (kk | op) ? 1u : 0u);
+                    }
+                }
+                umma_commit(&empty[s]);
+                umma_commit(&accfull[b]);
+                b ^= 1;
+                if (b == 0) bph ^= 1;
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+            umma_commit(drain);
+            mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+        }
+    } else {
+        const int tid = threadIdx.x - 64;
+        const int sub = warp & 3;
+        const int row = sub * 32 + lane;
+        int s = 0, b = 0, ob = 0;
+        uint32_t ph = 0, bph = 0;
+        long long prev_h = -1;
+        bool live = true;
+        float cur_isd = 1.f;
+
+        auto epilogue = [&](long long xe, int se, int be, uint32_t bphe) {
+            const int h = (int)(xe / nt), j = (int)(xe % nt);
+            bool got = live && LA_WAIT(&accfull[be], bphe, 0x10u);
+            got = __all_sync(0xffffffffu, got);
+            live = live && got;
+            const uint32_t da = tmem + (uint32_t)be * 128u + ((uint32_t)(32 * sub) << 16), db = da + 64u;
+            float dk[64], dv[64];
+            if (got) {
+                tc_fence_after();
+                tmem_row64(da, dk);
+                tmem_row64(db, dv);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[be]);
+                if (BIDIR) {
+                    float kf[64];
+                    load_row<BF16>(sK + se * kTileBytes, row, kf);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[se]);   // f(k) read: the stage may be reloaded
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) dk[c] = fmaf(dk[c], cur_isd, dz[c]) * fminf(kf[c], 1.f);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) dk[c] *= cur_isd;
+                }
+#pragma unroll
+                for (int c = 0; c < 64; ++c) dv[c] *= cur_isd;
+            } else if (BIDIR) {
+                __syncwarp();
+            }
+            if (tid == 0) tma_store_wait_read<OST - 1>();
+            named_bar(1, kWorkers);
+            if (got) {
+                store_row<BF16>(sDK + ob * kTileBytes, row, dk);
+                store_row<BF16>(sDV + ob * kTileBytes, row, dv);
+            }
+            fence_async_smem();
+            named_bar(1, kWorkers);
+            if (tid == 0 && live) {
+                tma_store_3d(&tmDK, sDK + ob * kTileBytes, 0, j * kRows, h);
+                tma_store_3d(&tmDV, sDV + ob * kTileBytes, 0, j * kRows, h);
+                tma_store_commit();
+            }
+            if (++ob == OST) ob = 0;
+        };
+
+        int s_prev = 0, b_prev = 0;
+        uint32_t bph_prev = 0;
+        for (long long x = x0; x < x1; ++x) {
+            const long long h = x / nt;
+            if (BIDIR) {
+                bool got = live && LA_WAIT(&full[s], ph, 0x8u);
+                got = __all_sync(0xffffffffu, got);
+                live = live && got;
+                if (got) {
+                    phi_row_inplace<BF16>(sK + s * kTileBytes, row, false);
+                    fence_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0 && got) mbar_arrive(&xf[s]);
+            }
+            if (x > x0) epilogue(x - 1, s_prev, b_prev, bph_prev);
+            if (h != prev_h) {
+                const float *srch = dpart + h * (long long)maxslots * kStateElems;
+                const int ns = P.last_cta((int)h) - P.first_cta((int)h) + 1;
+                float m = gather_state(srch, ns, stage, tid);
+                named_bar(1, kWorkers);
+                if (!BF16) m = workers_max(m, red, tid);
+                const float sd = operand_scale<BF16>(m);
+                if (tid < 64) {
+                    float xv[64];
+#pragma unroll
+                    for (int jj = 0; jj < 64; ++jj) xv[jj] = stage[tid * 65 + jj] * sd;
+                    operand_row<BF16, NOPS>(sOp, sOp + OPB, tid, xv);
+                    dz[tid] = BIDIR ? stage[tid * 65 + 64] : 0.f;
+                }
+                fence_async_smem();
+                named_bar(1, kWorkers);
+                cur_isd = 1.f / sd;
+                if (tid == 0) mbar_arrive(opready);
+                prev_h = h;
+            }
+            s_prev = s;
+            b_prev = b;
+            bph_prev = bph;
+            if (++s == NST) { s = 0; ph ^= 1; }
+            b ^= 1;
+            if (b == 0) bph ^= 1;
+        }
+        epilogue(x1 - 1, s_prev, b_prev, bph_prev);
+        if (tid == 0) tma_store_wait_all<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// =================================================================== host ==
+
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                              const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeFn encode_fn() {
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(p);
+    });
+    return fn;
+}
+
+// [BH, T, 64] 16-bit tensor, boxes of 128 rows x 64 columns, 128-byte swizzle, zero fill.
+static la_status tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16) {
+    EncodeFn enc = encode_fn();
+    if (!enc) {
+        set_error("cuTensorMapEncodeTiled is unavailable from the driver");
+        return LA_ERR_CUDA;
+    }
+    const cuuint64_t dims[3] = {(cuuint64_t)s.D, (cuuint64_t)s.T, (cuuint64_t)s.BH()};
+    const cuuint64_t strides[2] = {(cuuint64_t)s.D * 2, (cuuint64_t)s.T * s.D * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kRows, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                     const_cast<void *>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return LA_ERR_CUDA;
+    }
+    return LA_OK;
+}
+
+// state_reduce: 4 stages of (k, v) + the ones block, or 3 stages of (k, v, k_lo) for bf16 bidir
+constexpr size_t reduce_smem(bool klo) { return 1024 + (klo ? 9 : 8) * (size_t)kTileBytes + kTileBytes + 256; }
+constexpr size_t kOutputSmem = 1024 + 4 * kTileBytes + 2 * kTileBytes + 2 * 80 * 128 + kStateElems * 4 + 32 + 256;
+
+static size_t partial_bytes(const Shape &s) {
+    size_t b = (size_t)s.BH() * (size_t)max_slots((int)s.BH()) * kStateElems * sizeof(float);
+    return (b + 255) & ~(size_t)255;
+}
+
+template <bool BIDIR, bool BF16>
+static la_status launch_reduce(const CUtensorMap &mk, const CUtensorMap &mv, float *part, const Shape &s, int nt,
+                               cudaStream_t st) {
+    return launch(BIDIR ? "tc_state_reduce" : "tc_state_reduce_simple", state_reduce_kernel<BIDIR, BF16>,
+                  dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads), reduce_smem(BIDIR && BF16), st, mk, mv, part, s.T, (int)s.BH(), nt,
+                  max_slots((int)s.BH()));
+}
+
+template <bool BIDIR, bool BF16>
+static la_status fwd_t(const void *q, const void *k, const void *v, void *o, float *state, const Shape &s,
+                       float eps, void *ws, cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mo;
+    LA_TRY(tensor_map(&mq, q, s, BF16));
+    LA_TRY(tensor_map(&mk, k, s, BF16));
+    LA_TRY(tensor_map(&mv, v, s, BF16));
+    LA_TRY(tensor_map(&mo, o, s, BF16));
+    const int nt = (s.T + kRows - 1) / kRows;
+    const int ms = max_slots((int)s.BH());
+    float *part = (float *)ws;
+    LA_TRY((launch_reduce<BIDIR, BF16>(mk, mv, part, s, nt, st)));
+    return launch(BIDIR ? "tc_output" : "tc_output_simple", output_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
+                  kOutputSmem, st, mq, mo, (const float *)part, ms * kStateElems, 0, state, s.T, (int)s.BH(), nt,
+                  eps);
+}
+
+template <bool BIDIR, bool BF16>
+static la_status bwd_t(const void *q, const void *k, const void *v, const void *g, const float *state, void *dq,
+                       void *dk, void *dv, const Shape &s, float eps, void *ws, cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mg, mdq, mdk, mdv;
+    LA_TRY(tensor_map(&mq, q, s, BF16));
+    LA_TRY(tensor_map(&mk, k, s, BF16));
+    LA_TRY(tensor_map(&mv, v, s, BF16));
+    LA_TRY(tensor_map(&mg, g, s, BF16));
+    LA_TRY(tensor_map(&mdq, dq, s, BF16));
+    LA_TRY(tensor_map(&mdk, dk, s, BF16));
+    LA_TRY(tensor_map(&mdv, dv, s, BF16));
+    const int nt = (s.T + kRows - 1) / kRows;
+    const int ms = max_slots((int)s.BH());
+    float *dpart = (float *)ws;
+    float *spart = (float *)((char *)ws + partial_bytes(s));
+    const float *src = state;
+    int per_head = kStateElems, single = 1;
+    if (!state) {
+        LA_TRY((launch_reduce<BIDIR, BF16>(mk, mv, spart, s, nt, st)));
+        src = spart;
+        per_head = ms * kStateElems;
+        single = 0;
+    }
+    LA_TRY(launch(BIDIR ? "tc_bwd_q" : "tc_bwd_q_simple", bwd_q_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
+                  (size_t)BwdQLayout<BIDIR, BF16>::bytes, st, mq, mg, mdq, src, per_head, single, dpart, s.T, (int)s.BH(),
+                  nt, ms, eps));
+    return launch(BIDIR ? "tc_bwd_kv" : "tc_bwd_kv_simple", bwd_kv_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
+                  (size_t)BwdKvLayout::bytes, st, mk, mv, mdk, mdv, (const float *)dpart, s.T, (int)s.BH(), nt, ms);
+}
+
+}  // namespace
+
+size_t state_workspace_size(la_op op, const Shape &s) {
+    switch (op) {
+    case LA_OP_BIDIR_FWD:
+    case LA_OP_SIMPLE_FWD: return partial_bytes(s);
+    case LA_OP_BIDIR_BWD:
+    case LA_OP_SIMPLE_BWD: return 2 * partial_bytes(s);
+    default: return 0;
+    }
+}
+
+la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, void *o, float *state, const Shape &s,
+                    la_dtype dt, float eps, void *ws, cudaStream_t st) {
+    const bool bf = dt == LA_BF16;
+    if (bidir) return bf ? fwd_t<true, true>(q, k, v, o, state, s, eps, ws, st)
+                         : fwd_t<true, false>(q, k, v, o, state, s, eps, ws, st);
+    return bf ? fwd_t<false, true>(q, k, v, o, state, s, eps, ws, st)
+              : fwd_t<false, false>(q, k, v, o, state, s, eps, ws, st);
+}
+
+la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, const void *g, const float *state,
+                    void *dq, void *dk, void *dv, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st) {
+    const bool bf = dt == LA_BF16;
+    if (bidir) return bf ? bwd_t<true, true>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st)
+                         : bwd_t<true, false>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st);
+    return bf ? bwd_t<false, true>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st)
+              : bwd_t<false, false>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st);
+}
+
+unsigned int read_and_clear_fault() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tc_fault, sizeof v) != cudaSuccess) return 0xFFFFFFFFu;
+    if (v) cudaMemcpyToSymbol(g_tc_fault, &zero, sizeof zero);
+    return v;
+}
+
+}  // namespace tc
+}  // namespace la
