@@ -165,14 +165,42 @@ __device__ __forceinline__ void tmem_row64(uint32_t taddr, float (&v)[64]) {
 // ------------------------------------------------------------- state I/O --
 // stage[e] = sum over s in [0, nslots) of src[s * kStateElems + e], in slot order
 // (a fixed order: the result does not depend on which CTA finished first).
-// Returns this thread's max |stage[e]| over the elements it summed.
+// Blocks are 16-byte aligned, so the copy runs on float4s with all of a slot's
+// loads in flight at once.  Returns this thread's max |stage[e]| over its elements.
 __device__ __forceinline__ float gather_state(const float *__restrict__ src, int nslots, float *stage, int tid) {
+    constexpr int N4 = kStateElems / 4;                  // 1040 float4 per block
+    constexpr int PER = (N4 + kWorkers - 1) / kWorkers;  // 9 per thread
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+    float4 acc[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int e = tid + u * kWorkers;
+        acc[u] = e < N4 ? __ldg(s4 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int sl = 1; sl < nslots; ++sl) {
+        float4 nx[PER];
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int e = tid + u * kWorkers;
+            nx[u] = e < N4 ? __ldg(s4 + (long long)sl * N4 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            acc[u].x += nx[u].x;
+            acc[u].y += nx[u].y;
+            acc[u].z += nx[u].z;
+            acc[u].w += nx[u].w;
+        }
+    }
     float m = 0.f;
-    for (int e = tid; e < kStateElems; e += kWorkers) {
-        float acc = 0.f;
-        for (int s = 0; s < nslots; ++s) acc += src[(long long)s * kStateElems + e];
-        stage[e] = acc;
-        m = fmaxf(m, fabsf(acc));
+    float4 *st4 = reinterpret_cast<float4 *>(stage);
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int e = tid + u * kWorkers;
+        if (e < N4) {
+            st4[e] = acc[u];
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(acc[u].x), fabsf(acc[u].y)), fmaxf(fabsf(acc[u].z), fabsf(acc[u].w))));
+        }
     }
     return m;
 }
