@@ -14,8 +14,12 @@ namespace tc {
 
 constexpr int kGrid = 148;          // persistent CTAs; fixed so partial-slot layout depends on the shape only
 constexpr int kRows = 128;          // rows of q/k/v per tile (the UMMA M of the row-wise products)
-constexpr int kThreads = 192;       // warp 0: TMA producer, warp 1: UMMA issuer + TMEM, warps 2..5: workers
-constexpr int kWorkers = 128;
+// Warp roles: 0 TMA producer, 1 UMMA issuer + TMEM owner, 2..9 feature-map
+// ("transform") warps, 10..13 epilogue warps (warp w reads TMEM lanes 32*(w%4)..).
+constexpr int kXw0 = 2, kXWarps = 8, kXThreads = kXWarps * 32;
+constexpr int kEw0 = 10, kEWarps = 4;
+constexpr int kThreads = 448;
+constexpr int kWorkers = kEWarps * 32;   // epilogue threads (named barriers 1 and 2)
 constexpr int kTileBytes = kRows * 128;   // 128 rows x 64 16-bit elements, 128-byte swizzled
 constexpr int kStateElems = 64 * 65;      // one fp32 [64][65] state block: S | z
 
@@ -113,6 +117,85 @@ __device__ __forceinline__ void phi_row_split(uint8_t *tile, uint8_t *lo_tile, i
         }
         *reinterpret_cast<uint4 *>(p + off) = make_uint4(w[0], w[1], w[2], w[3]);
         *reinterpret_cast<uint4 *>(q + off) = make_uint4(l[0], l[1], l[2], l[3]);
+    }
+}
+
+// The transform warps split a tile into 256 half rows: thread xi handles row
+// xi % 128, logical chunks 4 * (xi / 128) .. + 3 (chunk order spreads banks).
+template <bool BF16>
+__device__ __forceinline__ void phi_half_row(uint8_t *tile, int xi, bool zero) {
+    const int row = xi & 127, c0 = (xi >> 7) * 4;
+    uint8_t *p = tile + row * 128;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        uint4 *c = reinterpret_cast<uint4 *>(p + (((c0 + it) ^ (row & 7)) << 4));
+        uint4 u = *c;
+        if (zero) {
+            u = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+            uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 f = h2<BF16>::to_f2(w[k]);
+                w[k] = h2<BF16>::from_f2(phi_f(f.x), phi_f(f.y));
+            }
+            u = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        *c = u;
+    }
+}
+
+// As phi_half_row, keeping lo = round(phi(x) - hi) in lo_tile (zeroing both when `zero`).
+template <bool BF16>
+__device__ __forceinline__ void phi_half_row_split(uint8_t *tile, uint8_t *lo_tile, int xi, bool zero) {
+    const int row = xi & 127, c0 = (xi >> 7) * 4;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        const int off = row * 128 + (((c0 + it) ^ (row & 7)) << 4);
+        uint4 u = *reinterpret_cast<uint4 *>(tile + off);
+        uint32_t w[4] = {u.x, u.y, u.z, u.w}, l[4] = {0u, 0u, 0u, 0u};
+        if (zero) {
+            w[0] = w[1] = w[2] = w[3] = 0u;
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 f = h2<BF16>::to_f2(w[k]);
+                const float a = phi_f(f.x), b = phi_f(f.y);
+                w[k] = h2<BF16>::from_f2(a, b);
+                const float2 hv = h2<BF16>::to_f2(w[k]);
+                l[k] = h2<BF16>::from_f2(a - hv.x, b - hv.y);
+            }
+        }
+        *reinterpret_cast<uint4 *>(tile + off) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4 *>(lo_tile + off) = make_uint4(l[0], l[1], l[2], l[3]);
+    }
+}
+
+// 16 elements (logical columns 16*c16 .. +15) of row `row` of a swizzled tile.
+template <bool BF16>
+__device__ __forceinline__ void load_chunk16(const uint8_t *tile, int row, int c16, float (&out)[16]) {
+    const uint8_t *p = tile + row * 128;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(p + (((2 * c16 + h) ^ (row & 7)) << 4));
+        const float2 a = h2<BF16>::to_f2(u.x), b = h2<BF16>::to_f2(u.y), d = h2<BF16>::to_f2(u.z),
+                     e = h2<BF16>::to_f2(u.w);
+        out[h * 8 + 0] = a.x; out[h * 8 + 1] = a.y; out[h * 8 + 2] = b.x; out[h * 8 + 3] = b.y;
+        out[h * 8 + 4] = d.x; out[h * 8 + 5] = d.y; out[h * 8 + 6] = e.x; out[h * 8 + 7] = e.y;
+    }
+}
+
+template <bool BF16>
+__device__ __forceinline__ void store_chunk16(uint8_t *tile, int row, int c16, const float (&v)[16]) {
+    uint8_t *p = tile + row * 128;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint4 u;
+        u.x = h2<BF16>::from_f2(v[h * 8 + 0], v[h * 8 + 1]);
+        u.y = h2<BF16>::from_f2(v[h * 8 + 2], v[h * 8 + 3]);
+        u.z = h2<BF16>::from_f2(v[h * 8 + 4], v[h * 8 + 5]);
+        u.w = h2<BF16>::from_f2(v[h * 8 + 6], v[h * 8 + 7]);
+        *reinterpret_cast<uint4 *>(p + (((2 * c16 + h) ^ (row & 7)) << 4)) = u;
     }
 }
 

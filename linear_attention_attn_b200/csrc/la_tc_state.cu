@@ -58,27 +58,44 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 // Partial (S | z) of every (CTA, head) segment.  UMMA M = 64 (the state row i),
 // N = 64 (+16 with the ones block that yields z), K = 128 tile rows:
 //   A = f(K)^T read MN-major from the k tile, B = [V | 1] read MN-major.
+// bf16 bidir also multiplies in lo = round(f(k) - hi) (its own tile), so S and z
+// carry f(k) to fp32 accuracy.
+template <bool BIDIR, bool BF16>
+struct ReduceLayout {
+    static constexpr bool KLO = BIDIR && BF16;
+    static constexpr int NST = KLO ? 4 : 6;
+    static constexpr int koff = 0;
+    static constexpr int voff = koff + NST * kTileBytes;
+    static constexpr int kloff = voff + NST * kTileBytes;
+    static constexpr int onesoff = kloff + (KLO ? NST * kTileBytes : 0);
+    static constexpr int baroff = onesoff + kTileBytes;
+    static constexpr int nbars = 3 * NST + 5;
+    static constexpr int misc = baroff + nbars * 8;
+    static constexpr int bytes = misc + 32 + 1024;
+};
+
 template <bool BIDIR, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     float *__restrict__ part, int T, int BH, int nt, int maxslots) {
-    constexpr bool KLO = BIDIR && BF16;      // bf16: f(k) = hi + lo, both multiplied in
-    constexpr int NST = KLO ? 3 : 4;
+    using L = ReduceLayout<BIDIR, BF16>;
+    constexpr int NST = L::NST;
+    constexpr bool KLO = L::KLO;
     constexpr int N = BIDIR ? 80 : 64;
     constexpr uint32_t IDESC = idesc_f16(64, N, BF16, true, true);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *sK = smem;
-    uint8_t *sV = sK + NST * kTileBytes;
-    uint8_t *sOnes = sV + NST * kTileBytes;
-    uint8_t *sKlo = sOnes + kTileBytes;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sKlo + (KLO ? NST * kTileBytes : 0));
+    uint8_t *sK = smem + L::koff;
+    uint8_t *sV = smem + L::voff;
+    uint8_t *sKlo = smem + L::kloff;
+    uint8_t *sOnes = smem + L::onesoff;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::baroff);
     uint64_t *xf = full + NST;
     uint64_t *empty = xf + NST;
     uint64_t *accfull = empty + NST;   // [2]
     uint64_t *accfree = accfull + 2;   // [2]
     uint64_t *drain = accfree + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc);
     int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -90,12 +107,12 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&xf[s], 4);
+            mbar_init(&xf[s], kXWarps);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&accfull[a], 1);
-            mbar_init(&accfree[a], 4);
+            mbar_init(&accfree[a], kEWarps);
         }
         mbar_init(drain, 1);
         *s_abort = 0;
@@ -105,9 +122,9 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         tma_prefetch(&tmK);
         tma_prefetch(&tmV);
     }
-    if (BIDIR && warp >= 2) {
+    if (BIDIR && warp >= kEw0) {
         // ones block: column 0 (state column 64) = 1 for every tile row, zeros elsewhere
-        const int r = threadIdx.x - 64;
+        const int r = threadIdx.x - kEw0 * 32;
         uint8_t *p = sOnes + r * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(p + c * 16) = make_uint4(0u, 0u, 0u, 0u);
@@ -137,8 +154,7 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 ++issued;
                 if (++s == NST) { s = 0; ph ^= 1; }
             }
-            // on an abort, let the loads in flight land before the CTA's smem goes away
-            if (*s_abort) {
+            if (*s_abort) {   // let the loads in flight land before the CTA's smem goes away
                 for (long long i = issued - 1; i >= 0 && i >= issued - NST; --i)
                     mbar_wait_slow(smem_u32(&full[i % NST]), (uint32_t)((i / NST) & 1), nullptr, &g_tc_fault, 0x200u);
             }
@@ -161,9 +177,9 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 const uint32_t lbo = BIDIR ? (smem_u32(sOnes) - aV) : (uint32_t)kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < kRows / 16; ++kk) {
-                    const uint64_t ad = sdesc_sw128(aK + kk * 2048, kTileBytes, 1024);
                     const uint64_t bd = sdesc_sw128(aV + kk * 2048, lbo, 1024);
-                    umma_f16_ss(d, ad, bd, IDESC, (seg_start && kk == 0) ? 0u : 1u);
+                    umma_f16_ss(d, sdesc_sw128(aK + kk * 2048, kTileBytes, 1024), bd, IDESC,
+                                (seg_start && kk == 0) ? 0u : 1u);
                     if (KLO)
                         umma_f16_ss(d, sdesc_sw128(smem_u32(sKlo + s * kTileBytes) + kk * 2048, kTileBytes, 1024), bd,
                                     IDESC, 1u);
@@ -180,61 +196,63 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             umma_commit(drain);
             mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
         }
-    } else {
-        const int sub = warp & 3;                 // TMEM subpartition of this warp
-        const int row = sub * 32 + lane;          // tile row this thread transforms
-        int s = 0, a = 0;
-        uint32_t ph = 0, aph = 0;
-        for (long long x = x0; x < x1; ++x) {
-            const int h = (int)(x / nt), j = (int)(x % nt);
-            const bool seg_end = (x + 1 == x1) || ((x + 1) / nt != h);
-            if (BIDIR) {
+    } else if (warp < kEw0) {
+        if (BIDIR) {
+            const int xi = threadIdx.x - kXw0 * 32;
+            int s = 0;
+            uint32_t ph = 0;
+            for (long long x = x0; x < x1; ++x) {
+                const int j = (int)(x % nt);
                 const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
                 if (!got) break;
-                if (KLO) {
-                    if (j * kRows + row >= T) {
-                        phi_row_inplace<BF16>(sK + s * kTileBytes, row, true);
-                        phi_row_inplace<BF16>(sKlo + s * kTileBytes, row, true);
-                    } else {
-                        phi_row_split<BF16>(sK + s * kTileBytes, sKlo + s * kTileBytes, row);
-                    }
-                } else {
-                    phi_row_inplace<BF16>(sK + s * kTileBytes, row, j * kRows + row >= T);
-                }
+                const bool pad = j * kRows + (xi & 127) >= T;   // rows past the end: f(0) = 1 must not count
+                if (KLO)
+                    phi_half_row_split<BF16>(sK + s * kTileBytes, sKlo + s * kTileBytes, xi, pad);
+                else
+                    phi_half_row<BF16>(sK + s * kTileBytes, xi, pad);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&xf[s]);
+                if (++s == NST) { s = 0; ph ^= 1; }
             }
-            if (++s == NST) { s = 0; ph ^= 1; }
-            if (seg_end) {
-                const bool got = __all_sync(0xffffffffu, LA_WAIT(&accfull[a], aph, 0x10u));
-                if (!got) break;
-                tc_fence_after();
-                // M = 64 accumulator: state row i = 16*sub + l sits in TMEM lane 32*sub + l (l < 16)
-                const uint32_t base = tmem + (uint32_t)a * 128u + ((uint32_t)(32 * sub) << 16);
-                float v[64];
-                tmem_row64(base, v);
-                float zz = 0.f;
-                if (BIDIR) {
-                    float t16[16];
-                    tmem_ld16(base + 64, t16);
-                    tmem_ld_wait();
-                    zz = t16[0];
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&accfree[a]);
-                if (lane < 16) {
-                    const int i = 16 * sub + lane;
-                    const int slot = cta - P.first_cta(h);
-                    float *dst = part + (((long long)h * maxslots + slot) * 64 + i) * 65;
+        }
+    } else {
+        const int sub = warp & 3;
+        int a = 0;
+        uint32_t aph = 0;
+        for (long long x = x0; x < x1; ++x) {
+            const int h = (int)(x / nt);
+            const bool seg_end = (x + 1 == x1) || ((x + 1) / nt != h);
+            if (!seg_end) continue;
+            const bool got = __all_sync(0xffffffffu, LA_WAIT(&accfull[a], aph, 0x10u));
+            if (!got) break;
+            tc_fence_after();
+            // M = 64 accumulator: state row i = 16*sub + l sits in TMEM lane 32*sub + l (l < 16)
+            const uint32_t base = tmem + (uint32_t)a * 128u + ((uint32_t)(32 * sub) << 16);
+            float v[64];
+            tmem_row64(base, v);
+            float zz = 0.f;
+            if (BIDIR) {
+                float t16[16];
+                tmem_ld16(base + 64, t16);
+                tmem_ld_wait();
+                zz = t16[0];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accfree[a]);
+            if (lane < 16) {
+                const int i = 16 * sub + lane;
+                const int slot = cta - P.first_cta(h);
+                float4 *dst = reinterpret_cast<float4 *>(part + ((long long)h * maxslots + slot) * kStateElems);
+                // row i of the [64][65] block: 65 floats starting at i*65 (not 16-byte aligned): scalar stores
+                float *d1 = reinterpret_cast<float *>(dst) + i * 65;
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) dst[c] = v[c];
-                    dst[64] = zz;
-                }
-                a ^= 1;
-                if (a == 0) aph ^= 1;
+                for (int c = 0; c < 64; ++c) d1[c] = v[c];
+                d1[64] = zz;
             }
+            a ^= 1;
+            if (a == 0) aph ^= 1;
         }
     }
     tc_fence_before();
@@ -247,35 +265,49 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 
 // ================================================================= output ==
 // o = f(q) [S | z] / n per tile: UMMA M = 128 rows, N = 80 (64 + z + pad) or 64,
-// K = 64, A = f(Q) tile K-major, B = state operand K-major (hi [+ lo]).
+// K = 64, A = f(Q) tile K-major, B = state operand K-major (hi [+ lo]).  The
+// epilogue warps build the operand of the CTA's next head into the second of
+// two operand buffers while the current head's tiles stream.
+struct OutputLayout {
+    static constexpr int NST = 6, OST = 2, OPB = 80 * 128;
+    static constexpr int qoff = 0;
+    static constexpr int ooff = qoff + NST * kTileBytes;
+    static constexpr int opoff = ooff + OST * kTileBytes;      // [buffer][hi, lo]
+    static constexpr int stageoff = opoff + 4 * OPB;
+    static constexpr int redoff = stageoff + kStateElems * 4;
+    static constexpr int baroff = redoff + 32;
+    static constexpr int nbars = 3 * NST + 2 + 2 + 2 + 1;
+    static constexpr int misc = baroff + nbars * 8;
+    static constexpr int bytes = misc + 32 + 1024;
+};
+
 template <bool BIDIR, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
               const float *__restrict__ src, int src_per_head, int src_single, float *__restrict__ state_out, int T,
               int BH, int nt, float eps) {
-    constexpr int NST = 4;
-    constexpr int OST = 2;
+    using L = OutputLayout;
+    constexpr int NST = L::NST, OST = L::OST, OPB = L::OPB;
     constexpr int NOPS = BF16 ? 2 : 1;
     constexpr int N = BIDIR ? 80 : 64;
-    constexpr int OPB = 80 * 128;                 // operand bytes (80 rows)
     constexpr uint32_t IDESC = idesc_f16(128, N, BF16, false, false);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *sQ = smem;
-    uint8_t *sO = sQ + NST * kTileBytes;
-    uint8_t *sOp = sO + OST * kTileBytes;          // NOPS x OPB (1024-aligned: OPB = 10 x 1024)
-    float *stage = reinterpret_cast<float *>(sOp + 2 * OPB);
-    float *red = stage + kStateElems;
-    uint64_t *full = reinterpret_cast<uint64_t *>(red + 8);
+    uint8_t *sQ = smem + L::qoff;
+    uint8_t *sO = smem + L::ooff;
+    uint8_t *sOp = smem + L::opoff;
+    float *stage = reinterpret_cast<float *>(smem + L::stageoff);
+    float *red = reinterpret_cast<float *>(smem + L::redoff);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::baroff);
     uint64_t *xf = full + NST;
     uint64_t *empty = xf + NST;
     uint64_t *accfull = empty + NST;
     uint64_t *accempty = accfull + 2;
-    uint64_t *opready = accempty + 2;
-    uint64_t *drain = opready + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *opready = accempty + 2;   // [2]
+    uint64_t *drain = opready + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc);
     int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
-    float *s_scale = reinterpret_cast<float *>(s_abort + 1);
+    float *s_scale = reinterpret_cast<float *>(tmem_slot + 2);   // [2]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Partition P{(long long)BH * nt, nt, grid_for((long long)BH * nt)};
@@ -286,14 +318,14 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&xf[s], 4);
+            mbar_init(&xf[s], kXWarps);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&accfull[a], 1);
-            mbar_init(&accempty[a], 4);
+            mbar_init(&accempty[a], kEWarps);
+            mbar_init(&opready[a], 1);
         }
-        mbar_init(opready, 1);
         mbar_init(drain, 1);
         *s_abort = 0;
         fence_mbar_init();
@@ -331,29 +363,28 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            int s = 0, a = 0;
-            uint32_t ph = 0, aph = 0, oph = 0;
+            int s = 0, a = 0, hidx = -1;
+            uint32_t ph = 0, aph = 0;
             long long prev_h = -1;
             for (long long x = x0; x < x1; ++x) {
                 const long long h = x / nt;
                 if (h != prev_h) {
-                    if (!LA_WAIT(opready, oph, 0x20u)) break;
-                    oph ^= 1;
+                    ++hidx;
                     prev_h = h;
+                    if (!LA_WAIT(&opready[hidx & 1], (uint32_t)((hidx >> 1) & 1), 0x20u)) break;
                 }
                 if (!LA_WAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
                 if (!LA_WAIT(&accempty[a], aph ^ 1, 0x2u)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)a * 128u;
                 const uint32_t aQ = smem_u32(sQ + s * kTileBytes);
+                const uint32_t aOp = smem_u32(sOp + (hidx & 1) * 2 * OPB);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
-                    for (int op = 0; op < NOPS; ++op) {
-                        const uint64_t ad = sdesc_sw128(aQ + kk * 32, 16, 1024);
-                        const uint64_t bd = sdesc_sw128(smem_u32(sOp + op * OPB) + kk * 32, 16, 1024);
-                        umma_f16_ss(d, ad, bd, IDESC, (kk | op) ? 1u : 0u);
-                    }
+                    for (int op = 0; op < NOPS; ++op)
+                        umma_f16_ss(d, sdesc_sw128(aQ + kk * 32, 16, 1024),
+                                    sdesc_sw128(aOp + op * OPB + kk * 32, 16, 1024), IDESC, (kk | op) ? 1u : 0u);
                 }
                 umma_commit(&empty[s]);
                 umma_commit(&accfull[a]);
@@ -364,102 +395,104 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             umma_commit(drain);
             mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
         }
+    } else if (warp < kEw0) {
+        if (BIDIR) {
+            const int xi = threadIdx.x - kXw0 * 32;
+            int s = 0;
+            uint32_t ph = 0;
+            for (long long x = x0; x < x1; ++x) {
+                const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
+                if (!got) break;
+                phi_half_row<BF16>(sQ + s * kTileBytes, xi, false);   // rows past T are never stored
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xf[s]);
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+        }
     } else {
-        // Workers.  Every named barrier below is reached by all 128 workers whatever
-        // happens to the mbarrier waits (a failed wait only skips the work), so an
-        // abort cannot leave a worker stuck at a barrier.
-        const int tid = threadIdx.x - 64;          // 0..127
+        // Epilogue warps.  Every named barrier is reached by all 128 of them whatever
+        // the mbarrier waits return (a failed wait only skips work).
+        const int tid = threadIdx.x - kEw0 * 32;
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
-        int s = 0, a = 0, ob = 0;
-        uint32_t ph = 0, aph = 0;
-        long long prev_h = -1;
+        int a = 0, ob = 0, hidx = -1;
+        uint32_t aph = 0;
+        long long cur_h = -1;
         bool live = true;
-        auto epilogue = [&](long long xe, int ae, uint32_t aphe) {
-            const int h = (int)(xe / nt), j = (int)(xe % nt);
-            bool got = live && LA_WAIT(&accfull[ae], aphe, 0x10u);
+        auto build = [&](long long h, int buf) {
+            const float *srch = src + h * (long long)src_per_head;
+            const int ns = src_single ? 1 : (P.last_cta((int)h) - P.first_cta((int)h) + 1);
+            float m = gather_state(srch, ns, stage, tid);
+            named_bar(1, kWorkers);
+            if (state_out && h * nt >= x0) {   // this CTA holds the head's first tile: it writes the state
+                float4 *dst = reinterpret_cast<float4 *>(state_out + h * (long long)kStateElems);
+                const float4 *st4 = reinterpret_cast<const float4 *>(stage);
+                for (int e = tid; e < kStateElems / 4; e += kWorkers) dst[e] = st4[e];
+            }
+            if (!BF16) m = workers_max(m, red, tid);
+            const float sc = operand_scale<BF16>(m);
+            uint8_t *op0 = sOp + buf * 2 * OPB;
+            if (tid < 80) {
+                float xv[64];
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    xv[i] = tid < 64 ? stage[i * 65 + tid] * sc : ((BIDIR && tid == 64) ? stage[i * 65 + 64] * sc : 0.f);
+                operand_row<BF16, NOPS>(op0, op0 + OPB, tid, xv);
+            }
+            if (tid == 0) s_scale[buf] = sc;
+            fence_async_smem();
+            named_bar(1, kWorkers);
+            if (tid == 0) mbar_arrive(&opready[buf]);
+        };
+        for (long long x = x0; x < x1; ++x) {
+            const long long h = x / nt;
+            const int j = (int)(x % nt);
+            if (h != cur_h) {
+                ++hidx;
+                cur_h = h;
+                if (hidx == 0) build(h, 0);
+            }
+            // ---- epilogue of tile x
+            if (tid == 0) tma_store_wait_read<OST - 1>();
+            named_bar(1, kWorkers);
+            bool got = live && LA_WAIT(&accfull[a], aph, 0x10u);
             got = __all_sync(0xffffffffu, got);
             live = live && got;
-            float v[64];
-            float nz = 0.f;
             if (got) {
                 tc_fence_after();
-                const uint32_t base = tmem + (uint32_t)ae * 128u + ((uint32_t)(32 * sub) << 16);
-                tmem_row64(base, v);
+                const uint32_t base = tmem + (uint32_t)a * 128u + ((uint32_t)(32 * sub) << 16);
+                const float sc = s_scale[hidx & 1];
+                float inv = 1.f / sc;
                 if (BIDIR) {
                     float t16[16];
                     tmem_ld16(base + 64, t16);
                     tmem_ld_wait();
-                    nz = t16[0];
+                    inv = 1.f / (t16[0] + eps * sc);
                 }
+                float v[64];
+                tmem_row64(base, v);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&accempty[ae]);
-                const float sc = *s_scale;
-                const float inv = BIDIR ? 1.f / (nz + eps * sc) : 1.f / sc;
+                if (lane == 0) mbar_arrive(&accempty[a]);
 #pragma unroll
                 for (int c = 0; c < 64; ++c) v[c] *= inv;
+                store_row<BF16>(sO + ob * kTileBytes, row, v);
             }
-            if (tid == 0) tma_store_wait_read<OST - 1>();
-            named_bar(1, kWorkers);
-            if (got) store_row<BF16>(sO + ob * kTileBytes, row, v);
             fence_async_smem();
             named_bar(1, kWorkers);
             if (tid == 0 && live) {
-                tma_store_3d(&tmO, sO + ob * kTileBytes, 0, j * kRows, h);
+                tma_store_3d(&tmO, sO + ob * kTileBytes, 0, j * kRows, (int)h);
                 tma_store_commit();
             }
             if (++ob == OST) ob = 0;
-        };
-        int a_prev = 0;
-        uint32_t aph_prev = 0;
-        for (long long x = x0; x < x1; ++x) {
-            const long long h = x / nt;
-            if (BIDIR) {
-                bool got = live && LA_WAIT(&full[s], ph, 0x8u);
-                got = __all_sync(0xffffffffu, got);
-                live = live && got;
-                if (got) {
-                    phi_row_inplace<BF16>(sQ + s * kTileBytes, row, false);
-                    fence_async_smem();
-                }
-                __syncwarp();
-                if (lane == 0 && got) mbar_arrive(&xf[s]);
-            }
-            if (++s == NST) { s = 0; ph ^= 1; }
-            if (x > x0) epilogue(x - 1, a_prev, aph_prev);
-            if (h != prev_h) {
-                // the previous head's UMMAs are complete: its last epilogue waited on them
-                const float *srch = src + h * (long long)src_per_head;
-                const int ns = src_single ? 1 : (P.last_cta((int)h) - P.first_cta((int)h) + 1);
-                float m = gather_state(srch, ns, stage, tid);
-                named_bar(1, kWorkers);
-                if (state_out && (x % nt) == 0) {
-                    float *dst = state_out + h * (long long)kStateElems;
-                    for (int e = tid; e < kStateElems; e += kWorkers) dst[e] = stage[e];
-                }
-                if (!BF16) m = workers_max(m, red, tid);
-                const float sc = operand_scale<BF16>(m);
-                if (tid < 80) {
-                    float xv[64];
-#pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        xv[i] = tid < 64 ? stage[i * 65 + tid] * sc
-                                         : ((BIDIR && tid == 64) ? stage[i * 65 + 64] * sc : 0.f);
-                    operand_row<BF16, NOPS>(sOp, sOp + OPB, tid, xv);
-                }
-                if (tid == 0) *s_scale = sc;
-                fence_async_smem();
-                named_bar(1, kWorkers);
-                if (tid == 0) mbar_arrive(opready);
-                prev_h = h;
-            }
-            a_prev = a;
-            aph_prev = aph;
             a ^= 1;
             if (a == 0) aph ^= 1;
+            // ---- the next head's operand, into the other buffer (its last user, the
+            //      head before this one, has finished all its UMMAs)
+            const bool first_of_head = (x == x0) || (j == 0);
+            if (first_of_head && (h + 1) * nt < x1) build(h + 1, (hidx + 1) & 1);
         }
-        epilogue(x1 - 1, a_prev, aph_prev);
         if (tid == 0) tma_store_wait_all<0>();
     }
     tc_fence_before();
@@ -470,18 +503,17 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
 }
 
-
 // ================================================================== bwd_q ==
 // Per tile: MMA1 [u | q.z] = f(Q) [S | z] (M=128, N=80), MMA2 g S^T (M=128, N=64,
-// B = the state operand read MN-major); the workers form n, o, g.o, dq and write
-// g/n (in place over the dO tile) and w = -(g.o)/n (column 0 of a zero block);
-// MMA3 accumulates [dS | dz] += f(Q)^T [g/n | w] (M=64, N=80, both MN-major).
-// bf16 bidir also keeps lo = round(f(q) - hi) of the feature map (one more tile per
-// stage): MMA1 then adds f(Q)_lo S_hi, and f'(q) = min(hi + lo, 1).
+// B = the state operand read MN-major); the epilogue warps form n, o, g.o and dq
+// and write g/n (in place over the dO tile) and w = -(g.o)/n (column 0 of a
+// zero block); MMA3 accumulates [dS | dz] += f(Q)^T [g/n | w] (M=64, N=80, both
+// MN-major).  bf16 bidir also keeps lo = round(f(q) - hi): MMA1 adds
+// f(Q)_lo S_hi and f'(q) = min(hi + lo, 1).
 template <bool BIDIR, bool BF16>
 struct BwdQLayout {
     static constexpr bool QLO = BIDIR && BF16;
-    static constexpr int NST = QLO ? 2 : 3, OST = 2, OPB = 80 * 128;
+    static constexpr int NST = BIDIR ? (QLO ? 2 : 3) : 4, OST = 1, OPB = 80 * 128;
     static constexpr int qoff = 0;
     static constexpr int goff = qoff + NST * kTileBytes;
     static constexpr int woff = goff + NST * kTileBytes;
@@ -492,7 +524,7 @@ struct BwdQLayout {
     static constexpr int zsoff = stageoff + kStateElems * 4;
     static constexpr int redoff = zsoff + 64 * 4;
     static constexpr int baroff = redoff + 32;
-    static constexpr int nbars = 4 * NST + 4 + 4;
+    static constexpr int nbars = 4 * NST + 8;
     static constexpr int misc = baroff + nbars * 8;
     static constexpr int bytes = misc + 32 + 1024;
 };
@@ -503,12 +535,11 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
              const __grid_constant__ CUtensorMap tmDQ, const float *__restrict__ src, int src_per_head,
              int src_single, float *__restrict__ dpart, int T, int BH, int nt, int maxslots, float eps) {
     using L = BwdQLayout<BIDIR, BF16>;
-    constexpr int NST = L::NST, OST = L::OST, OPB = L::OPB;
+    constexpr int NST = L::NST, OPB = L::OPB;
     constexpr bool QLO = L::QLO;
     constexpr int NOPS = BF16 ? 2 : 1;
-    constexpr int N1 = 80;
     constexpr int N3 = BIDIR ? 80 : 64;
-    constexpr uint32_t IDESC1 = idesc_f16(128, N1, BF16, false, false);
+    constexpr uint32_t IDESC1 = idesc_f16(128, 80, BF16, false, false);
     constexpr uint32_t IDESC2 = idesc_f16(128, 64, BF16, false, true);
     constexpr uint32_t IDESC3 = idesc_f16(64, N3, BF16, true, true);
     extern __shared__ uint8_t smem_raw[];
@@ -544,16 +575,16 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&xf[s], 4);
-            mbar_init(&gnready[s], 4);
+            mbar_init(&xf[s], kXWarps);
+            mbar_init(&gnready[s], kEWarps);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc12full[b], 1);
-            mbar_init(&acc12empty[b], 4);
+            mbar_init(&acc12empty[b], kEWarps);
         }
         mbar_init(accSfull, 1);
-        mbar_init(accSfree, 4);
+        mbar_init(accSfree, kEWarps);
         mbar_init(opready, 1);
         mbar_init(drain, 1);
         *s_abort = 0;
@@ -564,8 +595,8 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         tma_prefetch(&tmG);
         tma_prefetch(&tmDQ);
     }
-    if (BIDIR && warp >= 2) {
-        const int r = threadIdx.x - 64;
+    if (BIDIR && warp >= kEw0) {   // the w blocks: zero except column 0, written per tile
+        const int r = threadIdx.x - kEw0 * 32;
         for (int st = 0; st < NST; ++st) {
             uint8_t *p = sW + st * kTileBytes + r * 128;
 #pragma unroll
@@ -607,7 +638,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             int s = 0, b = 0;
             uint32_t ph = 0, bph = 0, oph = 0;
             long long prev_h = -1;
-            long long seg = 0;                     // segments started (for the accS free parity)
+            long long seg = 0;                     // segments started (accS free parity)
             bool dead = false;
             // MMA3 of tile xe (stage se, phase phe)
             auto issue3 = [&](long long xe, int se, uint32_t phe) {
@@ -622,11 +653,9 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 const uint32_t aQ = smem_u32(sQ + se * kTileBytes), aG = smem_u32(sG + se * kTileBytes);
                 const uint32_t lbo = BIDIR ? smem_u32(sW + se * kTileBytes) - aG : (uint32_t)kTileBytes;
 #pragma unroll
-                for (int kk = 0; kk < kRows / 16; ++kk) {
-                    const uint64_t ad = sdesc_sw128(aQ + kk * 2048, kTileBytes, 1024);
-                    const uint64_t bd = sdesc_sw128(aG + kk * 2048, lbo, 1024);
-                    umma_f16_ss(tmem + kAccS, ad, bd, IDESC3, (seg_start && kk == 0) ? 0u : 1u);
-                }
+                for (int kk = 0; kk < kRows / 16; ++kk)
+                    umma_f16_ss(tmem + kAccS, sdesc_sw128(aQ + kk * 2048, kTileBytes, 1024),
+                                sdesc_sw128(aG + kk * 2048, lbo, 1024), IDESC3, (seg_start && kk == 0) ? 0u : 1u);
                 umma_commit(&empty[se]);
                 if (seg_end) umma_commit(accSfull);
             };
@@ -636,6 +665,12 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             for (long long x = x0; x < x1 && !dead; ++x) {
                 const long long h = x / nt;
                 if (h != prev_h) {
+                    // finish the previous head (its dS partial) before waiting on the next operand
+                    if (xp >= 0) {
+                        issue3(xp, sp, php);
+                        xp = -1;
+                        if (dead) break;
+                    }
                     if (!LA_WAIT(opready, oph, 0x20u)) break;
                     oph ^= 1;
                     prev_h = h;
@@ -673,89 +708,66 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             umma_commit(drain);
             mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
         }
+    } else if (warp < kEw0) {
+        if (BIDIR) {
+            const int xi = threadIdx.x - kXw0 * 32;
+            int s = 0;
+            uint32_t ph = 0;
+            for (long long x = x0; x < x1; ++x) {
+                const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
+                if (!got) break;
+                if (QLO)
+                    phi_half_row_split<BF16>(sQ + s * kTileBytes, sQlo + s * kTileBytes, xi, false);
+                else
+                    phi_half_row<BF16>(sQ + s * kTileBytes, xi, false);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xf[s]);
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+        }
     } else {
-        // Workers (every named barrier is reached by all 128 whatever the waits return).
-        const int tid = threadIdx.x - 64;
+        // Epilogue warps (every named barrier is reached by all 128 whatever the waits return).
+        const int tid = threadIdx.x - kEw0 * 32;
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
-        int s = 0, b = 0, ob = 0;
-        uint32_t ph = 0, bph = 0;
-        long long prev_h = -1;
-        uint32_t sfull_ph = 0;
+        int s = 0, b = 0;
+        uint32_t ph = 0, bph = 0, sfull_ph = 0;
+        long long cur_h = -1;
         bool live = true;
         float cur_sc = 1.f, cur_scn = 1.f;
 
-        auto epilogue = [&](long long xe, int se, uint32_t phe, int be, uint32_t bphe) {
-            const int h = (int)(xe / nt), j = (int)(xe % nt);
-            bool got = live && LA_WAIT(&acc12full[be], bphe, 0x10u);
-            got = __all_sync(0xffffffffu, got);
-            live = live && got;
-            const uint32_t lanes = (uint32_t)(32 * sub) << 16;
-            const uint32_t d1 = tmem + (uint32_t)be * 256u + lanes, d2 = d1 + 96u;
-            uint8_t *tq = sQ + se * kTileBytes, *tg = sG + se * kTileBytes;
-            uint8_t *dqrow = sDQ + ob * kTileBytes;
-            float gdot = 0.f, inv = 1.f;
-            float dq[64];
-            if (got) {
-                tc_fence_after();
-                if (BIDIR) {
-                    float u[64], g[64];
-                    tmem_row64(d1, u);
-                    float t16[16];
-                    tmem_ld16(d1 + 64, t16);
-                    tmem_ld_wait();
-                    inv = 1.f / (t16[0] + eps * cur_sc);
-                    load_row<BF16>(tg, row, g);
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) gdot = fmaf(g[c], u[c] * inv, gdot);
-                    const float gsc = inv * cur_sc * cur_scn;
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) g[c] *= gsc;
-                    store_row<BF16>(tg, row, g);    // g/n (scaled) replaces dO in place: MMA2 is done
-                    const float w = -gdot * gsc;
-                    if (BF16) {
-                        __nv_bfloat16 wv = __float2bfloat16_rn(w);
-                        *reinterpret_cast<__nv_bfloat16 *>(sW + se * kTileBytes + sw128_offset(row, 0)) = wv;
-                    } else {
-                        __half wv = __float2half_rn(w);
-                        *reinterpret_cast<__half *>(sW + se * kTileBytes + sw128_offset(row, 0)) = wv;
-                    }
-                }
-                tmem_row64(d2, dq);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc12empty[be]);
-                if (BIDIR) {
-                    float qf[64];
-                    load_row<BF16>(tq, row, qf);
-                    if (QLO) {
-                        float ql[64];
-                        load_row<BF16>(sQlo + se * kTileBytes, row, ql);
-#pragma unroll
-                        for (int c = 0; c < 64; ++c) qf[c] += ql[c];
-                    }
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) dq[c] = (dq[c] - gdot * zs[c]) * inv * fminf(qf[c], 1.f);
-                } else {
-                    const float isc = 1.f / cur_sc;
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) dq[c] *= isc;
-                }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&gnready[se]);
-            }
-            if (tid == 0) tma_store_wait_read<OST - 1>();
+        auto build = [&](long long h) {
+            const float *srch = src + h * (long long)src_per_head;
+            const int ns = src_single ? 1 : (P.last_cta((int)h) - P.first_cta((int)h) + 1);
+            float m = gather_state(srch, ns, stage, tid);
             named_bar(1, kWorkers);
-            if (got) store_row<BF16>(dqrow, row, dq);
+            if (!BF16) m = workers_max(m, red, tid);
+            const float sc = operand_scale<BF16>(m);
+            float zsum = 0.f;
+            for (int i = 0; i < 64; ++i) zsum += fabsf(stage[i * 65 + 64]);
+            float scn = 1.f;
+            if (BIDIR && zsum > 0.f && isfinite(zsum)) {
+                int e;
+                frexpf(zsum, &e);
+                e = e < -100 ? -100 : (e > 100 ? 100 : e);
+                scn = ldexpf(1.f, e - 1);
+            }
+            if (tid < 80) {
+                float xv[64];
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    xv[i] = tid < 64 ? stage[i * 65 + tid] * sc : ((BIDIR && tid == 64) ? stage[i * 65 + 64] * sc : 0.f);
+                operand_row<BF16, NOPS>(sOp, sOp + OPB, tid, xv);
+            }
+            if (tid < 64) zs[tid] = stage[tid * 65 + 64] * sc;
             fence_async_smem();
             named_bar(1, kWorkers);
-            if (tid == 0 && live) {
-                tma_store_3d(&tmDQ, dqrow, 0, j * kRows, h);
-                tma_store_commit();
-            }
-            if (++ob == OST) ob = 0;
+            cur_sc = sc;
+            cur_scn = scn;
+            if (tid == 0) mbar_arrive(opready);
         };
+
         // [dS | dz] partial of the segment of head hs that just ended
         auto read_accS = [&](int hs, float scn) {
             bool got = live && LA_WAIT(accSfull, sfull_ph, 0x100u);
@@ -788,69 +800,96 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             }
         };
 
-        int s_prev = 0, b_prev = 0;
-        uint32_t ph_prev = 0, bph_prev = 0;
         for (long long x = x0; x < x1; ++x) {
             const long long h = x / nt;
-            if (BIDIR) {
-                bool got = live && LA_WAIT(&full[s], ph, 0x8u);
-                got = __all_sync(0xffffffffu, got);
-                live = live && got;
-                if (got) {
-                    if (QLO)
-                        phi_row_split<BF16>(sQ + s * kTileBytes, sQlo + s * kTileBytes, row);
-                    else
-                        phi_row_inplace<BF16>(sQ + s * kTileBytes, row, false);
-                    fence_async_smem();
-                }
-                __syncwarp();
-                if (lane == 0 && got) mbar_arrive(&xf[s]);
+            const int j = (int)(x % nt);
+            if (h != cur_h) {
+                build(h);
+                cur_h = h;
             }
-            if (x > x0) epilogue(x - 1, s_prev, ph_prev, b_prev, bph_prev);
-            const float prev_scn = cur_scn;
-            if (h != prev_h) {
-                const float *srch = src + h * (long long)src_per_head;
-                const int ns = src_single ? 1 : (P.last_cta((int)h) - P.first_cta((int)h) + 1);
-                float m = gather_state(srch, ns, stage, tid);
-                named_bar(1, kWorkers);
-                if (!BF16) m = workers_max(m, red, tid);
-                const float sc = operand_scale<BF16>(m);
-                float zsum = 0.f;
-                for (int i = 0; i < 64; ++i) zsum += fabsf(stage[i * 65 + 64]);
-                float scn = 1.f;
-                if (BIDIR && zsum > 0.f && isfinite(zsum)) {
-                    int e;
-                    frexpf(zsum, &e);
-                    e = e < -100 ? -100 : (e > 100 ? 100 : e);
-                    scn = ldexpf(1.f, e - 1);
-                }
-                if (tid < 80) {
-                    float xv[64];
+            // ---- epilogue of tile x (stage s, accumulator pair b)
+            if (tid == 0) tma_store_wait_read<0>();
+            named_bar(1, kWorkers);
+            bool got = live && LA_WAIT(&acc12full[b], bph, 0x10u);
+            got = __all_sync(0xffffffffu, got);
+            live = live && got;
+            if (got) {
+                tc_fence_after();
+                const uint32_t lanes = (uint32_t)(32 * sub) << 16;
+                const uint32_t d1 = tmem + (uint32_t)b * 256u + lanes, d2 = d1 + 96u;
+                uint8_t *tq = sQ + s * kTileBytes, *tg = sG + s * kTileBytes;
+                float gdot = 0.f, inv = 1.f;
+                if (BIDIR) {
+                    float t16[16];
+                    tmem_ld16(d1 + 64, t16);
+                    tmem_ld_wait();
+                    inv = 1.f / (t16[0] + eps * cur_sc);
+                    const float gsc = inv * cur_sc * cur_scn;
 #pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        xv[i] = tid < 64 ? stage[i * 65 + tid] * sc
-                                         : ((BIDIR && tid == 64) ? stage[i * 65 + 64] * sc : 0.f);
-                    operand_row<BF16, NOPS>(sOp, sOp + OPB, tid, xv);
+                    for (int c16 = 0; c16 < 4; ++c16) {
+                        float u[16], g[16];
+                        tmem_ld16(d1 + 16 * c16, u);
+                        load_chunk16<BF16>(tg, row, c16, g);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            gdot = fmaf(g[i], u[i], gdot);
+                            g[i] *= gsc;
+                        }
+                        store_chunk16<BF16>(tg, row, c16, g);   // g/n (scaled) over dO: MMA2 is done with it
+                    }
+                    gdot *= inv;
+                    const float w = -gdot * gsc;
+                    if (BF16)
+                        *reinterpret_cast<__nv_bfloat16 *>(sW + s * kTileBytes + sw128_offset(row, 0)) = __float2bfloat16_rn(w);
+                    else
+                        *reinterpret_cast<__half *>(sW + s * kTileBytes + sw128_offset(row, 0)) = __float2half_rn(w);
                 }
-                if (tid < 64) zs[tid] = stage[tid * 65 + 64] * sc;
+                const float isc = 1.f / cur_sc;
+#pragma unroll
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    float acc[16], dq[16];
+                    tmem_ld16(d2 + 16 * c16, acc);
+                    if (BIDIR) {
+                        float qf[16];
+                        load_chunk16<BF16>(tq, row, c16, qf);
+                        if (QLO) {
+                            float ql[16];
+                            load_chunk16<BF16>(sQlo + s * kTileBytes, row, c16, ql);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) qf[i] += ql[i];
+                        }
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            dq[i] = (acc[i] - gdot * zs[16 * c16 + i]) * inv * fminf(qf[i], 1.f);
+                    } else {
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) dq[i] = acc[i] * isc;
+                    }
+                    store_chunk16<BF16>(sDQ, row, c16, dq);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc12empty[b]);
                 fence_async_smem();
-                named_bar(1, kWorkers);
-                cur_sc = sc;
-                cur_scn = scn;
-                if (tid == 0) mbar_arrive(opready);
-                if (x > x0) read_accS((int)((x - 1) / nt), prev_scn);   // the previous head's segment ended
-                prev_h = h;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&gnready[s]);
+            } else {
+                fence_async_smem();
             }
-            s_prev = s;
-            ph_prev = ph;
-            b_prev = b;
-            bph_prev = bph;
+            named_bar(1, kWorkers);
+            if (tid == 0 && live) {
+                tma_store_3d(&tmDQ, sDQ, 0, j * kRows, (int)h);
+                tma_store_commit();
+            }
+            const bool seg_end = (x + 1 == x1) || ((x + 1) % nt == 0);
+            if (seg_end) read_accS((int)h, cur_scn);
             if (++s == NST) { s = 0; ph ^= 1; }
             b ^= 1;
             if (b == 0) bph ^= 1;
         }
-        epilogue(x1 - 1, s_prev, ph_prev, b_prev, bph_prev);
-        read_accS((int)((x1 - 1) / nt), cur_scn);
         if (tid == 0) tma_store_wait_all<0>();
     }
     tc_fence_before();
@@ -866,7 +905,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 //           MMA_b  f(K) dS (A = f(K) tile, B = dS operand read MN-major);
 // dk = (v dS^T + dz) f'(k), dv = f(k) dS.  The dS operand rows are dS's rows.
 struct BwdKvLayout {
-    static constexpr int NST = 3, OST = 2, OPB = 64 * 128;
+    static constexpr int NST = 4, OST = 1, OPB = 64 * 128;
     static constexpr int koff = 0;
     static constexpr int voff = koff + NST * kTileBytes;
     static constexpr int dkoff = voff + NST * kTileBytes;
@@ -887,7 +926,7 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
               const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
               const float *__restrict__ dpart, int T, int BH, int nt, int maxslots) {
     using L = BwdKvLayout;
-    constexpr int NST = L::NST, OST = L::OST, OPB = L::OPB;
+    constexpr int NST = L::NST, OPB = L::OPB;
     constexpr int NOPS = BF16 ? 2 : 1;
     constexpr uint32_t IDESC_A = idesc_f16(128, 64, BF16, false, false);
     constexpr uint32_t IDESC_B = idesc_f16(128, 64, BF16, false, true);
@@ -920,12 +959,12 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&xf[s], 4);
-            mbar_init(&empty[s], BIDIR ? 5 : 1);   // UMMA commit (+ the 4 worker warps that read f(k) for f'(k))
+            mbar_init(&xf[s], kXWarps);
+            mbar_init(&empty[s], BIDIR ? 1 + kEWarps : 1);   // UMMA commit (+ the epilogue warps read f(k))
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&accfull[b], 1);
-            mbar_init(&accempty[b], 4);
+            mbar_init(&accempty[b], kEWarps);
         }
         mbar_init(opready, 1);
         mbar_init(drain, 1);
@@ -1003,79 +1042,35 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             umma_commit(drain);
             mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
         }
+    } else if (warp < kEw0) {
+        if (BIDIR) {
+            const int xi = threadIdx.x - kXw0 * 32;
+            int s = 0;
+            uint32_t ph = 0;
+            for (long long x = x0; x < x1; ++x) {
+                const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
+                if (!got) break;
+                phi_half_row<BF16>(sK + s * kTileBytes, xi, false);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xf[s]);
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+        }
     } else {
-        const int tid = threadIdx.x - 64;
+        const int tid = threadIdx.x - kEw0 * 32;
         const int sub = warp & 3;
         const int row = sub * 32 + lane;
-        int s = 0, b = 0, ob = 0;
-        uint32_t ph = 0, bph = 0;
-        long long prev_h = -1;
+        int s = 0, b = 0;
+        uint32_t bph = 0;
+        long long cur_h = -1;
         bool live = true;
         float cur_isd = 1.f;
-
-        auto epilogue = [&](long long xe, int se, int be, uint32_t bphe) {
-            const int h = (int)(xe / nt), j = (int)(xe % nt);
-            bool got = live && LA_WAIT(&accfull[be], bphe, 0x10u);
-            got = __all_sync(0xffffffffu, got);
-            live = live && got;
-            const uint32_t da = tmem + (uint32_t)be * 128u + ((uint32_t)(32 * sub) << 16), db = da + 64u;
-            float dk[64], dv[64];
-            if (got) {
-                tc_fence_after();
-                tmem_row64(da, dk);
-                tmem_row64(db, dv);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&accempty[be]);
-                if (BIDIR) {
-                    float kf[64];
-                    load_row<BF16>(sK + se * kTileBytes, row, kf);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[se]);   // f(k) read: the stage may be reloaded
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) dk[c] = fmaf(dk[c], cur_isd, dz[c]) * fminf(kf[c], 1.f);
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) dk[c] *= cur_isd;
-                }
-#pragma unroll
-                for (int c = 0; c < 64; ++c) dv[c] *= cur_isd;
-            } else if (BIDIR) {
-                __syncwarp();
-            }
-            if (tid == 0) tma_store_wait_read<OST - 1>();
-            named_bar(1, kWorkers);
-            if (got) {
-                store_row<BF16>(sDK + ob * kTileBytes, row, dk);
-                store_row<BF16>(sDV + ob * kTileBytes, row, dv);
-            }
-            fence_async_smem();
-            named_bar(1, kWorkers);
-            if (tid == 0 && live) {
-                tma_store_3d(&tmDK, sDK + ob * kTileBytes, 0, j * kRows, h);
-                tma_store_3d(&tmDV, sDV + ob * kTileBytes, 0, j * kRows, h);
-                tma_store_commit();
-            }
-            if (++ob == OST) ob = 0;
-        };
-
-        int s_prev = 0, b_prev = 0;
-        uint32_t bph_prev = 0;
         for (long long x = x0; x < x1; ++x) {
             const long long h = x / nt;
-            if (BIDIR) {
-                bool got = live && LA_WAIT(&full[s], ph, 0x8u);
-                got = __all_sync(0xffffffffu, got);
-                live = live && got;
-                if (got) {
-                    phi_row_inplace<BF16>(sK + s * kTileBytes, row, false);
-                    fence_async_smem();
-                }
-                __syncwarp();
-                if (lane == 0 && got) mbar_arrive(&xf[s]);
-            }
-            if (x > x0) epilogue(x - 1, s_prev, b_prev, bph_prev);
-            if (h != prev_h) {
+            const int j = (int)(x % nt);
+            if (h != cur_h) {
+                // the previous head's UMMAs are complete (its last epilogue waited on them)
                 const float *srch = dpart + h * (long long)maxslots * kStateElems;
                 const int ns = P.last_cta((int)h) - P.first_cta((int)h) + 1;
                 float m = gather_state(srch, ns, stage, tid);
@@ -1093,16 +1088,56 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 named_bar(1, kWorkers);
                 cur_isd = 1.f / sd;
                 if (tid == 0) mbar_arrive(opready);
-                prev_h = h;
+                cur_h = h;
             }
-            s_prev = s;
-            b_prev = b;
-            bph_prev = bph;
-            if (++s == NST) { s = 0; ph ^= 1; }
+            // ---- epilogue of tile x
+            if (tid == 0) tma_store_wait_read<0>();
+            named_bar(1, kWorkers);
+            bool got = live && LA_WAIT(&accfull[b], bph, 0x10u);
+            got = __all_sync(0xffffffffu, got);
+            live = live && got;
+            if (got) {
+                tc_fence_after();
+                const uint32_t da = tmem + (uint32_t)b * 128u + ((uint32_t)(32 * sub) << 16), db = da + 64u;
+#pragma unroll
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    float aa[16], bb[16], out[16];
+                    tmem_ld16(da + 16 * c16, aa);
+                    tmem_ld16(db + 16 * c16, bb);
+                    if (BIDIR) {
+                        float kf[16];
+                        load_chunk16<BF16>(sK + s * kTileBytes, row, c16, kf);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) out[i] = fmaf(aa[i], cur_isd, dz[16 * c16 + i]) * fminf(kf[i], 1.f);
+                    } else {
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) out[i] = aa[i] * cur_isd;
+                    }
+                    store_chunk16<BF16>(sDK, row, c16, out);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) out[i] = bb[i] * cur_isd;
+                    store_chunk16<BF16>(sDV, row, c16, out);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&accempty[b]);
+                    if (BIDIR) mbar_arrive(&empty[s]);   // f(k) read: the stage may be reloaded
+                }
+            }
+            fence_async_smem();
+            named_bar(1, kWorkers);
+            if (tid == 0 && live) {
+                tma_store_3d(&tmDK, sDK, 0, j * kRows, (int)h);
+                tma_store_3d(&tmDV, sDV, 0, j * kRows, (int)h);
+                tma_store_commit();
+            }
+            if (++s == NST) s = 0;
             b ^= 1;
             if (b == 0) bph ^= 1;
         }
-        epilogue(x1 - 1, s_prev, b_prev, bph_prev);
         if (tid == 0) tma_store_wait_all<0>();
     }
     tc_fence_before();
@@ -1153,9 +1188,6 @@ static la_status tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, boo
     return LA_OK;
 }
 
-// state_reduce: 4 stages of (k, v) + the ones block, or 3 stages of (k, v, k_lo) for bf16 bidir
-constexpr size_t reduce_smem(bool klo) { return 1024 + (klo ? 9 : 8) * (size_t)kTileBytes + kTileBytes + 256; }
-constexpr size_t kOutputSmem = 1024 + 4 * kTileBytes + 2 * kTileBytes + 2 * 80 * 128 + kStateElems * 4 + 32 + 256;
 
 static size_t partial_bytes(const Shape &s) {
     size_t b = (size_t)s.BH() * (size_t)max_slots((int)s.BH()) * kStateElems * sizeof(float);
@@ -1166,7 +1198,7 @@ template <bool BIDIR, bool BF16>
 static la_status launch_reduce(const CUtensorMap &mk, const CUtensorMap &mv, float *part, const Shape &s, int nt,
                                cudaStream_t st) {
     return launch(BIDIR ? "tc_state_reduce" : "tc_state_reduce_simple", state_reduce_kernel<BIDIR, BF16>,
-                  dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads), reduce_smem(BIDIR && BF16), st, mk, mv, part, s.T, (int)s.BH(), nt,
+                  dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads), (size_t)ReduceLayout<BIDIR, BF16>::bytes, st, mk, mv, part, s.T, (int)s.BH(), nt,
                   max_slots((int)s.BH()));
 }
 
@@ -1183,7 +1215,7 @@ static la_status fwd_t(const void *q, const void *k, const void *v, void *o, flo
     float *part = (float *)ws;
     LA_TRY((launch_reduce<BIDIR, BF16>(mk, mv, part, s, nt, st)));
     return launch(BIDIR ? "tc_output" : "tc_output_simple", output_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
-                  kOutputSmem, st, mq, mo, (const float *)part, ms * kStateElems, 0, state, s.T, (int)s.BH(), nt,
+                  (size_t)OutputLayout::bytes, st, mq, mo, (const float *)part, ms * kStateElems, 0, state, s.T, (int)s.BH(), nt,
                   eps);
 }
 
