@@ -71,6 +71,22 @@ template <> struct h2<true> {
 
 __device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 
+// elu+1 on two packed fp16 values without leaving fp16:
+//   phi(x) = max(x, 0) + 2^(min(x, 0) * log2(e))
+// (x > 0 gives x + 2^0 = x + 1, x <= 0 gives e^x).  ex2.approx.f16x2 handles
+// both halves in one special-function operation.
+__device__ __forceinline__ uint32_t phi_h2(uint32_t x) {
+    const __half2 hx = *reinterpret_cast<__half2 *>(&x);
+    const __half2 zero = __float2half2_rn(0.f);
+    const __half2 l2e = __float2half2_rn(1.4426950408889634f);
+    __half2 a = __hmul2(__hmin2(hx, zero), l2e);
+    uint32_t ai = *reinterpret_cast<uint32_t *>(&a), ei;
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(ei) : "r"(ai));
+    const __half2 e = *reinterpret_cast<__half2 *>(&ei);
+    __half2 r = __hadd2(__hmax2(hx, zero), e);
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
 // Feature map elu+1 applied in place to row `row` of a 128-byte-swizzled tile
 // (the row's 8 chunks are visited in an order that spreads banks); rows that
 // lie past the sequence end are zeroed when `zero` is set.
@@ -132,6 +148,8 @@ __device__ __forceinline__ void phi_half_row(uint8_t *tile, int xi, bool zero) {
         uint4 u = *c;
         if (zero) {
             u = make_uint4(0u, 0u, 0u, 0u);
+        } else if (!BF16) {
+            u = make_uint4(phi_h2(u.x), phi_h2(u.y), phi_h2(u.z), phi_h2(u.w));
         } else {
             uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
