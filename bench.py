@@ -262,6 +262,32 @@ def config_of(w, args):
                   % (step_bytes / 1e6)}
 
 
+def time_step_at(la, w, dev, stream, steps, warmup):
+    """Device time (ms) of one fwd+bwd step of workload w, averaged over `steps`."""
+    host = synth.make_inputs(w, seed=0)
+    q, k, v, g = (host[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    state = torch.empty((w.B, w.H, w.D, w.D + 1), dtype=torch.float32, device=dev)
+    nws = max(la.la_workspace_size("bidir_fwd", w.B, w.H, w.T, w.D, q.dtype),
+              la.la_workspace_size("bidir_bwd", w.B, w.H, w.T, w.D, q.dtype))
+    ws = torch.empty(max(256, nws), dtype=torch.uint8, device=dev)
+
+    def step():
+        la.la_bidir_fwd(q, k, v, o, state, eps=w.eps, workspace=ws)
+        la.la_bidir_bwd(q, k, v, g, dq, dk, dv, state, eps=w.eps, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1) / steps
+
+
 def run_ours(args, w):
     import linear_attention_attn_b200 as la
     rank, world, local = dist_env()
@@ -369,6 +395,20 @@ def run_ours(args, w):
     step_roof = {"bytes_per_step": step_bytes, "achieved_gbs": step_bytes / (seconds / args.steps) / 1e9,
                  "frac": step_bytes / (seconds / args.steps) / 1e9 / peak, "peak": peak, "peak_source": peak_kind}
 
+    # ---- the same step at the longer sequence lengths of the metric (device events only)
+    sweep = []
+    if world == 1 and args.sweep:
+        del o, dq, dk, dv, q, k, v, g, ws
+        torch.cuda.empty_cache()
+        for Ts in (8192, 16384):
+            if Ts == T:
+                continue
+            ms_s = time_step_at(la, w.with_T(Ts), dev, stream, steps=max(3, min(args.steps, 50)), warmup=3)
+            b_s = 11 * w.B * w.H * Ts * w.D * 2
+            sweep.append({"T": Ts, "value": w.B * Ts / (ms_s / 1e3), "ms_per_step": ms_s,
+                          "achieved_gbs": b_s / (ms_s / 1e3) / 1e9,
+                          "frac": b_s / (ms_s / 1e3) / 1e9 / measured_peaks()[0]})
+
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
@@ -390,7 +430,7 @@ def run_ours(args, w):
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": vs, "dtype": "f16", "data": "synthetic", "config": config_of(w, args),
         "roofline": roof, "step_roofline": step_roof, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": launches, "clocks": clocks,
+        "gpu_launches": launches, "clocks": clocks, "t_sweep": sweep,
         "kernels": [{"name": n, "launches": c, "total_ms": t} for n, c, t in per_kernel],
     }
     print(json.dumps(line), flush=True)
@@ -407,6 +447,8 @@ def main(argv=None):
     ap.add_argument("--T", type=int, default=4096)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", dest="sweep", action="store_false",
+                    help="skip the extra T=8192/16384 device timings added to the JSON line")
     ap.add_argument("--profile-only", action="store_true",
                     help="run the warm-up and timed steps only (no e2e, CPU baseline or clock sampling): "
                          "the command profiled under ncu")
