@@ -11,8 +11,15 @@ bool supports(la_op op, const Shape &s, la_dtype dt) {
     case LA_OP_BIDIR_BWD:
     case LA_OP_SIMPLE_FWD:
     case LA_OP_SIMPLE_BWD: return s.D == 64;
+    case LA_OP_CHUNK_DECAY_FWD: return dt == LA_BF16 && s.D == 128;
     default: return false;
     }
+}
+
+unsigned int read_and_clear_fault() {
+    const unsigned int a = read_and_clear_state_fault(), b = read_and_clear_retention_fault();
+    if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu) return 0xFFFFFFFFu;
+    return a | b;
 }
 
 size_t workspace_size(la_op op, const Shape &s, la_dtype) {
@@ -25,9 +32,9 @@ size_t workspace_size(la_op op, const Shape &s, la_dtype) {
     }
 }
 
-la_status decay_fwd(const void *, const void *, const void *, void *, const DecayArgs &, const Shape &, la_dtype,
-                    void *, cudaStream_t) {
-    return LA_ERR_UNSUPPORTED;
+la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, const Shape &s,
+                    la_dtype, void *, cudaStream_t st) {
+    return retention_fwd(q, k, v, o, dec, s, st);
 }
 la_status decay_bwd(const void *, const void *, const void *, const void *, const DecayArgs &, void *, void *, void *,
                     const Shape &, la_dtype, void *, cudaStream_t) {

@@ -1,6 +1,8 @@
 // la_tc.cuh -- the tensor-core (tcgen05 / TMA) path for fp16 and bf16 (not part of the ABI).
 #pragma once
 
+#include <cuda.h>
+
 #include "la_internal.cuh"
 
 namespace la {
@@ -12,6 +14,15 @@ size_t workspace_size(la_op op, const Shape &s, la_dtype dt);
 size_t state_workspace_size(la_op op, const Shape &s);
 // Fault word of the tensor-core kernels (nonzero when a wait ran out); cleared on read.
 unsigned int read_and_clear_fault();
+unsigned int read_and_clear_state_fault();
+unsigned int read_and_clear_retention_fault();
+
+// [BH, T, D] 16-bit tensor map: boxes of box_rows x 64 columns, 128-byte swizzle.
+la_status make_tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16, int box_rows);
+la_status retention_map(CUtensorMap *m, const void *ptr, const Shape &s);
+// Chunked causal decay forward on tensor cores (bf16, D = 128).
+la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, const Shape &s,
+                        cudaStream_t st);
 la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, void *o, float *state,
                     const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
 la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, const void *g,

@@ -56,7 +56,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // After a short spin the thread backs off with __nanosleep (32 ns doubling to
 // 512 ns), so warps that wait long do not take issue slots from the warps
 // that share their scheduler.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                             unsigned int *fault_word, unsigned int code) {
 #pragma unroll 1
     for (int i = 0; i < 8; ++i)

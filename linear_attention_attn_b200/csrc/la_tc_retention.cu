@@ -1,0 +1,402 @@
+// la_tc_retention.cu -- tensor-core kernel of causal linear attention with a per-head
+// scalar decay (retention), forward, bf16 storage, D = 128, fp32 accumulation.
+//
+// "flash-linear-attention" README, "Benchmarks" (RetNet) and "Different forms of
+// linear attention" (FusedChunk: chunkwise, the inter-chunk state kept on chip,
+// one program per (b, h)).  With chunk c covering rows cC .. cC+C-1 (C = 64),
+// local indices i, j in [0, C), M_ij = gamma^(i-j) [i >= j], and the state
+// entering chunk c, S_c = sum_{s < cC} gamma^(cC-1-s) k_s^T v_s (S_0 = 0):
+//   O_c     = ((Q_c K_c^T) o M) V_c + diag(gamma^(i+1)) Q_c S_c
+//   S_{c+1} = gamma^C S_c + K_c^T diag(gamma^(C-1-j)) V_c
+// which is o_t = sum_{s<=t} gamma^(t-s) (q_t . k_s) v_s regrouped by chunk.
+//
+// One CTA per (b, h) walks the chunks in order.  Warp 0 streams q/k/v chunks
+// with TMA (two 64-column boxes per 64-row chunk, 128-byte swizzle); warp 1
+// issues the UMMAs; warps 2..9 form gamma^(C-1-j) k (hi + lo bf16); warps 10..13
+// apply the decay mask to P = Q K^T (hi + lo bf16), combine the two output
+// accumulators and carry the fp32 state S <- gamma^C S + dS, kept in shared
+// memory as a bf16 hi + lo pair that is also the B operand of Q S.
+//   P       M=64  N=64  K=128  A = Q (K-major)        B = K (K-major)
+//   O_intra M=64  N=128 K=64   A = P~ hi, lo (K-major) B = V (MN-major)
+//   O_inter M=64  N=128 K=128  A = Q (K-major)        B = S hi, lo (MN-major)
+//   dS      M=128 N=128 K=64   A = K^ hi, lo (MN-major) B = V (MN-major)
+#include "la_tc.cuh"
+#include "la_tc_common.cuh"
+
+#include <mutex>
+
+namespace la {
+namespace tc {
+
+__device__ unsigned int g_ret_fault = 0;
+
+namespace {
+
+#define LA_RWAIT(bar, par, code) mbar_wait((bar), (par), s_abort, &g_ret_fault, (code))
+
+constexpr int kC = 64;                    // chunk rows
+constexpr int kBox = kC * 128;            // one [64 rows x 64 cols] bf16 box, 8 KB
+constexpr int kTile128 = 2 * kBox;        // a [64 x 128] chunk tile: two boxes
+
+__device__ __forceinline__ uint8_t *align1024r(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// 16 columns (16*c16 .. +15, c16 in 0..7) of row `row` of a 128-column tile stored
+// as boxes of 64 columns, `box_bytes` apart.
+__device__ __forceinline__ void ld16_wide(const uint8_t *t, int box_bytes, int row, int c16, float (&v)[16]) {
+    load_chunk16<true>(t + (c16 >> 2) * box_bytes, row, c16 & 3, v);
+}
+__device__ __forceinline__ void st16_wide(uint8_t *t, int box_bytes, int row, int c16, const float (&v)[16]) {
+    store_chunk16<true>(t + (c16 >> 2) * box_bytes, row, c16 & 3, v);
+}
+
+struct RetLayout {
+    static constexpr int NST = 2;
+    static constexpr int qoff = 0;                              // [NST] q chunk (2 boxes)
+    static constexpr int koff = qoff + NST * kTile128;
+    static constexpr int voff = koff + NST * kTile128;
+    static constexpr int khoff = voff + NST * kTile128;         // k^ hi, lo
+    static constexpr int ptoff = khoff + 2 * kTile128;          // P~ hi, lo: [64 x 64] each
+    static constexpr int soff = ptoff + 2 * kBox;               // S hi, lo: [128 x 128] each (2 x 16 KB)
+    static constexpr int ooff = soff + 2 * 2 * 16384;           // output staging chunk
+    static constexpr int gpoff = ooff + kTile128;               // gamma^k, k = 0..128
+    static constexpr int baroff = gpoff + 132 * 4;
+    static constexpr int nbars = 2 * NST + 9;
+    static constexpr int misc = baroff + nbars * 8;
+    static constexpr int bytes = misc + 32 + 1024;
+};
+
+// Grid: one CTA per (b, h).  decay[h] = gamma_h.
+__global__ void __launch_bounds__(kThreads, 1)
+retention_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, DecayArgs dec,
+                     int T, int H) {
+    using L = RetLayout;
+    constexpr int NST = L::NST;
+    constexpr uint32_t ID_P = idesc_f16(64, 64, true, false, false);
+    constexpr uint32_t ID_OI = idesc_f16(64, 128, true, false, true);
+    constexpr uint32_t ID_DS = idesc_f16(128, 128, true, true, true);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024r(smem_raw);
+    uint8_t *sQ = smem + L::qoff;
+    uint8_t *sK = smem + L::koff;
+    uint8_t *sV = smem + L::voff;
+    uint8_t *sKh = smem + L::khoff;      // hi at +0, lo at +kTile128
+    uint8_t *sPt = smem + L::ptoff;      // hi at +0, lo at +kBox
+    uint8_t *sS = smem + L::soff;        // hi at +0 (2 atoms of 16 KB), lo at +32 KB
+    uint8_t *sO = smem + L::ooff;
+    float *gpow = reinterpret_cast<float *>(smem + L::gpoff);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::baroff);
+    uint64_t *empty = full + NST;
+    uint64_t *pfull = empty + NST;
+    uint64_t *ptready = pfull + 1;
+    uint64_t *khready = ptready + 1;
+    uint64_t *ofull = khready + 1;
+    uint64_t *oread = ofull + 1;
+    uint64_t *dsfull = oread + 1;
+    uint64_t *sready = dsfull + 1;
+    uint64_t *drain = sready + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc);
+    int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x;
+    const float gamma = dec.gamma[bh % H];
+    const int nchunks = (T + kC - 1) / kC;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(pfull, 1);
+        mbar_init(ptready, kEWarps);
+        mbar_init(khready, kXWarps);
+        mbar_init(ofull, 1);
+        mbar_init(oread, kEWarps);
+        mbar_init(dsfull, 1);
+        mbar_init(sready, kEWarps);
+        mbar_init(drain, 1);
+        *s_abort = 0;
+        fence_mbar_init();
+    }
+    if (threadIdx.x < 129) {
+        // gamma^k in fp32 as exp2(k log2 gamma): k = 0..C for the masks and row scales
+        const float l2g = log2f(gamma);
+        gpow[threadIdx.x] = threadIdx.x == 0 ? 1.f : exp2f((float)threadIdx.x * l2g);
+    }
+    if (warp >= kEw0) {
+        // S_0 = 0: both halves of the state operand
+        const int r = threadIdx.x - kEw0 * 32;
+        for (int part = 0; part < 4; ++part) {
+            uint8_t *p = sS + part * 16384 + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(p + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch(&tmQ);
+        tma_prefetch(&tmK);
+        tma_prefetch(&tmV);
+        tma_prefetch(&tmO);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    constexpr uint32_t cP = 0, cOI = 64, cOX = 192, cDS = 320;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int issued = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                if (!LA_RWAIT(&empty[s], ph ^ 1, 0x1u)) break;
+                mbar_arrive_expect_tx(&full[s], 3 * kTile128);
+                for (int b = 0; b < 2; ++b) {
+                    tma_load_3d(sQ + s * kTile128 + b * kBox, &tmQ, &full[s], 64 * b, c * kC, bh);
+                    tma_load_3d(sK + s * kTile128 + b * kBox, &tmK, &full[s], 64 * b, c * kC, bh);
+                    tma_load_3d(sV + s * kTile128 + b * kBox, &tmV, &full[s], 64 * b, c * kC, bh);
+                }
+                ++issued;
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+            if (*s_abort) {
+                for (int i = issued - 1; i >= 0 && i >= issued - NST; --i)
+                    mbar_wait_slow(smem_u32(&full[i % NST]), (uint32_t)((i / NST) & 1), nullptr, &g_ret_fault, 0x200u);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const uint32_t pc = (uint32_t)(c & 1), pp = (uint32_t)((c - 1) & 1);
+                if (!LA_RWAIT(&full[s], ph, 0x4u)) break;
+                if (c > 0 && !LA_RWAIT(ptready, pp, 0x8u)) break;   // P accumulator read
+                tc_fence_after();
+                const uint32_t aQ = smem_u32(sQ + s * kTile128), aK = smem_u32(sK + s * kTile128);
+                const uint32_t aV = smem_u32(sV + s * kTile128);
+                // P = Q K^T
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+                    umma_f16_ss(tmem + cP, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024), ID_P,
+                                kk ? 1u : 0u);
+                }
+                umma_commit(pfull);
+                // O_intra = P~ V and O_inter = Q S
+                if (!LA_RWAIT(ptready, pc, 0x10u)) break;
+                if (c > 0 && !LA_RWAIT(sready, pp, 0x20u)) break;
+                if (c > 0 && !LA_RWAIT(oread, pp, 0x40u)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t bv = sdesc_sw128(aV + kk * 2048, kBox, 1024);
+#pragma unroll
+                    for (int op = 0; op < 2; ++op)
+                        umma_f16_ss(tmem + cOI, sdesc_sw128(smem_u32(sPt + op * kBox) + kk * 32, 16, 1024), bv, ID_OI,
+                                    (kk | op) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+#pragma unroll
+                    for (int op = 0; op < 2; ++op)
+                        umma_f16_ss(tmem + cOX, sdesc_sw128(aQ + off, 16, 1024),
+                                    sdesc_sw128(smem_u32(sS + op * 32768) + kk * 2048, 16384, 1024), ID_OI,
+                                    (kk | op) ? 1u : 0u);
+                }
+                umma_commit(ofull);
+                // dS = K^^T V
+                if (!LA_RWAIT(khready, pc, 0x80u)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t bv = sdesc_sw128(aV + kk * 2048, kBox, 1024);
+#pragma unroll
+                    for (int op = 0; op < 2; ++op)
+                        umma_f16_ss(tmem + cDS, sdesc_sw128(smem_u32(sKh + op * kTile128) + kk * 2048, kBox, 1024), bv,
+                                    ID_DS, (kk | op) ? 1u : 0u);
+                }
+                umma_commit(dsfull);
+                umma_commit(&empty[s]);
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+            umma_commit(drain);
+            mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_ret_fault, 0x400u);
+        }
+    } else if (warp < kEw0) {
+        // K^ = diag(gamma^(C-1-j)) K as hi + lo; thread xi: row xi % 64, 8-element chunks 4*(xi/64) .. +3
+        const int xi = threadIdx.x - kXw0 * 32;
+        const int row = xi & 63, part = xi >> 6;
+        int s = 0;
+        uint32_t ph = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            bool got = LA_RWAIT(&full[s], ph, 0x100u);
+            if (got && c > 0) got = LA_RWAIT(dsfull, (uint32_t)((c - 1) & 1), 0x200u);   // K^ buffer free
+            got = __all_sync(0xffffffffu, got);
+            if (!got) break;
+            const float f = gpow[kC - 1 - row];
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+                const int ch = part * 4 + it;               // 0..15 across the two boxes
+                const int off = (ch >> 3) * kBox + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+                const uint4 u = *reinterpret_cast<const uint4 *>(sK + s * kTile128 + off);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float2 x = h2<true>::to_f2(w[k]);
+                    const float a = x.x * f, b = x.y * f;
+                    hi[k] = h2<true>::from_f2(a, b);
+                    const float2 hv = h2<true>::to_f2(hi[k]);
+                    lo[k] = h2<true>::from_f2(a - hv.x, b - hv.y);
+                }
+                *reinterpret_cast<uint4 *>(sKh + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(sKh + kTile128 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(khready);
+            if (++s == NST) { s = 0; ph ^= 1; }
+        }
+    } else {
+        // Epilogue warps: decay mask, output, state.  Named barrier 1 (128 threads) is
+        // reached by all of them whatever the waits return.
+        const int tid = threadIdx.x - kEw0 * 32;
+        const int sub = warp & 3;
+        const uint32_t lanes = (uint32_t)(32 * sub) << 16;
+        const int ri = 16 * sub + lane;           // M = 64 accumulators: chunk row of lanes 0..15
+        bool live = true;
+        for (int c = 0; c < nchunks; ++c) {
+            const uint32_t pc = (uint32_t)(c & 1);
+            // ---- P~ = (Q K^T) o M, hi + lo
+            bool got = live && LA_RWAIT(pfull, pc, 0x400u);
+            got = __all_sync(0xffffffffu, got);
+            live = live && got;
+            if (got) {
+                tc_fence_after();
+                float p[64];
+                tmem_row64(tmem + cP + lanes, p);
+                tc_fence_before();
+                if (lane < 16) {
+                    float hi[64], lo[64];
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) p[j] = j <= ri ? p[j] * gpow[ri - j] : 0.f;
+                    store_row<true>(sPt, ri, p);
+                    load_row<true>(sPt, ri, hi);
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) lo[j] = p[j] - hi[j];
+                    store_row<true>(sPt + kBox, ri, lo);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(ptready);
+            }
+            // ---- o = O_intra + diag(gamma^(i+1)) O_inter
+            got = live && LA_RWAIT(ofull, pc, 0x800u);
+            got = __all_sync(0xffffffffu, got);
+            live = live && got;
+            if (tid == 0) tma_store_wait_read<0>();
+            named_bar(1, kWorkers);
+            if (got) {
+                tc_fence_after();
+                const float g1 = gpow[ri + 1];
+#pragma unroll
+                for (int c16 = 0; c16 < 8; ++c16) {
+                    float a[16], b[16];
+                    tmem_ld16(tmem + cOI + lanes + 16 * c16, a);
+                    tmem_ld16(tmem + cOX + lanes + 16 * c16, b);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) a[i] = fmaf(g1, b[i], a[i]);
+                    if (lane < 16) st16_wide(sO, kBox, ri, c16, a);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(oread);
+            }
+            fence_async_smem();
+            named_bar(1, kWorkers);
+            if (tid == 0 && live) {
+                tma_store_3d(&tmO, sO, 0, c * kC, bh);
+                tma_store_3d(&tmO, sO + kBox, 64, c * kC, bh);
+                tma_store_commit();
+            }
+            // ---- S <- gamma^C S + dS (row d = this thread's TMEM lane), as hi + lo
+            got = live && LA_RWAIT(dsfull, pc, 0x1000u);
+            got = __all_sync(0xffffffffu, got);
+            live = live && got;
+            if (got) {
+                tc_fence_after();
+                const int d = 32 * sub + lane;             // the TMEM lane (state row) this thread reads
+                const float gC = gpow[kC];
+#pragma unroll 2
+                for (int c16 = 0; c16 < 8; ++c16) {
+                    float ds[16], hi[16], lo[16];
+                    tmem_ld16(tmem + cDS + lanes + 16 * c16, ds);
+                    ld16_wide(sS, 16384, d, c16, hi);
+                    ld16_wide(sS + 32768, 16384, d, c16, lo);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) ds[i] = fmaf(gC, hi[i] + lo[i], ds[i]);
+                    st16_wide(sS, 16384, d, c16, ds);
+                    ld16_wide(sS, 16384, d, c16, hi);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) lo[i] = ds[i] - hi[i];
+                    st16_wide(sS + 32768, 16384, d, c16, lo);
+                }
+                tc_fence_before();
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sready);
+            }
+        }
+        if (tid == 0) tma_store_wait_all<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+#ifndef LA_TRY
+#define LA_TRY(x)                     \
+    do {                              \
+        la_status _rc = (x);          \
+        if (_rc != LA_OK) return _rc; \
+    } while (0)
+#endif
+
+}  // namespace
+
+la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, const Shape &s,
+                        cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mo;
+    LA_TRY(retention_map(&mq, q, s));
+    LA_TRY(retention_map(&mk, k, s));
+    LA_TRY(retention_map(&mv, v, s));
+    LA_TRY(retention_map(&mo, o, s));
+    return launch("tc_retention_fwd", retention_fwd_kernel, dim3((unsigned)s.BH()), dim3(kThreads),
+                  (size_t)RetLayout::bytes, st, mq, mk, mv, mo, dec, s.T, s.H);
+}
+
+unsigned int read_and_clear_retention_fault() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_ret_fault, sizeof v) != cudaSuccess) return 0xFFFFFFFFu;
+    if (v) cudaMemcpyToSymbol(g_ret_fault, &zero, sizeof zero);
+    return v;
+}
+
+}  // namespace tc
+}  // namespace la

@@ -1167,8 +1167,10 @@ static EncodeFn encode_fn() {
     return fn;
 }
 
-// [BH, T, 64] 16-bit tensor, boxes of 128 rows x 64 columns, 128-byte swizzle, zero fill.
-static la_status tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16) {
+}  // namespace
+
+// [BH, T, D] 16-bit tensor, boxes of `box_rows` rows x 64 columns, 128-byte swizzle, zero fill.
+la_status make_tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16, int box_rows) {
     EncodeFn enc = encode_fn();
     if (!enc) {
         set_error("cuTensorMapEncodeTiled is unavailable from the driver");
@@ -1176,7 +1178,7 @@ static la_status tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, boo
     }
     const cuuint64_t dims[3] = {(cuuint64_t)s.D, (cuuint64_t)s.T, (cuuint64_t)s.BH()};
     const cuuint64_t strides[2] = {(cuuint64_t)s.D * 2, (cuuint64_t)s.T * s.D * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)kRows, 1};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     const cuuint32_t es[3] = {1, 1, 1};
     CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                      const_cast<void *>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1188,6 +1190,15 @@ static la_status tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, boo
     return LA_OK;
 }
 
+la_status retention_map(CUtensorMap *m, const void *ptr, const Shape &s) {
+    return make_tensor_map(m, ptr, s, true, 64);
+}
+
+namespace {
+
+static la_status tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16) {
+    return make_tensor_map(m, ptr, s, bf16, kRows);
+}
 
 static size_t partial_bytes(const Shape &s) {
     size_t b = (size_t)s.BH() * (size_t)max_slots((int)s.BH()) * kStateElems * sizeof(float);
@@ -1279,7 +1290,7 @@ la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, con
               : bwd_t<false, false>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st);
 }
 
-unsigned int read_and_clear_fault() {
+unsigned int read_and_clear_state_fault() {
     unsigned int v = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&v, g_tc_fault, sizeof v) != cudaSuccess) return 0xFFFFFFFFu;
     if (v) cudaMemcpyToSymbol(g_tc_fault, &zero, sizeof zero);
