@@ -49,6 +49,9 @@ PAGE_TIMINGS_MS = {128: (0.049152, 0.651264), 256: (0.056320, 0.625664), 512: (0
 KERNEL_TENSORS = {
     "simt_state_partial": 2, "simt_output": 2, "simt_bwd_q": 3, "simt_bwd_k": 4,
     "tc_state_reduce": 2, "tc_output": 2, "tc_bwd_q": 3, "tc_bwd_kv": 4,
+    "tc_state_reduce_simple": 2, "tc_output_simple": 2, "tc_bwd_q_simple": 3, "tc_bwd_kv_simple": 4,
+    "simt_ret_fwd": 4, "simt_ret_bwd_dq": 4, "simt_ret_bwd_dkdv": 6,
+    "tc_retention_fwd": 4, "tc_retention_bwd_dq": 4, "tc_retention_bwd_dkdv": 6,
 }
 
 
@@ -251,11 +254,19 @@ def run_reference(args, w):
 
 # ------------------------------------------------------------------- ours --
 
+WORKLOAD_TEXT = {
+    "bidir": "bidirectional linear attention fwd+bwd, fp16 storage / fp32 accumulate, B=%d H=%d T=%d D=%d, "
+             "phi=elu+1, eps=1e-06, Q,K,V ~ 0.5 N(0,1), dO ~ N(0,1)",
+    "simple": "simple_la fwd+bwd, bf16 storage / fp32 accumulate, B=%d H=%d T=%d D=%d, "
+              "q,k ~ N(0,1) D^-1/2, v, dO ~ N(0,1)",
+    "retention": "chunked causal decay (retention) fwd+bwd, bf16 storage / fp32 accumulate, B=%d H=%d T=%d D=%d, "
+                 "gamma_h = 1 - 2^(-5-7h/(H-1)), q ~ N(0,1) D^-1/2, k, v, dO ~ N(0,1)",
+}
+
+
 def config_of(w, args):
     step_bytes = 11 * w.B * w.H * w.T * w.D * 2
-    return {"workload": "bidirectional linear attention fwd+bwd, fp16 storage / fp32 accumulate, "
-                        "B=%d H=%d T=%d D=%d, phi=elu+1, eps=%g, Q,K,V ~ 0.5 N(0,1), dO ~ N(0,1)"
-                        % (w.B, w.H, w.T, w.D, w.eps),
+    return {"workload": WORKLOAD_TEXT[w.op] % (w.B, w.H, w.T, w.D),
             "B": w.B, "H": w.H, "T": w.T, "D": w.D, "global_batch": w.B * max(1, args.gpus), "seq_len": w.T,
             "parallelism": "dp%d (independent batches, no collective)" % max(1, args.gpus),
             "l2": "inputs larger than L2: %.0f MB of algorithmic traffic per step vs 126 MB L2, no flush"
@@ -301,13 +312,22 @@ def run_ours(args, w):
     B, H, T, D = w.B, w.H, w.T, w.D
     o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
     state = torch.empty((B, H, D, D + 1), dtype=torch.float32, device=dev)
-    ws_bytes = max(la.la_workspace_size("bidir_fwd", B, H, T, D, q.dtype),
-                   la.la_workspace_size("bidir_bwd", B, H, T, D, q.dtype))
+    names = {"bidir": ("bidir_fwd", "bidir_bwd"), "simple": ("simple_fwd", "simple_bwd"),
+             "retention": ("chunk_decay_fwd", "chunk_decay_bwd")}[w.op]
+    ws_bytes = max(la.la_workspace_size(n, B, H, T, D, q.dtype) for n in names)
     ws = torch.empty(max(256, ws_bytes), dtype=torch.uint8, device=dev)
+    gamma = host.get("gamma")
 
     def step():
-        la.la_bidir_fwd(q, k, v, o, state, eps=w.eps, workspace=ws)
-        la.la_bidir_bwd(q, k, v, g, dq, dk, dv, state, eps=w.eps, workspace=ws)
+        if w.op == "bidir":
+            la.la_bidir_fwd(q, k, v, o, state, eps=w.eps, workspace=ws)
+            la.la_bidir_bwd(q, k, v, g, dq, dk, dv, state, eps=w.eps, workspace=ws)
+        elif w.op == "simple":
+            la.la_simple_fwd(q, k, v, o, state, workspace=ws)
+            la.la_simple_bwd(q, k, v, g, dq, dk, dv, state, workspace=ws)
+        else:
+            la.la_chunk_decay_fwd(q, k, v, o, gamma, workspace=ws)
+            la.la_chunk_decay_bwd(q, k, v, g, gamma, dq, dk, dv, workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -397,7 +417,7 @@ def run_ours(args, w):
 
     # ---- the same step at the longer sequence lengths of the metric (device events only)
     sweep = []
-    if world == 1 and args.sweep:
+    if world == 1 and args.sweep and w.op == "bidir":
         del o, dq, dk, dv, q, k, v, g, ws
         torch.cuda.empty_cache()
         for Ts in (8192, 16384):
@@ -415,20 +435,21 @@ def run_ours(args, w):
         return 0
 
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and w.op == "bidir":
         cores = host_cores()
         r, dt, sample, used = oracle_step_sample(w, host, 15.0, cores)
         cpu = {"value": r, "unit": UNIT, "cores": used, "kind": "oracle", "sample": sample, "seconds": dt}
 
     vs = None
-    if T in PAGE_TIMINGS_MS and (B, H, D) == (8, 16, 64):
+    if w.op == "bidir" and T in PAGE_TIMINGS_MS and (B, H, D) == (8, 16, 64):
         page_rate = B * T / (sum(PAGE_TIMINGS_MS[T]) / 1e3)
         vs = value / page_rate
 
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC if w.op == "bidir" else "%s fwd+bwd tokens/s" % w.op, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": vs, "dtype": "f16", "data": "synthetic", "config": config_of(w, args),
+        "vs_baseline": vs, "dtype": w.dtype, "data": "synthetic", "config": config_of(w, args),
         "roofline": roof, "step_roofline": step_roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches, "clocks": clocks, "t_sweep": sweep,
         "kernels": [{"name": n, "launches": c, "total_ms": t} for n, c, t in per_kernel],
@@ -444,7 +465,10 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--T", type=int, default=4096)
+    ap.add_argument("--T", type=int, default=None, help="sequence length (default: the workload's)")
+    ap.add_argument("--workload", choices=["bidir", "simple", "retention"], default="bidir",
+                    help="bidir (the benchmark metric, B8 H16 D64 fp16), simple (B8 H16 D64 bf16) or "
+                         "retention (B8 H32 D128 bf16)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", dest="sweep", action="store_false",
@@ -455,7 +479,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    w = synth.WORKLOADS["bidir_f16"].with_T(args.T)
+    base = {"bidir": "bidir_f16", "simple": "simple_bf16", "retention": "retention_bf16"}[args.workload]
+    w = synth.WORKLOADS[base]
+    w = w.with_T(args.T if args.T is not None else (4096 if args.workload != "retention" else 8192))
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -11,7 +11,8 @@ bool supports(la_op op, const Shape &s, la_dtype dt) {
     case LA_OP_BIDIR_BWD:
     case LA_OP_SIMPLE_FWD:
     case LA_OP_SIMPLE_BWD: return s.D == 64;
-    case LA_OP_CHUNK_DECAY_FWD: return dt == LA_BF16 && s.D == 128;
+    case LA_OP_CHUNK_DECAY_FWD:
+    case LA_OP_CHUNK_DECAY_BWD: return dt == LA_BF16 && s.D == 128;
     default: return false;
     }
 }
@@ -36,9 +37,9 @@ la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const 
                     la_dtype, void *, cudaStream_t st) {
     return retention_fwd(q, k, v, o, dec, s, st);
 }
-la_status decay_bwd(const void *, const void *, const void *, const void *, const DecayArgs &, void *, void *, void *,
-                    const Shape &, la_dtype, void *, cudaStream_t) {
-    return LA_ERR_UNSUPPORTED;
+la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec, void *dq,
+                    void *dk, void *dv, const Shape &s, la_dtype, void *, cudaStream_t st) {
+    return retention_bwd(q, k, v, g, dec, dq, dk, dv, s, st);
 }
 
 }  // namespace tc

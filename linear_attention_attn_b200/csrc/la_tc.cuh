@@ -23,6 +23,8 @@ la_status retention_map(CUtensorMap *m, const void *ptr, const Shape &s);
 // Chunked causal decay forward on tensor cores (bf16, D = 128).
 la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, const Shape &s,
                         cudaStream_t st);
+la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec, void *dq,
+                        void *dk, void *dv, const Shape &s, cudaStream_t st);
 la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, void *o, float *state,
                     const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
 la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, const void *g,

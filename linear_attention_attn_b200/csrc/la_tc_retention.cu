@@ -20,10 +20,19 @@
 //   O_intra M=64  N=128 K=64   A = P~ hi, lo (K-major) B = V (MN-major)
 //   O_inter M=64  N=128 K=128  A = Q (K-major)        B = S hi, lo (MN-major)
 //   dS      M=128 N=128 K=64   A = K^ hi, lo (MN-major) B = V (MN-major)
+//
+// The backward reuses the same kernel: with R_s = sum_{t>=s} gamma^(t-s) q_t^T dO_t,
+//   dq_t = sum_{s<=t} gamma^(t-s) (dO_t . v_s) k_s   = retention(dO, V, K)
+//   dv_s = sum_{t>=s} gamma^(t-s) (k_s . q_t) dO_t   = retention run backwards in time on (K, Q, dO)
+//   dk_s = sum_{t>=s} gamma^(t-s) (v_s . dO_t) q_t   = retention run backwards in time on (V, dO, Q)
+// Backwards in time ("rev") the chunks are visited last to first, the mask is
+// gamma^(j-i) [j >= i], the inter-chunk row scale gamma^(C-i), and the state
+// update weights gamma^j k_j; the three passes run as one grid of 3 B H CTAs.
 #include "la_tc.cuh"
 #include "la_tc_common.cuh"
 
 #include <mutex>
+#include <string.h>
 
 namespace la {
 namespace tc {
@@ -67,11 +76,16 @@ struct RetLayout {
     static constexpr int bytes = misc + 32 + 1024;
 };
 
-// Grid: one CTA per (b, h).  decay[h] = gamma_h.
+// Up to three retention passes in one launch: pass p reads (q, k, v) through
+// maps q[p], k[p], v[p], writes o[p], forwards (rev = 0) or backwards in time.
+struct RetJobs {
+    CUtensorMap q[3], k[3], v[3], o[3];
+    int rev[3];
+};
+
+// Grid: one CTA per (pass, b, h), pass = blockIdx.x / BH.  decay[h] = gamma_h.
 __global__ void __launch_bounds__(kThreads, 1)
-retention_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, DecayArgs dec,
-                     int T, int H) {
+retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int H, int BH) {
     using L = RetLayout;
     constexpr int NST = L::NST;
     constexpr uint32_t ID_P = idesc_f16(64, 64, true, false, false);
@@ -101,7 +115,10 @@ retention_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.x;
+    const int pass = blockIdx.x / BH;
+    const int bh = blockIdx.x % BH;
+    const bool rev = jobs.rev[pass] != 0;
+    const CUtensorMap *tmQ = &jobs.q[pass], *tmK = &jobs.k[pass], *tmV = &jobs.v[pass], *tmO = &jobs.o[pass];
     const float gamma = dec.gamma[bh % H];
     const int nchunks = (T + kC - 1) / kC;
 
@@ -137,10 +154,10 @@ retention_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         fence_async_smem();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch(&tmQ);
-        tma_prefetch(&tmK);
-        tma_prefetch(&tmV);
-        tma_prefetch(&tmO);
+        tma_prefetch(tmQ);
+        tma_prefetch(tmK);
+        tma_prefetch(tmV);
+        tma_prefetch(tmO);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -157,13 +174,14 @@ retention_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             int s = 0;
             uint32_t ph = 0;
             int issued = 0;
-            for (int c = 0; c < nchunks; ++c) {
+            for (int it = 0; it < nchunks; ++it) {
+                const int c = rev ? nchunks - 1 - it : it;
                 if (!LA_RWAIT(&empty[s], ph ^ 1, 0x1u)) break;
                 mbar_arrive_expect_tx(&full[s], 3 * kTile128);
                 for (int b = 0; b < 2; ++b) {
-                    tma_load_3d(sQ + s * kTile128 + b * kBox, &tmQ, &full[s], 64 * b, c * kC, bh);
-                    tma_load_3d(sK + s * kTile128 + b * kBox, &tmK, &full[s], 64 * b, c * kC, bh);
-                    tma_load_3d(sV + s * kTile128 + b * kBox, &tmV, &full[s], 64 * b, c * kC, bh);
+                    tma_load_3d(sQ + s * kTile128 + b * kBox, tmQ, &full[s], 64 * b, c * kC, bh);
+                    tma_load_3d(sK + s * kTile128 + b * kBox, tmK, &full[s], 64 * b, c * kC, bh);
+                    tma_load_3d(sV + s * kTile128 + b * kBox, tmV, &full[s], 64 * b, c * kC, bh);
                 }
                 ++issued;
                 if (++s == NST) { s = 0; ph ^= 1; }
@@ -244,7 +262,7 @@ retention_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             if (got && c > 0) got = LA_RWAIT(dsfull, (uint32_t)((c - 1) & 1), 0x200u);   // K^ buffer free
             got = __all_sync(0xffffffffu, got);
             if (!got) break;
-            const float f = gpow[kC - 1 - row];
+            const float f = rev ? gpow[row] : gpow[kC - 1 - row];
 #pragma unroll
             for (int it = 0; it < 4; ++it) {
                 const int ch = part * 4 + it;               // 0..15 across the two boxes
@@ -276,8 +294,9 @@ retention_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         const uint32_t lanes = (uint32_t)(32 * sub) << 16;
         const int ri = 16 * sub + lane;           // M = 64 accumulators: chunk row of lanes 0..15
         bool live = true;
-        for (int c = 0; c < nchunks; ++c) {
-            const uint32_t pc = (uint32_t)(c & 1);
+        for (int it = 0; it < nchunks; ++it) {
+            const int c = rev ? nchunks - 1 - it : it;
+            const uint32_t pc = (uint32_t)(it & 1);
             // ---- P~ = (Q K^T) o M, hi + lo
             bool got = live && LA_RWAIT(pfull, pc, 0x400u);
             got = __all_sync(0xffffffffu, got);
@@ -290,7 +309,10 @@ retention_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 if (lane < 16) {
                     float hi[64], lo[64];
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) p[j] = j <= ri ? p[j] * gpow[ri - j] : 0.f;
+                    for (int j = 0; j < 64; ++j) {
+                        const int dlt = rev ? j - ri : ri - j;     // causal: i >= j; backwards: j >= i
+                        p[j] = dlt >= 0 ? p[j] * gpow[dlt] : 0.f;
+                    }
                     store_row<true>(sPt, ri, p);
                     load_row<true>(sPt, ri, hi);
 #pragma unroll
@@ -309,7 +331,7 @@ retention_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             named_bar(1, kWorkers);
             if (got) {
                 tc_fence_after();
-                const float g1 = gpow[ri + 1];
+                const float g1 = rev ? gpow[kC - ri] : gpow[ri + 1];
 #pragma unroll
                 for (int c16 = 0; c16 < 8; ++c16) {
                     float a[16], b[16];
@@ -327,8 +349,8 @@ retention_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             fence_async_smem();
             named_bar(1, kWorkers);
             if (tid == 0 && live) {
-                tma_store_3d(&tmO, sO, 0, c * kC, bh);
-                tma_store_3d(&tmO, sO + kBox, 64, c * kC, bh);
+                tma_store_3d(tmO, sO, 0, c * kC, bh);
+                tma_store_3d(tmO, sO + kBox, 64, c * kC, bh);
                 tma_store_commit();
             }
             // ---- S <- gamma^C S + dS (row d = this thread's TMEM lane), as hi + lo
@@ -382,13 +404,32 @@ retention_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 
 la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, const Shape &s,
                         cudaStream_t st) {
-    CUtensorMap mq, mk, mv, mo;
-    LA_TRY(retention_map(&mq, q, s));
-    LA_TRY(retention_map(&mk, k, s));
-    LA_TRY(retention_map(&mv, v, s));
-    LA_TRY(retention_map(&mo, o, s));
-    return launch("tc_retention_fwd", retention_fwd_kernel, dim3((unsigned)s.BH()), dim3(kThreads),
-                  (size_t)RetLayout::bytes, st, mq, mk, mv, mo, dec, s.T, s.H);
+    RetJobs jobs;
+    memset(&jobs, 0, sizeof jobs);
+    LA_TRY(retention_map(&jobs.q[0], q, s));
+    LA_TRY(retention_map(&jobs.k[0], k, s));
+    LA_TRY(retention_map(&jobs.v[0], v, s));
+    LA_TRY(retention_map(&jobs.o[0], o, s));
+    return launch("tc_retention_fwd", retention_kernel, dim3((unsigned)s.BH()), dim3(kThreads),
+                  (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
+}
+
+la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec, void *dq,
+                        void *dk, void *dv, const Shape &s, cudaStream_t st) {
+    RetJobs jobs;
+    memset(&jobs, 0, sizeof jobs);
+    // dq = retention(dO, V, K); dv = reverse retention(K, Q, dO); dk = reverse retention(V, dO, Q)
+    const void *in[3][3] = {{g, v, k}, {k, q, g}, {v, g, q}};
+    void *out[3] = {dq, dv, dk};
+    for (int p = 0; p < 3; ++p) {
+        LA_TRY(retention_map(&jobs.q[p], in[p][0], s));
+        LA_TRY(retention_map(&jobs.k[p], in[p][1], s));
+        LA_TRY(retention_map(&jobs.v[p], in[p][2], s));
+        LA_TRY(retention_map(&jobs.o[p], out[p], s));
+        jobs.rev[p] = p > 0;
+    }
+    return launch("tc_retention_bwd", retention_kernel, dim3((unsigned)(3 * s.BH())), dim3(kThreads),
+                  (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
 }
 
 unsigned int read_and_clear_retention_fault() {
