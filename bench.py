@@ -345,8 +345,6 @@ def run_ours(args, w):
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(gpu_selector(dev))
     sampler.start()
-    la.la_prof_enable(True)
-    la.la_prof_collect()              # drop anything recorded before
     launches0 = la.la_launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -355,8 +353,6 @@ def run_ours(args, w):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     launches = la.la_launch_count() - launches0
-    la.la_prof_enable(False)
-    per_kernel = la.la_prof_collect()
     if dist is not None:
         dist.barrier()
     clocks = sampler.stop()
@@ -365,6 +361,18 @@ def run_ours(args, w):
     seconds = ms / 1e3
     tokens_per_rank = B * T * args.steps
     value = aggregate_throughput(tokens_per_rank, world, seconds)
+
+    # ---- per-kernel device times: the same steps again with two events around every
+    #      launch (events between kernels keep them from overlapping, so this pass is
+    #      separate from the timed one)
+    k_prof = max(3, min(args.steps, 50))
+    la.la_prof_enable(True)
+    la.la_prof_collect()              # drop anything recorded before
+    for _ in range(k_prof):
+        step()
+    torch.cuda.synchronize(dev)
+    la.la_prof_enable(False)
+    per_kernel = la.la_prof_collect()
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
     e2e = None
@@ -453,6 +461,7 @@ def run_ours(args, w):
         "roofline": roof, "step_roofline": step_roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches, "clocks": clocks, "t_sweep": sweep,
         "kernels": [{"name": n, "launches": c, "total_ms": t} for n, c, t in per_kernel],
+        "kernel_timing": "per-kernel CUDA events on the launch stream over %d further steps after the timed region" % k_prof,
     }
     print(json.dumps(line), flush=True)
     if dist is not None:

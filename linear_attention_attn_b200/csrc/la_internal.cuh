@@ -39,6 +39,38 @@ la_status launch(const char *name, Kernel kernel, dim3 grid, dim3 block, size_t 
     return LA_OK;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous kernel in the stream is finishing.  Only for kernels that execute
+// griddepcontrol.wait before touching global memory (the tensor-core kernels).
+// (With per-kernel profiling on, the events between kernels keep plain order.)
+
+template <typename Kernel, typename... Args>
+la_status launch_pdl(const char *name, Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                     Args... args) {
+    if (grid.x == 0 || grid.y == 0 || grid.z == 0) return LA_OK;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, name);
+    }
+    prof_before(name, stream);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    prof_after(stream);
+    count_launch();
+    if (e != cudaSuccess) return cuda_fail(e, name);
+    return LA_OK;
+}
+
 // ---------------------------------------------------------- element I/O --
 template <typename T> struct io;
 template <> struct io<float> {

@@ -167,6 +167,10 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Everything above touched only shared memory and TMEM: with a programmatic
+    // launch it overlapped the previous kernel.  Global memory waits for it here.
+    grid_launch_dependents();
+    grid_dependency_wait();
     constexpr uint32_t cP = 0, cOI = 64, cOX = 192, cDS = 320;
 
     if (warp == 0) {
@@ -410,7 +414,7 @@ la_status retention_fwd(const void *q, const void *k, const void *v, void *o, co
     LA_TRY(retention_map(&jobs.k[0], k, s));
     LA_TRY(retention_map(&jobs.v[0], v, s));
     LA_TRY(retention_map(&jobs.o[0], o, s));
-    return launch("tc_retention_fwd", retention_kernel, dim3((unsigned)s.BH()), dim3(kThreads),
+    return launch_pdl("tc_retention_fwd", retention_kernel, dim3((unsigned)s.BH()), dim3(kThreads),
                   (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
 }
 
@@ -428,7 +432,7 @@ la_status retention_bwd(const void *q, const void *k, const void *v, const void 
         LA_TRY(retention_map(&jobs.o[p], out[p], s));
         jobs.rev[p] = p > 0;
     }
-    return launch("tc_retention_bwd", retention_kernel, dim3((unsigned)(3 * s.BH())), dim3(kThreads),
+    return launch_pdl("tc_retention_bwd", retention_kernel, dim3((unsigned)(3 * s.BH())), dim3(kThreads),
                   (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
 }
 

@@ -139,6 +139,10 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Everything above touched only shared memory and TMEM: with a programmatic
+    // launch it overlapped the previous kernel.  Global memory waits for it here.
+    grid_launch_dependents();
+    grid_dependency_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -342,6 +346,10 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Everything above touched only shared memory and TMEM: with a programmatic
+    // launch it overlapped the previous kernel.  Global memory waits for it here.
+    grid_launch_dependents();
+    grid_dependency_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -612,6 +620,10 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Everything above touched only shared memory and TMEM: with a programmatic
+    // launch it overlapped the previous kernel.  Global memory waits for it here.
+    grid_launch_dependents();
+    grid_dependency_wait();
     constexpr uint32_t kAccS = 176;    // columns 176..255: the M=64 [dS | dz] accumulator
 
     if (warp == 0) {
@@ -985,6 +997,10 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Everything above touched only shared memory and TMEM: with a programmatic
+    // launch it overlapped the previous kernel.  Global memory waits for it here.
+    grid_launch_dependents();
+    grid_dependency_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -1208,7 +1224,7 @@ static size_t partial_bytes(const Shape &s) {
 template <bool BIDIR, bool BF16>
 static la_status launch_reduce(const CUtensorMap &mk, const CUtensorMap &mv, float *part, const Shape &s, int nt,
                                cudaStream_t st) {
-    return launch(BIDIR ? "tc_state_reduce" : "tc_state_reduce_simple", state_reduce_kernel<BIDIR, BF16>,
+    return launch_pdl(BIDIR ? "tc_state_reduce" : "tc_state_reduce_simple", state_reduce_kernel<BIDIR, BF16>,
                   dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads), (size_t)ReduceLayout<BIDIR, BF16>::bytes, st, mk, mv, part, s.T, (int)s.BH(), nt,
                   max_slots((int)s.BH()));
 }
@@ -1225,7 +1241,7 @@ static la_status fwd_t(const void *q, const void *k, const void *v, void *o, flo
     const int ms = max_slots((int)s.BH());
     float *part = (float *)ws;
     LA_TRY((launch_reduce<BIDIR, BF16>(mk, mv, part, s, nt, st)));
-    return launch(BIDIR ? "tc_output" : "tc_output_simple", output_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
+    return launch_pdl(BIDIR ? "tc_output" : "tc_output_simple", output_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
                   (size_t)OutputLayout::bytes, st, mq, mo, (const float *)part, ms * kStateElems, 0, state, s.T, (int)s.BH(), nt,
                   eps);
 }
@@ -1253,10 +1269,10 @@ static la_status bwd_t(const void *q, const void *k, const void *v, const void *
         per_head = ms * kStateElems;
         single = 0;
     }
-    LA_TRY(launch(BIDIR ? "tc_bwd_q" : "tc_bwd_q_simple", bwd_q_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
+    LA_TRY(launch_pdl(BIDIR ? "tc_bwd_q" : "tc_bwd_q_simple", bwd_q_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
                   (size_t)BwdQLayout<BIDIR, BF16>::bytes, st, mq, mg, mdq, src, per_head, single, dpart, s.T, (int)s.BH(),
                   nt, ms, eps));
-    return launch(BIDIR ? "tc_bwd_kv" : "tc_bwd_kv_simple", bwd_kv_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
+    return launch_pdl(BIDIR ? "tc_bwd_kv" : "tc_bwd_kv_simple", bwd_kv_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
                   (size_t)BwdKvLayout::bytes, st, mk, mv, mdk, mdv, (const float *)dpart, s.T, (int)s.BH(), nt, ms);
 }
 
