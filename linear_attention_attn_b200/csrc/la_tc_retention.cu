@@ -168,9 +168,10 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // Everything above touched only shared memory and TMEM: with a programmatic
-    // launch it overlapped the previous kernel.  Global memory waits for it here.
-    grid_launch_dependents();
+    // launch it overlapped the previous kernel.  Global memory waits for it here;
+    // dependents are released only once this kernel is past its own wait.
     grid_dependency_wait();
+    if (threadIdx.x == 0) grid_launch_dependents();
     constexpr uint32_t cP = 0, cOI = 64, cOX = 192, cDS = 320;
 
     if (warp == 0) {

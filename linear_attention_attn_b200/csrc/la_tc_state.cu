@@ -140,9 +140,10 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // Everything above touched only shared memory and TMEM: with a programmatic
-    // launch it overlapped the previous kernel.  Global memory waits for it here.
-    grid_launch_dependents();
+    // launch it overlapped the previous kernel.  Global memory waits for it here;
+    // dependents are released only once this kernel is past its own wait.
     grid_dependency_wait();
+    if (threadIdx.x == 0) grid_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -289,7 +290,7 @@ template <bool BIDIR, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
               const float *__restrict__ src, int src_per_head, int src_single, float *__restrict__ state_out, int T,
-              int BH, int nt, float eps) {
+              int BH, int nt, float eps, int early_loads) {
     using L = OutputLayout;
     constexpr int NST = L::NST, OST = L::OST, OPB = L::OPB;
     constexpr int NOPS = BF16 ? 2 : 1;
@@ -347,9 +348,12 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // Everything above touched only shared memory and TMEM: with a programmatic
-    // launch it overlapped the previous kernel.  Global memory waits for it here.
-    grid_launch_dependents();
-    grid_dependency_wait();
+    // launch it overlapped the previous kernel.  With `early_loads` (the previous
+    // kernel is the first kernel of the same call, which writes none of this
+    // kernel's inputs) the TMA producer starts streaming inputs right away; every
+    // other access to global memory waits for the previous kernel here.
+    if (!(early_loads && warp == 0)) grid_dependency_wait();
+    if (threadIdx.x == 64) grid_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -541,7 +545,8 @@ template <bool BIDIR, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
              const __grid_constant__ CUtensorMap tmDQ, const float *__restrict__ src, int src_per_head,
-             int src_single, float *__restrict__ dpart, int T, int BH, int nt, int maxslots, float eps) {
+             int src_single, float *__restrict__ dpart, int T, int BH, int nt, int maxslots, float eps,
+             int early_loads) {
     using L = BwdQLayout<BIDIR, BF16>;
     constexpr int NST = L::NST, OPB = L::OPB;
     constexpr bool QLO = L::QLO;
@@ -621,9 +626,12 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // Everything above touched only shared memory and TMEM: with a programmatic
-    // launch it overlapped the previous kernel.  Global memory waits for it here.
-    grid_launch_dependents();
-    grid_dependency_wait();
+    // launch it overlapped the previous kernel.  With `early_loads` (the previous
+    // kernel is the first kernel of the same call, which writes none of this
+    // kernel's inputs) the TMA producer starts streaming inputs right away; every
+    // other access to global memory waits for the previous kernel here.
+    if (!(early_loads && warp == 0)) grid_dependency_wait();
+    if (threadIdx.x == 64) grid_launch_dependents();
     constexpr uint32_t kAccS = 176;    // columns 176..255: the M=64 [dS | dz] accumulator
 
     if (warp == 0) {
@@ -936,7 +944,7 @@ template <bool BIDIR, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
               const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
-              const float *__restrict__ dpart, int T, int BH, int nt, int maxslots) {
+              const float *__restrict__ dpart, int T, int BH, int nt, int maxslots, int early_loads) {
     using L = BwdKvLayout;
     constexpr int NST = L::NST, OPB = L::OPB;
     constexpr int NOPS = BF16 ? 2 : 1;
@@ -998,9 +1006,12 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // Everything above touched only shared memory and TMEM: with a programmatic
-    // launch it overlapped the previous kernel.  Global memory waits for it here.
-    grid_launch_dependents();
-    grid_dependency_wait();
+    // launch it overlapped the previous kernel.  With `early_loads` (the previous
+    // kernel is the first kernel of the same call, which writes none of this
+    // kernel's inputs) the TMA producer starts streaming inputs right away; every
+    // other access to global memory waits for the previous kernel here.
+    if (!(early_loads && warp == 0)) grid_dependency_wait();
+    if (threadIdx.x == 64) grid_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -1243,7 +1254,7 @@ static la_status fwd_t(const void *q, const void *k, const void *v, void *o, flo
     LA_TRY((launch_reduce<BIDIR, BF16>(mk, mv, part, s, nt, st)));
     return launch_pdl(BIDIR ? "tc_output" : "tc_output_simple", output_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
                   (size_t)OutputLayout::bytes, st, mq, mo, (const float *)part, ms * kStateElems, 0, state, s.T, (int)s.BH(), nt,
-                  eps);
+                  eps, 1);
 }
 
 template <bool BIDIR, bool BF16>
@@ -1271,9 +1282,9 @@ static la_status bwd_t(const void *q, const void *k, const void *v, const void *
     }
     LA_TRY(launch_pdl(BIDIR ? "tc_bwd_q" : "tc_bwd_q_simple", bwd_q_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
                   (size_t)BwdQLayout<BIDIR, BF16>::bytes, st, mq, mg, mdq, src, per_head, single, dpart, s.T, (int)s.BH(),
-                  nt, ms, eps));
+                  nt, ms, eps, state ? 0 : 1));
     return launch_pdl(BIDIR ? "tc_bwd_kv" : "tc_bwd_kv_simple", bwd_kv_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
-                  (size_t)BwdKvLayout::bytes, st, mk, mv, mdk, mdv, (const float *)dpart, s.T, (int)s.BH(), nt, ms);
+                  (size_t)BwdKvLayout::bytes, st, mk, mv, mdk, mdv, (const float *)dpart, s.T, (int)s.BH(), nt, ms, 1);
 }
 
 }  // namespace
