@@ -205,14 +205,14 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                 if (!LA_RWAIT(&full[s], ph, 0x4u)) break;
                 if (c > 0 && !LA_RWAIT(ptready, pp, 0x8u)) break;   // P accumulator read
                 tc_fence_after();
-                const uint32_t aQ = smem_u32(sQ + s * kTile128), aK = smem_u32(sK + s * kTile128);
-                const uint32_t aV = smem_u32(sV + s * kTile128);
+                const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTile128), 16, 1024);
+                const uint64_t dk = sdesc_sw128(smem_u32(sK + s * kTile128), 16, 1024);
+                const uint64_t dv = sdesc_sw128(smem_u32(sV + s * kTile128), kBox, 1024);
                 // P = Q K^T
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                    umma_f16_ss(tmem + cP, sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024), ID_P,
-                                kk ? 1u : 0u);
+                    umma_f16_ss(tmem + cP, desc_at(dq, off), desc_at(dk, off), ID_P, kk ? 1u : 0u);
                 }
                 umma_commit(pfull);
                 // O_intra = P~ V and O_inter = Q S
@@ -220,12 +220,13 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                 if (c > 0 && !LA_RWAIT(sready, pp, 0x20u)) break;
                 if (c > 0 && !LA_RWAIT(oread, pp, 0x40u)) break;
                 tc_fence_after();
+                const uint64_t dpt = sdesc_sw128(smem_u32(sPt), 16, 1024);
+                const uint64_t ds = sdesc_sw128(smem_u32(sS), 16384, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bv = sdesc_sw128(aV + kk * 2048, kBox, 1024);
 #pragma unroll
                     for (int op = 0; op < 2; ++op)
-                        umma_f16_ss(tmem + cOI, sdesc_sw128(smem_u32(sPt + op * kBox) + kk * 32, 16, 1024), bv, ID_OI,
+                        umma_f16_ss(tmem + cOI, desc_at(dpt, op * kBox + kk * 32), desc_at(dv, kk * 2048), ID_OI,
                                     (kk | op) ? 1u : 0u);
                 }
 #pragma unroll
@@ -233,21 +234,20 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                     const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
 #pragma unroll
                     for (int op = 0; op < 2; ++op)
-                        umma_f16_ss(tmem + cOX, sdesc_sw128(aQ + off, 16, 1024),
-                                    sdesc_sw128(smem_u32(sS + op * 32768) + kk * 2048, 16384, 1024), ID_OI,
+                        umma_f16_ss(tmem + cOX, desc_at(dq, off), desc_at(ds, op * 32768 + kk * 2048), ID_OI,
                                     (kk | op) ? 1u : 0u);
                 }
                 umma_commit(ofull);
                 // dS = K^^T V
                 if (!LA_RWAIT(khready, pc, 0x80u)) break;
                 tc_fence_after();
+                const uint64_t dkh = sdesc_sw128(smem_u32(sKh), kBox, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bv = sdesc_sw128(aV + kk * 2048, kBox, 1024);
 #pragma unroll
                     for (int op = 0; op < 2; ++op)
-                        umma_f16_ss(tmem + cDS, sdesc_sw128(smem_u32(sKh + op * kTile128) + kk * 2048, kBox, 1024), bv,
-                                    ID_DS, (kk | op) ? 1u : 0u);
+                        umma_f16_ss(tmem + cDS, desc_at(dkh, op * kTile128 + kk * 2048), desc_at(dv, kk * 2048), ID_DS,
+                                    (kk | op) ? 1u : 0u);
                 }
                 umma_commit(dsfull);
                 umma_commit(&empty[s]);

@@ -178,16 +178,16 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 if (!LA_WAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)a * 128u;
-                const uint32_t aK = smem_u32(sK + s * kTileBytes), aV = smem_u32(sV + s * kTileBytes);
+                const uint32_t aV = smem_u32(sV + s * kTileBytes);
                 const uint32_t lbo = BIDIR ? (smem_u32(sOnes) - aV) : (uint32_t)kTileBytes;
+                const uint64_t dk = sdesc_sw128(smem_u32(sK + s * kTileBytes), kTileBytes, 1024);
+                const uint64_t dkl = sdesc_sw128(smem_u32(sKlo + s * kTileBytes), kTileBytes, 1024);
+                const uint64_t dv = sdesc_sw128(aV, lbo, 1024);
 #pragma unroll
                 for (int kk = 0; kk < kRows / 16; ++kk) {
-                    const uint64_t bd = sdesc_sw128(aV + kk * 2048, lbo, 1024);
-                    umma_f16_ss(d, sdesc_sw128(aK + kk * 2048, kTileBytes, 1024), bd, IDESC,
+                    umma_f16_ss(d, desc_at(dk, kk * 2048), desc_at(dv, kk * 2048), IDESC,
                                 (seg_start && kk == 0) ? 0u : 1u);
-                    if (KLO)
-                        umma_f16_ss(d, sdesc_sw128(smem_u32(sKlo + s * kTileBytes) + kk * 2048, kTileBytes, 1024), bd,
-                                    IDESC, 1u);
+                    if (KLO) umma_f16_ss(d, desc_at(dkl, kk * 2048), desc_at(dv, kk * 2048), IDESC, 1u);
                 }
                 umma_commit(&empty[s]);
                 if (seg_end) {
@@ -389,14 +389,14 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 if (!LA_WAIT(&accempty[a], aph ^ 1, 0x2u)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)a * 128u;
-                const uint32_t aQ = smem_u32(sQ + s * kTileBytes);
-                const uint32_t aOp = smem_u32(sOp + (hidx & 1) * 2 * OPB);
+                const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTileBytes), 16, 1024);
+                const uint64_t dop = sdesc_sw128(smem_u32(sOp + (hidx & 1) * 2 * OPB), 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
                     for (int op = 0; op < NOPS; ++op)
-                        umma_f16_ss(d, sdesc_sw128(aQ + kk * 32, 16, 1024),
-                                    sdesc_sw128(aOp + op * OPB + kk * 32, 16, 1024), IDESC, (kk | op) ? 1u : 0u);
+                        umma_f16_ss(d, desc_at(dq, kk * 32), desc_at(dop, op * OPB + kk * 32), IDESC,
+                                    (kk | op) ? 1u : 0u);
                 }
                 umma_commit(&empty[s]);
                 umma_commit(&accfull[a]);
@@ -670,12 +670,14 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 }
                 if (!LA_WAIT(&gnready[se], phe, 0x80u)) { dead = true; return; }
                 tc_fence_after();
-                const uint32_t aQ = smem_u32(sQ + se * kTileBytes), aG = smem_u32(sG + se * kTileBytes);
+                const uint32_t aG = smem_u32(sG + se * kTileBytes);
                 const uint32_t lbo = BIDIR ? smem_u32(sW + se * kTileBytes) - aG : (uint32_t)kTileBytes;
+                const uint64_t dq = sdesc_sw128(smem_u32(sQ + se * kTileBytes), kTileBytes, 1024);
+                const uint64_t dg = sdesc_sw128(aG, lbo, 1024);
 #pragma unroll
                 for (int kk = 0; kk < kRows / 16; ++kk)
-                    umma_f16_ss(tmem + kAccS, sdesc_sw128(aQ + kk * 2048, kTileBytes, 1024),
-                                sdesc_sw128(aG + kk * 2048, lbo, 1024), IDESC3, (seg_start && kk == 0) ? 0u : 1u);
+                    umma_f16_ss(tmem + kAccS, desc_at(dq, kk * 2048), desc_at(dg, kk * 2048), IDESC3,
+                                (seg_start && kk == 0) ? 0u : 1u);
                 umma_commit(&empty[se]);
                 if (seg_end) umma_commit(accSfull);
             };
@@ -699,21 +701,22 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 if (!LA_WAIT(&acc12empty[b], bph ^ 1, 0x2u)) break;
                 tc_fence_after();
                 const uint32_t d1 = tmem + (uint32_t)b * 256u, d2 = d1 + 96u;
-                const uint32_t aQ = smem_u32(sQ + s * kTileBytes), aG = smem_u32(sG + s * kTileBytes);
+                const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTileBytes), 16, 1024);
+                const uint64_t dg = sdesc_sw128(smem_u32(sG + s * kTileBytes), 16, 1024);
+                const uint64_t dql = sdesc_sw128(smem_u32(sQlo + s * kTileBytes), 16, 1024);
+                const uint64_t dok = sdesc_sw128(smem_u32(sOp), 16, 1024);     // state operand read K-major
+                const uint64_t dom = sdesc_sw128(smem_u32(sOp), OPB, 1024);    // ... and MN-major
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
                     for (int op = 0; op < NOPS; ++op) {
-                        const uint32_t aO = smem_u32(sOp + op * OPB);
                         if (BIDIR)
-                            umma_f16_ss(d1, sdesc_sw128(aQ + kk * 32, 16, 1024), sdesc_sw128(aO + kk * 32, 16, 1024),
-                                        IDESC1, (kk | op) ? 1u : 0u);
-                        umma_f16_ss(d2, sdesc_sw128(aG + kk * 32, 16, 1024), sdesc_sw128(aO + kk * 2048, OPB, 1024),
-                                    IDESC2, (kk | op) ? 1u : 0u);
+                            umma_f16_ss(d1, desc_at(dq, kk * 32), desc_at(dok, op * OPB + kk * 32), IDESC1,
+                                        (kk | op) ? 1u : 0u);
+                        umma_f16_ss(d2, desc_at(dg, kk * 32), desc_at(dom, op * OPB + kk * 2048), IDESC2,
+                                    (kk | op) ? 1u : 0u);
                     }
-                    if (QLO)
-                        umma_f16_ss(d1, sdesc_sw128(smem_u32(sQlo + s * kTileBytes) + kk * 32, 16, 1024),
-                                    sdesc_sw128(smem_u32(sOp) + kk * 32, 16, 1024), IDESC1, 1u);
+                    if (QLO) umma_f16_ss(d1, desc_at(dql, kk * 32), desc_at(dok, kk * 32), IDESC1, 1u);
                 }
                 umma_commit(&acc12full[b]);
                 b ^= 1;
@@ -1048,16 +1051,18 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 if (!LA_WAIT(&accempty[b], bph ^ 1, 0x2u)) break;
                 tc_fence_after();
                 const uint32_t da = tmem + (uint32_t)b * 128u, db = da + 64u;
-                const uint32_t aK = smem_u32(sK + s * kTileBytes), aV = smem_u32(sV + s * kTileBytes);
+                const uint64_t dk = sdesc_sw128(smem_u32(sK + s * kTileBytes), 16, 1024);
+                const uint64_t dv = sdesc_sw128(smem_u32(sV + s * kTileBytes), 16, 1024);
+                const uint64_t dok = sdesc_sw128(smem_u32(sOp), 16, 1024);
+                const uint64_t dom = sdesc_sw128(smem_u32(sOp), OPB, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
                     for (int op = 0; op < NOPS; ++op) {
-                        const uint32_t aO = smem_u32(sOp + op * OPB);
-                        umma_f16_ss(da, sdesc_sw128(aV + kk * 32, 16, 1024), sdesc_sw128(aO + kk * 32, 16, 1024),
-                                    IDESC_A, (kk | op) ? 1u : 0u);
-                        umma_f16_ss(db, sdesc_sw128(aK + kk * 32, 16, 1024), sdesc_sw128(aO + kk * 2048, OPB, 1024),
-                                    IDESC_B, (kk | op) ? 1u : 0u);
+                        umma_f16_ss(da, desc_at(dv, kk * 32), desc_at(dok, op * OPB + kk * 32), IDESC_A,
+                                    (kk | op) ? 1u : 0u);
+                        umma_f16_ss(db, desc_at(dk, kk * 32), desc_at(dom, op * OPB + kk * 2048), IDESC_B,
+                                    (kk | op) ? 1u : 0u);
                     }
                 }
                 umma_commit(&empty[s]);
