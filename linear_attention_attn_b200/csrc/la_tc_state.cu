@@ -13,10 +13,10 @@
 //
 // Every kernel is persistent: kGrid CTAs split the head-major list of 128-row
 // tiles into contiguous ranges (Partition).  Warp 0 streams q/k/v/dO tiles with
-// TMA into a ring of 128-byte-swizzled stages; warp 1 issues tcgen05 UMMAs
-// (fp32 accumulators in TMEM); warps 2..5 apply the feature map in place, run
-// the epilogues (TMEM -> registers -> swizzled staging -> TMA store) and build
-// the per-head state operand.  A reduction's per-CTA partial goes to slot
+// TMA into a ring of 128-byte-swizzled stages; warp 1 owns TMEM and issues the
+// tcgen05 UMMAs (fp32 accumulators in TMEM); warps 2..9 apply the feature map in
+// place (half a row each); warps 10..13 run the epilogues (TMEM -> registers ->
+// swizzled staging -> TMA store) and build the per-head state operand.  A reduction's per-CTA partial goes to slot
 // (cta - first_cta(head)) of the workspace; its consumer sums the slots in slot
 // order, so results are deterministic.
 //
