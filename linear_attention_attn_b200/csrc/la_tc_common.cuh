@@ -329,19 +329,71 @@ __device__ __forceinline__ float operand_scale(float m) {
     return ldexpf(1.f, e);
 }
 
-// One row of a K-major 128-byte-swizzled 16-bit operand from 64 fp32 values
-// scaled by sc: hi = round(x), lo = round(x - hi) (lo only with NOPS == 2).
-template <bool BF16, int NOPS>
-__device__ __forceinline__ void operand_row(uint8_t *op0, uint8_t *op1, int row, const float (&x)[64]) {
-    float hi[64];
-    store_row<BF16>(op0, row, x);
-    if (NOPS == 2) {
-        load_row<BF16>(op0, row, hi);
-        float lo[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) lo[i] = x[i] - hi[i];
-        store_row<BF16>(op1, row, lo);
+// (head, tile-in-head) of the tile indices x0, x0 + 1, ... of a Partition, advanced
+// without a 64-bit division per tile (an emulated division costs hundreds of cycles).
+struct TileCursor {
+    long long x;
+    int h, j, nt;
+    __device__ __forceinline__ TileCursor(long long x0, int nt_)
+        : x(x0), h((int)(x0 / nt_)), j((int)(x0 % nt_)), nt(nt_) {}
+    __device__ __forceinline__ void next() {
+        ++x;
+        if (++j == nt) { j = 0; ++h; }
     }
+    __device__ __forceinline__ bool last_of_head() const { return j + 1 == nt; }
+};
+
+// Rows [0, nrows) of a K-major 128-byte-swizzled 16-bit operand (64 K values per
+// row) from the fp32 state block [64][65] in shared memory, scaled by sc:
+//   COLUMNS:  row n, element i = stage[i][n]  (column n of S; n == 64 is z when
+//             with_z, and rows without a source are zero)
+//   !COLUMNS: row n, element i = stage[n][i]  (row n of S)
+// hi = round(x), lo = round(x - hi) (lo only with NOPS == 2).  The 128 worker
+// threads take (row, 8-element chunk) pairs, consecutive rows in consecutive
+// threads, so neither the reads (row stride 65 words) nor the swizzled 16-byte
+// writes conflict.  The loop stays rolled: this runs once per head, and an
+// unrolled copy costs more in cold instruction fetch than it saves.
+template <bool BF16, int NOPS, bool COLUMNS>
+__device__ __forceinline__ void build_state_operand(const float *stage, float sc, int nrows, bool with_z, uint8_t *op0,
+                                                    uint8_t *op1, int tid) {
+#pragma unroll 1
+    for (int task = tid; task < nrows * 8; task += kWorkers) {
+        const int n = task % nrows, c = task / nrows;
+        float x[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int i = 8 * c + k;
+            if (COLUMNS)
+                x[k] = (n < 64 || (n == 64 && with_z)) ? stage[i * 65 + n] * sc : 0.f;
+            else
+                x[k] = stage[n * 65 + i] * sc;
+        }
+        const int off = n * 128 + ((c ^ (n & 7)) << 4);
+        uint4 u;
+        u.x = h2<BF16>::from_f2(x[0], x[1]);
+        u.y = h2<BF16>::from_f2(x[2], x[3]);
+        u.z = h2<BF16>::from_f2(x[4], x[5]);
+        u.w = h2<BF16>::from_f2(x[6], x[7]);
+        *reinterpret_cast<uint4 *>(op0 + off) = u;
+        if (NOPS == 2) {
+            const uint32_t hw[4] = {u.x, u.y, u.z, u.w};
+            uint32_t lw[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 hv = h2<BF16>::to_f2(hw[k]);
+                lw[k] = h2<BF16>::from_f2(x[2 * k] - hv.x, x[2 * k + 1] - hv.y);
+            }
+            *reinterpret_cast<uint4 *>(op1 + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+    }
+}
+
+// sum_i |stage[i][64]| (the z column), the same value in every lane of the warp.
+__device__ __forceinline__ float warp_abs_z_sum(const float *stage, int lane) {
+    float v = fabsf(stage[lane * 65 + 64]) + fabsf(stage[(lane + 32) * 65 + 64]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
 }
 
 }  // namespace tc

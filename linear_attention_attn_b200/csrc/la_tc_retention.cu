@@ -74,6 +74,7 @@ struct RetLayout {
     static constexpr int nbars = 2 * NST + 9;
     static constexpr int misc = baroff + nbars * 8;
     static constexpr int bytes = misc + 32 + 1024;
+    static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 // Up to three retention passes in one launch: pass p reads (q, k, v) through

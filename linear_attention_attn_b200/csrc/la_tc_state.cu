@@ -72,6 +72,7 @@ struct ReduceLayout {
     static constexpr int nbars = 3 * NST + 5;
     static constexpr int misc = baroff + nbars * 8;
     static constexpr int bytes = misc + 32 + 1024;
+    static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 template <bool BIDIR, bool BF16>
@@ -150,8 +151,9 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             int s = 0;
             uint32_t ph = 0;
             long long issued = 0;
-            for (long long x = x0; x < x1; ++x) {
-                const int h = (int)(x / nt), j = (int)(x % nt);
+            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
+                const int h = t.h, j = t.j;
                 if (!LA_WAIT(&empty[s], ph ^ 1, 0x1u)) break;
                 mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
                 tma_load_3d(sK + s * kTileBytes, &tmK, &full[s], 0, j * kRows, h);
@@ -169,9 +171,10 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             int s = 0, a = 0;
             uint32_t ph = 0, aph = 0;
             bool seg_start = true;
-            for (long long x = x0; x < x1; ++x) {
-                const long long h = x / nt;
-                const bool seg_end = (x + 1 == x1) || ((x + 1) / nt != h);
+            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
+                const long long h = t.h;
+                const bool seg_end = (x + 1 == x1) || t.last_of_head();
                 if (seg_start) {
                     if (!LA_WAIT(&accfree[a], aph ^ 1, 0x2u)) break;
                 }
@@ -206,8 +209,9 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             const int xi = threadIdx.x - kXw0 * 32;
             int s = 0;
             uint32_t ph = 0;
-            for (long long x = x0; x < x1; ++x) {
-                const int j = (int)(x % nt);
+            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
+                const int j = t.j;
                 const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
                 if (!got) break;
                 const bool pad = j * kRows + (xi & 127) >= T;   // rows past the end: f(0) = 1 must not count
@@ -225,9 +229,10 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const int sub = warp & 3;
         int a = 0;
         uint32_t aph = 0;
-        for (long long x = x0; x < x1; ++x) {
-            const int h = (int)(x / nt);
-            const bool seg_end = (x + 1 == x1) || ((x + 1) / nt != h);
+        for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
+            const int h = t.h;
+            const bool seg_end = (x + 1 == x1) || t.last_of_head();
             if (!seg_end) continue;
             const bool got = __all_sync(0xffffffffu, LA_WAIT(&accfull[a], aph, 0x10u));
             if (!got) break;
@@ -284,6 +289,7 @@ struct OutputLayout {
     static constexpr int nbars = 3 * NST + 2 + 2 + 2 + 1;
     static constexpr int misc = baroff + nbars * 8;
     static constexpr int bytes = misc + 32 + 1024;
+    static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 template <bool BIDIR, bool BF16>
@@ -360,8 +366,9 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             int s = 0;
             uint32_t ph = 0;
             long long issued = 0;
-            for (long long x = x0; x < x1; ++x) {
-                const int h = (int)(x / nt), j = (int)(x % nt);
+            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
+                const int h = t.h, j = t.j;
                 if (!LA_WAIT(&empty[s], ph ^ 1, 0x1u)) break;
                 mbar_arrive_expect_tx(&full[s], kTileBytes);
                 tma_load_3d(sQ + s * kTileBytes, &tmQ, &full[s], 0, j * kRows, h);
@@ -378,8 +385,9 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             int s = 0, a = 0, hidx = -1;
             uint32_t ph = 0, aph = 0;
             long long prev_h = -1;
-            for (long long x = x0; x < x1; ++x) {
-                const long long h = x / nt;
+            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
+                const long long h = t.h;
                 if (h != prev_h) {
                     ++hidx;
                     prev_h = h;
@@ -412,7 +420,8 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const int xi = threadIdx.x - kXw0 * 32;
             int s = 0;
             uint32_t ph = 0;
-            for (long long x = x0; x < x1; ++x) {
+            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
                 const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
                 if (!got) break;
                 phi_half_row<BF16>(sQ + s * kTileBytes, xi, false);   // rows past T are never stored
@@ -445,21 +454,16 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (!BF16) m = workers_max(m, red, tid);
             const float sc = operand_scale<BF16>(m);
             uint8_t *op0 = sOp + buf * 2 * OPB;
-            if (tid < 80) {
-                float xv[64];
-#pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    xv[i] = tid < 64 ? stage[i * 65 + tid] * sc : ((BIDIR && tid == 64) ? stage[i * 65 + 64] * sc : 0.f);
-                operand_row<BF16, NOPS>(op0, op0 + OPB, tid, xv);
-            }
+            build_state_operand<BF16, NOPS, true>(stage, sc, 80, BIDIR, op0, op0 + OPB, tid);
             if (tid == 0) s_scale[buf] = sc;
             fence_async_smem();
             named_bar(1, kWorkers);
             if (tid == 0) mbar_arrive(&opready[buf]);
         };
-        for (long long x = x0; x < x1; ++x) {
-            const long long h = x / nt;
-            const int j = (int)(x % nt);
+        for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
+            const long long h = t.h;
+            const int j = t.j;
             if (h != cur_h) {
                 ++hidx;
                 cur_h = h;
@@ -525,7 +529,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 template <bool BIDIR, bool BF16>
 struct BwdQLayout {
     static constexpr bool QLO = BIDIR && BF16;
-    static constexpr int NST = BIDIR ? (QLO ? 2 : 3) : 4, OST = 1, OPB = 80 * 128;
+    static constexpr int NST = BIDIR ? (QLO ? 2 : 3) : 4, OST = 2, OPB = 80 * 128;
     static constexpr int qoff = 0;
     static constexpr int goff = qoff + NST * kTileBytes;
     static constexpr int woff = goff + NST * kTileBytes;
@@ -539,6 +543,7 @@ struct BwdQLayout {
     static constexpr int nbars = 4 * NST + 8;
     static constexpr int misc = baroff + nbars * 8;
     static constexpr int bytes = misc + 32 + 1024;
+    static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 template <bool BIDIR, bool BF16>
@@ -639,8 +644,9 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             int s = 0;
             uint32_t ph = 0;
             long long issued = 0;
-            for (long long x = x0; x < x1; ++x) {
-                const int h = (int)(x / nt), j = (int)(x % nt);
+            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
+                const int h = t.h, j = t.j;
                 if (!LA_WAIT(&empty[s], ph ^ 1, 0x1u)) break;
                 mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
                 tma_load_3d(sQ + s * kTileBytes, &tmQ, &full[s], 0, j * kRows, h);
@@ -661,9 +667,9 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             long long seg = 0;                     // segments started (accS free parity)
             bool dead = false;
             // MMA3 of tile xe (stage se, phase phe)
-            auto issue3 = [&](long long xe, int se, uint32_t phe) {
-                const bool seg_start = (xe == x0) || (xe % nt == 0);
-                const bool seg_end = (xe + 1 == x1) || ((xe + 1) % nt == 0);
+            auto issue3 = [&](long long xe, int je, int se, uint32_t phe) {
+                const bool seg_start = (xe == x0) || je == 0;
+                const bool seg_end = (xe + 1 == x1) || je + 1 == nt;
                 if (seg_start) {
                     if (!LA_WAIT(accSfree, (uint32_t)((seg & 1) ^ 1), 0x40u)) { dead = true; return; }
                     ++seg;
@@ -682,14 +688,15 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 if (seg_end) umma_commit(accSfull);
             };
             long long xp = -1;
-            int sp = 0;
+            int sp = 0, jp = 0;
             uint32_t php = 0;
-            for (long long x = x0; x < x1 && !dead; ++x) {
-                const long long h = x / nt;
+            for (TileCursor t(x0, nt); t.x < x1 && !dead; t.next()) {
+                const long long x = t.x;
+                const long long h = t.h;
                 if (h != prev_h) {
                     // finish the previous head (its dS partial) before waiting on the next operand
                     if (xp >= 0) {
-                        issue3(xp, sp, php);
+                        issue3(xp, jp, sp, php);
                         xp = -1;
                         if (dead) break;
                     }
@@ -721,13 +728,14 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 umma_commit(&acc12full[b]);
                 b ^= 1;
                 if (b == 0) bph ^= 1;
-                if (xp >= 0) issue3(xp, sp, php);
+                if (xp >= 0) issue3(xp, jp, sp, php);
                 xp = x;
+                jp = t.j;
                 sp = s;
                 php = ph;
                 if (++s == NST) { s = 0; ph ^= 1; }
             }
-            if (xp >= 0 && !dead && !*s_abort) issue3(xp, sp, php);
+            if (xp >= 0 && !dead && !*s_abort) issue3(xp, jp, sp, php);
             umma_commit(drain);
             mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
         }
@@ -736,7 +744,8 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             const int xi = threadIdx.x - kXw0 * 32;
             int s = 0;
             uint32_t ph = 0;
-            for (long long x = x0; x < x1; ++x) {
+            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
                 const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
                 if (!got) break;
                 if (QLO)
@@ -767,8 +776,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             named_bar(1, kWorkers);
             if (!BF16) m = workers_max(m, red, tid);
             const float sc = operand_scale<BF16>(m);
-            float zsum = 0.f;
-            for (int i = 0; i < 64; ++i) zsum += fabsf(stage[i * 65 + 64]);
+            const float zsum = BIDIR ? warp_abs_z_sum(stage, tid & 31) : 0.f;
             float scn = 1.f;
             if (BIDIR && zsum > 0.f && isfinite(zsum)) {
                 int e;
@@ -776,13 +784,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 e = e < -100 ? -100 : (e > 100 ? 100 : e);
                 scn = ldexpf(1.f, e - 1);
             }
-            if (tid < 80) {
-                float xv[64];
-#pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    xv[i] = tid < 64 ? stage[i * 65 + tid] * sc : ((BIDIR && tid == 64) ? stage[i * 65 + 64] * sc : 0.f);
-                operand_row<BF16, NOPS>(sOp, sOp + OPB, tid, xv);
-            }
+            build_state_operand<BF16, NOPS, true>(stage, sc, 80, BIDIR, sOp, sOp + OPB, tid);
             if (tid < 64) zs[tid] = stage[tid * 65 + 64] * sc;
             fence_async_smem();
             named_bar(1, kWorkers);
@@ -823,16 +825,18 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             }
         };
 
-        for (long long x = x0; x < x1; ++x) {
-            const long long h = x / nt;
-            const int j = (int)(x % nt);
+        for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
+            const long long h = t.h;
+            const int j = t.j;
             if (h != cur_h) {
                 build(h);
                 cur_h = h;
             }
-            // ---- epilogue of tile x (stage s, accumulator pair b)
-            if (tid == 0) tma_store_wait_read<0>();
+            // ---- epilogue of tile x (stage s, accumulator pair b, dq staging buffer x % OST)
+            if (tid == 0) tma_store_wait_read<L::OST - 1>();
             named_bar(1, kWorkers);
+            uint8_t *sDQx = sDQ + (int)(x & (L::OST - 1)) * kTileBytes;
             bool got = live && LA_WAIT(&acc12full[b], bph, 0x10u);
             got = __all_sync(0xffffffffu, got);
             live = live && got;
@@ -843,20 +847,19 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 uint8_t *tq = sQ + s * kTileBytes, *tg = sG + s * kTileBytes;
                 float gdot = 0.f, inv = 1.f;
                 if (BIDIR) {
-                    float t16[16];
+                    // u = f(q) S and q.z (one wait for all five loads)
+                    float u[64], t16[16];
                     tmem_ld16(d1 + 64, t16);
-                    tmem_ld_wait();
+                    tmem_row64(d1, u);
                     inv = 1.f / (t16[0] + eps * cur_sc);
                     const float gsc = inv * cur_sc * cur_scn;
 #pragma unroll
                     for (int c16 = 0; c16 < 4; ++c16) {
-                        float u[16], g[16];
-                        tmem_ld16(d1 + 16 * c16, u);
+                        float g[16];
                         load_chunk16<BF16>(tg, row, c16, g);
-                        tmem_ld_wait();
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            gdot = fmaf(g[i], u[i], gdot);
+                            gdot = fmaf(g[i], u[16 * c16 + i], gdot);
                             g[i] *= gsc;
                         }
                         store_chunk16<BF16>(tg, row, c16, g);   // g/n (scaled) over dO: MMA2 is done with it
@@ -869,33 +872,58 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                         *reinterpret_cast<__half *>(sW + s * kTileBytes + sw128_offset(row, 0)) = __float2half_rn(w);
                 }
                 const float isc = 1.f / cur_sc;
+                // g S^T in two halves of 32 columns (one wait each)
 #pragma unroll
-                for (int c16 = 0; c16 < 4; ++c16) {
-                    float acc[16], dq[16];
-                    tmem_ld16(d2 + 16 * c16, acc);
-                    if (BIDIR) {
-                        float qf[16];
-                        load_chunk16<BF16>(tq, row, c16, qf);
-                        if (QLO) {
-                            float ql[16];
-                            load_chunk16<BF16>(sQlo + s * kTileBytes, row, c16, ql);
+                for (int hf = 0; hf < 2; ++hf) {
+                    float acc[32];
+                    {
+                        float a0[16], a1[16];
+                        tmem_ld16(d2 + 32 * hf, a0);
+                        tmem_ld16(d2 + 32 * hf + 16, a1);
+                        tmem_ld_wait();
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) qf[i] += ql[i];
+                        for (int i = 0; i < 16; ++i) {
+                            acc[i] = a0[i];
+                            acc[16 + i] = a1[i];
                         }
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            dq[i] = (acc[i] - gdot * zs[16 * c16 + i]) * inv * fminf(qf[i], 1.f);
-                    } else {
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) dq[i] = acc[i] * isc;
                     }
-                    store_chunk16<BF16>(sDQ, row, c16, dq);
+                    if (hf == 1) {
+                        // every TMEM read of this accumulator pair is complete
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&acc12empty[b]);
+                    }
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c16 = 2 * hf + cc;
+                        float dq[16];
+                        if (BIDIR) {
+                            float qf[16];
+                            load_chunk16<BF16>(tq, row, c16, qf);
+                            if (QLO) {
+                                float ql[16];
+                                load_chunk16<BF16>(sQlo + s * kTileBytes, row, c16, ql);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) qf[i] += ql[i];
+                            }
+                            const float4 *z4 = reinterpret_cast<const float4 *>(zs + 16 * c16);
+#pragma unroll
+                            for (int i4 = 0; i4 < 4; ++i4) {
+                                const float4 zz = z4[i4];
+                                const float zv[4] = {zz.x, zz.y, zz.z, zz.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int i = 4 * i4 + e;
+                                    dq[i] = (acc[16 * cc + i] - gdot * zv[e]) * inv * fminf(qf[i], 1.f);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) dq[i] = acc[16 * cc + i] * isc;
+                        }
+                        store_chunk16<BF16>(sDQx, row, c16, dq);
+                    }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc12empty[b]);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&gnready[s]);
@@ -904,10 +932,10 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             }
             named_bar(1, kWorkers);
             if (tid == 0 && live) {
-                tma_store_3d(&tmDQ, sDQ, 0, j * kRows, (int)h);
+                tma_store_3d(&tmDQ, sDQx, 0, j * kRows, (int)h);
                 tma_store_commit();
             }
-            const bool seg_end = (x + 1 == x1) || ((x + 1) % nt == 0);
+            const bool seg_end = (x + 1 == x1) || t.last_of_head();
             if (seg_end) read_accS((int)h, cur_scn);
             if (++s == NST) { s = 0; ph ^= 1; }
             b ^= 1;
@@ -941,6 +969,7 @@ struct BwdKvLayout {
     static constexpr int nbars = 3 * NST + 4 + 2;
     static constexpr int misc = baroff + nbars * 8;
     static constexpr int bytes = misc + 32 + 1024;
+    static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 template <bool BIDIR, bool BF16>
@@ -1021,8 +1050,9 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             int s = 0;
             uint32_t ph = 0;
             long long issued = 0;
-            for (long long x = x0; x < x1; ++x) {
-                const int h = (int)(x / nt), j = (int)(x % nt);
+            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
+                const int h = t.h, j = t.j;
                 if (!LA_WAIT(&empty[s], ph ^ 1, 0x1u)) break;
                 mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
                 tma_load_3d(sK + s * kTileBytes, &tmK, &full[s], 0, j * kRows, h);
@@ -1040,8 +1070,9 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             int s = 0, b = 0;
             uint32_t ph = 0, bph = 0, oph = 0;
             long long prev_h = -1;
-            for (long long x = x0; x < x1; ++x) {
-                const long long h = x / nt;
+            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
+                const long long h = t.h;
                 if (h != prev_h) {
                     if (!LA_WAIT(opready, oph, 0x20u)) break;
                     oph ^= 1;
@@ -1079,7 +1110,8 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             const int xi = threadIdx.x - kXw0 * 32;
             int s = 0;
             uint32_t ph = 0;
-            for (long long x = x0; x < x1; ++x) {
+            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
                 const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
                 if (!got) break;
                 phi_half_row<BF16>(sK + s * kTileBytes, xi, false);
@@ -1098,9 +1130,10 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         long long cur_h = -1;
         bool live = true;
         float cur_isd = 1.f;
-        for (long long x = x0; x < x1; ++x) {
-            const long long h = x / nt;
-            const int j = (int)(x % nt);
+        for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const long long x = t.x;
+            const long long h = t.h;
+            const int j = t.j;
             if (h != cur_h) {
                 // the previous head's UMMAs are complete (its last epilogue waited on them)
                 const float *srch = dpart + h * (long long)maxslots * kStateElems;
@@ -1109,13 +1142,8 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 named_bar(1, kWorkers);
                 if (!BF16) m = workers_max(m, red, tid);
                 const float sd = operand_scale<BF16>(m);
-                if (tid < 64) {
-                    float xv[64];
-#pragma unroll
-                    for (int jj = 0; jj < 64; ++jj) xv[jj] = stage[tid * 65 + jj] * sd;
-                    operand_row<BF16, NOPS>(sOp, sOp + OPB, tid, xv);
-                    dz[tid] = BIDIR ? stage[tid * 65 + 64] : 0.f;
-                }
+                build_state_operand<BF16, NOPS, false>(stage, sd, 64, false, sOp, sOp + OPB, tid);
+                if (tid < 64) dz[tid] = BIDIR ? stage[tid * 65 + 64] : 0.f;
                 fence_async_smem();
                 named_bar(1, kWorkers);
                 cur_isd = 1.f / sd;
