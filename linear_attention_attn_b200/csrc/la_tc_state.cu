@@ -522,18 +522,21 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 // ================================================================== bwd_q ==
 // Per tile: MMA1 [u | q.z] = f(Q) [S | z] (M=128, N=80), MMA2 g S^T (M=128, N=64,
 // B = the state operand read MN-major); the epilogue warps form n, o, g.o and dq
-// and write g/n (in place over the dO tile) and w = -(g.o)/n (column 0 of a
-// zero block); MMA3 accumulates [dS | dz] += f(Q)^T [g/n | w] (M=64, N=80, both
-// MN-major).  bf16 bidir also keeps lo = round(f(q) - hi): MMA1 adds
-// f(Q)_lo S_hi and f'(q) = min(hi + lo, 1).
+// and write g/n (in place over the dO tile) and w = -(g.o)/n; MMA3 accumulates
+// [dS | dz] += f(Q)^T [g/n | w] (M=64, N=80, both MN-major).  The 16 columns of
+// w's MN atom live in one zero-filled tile shared by the stages: stage s owns
+// columns 16 s .. 16 s + 15 (w in the first, zeros after), and MMA3's
+// descriptor points its second atom there (a start 32 s bytes into a 128-byte
+// row, as a K step does for K-major operands).  bf16 bidir also keeps
+// lo = round(f(q) - hi): MMA1 adds f(Q)_lo S_hi and f'(q) = min(hi + lo, 1).
 template <bool BIDIR, bool BF16>
 struct BwdQLayout {
     static constexpr bool QLO = BIDIR && BF16;
-    static constexpr int NST = BIDIR ? (QLO ? 2 : 3) : 4, OST = 2, OPB = 80 * 128;
+    static constexpr int NST = BIDIR ? (QLO ? 2 : 4) : 4, OST = 2, OPB = 80 * 128;
     static constexpr int qoff = 0;
     static constexpr int goff = qoff + NST * kTileBytes;
     static constexpr int woff = goff + NST * kTileBytes;
-    static constexpr int qloff = woff + (BIDIR ? NST * kTileBytes : 0);
+    static constexpr int qloff = woff + (BIDIR ? kTileBytes : 0);   // one w tile shared by the stages
     static constexpr int dqoff = qloff + (QLO ? NST * kTileBytes : 0);
     static constexpr int opoff = dqoff + OST * kTileBytes;
     static constexpr int stageoff = opoff + 2 * OPB;
@@ -613,13 +616,11 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         tma_prefetch(&tmG);
         tma_prefetch(&tmDQ);
     }
-    if (BIDIR && warp >= kEw0) {   // the w blocks: zero except column 0, written per tile
+    if (BIDIR && warp >= kEw0) {   // the w tile: zero except column 16 s of stage s, written per tile
         const int r = threadIdx.x - kEw0 * 32;
-        for (int st = 0; st < NST; ++st) {
-            uint8_t *p = sW + st * kTileBytes + r * 128;
+        uint8_t *p = sW + r * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(p + c * 16) = make_uint4(0u, 0u, 0u, 0u);
-        }
+        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(p + c * 16) = make_uint4(0u, 0u, 0u, 0u);
         fence_async_smem();
     }
     if (warp == 1) {
@@ -677,7 +678,8 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 if (!LA_WAIT(&gnready[se], phe, 0x80u)) { dead = true; return; }
                 tc_fence_after();
                 const uint32_t aG = smem_u32(sG + se * kTileBytes);
-                const uint32_t lbo = BIDIR ? smem_u32(sW + se * kTileBytes) - aG : (uint32_t)kTileBytes;
+                // the second MN atom of [g/n | w] starts at column 16 se of the shared w tile
+                const uint32_t lbo = BIDIR ? smem_u32(sW) + 32u * (uint32_t)se - aG : (uint32_t)kTileBytes;
                 const uint64_t dq = sdesc_sw128(smem_u32(sQ + se * kTileBytes), kTileBytes, 1024);
                 const uint64_t dg = sdesc_sw128(aG, lbo, 1024);
 #pragma unroll
@@ -866,10 +868,10 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                     }
                     gdot *= inv;
                     const float w = -gdot * gsc;
-                    if (BF16)
-                        *reinterpret_cast<__nv_bfloat16 *>(sW + s * kTileBytes + sw128_offset(row, 0)) = __float2bfloat16_rn(w);
-                    else
-                        *reinterpret_cast<__half *>(sW + s * kTileBytes + sw128_offset(row, 0)) = __float2half_rn(w);
+                    // columns 16 s .. 16 s + 7 of the w tile: (w, 0, ..., 0)
+                    const uint32_t wbits = BF16 ? (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(w))
+                                                : (uint32_t)__half_as_ushort(__float2half_rn(w));
+                    *reinterpret_cast<uint4 *>(sW + sw128_offset(row, 16 * s)) = make_uint4(wbits, 0u, 0u, 0u);
                 }
                 const float isc = 1.f / cur_sc;
                 // g S^T in two halves of 32 columns (one wait each)
