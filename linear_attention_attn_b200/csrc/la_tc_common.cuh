@@ -112,6 +112,38 @@ __device__ __forceinline__ void phi_row_inplace(uint8_t *tile, int row, bool zer
     }
 }
 
+// Feature map of one whole row of a 128-byte-swizzled tile in place, all eight
+// 16-byte chunks loaded before any is transformed (one shared-memory round trip
+// per row).  SPLIT keeps lo = round(phi(x) - hi) at the same position of lo_tile.
+template <bool BF16, bool SPLIT>
+__device__ __forceinline__ void phi_row_batched(uint8_t *tile, uint8_t *lo_tile, int row) {
+    uint8_t *p = tile + row * 128;
+    uint4 u[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) u[c] = *reinterpret_cast<const uint4 *>(p + ((c ^ (row & 7)) << 4));
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint32_t w[4] = {u[c].x, u[c].y, u[c].z, u[c].w}, l[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (!BF16 && !SPLIT) {
+                w[k] = phi_h2(w[k]);
+            } else {
+                const float2 f = h2<BF16>::to_f2(w[k]);
+                const float a = phi_f(f.x), b = phi_f(f.y);
+                w[k] = h2<BF16>::from_f2(a, b);
+                if (SPLIT) {
+                    const float2 hv = h2<BF16>::to_f2(w[k]);
+                    l[k] = h2<BF16>::from_f2(a - hv.x, b - hv.y);
+                }
+            }
+        }
+        const int off = (c ^ (row & 7)) << 4;
+        *reinterpret_cast<uint4 *>(p + off) = make_uint4(w[0], w[1], w[2], w[3]);
+        if (SPLIT) *reinterpret_cast<uint4 *>(lo_tile + row * 128 + off) = make_uint4(l[0], l[1], l[2], l[3]);
+    }
+}
+
 // Feature map with a two-term result: hi = round(phi(x)) replaces x in place,
 // lo = round(phi(x) - hi) goes to the same position of `lo_tile`.
 template <bool BF16>

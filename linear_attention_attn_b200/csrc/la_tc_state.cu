@@ -529,6 +529,10 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 // descriptor points its second atom there (a start 32 s bytes into a 128-byte
 // row, as a K step does for K-major operands).  bf16 bidir also keeps
 // lo = round(f(q) - hi): MMA1 adds f(Q)_lo S_hi and f'(q) = min(hi + lo, 1).
+// Warp roles of bwd_q: 0 TMA, 1 UMMA, 2..5 feature map, 6..9 dq, 10..13 epilogue.
+constexpr int kQXWarps = 4, kQDw0 = kXw0 + kQXWarps, kQDWarps = 4;
+static_assert(kQDw0 + kQDWarps == kEw0, "bwd_q warp roles");
+
 template <bool BIDIR, bool BF16>
 struct BwdQLayout {
     static constexpr bool QLO = BIDIR && BF16;
@@ -540,8 +544,10 @@ struct BwdQLayout {
     static constexpr int dqoff = qloff + (QLO ? NST * kTileBytes : 0);
     static constexpr int opoff = dqoff + OST * kTileBytes;
     static constexpr int stageoff = opoff + 2 * OPB;
-    static constexpr int zsoff = stageoff + kStateElems * 4;
-    static constexpr int redoff = zsoff + 64 * 4;
+    static constexpr int zsoff = stageoff + kStateElems * 4;        // [3][64] z of three heads
+    static constexpr int iscoff = zsoff + 3 * 64 * 4;                // [3] 1 / operand scale
+    static constexpr int rioff = iscoff + 16;                        // [2][128] (g.o, 1/n) per row
+    static constexpr int redoff = rioff + 2 * 128 * 8;
     static constexpr int baroff = redoff + 32;
     static constexpr int nbars = 4 * NST + 8;
     static constexpr int misc = baroff + nbars * 8;
@@ -596,13 +602,13 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&xf[s], kXWarps);
+            mbar_init(&xf[s], kQXWarps);
             mbar_init(&gnready[s], kEWarps);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], BIDIR ? 1 + kQDWarps : 1);   // MMA3, and the dq pass that reads f(q)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc12full[b], 1);
-            mbar_init(&acc12empty[b], kEWarps);
+            mbar_init(&acc12empty[b], BIDIR ? kEWarps + kQDWarps : kQDWarps);
         }
         mbar_init(accSfull, 1);
         mbar_init(accSfree, kEWarps);
@@ -741,25 +747,118 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             umma_commit(drain);
             mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
         }
-    } else if (warp < kEw0) {
+    } else if (warp < kQDw0) {
+        // Feature-map warps (bidir): f(q) in place, one row per thread.
         if (BIDIR) {
-            const int xi = threadIdx.x - kXw0 * 32;
+            const int r = threadIdx.x - kXw0 * 32;
             int s = 0;
             uint32_t ph = 0;
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
                 const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
                 if (!got) break;
-                if (QLO)
-                    phi_half_row_split<BF16>(sQ + s * kTileBytes, sQlo + s * kTileBytes, xi, false);
-                else
-                    phi_half_row<BF16>(sQ + s * kTileBytes, xi, false);
+                phi_row_batched<BF16, QLO>(sQ + s * kTileBytes, sQlo + s * kTileBytes, r);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&xf[s]);
                 if (++s == NST) { s = 0; ph ^= 1; }
             }
         }
+    } else if (warp < kEw0) {
+        // dq warps: dq = ((g S^T - (g.o) z) / n) f'(q) from TMEM (g S^T) and the
+        // epilogue warps' per-row (g.o, 1/n); warp w reads TMEM lane quadrant w % 4.
+        // Named barrier 3 (these 128 threads) is reached by all whatever the waits return.
+        const int sub = warp & 3;
+        const int row = sub * 32 + lane;
+        const bool storer = threadIdx.x == kQDw0 * 32;
+        const float2 *rinfo = reinterpret_cast<const float2 *>(smem + L::rioff);
+        const float *isc3 = reinterpret_cast<const float *>(smem + L::iscoff);
+        bool live = true;
+        int s = 0, b = 0, hidx = -1;
+        uint32_t ph = 0, bph = 0;
+        long long prev_h = -1;
+        for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+            if (t.h != prev_h) {
+                ++hidx;
+                prev_h = t.h;
+            }
+            const int zb = hidx % 3;
+            if (storer) tma_store_wait_read<L::OST - 1>();   // staging buffer x % OST is free
+            named_bar(3, kQDWarps * 32);
+            uint8_t *sDQx = sDQ + (int)(t.x & (L::OST - 1)) * kTileBytes;
+            bool got = live && LA_WAIT(&gnready[s], ph, 0x80u);
+            got = got && LA_WAIT(&acc12full[b], bph, 0x10u);
+            got = __all_sync(0xffffffffu, got);
+            live = live && got;
+            if (got) {
+                tc_fence_after();
+                float gdot = 0.f, inv = 1.f;
+                if (BIDIR) {
+                    const float2 ri = rinfo[b * 128 + row];
+                    gdot = ri.x;
+                    inv = ri.y;
+                }
+                const float *zsb = zs + zb * 64;
+                const float isc = isc3[zb];
+                const uint32_t d2 = tmem + (uint32_t)b * 256u + 96u + ((uint32_t)(32 * sub) << 16);
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float a0[16], a1[16];
+                    tmem_ld16(d2 + 32 * hf, a0);
+                    tmem_ld16(d2 + 32 * hf + 16, a1);
+                    tmem_ld_wait();
+                    if (hf == 1) {   // every TMEM read of this accumulator pair is complete
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&acc12empty[b]);
+                    }
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c16 = 2 * hf + cc;
+                        float dq[16];
+                        if (BIDIR) {
+                            float qf[16];
+                            load_chunk16<BF16>(sQ + s * kTileBytes, row, c16, qf);
+                            if (QLO) {
+                                float ql[16];
+                                load_chunk16<BF16>(sQlo + s * kTileBytes, row, c16, ql);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) qf[i] += ql[i];
+                            }
+                            const float4 *z4 = reinterpret_cast<const float4 *>(zsb + 16 * c16);
+#pragma unroll
+                            for (int i4 = 0; i4 < 4; ++i4) {
+                                const float4 zz = z4[i4];
+                                const float zv[4] = {zz.x, zz.y, zz.z, zz.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int i = 4 * i4 + e;
+                                    const float acc = cc ? a1[i] : a0[i];
+                                    dq[i] = (acc - gdot * zv[e]) * inv * fminf(qf[i], 1.f);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) dq[i] = (cc ? a1[i] : a0[i]) * isc;
+                        }
+                        store_chunk16<BF16>(sDQx, row, c16, dq);
+                    }
+                }
+                if (BIDIR) {   // f(q) of this stage is no longer read
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[s]);
+                }
+            }
+            fence_async_smem();
+            named_bar(3, kQDWarps * 32);
+            if (storer && live) {
+                tma_store_3d(&tmDQ, sDQx, 0, t.j * kRows, t.h);
+                tma_store_commit();
+            }
+            if (++s == NST) { s = 0; ph ^= 1; }
+            b ^= 1;
+            if (b == 0) bph ^= 1;
+        }
+        if (storer) tma_store_wait_all<0>();
     } else {
         // Epilogue warps (every named barrier is reached by all 128 whatever the waits return).
         const int tid = threadIdx.x - kEw0 * 32;
@@ -771,7 +870,8 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         bool live = true;
         float cur_sc = 1.f, cur_scn = 1.f;
 
-        auto build = [&](long long h) {
+        float *isc3 = reinterpret_cast<float *>(smem + L::iscoff);
+        auto build = [&](long long h, int zb) {
             const float *srch = src + h * (long long)src_per_head;
             const int ns = src_single ? 1 : (P.last_cta((int)h) - P.first_cta((int)h) + 1);
             float m = gather_state(srch, ns, stage, tid);
@@ -787,7 +887,8 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 scn = ldexpf(1.f, e - 1);
             }
             build_state_operand<BF16, NOPS, true>(stage, sc, 80, BIDIR, sOp, sOp + OPB, tid);
-            if (tid < 64) zs[tid] = stage[tid * 65 + 64] * sc;
+            if (tid < 64) zs[zb * 64 + tid] = stage[tid * 65 + 64] * sc;
+            if (tid == 0) isc3[zb] = 1.f / sc;
             fence_async_smem();
             named_bar(1, kWorkers);
             cur_sc = sc;
@@ -827,123 +928,62 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             }
         };
 
+        float2 *rinfo = reinterpret_cast<float2 *>(smem + L::rioff);
+        int hidx = -1;
         for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
+            const long long x = t.x;
             const long long h = t.h;
-            const int j = t.j;
             if (h != cur_h) {
-                build(h);
+                ++hidx;
+                build(h, hidx % 3);
                 cur_h = h;
             }
-            // ---- epilogue of tile x (stage s, accumulator pair b, dq staging buffer x % OST)
-            if (tid == 0) tma_store_wait_read<L::OST - 1>();
-            named_bar(1, kWorkers);
-            uint8_t *sDQx = sDQ + (int)(x & (L::OST - 1)) * kTileBytes;
+            // ---- first half of the epilogue of tile x (stage s, accumulator pair b):
+            //      n, g.o, g/n and w; the feature-map warps form dq from g S^T
             bool got = live && LA_WAIT(&acc12full[b], bph, 0x10u);
             got = __all_sync(0xffffffffu, got);
             live = live && got;
-            if (got) {
+            if (got && BIDIR) {
                 tc_fence_after();
-                const uint32_t lanes = (uint32_t)(32 * sub) << 16;
-                const uint32_t d1 = tmem + (uint32_t)b * 256u + lanes, d2 = d1 + 96u;
-                uint8_t *tq = sQ + s * kTileBytes, *tg = sG + s * kTileBytes;
-                float gdot = 0.f, inv = 1.f;
-                if (BIDIR) {
-                    // u = f(q) S and q.z (one wait for all five loads)
-                    float u[64], t16[16];
-                    tmem_ld16(d1 + 64, t16);
-                    tmem_row64(d1, u);
-                    inv = 1.f / (t16[0] + eps * cur_sc);
-                    const float gsc = inv * cur_sc * cur_scn;
-#pragma unroll
-                    for (int c16 = 0; c16 < 4; ++c16) {
-                        float g[16];
-                        load_chunk16<BF16>(tg, row, c16, g);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            gdot = fmaf(g[i], u[16 * c16 + i], gdot);
-                            g[i] *= gsc;
-                        }
-                        store_chunk16<BF16>(tg, row, c16, g);   // g/n (scaled) over dO: MMA2 is done with it
-                    }
-                    gdot *= inv;
-                    const float w = -gdot * gsc;
-                    // columns 16 s .. 16 s + 7 of the w tile: (w, 0, ..., 0)
-                    const uint32_t wbits = BF16 ? (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(w))
-                                                : (uint32_t)__half_as_ushort(__float2half_rn(w));
-                    *reinterpret_cast<uint4 *>(sW + sw128_offset(row, 16 * s)) = make_uint4(wbits, 0u, 0u, 0u);
-                }
-                const float isc = 1.f / cur_sc;
-                // g S^T in two halves of 32 columns (one wait each)
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float acc[32];
-                    {
-                        float a0[16], a1[16];
-                        tmem_ld16(d2 + 32 * hf, a0);
-                        tmem_ld16(d2 + 32 * hf + 16, a1);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            acc[i] = a0[i];
-                            acc[16 + i] = a1[i];
-                        }
-                    }
-                    if (hf == 1) {
-                        // every TMEM read of this accumulator pair is complete
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&acc12empty[b]);
-                    }
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        const int c16 = 2 * hf + cc;
-                        float dq[16];
-                        if (BIDIR) {
-                            float qf[16];
-                            load_chunk16<BF16>(tq, row, c16, qf);
-                            if (QLO) {
-                                float ql[16];
-                                load_chunk16<BF16>(sQlo + s * kTileBytes, row, c16, ql);
-#pragma unroll
-                                for (int i = 0; i < 16; ++i) qf[i] += ql[i];
-                            }
-                            const float4 *z4 = reinterpret_cast<const float4 *>(zs + 16 * c16);
-#pragma unroll
-                            for (int i4 = 0; i4 < 4; ++i4) {
-                                const float4 zz = z4[i4];
-                                const float zv[4] = {zz.x, zz.y, zz.z, zz.w};
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int i = 4 * i4 + e;
-                                    dq[i] = (acc[16 * cc + i] - gdot * zv[e]) * inv * fminf(qf[i], 1.f);
-                                }
-                            }
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) dq[i] = acc[16 * cc + i] * isc;
-                        }
-                        store_chunk16<BF16>(sDQx, row, c16, dq);
-                    }
-                }
-                fence_async_smem();
+                const uint32_t d1 = tmem + (uint32_t)b * 256u + ((uint32_t)(32 * sub) << 16);
+                float u[64], t16[16];   // u = f(q) S, t16[0] = f(q).z (one wait for all five loads)
+                tmem_ld16(d1 + 64, t16);
+                tmem_row64(d1, u);
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&gnready[s]);
-            } else {
+                if (lane == 0) mbar_arrive(&acc12empty[b]);
+                const float inv = 1.f / (t16[0] + eps * cur_sc);
+                const float gsc = inv * cur_sc * cur_scn;
+                uint8_t *tg = sG + s * kTileBytes;
+                float gdot = 0.f;
+#pragma unroll
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    float g[16];
+                    load_chunk16<BF16>(tg, row, c16, g);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        gdot = fmaf(g[i], u[16 * c16 + i], gdot);
+                        g[i] *= gsc;
+                    }
+                    store_chunk16<BF16>(tg, row, c16, g);   // g/n (scaled) over dO: MMA2 is done with it
+                }
+                gdot *= inv;
+                rinfo[b * 128 + row] = make_float2(gdot, inv);
+                const float w = -gdot * gsc;
+                // columns 16 s .. 16 s + 7 of the w tile: (w, 0, ..., 0)
+                const uint32_t wbits = BF16 ? (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(w))
+                                            : (uint32_t)__half_as_ushort(__float2half_rn(w));
+                *reinterpret_cast<uint4 *>(sW + sw128_offset(row, 16 * s)) = make_uint4(wbits, 0u, 0u, 0u);
                 fence_async_smem();
             }
-            named_bar(1, kWorkers);
-            if (tid == 0 && live) {
-                tma_store_3d(&tmDQ, sDQx, 0, j * kRows, (int)h);
-                tma_store_commit();
-            }
+            __syncwarp();
+            if (lane == 0 && got) mbar_arrive(&gnready[s]);
             const bool seg_end = (x + 1 == x1) || t.last_of_head();
             if (seg_end) read_accS((int)h, cur_scn);
             if (++s == NST) { s = 0; ph ^= 1; }
             b ^= 1;
             if (b == 0) bph ^= 1;
         }
-        if (tid == 0) tma_store_wait_all<0>();
     }
     tc_fence_before();
     __syncthreads();
