@@ -53,26 +53,27 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // abort_flag may be null: the wait then ignores aborts and ends only on
 // completion or on the time limit (used to drain copies and UMMAs in flight).
-// After a short spin the thread backs off with __nanosleep (32 ns doubling to
-// 512 ns), so warps that wait long do not take issue slots from the warps
-// that share their scheduler.
+// mbarrier.try_wait itself suspends the thread until the phase completes or a
+// hardware time limit passes, so the loop re-tries at once: a sleep between
+// tries would add its own length to the wait of a phase that completes during
+// it.  Only a wait that has lasted 20 us (a pipeline fill, a head change) backs
+// off with __nanosleep, to leave issue slots to the warps that share its
+// scheduler.
 static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                             unsigned int *fault_word, unsigned int code) {
-#pragma unroll 1
-    for (int i = 0; i < 8; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    unsigned int ns = 32;
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+        for (int i = 0; i < 16; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
         if (abort_flag && *abort_flag) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        const uint64_t dt = globaltimer_ns() - t0;
+        if (dt > kWaitLimitNs) {
             if (abort_flag) *abort_flag = 1;
             atomicOr(fault_word, code | 0x80000000u);
             return false;
         }
-        __nanosleep(ns);
-        if (ns < 512) ns <<= 1;
+        if (dt > 20000) __nanosleep(256);
     }
 }
 
