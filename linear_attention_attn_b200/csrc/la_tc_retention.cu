@@ -12,10 +12,14 @@
 //
 // One CTA per (b, h) walks the chunks in order.  Warp 0 streams q/k/v chunks
 // with TMA (two 64-column boxes per 64-row chunk, 128-byte swizzle); warp 1
-// issues the UMMAs; warps 2..9 form gamma^(C-1-j) k (hi + lo bf16); warps 10..13
-// apply the decay mask to P = Q K^T (hi + lo bf16), combine the two output
-// accumulators and carry the fp32 state S <- gamma^C S + dS, kept in shared
-// memory as a bf16 hi + lo pair that is also the B operand of Q S.
+// issues the UMMAs in the order P, dS, O_intra, O_inter, so that dS (which does
+// not depend on the state) and O_intra run while the state of the previous
+// chunk is being carried; warps 2..5 form gamma^(C-1-j) k and the masked
+// P~ = P o M (hi + lo bf16 each); warps 6..9 combine the two output
+// accumulators and store o; warps 10..13 carry the fp32 state
+// S <- gamma^C S + dS, kept in shared memory as a bf16 hi + lo pair that is
+// also the B operand of Q S.  The chain from one chunk to the next is only
+// O_inter (reads S_c) -> state update -> O_inter of the next chunk.
 //   P       M=64  N=64  K=128  A = Q (K-major)        B = K (K-major)
 //   O_intra M=64  N=128 K=64   A = P~ hi, lo (K-major) B = V (MN-major)
 //   O_inter M=64  N=128 K=128  A = Q (K-major)        B = S hi, lo (MN-major)
@@ -60,6 +64,10 @@ __device__ __forceinline__ void st16_wide(uint8_t *t, int box_bytes, int row, in
     store_chunk16<true>(t + (c16 >> 2) * box_bytes, row, c16 & 3, v);
 }
 
+// Warp roles: 0 TMA, 1 UMMA, 2..5 K^ and decay mask, 6..9 output, 10..13 state.
+constexpr int kRXw0 = 2, kRXWarps = 4, kROw0 = 6, kROWarps = 4, kRSw0 = 10, kRSWarps = 4;
+static_assert(kRSw0 + kRSWarps == kThreads / 32, "retention warp roles");
+
 struct RetLayout {
     static constexpr int NST = 2;
     static constexpr int qoff = 0;                              // [NST] q chunk (2 boxes)
@@ -71,7 +79,7 @@ struct RetLayout {
     static constexpr int ooff = soff + 2 * 2 * 16384;           // output staging chunk
     static constexpr int gpoff = ooff + kTile128;               // gamma^k, k = 0..128
     static constexpr int baroff = gpoff + 132 * 4;
-    static constexpr int nbars = 2 * NST + 9;
+    static constexpr int nbars = 2 * NST + 10;
     static constexpr int misc = baroff + nbars * 8;
     static constexpr int bytes = misc + 32 + 1024;
     static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
@@ -104,14 +112,16 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
     float *gpow = reinterpret_cast<float *>(smem + L::gpoff);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::baroff);
     uint64_t *empty = full + NST;
-    uint64_t *pfull = empty + NST;
-    uint64_t *ptready = pfull + 1;
-    uint64_t *khready = ptready + 1;
-    uint64_t *ofull = khready + 1;
-    uint64_t *oread = ofull + 1;
-    uint64_t *dsfull = oread + 1;
-    uint64_t *sready = dsfull + 1;
-    uint64_t *drain = sready + 1;
+    uint64_t *pfull = empty + NST;       // P = Q K^T in TMEM
+    uint64_t *ptready = pfull + 1;       // P read, P~ written (feature-map warps)
+    uint64_t *khready = ptready + 1;     // K^ written
+    uint64_t *dsfull = khready + 1;      // dS = K^^T V in TMEM
+    uint64_t *dsread = dsfull + 1;       // dS read (state warps)
+    uint64_t *sready = dsread + 1;       // state operand holds S_c (phase c)
+    uint64_t *sfree = sready + 1;        // Q S of the chunk done reading the state operand
+    uint64_t *ofull = sfree + 1;         // O_intra and O_inter in TMEM
+    uint64_t *oread = ofull + 1;         // ... read (output warps)
+    uint64_t *drain = oread + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc);
     int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
 
@@ -129,12 +139,14 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             mbar_init(&empty[s], 1);
         }
         mbar_init(pfull, 1);
-        mbar_init(ptready, kEWarps);
-        mbar_init(khready, kXWarps);
-        mbar_init(ofull, 1);
-        mbar_init(oread, kEWarps);
+        mbar_init(ptready, kRXWarps);
+        mbar_init(khready, kRXWarps);
         mbar_init(dsfull, 1);
-        mbar_init(sready, kEWarps);
+        mbar_init(dsread, kRSWarps);
+        mbar_init(sready, kRSWarps);
+        mbar_init(sfree, 1);
+        mbar_init(ofull, 1);
+        mbar_init(oread, kROWarps);
         mbar_init(drain, 1);
         *s_abort = 0;
         fence_mbar_init();
@@ -144,9 +156,9 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         const float l2g = log2f(gamma);
         gpow[threadIdx.x] = threadIdx.x == 0 ? 1.f : exp2f((float)threadIdx.x * l2g);
     }
-    if (warp >= kEw0) {
+    if (warp >= kRSw0) {
         // S_0 = 0: both halves of the state operand
-        const int r = threadIdx.x - kEw0 * 32;
+        const int r = threadIdx.x - kRSw0 * 32;
         for (int part = 0; part < 4; ++part) {
             uint8_t *p = sS + part * 16384 + r * 128;
 #pragma unroll
@@ -198,13 +210,15 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             }
         }
     } else if (warp == 1) {
+        // UMMA issue, per chunk: P, then dS (independent of the state), then
+        // O_intra, then Q S once the state warps have written S_c.
         if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
-            for (int c = 0; c < nchunks; ++c) {
-                const uint32_t pc = (uint32_t)(c & 1), pp = (uint32_t)((c - 1) & 1);
+            for (int it = 0; it < nchunks; ++it) {
+                const uint32_t pc = (uint32_t)(it & 1), pp = pc ^ 1u;
                 if (!LA_RWAIT(&full[s], ph, 0x4u)) break;
-                if (c > 0 && !LA_RWAIT(ptready, pp, 0x8u)) break;   // P accumulator read
+                if (it > 0 && !LA_RWAIT(ptready, pp, 0x8u)) break;   // P accumulator read
                 tc_fence_after();
                 const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTile128), 16, 1024);
                 const uint64_t dk = sdesc_sw128(smem_u32(sK + s * kTile128), 16, 1024);
@@ -216,31 +230,9 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                     umma_f16_ss(tmem + cP, desc_at(dq, off), desc_at(dk, off), ID_P, kk ? 1u : 0u);
                 }
                 umma_commit(pfull);
-                // O_intra = P~ V and O_inter = Q S
-                if (!LA_RWAIT(ptready, pc, 0x10u)) break;
-                if (c > 0 && !LA_RWAIT(sready, pp, 0x20u)) break;
-                if (c > 0 && !LA_RWAIT(oread, pp, 0x40u)) break;
-                tc_fence_after();
-                const uint64_t dpt = sdesc_sw128(smem_u32(sPt), 16, 1024);
-                const uint64_t ds = sdesc_sw128(smem_u32(sS), 16384, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-                    for (int op = 0; op < 2; ++op)
-                        umma_f16_ss(tmem + cOI, desc_at(dpt, op * kBox + kk * 32), desc_at(dv, kk * 2048), ID_OI,
-                                    (kk | op) ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-#pragma unroll
-                    for (int op = 0; op < 2; ++op)
-                        umma_f16_ss(tmem + cOX, desc_at(dq, off), desc_at(ds, op * 32768 + kk * 2048), ID_OI,
-                                    (kk | op) ? 1u : 0u);
-                }
-                umma_commit(ofull);
                 // dS = K^^T V
                 if (!LA_RWAIT(khready, pc, 0x80u)) break;
+                if (it > 0 && !LA_RWAIT(dsread, pp, 0x40u)) break;
                 tc_fence_after();
                 const uint64_t dkh = sdesc_sw128(smem_u32(sKh), kBox, 1024);
 #pragma unroll
@@ -251,28 +243,60 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                                     (kk | op) ? 1u : 0u);
                 }
                 umma_commit(dsfull);
+                // O_intra = P~ V
+                if (!LA_RWAIT(ptready, pc, 0x10u)) break;
+                if (it > 0 && !LA_RWAIT(oread, pp, 0x20u)) break;
+                tc_fence_after();
+                const uint64_t dpt = sdesc_sw128(smem_u32(sPt), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                    for (int op = 0; op < 2; ++op)
+                        umma_f16_ss(tmem + cOI, desc_at(dpt, op * kBox + kk * 32), desc_at(dv, kk * 2048), ID_OI,
+                                    (kk | op) ? 1u : 0u);
+                }
+                // O_inter = Q S_c
+                if (!LA_RWAIT(sready, pc, 0x1000u)) break;
+                tc_fence_after();
+                const uint64_t ds = sdesc_sw128(smem_u32(sS), 16384, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+#pragma unroll
+                    for (int op = 0; op < 2; ++op)
+                        umma_f16_ss(tmem + cOX, desc_at(dq, off), desc_at(ds, op * 32768 + kk * 2048), ID_OI,
+                                    (kk | op) ? 1u : 0u);
+                }
+                umma_commit(ofull);
+                umma_commit(sfree);
                 umma_commit(&empty[s]);
                 if (++s == NST) { s = 0; ph ^= 1; }
             }
             umma_commit(drain);
             mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_ret_fault, 0x400u);
         }
-    } else if (warp < kEw0) {
-        // K^ = diag(gamma^(C-1-j)) K as hi + lo; thread xi: row xi % 64, 8-element chunks 4*(xi/64) .. +3
-        const int xi = threadIdx.x - kXw0 * 32;
-        const int row = xi & 63, part = xi >> 6;
+    } else if (warp < kROw0) {
+        // Feature-map warps: K^ = diag(gamma^(C-1-j)) K as hi + lo (thread xt: row xt % 64,
+        // 8-element chunks 8 (xt / 64) .. + 7), then the decay mask P~ = P o M as hi + lo
+        // (warp w reads TMEM lane quadrant w % 4; lanes 0..15 hold chunk rows 16 (w % 4) + l).
+        const int xt = threadIdx.x - kRXw0 * 32;
+        const int krow = xt & 63, part = xt >> 6;
+        const int sub = warp & 3;
+        const uint32_t lanes = (uint32_t)(32 * sub) << 16;
+        const int ri = 16 * sub + lane;
         int s = 0;
         uint32_t ph = 0;
-        for (int c = 0; c < nchunks; ++c) {
+        for (int it = 0; it < nchunks; ++it) {
+            const uint32_t pc = (uint32_t)(it & 1);
             bool got = LA_RWAIT(&full[s], ph, 0x100u);
-            if (got && c > 0) got = LA_RWAIT(dsfull, (uint32_t)((c - 1) & 1), 0x200u);   // K^ buffer free
+            if (got && it > 0) got = LA_RWAIT(dsfull, pc ^ 1u, 0x200u);   // K^ buffer free
             got = __all_sync(0xffffffffu, got);
             if (!got) break;
-            const float f = rev ? gpow[row] : gpow[kC - 1 - row];
+            const float f = rev ? gpow[krow] : gpow[kC - 1 - krow];
 #pragma unroll
-            for (int it = 0; it < 4; ++it) {
-                const int ch = part * 4 + it;               // 0..15 across the two boxes
-                const int off = (ch >> 3) * kBox + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+            for (int i = 0; i < 8; ++i) {
+                const int ch = part * 8 + i;               // 0..15 across the two boxes
+                const int off = (ch >> 3) * kBox + krow * 128 + (((ch & 7) ^ (krow & 7)) << 4);
                 const uint4 u = *reinterpret_cast<const uint4 *>(sK + s * kTile128 + off);
                 const uint32_t w[4] = {u.x, u.y, u.z, u.w};
                 uint32_t hi[4], lo[4];
@@ -290,51 +314,49 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(khready);
+            // ---- P~ = (Q K^T) o M, hi + lo (P~ of the previous chunk: its O_intra
+            //      completed before this chunk's P, which pfull tracks)
+            got = __all_sync(0xffffffffu, LA_RWAIT(pfull, pc, 0x400u));
+            if (!got) break;
+            tc_fence_after();
+            float p[64];
+            tmem_row64(tmem + cP + lanes, p);
+            tc_fence_before();
+            if (lane < 16) {
+                float hi[64], lo[64];
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    const int dlt = rev ? j - ri : ri - j;     // causal: i >= j; backwards: j >= i
+                    p[j] = dlt >= 0 ? p[j] * gpow[dlt] : 0.f;
+                }
+                store_row<true>(sPt, ri, p);
+                load_row<true>(sPt, ri, hi);
+#pragma unroll
+                for (int j = 0; j < 64; ++j) lo[j] = p[j] - hi[j];
+                store_row<true>(sPt + kBox, ri, lo);
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ptready);
             if (++s == NST) { s = 0; ph ^= 1; }
         }
-    } else {
-        // Epilogue warps: decay mask, output, state.  Named barrier 1 (128 threads) is
+    } else if (warp < kRSw0) {
+        // Output warps: o = O_intra + diag(gamma^(i+1)) O_inter (backwards: gamma^(C-i)),
+        // staged and stored with TMA.  Named barrier 1 (these 128 threads) is
         // reached by all of them whatever the waits return.
-        const int tid = threadIdx.x - kEw0 * 32;
+        const int ot = threadIdx.x - kROw0 * 32;
         const int sub = warp & 3;
         const uint32_t lanes = (uint32_t)(32 * sub) << 16;
-        const int ri = 16 * sub + lane;           // M = 64 accumulators: chunk row of lanes 0..15
+        const int ri = 16 * sub + lane;
         bool live = true;
         for (int it = 0; it < nchunks; ++it) {
             const int c = rev ? nchunks - 1 - it : it;
             const uint32_t pc = (uint32_t)(it & 1);
-            // ---- P~ = (Q K^T) o M, hi + lo
-            bool got = live && LA_RWAIT(pfull, pc, 0x400u);
+            if (ot == 0) tma_store_wait_read<0>();
+            named_bar(1, kROWarps * 32);
+            bool got = live && LA_RWAIT(ofull, pc, 0x800u);
             got = __all_sync(0xffffffffu, got);
             live = live && got;
-            if (got) {
-                tc_fence_after();
-                float p[64];
-                tmem_row64(tmem + cP + lanes, p);
-                tc_fence_before();
-                if (lane < 16) {
-                    float hi[64], lo[64];
-#pragma unroll
-                    for (int j = 0; j < 64; ++j) {
-                        const int dlt = rev ? j - ri : ri - j;     // causal: i >= j; backwards: j >= i
-                        p[j] = dlt >= 0 ? p[j] * gpow[dlt] : 0.f;
-                    }
-                    store_row<true>(sPt, ri, p);
-                    load_row<true>(sPt, ri, hi);
-#pragma unroll
-                    for (int j = 0; j < 64; ++j) lo[j] = p[j] - hi[j];
-                    store_row<true>(sPt + kBox, ri, lo);
-                }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(ptready);
-            }
-            // ---- o = O_intra + diag(gamma^(i+1)) O_inter
-            got = live && LA_RWAIT(ofull, pc, 0x800u);
-            got = __all_sync(0xffffffffu, got);
-            live = live && got;
-            if (tid == 0) tma_store_wait_read<0>();
-            named_bar(1, kWorkers);
             if (got) {
                 tc_fence_after();
                 const float g1 = rev ? gpow[kC - ri] : gpow[ri + 1];
@@ -353,42 +375,52 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                 if (lane == 0) mbar_arrive(oread);
             }
             fence_async_smem();
-            named_bar(1, kWorkers);
-            if (tid == 0 && live) {
+            named_bar(1, kROWarps * 32);
+            if (ot == 0 && live) {
                 tma_store_3d(tmO, sO, 0, c * kC, bh);
                 tma_store_3d(tmO, sO + kBox, 64, c * kC, bh);
                 tma_store_commit();
             }
-            // ---- S <- gamma^C S + dS (row d = this thread's TMEM lane), as hi + lo
-            got = live && LA_RWAIT(dsfull, pc, 0x1000u);
-            got = __all_sync(0xffffffffu, got);
-            live = live && got;
-            if (got) {
-                tc_fence_after();
-                const int d = 32 * sub + lane;             // the TMEM lane (state row) this thread reads
-                const float gC = gpow[kC];
-#pragma unroll 2
-                for (int c16 = 0; c16 < 8; ++c16) {
-                    float ds[16], hi[16], lo[16];
-                    tmem_ld16(tmem + cDS + lanes + 16 * c16, ds);
-                    ld16_wide(sS, 16384, d, c16, hi);
-                    ld16_wide(sS + 32768, 16384, d, c16, lo);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) ds[i] = fmaf(gC, hi[i] + lo[i], ds[i]);
-                    st16_wide(sS, 16384, d, c16, ds);
-                    ld16_wide(sS, 16384, d, c16, hi);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) lo[i] = ds[i] - hi[i];
-                    st16_wide(sS + 32768, 16384, d, c16, lo);
-                }
-                tc_fence_before();
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(sready);
-            }
         }
-        if (tid == 0) tma_store_wait_all<0>();
+        if (ot == 0) tma_store_wait_all<0>();
+    } else {
+        // State warps: S_{c+1} = gamma^C S_c + dS_c; thread d holds state row d (its
+        // TMEM lane), kept in shared memory as the bf16 hi + lo operand of Q S.
+        const int sub = warp & 3;
+        const uint32_t lanes = (uint32_t)(32 * sub) << 16;
+        const int d = 32 * sub + lane;
+        const float gC = gpow[kC];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sready);                // S_0 (zeroed above)
+        for (int it = 0; it < nchunks; ++it) {
+            const uint32_t pc = (uint32_t)(it & 1);
+            bool got = LA_RWAIT(dsfull, pc, 0x1000u);
+            if (got) got = LA_RWAIT(sfree, pc, 0x2000u);   // Q S_c has read the operand
+            got = __all_sync(0xffffffffu, got);
+            if (!got) break;
+            tc_fence_after();
+#pragma unroll 2
+            for (int c16 = 0; c16 < 8; ++c16) {
+                float dsv[16], hi[16], lo[16];
+                tmem_ld16(tmem + cDS + lanes + 16 * c16, dsv);
+                ld16_wide(sS, 16384, d, c16, hi);
+                ld16_wide(sS + 32768, 16384, d, c16, lo);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) dsv[i] = fmaf(gC, hi[i] + lo[i], dsv[i]);
+                st16_wide(sS, 16384, d, c16, dsv);
+                ld16_wide(sS, 16384, d, c16, hi);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) lo[i] = dsv[i] - hi[i];
+                st16_wide(sS + 32768, 16384, d, c16, lo);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dsread);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sready);
+        }
     }
     tc_fence_before();
     __syncthreads();
