@@ -32,6 +32,18 @@ la_status cuda_fail(cudaError_t e, const char *what) {
     return LA_ERR_CUDA;
 }
 
+la_status launch_fail(cudaError_t e, const char *what, const void *kernel, dim3 block, size_t smem) {
+    cudaFuncAttributes fa;
+    memset(&fa, 0, sizeof fa);
+    cudaGetLastError();
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) cudaGetLastError();
+    set_error("%s: %s (%s); block %u threads, %zu B dynamic shared memory; kernel: %d registers, "
+              "%zu B local, %zu B static shared, at most %d threads",
+              what, cudaGetErrorString(e), cudaGetErrorName(e), block.x * block.y * block.z, smem, fa.numRegs,
+              (size_t)fa.localSizeBytes, (size_t)fa.sharedSizeBytes, fa.maxThreadsPerBlock);
+    return LA_ERR_CUDA;
+}
+
 static la_status fail(la_status s, const char *fmt, ...) {
     char buf[512];
     va_list ap;

@@ -13,6 +13,9 @@ namespace la {
 // ---------------------------------------------------------------- errors --
 void set_error(const char *fmt, ...);
 la_status cuda_fail(cudaError_t e, const char *what);
+// A failed launch: the error text also gives the kernel's registers, local memory
+// and thread limit next to the block and shared memory asked for.
+la_status launch_fail(cudaError_t e, const char *what, const void *kernel, dim3 block, size_t smem);
 
 // ------------------------------------------------------------- launching --
 // Every kernel goes through launch(): it counts launches and, when profiling
@@ -67,7 +70,7 @@ la_status launch_pdl(const char *name, Kernel kernel, dim3 grid, dim3 block, siz
     if (e == cudaSuccess) e = cudaGetLastError();
     prof_after(stream);
     count_launch();
-    if (e != cudaSuccess) return cuda_fail(e, name);
+    if (e != cudaSuccess) return launch_fail(e, name, reinterpret_cast<const void *>(kernel), block, smem);
     return LA_OK;
 }
 

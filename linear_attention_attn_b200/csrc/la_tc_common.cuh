@@ -361,6 +361,26 @@ __device__ __forceinline__ float operand_scale(float m) {
     return ldexpf(1.f, e);
 }
 
+// Two-term bf16 split of 16 fp32 values, packed in pairs: hi = round(x),
+// lo = round(x - hi) (x - hi is exact in fp32).
+__device__ __forceinline__ void split_hi_lo16_packed(const float (&x)[16], uint32_t (&hw)[8], uint32_t (&lw)[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        hw[k] = h2<true>::from_f2(x[2 * k], x[2 * k + 1]);
+        const float2 hv = h2<true>::to_f2(hw[k]);
+        lw[k] = h2<true>::from_f2(x[2 * k] - hv.x, x[2 * k + 1] - hv.y);
+    }
+}
+
+// store_chunk16 with the 16 values already packed in pairs.
+__device__ __forceinline__ void store_chunk16_packed(uint8_t *tile, int row, int c16, const uint32_t (&w)[8]) {
+    uint8_t *p = tile + row * 128;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+        *reinterpret_cast<uint4 *>(p + (((2 * c16 + h) ^ (row & 7)) << 4)) =
+            make_uint4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]);
+}
+
 // (head, tile-in-head) of the tile indices x0, x0 + 1, ... of a Partition, advanced
 // without a 64-bit division per tile (an emulated division costs hundreds of cycles).
 struct TileCursor {

@@ -55,18 +55,16 @@ __device__ __forceinline__ uint8_t *align1024r(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// 16 columns (16*c16 .. +15, c16 in 0..7) of row `row` of a 128-column tile stored
-// as boxes of 64 columns, `box_bytes` apart.
-__device__ __forceinline__ void ld16_wide(const uint8_t *t, int box_bytes, int row, int c16, float (&v)[16]) {
-    load_chunk16<true>(t + (c16 >> 2) * box_bytes, row, c16 & 3, v);
-}
+// Stores 16 columns (16*c16 .. +15, c16 in 0..7) of row `row` of a 128-column tile
+// kept as boxes of 64 columns, `box_bytes` apart.
 __device__ __forceinline__ void st16_wide(uint8_t *t, int box_bytes, int row, int c16, const float (&v)[16]) {
     store_chunk16<true>(t + (c16 >> 2) * box_bytes, row, c16 & 3, v);
 }
 
-// Warp roles: 0 TMA, 1 UMMA, 2..5 K^ and decay mask, 6..9 output, 10..13 state.
-constexpr int kRXw0 = 2, kRXWarps = 4, kROw0 = 6, kROWarps = 4, kRSw0 = 10, kRSWarps = 4;
-static_assert(kRSw0 + kRSWarps == kThreads / 32, "retention warp roles");
+// Warp roles: 0 TMA, 1 UMMA, 2..5 K^ and decay mask, 6..9 output, 10..17 state
+// (two warps per TMEM lane quadrant, 64 state columns each).
+constexpr int kRXw0 = 2, kRXWarps = 4, kROw0 = 6, kROWarps = 4, kRSw0 = 10, kRSWarps = 8;
+constexpr int kRThreads = (kRSw0 + kRSWarps) * 32;
 
 struct RetLayout {
     static constexpr int NST = 2;
@@ -93,7 +91,7 @@ struct RetJobs {
 };
 
 // Grid: one CTA per (pass, b, h), pass = blockIdx.x / BH.  decay[h] = gamma_h.
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kRThreads, 1)
 retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int H, int BH) {
     using L = RetLayout;
     constexpr int NST = L::NST;
@@ -157,13 +155,9 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         gpow[threadIdx.x] = threadIdx.x == 0 ? 1.f : exp2f((float)threadIdx.x * l2g);
     }
     if (warp >= kRSw0) {
-        // S_0 = 0: both halves of the state operand
-        const int r = threadIdx.x - kRSw0 * 32;
-        for (int part = 0; part < 4; ++part) {
-            uint8_t *p = sS + part * 16384 + r * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(p + c * 16) = make_uint4(0u, 0u, 0u, 0u);
-        }
+        // S_0 = 0: the state operand (hi and lo, 4 x 16 KB), 16 bytes per thread per step
+        for (int i = threadIdx.x - kRSw0 * 32; i < 4 * 16384 / 16; i += kRSWarps * 32)
+            reinterpret_cast<uint4 *>(sS)[i] = make_uint4(0u, 0u, 0u, 0u);
         fence_async_smem();
     }
     if (warp == 0 && lane == 0) {
@@ -210,26 +204,33 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             }
         }
     } else if (warp == 1) {
-        // UMMA issue, per chunk: P, then dS (independent of the state), then
-        // O_intra, then Q S once the state warps have written S_c.
+        // UMMA issue, per chunk c: dS (independent of the state), O_intra, P of
+        // chunk c + 1 (so that its decay mask overlaps the rest of chunk c), then
+        // Q S once the state warps have written S_c.
         if (lane == 0) {
-            int s = 0;
-            uint32_t ph = 0;
-            for (int it = 0; it < nchunks; ++it) {
-                const uint32_t pc = (uint32_t)(it & 1), pp = pc ^ 1u;
-                if (!LA_RWAIT(&full[s], ph, 0x4u)) break;
-                if (it > 0 && !LA_RWAIT(ptready, pp, 0x8u)) break;   // P accumulator read
-                tc_fence_after();
-                const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTile128), 16, 1024);
-                const uint64_t dk = sdesc_sw128(smem_u32(sK + s * kTile128), 16, 1024);
-                const uint64_t dv = sdesc_sw128(smem_u32(sV + s * kTile128), kBox, 1024);
-                // P = Q K^T
+            auto issue_p = [&](int sp) {
+                const uint64_t dq = sdesc_sw128(smem_u32(sQ + sp * kTile128), 16, 1024);
+                const uint64_t dk = sdesc_sw128(smem_u32(sK + sp * kTile128), 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
                     umma_f16_ss(tmem + cP, desc_at(dq, off), desc_at(dk, off), ID_P, kk ? 1u : 0u);
                 }
                 umma_commit(pfull);
+            };
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = nchunks > 0 && LA_RWAIT(&full[0], 0, 0x4u);
+            if (ok) {
+                tc_fence_after();
+                issue_p(0);
+            }
+            for (int it = 0; it < nchunks && ok; ++it) {
+                const uint32_t pc = (uint32_t)(it & 1), pp = pc ^ 1u;
+                const int sn = s + 1 == NST ? 0 : s + 1;
+                const uint32_t phn = s + 1 == NST ? ph ^ 1u : ph;
+                const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTile128), 16, 1024);
+                const uint64_t dv = sdesc_sw128(smem_u32(sV + s * kTile128), kBox, 1024);
                 // dS = K^^T V
                 if (!LA_RWAIT(khready, pc, 0x80u)) break;
                 if (it > 0 && !LA_RWAIT(dsread, pp, 0x40u)) break;
@@ -243,7 +244,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                                     (kk | op) ? 1u : 0u);
                 }
                 umma_commit(dsfull);
-                // O_intra = P~ V
+                // O_intra = P~ V (the mask has read P: its accumulator is free)
                 if (!LA_RWAIT(ptready, pc, 0x10u)) break;
                 if (it > 0 && !LA_RWAIT(oread, pp, 0x20u)) break;
                 tc_fence_after();
@@ -254,6 +255,12 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                     for (int op = 0; op < 2; ++op)
                         umma_f16_ss(tmem + cOI, desc_at(dpt, op * kBox + kk * 32), desc_at(dv, kk * 2048), ID_OI,
                                     (kk | op) ? 1u : 0u);
+                }
+                // P of the next chunk
+                if (it + 1 < nchunks) {
+                    if (!LA_RWAIT(&full[sn], phn, 0x4u)) break;
+                    tc_fence_after();
+                    issue_p(sn);
                 }
                 // O_inter = Q S_c
                 if (!LA_RWAIT(sready, pc, 0x1000u)) break;
@@ -270,7 +277,8 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                 umma_commit(ofull);
                 umma_commit(sfree);
                 umma_commit(&empty[s]);
-                if (++s == NST) { s = 0; ph ^= 1; }
+                s = sn;
+                ph = phn;
             }
             umma_commit(drain);
             mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_ret_fault, 0x400u);
@@ -319,22 +327,25 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             got = __all_sync(0xffffffffu, LA_RWAIT(pfull, pc, 0x400u));
             if (!got) break;
             tc_fence_after();
-            float p[64];
-            tmem_row64(tmem + cP + lanes, p);
-            tc_fence_before();
-            if (lane < 16) {
-                float hi[64], lo[64];
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    const int dlt = rev ? j - ri : ri - j;     // causal: i >= j; backwards: j >= i
-                    p[j] = dlt >= 0 ? p[j] * gpow[dlt] : 0.f;
+            for (int c16 = 0; c16 < 4; ++c16) {
+                float x[16];
+                tmem_ld16(tmem + cP + lanes + 16 * c16, x);
+                tmem_ld_wait();
+                if (lane < 16) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int j = 16 * c16 + e;
+                        const int dlt = rev ? j - ri : ri - j;     // causal: i >= j; backwards: j >= i
+                        x[e] = dlt >= 0 ? x[e] * gpow[dlt] : 0.f;
+                    }
+                    uint32_t hw[8], lw[8];
+                    split_hi_lo16_packed(x, hw, lw);
+                    store_chunk16_packed(sPt, ri, c16, hw);
+                    store_chunk16_packed(sPt + kBox, ri, c16, lw);
                 }
-                store_row<true>(sPt, ri, p);
-                load_row<true>(sPt, ri, hi);
-#pragma unroll
-                for (int j = 0; j < 64; ++j) lo[j] = p[j] - hi[j];
-                store_row<true>(sPt + kBox, ri, lo);
             }
+            tc_fence_before();
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(ptready);
@@ -384,39 +395,45 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         }
         if (ot == 0) tma_store_wait_all<0>();
     } else {
-        // State warps: S_{c+1} = gamma^C S_c + dS_c; thread d holds state row d (its
-        // TMEM lane), kept in shared memory as the bf16 hi + lo operand of Q S.
-        const int sub = warp & 3;
+        // State warps: S_{c+1} = gamma^C S_c + dS_c in fp32 registers; thread (d, half)
+        // holds columns 64 half .. 64 half + 63 of state row d (its TMEM lane) and
+        // writes them as the bf16 hi + lo operand of Q S.
+        const int sub = warp & 3, half = (warp - kRSw0) >> 2;
         const uint32_t lanes = (uint32_t)(32 * sub) << 16;
         const int d = 32 * sub + lane;
         const float gC = gpow[kC];
+        float st[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) st[i] = 0.f;
         __syncwarp();
         if (lane == 0) mbar_arrive(sready);                // S_0 (zeroed above)
         for (int it = 0; it < nchunks; ++it) {
             const uint32_t pc = (uint32_t)(it & 1);
-            bool got = LA_RWAIT(dsfull, pc, 0x1000u);
-            if (got) got = LA_RWAIT(sfree, pc, 0x2000u);   // Q S_c has read the operand
-            got = __all_sync(0xffffffffu, got);
+            bool got = __all_sync(0xffffffffu, LA_RWAIT(dsfull, pc, 0x1000u));
             if (!got) break;
             tc_fence_after();
-#pragma unroll 2
-            for (int c16 = 0; c16 < 8; ++c16) {
-                float dsv[16], hi[16], lo[16];
-                tmem_ld16(tmem + cDS + lanes + 16 * c16, dsv);
-                ld16_wide(sS, 16384, d, c16, hi);
-                ld16_wide(sS + 32768, 16384, d, c16, lo);
+            const uint32_t base = tmem + cDS + lanes + 64u * half;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                float a[16];
+                tmem_ld16(base + 16 * c4, a);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) dsv[i] = fmaf(gC, hi[i] + lo[i], dsv[i]);
-                st16_wide(sS, 16384, d, c16, dsv);
-                ld16_wide(sS, 16384, d, c16, hi);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) lo[i] = dsv[i] - hi[i];
-                st16_wide(sS + 32768, 16384, d, c16, lo);
+                for (int i = 0; i < 16; ++i) st[16 * c4 + i] = fmaf(gC, st[16 * c4 + i], a[i]);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(dsread);
+            got = __all_sync(0xffffffffu, LA_RWAIT(sfree, pc, 0x2000u));   // Q S_c has read the operand
+            if (!got) break;
+            // the 64 columns are columns 0..63 of box `half` (each box holds 64 state columns)
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t hw[8], lw[8];
+                split_hi_lo16_packed(*reinterpret_cast<const float(*)[16]>(&st[16 * c4]), hw, lw);
+                store_chunk16_packed(sS + half * 16384, d, c4, hw);
+                store_chunk16_packed(sS + 32768 + half * 16384, d, c4, lw);
+            }
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(sready);
@@ -448,7 +465,7 @@ la_status retention_fwd(const void *q, const void *k, const void *v, void *o, co
     LA_TRY(retention_map(&jobs.k[0], k, s));
     LA_TRY(retention_map(&jobs.v[0], v, s));
     LA_TRY(retention_map(&jobs.o[0], o, s));
-    return launch_pdl("tc_retention_fwd", retention_kernel, dim3((unsigned)s.BH()), dim3(kThreads),
+    return launch_pdl("tc_retention_fwd", retention_kernel, dim3((unsigned)s.BH()), dim3(kRThreads),
                   (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
 }
 
@@ -466,7 +483,7 @@ la_status retention_bwd(const void *q, const void *k, const void *v, const void 
         LA_TRY(retention_map(&jobs.o[p], out[p], s));
         jobs.rev[p] = p > 0;
     }
-    return launch_pdl("tc_retention_bwd", retention_kernel, dim3((unsigned)(3 * s.BH())), dim3(kThreads),
+    return launch_pdl("tc_retention_bwd", retention_kernel, dim3((unsigned)(3 * s.BH())), dim3(kRThreads),
                   (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
 }
 
