@@ -486,15 +486,160 @@ def run_ours(args, w):
     return 0
 
 
+# ---------------------------------------------------------------- decode --
+
+DECODE_SHAPE = (64, 32, 128)   # B, H, D: a serving batch whose fp32 state (134 MB) exceeds the 126 MB L2
+
+
+def run_decode_reference(args):
+    """The oracle's decode step on the host cores, on a bounded sample of the decode workload."""
+    import oracle
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    B, H, D = DECODE_SHAPE
+    nh = 64
+    gam = synth.retention_gammas(H)
+    qs, ks, vs = (synth.normal((B, H, D), 0, i).reshape(B * H, D)[:nh].double().numpy()[None] for i in range(3))
+    st = synth.normal((B, H, D, D), 0, 3).reshape(B * H, D, D)[:nh].double().numpy()[None] * D ** -0.5
+    gs = gam.double().numpy()[:1].repeat(nh)
+    for _ in range(args.warmup):
+        _, st = oracle.retention_step(qs, ks, vs, gs, st)
+    rates, secs = [], 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        _, st = oracle.retention_step(qs, ks, vs, gs, st)
+        dt_s = time.perf_counter() - t0
+        secs += dt_s
+        rates.append(nh / H / dt_s)
+    value = statistics.median(rates)
+    sample = "%d of %d (b,h) heads per step, fp64, one thread" % (nh, B * H)
+    print(json.dumps({
+        "impl": "reference", "metric": "retention decode tokens/s", "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "recurrent decode step of the decay op, B=%d H=%d D=%d" % (B, H, D)},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+    return 0
+
+
+def run_decode(args):
+    """Recurrent decode steps of the decay op: every step reads and writes the fp32 state of all
+    B*H heads once (S <- gamma S + k^T v, o = q S), B new tokens per step."""
+    import linear_attention_attn_b200 as la
+    rank, world, local = dist_env()
+    dist = init_dist(world, local)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    B, H, D = DECODE_SHAPE
+    dt = torch.bfloat16
+    pool = 8                                   # distinct token inputs cycled through the steps
+    gam = synth.retention_gammas(H)
+    hq = [synth.normal((B, H, D), rank * 100 + i, 0).mul(D ** -0.5).to(dt) for i in range(pool)]
+    hk = [synth.normal((B, H, D), rank * 100 + i, 1).to(dt) for i in range(pool)]
+    hv = [synth.normal((B, H, D), rank * 100 + i, 2).to(dt) for i in range(pool)]
+    q, k, v = ([t.to(dev) for t in x] for x in (hq, hk, hv))
+    o = torch.empty((B, H, D), dtype=dt, device=dev)
+    state = (synth.normal((B, H, D, D), rank, 3) * (D ** -0.5)).to(dev)
+
+    def step(i):
+        la.la_chunk_decay_step(q[i % pool], k[i % pool], v[i % pool], o, state, gam)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    sampler = ClockSampler(gpu_selector(dev))
+    sampler.start()
+    launches0 = la.la_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = la.la_launch_count() - launches0
+    if dist is not None:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    value = aggregate_throughput(B * args.steps, world, ms / 1e3)
+
+    # end to end: this step's q, k, v from pinned host memory, o back to the host; the state stays on the GPU
+    pq, pk, pv = (x[0].pin_memory() for x in (hq, hk, hv))
+    po = torch.empty((B, H, D), dtype=dt).pin_memory()
+    k_e2e = max(3, min(args.steps, 50))
+    for it in range(2 + k_e2e):
+        if it == 2:
+            torch.cuda.synchronize(dev)
+            x0 = torch.cuda.Event(enable_timing=True)
+            x0.record(stream)
+        q[0].copy_(pq, non_blocking=True)
+        k[0].copy_(pk, non_blocking=True)
+        v[0].copy_(pv, non_blocking=True)
+        step(0)
+        po.copy_(o, non_blocking=True)
+    x1 = torch.cuda.Event(enable_timing=True)
+    x1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1), dist, dev)
+    tok_bytes = B * H * D * 2
+    e2e = {"value": aggregate_throughput(B * k_e2e, world, e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": 3 * tok_bytes, "d2h_bytes_per_step": tok_bytes, "steps": k_e2e,
+           "note": "pinned host q, k, v copied in and o copied out every step; the fp32 state stays on the GPU"}
+
+    step_bytes = B * H * (2 * D * D * 4 + 4 * D * 2)
+    peak, peak_kind = measured_peaks()
+    achieved = step_bytes / (ms / args.steps / 1e3) / 1e9
+    roof = {"bound": "hbm", "kernel": "decay_step", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_source": peak_kind, "traffic": None,
+            "algorithmic_bytes_per_launch": step_bytes, "avg_launch_ms": ms / args.steps}
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        nh = 64                                  # a bounded sample: 64 of the B*H heads, 20 steps
+        qs, ks, vs = (x[0].reshape(B * H, D)[:nh].double().numpy()[None] for x in (hq, hk, hv))
+        st = state.reshape(B * H, D, D)[:nh].double().cpu().numpy()[None]
+        gs = gam.double().numpy()[:1].repeat(nh)
+        t0 = time.perf_counter()
+        for _ in range(20):
+            _, st = oracle.retention_step(qs, ks, vs, gs, st)
+        dt_s = time.perf_counter() - t0
+        cpu = {"value": 20 * nh / H / dt_s, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": "%d of %d (b,h) heads x 20 steps, fp64, one thread" % (nh, B * H), "seconds": dt_s}
+    line = {
+        "metric": "retention decode tokens/s", "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "recurrent decode step of the decay op (S <- gamma S + k^T v, o = q S), bf16 q/k/v/o, "
+                               "fp32 state, B=%d H=%d D=%d, gamma_h = 1 - 2^(-5-7h/(H-1))" % (B, H, D),
+                   "B": B, "H": H, "D": D, "global_batch": B * max(1, world),
+                   "parallelism": "dp%d (independent batches, no collective)" % max(1, world),
+                   "l2": "state of %.0f MB per step vs 126 MB L2, no flush" % (B * H * D * D * 4 / 1e6)},
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--T", type=int, default=None, help="sequence length (default: the workload's)")
-    ap.add_argument("--workload", choices=["bidir", "simple", "retention"], default="bidir",
-                    help="bidir (the benchmark metric, B8 H16 D64 fp16), simple (B8 H16 D64 bf16) or "
-                         "retention (B8 H32 D128 bf16)")
+    ap.add_argument("--workload", choices=["bidir", "simple", "retention", "decode"], default="bidir",
+                    help="bidir (the benchmark metric, B8 H16 D64 fp16), simple (B8 H16 D64 bf16), "
+                         "retention (B8 H32 D128 bf16) or decode (recurrent decay step, B64 H32 D128)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", dest="sweep", action="store_false",
@@ -505,6 +650,10 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload == "decode":
+        if args.impl == "reference":
+            return run_decode_reference(args)
+        return run_decode(args)
     base = {"bidir": "bidir_f16", "simple": "simple_bf16", "retention": "retention_bf16"}[args.workload]
     w = synth.WORKLOADS[base]
     w = w.with_T(args.T if args.T is not None else (4096 if args.workload != "retention" else 8192))

@@ -155,6 +155,21 @@ la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const 
                              int B, int H, int T, int D, la_dtype dtype,
                              void *workspace, size_t workspace_bytes, void *stream);
 
+/* One recurrent step of retention (decode): for every (b, h), with the state
+ * S = sum_{s<=t-1} gamma^(t-1-s) k_s^T v_s of the tokens seen so far,
+ *      S <- gamma_h S + k^T v,     o = q S
+ * i.e. S[i][j] <- gamma S[i][j] + k[i] v[j] and o[j] = sum_i q[i] S[i][j].
+ * Source: "flash-linear-attention" README, "Different forms of linear
+ * attention" (FusedRecurrent: the recurrent form, one token at a time).  The
+ * library's addition for serving after a chunked prefill; T is 1.
+ *  q, k, v  in  [B,H,D] device tensors of `dtype` (16-byte aligned)
+ *  o        out [B,H,D] of `dtype`
+ *  state    in/out [B,H,D,D] fp32 device array (16-byte aligned), updated in place
+ *  decay    HOST pointer to H floats in (0, 1], read during the call
+ * D must be 64 or 128.  No workspace.  Errors as for the other entry points. */
+la_status la_chunk_decay_step(const void *q, const void *k, const void *v, void *o, float *state,
+                              const float *decay, int B, int H, int D, la_dtype dtype, void *stream);
+
 /* Reports, and clears, the fault word of this library's tensor-core kernels on
  * the current device.  Every wait inside those kernels is bounded (2 s); a wait
  * that runs out makes the kernel wind down early (its outputs are then invalid)

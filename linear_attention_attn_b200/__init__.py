@@ -50,8 +50,9 @@ _lib.la_bidir_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I
 _lib.la_simple_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_chunk_decay_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_chunk_decay_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
+_lib.la_chunk_decay_step.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]
 for _n in ("la_bidir_fwd", "la_simple_fwd", "la_bidir_bwd", "la_simple_bwd", "la_chunk_decay_fwd",
-           "la_chunk_decay_bwd"):
+           "la_chunk_decay_bwd", "la_chunk_decay_step"):
     getattr(_lib, _n).restype = _I
 _lib.la_bidir_fwd_static.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.la_bidir_fwd_static.restype = _I
@@ -229,6 +230,26 @@ def la_chunk_decay_bwd(q, k, v, dout, decay, dq, dk, dv, workspace=None, stream=
     _check(_lib.la_chunk_decay_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), ctypes.cast(dec, _P), _ptr(dq),
                                    _ptr(dk), _ptr(dv), B, H, T, D, dt, wp, wn, _stream(stream, q.device)),
            "la_chunk_decay_bwd")
+
+
+def la_chunk_decay_step(q, k, v, o, state, decay, stream=None):
+    """One decode step: state <- decay[h] state + k^T v, o <- q state.  q, k, v, o are [B, H, D]
+    tensors of one dtype; state is a float32 [B, H, D, D] tensor updated in place."""
+    import torch
+    if q.dim() != 3:
+        raise ValueError("expected [B, H, D] tensors, got %r" % (tuple(q.shape),))
+    for t in (k, v, o):
+        if tuple(t.shape) != tuple(q.shape) or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("q, k, v, o must share shape, dtype and device")
+    for t in (q, k, v, o, state):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    B, H, D = (int(x) for x in q.shape)
+    if tuple(state.shape) != (B, H, D, D) or state.dtype != torch.float32 or state.device != q.device:
+        raise ValueError("state must be a float32 [B, H, D, D] tensor on the inputs' device")
+    dec = _decay(decay, H)
+    _check(_lib.la_chunk_decay_step(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), ctypes.cast(dec, _P), B, H, D,
+                                    _dtype_code(q), _stream(stream, q.device)), "la_chunk_decay_step")
 
 
 def la_status_string(status: int) -> str:

@@ -302,6 +302,20 @@ la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const 
     return simt::decay_bwd(q, k, v, dout, dec, dq, dk, dv, s, dtype, st);
 }
 
+la_status la_chunk_decay_step(const void *q, const void *k, const void *v, void *o, float *state,
+                              const float *decay, int B, int H, int D, la_dtype dtype, void *stream) {
+    const Shape s{B, H, 1, D};
+    LA_TRY(validate(s, dtype));
+    LA_TRY(check_ptr(q, "q"));
+    LA_TRY(check_ptr(k, "k"));
+    LA_TRY(check_ptr(v, "v"));
+    LA_TRY(check_ptr(o, "o"));
+    LA_TRY(check_ptr(state, "state"));
+    DecayArgs dec;
+    LA_TRY(decay_args(decay, H, &dec));
+    return decay_step(q, k, v, o, state, dec, B, H, D, dtype, (cudaStream_t)stream);
+}
+
 const char *la_status_string(la_status status) {
     switch (status) {
     case LA_OK: return "LA_OK";

@@ -112,6 +112,11 @@ int state_splits(const Shape &s, int rows_per_unit);
 // Bytes of one [BH, D, D+1] fp32 state block, rounded up to 256.
 size_t state_bytes(const Shape &s, long long copies);
 
+// One recurrent (decode) step of the decay op: S <- gamma S + k^T v, o = q S,
+// with q, k, v, o [B,H,D] and the fp32 state [B,H,D,D] updated in place.
+la_status decay_step(const void *q, const void *k, const void *v, void *o, float *state, const DecayArgs &dec, int B,
+                     int H, int D, la_dtype dt, cudaStream_t st);
+
 // ------------------------------------------------------------ SIMT path --
 // Plain CUDA-core kernels (fp32 FMA).  They implement every op for every
 // dtype; the fp16/bf16 ops at D in {64,128} normally run on the tensor-core

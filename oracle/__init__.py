@@ -59,8 +59,10 @@ def _bind(lib):
     lib.oracle_simple_bwd.argtypes = [P, P, P, P, P, P, P, L, L, L, L, I]
     lib.oracle_retention_fwd.argtypes = [P, P, P, P, P, L, L, L, L, I]
     lib.oracle_retention_bwd.argtypes = [P, P, P, P, P, P, P, P, L, L, L, L, I]
+    lib.oracle_retention_step.argtypes = [P, P, P, P, P, P, L, L, L]
     for name in ("oracle_bidir_fwd", "oracle_simple_fwd", "oracle_bidir_bwd",
-                 "oracle_simple_bwd", "oracle_retention_fwd", "oracle_retention_bwd"):
+                 "oracle_simple_bwd", "oracle_retention_fwd", "oracle_retention_bwd",
+                 "oracle_retention_step"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -175,6 +177,24 @@ class Oracle:
         _check(rc, "oracle_retention_bwd")
         return dq, dk, dv
 
+    def retention_step(self, q, k, v, gamma, state):
+        """One decode step: returns (o, new_state) with new_state = gamma_h state + k^T v and
+        o = q new_state; q, k, v are [B, H, D], state is [B, H, D, D] (not modified)."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        if q.ndim != 3:
+            raise ValueError("expected [B, H, D] arrays")
+        B, H, D = q.shape
+        S = np.array(_f64(state), dtype=np.float64, copy=True, order="C")
+        if S.shape != (B, H, D, D):
+            raise ValueError("state must be [B, H, D, D]")
+        gm = _f64(gamma).reshape(-1)
+        if gm.shape[0] != H:
+            raise ValueError("gamma must have H=%d entries" % H)
+        o = np.empty_like(q)
+        rc = self._lib.oracle_retention_step(_p(q), _p(k), _p(v), _p(gm), _p(S), _p(o), B, H, D)
+        _check(rc, "oracle_retention_step")
+        return o, S
+
 
 _inst = None
 
@@ -213,3 +233,7 @@ def retention_fwd(*a, **kw):
 
 def retention_bwd(*a, **kw):
     return _instance().retention_bwd(*a, **kw)
+
+
+def retention_step(*a, **kw):
+    return _instance().retention_step(*a, **kw)

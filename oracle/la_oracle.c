@@ -344,6 +344,30 @@ int oracle_retention_fwd(const double *q, const double *k, const double *v, cons
     return for_each_head(&jb, retention_fwd_head, (size_t)(D * D), nthreads);
 }
 
+/* One recurrent step of retention (decode), every head (the FusedRecurrent
+ * update applied to a single token):
+ *   S <- gamma_h S + k^T v,    o = q S
+ * q, k, v, o are [B, H, D]; S is [B, H, D, D] (row i = key index i, column j =
+ * value index j) and is updated in place. */
+int oracle_retention_step(const double *q, const double *k, const double *v, const double *gamma,
+                          double *S, double *o, long B, long H, long D) {
+    if (B < 1 || H < 1 || D < 1 || !q || !k || !v || !gamma || !S || !o) return -1;
+    for (long bh = 0; bh < B * H; ++bh) {
+        const double g = gamma[bh % H];
+        const double *qh = q + bh * D, *kh = k + bh * D, *vh = v + bh * D;
+        double *Sh = S + bh * D * D, *oh = o + bh * D;
+        for (long i = 0; i < D; ++i)
+            for (long j = 0; j < D; ++j)
+                Sh[i * D + j] = g * Sh[i * D + j] + kh[i] * vh[j];
+        for (long j = 0; j < D; ++j) {
+            double a = 0.0;
+            for (long i = 0; i < D; ++i) a += qh[i] * Sh[i * D + j];
+            oh[j] = a;
+        }
+    }
+    return 0;
+}
+
 int oracle_retention_bwd(const double *q, const double *k, const double *v, const double *dout,
                          const double *gamma, double *dq, double *dk, double *dv,
                          long B, long H, long T, long D, int nthreads) {

@@ -16,7 +16,8 @@ The facts used:
   * invariances: permutation of tokens, linearity in V, per-head independence,
     thread-count independence;
   * gradients: central finite differences of the oracle's forward, and torch
-    autograd through an independently written pairwise form in float64.
+    autograd through an independently written pairwise form in float64;
+  * the decode step: T steps from a zero state against the pairwise causal form.
 """
 from __future__ import annotations
 
@@ -72,6 +73,13 @@ def _parse(x):
 def check_golden(orc):
     cases = json.load(open(GOLDEN))["cases"]
     for c in cases:
+        if c["op"] == "retention_step":
+            q, k, v = (np.asarray(_parse(c[n]), dtype=np.float64)[None, None] for n in ("q", "k", "v"))
+            st = np.asarray(_parse(c["state"]), dtype=np.float64)[None, None]
+            o, st2 = orc.retention_step(q, k, v, np.array([c["gamma"]]), st)
+            _close(o[0, 0], _parse(c["o"]), what=c["name"] + " o")
+            _close(st2[0, 0], _parse(c["state_out"]), what=c["name"] + " state")
+            continue
         q, k, v = (_as4(_parse(c[n])) for n in ("q", "k", "v"))
         if c["op"] == "bidir":
             o = orc.bidir_fwd(q, k, v, eps=c["eps"])
@@ -298,5 +306,29 @@ def check_autograd(orc):
             _close(a, b.numpy(), rtol=1e-10, atol=1e-11, what="%s %s vs autograd" % (op, n))
 
 
+# ------------------------------------------------------------- decode step --
+
+def check_decode_step(orc):
+    """T recurrent steps from a zero state give the pairwise causal outputs, and leave the
+    state sum_s gamma^(T-1-s) k_s^T v_s; a step from a nonzero state continues a prefix."""
+    B, H, T, D = 2, 3, 9, 5
+    q, k, v = _rand((B, H, T, D), 41), _rand((B, H, T, D), 42), _rand((B, H, T, D), 43)
+    gam = np.array([0.5, 0.9, 1.0])
+    want = brute_retention(q, k, v, gam)
+    st = np.zeros((B, H, D, D))
+    for t in range(T):
+        o, st = orc.retention_step(q[:, :, t], k[:, :, t], v[:, :, t], gam, st)
+        _close(o, want[:, :, t], rtol=1e-11, atol=1e-12, what="step %d vs pairwise" % t)
+    w = gam[None, :, None] ** (T - 1 - np.arange(T))[None, None, :]
+    _close(st, np.einsum("bhs,bhsi,bhsj->bhij", w, k, v), rtol=1e-12, atol=1e-12, what="state after T steps")
+    # a prefix of T - 3 tokens as the state, then the last 3 tokens one by one
+    p = T - 3
+    wp = gam[None, :, None] ** (p - 1 - np.arange(p))[None, None, :]
+    st = np.einsum("bhs,bhsi,bhsj->bhij", wp, k[:, :, :p], v[:, :, :p])
+    for t in range(p, T):
+        o, st = orc.retention_step(q[:, :, t], k[:, :, t], v[:, :, t], gam, st)
+        _close(o, want[:, :, t], rtol=1e-11, atol=1e-12, what="step %d after a prefix state" % t)
+
+
 ALL_CHECKS = (check_golden, check_brute, check_closed_forms, check_invariances,
-              check_fd_gradients, check_autograd)
+              check_fd_gradients, check_autograd, check_decode_step)

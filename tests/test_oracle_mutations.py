@@ -35,6 +35,11 @@ MUTATIONS = [
     ("ret_fwd_gamma_head_index", "const double gamma = jb->gamma[bh % jb->H];", "const double gamma = jb->gamma[0];", 0),
     ("ret_bwd_gamma_head_index", "const double gamma = jb->gamma[bh % jb->H];", "const double gamma = jb->gamma[0];", 1),
     ("head_offset_dropped", "const long off = bh * T * D;", "const long off = 0;", 0),
+    ("step_no_decay", "Sh[i * D + j] = g * Sh[i * D + j] + kh[i] * vh[j];",
+     "Sh[i * D + j] = Sh[i * D + j] + kh[i] * vh[j];", 0),
+    ("step_output_transposed", "a += qh[i] * Sh[i * D + j];", "a += qh[i] * Sh[j * D + i];", 0),
+    ("step_outer_product_transposed", "+ kh[i] * vh[j];", "+ kh[j] * vh[i];", 0),
+    ("step_gamma_head_index", "const double g = gamma[bh % H];", "const double g = gamma[0];", 0),
 ]
 
 
