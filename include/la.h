@@ -70,8 +70,16 @@ typedef enum {
     LA_OP_SIMPLE_FWD = 2,
     LA_OP_SIMPLE_BWD = 3,
     LA_OP_CHUNK_DECAY_FWD = 4,
-    LA_OP_CHUNK_DECAY_BWD = 5
+    LA_OP_CHUNK_DECAY_BWD = 5,
+    LA_OP_STATE_REDUCE = 6,
+    LA_OP_STATE_APPLY = 7,
+    LA_OP_STATE_BWD_Q = 8,
+    LA_OP_STATE_BWD_KV = 9
 } la_op;
+
+/* Feature map of the sequence-parallel stages: elu+1 with the norm term (the
+ * la_bidir_* op) or the identity without it (the la_simple_* op). */
+typedef enum { LA_FEATURE_IDENTITY = 0, LA_FEATURE_ELU1 = 1 } la_feature;
 
 /* Largest H accepted by la_chunk_decay_* (the decays travel as kernel arguments). */
 #define LA_MAX_DECAY_HEADS 512
@@ -154,6 +162,47 @@ la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const 
                              const float *decay, void *dq, void *dk, void *dv,
                              int B, int H, int T, int D, la_dtype dtype,
                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---- the state form in stages, for a sequence split along T -------------
+ * A sequence cut into shards along T (one per rank or per call) gives each
+ * shard's partial state; their sum over the shards is the state of the whole
+ * sequence, so the op runs as: la_state_reduce on every shard, a sum of the
+ * states over the shards (an all-reduce: the caller's collective), la_state_apply
+ * on every shard.  The backward likewise: la_state_bwd_q on every shard with
+ * the whole sequence's state, a sum of the shards' [dS | dz], la_state_bwd_kv
+ * on every shard.  With one shard the stages compute exactly la_bidir_* /
+ * la_simple_* (feature = LA_FEATURE_ELU1 / LA_FEATURE_IDENTITY).  The library's
+ * addition: the pages only motivate long sequences ("Flash Bi-directional
+ * Linear Attention" README: intro), the split is the state form's own.
+ * Shapes, dtypes and alignment as for la_bidir_fwd; T is the shard's length
+ * (0 allowed: a reduce then writes zeros).  States are [B,H,D,D+1] fp32 device
+ * arrays as in la_bidir_fwd (column D holds z, 0 for LA_FEATURE_IDENTITY).
+ * Workspace: la_workspace_size(LA_OP_STATE_REDUCE / LA_OP_STATE_BWD_Q, ...);
+ * the apply and bwd_kv stages take none. */
+
+/* state <- [S | z] of the shard: S = sum_s f(k_s)^T v_s, z = sum_s f(k_s). */
+la_status la_state_reduce(const void *k, const void *v, float *state, int B, int H, int T, int D,
+                          la_dtype dtype, la_feature feature, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
+/* o <- f(q_t) S / (f(q_t) . z + eps) (elu+1), or q_t S (identity), with the
+ * whole sequence's state. */
+la_status la_state_apply(const void *q, const float *state, void *o, int B, int H, int T, int D,
+                         la_dtype dtype, la_feature feature, float eps, void *stream);
+
+/* dq of the shard and its [dS | dz] (dstate, out), from the whole sequence's
+ * state: with n_t = f(q_t).z + eps and o_t = f(q_t) S / n_t,
+ *   dq_t = ((dout_t S^T - (dout_t . o_t) z) / n_t) * f'(q_t),
+ *   dS = sum_t f(q_t)^T dout_t / n_t,   dz = -sum_t f(q_t) (dout_t . o_t) / n_t
+ * (identity: dq_t = dout_t S^T, dS = sum_t q_t^T dout_t, dz = 0). */
+la_status la_state_bwd_q(const void *q, const void *dout, const float *state, void *dq, float *dstate,
+                         int B, int H, int T, int D, la_dtype dtype, la_feature feature, float eps,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/* dk, dv of the shard from the whole sequence's [dS | dz]:
+ *   dk_s = (v_s dS^T + dz) * f'(k_s),   dv_s = f(k_s) dS. */
+la_status la_state_bwd_kv(const void *k, const void *v, const float *dstate, void *dk, void *dv,
+                          int B, int H, int T, int D, la_dtype dtype, la_feature feature, void *stream);
 
 /* One recurrent step of retention (decode): for every (b, h), with the state
  * S = sum_{s<=t-1} gamma^(t-1-s) k_s^T v_s of the tokens seen so far,

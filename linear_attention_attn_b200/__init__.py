@@ -27,7 +27,9 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 LA_F32, LA_F16, LA_BF16 = 0, 1, 2
 OPS = {"bidir_fwd": 0, "bidir_bwd": 1, "simple_fwd": 2, "simple_bwd": 3,
-       "chunk_decay_fwd": 4, "chunk_decay_bwd": 5}
+       "chunk_decay_fwd": 4, "chunk_decay_bwd": 5, "state_reduce": 6, "state_apply": 7,
+       "state_bwd_q": 8, "state_bwd_kv": 9}
+FEATURES = {"identity": 0, "elu1": 1}
 STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_ALIGNMENT",
           4: "LA_ERR_WORKSPACE", 5: "LA_ERR_CUDA", 6: "LA_ERR_TIMEOUT"}
 MAX_DECAY_HEADS = 512
@@ -51,8 +53,13 @@ _lib.la_simple_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _
 _lib.la_chunk_decay_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_chunk_decay_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_chunk_decay_step.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]
+_lib.la_state_reduce.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P]
+_lib.la_state_apply.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
+_lib.la_state_bwd_q.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
+_lib.la_state_bwd_kv.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]
 for _n in ("la_bidir_fwd", "la_simple_fwd", "la_bidir_bwd", "la_simple_bwd", "la_chunk_decay_fwd",
-           "la_chunk_decay_bwd", "la_chunk_decay_step"):
+           "la_chunk_decay_bwd", "la_chunk_decay_step", "la_state_reduce", "la_state_apply", "la_state_bwd_q",
+           "la_state_bwd_kv"):
     getattr(_lib, _n).restype = _I
 _lib.la_bidir_fwd_static.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.la_bidir_fwd_static.restype = _I
@@ -250,6 +257,58 @@ def la_chunk_decay_step(q, k, v, o, state, decay, stream=None):
     dec = _decay(decay, H)
     _check(_lib.la_chunk_decay_step(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state), ctypes.cast(dec, _P), B, H, D,
                                     _dtype_code(q), _stream(stream, q.device)), "la_chunk_decay_step")
+
+
+def _feature(feature):
+    if isinstance(feature, str):
+        if feature not in FEATURES:
+            raise ValueError("feature must be one of %s" % sorted(FEATURES))
+        return FEATURES[feature]
+    return int(feature)
+
+
+def _full_state_check(state, B, H, D, dev, name="state"):
+    import torch
+    if (state is None or tuple(state.shape) != (B, H, D, D + 1) or state.dtype != torch.float32
+            or not state.is_cuda or not state.is_contiguous() or state.device != dev):
+        raise ValueError("%s must be a contiguous float32 CUDA tensor [B, H, D, D+1] on the inputs' device" % name)
+
+
+def la_state_reduce(k, v, state, feature="elu1", workspace=None, stream=None):
+    """state <- (S | z) of the tokens of k, v (one shard of a sequence split along T)."""
+    B, H, T, D = _shape(k, v)
+    _full_state_check(state, B, H, D, k.device)
+    dt = _dtype_code(k)
+    wp, wn, _keep = _workspace("state_reduce", (B, H, T, D), dt, workspace, k.device, stream)
+    _check(_lib.la_state_reduce(_ptr(k), _ptr(v), _ptr(state), B, H, T, D, dt, _feature(feature), wp, wn,
+                                _stream(stream, k.device)), "la_state_reduce")
+
+
+def la_state_apply(q, state, o, feature="elu1", eps: float = 1e-6, stream=None):
+    """o <- the op's output for the tokens of q, given the whole sequence's (S | z)."""
+    B, H, T, D = _shape(q, o)
+    _full_state_check(state, B, H, D, q.device)
+    _check(_lib.la_state_apply(_ptr(q), _ptr(state), _ptr(o), B, H, T, D, _dtype_code(q), _feature(feature),
+                               float(eps), _stream(stream, q.device)), "la_state_apply")
+
+
+def la_state_bwd_q(q, dout, state, dq, dstate, feature="elu1", eps: float = 1e-6, workspace=None, stream=None):
+    """dq of the shard and its (dS | dz) into dstate, given the whole sequence's (S | z)."""
+    B, H, T, D = _shape(q, dout, dq)
+    _full_state_check(state, B, H, D, q.device)
+    _full_state_check(dstate, B, H, D, q.device, "dstate")
+    dt = _dtype_code(q)
+    wp, wn, _keep = _workspace("state_bwd_q", (B, H, T, D), dt, workspace, q.device, stream)
+    _check(_lib.la_state_bwd_q(_ptr(q), _ptr(dout), _ptr(state), _ptr(dq), _ptr(dstate), B, H, T, D, dt,
+                               _feature(feature), float(eps), wp, wn, _stream(stream, q.device)), "la_state_bwd_q")
+
+
+def la_state_bwd_kv(k, v, dstate, dk, dv, feature="elu1", stream=None):
+    """dk, dv of the shard given the whole sequence's (dS | dz)."""
+    B, H, T, D = _shape(k, v, dk, dv)
+    _full_state_check(dstate, B, H, D, k.device, "dstate")
+    _check(_lib.la_state_bwd_kv(_ptr(k), _ptr(v), _ptr(dstate), _ptr(dk), _ptr(dv), B, H, T, D, _dtype_code(k),
+                                _feature(feature), _stream(stream, k.device)), "la_state_bwd_kv")
 
 
 def la_status_string(status: int) -> str:

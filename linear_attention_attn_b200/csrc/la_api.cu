@@ -1,5 +1,6 @@
 // la_api.cu -- the C entry points: argument validation, workspace layout,
 // path selection, launch accounting and the optional per-kernel timing.
+#include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -226,6 +227,42 @@ static la_status decay_args(const float *decay, int H, DecayArgs *out) {
     return LA_OK;
 }
 
+// Front half of the sequence-parallel stage entry points.
+static la_status check_state(const void *p, const char *name) {
+    if (!p) return fail(LA_ERR_INVALID_ARG, "%s is NULL", name);
+    if (((uintptr_t)p) & 15) return fail(LA_ERR_ALIGNMENT, "%s is not 16-byte aligned", name);
+    return LA_OK;
+}
+
+static la_status stage_entry(Stage stage, la_op op, la_feature f, const void *x, const void *y, const float *sin,
+                             float *sout, void *out1, void *out2, int B, int H, int T, int D, la_dtype dt, float eps,
+                             void *ws, size_t ws_bytes, void *stream) {
+    const Shape s{B, H, T, D};
+    LA_TRY(validate(s, dt));
+    if (f != LA_FEATURE_IDENTITY && f != LA_FEATURE_ELU1) return fail(LA_ERR_UNSUPPORTED, "unknown feature map %d", (int)f);
+    if (!(eps >= 0.f) || !isfinite(eps)) return fail(LA_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    const char *xn = stage == Stage::Reduce || stage == Stage::BwdKV ? "k" : "q";
+    LA_TRY(check_ptr(x, xn));
+    if (stage != Stage::Apply) LA_TRY(check_ptr(y, stage == Stage::BwdQ ? "dout" : "v"));
+    if (sin) LA_TRY(check_state(sin, "state"));
+    if (stage != Stage::Reduce && !sin) return fail(LA_ERR_INVALID_ARG, "state is NULL");
+    if (stage == Stage::Reduce || stage == Stage::BwdQ) LA_TRY(check_state(sout, stage == Stage::Reduce ? "state" : "dstate"));
+    if (stage != Stage::Reduce) LA_TRY(check_ptr(out1, stage == Stage::Apply ? "o" : (stage == Stage::BwdQ ? "dq" : "dk")));
+    if (stage == Stage::BwdKV) LA_TRY(check_ptr(out2, "dv"));
+    LA_TRY(check_ws(op, s, dt, ws, ws_bytes));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (T == 0) {
+        if (sout) {
+            cudaError_t e = cudaMemsetAsync(sout, 0, state_bytes(s, 1), st);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+        }
+        return LA_OK;
+    }
+    const bool bidir = f == LA_FEATURE_ELU1;
+    if (path_tc(op, s, dt)) return tc::state_stage(stage, bidir, x, y, sin, sout, out1, out2, s, dt, eps, ws, st);
+    return simt::state_stage(stage, bidir, x, y, sin, sout, out1, out2, s, dt, eps, ws, st);
+}
+
 }  // namespace la
 
 using namespace la;
@@ -236,7 +273,7 @@ size_t la_workspace_size(la_op op, int B, int H, int T, int D, la_dtype dtype) {
     const Shape s{B, H, T, D};
     if (s.B < 1 || s.H < 1 || s.T < 0 || (s.D != 64 && s.D != 128)) return 0;
     if (dtype != LA_F32 && dtype != LA_F16 && dtype != LA_BF16) return 0;
-    if ((int)op < 0 || (int)op > 5) return 0;
+    if ((int)op < 0 || (int)op > (int)LA_OP_STATE_BWD_KV) return 0;
     return ws_size(op, s, dtype);
 }
 
@@ -300,6 +337,31 @@ la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const 
     cudaStream_t st = (cudaStream_t)stream;
     if (path_tc(LA_OP_CHUNK_DECAY_BWD, s, dtype)) return tc::decay_bwd(q, k, v, dout, dec, dq, dk, dv, s, dtype, workspace, st);
     return simt::decay_bwd(q, k, v, dout, dec, dq, dk, dv, s, dtype, st);
+}
+
+la_status la_state_reduce(const void *k, const void *v, float *state, int B, int H, int T, int D, la_dtype dtype,
+                          la_feature feature, void *workspace, size_t workspace_bytes, void *stream) {
+    return stage_entry(Stage::Reduce, LA_OP_STATE_REDUCE, feature, k, v, nullptr, state, nullptr, nullptr, B, H, T, D,
+                       dtype, 0.f, workspace, workspace_bytes, stream);
+}
+
+la_status la_state_apply(const void *q, const float *state, void *o, int B, int H, int T, int D, la_dtype dtype,
+                         la_feature feature, float eps, void *stream) {
+    return stage_entry(Stage::Apply, LA_OP_STATE_APPLY, feature, q, nullptr, state, nullptr, o, nullptr, B, H, T, D,
+                       dtype, eps, nullptr, 0, stream);
+}
+
+la_status la_state_bwd_q(const void *q, const void *dout, const float *state, void *dq, float *dstate, int B, int H,
+                         int T, int D, la_dtype dtype, la_feature feature, float eps, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    return stage_entry(Stage::BwdQ, LA_OP_STATE_BWD_Q, feature, q, dout, state, dstate, dq, nullptr, B, H, T, D, dtype,
+                       eps, workspace, workspace_bytes, stream);
+}
+
+la_status la_state_bwd_kv(const void *k, const void *v, const float *dstate, void *dk, void *dv, int B, int H, int T,
+                          int D, la_dtype dtype, la_feature feature, void *stream) {
+    return stage_entry(Stage::BwdKV, LA_OP_STATE_BWD_KV, feature, k, v, dstate, nullptr, dk, dv, B, H, T, D, dtype,
+                       0.f, nullptr, 0, stream);
 }
 
 la_status la_chunk_decay_step(const void *q, const void *k, const void *v, void *o, float *state,

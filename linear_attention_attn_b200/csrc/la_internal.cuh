@@ -99,6 +99,13 @@ struct DecayArgs {
     float gamma[LA_MAX_DECAY_HEADS];
 };
 
+// Stages of the state form, run separately for a sequence split along T:
+//   Reduce  k, v            -> [S | z] of the tokens passed
+//   Apply   q, [S | z]      -> o
+//   BwdQ    q, dO, [S | z]  -> dq and the tokens' [dS | dz]
+//   BwdKV   k, v, [dS | dz] -> dk, dv
+enum class Stage { Reduce, Apply, BwdQ, BwdKV };
+
 // ------------------------------------------------------ shape / workspace --
 struct Shape {
     int B, H, T, D;
@@ -132,6 +139,8 @@ la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const 
                     const Shape &s, la_dtype dt, cudaStream_t st);
 la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec,
                     void *dq, void *dk, void *dv, const Shape &s, la_dtype dt, cudaStream_t st);
+la_status state_stage(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout,
+                      void *out1, void *out2, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
 }  // namespace simt
 
 }  // namespace la

@@ -505,6 +505,58 @@ la_status state_bwd_t(bool bidir, const T *q, const T *k, const T *v, const T *g
                           (const float *)dstate, dk, dv, s.T);
 }
 
+// One stage of the state form (see Stage): the same kernels as state_fwd_t /
+// state_bwd_t, with the state passed in or handed out instead of kept inside.
+template <typename T, int D>
+la_status stage_t(Stage stage, bool bidir, const T *x, const T *y, const float *sin, float *sout, T *out1, T *out2,
+                  const Shape &s, float eps, void *ws, cudaStream_t st) {
+    const int nsplit = simt_splits(s);
+    const int rps = (s.T + nsplit - 1) / nsplit;
+    float *part = (float *)ws;
+    const dim3 g1(nsplit, (unsigned)s.BH());
+    const dim3 g2((s.T + kTile - 1) / kTile, (unsigned)s.BH());
+    la_status rc;
+    switch (stage) {
+    case Stage::Reduce:
+        rc = bidir ? launch("simt_state_partial", state_partial<T, D, true>, g1, dim3(kThreads), 0, st, x, y, part,
+                            s.T, nsplit, rps)
+                   : launch("simt_state_partial", state_partial<T, D, false>, g1, dim3(kThreads), 0, st, x, y, part,
+                            s.T, nsplit, rps);
+        if (rc) return rc;
+        return launch("simt_combine", combine, dim3((unsigned)s.BH()), dim3(kThreads), 0, st, (const float *)part, sout,
+                      nsplit, D * (D + 1));
+    case Stage::Apply: {
+        const size_t smem = (size_t)(D * D + D + kTile * (D + 1)) * sizeof(float);
+        return bidir ? launch("simt_output", output<T, D, true>, g2, dim3(kThreads), smem, st, x, sin, out1, s.T, eps)
+                     : launch("simt_output", output<T, D, false>, g2, dim3(kThreads), smem, st, x, sin, out1, s.T, eps);
+    }
+    case Stage::BwdQ: {
+        const size_t smemq = (size_t)(D * (D + 1) + D + 3 * kTile * (D + 1) + kTile) * sizeof(float);
+        rc = bidir ? launch("simt_bwd_q", bwd_q<T, D, true>, g1, dim3(kThreads), smemq, st, x, y, sin, out1, part, s.T,
+                            nsplit, rps, eps)
+                   : launch("simt_bwd_q", bwd_q<T, D, false>, g1, dim3(kThreads), smemq, st, x, y, sin, out1, part, s.T,
+                            nsplit, rps, eps);
+        if (rc) return rc;
+        return launch("simt_combine", combine, dim3((unsigned)s.BH()), dim3(kThreads), 0, st, (const float *)part, sout,
+                      nsplit, D * (D + 1));
+    }
+    default: {
+        const size_t smemk = (size_t)(D * (D + 1) + D + 3 * kTile * (D + 1)) * sizeof(float);
+        return bidir ? launch("simt_bwd_k", bwd_k<T, D, true>, g2, dim3(kThreads), smemk, st, x, y, sin, out1, out2, s.T)
+                     : launch("simt_bwd_k", bwd_k<T, D, false>, g2, dim3(kThreads), smemk, st, x, y, sin, out1, out2,
+                              s.T);
+    }
+    }
+}
+
+template <typename T>
+la_status stage_d(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout, void *out1,
+                  void *out2, const Shape &s, float eps, void *ws, cudaStream_t st) {
+    if (s.D == 64)
+        return stage_t<T, 64>(stage, bidir, (const T *)x, (const T *)y, sin, sout, (T *)out1, (T *)out2, s, eps, ws, st);
+    return stage_t<T, 128>(stage, bidir, (const T *)x, (const T *)y, sin, sout, (T *)out1, (T *)out2, s, eps, ws, st);
+}
+
 template <typename T>
 la_status state_fwd_d(bool bidir, const void *q, const void *k, const void *v, void *o, float *state, const Shape &s,
                       float eps, void *ws, cudaStream_t st) {
@@ -549,8 +601,20 @@ size_t workspace_size(la_op op, const Shape &s) {
     case LA_OP_BIDIR_BWD:
     case LA_OP_SIMPLE_BWD:
         return state_bytes(s, simt_splits(s)) + 2 * state_bytes(s, 1);
+    case LA_OP_STATE_REDUCE:
+    case LA_OP_STATE_BWD_Q:
+        return state_bytes(s, simt_splits(s));
     default:
         return 0;
+    }
+}
+
+la_status state_stage(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout,
+                      void *out1, void *out2, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st) {
+    switch (dt) {
+    case LA_F32: return stage_d<float>(stage, bidir, x, y, sin, sout, out1, out2, s, eps, ws, st);
+    case LA_F16: return stage_d<__half>(stage, bidir, x, y, sin, sout, out1, out2, s, eps, ws, st);
+    default: return stage_d<__nv_bfloat16>(stage, bidir, x, y, sin, sout, out1, out2, s, eps, ws, st);
     }
 }
 

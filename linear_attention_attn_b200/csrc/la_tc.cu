@@ -10,7 +10,11 @@ bool supports(la_op op, const Shape &s, la_dtype dt) {
     case LA_OP_BIDIR_FWD:
     case LA_OP_BIDIR_BWD:
     case LA_OP_SIMPLE_FWD:
-    case LA_OP_SIMPLE_BWD: return s.D == 64;
+    case LA_OP_SIMPLE_BWD:
+    case LA_OP_STATE_REDUCE:
+    case LA_OP_STATE_APPLY:
+    case LA_OP_STATE_BWD_Q:
+    case LA_OP_STATE_BWD_KV: return s.D == 64;
     case LA_OP_CHUNK_DECAY_FWD:
     case LA_OP_CHUNK_DECAY_BWD: return dt == LA_BF16 && s.D == 128;
     default: return false;
@@ -28,7 +32,9 @@ size_t workspace_size(la_op op, const Shape &s, la_dtype) {
     case LA_OP_BIDIR_FWD:
     case LA_OP_BIDIR_BWD:
     case LA_OP_SIMPLE_FWD:
-    case LA_OP_SIMPLE_BWD: return state_workspace_size(op, s);
+    case LA_OP_SIMPLE_BWD:
+    case LA_OP_STATE_REDUCE:
+    case LA_OP_STATE_BWD_Q: return state_workspace_size(op, s);
     default: return 0;
     }
 }

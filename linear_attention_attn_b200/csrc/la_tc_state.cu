@@ -1018,7 +1018,8 @@ template <bool BIDIR, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
               const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
-              const float *__restrict__ dpart, int T, int BH, int nt, int maxslots, int early_loads) {
+              const float *__restrict__ src, int src_per_head, int src_single, int T, int BH, int nt,
+              int early_loads) {
     using L = BwdKvLayout;
     constexpr int NST = L::NST, OPB = L::OPB;
     constexpr int NOPS = BF16 ? 2 : 1;
@@ -1178,8 +1179,8 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             const int j = t.j;
             if (h != cur_h) {
                 // the previous head's UMMAs are complete (its last epilogue waited on them)
-                const float *srch = dpart + h * (long long)maxslots * kStateElems;
-                const int ns = P.last_cta((int)h) - P.first_cta((int)h) + 1;
+                const float *srch = src + h * (long long)src_per_head;
+                const int ns = src_single ? 1 : (P.last_cta((int)h) - P.first_cta((int)h) + 1);
                 float m = gather_state(srch, ns, stage, tid);
                 named_bar(1, kWorkers);
                 if (!BF16) m = workers_max(m, red, tid);
@@ -1247,6 +1248,29 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 256);
+    }
+}
+
+// ================================================================ combine ==
+// state[h] = sum over the head's partial slots 0 .. ns(h) - 1 in slot order (the
+// order every consumer's gather uses, so the sum is the same bits).
+__global__ void __launch_bounds__(256)
+combine_partials_kernel(const float *__restrict__ part, float *__restrict__ out, int BH, int nt, int maxslots) {
+    const Partition P{(long long)BH * nt, nt, grid_for((long long)BH * nt)};
+    const int h = blockIdx.x;
+    const int ns = P.last_cta(h) - P.first_cta(h) + 1;
+    const float4 *src = reinterpret_cast<const float4 *>(part + (long long)h * maxslots * kStateElems);
+    float4 *dst = reinterpret_cast<float4 *>(out + (long long)h * kStateElems);
+    for (int e = threadIdx.x; e < kStateElems / 4; e += blockDim.x) {
+        float4 a = src[e];
+        for (int sl = 1; sl < ns; ++sl) {
+            const float4 b = src[(long long)sl * (kStateElems / 4) + e];
+            a.x += b.x;
+            a.y += b.y;
+            a.z += b.z;
+            a.w += b.w;
+        }
+        dst[e] = a;
     }
 }
 
@@ -1359,7 +1383,58 @@ static la_status bwd_t(const void *q, const void *k, const void *v, const void *
                   (size_t)BwdQLayout<BIDIR, BF16>::bytes, st, mq, mg, mdq, src, per_head, single, dpart, s.T, (int)s.BH(),
                   nt, ms, eps, state ? 0 : 1));
     return launch_pdl(BIDIR ? "tc_bwd_kv" : "tc_bwd_kv_simple", bwd_kv_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
-                  (size_t)BwdKvLayout::bytes, st, mk, mv, mdk, mdv, (const float *)dpart, s.T, (int)s.BH(), nt, ms, 1);
+                  (size_t)BwdKvLayout::bytes, st, mk, mv, mdk, mdv, (const float *)dpart, ms * kStateElems, 0, s.T,
+                  (int)s.BH(), nt, 1);
+}
+
+// The state form in separate stages, for a sequence split along T (see the
+// sequence-parallel entry points): the caller sums the stages' states across
+// the shards between them.
+template <bool BIDIR, bool BF16>
+static la_status stage_t(Stage stage, const void *x, const void *y, const float *sin, float *sout, void *out1,
+                         void *out2, const Shape &s, float eps, void *ws, cudaStream_t st) {
+    const int nt = (s.T + kRows - 1) / kRows;
+    const int ms = max_slots((int)s.BH());
+    float *part = (float *)ws;
+    switch (stage) {
+    case Stage::Reduce: {   // x = k, y = v -> sout = [S | z]
+        CUtensorMap mk, mv;
+        LA_TRY(tensor_map(&mk, x, s, BF16));
+        LA_TRY(tensor_map(&mv, y, s, BF16));
+        LA_TRY((launch_reduce<BIDIR, BF16>(mk, mv, part, s, nt, st)));
+        return launch("tc_combine", combine_partials_kernel, dim3((unsigned)s.BH()), dim3(256), 0, st,
+                      (const float *)part, sout, (int)s.BH(), nt, ms);
+    }
+    case Stage::Apply: {    // x = q, sin = [S | z] -> out1 = o
+        CUtensorMap mq, mo;
+        LA_TRY(tensor_map(&mq, x, s, BF16));
+        LA_TRY(tensor_map(&mo, out1, s, BF16));
+        return launch_pdl(BIDIR ? "tc_output" : "tc_output_simple", output_kernel<BIDIR, BF16>,
+                          dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads), (size_t)OutputLayout::bytes, st, mq,
+                          mo, sin, kStateElems, 1, (float *)nullptr, s.T, (int)s.BH(), nt, eps, 0);
+    }
+    case Stage::BwdQ: {     // x = q, y = dO, sin = [S | z] -> out1 = dq, sout = [dS | dz]
+        CUtensorMap mq, mg, mdq;
+        LA_TRY(tensor_map(&mq, x, s, BF16));
+        LA_TRY(tensor_map(&mg, y, s, BF16));
+        LA_TRY(tensor_map(&mdq, out1, s, BF16));
+        LA_TRY(launch_pdl(BIDIR ? "tc_bwd_q" : "tc_bwd_q_simple", bwd_q_kernel<BIDIR, BF16>,
+                          dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads), (size_t)BwdQLayout<BIDIR, BF16>::bytes,
+                          st, mq, mg, mdq, sin, kStateElems, 1, part, s.T, (int)s.BH(), nt, ms, eps, 0));
+        return launch("tc_combine", combine_partials_kernel, dim3((unsigned)s.BH()), dim3(256), 0, st,
+                      (const float *)part, sout, (int)s.BH(), nt, ms);
+    }
+    default: {              // x = k, y = v, sin = [dS | dz] -> out1 = dk, out2 = dv
+        CUtensorMap mk, mv, mdk, mdv;
+        LA_TRY(tensor_map(&mk, x, s, BF16));
+        LA_TRY(tensor_map(&mv, y, s, BF16));
+        LA_TRY(tensor_map(&mdk, out1, s, BF16));
+        LA_TRY(tensor_map(&mdv, out2, s, BF16));
+        return launch_pdl(BIDIR ? "tc_bwd_kv" : "tc_bwd_kv_simple", bwd_kv_kernel<BIDIR, BF16>,
+                          dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads), (size_t)BwdKvLayout::bytes, st, mk,
+                          mv, mdk, mdv, sin, kStateElems, 1, s.T, (int)s.BH(), nt, 0);
+    }
+    }
 }
 
 }  // namespace
@@ -1370,8 +1445,19 @@ size_t state_workspace_size(la_op op, const Shape &s) {
     case LA_OP_SIMPLE_FWD: return partial_bytes(s);
     case LA_OP_BIDIR_BWD:
     case LA_OP_SIMPLE_BWD: return 2 * partial_bytes(s);
+    case LA_OP_STATE_REDUCE:
+    case LA_OP_STATE_BWD_Q: return partial_bytes(s);
     default: return 0;
     }
+}
+
+la_status state_stage(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout,
+                      void *out1, void *out2, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st) {
+    const bool bf = dt == LA_BF16;
+    if (bidir) return bf ? stage_t<true, true>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st)
+                         : stage_t<true, false>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st);
+    return bf ? stage_t<false, true>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st)
+              : stage_t<false, false>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st);
 }
 
 la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, void *o, float *state, const Shape &s,

@@ -1,0 +1,125 @@
+"""Sequence parallelism on CPU: two gloo ranks each hold half of a sequence and run
+linear_attention_attn_b200.seqpar with a float64 torch implementation of the four stages
+(written here from their definitions); the shards' outputs and gradients must equal the
+oracle's on the whole sequence.  This checks the split (local reduce, all-reduce, local
+apply; local dq pass, all-reduce of (dS | dz), local dk, dv pass) and the collective plumbing."""
+import os
+import socket
+import sys
+import types
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _phi(x, feature):
+    return torch.where(x > 0, x + 1.0, torch.exp(torch.clamp(x, max=0.0))) if feature == "elu1" else x
+
+
+def _dphi(x, feature):
+    return torch.where(x > 0, torch.ones_like(x), torch.exp(torch.clamp(x, max=0.0))) if feature == "elu1" \
+        else torch.ones_like(x)
+
+
+def _stages():
+    """The four stages on float64 CPU tensors, from the formulas of include/la.h."""
+    def la_state_reduce(k, v, state, feature="elu1", stream=None):
+        D = k.shape[-1]
+        fk = _phi(k, feature)
+        state[..., :D] = torch.einsum("bhti,bhtj->bhij", fk, v)
+        state[..., D] = fk.sum(2) if feature == "elu1" else 0.0
+
+    def la_state_apply(q, state, o, feature="elu1", eps=1e-6, stream=None):
+        D = q.shape[-1]
+        fq = _phi(q, feature)
+        u = torch.einsum("bhti,bhij->bhtj", fq, state[..., :D])
+        if feature == "elu1":
+            u = u / (torch.einsum("bhti,bhi->bht", fq, state[..., D]) + eps)[..., None]
+        o.copy_(u)
+
+    def la_state_bwd_q(q, dout, state, dq, dstate, feature="elu1", eps=1e-6, stream=None):
+        D = q.shape[-1]
+        S, z = state[..., :D], state[..., D]
+        fq = _phi(q, feature)
+        gs = torch.einsum("bhtj,bhij->bhti", dout, S)                 # dout S^T
+        if feature == "elu1":
+            n = torch.einsum("bhti,bhi->bht", fq, z) + eps
+            o = torch.einsum("bhti,bhij->bhtj", fq, S) / n[..., None]
+            go = (dout * o).sum(-1)
+            dq.copy_((gs - go[..., None] * z[:, :, None, :]) / n[..., None] * _dphi(q, feature))
+            dstate[..., :D] = torch.einsum("bhti,bhtj->bhij", fq, dout / n[..., None])
+            dstate[..., D] = -torch.einsum("bhti,bht->bhi", fq, go / n)
+        else:
+            dq.copy_(gs)
+            dstate[..., :D] = torch.einsum("bhti,bhtj->bhij", q, dout)
+            dstate[..., D] = 0.0
+
+    def la_state_bwd_kv(k, v, dstate, dk, dv, feature="elu1", stream=None):
+        D = k.shape[-1]
+        dS, dz = dstate[..., :D], dstate[..., D]
+        dk.copy_((torch.einsum("bhsj,bhij->bhsi", v, dS) + dz[:, :, None, :]) * _dphi(k, feature))
+        dv.copy_(torch.einsum("bhsi,bhij->bhsj", _phi(k, feature), dS))
+
+    return types.SimpleNamespace(la_state_reduce=la_state_reduce, la_state_apply=la_state_apply,
+                                 la_state_bwd_q=la_state_bwd_q, la_state_bwd_kv=la_state_bwd_kv)
+
+
+def _inputs(B, H, T, D):
+    g = torch.Generator().manual_seed(7)
+    return [torch.randn(B, H, T, D, generator=g, dtype=torch.float64) * s for s in (0.5, 0.5, 1.0, 1.0)]
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, feature, cuts, out):
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    from linear_attention_attn_b200 import seqpar
+    B, H, T, D = 2, 3, cuts[-1], 8
+    q, k, v, g = _inputs(B, H, T, D)
+    sl = slice(cuts[rank], cuts[rank + 1])
+    qs, ks, vs, gs = (x[:, :, sl].contiguous() for x in (q, k, v, g))
+    ops = _stages()
+    state = torch.empty(B, H, D, D + 1, dtype=torch.float64)
+    o = torch.empty_like(qs)
+    seqpar.forward(qs, ks, vs, o, state, feature=feature, eps=1e-3, ops=ops)
+    dq, dk, dv = torch.empty_like(qs), torch.empty_like(qs), torch.empty_like(qs)
+    dstate = torch.empty_like(state)
+    seqpar.backward(qs, ks, vs, gs, state, dq, dk, dv, dstate, feature=feature, eps=1e-3, ops=ops)
+    out[rank] = [t.numpy() for t in (o, dq, dk, dv)]
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("feature", ["elu1", "identity"])
+def test_two_ranks_match_the_whole_sequence(feature):
+    import oracle
+    cuts = [0, 11, 30]                    # uneven shards
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, feature, cuts, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    q, k, v, g = (x.numpy() for x in _inputs(2, 3, cuts[-1], 8))
+    if feature == "elu1":
+        want = [oracle.bidir_fwd(q, k, v, eps=1e-3)] + list(oracle.bidir_bwd(q, k, v, g, eps=1e-3))
+    else:
+        want = [oracle.simple_fwd(q, k, v)] + list(oracle.simple_bwd(q, k, v, g))
+    for i, name in enumerate(("o", "dq", "dk", "dv")):
+        got = np.concatenate([out[0][i], out[1][i]], axis=2)
+        np.testing.assert_allclose(got, want[i], rtol=1e-10, atol=1e-12, err_msg=name)
