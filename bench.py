@@ -324,19 +324,35 @@ def run_ours(args, w):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
 
-    host = synth.make_inputs(w, seed=rank)
+    seqpar = getattr(args, "seqpar", False)
+    if seqpar:
+        # the workload's T is the whole sequence; this rank holds a shard of T / world tokens
+        from linear_attention_attn_b200 import seqpar as sp
+        if w.op == "retention" or w.T % world:
+            raise SystemExit("--seqpar needs the bidir or simple workload and T divisible by the GPU count")
+        host = synth.make_inputs(w.with_T(w.T // world), seed=rank)
+    else:
+        host = synth.make_inputs(w, seed=rank)
     q, k, v, g = (host[n].to(dev) for n in ("q", "k", "v", "do"))
-    B, H, T, D = w.B, w.H, w.T, w.D
+    B, H, D = w.B, w.H, w.D
+    T = q.shape[2]
     o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
     state = torch.empty((B, H, D, D + 1), dtype=torch.float32, device=dev)
+    dstate = torch.empty_like(state)
     names = {"bidir": ("bidir_fwd", "bidir_bwd"), "simple": ("simple_fwd", "simple_bwd"),
              "retention": ("chunk_decay_fwd", "chunk_decay_bwd")}[w.op]
+    if seqpar:
+        names = ("state_reduce", "state_bwd_q")
     ws_bytes = max(la.la_workspace_size(n, B, H, T, D, q.dtype) for n in names)
     ws = torch.empty(max(256, ws_bytes), dtype=torch.uint8, device=dev)
     gamma = host.get("gamma")
+    feature = "elu1" if w.op == "bidir" else "identity"
 
     def step():
-        if w.op == "bidir":
+        if seqpar:
+            sp.forward(q, k, v, o, state, feature=feature, eps=w.eps, workspace=ws)
+            sp.backward(q, k, v, g, state, dq, dk, dv, dstate, feature=feature, eps=w.eps, workspace=ws)
+        elif w.op == "bidir":
             la.la_bidir_fwd(q, k, v, o, state, eps=w.eps, workspace=ws)
             la.la_bidir_bwd(q, k, v, g, dq, dk, dv, state, eps=w.eps, workspace=ws)
         elif w.op == "simple":
@@ -442,7 +458,7 @@ def run_ours(args, w):
 
     # ---- the same step at the longer sequence lengths of the metric (device events only)
     sweep = []
-    if world == 1 and args.sweep and w.op == "bidir":
+    if world == 1 and args.sweep and w.op == "bidir" and not seqpar:
         del o, dq, dk, dv, q, k, v, g, ws
         torch.cuda.empty_cache()
         for Ts in (8192, 16384):
@@ -466,20 +482,26 @@ def run_ours(args, w):
         cpu = {"value": r, "unit": UNIT, "cores": used, "kind": "oracle", "sample": sample, "seconds": dt}
 
     vs = None
-    if w.op == "bidir" and T in PAGE_TIMINGS_MS and (B, H, D) == (8, 16, 64):
+    if w.op == "bidir" and not seqpar and T in PAGE_TIMINGS_MS and (B, H, D) == (8, 16, 64):
         page_rate = B * T / (sum(PAGE_TIMINGS_MS[T]) / 1e3)
         vs = value / page_rate
 
     line = {
         "metric": METRIC if w.op == "bidir" else "%s fwd+bwd tokens/s" % w.op, "value": value, "unit": UNIT,
         "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "strong" if seqpar else "weak",
         "vs_baseline": vs, "dtype": w.dtype, "data": "synthetic", "config": config_of(w, args),
         "roofline": roof, "step_roofline": step_roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches, "clocks": clocks, "t_sweep": sweep,
         "kernels": [{"name": n, "launches": c, "total_ms": t} for n, c, t in per_kernel],
         "kernel_timing": "per-kernel CUDA events on the launch stream over %d further steps after the timed region" % k_prof,
     }
+    if seqpar:
+        line["config"]["parallelism"] = ("sp%d (the sequence split along T: %d tokens per GPU, one all-reduce of the "
+                                         "[B,H,D,D+1] state per pass)" % (world, T))
+        line["config"]["shard_T"] = T
+        line["config"]["global_batch"] = B
     print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
@@ -641,6 +663,9 @@ def main(argv=None):
                     help="bidir (the benchmark metric, B8 H16 D64 fp16), simple (B8 H16 D64 bf16), "
                          "retention (B8 H32 D128 bf16) or decode (recurrent decay step, B64 H32 D128)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seqpar", action="store_true",
+                    help="bidir/simple: split the workload's sequence along T across the GPUs (one all-reduce of "
+                         "the state per pass; strong scaling) instead of independent batches per GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", dest="sweep", action="store_false",
                     help="skip the extra T=8192/16384 device timings added to the JSON line")

@@ -16,26 +16,31 @@ def _all_reduce(t, group):
         dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
 
 
-def forward(q, k, v, o, state, feature="elu1", eps: float = 1e-6, group=None, ops=None, stream=None):
-    """o <- the op's output for this rank's shard; state <- the whole sequence's (S | z)."""
+def forward(q, k, v, o, state, feature="elu1", eps: float = 1e-6, group=None, ops=None, stream=None,
+            workspace=None):
+    """o <- the op's output for this rank's shard; state <- the whole sequence's (S | z).
+    workspace: optional device buffer of la_workspace_size("state_reduce", ...) bytes."""
     if ops is None:
         from linear_attention_attn_b200 import la_state_apply, la_state_reduce
     else:
         la_state_reduce, la_state_apply = ops.la_state_reduce, ops.la_state_apply
-    la_state_reduce(k, v, state, feature=feature, stream=stream)
+    kw = {} if workspace is None else {"workspace": workspace}
+    la_state_reduce(k, v, state, feature=feature, stream=stream, **kw)
     _all_reduce(state, group)
     la_state_apply(q, state, o, feature=feature, eps=eps, stream=stream)
     return state
 
 
 def backward(q, k, v, dout, state, dq, dk, dv, dstate, feature="elu1", eps: float = 1e-6, group=None, ops=None,
-             stream=None):
-    """dq, dk, dv of this rank's shard from the whole sequence's state (from forward)."""
+             stream=None, workspace=None):
+    """dq, dk, dv of this rank's shard from the whole sequence's state (from forward).
+    workspace: optional device buffer of la_workspace_size("state_bwd_q", ...) bytes."""
     if ops is None:
         from linear_attention_attn_b200 import la_state_bwd_kv, la_state_bwd_q
     else:
         la_state_bwd_q, la_state_bwd_kv = ops.la_state_bwd_q, ops.la_state_bwd_kv
-    la_state_bwd_q(q, dout, state, dq, dstate, feature=feature, eps=eps, stream=stream)
+    kw = {} if workspace is None else {"workspace": workspace}
+    la_state_bwd_q(q, dout, state, dq, dstate, feature=feature, eps=eps, stream=stream, **kw)
     _all_reduce(dstate, group)
     la_state_bwd_kv(k, v, dstate, dk, dv, feature=feature, stream=stream)
     return dstate
