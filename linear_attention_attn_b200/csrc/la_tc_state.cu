@@ -902,30 +902,37 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             got = __all_sync(0xffffffffu, got);
             live = live && got;
             sfull_ph ^= 1;
-            if (!got) return;
-            tc_fence_after();
-            const uint32_t base = tmem + kAccS + ((uint32_t)(32 * sub) << 16);
-            float v[64];
-            tmem_row64(base, v);
-            float zz = 0.f;
-            if (BIDIR) {
-                float t16[16];
-                tmem_ld16(base + 64, t16);
-                tmem_ld_wait();
-                zz = t16[0];
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(accSfree);
-            if (lane < 16) {
-                const int i = 16 * sub + lane;
-                const int slot = cta - P.first_cta(hs);
-                float *dst = dpart + (((long long)hs * maxslots + slot) * 64 + i) * 65;
-                const float is = 1.f / scn;
+            if (got) {
+                tc_fence_after();
+                const uint32_t base = tmem + kAccS + ((uint32_t)(32 * sub) << 16);
+                float v[64];
+                tmem_row64(base, v);
+                float zz = 0.f;
+                if (BIDIR) {
+                    float t16[16];
+                    tmem_ld16(base + 64, t16);
+                    tmem_ld_wait();
+                    zz = t16[0];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(accSfree);
+                if (lane < 16) {   // row i of [dS | dz] into the staging block (stride 65: no bank conflicts)
+                    const int i = 16 * sub + lane;
+                    const float is = 1.f / scn;
 #pragma unroll
-                for (int c = 0; c < 64; ++c) dst[c] = v[c] * is;
-                dst[64] = zz * is;
+                    for (int c = 0; c < 64; ++c) stage[i * 65 + c] = v[c] * is;
+                    stage[i * 65 + 64] = zz * is;
+                }
             }
+            named_bar(1, kWorkers);
+            if (live) {            // the slot as one contiguous, coalesced 16.6 KB copy
+                float4 *dst = reinterpret_cast<float4 *>(dpart + ((long long)hs * maxslots + (cta - P.first_cta(hs))) *
+                                                                     kStateElems);
+                const float4 *src4 = reinterpret_cast<const float4 *>(stage);
+                for (int e = tid; e < kStateElems / 4; e += kWorkers) dst[e] = src4[e];
+            }
+            named_bar(1, kWorkers);   // the staging block is free for the next head's gather
         };
 
         float2 *rinfo = reinterpret_cast<float2 *>(smem + L::rioff);
