@@ -529,8 +529,10 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 // descriptor points its second atom there (a start 32 s bytes into a 128-byte
 // row, as a K step does for K-major operands).  bf16 bidir also keeps
 // lo = round(f(q) - hi): MMA1 adds f(Q)_lo S_hi and f'(q) = min(hi + lo, 1).
-// Warp roles of bwd_q: 0 TMA, 1 UMMA, 2..5 feature map, 6..9 dq, 10..13 epilogue.
-constexpr int kQXWarps = 4, kQDw0 = kXw0 + kQXWarps, kQDWarps = 4;
+// Warp roles of bwd_q: 0 TMA, 1 UMMA (MMA1, MMA2), 2..5 feature map, 6..9 dq,
+// 10..13 epilogue, 14 UMMA (MMA3).
+constexpr int kQXWarps = 4, kQDw0 = kXw0 + kQXWarps, kQDWarps = 4, kQU2 = kEw0 + kEWarps;
+constexpr int kQThreads = (kQU2 + 1) * 32;
 static_assert(kQDw0 + kQDWarps == kEw0, "bwd_q warp roles");
 
 template <bool BIDIR, bool BF16>
@@ -549,14 +551,14 @@ struct BwdQLayout {
     static constexpr int rioff = iscoff + 16;                        // [2][128] (g.o, 1/n) per row
     static constexpr int redoff = rioff + 2 * 128 * 8;
     static constexpr int baroff = redoff + 32;
-    static constexpr int nbars = 4 * NST + 8;
+    static constexpr int nbars = 4 * NST + 9;
     static constexpr int misc = baroff + nbars * 8;
     static constexpr int bytes = misc + 32 + 1024;
     static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 template <bool BIDIR, bool BF16>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kQThreads, 1)
 bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
              const __grid_constant__ CUtensorMap tmDQ, const float *__restrict__ src, int src_per_head,
              int src_single, float *__restrict__ dpart, int T, int BH, int nt, int maxslots, float eps,
@@ -590,6 +592,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     uint64_t *accSfree = accSfull + 1;
     uint64_t *opready = accSfree + 1;
     uint64_t *drain = opready + 1;
+    uint64_t *drain2 = drain + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc);
     int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
 
@@ -614,6 +617,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         mbar_init(accSfree, kEWarps);
         mbar_init(opready, 1);
         mbar_init(drain, 1);
+        mbar_init(drain2, 1);
         *s_abort = 0;
         fence_mbar_init();
     }
@@ -622,7 +626,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         tma_prefetch(&tmG);
         tma_prefetch(&tmDQ);
     }
-    if (BIDIR && warp >= kEw0) {   // the w tile: zero except column 16 s of stage s, written per tile
+    if (BIDIR && warp >= kEw0 && warp < kQU2) {   // the w tile: zero except column 16 s of stage s, written per tile
         const int r = threadIdx.x - kEw0 * 32;
         uint8_t *p = sW + r * 128;
 #pragma unroll
@@ -673,41 +677,9 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             long long prev_h = -1;
             long long seg = 0;                     // segments started (accS free parity)
             bool dead = false;
-            // MMA3 of tile xe (stage se, phase phe)
-            auto issue3 = [&](long long xe, int je, int se, uint32_t phe) {
-                const bool seg_start = (xe == x0) || je == 0;
-                const bool seg_end = (xe + 1 == x1) || je + 1 == nt;
-                if (seg_start) {
-                    if (!LA_WAIT(accSfree, (uint32_t)((seg & 1) ^ 1), 0x40u)) { dead = true; return; }
-                    ++seg;
-                }
-                if (!LA_WAIT(&gnready[se], phe, 0x80u)) { dead = true; return; }
-                tc_fence_after();
-                const uint32_t aG = smem_u32(sG + se * kTileBytes);
-                // the second MN atom of [g/n | w] starts at column 16 se of the shared w tile
-                const uint32_t lbo = BIDIR ? smem_u32(sW) + 32u * (uint32_t)se - aG : (uint32_t)kTileBytes;
-                const uint64_t dq = sdesc_sw128(smem_u32(sQ + se * kTileBytes), kTileBytes, 1024);
-                const uint64_t dg = sdesc_sw128(aG, lbo, 1024);
-#pragma unroll
-                for (int kk = 0; kk < kRows / 16; ++kk)
-                    umma_f16_ss(tmem + kAccS, desc_at(dq, kk * 2048), desc_at(dg, kk * 2048), IDESC3,
-                                (seg_start && kk == 0) ? 0u : 1u);
-                umma_commit(&empty[se]);
-                if (seg_end) umma_commit(accSfull);
-            };
-            long long xp = -1;
-            int sp = 0, jp = 0;
-            uint32_t php = 0;
             for (TileCursor t(x0, nt); t.x < x1 && !dead; t.next()) {
-                const long long x = t.x;
                 const long long h = t.h;
                 if (h != prev_h) {
-                    // finish the previous head (its dS partial) before waiting on the next operand
-                    if (xp >= 0) {
-                        issue3(xp, jp, sp, php);
-                        xp = -1;
-                        if (dead) break;
-                    }
                     if (!LA_WAIT(opready, oph, 0x20u)) break;
                     oph ^= 1;
                     prev_h = h;
@@ -736,16 +708,44 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 umma_commit(&acc12full[b]);
                 b ^= 1;
                 if (b == 0) bph ^= 1;
-                if (xp >= 0) issue3(xp, jp, sp, php);
-                xp = x;
-                jp = t.j;
-                sp = s;
-                php = ph;
                 if (++s == NST) { s = 0; ph ^= 1; }
             }
-            if (xp >= 0 && !dead && !*s_abort) issue3(xp, jp, sp, php);
             umma_commit(drain);
             mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+        }
+    } else if (warp == kQU2) {
+        // Second UMMA issuer: MMA3 of every tile, in tile order, once the epilogue
+        // warps have written its g/n and w.  A thread's issue rate, not the tensor
+        // pipe, bounds these small-N UMMAs while the other warps of its scheduler
+        // are busy, so the two UMMA groups of a tile come from two schedulers.
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            long long seg = 0;                     // segments started (accS free parity)
+            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+                const bool seg_start = (t.x == x0) || t.j == 0;
+                const bool seg_end = (t.x + 1 == x1) || t.last_of_head();
+                if (seg_start) {
+                    if (!LA_WAIT(accSfree, (uint32_t)((seg & 1) ^ 1), 0x40u)) break;
+                    ++seg;
+                }
+                if (!LA_WAIT(&gnready[s], ph, 0x80u)) break;
+                tc_fence_after();
+                const uint32_t aG = smem_u32(sG + s * kTileBytes);
+                // the second MN atom of [g/n | w] starts at column 16 s of the shared w tile
+                const uint32_t lbo = BIDIR ? smem_u32(sW) + 32u * (uint32_t)s - aG : (uint32_t)kTileBytes;
+                const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTileBytes), kTileBytes, 1024);
+                const uint64_t dg = sdesc_sw128(aG, lbo, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kRows / 16; ++kk)
+                    umma_f16_ss(tmem + kAccS, desc_at(dq, kk * 2048), desc_at(dg, kk * 2048), IDESC3,
+                                (seg_start && kk == 0) ? 0u : 1u);
+                umma_commit(&empty[s]);
+                if (seg_end) umma_commit(accSfull);
+                if (++s == NST) { s = 0; ph ^= 1; }
+            }
+            umma_commit(drain2);
+            mbar_wait_slow(smem_u32(drain2), 0, nullptr, &g_tc_fault, 0x400u);
         }
     } else if (warp < kQDw0) {
         // Feature-map warps (bidir): f(q) in place, one row per thread.
@@ -859,7 +859,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             if (b == 0) bph ^= 1;
         }
         if (storer) tma_store_wait_all<0>();
-    } else {
+    } else if (warp < kQU2) {
         // Epilogue warps (every named barrier is reached by all 128 whatever the waits return).
         const int tid = threadIdx.x - kEw0 * 32;
         const int sub = warp & 3;
@@ -1386,7 +1386,7 @@ static la_status bwd_t(const void *q, const void *k, const void *v, const void *
         per_head = ms * kStateElems;
         single = 0;
     }
-    LA_TRY(launch_pdl(BIDIR ? "tc_bwd_q" : "tc_bwd_q_simple", bwd_q_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
+    LA_TRY(launch_pdl(BIDIR ? "tc_bwd_q" : "tc_bwd_q_simple", bwd_q_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kQThreads),
                   (size_t)BwdQLayout<BIDIR, BF16>::bytes, st, mq, mg, mdq, src, per_head, single, dpart, s.T, (int)s.BH(),
                   nt, ms, eps, state ? 0 : 1));
     return launch_pdl(BIDIR ? "tc_bwd_kv" : "tc_bwd_kv_simple", bwd_kv_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
@@ -1426,7 +1426,7 @@ static la_status stage_t(Stage stage, const void *x, const void *y, const float 
         LA_TRY(tensor_map(&mg, y, s, BF16));
         LA_TRY(tensor_map(&mdq, out1, s, BF16));
         LA_TRY(launch_pdl(BIDIR ? "tc_bwd_q" : "tc_bwd_q_simple", bwd_q_kernel<BIDIR, BF16>,
-                          dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads), (size_t)BwdQLayout<BIDIR, BF16>::bytes,
+                          dim3(grid_for((long long)s.BH() * nt)), dim3(kQThreads), (size_t)BwdQLayout<BIDIR, BF16>::bytes,
                           st, mq, mg, mdq, sin, kStateElems, 1, part, s.T, (int)s.BH(), nt, ms, eps, 0));
         return launch("tc_combine", combine_partials_kernel, dim3((unsigned)s.BH()), dim3(256), 0, st,
                       (const float *)part, sout, (int)s.BH(), nt, ms);
