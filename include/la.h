@@ -155,6 +155,22 @@ la_status la_chunk_decay_fwd(const void *q, const void *k, const void *v, void *
                              int B, int H, int T, int D, la_dtype dtype,
                              void *workspace, size_t workspace_bytes, void *stream);
 
+/* la_chunk_decay_fwd continuing from a state and handing its state on: with
+ * S_in the state of the tokens before this call (state_in, or zero if NULL),
+ *  o_t = q_t (gamma^(t+1) S_in + sum_{s<=t} gamma^(t-s) k_s^T v_s)
+ * and state_out (if not NULL) <- gamma^T S_in + sum_s gamma^(T-1-s) k_s^T v_s, the
+ * state after the last token (what la_chunk_decay_step continues from, or the
+ * next segment of the sequence starts with).  state_in, state_out: [B,H,D,D]
+ * fp32 device arrays, 16-byte aligned (row i = key index); they may alias. With
+ * T = 0 state_out <- state_in.  The library's addition for chunked prefill and
+ * for splitting a sequence into segments; source of the form as for
+ * la_chunk_decay_fwd ("flash-linear-attention" README, FusedChunk: the
+ * inter-chunk state carried from chunk to chunk). */
+la_status la_chunk_decay_fwd_state(const void *q, const void *k, const void *v, void *o,
+                                   const float *state_in, float *state_out, const float *decay,
+                                   int B, int H, int T, int D, la_dtype dtype,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
 /* Retention backward.  With R_s = sum_{t>=s} gamma^(t-s) q_t^T dout_t and
  * S_t = sum_{s<=t} gamma^(t-s) k_s^T v_s:
  *  dq_t = dout_t S_t^T,  dk_s = v_s R_s^T,  dv_s = k_s R_s.                   */

@@ -53,12 +53,13 @@ _lib.la_simple_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _
 _lib.la_chunk_decay_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_chunk_decay_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_chunk_decay_step.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]
+_lib.la_chunk_decay_fwd_state.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_state_reduce.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_state_apply.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
 _lib.la_state_bwd_q.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
 _lib.la_state_bwd_kv.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]
 for _n in ("la_bidir_fwd", "la_simple_fwd", "la_bidir_bwd", "la_simple_bwd", "la_chunk_decay_fwd",
-           "la_chunk_decay_bwd", "la_chunk_decay_step", "la_state_reduce", "la_state_apply", "la_state_bwd_q",
+           "la_chunk_decay_bwd", "la_chunk_decay_step", "la_chunk_decay_fwd_state", "la_state_reduce", "la_state_apply", "la_state_bwd_q",
            "la_state_bwd_kv"):
     getattr(_lib, _n).restype = _I
 _lib.la_bidir_fwd_static.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
@@ -226,6 +227,23 @@ def la_chunk_decay_fwd(q, k, v, o, decay, workspace=None, stream=None):
     wp, wn, _keep = _workspace("chunk_decay_fwd", (B, H, T, D), dt, workspace, q.device, stream)
     _check(_lib.la_chunk_decay_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.cast(dec, _P), B, H, T, D, dt,
                                    wp, wn, _stream(stream, q.device)), "la_chunk_decay_fwd")
+
+
+def la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=None, state_out=None, workspace=None, stream=None):
+    """la_chunk_decay_fwd continuing from state_in ([B, H, D, D] float32, zero if None) and
+    writing the state after the last token to state_out (if given); they may be the same tensor."""
+    import torch
+    B, H, T, D = _shape(q, k, v, o)
+    for st, name in ((state_in, "state_in"), (state_out, "state_out")):
+        if st is not None and (tuple(st.shape) != (B, H, D, D) or st.dtype != torch.float32 or not st.is_cuda
+                               or not st.is_contiguous() or st.device != q.device):
+            raise ValueError("%s must be a contiguous float32 CUDA tensor [B, H, D, D] on the inputs' device" % name)
+    dt = _dtype_code(q)
+    dec = _decay(decay, H)
+    wp, wn, _keep = _workspace("chunk_decay_fwd", (B, H, T, D), dt, workspace, q.device, stream)
+    _check(_lib.la_chunk_decay_fwd_state(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state_in), _ptr(state_out),
+                                         ctypes.cast(dec, _P), B, H, T, D, dt, wp, wn, _stream(stream, q.device)),
+           "la_chunk_decay_fwd_state")
 
 
 def la_chunk_decay_bwd(q, k, v, dout, decay, dq, dk, dv, workspace=None, stream=None):

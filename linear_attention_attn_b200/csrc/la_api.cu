@@ -301,21 +301,43 @@ la_status la_simple_bwd(const void *q, const void *k, const void *v, const void 
                            workspace_bytes, stream);
 }
 
-la_status la_chunk_decay_fwd(const void *q, const void *k, const void *v, void *o, const float *decay, int B, int H,
-                             int T, int D, la_dtype dtype, void *workspace, size_t workspace_bytes, void *stream) {
+static la_status decay_fwd_entry(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
+                                 const float *decay, int B, int H, int T, int D, la_dtype dtype, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
     const Shape s{B, H, T, D};
     LA_TRY(validate(s, dtype));
     LA_TRY(check_ptr(q, "q"));
     LA_TRY(check_ptr(k, "k"));
     LA_TRY(check_ptr(v, "v"));
     LA_TRY(check_ptr(o, "o"));
+    if (sin) LA_TRY(check_state(sin, "state_in"));
+    if (sout) LA_TRY(check_state(sout, "state_out"));
     DecayArgs dec;
     LA_TRY(decay_args(decay, H, &dec));
     LA_TRY(check_ws(LA_OP_CHUNK_DECAY_FWD, s, dtype, workspace, workspace_bytes));
-    if (T == 0) return LA_OK;
     cudaStream_t st = (cudaStream_t)stream;
-    if (path_tc(LA_OP_CHUNK_DECAY_FWD, s, dtype)) return tc::decay_fwd(q, k, v, o, dec, s, dtype, workspace, st);
-    return simt::decay_fwd(q, k, v, o, dec, s, dtype, st);
+    if (T == 0) {   // the state passes through unchanged
+        if (!sout) return LA_OK;
+        const size_t bytes = (size_t)s.BH() * D * D * sizeof(float);
+        cudaError_t e = sin ? (sin == sout ? cudaSuccess : cudaMemcpyAsync(sout, sin, bytes, cudaMemcpyDeviceToDevice, st))
+                            : cudaMemsetAsync(sout, 0, bytes, st);
+        return e == cudaSuccess ? LA_OK : cuda_fail(e, "state copy");
+    }
+    if (path_tc(LA_OP_CHUNK_DECAY_FWD, s, dtype))
+        return tc::decay_fwd(q, k, v, o, sin, sout, dec, s, dtype, workspace, st);
+    return simt::decay_fwd(q, k, v, o, sin, sout, dec, s, dtype, st);
+}
+
+la_status la_chunk_decay_fwd(const void *q, const void *k, const void *v, void *o, const float *decay, int B, int H,
+                             int T, int D, la_dtype dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    return decay_fwd_entry(q, k, v, o, nullptr, nullptr, decay, B, H, T, D, dtype, workspace, workspace_bytes, stream);
+}
+
+la_status la_chunk_decay_fwd_state(const void *q, const void *k, const void *v, void *o, const float *state_in,
+                                   float *state_out, const float *decay, int B, int H, int T, int D, la_dtype dtype,
+                                   void *workspace, size_t workspace_bytes, void *stream) {
+    return decay_fwd_entry(q, k, v, o, state_in, state_out, decay, B, H, T, D, dtype, workspace, workspace_bytes,
+                           stream);
 }
 
 la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const void *dout, const float *decay,

@@ -135,8 +135,8 @@ la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, voi
 la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, const void *g,
                     const float *state, void *dq, void *dk, void *dv, const Shape &s, la_dtype dt,
                     float eps, void *ws, cudaStream_t st);
-la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec,
-                    const Shape &s, la_dtype dt, cudaStream_t st);
+la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
+                    const DecayArgs &dec, const Shape &s, la_dtype dt, cudaStream_t st);
 la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec,
                     void *dq, void *dk, void *dv, const Shape &s, la_dtype dt, cudaStream_t st);
 la_status state_stage(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout,

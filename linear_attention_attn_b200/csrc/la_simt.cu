@@ -329,15 +329,15 @@ __device__ __forceinline__ void load_rows(const T *const (&src)[N], float (*dst)
 template <typename T, int D>
 __global__ void __launch_bounds__(D)
 ret_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, T *__restrict__ o,
-        DecayArgs dec, int T_len, int H) {
+        DecayArgs dec, int T_len, int H, const float *__restrict__ sin, float *__restrict__ sout) {
     __shared__ float tiles[3][kRetTile][D];
     const int bh = blockIdx.x;
     const float gamma = dec.gamma[bh % H];
     const long long base = (long long)bh * T_len * D;
     const int j = threadIdx.x;
-    float S[D];
+    float S[D];   // column j of the state (S[i] = S[i][j]); the entering state, or zero
 #pragma unroll
-    for (int i = 0; i < D; ++i) S[i] = 0.f;
+    for (int i = 0; i < D; ++i) S[i] = sin ? sin[((long long)bh * D + i) * D + j] : 0.f;
     const T *const src[3] = {q, k, v};
     for (int ts = 0; ts < T_len; ts += kRetTile) {
         __syncthreads();
@@ -354,6 +354,10 @@ ret_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ 
             }
             io<T>::st(o + base + (long long)(ts + r) * D + j, acc);
         }
+    }
+    if (sout) {
+#pragma unroll
+        for (int i = 0; i < D; ++i) sout[((long long)bh * D + i) * D + j] = S[i];
     }
 }
 
@@ -576,9 +580,10 @@ la_status state_bwd_d(bool bidir, const void *q, const void *k, const void *v, c
 }
 
 template <typename T, int D>
-la_status decay_fwd_t(const T *q, const T *k, const T *v, T *o, const DecayArgs &dec, const Shape &s,
-                      cudaStream_t st) {
-    return launch("simt_ret_fwd", ret_fwd<T, D>, dim3((unsigned)s.BH()), dim3(D), 0, st, q, k, v, o, dec, s.T, s.H);
+la_status decay_fwd_t(const T *q, const T *k, const T *v, T *o, const float *sin, float *sout, const DecayArgs &dec,
+                      const Shape &s, cudaStream_t st) {
+    return launch("simt_ret_fwd", ret_fwd<T, D>, dim3((unsigned)s.BH()), dim3(D), 0, st, q, k, v, o, dec, s.T, s.H,
+                  sin, sout);
 }
 
 template <typename T, int D>
@@ -636,11 +641,11 @@ la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, con
     }
 }
 
-la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, const Shape &s,
-                    la_dtype dt, cudaStream_t st) {
-#define LA_RET_FWD(TY)                                                                                     \
-    return s.D == 64 ? decay_fwd_t<TY, 64>((const TY *)q, (const TY *)k, (const TY *)v, (TY *)o, dec, s, st) \
-                     : decay_fwd_t<TY, 128>((const TY *)q, (const TY *)k, (const TY *)v, (TY *)o, dec, s, st)
+la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
+                    const DecayArgs &dec, const Shape &s, la_dtype dt, cudaStream_t st) {
+#define LA_RET_FWD(TY)                                                                                                 \
+    return s.D == 64 ? decay_fwd_t<TY, 64>((const TY *)q, (const TY *)k, (const TY *)v, (TY *)o, sin, sout, dec, s, st) \
+                     : decay_fwd_t<TY, 128>((const TY *)q, (const TY *)k, (const TY *)v, (TY *)o, sin, sout, dec, s, st)
     switch (dt) {
     case LA_F32: LA_RET_FWD(float);
     case LA_F16: LA_RET_FWD(__half);

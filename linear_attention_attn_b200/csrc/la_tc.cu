@@ -39,9 +39,9 @@ size_t workspace_size(la_op op, const Shape &s, la_dtype) {
     }
 }
 
-la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, const Shape &s,
-                    la_dtype, void *, cudaStream_t st) {
-    return retention_fwd(q, k, v, o, dec, s, st);
+la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
+                    const DecayArgs &dec, const Shape &s, la_dtype, void *, cudaStream_t st) {
+    return retention_fwd(q, k, v, o, sin, sout, dec, s, st);
 }
 la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec, void *dq,
                     void *dk, void *dv, const Shape &s, la_dtype, void *, cudaStream_t st) {

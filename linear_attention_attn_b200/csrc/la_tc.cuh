@@ -21,8 +21,8 @@ unsigned int read_and_clear_retention_fault();
 la_status make_tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16, int box_rows);
 la_status retention_map(CUtensorMap *m, const void *ptr, const Shape &s);
 // Chunked causal decay forward on tensor cores (bf16, D = 128).
-la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, const Shape &s,
-                        cudaStream_t st);
+la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
+                        const DecayArgs &dec, const Shape &s, cudaStream_t st);
 la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec, void *dq,
                         void *dk, void *dv, const Shape &s, cudaStream_t st);
 la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, void *o, float *state,
@@ -30,8 +30,8 @@ la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, voi
 la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, const void *g,
                     const float *state, void *dq, void *dk, void *dv, const Shape &s, la_dtype dt,
                     float eps, void *ws, cudaStream_t st);
-la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec,
-                    const Shape &s, la_dtype dt, void *ws, cudaStream_t st);
+la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
+                    const DecayArgs &dec, const Shape &s, la_dtype dt, void *ws, cudaStream_t st);
 // One stage of the state form (Stage in la_internal.cuh).
 la_status state_stage(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout,
                       void *out1, void *out2, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);

@@ -88,6 +88,8 @@ struct RetLayout {
 struct RetJobs {
     CUtensorMap q[3], k[3], v[3], o[3];
     int rev[3];
+    const float *sin;    // pass 0 (forward in time): state entering the sequence [BH, D, D], or null (zero)
+    float *sout;         // pass 0: state after the sequence [BH, D, D], or null
 };
 
 // Grid: one CTA per (pass, b, h), pass = blockIdx.x / BH.  decay[h] = gamma_h.
@@ -300,7 +302,10 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             if (got && it > 0) got = LA_RWAIT(dsfull, pc ^ 1u, 0x200u);   // K^ buffer free
             got = __all_sync(0xffffffffu, got);
             if (!got) break;
-            const float f = rev ? gpow[krow] : gpow[kC - 1 - krow];
+            // forwards in time the weights count back from the chunk's last valid row, so
+            // that the state after a partial last chunk is the state after token T - 1
+            const int rows = min(kC, T - (rev ? nchunks - 1 - it : it) * kC);
+            const float f = rev ? gpow[krow] : (krow < rows ? gpow[rows - 1 - krow] : 0.f);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int ch = part * 8 + i;               // 0..15 across the two boxes
@@ -402,24 +407,48 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         const uint32_t lanes = (uint32_t)(32 * sub) << 16;
         const int d = 32 * sub + lane;
         const float gC = gpow[kC];
+        const float gLast = gpow[min(kC, T - (nchunks - 1) * kC)];   // decay over a partial last chunk
         float st[64];
+        const float *sin = pass == 0 ? jobs.sin : nullptr;
+        float *sout = pass == 0 ? jobs.sout : nullptr;
+        const long long srow = ((long long)bh * 128 + d) * 128 + 64 * half;   // this thread's 64 state entries
+        if (sin) {   // S_0 given: registers and the hi + lo operand of the first Q S
 #pragma unroll
-        for (int i = 0; i < 64; ++i) st[i] = 0.f;
+            for (int c4 = 0; c4 < 16; ++c4) {
+                const float4 x = *reinterpret_cast<const float4 *>(sin + srow + 4 * c4);
+                st[4 * c4] = x.x;
+                st[4 * c4 + 1] = x.y;
+                st[4 * c4 + 2] = x.z;
+                st[4 * c4 + 3] = x.w;
+            }
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                uint32_t hw[8], lw[8];
+                split_hi_lo16_packed(*reinterpret_cast<const float(*)[16]>(&st[16 * c4]), hw, lw);
+                store_chunk16_packed(sS + half * 16384, d, c4, hw);
+                store_chunk16_packed(sS + 32768 + half * 16384, d, c4, lw);
+            }
+            fence_async_smem();
+        } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) st[i] = 0.f;
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(sready);                // S_0 (zeroed above)
+        if (lane == 0) mbar_arrive(sready);                // S_0
         for (int it = 0; it < nchunks; ++it) {
             const uint32_t pc = (uint32_t)(it & 1);
             bool got = __all_sync(0xffffffffu, LA_RWAIT(dsfull, pc, 0x1000u));
             if (!got) break;
             tc_fence_after();
             const uint32_t base = tmem + cDS + lanes + 64u * half;
+            const float g = (!rev && it == nchunks - 1) ? gLast : gC;
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
                 float a[16];
                 tmem_ld16(base + 16 * c4, a);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) st[16 * c4 + i] = fmaf(gC, st[16 * c4 + i], a[i]);
+                for (int i = 0; i < 16; ++i) st[16 * c4 + i] = fmaf(g, st[16 * c4 + i], a[i]);
             }
             tc_fence_before();
             __syncwarp();
@@ -437,6 +466,12 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(sready);
+        }
+        if (sout && !*s_abort) {   // S after the last chunk
+#pragma unroll
+            for (int c4 = 0; c4 < 16; ++c4)
+                *reinterpret_cast<float4 *>(sout + srow + 4 * c4) =
+                    make_float4(st[4 * c4], st[4 * c4 + 1], st[4 * c4 + 2], st[4 * c4 + 3]);
         }
     }
     tc_fence_before();
@@ -457,10 +492,12 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
 
 }  // namespace
 
-la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, const Shape &s,
-                        cudaStream_t st) {
+la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
+                        const DecayArgs &dec, const Shape &s, cudaStream_t st) {
     RetJobs jobs;
     memset(&jobs, 0, sizeof jobs);
+    jobs.sin = sin;
+    jobs.sout = sout;
     LA_TRY(retention_map(&jobs.q[0], q, s));
     LA_TRY(retention_map(&jobs.k[0], k, s));
     LA_TRY(retention_map(&jobs.v[0], v, s));

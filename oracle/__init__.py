@@ -60,9 +60,10 @@ def _bind(lib):
     lib.oracle_retention_fwd.argtypes = [P, P, P, P, P, L, L, L, L, I]
     lib.oracle_retention_bwd.argtypes = [P, P, P, P, P, P, P, P, L, L, L, L, I]
     lib.oracle_retention_step.argtypes = [P, P, P, P, P, P, L, L, L]
+    lib.oracle_retention_fwd_state.argtypes = [P, P, P, P, P, P, P, L, L, L, L, I]
     for name in ("oracle_bidir_fwd", "oracle_simple_fwd", "oracle_bidir_bwd",
                  "oracle_simple_bwd", "oracle_retention_fwd", "oracle_retention_bwd",
-                 "oracle_retention_step"):
+                 "oracle_retention_step", "oracle_retention_fwd_state"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -177,6 +178,24 @@ class Oracle:
         _check(rc, "oracle_retention_bwd")
         return dq, dk, dv
 
+    def retention_fwd_state(self, q, k, v, gamma, state_in=None, nthreads: int | None = None):
+        """retention_fwd starting from state_in ([B, H, D, D], zero if None); returns
+        (o, state after the last token)."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, H, T, D = _shape4(q)
+        gm = _f64(gamma).reshape(-1)
+        if gm.shape[0] != H:
+            raise ValueError("gamma must have H=%d entries" % H)
+        sin = None if state_in is None else np.ascontiguousarray(_f64(state_in))
+        if sin is not None and sin.shape != (B, H, D, D):
+            raise ValueError("state_in must be [B, H, D, D]")
+        o = np.empty_like(q)
+        sout = np.empty((B, H, D, D))
+        rc = self._lib.oracle_retention_fwd_state(_p(q), _p(k), _p(v), _p(gm), None if sin is None else _p(sin),
+                                                 _p(o), _p(sout), B, H, T, D, nthreads or default_threads())
+        _check(rc, "oracle_retention_fwd_state")
+        return o, sout
+
     def retention_step(self, q, k, v, gamma, state):
         """One decode step: returns (o, new_state) with new_state = gamma_h state + k^T v and
         o = q new_state; q, k, v are [B, H, D], state is [B, H, D, D] (not modified)."""
@@ -237,3 +256,7 @@ def retention_bwd(*a, **kw):
 
 def retention_step(*a, **kw):
     return _instance().retention_step(*a, **kw)
+
+
+def retention_fwd_state(*a, **kw):
+    return _instance().retention_fwd_state(*a, **kw)

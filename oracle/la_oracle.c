@@ -59,6 +59,8 @@ typedef struct {
     const double *q, *k, *v, *g;   /* g = upstream gradient dO (bwd only) */
     double *o, *state, *dq, *dk, *dv;
     const double *gamma;           /* [H] (retention only) */
+    const double *state_in;        /* [B, H, D, D] state entering the sequence, or NULL (retention fwd) */
+    double *state_out;             /* [B, H, D, D] state after the last token, or NULL (retention fwd) */
     long B, H, T, D;
     double eps;
     int use_phi, use_norm;
@@ -282,7 +284,10 @@ static void retention_fwd_head(job_t *jb, long bh, double *scratch) {
     const double *q = jb->q + off, *k = jb->k + off, *v = jb->v + off;
     double *o = jb->o + off;
     double *S = scratch;
-    memset(S, 0, (size_t)(D * D) * sizeof(double));
+    if (jb->state_in)
+        memcpy(S, jb->state_in + bh * D * D, (size_t)(D * D) * sizeof(double));
+    else
+        memset(S, 0, (size_t)(D * D) * sizeof(double));
     for (long t = 0; t < T; ++t) {
         for (long i = 0; i < D; ++i)
             for (long j = 0; j < D; ++j)
@@ -293,6 +298,7 @@ static void retention_fwd_head(job_t *jb, long bh, double *scratch) {
             o[t * D + j] = a;
         }
     }
+    if (jb->state_out) memcpy(jb->state_out + bh * D * D, S, (size_t)(D * D) * sizeof(double));
 }
 
 /* Backward, one head.
@@ -366,6 +372,20 @@ int oracle_retention_step(const double *q, const double *k, const double *v, con
         }
     }
     return 0;
+}
+
+/* oracle_retention_fwd from a given state: S starts at state_in (zero if NULL)
+ * instead of zero, and the state after the last token goes to state_out (if not
+ * NULL).  Arrays [B, H, D, D]. */
+int oracle_retention_fwd_state(const double *q, const double *k, const double *v, const double *gamma,
+                               const double *state_in, double *o, double *state_out,
+                               long B, long H, long T, long D, int nthreads) {
+    if (check_dims(B, H, T, D) || (T > 0 && (!q || !k || !v || !o)) || !gamma) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.gamma = gamma; jb.o = o;
+    jb.state_in = state_in; jb.state_out = state_out;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D;
+    return for_each_head(&jb, retention_fwd_head, (size_t)(D * D), nthreads);
 }
 
 int oracle_retention_bwd(const double *q, const double *k, const double *v, const double *dout,

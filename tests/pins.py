@@ -330,5 +330,27 @@ def check_decode_step(orc):
         _close(o, want[:, :, t], rtol=1e-11, atol=1e-12, what="step %d after a prefix state" % t)
 
 
+def check_state_segments(orc):
+    """The forward from a given state: o_t = pairwise output + gamma^(t+1) q_t S_in, the state
+    after T tokens is gamma^T S_in + sum_s gamma^(T-1-s) k_s^T v_s, and two segments chained
+    through the state give the whole sequence."""
+    B, H, T, D = 2, 3, 11, 5
+    q, k, v = _rand((B, H, T, D), 51), _rand((B, H, T, D), 52), _rand((B, H, T, D), 53)
+    gam = np.array([0.5, 0.9, 1.0])
+    sin = _rand((B, H, D, D), 54)
+    o, sout = orc.retention_fwd_state(q, k, v, gam, sin)
+    decay_t = gam[None, :, None] ** (np.arange(T) + 1)[None, None, :]            # gamma^(t+1)
+    want = brute_retention(q, k, v, gam) + decay_t[..., None] * np.einsum("bhti,bhij->bhtj", q, sin)
+    _close(o, want, rtol=1e-11, atol=1e-12, what="fwd from a state")
+    w = gam[None, :, None] ** (T - 1 - np.arange(T))[None, None, :]
+    want_s = (gam ** T)[None, :, None, None] * sin + np.einsum("bhs,bhsi,bhsj->bhij", w, k, v)
+    _close(sout, want_s, rtol=1e-12, atol=1e-12, what="state after the sequence")
+    p = 4
+    o1, s1 = orc.retention_fwd_state(q[:, :, :p], k[:, :, :p], v[:, :, :p], gam)
+    o2, s2 = orc.retention_fwd_state(q[:, :, p:].copy(), k[:, :, p:].copy(), v[:, :, p:].copy(), gam, s1)
+    _close(np.concatenate([o1, o2], axis=2), orc.retention_fwd(q, k, v, gam), rtol=1e-12, atol=1e-12,
+           what="two segments vs the whole")
+
+
 ALL_CHECKS = (check_golden, check_brute, check_closed_forms, check_invariances,
-              check_fd_gradients, check_autograd, check_decode_step)
+              check_fd_gradients, check_autograd, check_decode_step, check_state_segments)

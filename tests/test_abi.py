@@ -26,7 +26,7 @@ def declared_functions():
 def test_header_declares_the_api():
     names = declared_functions()
     for n in ("la_bidir_fwd", "la_bidir_bwd", "la_simple_fwd", "la_simple_bwd", "la_chunk_decay_fwd",
-              "la_chunk_decay_bwd", "la_chunk_decay_step", "la_workspace_size", "la_status_string", "la_last_error"):
+              "la_chunk_decay_bwd", "la_chunk_decay_step", "la_chunk_decay_fwd_state", "la_workspace_size", "la_status_string", "la_last_error"):
         assert n in names
 
 

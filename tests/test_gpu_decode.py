@@ -78,3 +78,60 @@ def test_decode_rejects_bad_state_shape():
     q = torch.zeros((1, 2, 64), dtype=torch.bfloat16, device=dev)
     with pytest.raises(ValueError):
         la.la_chunk_decay_step(q, q, q, torch.empty_like(q), torch.zeros((1, 2, 64, 65), device=dev), [0.5, 0.5])
+
+
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f16", 64), ("f32", 128)])
+def test_forward_from_a_state(dtype, D):
+    """A random entering state: outputs and the state after the sequence against the oracle."""
+    import linear_attention_attn_b200 as la
+    w = synth.Workload("case", "retention", 2, 3, 300, D, dtype, q_scale=D ** -0.5)
+    inp = synth.make_inputs(w, seed=6, with_grad=False)
+    dev = torch.device("cuda", 0)
+    sin = synth.normal((w.B, w.H, D, D), 8, 0) * (D ** -0.5)
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    sout = torch.empty_like(sin, device=dev)
+    la.la_chunk_decay_fwd_state(q, k, v, o, inp["gamma"], state_in=sin.to(dev), state_out=sout)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.retention_fwd_state(inp["q"], inp["k"], inp["v"], inp["gamma"], sin.double().numpy())
+    pu.assert_fwd(o.cpu().double().numpy(), o_ref, "o from a state")
+    assert _rel_l2(sout.cpu().numpy(), s_ref) <= 2e-3
+
+
+def test_segments_chained_through_the_state():
+    """Two segments of one sequence, the second starting from the first's state (the same
+    buffer in and out), match the op on the whole sequence."""
+    import linear_attention_attn_b200 as la
+    w = synth.Workload("case", "retention", 2, 4, 700, 128, "bf16", q_scale=128 ** -0.5)
+    inp = synth.make_inputs(w, seed=9, with_grad=False)
+    dev = torch.device("cuda", 0)
+    cut = 257
+    st = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+    outs = []
+    for a, b, sin in ((0, cut, None), (cut, w.T, st)):
+        q, k, v = (inp[n][:, :, a:b].contiguous().to(dev) for n in ("q", "k", "v"))
+        o = torch.empty_like(q)
+        la.la_chunk_decay_fwd_state(q, k, v, o, inp["gamma"], state_in=sin, state_out=st)
+        outs.append(o)
+    torch.cuda.synchronize()
+    got = torch.cat(outs, dim=2).cpu().double().numpy()
+    pu.assert_fwd(got, oracle.retention_fwd(inp["q"], inp["k"], inp["v"], inp["gamma"]), "two segments")
+
+
+def test_prefill_then_decode():
+    """Chunked prefill of T tokens hands its state to the decode step for token T + 1."""
+    import linear_attention_attn_b200 as la
+    w = synth.Workload("case", "retention", 2, 4, 401, 128, "bf16", q_scale=128 ** -0.5)
+    inp = synth.make_inputs(w, seed=10, with_grad=False)
+    dev = torch.device("cuda", 0)
+    T = w.T - 1
+    q, k, v = (inp[n][:, :, :T].contiguous().to(dev) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    st = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+    la.la_chunk_decay_fwd_state(q, k, v, o, inp["gamma"], state_out=st)
+    o1 = torch.empty((w.B, w.H, w.D), dtype=q.dtype, device=dev)
+    la.la_chunk_decay_step(*(inp[n][:, :, T].contiguous().to(dev) for n in ("q", "k", "v")), o1, st, inp["gamma"])
+    torch.cuda.synchronize()
+    full = oracle.retention_fwd(inp["q"], inp["k"], inp["v"], inp["gamma"])
+    pu.assert_fwd(o.cpu().double().numpy(), full[:, :, :T], "prefill")
+    pu.assert_fwd(o1.cpu().double().numpy(), full[:, :, T], "decode after prefill")

@@ -40,6 +40,9 @@ MUTATIONS = [
     ("step_output_transposed", "a += qh[i] * Sh[i * D + j];", "a += qh[i] * Sh[j * D + i];", 0),
     ("step_outer_product_transposed", "+ kh[i] * vh[j];", "+ kh[j] * vh[i];", 0),
     ("step_gamma_head_index", "const double g = gamma[bh % H];", "const double g = gamma[0];", 0),
+    ("fwd_state_in_ignored", "    if (jb->state_in)\n", "    if (0)\n", 0),
+    ("fwd_state_out_before_last_token", "    if (jb->state_out) memcpy(jb->state_out + bh * D * D, S,",
+     "    if (jb->state_out) memcpy(jb->state_out + bh * D * D, jb->state_in ? jb->state_in + bh * D * D : S,", 0),
 ]
 
 
