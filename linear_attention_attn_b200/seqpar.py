@@ -44,3 +44,43 @@ def backward(q, k, v, dout, state, dq, dk, dv, dstate, feature="elu1", eps: floa
     _all_reduce(dstate, group)
     la_state_bwd_kv(k, v, dstate, dk, dv, feature=feature, stream=stream)
     return dstate
+
+
+def decay_forward(q, k, v, o, decay, state_out=None, group=None, ops=None, stream=None, workspace=None):
+    """The decay op (retention) forward for this rank's segment of a sequence split along T
+    (rank r holds the r-th segment).  A segment's output needs the state of every token before
+    it: pass 1 gives each segment's own end state E_r (from a zero state), an all-gather shares
+    them with the segment lengths, rank r forms S_r = sum_{r' < r} (prod of gamma^T over the
+    segments between) E_r' as the running state gamma^{T_r'} S + E_r', and pass 2 recomputes the
+    segment from S_r.  state_out (optional, [B, H, D, D] fp32) receives the state after this
+    rank's segment (on the last rank: after the whole sequence)."""
+    import torch
+    if ops is None:
+        from linear_attention_attn_b200 import la_chunk_decay_fwd_state
+    else:
+        la_chunk_decay_fwd_state = ops.la_chunk_decay_fwd_state
+    import torch.distributed as dist
+    B, H, T, D = (int(x) for x in q.shape)
+    kw = {} if workspace is None else {"workspace": workspace}
+    end = torch.empty((B, H, D, D), dtype=torch.float32 if q.is_cuda else torch.float64, device=q.device)
+    la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=None, state_out=end, stream=stream, **kw)
+    world = dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
+    if world == 1:
+        if state_out is not None:
+            state_out.copy_(end)
+        return state_out
+    rank = dist.get_rank(group)
+    ends = [torch.empty_like(end) for _ in range(world)]
+    dist.all_gather(ends, end, group=group)
+    lens = torch.tensor([T], dtype=torch.int64, device=end.device)
+    all_lens = [torch.empty_like(lens) for _ in range(world)]
+    dist.all_gather(all_lens, lens, group=group)
+    gam = torch.as_tensor([float(x) for x in (decay.tolist() if hasattr(decay, "tolist") else decay)],
+                          dtype=torch.float64)
+    state = torch.zeros((B, H, D, D), dtype=torch.float64, device=end.device)
+    for r in range(rank):
+        f = torch.pow(gam, float(all_lens[r].item())).to(end.device)
+        state = f[None, :, None, None] * state + ends[r].to(torch.float64)
+    sin = state.to(end.dtype).contiguous()
+    la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=sin, state_out=state_out, stream=stream, **kw)
+    return state_out

@@ -123,3 +123,55 @@ def test_two_ranks_match_the_whole_sequence(feature):
     for i, name in enumerate(("o", "dq", "dk", "dv")):
         got = np.concatenate([out[0][i], out[1][i]], axis=2)
         np.testing.assert_allclose(got, want[i], rtol=1e-10, atol=1e-12, err_msg=name)
+
+
+def _decay_ops():
+    """la_chunk_decay_fwd_state on float64 CPU tensors: the recurrent form, from its definition."""
+    def la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=None, state_out=None, stream=None):
+        B, H, T, D = q.shape
+        g = torch.as_tensor(list(decay), dtype=torch.float64)[None, :, None, None]
+        S = state_in.clone() if state_in is not None else torch.zeros(B, H, D, D, dtype=torch.float64)
+        for t in range(T):
+            S = g * S + torch.einsum("bhi,bhj->bhij", k[:, :, t], v[:, :, t])
+            o[:, :, t] = torch.einsum("bhi,bhij->bhj", q[:, :, t], S)
+        if state_out is not None:
+            state_out.copy_(S)
+    return types.SimpleNamespace(la_chunk_decay_fwd_state=la_chunk_decay_fwd_state)
+
+
+def _decay_rank_main(rank, world, port, cuts, gam, out):
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    from linear_attention_attn_b200 import seqpar
+    q, k, v, _ = _inputs(2, 3, cuts[-1], 6)
+    sl = slice(cuts[rank], cuts[rank + 1])
+    qs, ks, vs = (x[:, :, sl].contiguous() for x in (q, k, v))
+    o = torch.empty_like(qs)
+    st = torch.empty(2, 3, 6, 6, dtype=torch.float64)
+    seqpar.decay_forward(qs, ks, vs, o, gam, state_out=st, ops=_decay_ops())
+    out[rank] = (o.numpy(), st.numpy())
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_decay_forward_over_three_ranks():
+    import oracle
+    cuts = [0, 7, 19, 30]
+    gam = [0.6, 0.9, 1.0]
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_decay_rank_main, args=(r, 3, port, cuts, gam, out)) for r in range(3)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    q, k, v, _ = (x.numpy() for x in _inputs(2, 3, cuts[-1], 6))
+    want_o, want_s = oracle.retention_fwd_state(q, k, v, np.array(gam))
+    got = np.concatenate([out[r][0] for r in range(3)], axis=2)
+    np.testing.assert_allclose(got, want_o, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(out[2][1], want_s, rtol=1e-10, atol=1e-12)    # the last rank: whole sequence
