@@ -361,6 +361,17 @@ __device__ __forceinline__ float operand_scale(float m) {
     return ldexpf(1.f, e);
 }
 
+// This worker thread's max |stage[e]| over the float4s gather_state would have given it.
+__device__ __forceinline__ float stage_absmax(const float *stage, int tid) {
+    const float4 *st4 = reinterpret_cast<const float4 *>(stage);
+    float m = 0.f;
+    for (int e = tid; e < kStateElems / 4; e += kWorkers) {
+        const float4 a = st4[e];
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+    }
+    return m;
+}
+
 // Two-term bf16 split of 16 fp32 values, packed in pairs: hi = round(x),
 // lo = round(x - hi) (x - hi is exact in fp32).
 __device__ __forceinline__ void split_hi_lo16_packed(const float (&x)[16], uint32_t (&hw)[8], uint32_t (&lw)[8]) {

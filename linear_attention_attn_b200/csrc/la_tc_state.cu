@@ -551,7 +551,7 @@ struct BwdQLayout {
     static constexpr int rioff = iscoff + 16;                        // [2][128] (g.o, 1/n) per row
     static constexpr int redoff = rioff + 2 * 128 * 8;
     static constexpr int baroff = redoff + 32;
-    static constexpr int nbars = 4 * NST + 9;
+    static constexpr int nbars = 4 * NST + 10;
     static constexpr int misc = baroff + nbars * 8;
     static constexpr int bytes = misc + 32 + 1024;
     static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
@@ -593,6 +593,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     uint64_t *opready = accSfree + 1;
     uint64_t *drain = opready + 1;
     uint64_t *drain2 = drain + 1;
+    uint64_t *stfull = drain2 + 1;       // the first head's state copied into the staging block
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc);
     int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
 
@@ -618,6 +619,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         mbar_init(opready, 1);
         mbar_init(drain, 1);
         mbar_init(drain2, 1);
+        mbar_init(stfull, 1);
         *s_abort = 0;
         fence_mbar_init();
     }
@@ -655,6 +657,10 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             int s = 0;
             uint32_t ph = 0;
             long long issued = 0;
+            if (src_single) {   // the first head's state, ahead of the tile stream
+                mbar_arrive_expect_tx(stfull, kStateElems * 4);
+                bulk_load(stage, src + (x0 / nt) * (long long)src_per_head, kStateElems * 4, stfull);
+            }
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
                 const long long x = t.x;
                 const int h = t.h, j = t.j;
@@ -668,6 +674,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             if (*s_abort) {
                 for (long long i = issued - 1; i >= 0 && i >= issued - NST; --i)
                     mbar_wait_slow(smem_u32(&full[i % NST]), (uint32_t)((i / NST) & 1), nullptr, &g_tc_fault, 0x200u);
+                if (src_single) mbar_wait_slow(smem_u32(stfull), 0, nullptr, &g_tc_fault, 0x200u);
             }
         }
     } else if (warp == 1) {
@@ -871,10 +878,17 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         float cur_sc = 1.f, cur_scn = 1.f;
 
         float *isc3 = reinterpret_cast<float *>(smem + L::iscoff);
+        int hidx = -1;
         auto build = [&](long long h, int zb) {
             const float *srch = src + h * (long long)src_per_head;
             const int ns = src_single ? 1 : (P.last_cta((int)h) - P.first_cta((int)h) + 1);
-            float m = gather_state(srch, ns, stage, tid);
+            float m;
+            if (src_single && hidx == 0) {   // copied by the TMA thread at the start
+                if (!LA_WAIT(stfull, 0, 0x800u)) live = false;
+                m = stage_absmax(stage, tid);
+            } else {
+                m = gather_state(srch, ns, stage, tid);
+            }
             named_bar(1, kWorkers);
             if (!BF16) m = workers_max(m, red, tid);
             const float sc = operand_scale<BF16>(m);
@@ -936,7 +950,6 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         };
 
         float2 *rinfo = reinterpret_cast<float2 *>(smem + L::rioff);
-        int hidx = -1;
         for (TileCursor t(x0, nt); t.x < x1; t.next()) {
             const long long x = t.x;
             const long long h = t.h;
