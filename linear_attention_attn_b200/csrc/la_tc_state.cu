@@ -152,7 +152,6 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             uint32_t ph = 0;
             long long issued = 0;
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
                 const int h = t.h, j = t.j;
                 if (!LA_WAIT(&empty[s], ph ^ 1, 0x1u)) break;
                 mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
@@ -173,7 +172,6 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             bool seg_start = true;
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
                 const long long x = t.x;
-                const long long h = t.h;
                 const bool seg_end = (x + 1 == x1) || t.last_of_head();
                 if (seg_start) {
                     if (!LA_WAIT(&accfree[a], aph ^ 1, 0x2u)) break;
@@ -210,7 +208,6 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             int s = 0;
             uint32_t ph = 0;
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
                 const int j = t.j;
                 const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
                 if (!got) break;
@@ -367,7 +364,6 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             uint32_t ph = 0;
             long long issued = 0;
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
                 const int h = t.h, j = t.j;
                 if (!LA_WAIT(&empty[s], ph ^ 1, 0x1u)) break;
                 mbar_arrive_expect_tx(&full[s], kTileBytes);
@@ -386,7 +382,6 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             uint32_t ph = 0, aph = 0;
             long long prev_h = -1;
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
                 const long long h = t.h;
                 if (h != prev_h) {
                     ++hidx;
@@ -421,7 +416,6 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             int s = 0;
             uint32_t ph = 0;
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
                 const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
                 if (!got) break;
                 phi_half_row<BF16>(sQ + s * kTileBytes, xi, false);   // rows past T are never stored
@@ -662,7 +656,6 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 bulk_load(stage, src + (x0 / nt) * (long long)src_per_head, kStateElems * 4, stfull);
             }
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
                 const int h = t.h, j = t.j;
                 if (!LA_WAIT(&empty[s], ph ^ 1, 0x1u)) break;
                 mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
@@ -682,7 +675,6 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             int s = 0, b = 0;
             uint32_t ph = 0, bph = 0, oph = 0;
             long long prev_h = -1;
-            long long seg = 0;                     // segments started (accS free parity)
             bool dead = false;
             for (TileCursor t(x0, nt); t.x < x1 && !dead; t.next()) {
                 const long long h = t.h;
@@ -1114,7 +1106,6 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             uint32_t ph = 0;
             long long issued = 0;
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
                 const int h = t.h, j = t.j;
                 if (!LA_WAIT(&empty[s], ph ^ 1, 0x1u)) break;
                 mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
@@ -1134,7 +1125,6 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             uint32_t ph = 0, bph = 0, oph = 0;
             long long prev_h = -1;
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
                 const long long h = t.h;
                 if (h != prev_h) {
                     if (!LA_WAIT(opready, oph, 0x20u)) break;
@@ -1174,7 +1164,6 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             int s = 0;
             uint32_t ph = 0;
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
                 const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
                 if (!got) break;
                 phi_half_row<BF16>(sK + s * kTileBytes, xi, false);
@@ -1194,7 +1183,6 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
         bool live = true;
         float cur_isd = 1.f;
         for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
             const long long h = t.h;
             const int j = t.j;
             if (h != cur_h) {
