@@ -84,6 +84,9 @@ typedef enum { LA_FEATURE_IDENTITY = 0, LA_FEATURE_ELU1 = 1 } la_feature;
 /* Largest H accepted by la_chunk_decay_* (the decays travel as kernel arguments). */
 #define LA_MAX_DECAY_HEADS 512
 
+/* Most segments la_chunk_decay_scan combines in one call. */
+#define LA_MAX_SCAN_SEGMENTS 128
+
 /* Bytes of device workspace the call `op` needs for this shape (0 if none).
  * Depends only on its arguments.  Returns 0 for invalid arguments too. */
 size_t la_workspace_size(la_op op, int B, int H, int T, int D, la_dtype dtype);
@@ -178,6 +181,50 @@ la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const 
                              const float *decay, void *dq, void *dk, void *dv,
                              int B, int H, int T, int D, la_dtype dtype,
                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* la_chunk_decay_bwd of one segment of a longer sequence, the backward of
+ * la_chunk_decay_fwd_state.  Rows t = 0..T-1 are the segment's; S_in (state_in,
+ * or zero if NULL) is the state of the tokens before it and R_in (dstate_in, or
+ * zero if NULL) = sum_{u after the segment} gamma^(u-T) q_u^T dout_u comes from the
+ * tokens after it (u counted from the segment's first row).  Then
+ *  S_t = gamma^(t+1) S_in + sum_{s<=t} gamma^(t-s) k_s^T v_s,
+ *  R_s = gamma^(T-s) R_in + sum_{s<=t<T} gamma^(t-s) q_t^T dout_t,
+ *  dq_t = dout_t S_t^T,  dk_s = v_s R_s^T,  dv_s = k_s R_s,
+ * and dstate_out (if not NULL) <- R_0, the dstate_in of the segment before this
+ * one.  The gradient of the loss with respect to state_in is gamma R_0.  All
+ * three are [B,H,D,D] fp32 device arrays, 16-byte aligned, row i = the index
+ * of q (R) or k (S); dstate_out must not overlap state_in or dstate_in
+ * (LA_ERR_INVALID_ARG).  dq may be NULL: then only dk and dv are computed
+ * (state_in is not read).  With T = 0, dstate_out <- dstate_in.  The library's
+ * addition for splitting a sequence into segments (the reverse-time
+ * recurrence is the backward of the FusedChunk form, "flash-linear-attention"
+ * README). */
+la_status la_chunk_decay_bwd_state(const void *q, const void *k, const void *v, const void *dout,
+                                   const float *state_in, const float *dstate_in, float *dstate_out,
+                                   const float *decay, void *dq, void *dk, void *dv,
+                                   int B, int H, int T, int D, la_dtype dtype,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Combine of per-segment states for a sequence split into n segments:
+ *   out[b,h] = sum over i < n with gaps[i] >= 0 of decay[h]^gaps[i] states[i,b,h],
+ * summed in the order i = 0, 1, ... in fp32 (deterministic).  With E_i the
+ * state_out of la_chunk_decay_fwd_state on segment i from a zero state, and
+ * gaps[i] = the number of tokens strictly between segment i and segment r (-1
+ * for i >= r), out is the state_in of segment r.  With F_i the dstate_out of
+ * la_chunk_decay_bwd_state on segment i from a zero dstate_in, and gaps[i] = the
+ * number of tokens strictly between segment r and segment i (-1 for i <= r),
+ * out is the dstate_in of segment r.  Both follow from the recurrent form: a
+ * span of L tokens maps a state S to gamma^L S + (the span's own state)
+ * ("flash-linear-attention" README, FusedRecurrent).  The library's addition
+ * for sequence parallelism (one segment per rank, the states all-gathered).
+ *  states  in  [n,B,H,D,D] fp32 device array, 16-byte aligned
+ *  gaps    HOST array of n values, read during the call
+ *  decay   HOST array of H values in (0, 1]
+ *  out     out [B,H,D,D] fp32 device array, 16-byte aligned; it may be one of
+ *          the states (each element is read before it is written).
+ * 1 <= n <= LA_MAX_SCAN_SEGMENTS (else LA_ERR_UNSUPPORTED). */
+la_status la_chunk_decay_scan(const float *states, const long long *gaps, int n, const float *decay,
+                              float *out, int B, int H, int D, void *stream);
 
 /* ---- the state form in stages, for a sequence split along T -------------
  * A sequence cut into shards along T (one per rank or per call) gives each

@@ -54,13 +54,16 @@ _lib.la_chunk_decay_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, 
 _lib.la_chunk_decay_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_chunk_decay_step.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]
 _lib.la_chunk_decay_fwd_state.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
+_lib.la_chunk_decay_bwd_state.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z,
+                                          _P]
+_lib.la_chunk_decay_scan.argtypes = [_P, _P, _I, _P, _P, _I, _I, _I, _P]
 _lib.la_state_reduce.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_state_apply.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
 _lib.la_state_bwd_q.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
 _lib.la_state_bwd_kv.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]
 for _n in ("la_bidir_fwd", "la_simple_fwd", "la_bidir_bwd", "la_simple_bwd", "la_chunk_decay_fwd",
-           "la_chunk_decay_bwd", "la_chunk_decay_step", "la_chunk_decay_fwd_state", "la_state_reduce", "la_state_apply", "la_state_bwd_q",
-           "la_state_bwd_kv"):
+           "la_chunk_decay_bwd", "la_chunk_decay_step", "la_chunk_decay_fwd_state", "la_chunk_decay_bwd_state",
+           "la_chunk_decay_scan", "la_state_reduce", "la_state_apply", "la_state_bwd_q", "la_state_bwd_kv"):
     getattr(_lib, _n).restype = _I
 _lib.la_bidir_fwd_static.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.la_bidir_fwd_static.restype = _I
@@ -246,6 +249,27 @@ def la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=None, state_out=None, w
            "la_chunk_decay_fwd_state")
 
 
+def la_chunk_decay_bwd_state(q, k, v, dout, decay, dq, dk, dv, state_in=None, dstate_in=None, dstate_out=None,
+                             workspace=None, stream=None):
+    """la_chunk_decay_bwd of one segment: state_in is the state of the tokens before it,
+    dstate_in R = sum gamma^(u-T) q_u^T dout_u of the tokens after it (both [B, H, D, D] float32,
+    zero if None); dstate_out (if given, not overlapping either) receives R at the segment's
+    first row.  dq may be None: then only dk and dv are computed."""
+    import torch
+    B, H, T, D = _shape(q, k, v, dout, dq, dk, dv)
+    for st, name in ((state_in, "state_in"), (dstate_in, "dstate_in"), (dstate_out, "dstate_out")):
+        if st is not None and (tuple(st.shape) != (B, H, D, D) or st.dtype != torch.float32 or not st.is_cuda
+                               or not st.is_contiguous() or st.device != q.device):
+            raise ValueError("%s must be a contiguous float32 CUDA tensor [B, H, D, D] on the inputs' device" % name)
+    dt = _dtype_code(q)
+    dec = _decay(decay, H)
+    wp, wn, _keep = _workspace("chunk_decay_bwd", (B, H, T, D), dt, workspace, q.device, stream)
+    _check(_lib.la_chunk_decay_bwd_state(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(state_in), _ptr(dstate_in),
+                                         _ptr(dstate_out), ctypes.cast(dec, _P), _ptr(dq), _ptr(dk), _ptr(dv), B, H,
+                                         T, D, dt, wp, wn, _stream(stream, q.device)),
+           "la_chunk_decay_bwd_state")
+
+
 def la_chunk_decay_bwd(q, k, v, dout, decay, dq, dk, dv, workspace=None, stream=None):
     """dq, dk, dv <- gradients of sum(o * dout) for la_chunk_decay_fwd."""
     B, H, T, D = _shape(q, k, v, dout, dq, dk, dv)
@@ -255,6 +279,27 @@ def la_chunk_decay_bwd(q, k, v, dout, decay, dq, dk, dv, workspace=None, stream=
     _check(_lib.la_chunk_decay_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), ctypes.cast(dec, _P), _ptr(dq),
                                    _ptr(dk), _ptr(dv), B, H, T, D, dt, wp, wn, _stream(stream, q.device)),
            "la_chunk_decay_bwd")
+
+
+def la_chunk_decay_scan(states, gaps, decay, out, stream=None):
+    """out[b, h] <- sum over i with gaps[i] >= 0 of decay[h]^gaps[i] * states[i, b, h]: the state
+    entering (or, backwards, the R leaving into) one segment of a sequence split into segments.
+    states is a float32 [n, B, H, D, D] CUDA tensor, out a float32 [B, H, D, D] one, gaps a
+    length-n host sequence of ints (-1 = leave segment i out)."""
+    import torch
+    if states.dim() != 5 or states.dtype != torch.float32 or not states.is_cuda or not states.is_contiguous():
+        raise ValueError("states must be a contiguous float32 CUDA tensor [n, B, H, D, D]")
+    n, B, H, D, D2 = (int(x) for x in states.shape)
+    if D2 != D or tuple(out.shape) != (B, H, D, D) or out.dtype != torch.float32 or not out.is_cuda \
+            or not out.is_contiguous() or out.device != states.device:
+        raise ValueError("out must be a contiguous float32 CUDA tensor [B, H, D, D] on the states' device")
+    g = [int(x) for x in gaps]
+    if len(g) != n:
+        raise ValueError("gaps must have n=%d entries" % n)
+    garr = (ctypes.c_longlong * n)(*g)
+    dec = _decay(decay, H)
+    _check(_lib.la_chunk_decay_scan(_ptr(states), ctypes.cast(garr, _P), n, ctypes.cast(dec, _P), _ptr(out), B, H,
+                                    D, _stream(stream, states.device)), "la_chunk_decay_scan")
 
 
 def la_chunk_decay_step(q, k, v, o, state, decay, stream=None):

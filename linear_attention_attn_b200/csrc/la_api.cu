@@ -340,25 +340,73 @@ la_status la_chunk_decay_fwd_state(const void *q, const void *k, const void *v, 
                            stream);
 }
 
-la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const void *dout, const float *decay,
-                             void *dq, void *dk, void *dv, int B, int H, int T, int D, la_dtype dtype,
-                             void *workspace, size_t workspace_bytes, void *stream) {
+static la_status decay_bwd_entry(const void *q, const void *k, const void *v, const void *dout, const float *sin,
+                                 const float *rin, float *rout, const float *decay, void *dq, void *dk, void *dv,
+                                 int B, int H, int T, int D, la_dtype dtype, void *workspace, size_t workspace_bytes,
+                                 void *stream, bool dq_optional) {
     const Shape s{B, H, T, D};
     LA_TRY(validate(s, dtype));
     LA_TRY(check_ptr(q, "q"));
     LA_TRY(check_ptr(k, "k"));
     LA_TRY(check_ptr(v, "v"));
     LA_TRY(check_ptr(dout, "dout"));
-    LA_TRY(check_ptr(dq, "dq"));
+    if (dq || !dq_optional) LA_TRY(check_ptr(dq, "dq"));
     LA_TRY(check_ptr(dk, "dk"));
     LA_TRY(check_ptr(dv, "dv"));
+    if (sin) LA_TRY(check_state(sin, "state_in"));
+    if (rin) LA_TRY(check_state(rin, "dstate_in"));
+    if (rout) {
+        LA_TRY(check_state(rout, "dstate_out"));
+        // dstate_out is written while other CTAs still read state_in and dstate_in
+        const size_t bytes = (size_t)s.BH() * D * D * sizeof(float);
+        auto overlaps = [&](const float *a) {
+            return a && (const char *)a < (const char *)rout + bytes && (const char *)rout < (const char *)a + bytes;
+        };
+        if (overlaps(sin) || overlaps(rin))
+            return fail(LA_ERR_INVALID_ARG, "dstate_out overlaps state_in or dstate_in");
+    }
     DecayArgs dec;
     LA_TRY(decay_args(decay, H, &dec));
     LA_TRY(check_ws(LA_OP_CHUNK_DECAY_BWD, s, dtype, workspace, workspace_bytes));
-    if (T == 0) return LA_OK;
     cudaStream_t st = (cudaStream_t)stream;
-    if (path_tc(LA_OP_CHUNK_DECAY_BWD, s, dtype)) return tc::decay_bwd(q, k, v, dout, dec, dq, dk, dv, s, dtype, workspace, st);
-    return simt::decay_bwd(q, k, v, dout, dec, dq, dk, dv, s, dtype, st);
+    if (T == 0) {   // R passes through unchanged
+        if (!rout) return LA_OK;
+        const size_t bytes = (size_t)s.BH() * D * D * sizeof(float);
+        cudaError_t e = rin ? cudaMemcpyAsync(rout, rin, bytes, cudaMemcpyDeviceToDevice, st)
+                            : cudaMemsetAsync(rout, 0, bytes, st);
+        return e == cudaSuccess ? LA_OK : cuda_fail(e, "dstate copy");
+    }
+    if (path_tc(LA_OP_CHUNK_DECAY_BWD, s, dtype))
+        return tc::decay_bwd(q, k, v, dout, sin, rin, rout, dec, dq, dk, dv, s, dtype, workspace, st);
+    return simt::decay_bwd(q, k, v, dout, sin, rin, rout, dec, dq, dk, dv, s, dtype, st);
+}
+
+la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const void *dout, const float *decay,
+                             void *dq, void *dk, void *dv, int B, int H, int T, int D, la_dtype dtype,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    return decay_bwd_entry(q, k, v, dout, nullptr, nullptr, nullptr, decay, dq, dk, dv, B, H, T, D, dtype, workspace,
+                           workspace_bytes, stream, false);
+}
+
+la_status la_chunk_decay_bwd_state(const void *q, const void *k, const void *v, const void *dout,
+                                   const float *state_in, const float *dstate_in, float *dstate_out,
+                                   const float *decay, void *dq, void *dk, void *dv, int B, int H, int T, int D,
+                                   la_dtype dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    return decay_bwd_entry(q, k, v, dout, state_in, dstate_in, dstate_out, decay, dq, dk, dv, B, H, T, D, dtype,
+                           workspace, workspace_bytes, stream, true);
+}
+
+la_status la_chunk_decay_scan(const float *states, const long long *gaps, int n, const float *decay, float *out,
+                              int B, int H, int D, void *stream) {
+    LA_TRY(validate(Shape{B, H, 1, D}, LA_F32));
+    if (n < 1 || n > LA_MAX_SCAN_SEGMENTS)
+        return fail(LA_ERR_UNSUPPORTED, "n=%d segments, must be in [1, %d]", n, LA_MAX_SCAN_SEGMENTS);
+    if (!gaps) return fail(LA_ERR_INVALID_ARG, "gaps is NULL");
+    LA_TRY(check_state(states, "states"));
+    LA_TRY(check_state(out, "out"));
+    DecayArgs dec;
+    LA_TRY(decay_args(decay, H, &dec));
+    return decay_scan(states, gaps, n, dec, out, B, H, D, (cudaStream_t)stream);
 }
 
 la_status la_state_reduce(const void *k, const void *v, float *state, int B, int H, int T, int D, la_dtype dtype,

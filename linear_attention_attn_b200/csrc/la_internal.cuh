@@ -119,6 +119,11 @@ int state_splits(const Shape &s, int rows_per_unit);
 // Bytes of one [BH, D, D+1] fp32 state block, rounded up to 256.
 size_t state_bytes(const Shape &s, long long copies);
 
+// Combine of per-segment states of the decay op: out = sum_i gamma^gaps[i] states[i]
+// over the i with gaps[i] >= 0 (n <= LA_MAX_SCAN_SEGMENTS, gaps on the host).
+la_status decay_scan(const float *states, const long long *gaps, int n, const DecayArgs &dec, float *out, int B,
+                     int H, int D, cudaStream_t st);
+
 // One recurrent (decode) step of the decay op: S <- gamma S + k^T v, o = q S,
 // with q, k, v, o [B,H,D] and the fp32 state [B,H,D,D] updated in place.
 la_status decay_step(const void *q, const void *k, const void *v, void *o, float *state, const DecayArgs &dec, int B,
@@ -137,8 +142,9 @@ la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, con
                     float eps, void *ws, cudaStream_t st);
 la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
                     const DecayArgs &dec, const Shape &s, la_dtype dt, cudaStream_t st);
-la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec,
-                    void *dq, void *dk, void *dv, const Shape &s, la_dtype dt, cudaStream_t st);
+la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin,
+                    const float *rin, float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv,
+                    const Shape &s, la_dtype dt, cudaStream_t st);
 la_status state_stage(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout,
                       void *out1, void *out2, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
 }  // namespace simt

@@ -361,11 +361,12 @@ ret_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ 
     }
 }
 
-// Backward, forward sweep, thread i holds row i of S: dq_t[i] = sum_j S_t[i][j] g_t[j].
+// Backward, forward sweep, thread i holds row i of S: dq_t[i] = sum_j S_t[i][j] g_t[j],
+// S starting from the state entering the segment (sin) or zero.
 template <typename T, int D>
 __global__ void __launch_bounds__(D)
 ret_bwd_dq(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g, T *__restrict__ dq,
-           DecayArgs dec, int T_len, int H) {
+           DecayArgs dec, int T_len, int H, const float *__restrict__ sin) {
     __shared__ float tiles[3][kRetTile][D];
     const int bh = blockIdx.x;
     const float gamma = dec.gamma[bh % H];
@@ -373,7 +374,7 @@ ret_bwd_dq(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict
     const int i = threadIdx.x;
     float S[D];
 #pragma unroll
-    for (int j = 0; j < D; ++j) S[j] = 0.f;
+    for (int j = 0; j < D; ++j) S[j] = sin ? sin[((long long)bh * D + i) * D + j] : 0.f;
     const T *const src[3] = {k, v, g};
     for (int ts = 0; ts < T_len; ts += kRetTile) {
         __syncthreads();
@@ -395,11 +396,13 @@ ret_bwd_dq(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict
 
 // Backward, reverse sweep over R_s = gamma R_{s+1} + q_s^T g_s.  Threads
 // 0..D-1 hold row i of R (dk_s[i] = sum_j R[i][j] v_s[j]); threads D..2D-1
-// hold column j of R (dv_s[j] = sum_i k_s[i] R[i][j]).
+// hold column j of R (dv_s[j] = sum_i k_s[i] R[i][j]).  R starts from rin (R one
+// past the segment's last row) or zero; rout receives R at the segment's first row.
 template <typename T, int D>
 __global__ void __launch_bounds__(2 * D)
 ret_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-             const T *__restrict__ g, T *__restrict__ dk, T *__restrict__ dv, DecayArgs dec, int T_len, int H) {
+             const T *__restrict__ g, T *__restrict__ dk, T *__restrict__ dv, DecayArgs dec, int T_len, int H,
+             const float *__restrict__ rin, float *__restrict__ rout) {
     __shared__ float tiles[4][kRetTile][D];
     const int bh = blockIdx.x;
     const float gamma = dec.gamma[bh % H];
@@ -407,8 +410,9 @@ ret_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
     const bool row_side = threadIdx.x < D;
     const int idx = row_side ? threadIdx.x : threadIdx.x - D;
     float Rr[D];
+    const float *rb = rin ? rin + (long long)bh * D * D : nullptr;
 #pragma unroll
-    for (int m = 0; m < D; ++m) Rr[m] = 0.f;
+    for (int m = 0; m < D; ++m) Rr[m] = rin ? (row_side ? rb[idx * D + m] : rb[m * D + idx]) : 0.f;
     const T *const src[4] = {q, k, v, g};
     const int ntiles = (T_len + kRetTile - 1) / kRetTile;
     for (int tile = ntiles - 1; tile >= 0; --tile) {
@@ -437,6 +441,10 @@ ret_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
                 io<T>::st(dv + base + (long long)(ts + r) * D + idx, acc);
             }
         }
+    }
+    if (rout && row_side) {
+#pragma unroll
+        for (int j = 0; j < D; ++j) rout[((long long)bh * D + idx) * D + j] = Rr[j];
     }
 }
 
@@ -587,13 +595,15 @@ la_status decay_fwd_t(const T *q, const T *k, const T *v, T *o, const float *sin
 }
 
 template <typename T, int D>
-la_status decay_bwd_t(const T *q, const T *k, const T *v, const T *g, const DecayArgs &dec, T *dq, T *dk, T *dv,
-                      const Shape &s, cudaStream_t st) {
-    la_status rc = launch("simt_ret_bwd_dq", ret_bwd_dq<T, D>, dim3((unsigned)s.BH()), dim3(D), 0, st, k, v, g, dq,
-                          dec, s.T, s.H);
-    if (rc) return rc;
+la_status decay_bwd_t(const T *q, const T *k, const T *v, const T *g, const float *sin, const float *rin, float *rout,
+                      const DecayArgs &dec, T *dq, T *dk, T *dv, const Shape &s, cudaStream_t st) {
+    if (dq) {   // dq == null: dk, dv only
+        la_status rc = launch("simt_ret_bwd_dq", ret_bwd_dq<T, D>, dim3((unsigned)s.BH()), dim3(D), 0, st, k, v, g,
+                              dq, dec, s.T, s.H, sin);
+        if (rc) return rc;
+    }
     return launch("simt_ret_bwd_dkdv", ret_bwd_dkdv<T, D>, dim3((unsigned)s.BH()), dim3(2 * D), 0, st, q, k, v, g,
-                  dk, dv, dec, s.T, s.H);
+                  dk, dv, dec, s.T, s.H, rin, rout);
 }
 
 }  // namespace
@@ -654,13 +664,14 @@ la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const 
 #undef LA_RET_FWD
 }
 
-la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec, void *dq,
-                    void *dk, void *dv, const Shape &s, la_dtype dt, cudaStream_t st) {
-#define LA_RET_BWD(TY)                                                                                          \
-    return s.D == 64 ? decay_bwd_t<TY, 64>((const TY *)q, (const TY *)k, (const TY *)v, (const TY *)g, dec,       \
-                                           (TY *)dq, (TY *)dk, (TY *)dv, s, st)                                  \
-                     : decay_bwd_t<TY, 128>((const TY *)q, (const TY *)k, (const TY *)v, (const TY *)g, dec,      \
-                                            (TY *)dq, (TY *)dk, (TY *)dv, s, st)
+la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin, const float *rin,
+                    float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv, const Shape &s, la_dtype dt,
+                    cudaStream_t st) {
+#define LA_RET_BWD(TY)                                                                                              \
+    return s.D == 64 ? decay_bwd_t<TY, 64>((const TY *)q, (const TY *)k, (const TY *)v, (const TY *)g, sin, rin,      \
+                                           rout, dec, (TY *)dq, (TY *)dk, (TY *)dv, s, st)                           \
+                     : decay_bwd_t<TY, 128>((const TY *)q, (const TY *)k, (const TY *)v, (const TY *)g, sin, rin,     \
+                                            rout, dec, (TY *)dq, (TY *)dk, (TY *)dv, s, st)
     switch (dt) {
     case LA_F32: LA_RET_BWD(float);
     case LA_F16: LA_RET_BWD(__half);

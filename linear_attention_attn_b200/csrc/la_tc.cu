@@ -43,9 +43,10 @@ la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const 
                     const DecayArgs &dec, const Shape &s, la_dtype, void *, cudaStream_t st) {
     return retention_fwd(q, k, v, o, sin, sout, dec, s, st);
 }
-la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec, void *dq,
-                    void *dk, void *dv, const Shape &s, la_dtype, void *, cudaStream_t st) {
-    return retention_bwd(q, k, v, g, dec, dq, dk, dv, s, st);
+la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin, const float *rin,
+                    float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv, const Shape &s, la_dtype, void *,
+                    cudaStream_t st) {
+    return retention_bwd(q, k, v, g, sin, rin, rout, dec, dq, dk, dv, s, st);
 }
 
 }  // namespace tc

@@ -23,8 +23,11 @@ la_status retention_map(CUtensorMap *m, const void *ptr, const Shape &s);
 // Chunked causal decay forward on tensor cores (bf16, D = 128).
 la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
                         const DecayArgs &dec, const Shape &s, cudaStream_t st);
-la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec, void *dq,
-                        void *dk, void *dv, const Shape &s, cudaStream_t st);
+// sin: state S entering the segment (or null); rin: R = sum_{t >= end} gamma^(t-end) q_t^T dO_t
+// entering from the right (or null); rout: R at the segment's first row (or null).  [BH, D, D].
+la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin,
+                        const float *rin, float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv,
+                        const Shape &s, cudaStream_t st);
 la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, void *o, float *state,
                     const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
 la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, const void *g,
@@ -35,8 +38,9 @@ la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const 
 // One stage of the state form (Stage in la_internal.cuh).
 la_status state_stage(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout,
                       void *out1, void *out2, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
-la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec,
-                    void *dq, void *dk, void *dv, const Shape &s, la_dtype dt, void *ws, cudaStream_t st);
+la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin,
+                    const float *rin, float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv,
+                    const Shape &s, la_dtype dt, void *ws, cudaStream_t st);
 
 }  // namespace tc
 }  // namespace la

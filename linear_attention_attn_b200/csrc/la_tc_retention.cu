@@ -88,8 +88,12 @@ struct RetLayout {
 struct RetJobs {
     CUtensorMap q[3], k[3], v[3], o[3];
     int rev[3];
-    const float *sin;    // pass 0 (forward in time): state entering the sequence [BH, D, D], or null (zero)
-    float *sout;         // pass 0: state after the sequence [BH, D, D], or null
+    // Per pass: the state entering the pass's first chunk in its own direction of time
+    // [BH, D, D] fp32 (row = key-side index), or null for zero; sin_t[p] != 0 reads it
+    // transposed.  sout[p]: the state after the pass's last chunk, or null.
+    const float *sin[3];
+    float *sout[3];
+    int sin_t[3];
 };
 
 // Grid: one CTA per (pass, b, h), pass = blockIdx.x / BH.  decay[h] = gamma_h.
@@ -375,7 +379,9 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             live = live && got;
             if (got) {
                 tc_fence_after();
-                const float g1 = rev ? gpow[kC - ri] : gpow[ri + 1];
+                // backwards the entering state sits one past the chunk's last valid row
+                const int rows = min(kC, T - c * kC);
+                const float g1 = rev ? (ri < rows ? gpow[rows - ri] : 0.f) : gpow[ri + 1];
 #pragma unroll
                 for (int c16 = 0; c16 < 8; ++c16) {
                     float a[16], b[16];
@@ -407,19 +413,27 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         const uint32_t lanes = (uint32_t)(32 * sub) << 16;
         const int d = 32 * sub + lane;
         const float gC = gpow[kC];
-        const float gLast = gpow[min(kC, T - (nchunks - 1) * kC)];   // decay over a partial last chunk
+        // decay over the partial chunk at the end of the sequence: the last chunk
+        // forwards, the first one backwards
+        const float gLast = gpow[min(kC, T - (nchunks - 1) * kC)];
         float st[64];
-        const float *sin = pass == 0 ? jobs.sin : nullptr;
-        float *sout = pass == 0 ? jobs.sout : nullptr;
+        const float *sin = jobs.sin[pass];
+        float *sout = jobs.sout[pass];
         const long long srow = ((long long)bh * 128 + d) * 128 + 64 * half;   // this thread's 64 state entries
         if (sin) {   // S_0 given: registers and the hi + lo operand of the first Q S
+            if (jobs.sin_t[pass]) {   // st[c] = sin[64 half + c][d]: lanes read consecutive d
+                const float *col = sin + (long long)bh * 128 * 128 + (long long)(64 * half) * 128 + d;
 #pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) {
-                const float4 x = *reinterpret_cast<const float4 *>(sin + srow + 4 * c4);
-                st[4 * c4] = x.x;
-                st[4 * c4 + 1] = x.y;
-                st[4 * c4 + 2] = x.z;
-                st[4 * c4 + 3] = x.w;
+                for (int c = 0; c < 64; ++c) st[c] = col[(long long)c * 128];
+            } else {
+#pragma unroll
+                for (int c4 = 0; c4 < 16; ++c4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(sin + srow + 4 * c4);
+                    st[4 * c4] = x.x;
+                    st[4 * c4 + 1] = x.y;
+                    st[4 * c4 + 2] = x.z;
+                    st[4 * c4 + 3] = x.w;
+                }
             }
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
@@ -441,7 +455,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             if (!got) break;
             tc_fence_after();
             const uint32_t base = tmem + cDS + lanes + 64u * half;
-            const float g = (!rev && it == nchunks - 1) ? gLast : gC;
+            const float g = (it == (rev ? 0 : nchunks - 1)) ? gLast : gC;
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
                 float a[16];
@@ -496,8 +510,8 @@ la_status retention_fwd(const void *q, const void *k, const void *v, void *o, co
                         const DecayArgs &dec, const Shape &s, cudaStream_t st) {
     RetJobs jobs;
     memset(&jobs, 0, sizeof jobs);
-    jobs.sin = sin;
-    jobs.sout = sout;
+    jobs.sin[0] = sin;
+    jobs.sout[0] = sout;
     LA_TRY(retention_map(&jobs.q[0], q, s));
     LA_TRY(retention_map(&jobs.k[0], k, s));
     LA_TRY(retention_map(&jobs.v[0], v, s));
@@ -506,21 +520,37 @@ la_status retention_fwd(const void *q, const void *k, const void *v, void *o, co
                   (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
 }
 
-la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const DecayArgs &dec, void *dq,
-                        void *dk, void *dv, const Shape &s, cudaStream_t st) {
+la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin,
+                        const float *rin, float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv,
+                        const Shape &s, cudaStream_t st) {
     RetJobs jobs;
     memset(&jobs, 0, sizeof jobs);
-    // dq = retention(dO, V, K); dv = reverse retention(K, Q, dO); dk = reverse retention(V, dO, Q)
-    const void *in[3][3] = {{g, v, k}, {k, q, g}, {v, g, q}};
-    void *out[3] = {dq, dv, dk};
-    for (int p = 0; p < 3; ++p) {
-        LA_TRY(retention_map(&jobs.q[p], in[p][0], s));
-        LA_TRY(retention_map(&jobs.k[p], in[p][1], s));
-        LA_TRY(retention_map(&jobs.v[p], in[p][2], s));
-        LA_TRY(retention_map(&jobs.o[p], out[p], s));
-        jobs.rev[p] = p > 0;
+    // dq = retention(dO, V, K); dv = reverse retention(K, Q, dO); dk = reverse retention(V, dO, Q).
+    // Their states are S^T (S = sum k^T v), R and R^T (R = sum gamma^(t-s) q_t^T dO_t).
+    // dq == null leaves out the first pass.
+    struct Pass {
+        const void *q, *k, *v;
+        void *o;
+        int rev;
+        const float *sin;
+        int sin_t;
+        float *sout;
+    };
+    const Pass all[3] = {{g, v, k, dq, 0, sin, 1, nullptr},
+                         {k, q, g, dv, 1, rin, 0, rout},
+                         {v, g, q, dk, 1, rin, 1, nullptr}};
+    int np = 0;
+    for (int p = dq ? 0 : 1; p < 3; ++p, ++np) {
+        LA_TRY(retention_map(&jobs.q[np], all[p].q, s));
+        LA_TRY(retention_map(&jobs.k[np], all[p].k, s));
+        LA_TRY(retention_map(&jobs.v[np], all[p].v, s));
+        LA_TRY(retention_map(&jobs.o[np], all[p].o, s));
+        jobs.rev[np] = all[p].rev;
+        jobs.sin[np] = all[p].sin;
+        jobs.sin_t[np] = all[p].sin_t;
+        jobs.sout[np] = all[p].sout;
     }
-    return launch_pdl("tc_retention_bwd", retention_kernel, dim3((unsigned)(3 * s.BH())), dim3(kRThreads),
+    return launch_pdl("tc_retention_bwd", retention_kernel, dim3((unsigned)(np * s.BH())), dim3(kRThreads),
                   (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
 }
 

@@ -1,11 +1,16 @@
-"""Sequence parallelism for the state form (bidirectional linear attention and simple_la).
+"""Sequence parallelism for the state form (bidirectional linear attention and simple_la) and
+for the decay op (retention).
 
 Every rank holds one shard of the sequence along T (the same B, H, D on every rank).  A
 shard's state is a sum over its tokens, so the whole sequence's state is the sum of the
 shards' states: the forward is a local reduce, one all-reduce of the [B, H, D, D+1] fp32
 state, and a local apply; the backward is a local dq pass, one all-reduce of (dS | dz), and a
-local dk, dv pass.  The collective is torch.distributed's (NCCL over NVLink for CUDA
-tensors); `ops` is the module that provides the four stages, the CUDA binding by default.
+local dk, dv pass.  The decay op's segments are not a sum but a scan (the state entering a
+segment decays across the segments in between): its end states are all-gathered and
+combined per rank (decay_forward, decay_backward).  The collective is torch.distributed's
+(NCCL over NVLink for CUDA tensors); `ops` is the module that provides the stages, the CUDA
+binding by default.  The collectives and the stages run in the order of torch's current stream:
+pass stream=None, or that stream.
 """
 from __future__ import annotations
 
@@ -46,41 +51,96 @@ def backward(q, k, v, dout, state, dq, dk, dv, dstate, feature="elu1", eps: floa
     return dstate
 
 
-def decay_forward(q, k, v, o, decay, state_out=None, group=None, ops=None, stream=None, workspace=None):
-    """The decay op (retention) forward for this rank's segment of a sequence split along T
-    (rank r holds the r-th segment).  A segment's output needs the state of every token before
-    it: pass 1 gives each segment's own end state E_r (from a zero state), an all-gather shares
-    them with the segment lengths, rank r forms S_r = sum_{r' < r} (prod of gamma^T over the
-    segments between) E_r' as the running state gamma^{T_r'} S + E_r', and pass 2 recomputes the
-    segment from S_r.  state_out (optional, [B, H, D, D] fp32) receives the state after this
-    rank's segment (on the last rank: after the whole sequence)."""
-    import torch
-    if ops is None:
-        from linear_attention_attn_b200 import la_chunk_decay_fwd_state
-    else:
-        la_chunk_decay_fwd_state = ops.la_chunk_decay_fwd_state
+def _world(group):
     import torch.distributed as dist
-    B, H, T, D = (int(x) for x in q.shape)
-    kw = {} if workspace is None else {"workspace": workspace}
-    end = torch.empty((B, H, D, D), dtype=torch.float32 if q.is_cuda else torch.float64, device=q.device)
-    la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=None, state_out=end, stream=stream, **kw)
-    world = dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
-    if world == 1:
-        if state_out is not None:
-            state_out.copy_(end)
-        return state_out
-    rank = dist.get_rank(group)
-    ends = [torch.empty_like(end) for _ in range(world)]
-    dist.all_gather(ends, end, group=group)
-    lens = torch.tensor([T], dtype=torch.int64, device=end.device)
+    if dist.is_available() and dist.is_initialized():
+        return dist.get_world_size(group), dist.get_rank(group)
+    return 1, 0
+
+
+def _gather_states(x, T, group):
+    """All-gather this rank's [B, H, D, D] state and segment length: ([world, B, H, D, D], lengths)."""
+    import torch
+    import torch.distributed as dist
+    world, _ = _world(group)
+    buf = torch.empty((world,) + tuple(x.shape), dtype=x.dtype, device=x.device)
+    dist.all_gather(list(buf.unbind(0)), x, group=group)
+    lens = torch.tensor([T], dtype=torch.int64, device=x.device)
     all_lens = [torch.empty_like(lens) for _ in range(world)]
     dist.all_gather(all_lens, lens, group=group)
-    gam = torch.as_tensor([float(x) for x in (decay.tolist() if hasattr(decay, "tolist") else decay)],
-                          dtype=torch.float64)
-    state = torch.zeros((B, H, D, D), dtype=torch.float64, device=end.device)
-    for r in range(rank):
-        f = torch.pow(gam, float(all_lens[r].item())).to(end.device)
-        state = f[None, :, None, None] * state + ends[r].to(torch.float64)
-    sin = state.to(end.dtype).contiguous()
-    la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=sin, state_out=state_out, stream=stream, **kw)
+    return buf, [int(t.item()) for t in all_lens]
+
+
+def entering_gaps(lens, rank):
+    """Gaps for the state entering segment `rank`: segment i < rank is followed by the tokens of
+    segments i+1 .. rank-1 before it reaches `rank` (-1: segment not included)."""
+    return [sum(lens[i + 1:rank]) if i < rank else -1 for i in range(len(lens))]
+
+
+def leaving_gaps(lens, rank):
+    """Gaps for the reverse-sweep state R arriving at segment `rank` from the right: segment
+    i > rank is preceded by the tokens of segments rank+1 .. i-1 (-1: not included)."""
+    return [sum(lens[rank + 1:i]) if i > rank else -1 for i in range(len(lens))]
+
+
+def _decay_ops(ops):
+    if ops is None:
+        import linear_attention_attn_b200 as ops
+    return ops
+
+
+def decay_forward(q, k, v, o, decay, state_out=None, entering=None, group=None, ops=None, stream=None,
+                  workspace=None):
+    """The decay op (retention) forward for this rank's segment of a sequence split along T
+    (rank r holds the r-th segment).  A segment's output needs the state of every token before
+    it: pass 1 gives each segment's own end state E_r (from a zero state) and, on rank 0, its
+    final output; an all-gather shares the E_r and the segment lengths; la_chunk_decay_scan forms
+    S_r = sum_{r' < r} gamma^(tokens between) E_r'; pass 2 recomputes the segment from S_r.
+    state_out (optional, [B, H, D, D] fp32) receives the state after this rank's segment (on the
+    last rank: after the whole sequence); entering (optional, same shape) receives S_r, which
+    decay_backward needs."""
+    import torch
+    ops = _decay_ops(ops)
+    B, H, T, D = (int(x) for x in q.shape)
+    kw = {} if workspace is None else {"workspace": workspace}
+    world, rank = _world(group)
+    sdt = torch.float32 if q.is_cuda else torch.float64
+    end = state_out if state_out is not None else torch.empty((B, H, D, D), dtype=sdt, device=q.device)
+    if entering is not None:
+        entering.zero_()
+    ops.la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=None, state_out=end, stream=stream, **kw)
+    if world == 1:
+        return state_out
+    ends, lens = _gather_states(end, T, group)
+    if rank == 0:                                  # nothing enters the first segment: pass 1 is final
+        return state_out
+    sin = entering if entering is not None else torch.empty_like(end)
+    ops.la_chunk_decay_scan(ends, entering_gaps(lens, rank), decay, sin, stream=stream)
+    ops.la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=sin, state_out=state_out, stream=stream, **kw)
     return state_out
+
+
+def decay_backward(q, k, v, dout, decay, dq, dk, dv, entering=None, group=None, ops=None, stream=None,
+                   workspace=None):
+    """The decay op's backward for this rank's segment, with `entering` the state S_r entering it
+    (from decay_forward; None for zero).  dq needs only S_r, so pass 1 (the whole backward from
+    S_r and a zero R) gives the final dq and each segment's own reverse-sweep state F_r at its
+    first token; an all-gather shares the F_r; la_chunk_decay_scan forms the R arriving from the
+    segments to the right, R_r = sum_{r' > r} gamma^(tokens between) F_r'; pass 2 recomputes dk
+    and dv from R_r (the last rank has none and skips it)."""
+    import torch
+    ops = _decay_ops(ops)
+    B, H, T, D = (int(x) for x in q.shape)
+    kw = {} if workspace is None else {"workspace": workspace}
+    world, rank = _world(group)
+    f = torch.empty((B, H, D, D), dtype=torch.float32 if q.is_cuda else torch.float64, device=q.device)
+    ops.la_chunk_decay_bwd_state(q, k, v, dout, decay, dq, dk, dv, state_in=entering, dstate_in=None,
+                                 dstate_out=f, stream=stream, **kw)
+    if world == 1:
+        return
+    fs, lens = _gather_states(f, T, group)
+    if rank == world - 1:                          # nothing arrives from after the last segment
+        return
+    rin = torch.empty_like(f)
+    ops.la_chunk_decay_scan(fs, leaving_gaps(lens, rank), decay, rin, stream=stream)
+    ops.la_chunk_decay_bwd_state(q, k, v, dout, decay, None, dk, dv, dstate_in=rin, stream=stream, **kw)

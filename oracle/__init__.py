@@ -61,9 +61,10 @@ def _bind(lib):
     lib.oracle_retention_bwd.argtypes = [P, P, P, P, P, P, P, P, L, L, L, L, I]
     lib.oracle_retention_step.argtypes = [P, P, P, P, P, P, L, L, L]
     lib.oracle_retention_fwd_state.argtypes = [P, P, P, P, P, P, P, L, L, L, L, I]
+    lib.oracle_retention_bwd_state.argtypes = [P, P, P, P, P, P, P, P, P, P, P, L, L, L, L, I]
     for name in ("oracle_bidir_fwd", "oracle_simple_fwd", "oracle_bidir_bwd",
                  "oracle_simple_bwd", "oracle_retention_fwd", "oracle_retention_bwd",
-                 "oracle_retention_step", "oracle_retention_fwd_state"):
+                 "oracle_retention_step", "oracle_retention_fwd_state", "oracle_retention_bwd_state"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -196,6 +197,32 @@ class Oracle:
         _check(rc, "oracle_retention_fwd_state")
         return o, sout
 
+    def retention_bwd_state(self, q, k, v, dout, gamma, state_in=None, dstate_in=None,
+                            nthreads: int | None = None):
+        """retention_bwd of one segment of a longer sequence: state_in is the state of the
+        tokens before it, dstate_in the reverse-sweep R = sum_u gamma^(u-T) q_u^T dout_u of the
+        tokens after it ([B, H, D, D], zero if None).  Returns (dq, dk, dv, R at the segment's
+        first token)."""
+        q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(dout)
+        B, H, T, D = _shape4(q)
+        gm = _f64(gamma).reshape(-1)
+        if gm.shape[0] != H:
+            raise ValueError("gamma must have H=%d entries" % H)
+        ins = []
+        for a, name in ((state_in, "state_in"), (dstate_in, "dstate_in")):
+            a = None if a is None else np.ascontiguousarray(_f64(a))
+            if a is not None and a.shape != (B, H, D, D):
+                raise ValueError("%s must be [B, H, D, D]" % name)
+            ins.append(a)
+        dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+        rout = np.empty((B, H, D, D))
+        rc = self._lib.oracle_retention_bwd_state(
+            _p(q), _p(k), _p(v), _p(g), _p(gm), None if ins[0] is None else _p(ins[0]),
+            None if ins[1] is None else _p(ins[1]), _p(dq), _p(dk), _p(dv), _p(rout), B, H, T, D,
+            nthreads or default_threads())
+        _check(rc, "oracle_retention_bwd_state")
+        return dq, dk, dv, rout
+
     def retention_step(self, q, k, v, gamma, state):
         """One decode step: returns (o, new_state) with new_state = gamma_h state + k^T v and
         o = q new_state; q, k, v are [B, H, D], state is [B, H, D, D] (not modified)."""
@@ -260,3 +287,7 @@ def retention_step(*a, **kw):
 
 def retention_fwd_state(*a, **kw):
     return _instance().retention_fwd_state(*a, **kw)
+
+
+def retention_bwd_state(*a, **kw):
+    return _instance().retention_bwd_state(*a, **kw)

@@ -59,8 +59,10 @@ typedef struct {
     const double *q, *k, *v, *g;   /* g = upstream gradient dO (bwd only) */
     double *o, *state, *dq, *dk, *dv;
     const double *gamma;           /* [H] (retention only) */
-    const double *state_in;        /* [B, H, D, D] state entering the sequence, or NULL (retention fwd) */
+    const double *state_in;        /* [B, H, D, D] state entering the sequence, or NULL (retention) */
     double *state_out;             /* [B, H, D, D] state after the last token, or NULL (retention fwd) */
+    const double *dstate_in;       /* [B, H, D, D] R entering from after the sequence, or NULL (retention bwd) */
+    double *dstate_out;            /* [B, H, D, D] R at the first token, or NULL (retention bwd) */
     long B, H, T, D;
     double eps;
     int use_phi, use_norm;
@@ -305,7 +307,9 @@ static void retention_fwd_head(job_t *jb, long bh, double *scratch) {
  *   dq_t[i] = sum_j S_t[i][j] g_t[j]                        (forward sweep)
  *   R_t     = gamma R_{t+1} + q_t^T g_t   (R_T = 0)          (reverse sweep)
  *             i.e. R_s = sum_{t>=s} gamma^(t-s) q_t^T g_t
- *   dk_s[i] = sum_j R_s[i][j] v_s[j],   dv_s[j] = sum_i k_s[i] R_s[i][j]. */
+ *   dk_s[i] = sum_j R_s[i][j] v_s[j],   dv_s[j] = sum_i k_s[i] R_s[i][j].
+ * For a segment of a longer sequence S_{-1} = state_in (the tokens before it) and
+ * R_T = dstate_in (the tokens after it) instead of zero; R_0 goes to dstate_out. */
 static void retention_bwd_head(job_t *jb, long bh, double *scratch) {
     const long T = jb->T, D = jb->D;
     const double gamma = jb->gamma[bh % jb->H];
@@ -314,6 +318,8 @@ static void retention_bwd_head(job_t *jb, long bh, double *scratch) {
     double *dq = jb->dq + off, *dk = jb->dk + off, *dv = jb->dv + off;
     double *S = scratch, *R = S + D * D;
     memset(S, 0, (size_t)(2 * D * D) * sizeof(double));
+    if (jb->state_in) memcpy(S, jb->state_in + bh * D * D, (size_t)(D * D) * sizeof(double));
+    if (jb->dstate_in) memcpy(R, jb->dstate_in + bh * D * D, (size_t)(D * D) * sizeof(double));
     for (long t = 0; t < T; ++t) {
         for (long i = 0; i < D; ++i)
             for (long j = 0; j < D; ++j)
@@ -339,6 +345,7 @@ static void retention_bwd_head(job_t *jb, long bh, double *scratch) {
             dv[s * D + j] = a;
         }
     }
+    if (jb->dstate_out) memcpy(jb->dstate_out + bh * D * D, R, (size_t)(D * D) * sizeof(double));
 }
 
 int oracle_retention_fwd(const double *q, const double *k, const double *v, const double *gamma,
@@ -394,6 +401,22 @@ int oracle_retention_bwd(const double *q, const double *k, const double *v, cons
     if (check_dims(B, H, T, D) || !q || !k || !v || !dout || !gamma || !dq || !dk || !dv) return -1;
     job_t jb; memset(&jb, 0, sizeof jb);
     jb.q = q; jb.k = k; jb.v = v; jb.g = dout; jb.gamma = gamma; jb.dq = dq; jb.dk = dk; jb.dv = dv;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D;
+    return for_each_head(&jb, retention_bwd_head, (size_t)(2 * D * D), nthreads);
+}
+
+/* oracle_retention_bwd of one segment of a longer sequence: state_in is the state
+ * of the tokens before it, dstate_in the reverse-sweep R of the tokens after it
+ * (both zero if NULL); R at the segment's first token goes to dstate_out (if not
+ * NULL).  Arrays [B, H, D, D]. */
+int oracle_retention_bwd_state(const double *q, const double *k, const double *v, const double *dout,
+                               const double *gamma, const double *state_in, const double *dstate_in,
+                               double *dq, double *dk, double *dv, double *dstate_out,
+                               long B, long H, long T, long D, int nthreads) {
+    if (check_dims(B, H, T, D) || (T > 0 && (!q || !k || !v || !dout || !dq || !dk || !dv)) || !gamma) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.g = dout; jb.gamma = gamma; jb.dq = dq; jb.dk = dk; jb.dv = dv;
+    jb.state_in = state_in; jb.dstate_in = dstate_in; jb.dstate_out = dstate_out;
     jb.B = B; jb.H = H; jb.T = T; jb.D = D;
     return for_each_head(&jb, retention_bwd_head, (size_t)(2 * D * D), nthreads);
 }

@@ -352,5 +352,52 @@ def check_state_segments(orc):
            what="two segments vs the whole")
 
 
+def check_segment_backward(orc):
+    """The backward of one segment, with S_in from the tokens before it and R_in from the tokens
+    after it.  The tokens after the segment see its state only through S_out, and their loss
+    changes by gamma <R_in, dS_out> to first order, so the segment's gradients are those of
+    L = sum(o * g) + gamma <R_in, S_out>: finite differences of the forward from a state give
+    dq, dk, dv and, with respect to S_in, gamma R_0.  Then R_0 of a lone segment is
+    sum_t gamma^t q_t^T g_t, and two segments chained (S forwards, R backwards) give the whole
+    sequence's gradients."""
+    B, H, T, D = 1, 2, 5, 3
+    q, k, v, g = (_rand((B, H, T, D), 61 + i) for i in range(4))
+    gam = np.array([0.6, 0.95])
+    gm = gam[None, :, None, None]
+    sin, rin = _rand((B, H, D, D), 65), _rand((B, H, D, D), 66)
+    dq, dk, dv, r0 = orc.retention_bwd_state(q, k, v, g, gam, sin, rin)
+
+    def loss(a, b, c, s):
+        o, so = orc.retention_fwd_state(a, b, c, gam, s)
+        return float((o * g).sum() + (gm * rin * so).sum())
+
+    h = 1e-6
+    args = [q, k, v, sin]
+    for idx, (name, got) in enumerate((("dq", dq), ("dk", dk), ("dv", dv), ("dS_in", gm * r0))):
+        fd = np.zeros_like(args[idx])
+        for mi in np.ndindex(*args[idx].shape):
+            a = [x.copy() for x in args]
+            a[idx][mi] += h
+            lp = loss(*a)
+            a[idx][mi] -= 2 * h
+            fd[mi] = (lp - loss(*a)) / (2 * h)
+        _close(got, fd, rtol=1e-6, atol=1e-7, what="segment backward %s vs finite differences" % name)
+    # a lone segment: R_0 = sum_t gamma^t q_t^T g_t
+    _, _, _, r_lone = orc.retention_bwd_state(q, k, v, g, gam)
+    w = gam[None, :, None] ** np.arange(T)[None, None, :]
+    _close(r_lone, np.einsum("bht,bhti,bhtj->bhij", w, q, g), rtol=1e-12, atol=1e-13, what="R_0 closed form")
+    # two segments of a sequence of 11 chained through S (forwards) and R (backwards)
+    T2, p = 11, 4
+    q, k, v, g = (_rand((B, H, T2, D), 71 + i) for i in range(4))
+    cut = lambda x, a, b: np.ascontiguousarray(x[:, :, a:b])
+    _, s1 = orc.retention_fwd_state(cut(q, 0, p), cut(k, 0, p), cut(v, 0, p), gam)
+    dq2, dk2, dv2, r2 = orc.retention_bwd_state(cut(q, p, T2), cut(k, p, T2), cut(v, p, T2), cut(g, p, T2), gam, s1)
+    dq1, dk1, dv1, _ = orc.retention_bwd_state(cut(q, 0, p), cut(k, 0, p), cut(v, 0, p), cut(g, 0, p), gam, None, r2)
+    whole = orc.retention_bwd(q, k, v, g, gam)
+    for n, a, b, c in zip(("dq", "dk", "dv"), (dq1, dk1, dv1), (dq2, dk2, dv2), whole):
+        _close(np.concatenate([a, b], axis=2), c, rtol=1e-12, atol=1e-12, what="segments vs whole %s" % n)
+
+
 ALL_CHECKS = (check_golden, check_brute, check_closed_forms, check_invariances,
-              check_fd_gradients, check_autograd, check_decode_step, check_state_segments)
+              check_fd_gradients, check_autograd, check_decode_step, check_state_segments,
+              check_segment_backward)

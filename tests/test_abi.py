@@ -26,7 +26,8 @@ def declared_functions():
 def test_header_declares_the_api():
     names = declared_functions()
     for n in ("la_bidir_fwd", "la_bidir_bwd", "la_simple_fwd", "la_simple_bwd", "la_chunk_decay_fwd",
-              "la_chunk_decay_bwd", "la_chunk_decay_step", "la_chunk_decay_fwd_state", "la_workspace_size", "la_status_string", "la_last_error"):
+              "la_chunk_decay_bwd", "la_chunk_decay_step", "la_chunk_decay_fwd_state", "la_chunk_decay_bwd_state",
+              "la_workspace_size", "la_status_string", "la_last_error"):
         assert n in names
 
 
@@ -93,6 +94,44 @@ def test_decay_validation(lib):
     many = (ctypes.c_float * 600)(*([0.5] * 600))
     assert f(P(0x1000), P(0x1000), P(0x1000), P(0x1000), ctypes.cast(many, P), 1, 600, 16, 64, 2, P(0x100000),
              ctypes.c_size_t(1 << 30), P(0)) == 2
+
+
+def test_decay_bwd_state_validation(lib):
+    # dstate_out is written while other CTAs still read state_in and dstate_in: overlap is refused
+    P = ctypes.c_void_p
+    f = lib.la_chunk_decay_bwd_state
+    f.restype = ctypes.c_int
+    gam = (ctypes.c_float * 2)(0.5, 0.9)
+    nbytes = 1 * 2 * 64 * 64 * 4
+
+    def call(sin, rin, rout):
+        return f(P(0x1000), P(0x1000), P(0x1000), P(0x1000), P(sin), P(rin), P(rout), ctypes.cast(gam, P),
+                 P(0x1000), P(0x1000), P(0x1000), 1, 2, 16, 64, 2, P(0x100000), ctypes.c_size_t(1 << 30), P(0))
+    assert call(0x200000, 0x400000, 0x400000) == 1
+    assert call(0x200000, 0x400000, 0x400000 + nbytes - 16) == 1
+    assert call(0x200000 + nbytes - 16, 0x800000, 0x200000) == 1
+    assert call(0x200000, 0x400000, 0x400008) == 3     # 16-byte alignment
+    lib.la_last_error.restype = ctypes.c_char_p
+    assert call(0x200000, 0x400000, 0x400000 + nbytes - 16) == 1 and b"overlaps" in lib.la_last_error()
+
+
+def test_decay_scan_validation(lib):
+    P = ctypes.c_void_p
+    f = lib.la_chunk_decay_scan
+    f.restype = ctypes.c_int
+    gam = (ctypes.c_float * 2)(0.5, 0.9)
+    gaps = (ctypes.c_longlong * 200)(*([0] * 200))
+
+    def call(n=2, st=0x200000, gp=True, out=0x400000, D=128, dec=gam):
+        return f(P(st), ctypes.cast(gaps, P) if gp else P(0), n, ctypes.cast(dec, P), P(out), 1, 2, D, P(0))
+    assert call(n=0) == 2
+    assert call(n=129) == 2
+    assert call(D=96) == 2
+    assert call(gp=False) == 1
+    assert call(st=0) == 1
+    assert call(out=0x400004) == 3
+    bad = (ctypes.c_float * 2)(0.5, 0.0)
+    assert call(dec=bad) == 1
 
 
 def test_status_strings(lib):

@@ -41,6 +41,9 @@ MUTATIONS = [
     ("step_outer_product_transposed", "+ kh[i] * vh[j];", "+ kh[j] * vh[i];", 0),
     ("step_gamma_head_index", "const double g = gamma[bh % H];", "const double g = gamma[0];", 0),
     ("fwd_state_in_ignored", "    if (jb->state_in)\n", "    if (0)\n", 0),
+    ("bwd_state_in_ignored", "    if (jb->state_in) memcpy(S,", "    if (0) memcpy(S,", 0),
+    ("bwd_dstate_in_ignored", "    if (jb->dstate_in) memcpy(R,", "    if (0) memcpy(R,", 0),
+    ("bwd_dstate_out_is_state", "memcpy(jb->dstate_out + bh * D * D, R,", "memcpy(jb->dstate_out + bh * D * D, S,", 0),
     ("fwd_state_out_before_last_token", "    if (jb->state_out) memcpy(jb->state_out + bh * D * D, S,",
      "    if (jb->state_out) memcpy(jb->state_out + bh * D * D, jb->state_in ? jb->state_in + bh * D * D : S,", 0),
 ]

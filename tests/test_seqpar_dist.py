@@ -126,17 +126,49 @@ def test_two_ranks_match_the_whole_sequence(feature):
 
 
 def _decay_ops():
-    """la_chunk_decay_fwd_state on float64 CPU tensors: the recurrent form, from its definition."""
+    """The decay op's segment calls on float64 CPU tensors, from their definitions in
+    include/la.h: the recurrent form forwards (S) and backwards (R), and the combine."""
+    def gam4(decay):
+        return torch.as_tensor(list(decay), dtype=torch.float64)[None, :, None, None]
+
     def la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=None, state_out=None, stream=None):
         B, H, T, D = q.shape
-        g = torch.as_tensor(list(decay), dtype=torch.float64)[None, :, None, None]
+        g = gam4(decay)
         S = state_in.clone() if state_in is not None else torch.zeros(B, H, D, D, dtype=torch.float64)
         for t in range(T):
             S = g * S + torch.einsum("bhi,bhj->bhij", k[:, :, t], v[:, :, t])
             o[:, :, t] = torch.einsum("bhi,bhij->bhj", q[:, :, t], S)
         if state_out is not None:
             state_out.copy_(S)
-    return types.SimpleNamespace(la_chunk_decay_fwd_state=la_chunk_decay_fwd_state)
+
+    def la_chunk_decay_bwd_state(q, k, v, dout, decay, dq, dk, dv, state_in=None, dstate_in=None,
+                                 dstate_out=None, stream=None):
+        B, H, T, D = q.shape
+        g = gam4(decay)
+        if dq is not None:
+            S = state_in.clone() if state_in is not None else torch.zeros(B, H, D, D, dtype=torch.float64)
+            for t in range(T):
+                S = g * S + torch.einsum("bhi,bhj->bhij", k[:, :, t], v[:, :, t])
+                dq[:, :, t] = torch.einsum("bhij,bhj->bhi", S, dout[:, :, t])
+        R = dstate_in.clone() if dstate_in is not None else torch.zeros(B, H, D, D, dtype=torch.float64)
+        for s in reversed(range(T)):
+            R = g * R + torch.einsum("bhi,bhj->bhij", q[:, :, s], dout[:, :, s])
+            dk[:, :, s] = torch.einsum("bhij,bhj->bhi", R, v[:, :, s])
+            dv[:, :, s] = torch.einsum("bhi,bhij->bhj", k[:, :, s], R)
+        if dstate_out is not None:
+            dstate_out.copy_(R)
+
+    def la_chunk_decay_scan(states, gaps, decay, out, stream=None):
+        g = gam4(decay)
+        acc = torch.zeros_like(out)
+        for i, gap in enumerate(gaps):
+            if gap >= 0:
+                acc += g ** gap * states[i]
+        out.copy_(acc)
+
+    return types.SimpleNamespace(la_chunk_decay_fwd_state=la_chunk_decay_fwd_state,
+                                 la_chunk_decay_bwd_state=la_chunk_decay_bwd_state,
+                                 la_chunk_decay_scan=la_chunk_decay_scan)
 
 
 def _decay_rank_main(rank, world, port, cuts, gam, out):
@@ -146,18 +178,31 @@ def _decay_rank_main(rank, world, port, cuts, gam, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     from linear_attention_attn_b200 import seqpar
-    q, k, v, _ = _inputs(2, 3, cuts[-1], 6)
+    q, k, v, g = _inputs(2, 3, cuts[-1], 6)
     sl = slice(cuts[rank], cuts[rank + 1])
-    qs, ks, vs = (x[:, :, sl].contiguous() for x in (q, k, v))
+    qs, ks, vs, gs = (x[:, :, sl].contiguous() for x in (q, k, v, g))
     o = torch.empty_like(qs)
     st = torch.empty(2, 3, 6, 6, dtype=torch.float64)
-    seqpar.decay_forward(qs, ks, vs, o, gam, state_out=st, ops=_decay_ops())
-    out[rank] = (o.numpy(), st.numpy())
+    ent = torch.empty_like(st)
+    ops = _decay_ops()
+    seqpar.decay_forward(qs, ks, vs, o, gam, state_out=st, entering=ent, ops=ops)
+    dq, dk, dv = (torch.empty_like(qs) for _ in range(3))
+    seqpar.decay_backward(qs, ks, vs, gs, gam, dq, dk, dv, entering=ent, ops=ops)
+    out[rank] = (o.numpy(), st.numpy(), dq.numpy(), dk.numpy(), dv.numpy())
     dist.barrier()
     dist.destroy_process_group()
 
 
-def test_decay_forward_over_three_ranks():
+def test_segment_gaps():
+    from linear_attention_attn_b200 import seqpar
+    lens = [5, 7, 0, 4]
+    assert seqpar.entering_gaps(lens, 0) == [-1, -1, -1, -1]
+    assert seqpar.entering_gaps(lens, 3) == [7, 0, 0, -1]
+    assert seqpar.leaving_gaps(lens, 0) == [-1, 0, 7, 7]
+    assert seqpar.leaving_gaps(lens, 3) == [-1, -1, -1, -1]
+
+
+def test_decay_forward_and_backward_over_three_ranks():
     import oracle
     cuts = [0, 7, 19, 30]
     gam = [0.6, 0.9, 1.0]
@@ -170,8 +215,12 @@ def test_decay_forward_over_three_ranks():
     for p in procs:
         p.join(180)
         assert p.exitcode == 0
-    q, k, v, _ = (x.numpy() for x in _inputs(2, 3, cuts[-1], 6))
+    q, k, v, g = (x.numpy() for x in _inputs(2, 3, cuts[-1], 6))
     want_o, want_s = oracle.retention_fwd_state(q, k, v, np.array(gam))
     got = np.concatenate([out[r][0] for r in range(3)], axis=2)
     np.testing.assert_allclose(got, want_o, rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(out[2][1], want_s, rtol=1e-10, atol=1e-12)    # the last rank: whole sequence
+    want = oracle.retention_bwd(q, k, v, g, np.array(gam))
+    for i, name in enumerate(("dq", "dk", "dv")):
+        got = np.concatenate([out[r][2 + i] for r in range(3)], axis=2)
+        np.testing.assert_allclose(got, want[i], rtol=1e-10, atol=1e-12, err_msg=name)
