@@ -5,6 +5,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <string.h>
 
 #include "la_internal.cuh"
 #include "la_tc_ptx.cuh"
@@ -45,26 +46,34 @@ __host__ __device__ inline int grid_for(long long N) { return N < kGrid ? (int)N
 __host__ __device__ inline int max_slots(int BH) { return (kGrid + BH - 1) / BH + 1; }
 
 // ------------------------------------------------------------ 16-bit I/O --
+// Packed pairs travel as uint32_t.  Reinterpreting a local through a pointer of
+// another type breaks C++'s aliasing rules, and the optimiser is then free to
+// read a value that was never stored (a bf16 pair read back as zero after it was
+// packed made a hi + lo split return lo = x); memcpy is the defined bit copy and
+// compiles to a register move.
+template <typename To, typename From>
+__device__ __forceinline__ To bit_cast32(const From &x) {
+    static_assert(sizeof(To) == 4 && sizeof(From) == 4, "32-bit values only");
+    To t;
+    memcpy(&t, &x, 4);
+    return t;
+}
+
 template <bool BF16> struct h2;
 template <> struct h2<false> {
-    static __device__ __forceinline__ float2 to_f2(uint32_t u) {
-        __half2 h = *reinterpret_cast<__half2 *>(&u);
-        return __half22float2(h);
-    }
+    static __device__ __forceinline__ float2 to_f2(uint32_t u) { return __half22float2(bit_cast32<__half2>(u)); }
     static __device__ __forceinline__ uint32_t from_f2(float a, float b) {
-        __half2 h = __floats2half2_rn(a, b);
-        return *reinterpret_cast<uint32_t *>(&h);
+        return bit_cast32<uint32_t>(__floats2half2_rn(a, b));
     }
     static __device__ __forceinline__ uint16_t one() { return 0x3C00u; }
 };
 template <> struct h2<true> {
+    // bf16 is the upper half of an fp32: widening is a shift
     static __device__ __forceinline__ float2 to_f2(uint32_t u) {
-        __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162 *>(&u);
-        return __bfloat1622float2(h);
+        return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
     }
     static __device__ __forceinline__ uint32_t from_f2(float a, float b) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-        return *reinterpret_cast<uint32_t *>(&h);
+        return bit_cast32<uint32_t>(__floats2bfloat162_rn(a, b));
     }
     static __device__ __forceinline__ uint16_t one() { return 0x3F80u; }
 };
@@ -76,15 +85,14 @@ __device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : __e
 // (x > 0 gives x + 2^0 = x + 1, x <= 0 gives e^x).  ex2.approx.f16x2 handles
 // both halves in one special-function operation.
 __device__ __forceinline__ uint32_t phi_h2(uint32_t x) {
-    const __half2 hx = *reinterpret_cast<__half2 *>(&x);
+    const __half2 hx = bit_cast32<__half2>(x);
     const __half2 zero = __float2half2_rn(0.f);
     const __half2 l2e = __float2half2_rn(1.4426950408889634f);
-    __half2 a = __hmul2(__hmin2(hx, zero), l2e);
-    uint32_t ai = *reinterpret_cast<uint32_t *>(&a), ei;
+    const __half2 a = __hmul2(__hmin2(hx, zero), l2e);
+    const uint32_t ai = bit_cast32<uint32_t>(a);
+    uint32_t ei;
     asm("ex2.approx.f16x2 %0, %1;" : "=r"(ei) : "r"(ai));
-    const __half2 e = *reinterpret_cast<__half2 *>(&ei);
-    __half2 r = __hadd2(__hmax2(hx, zero), e);
-    return *reinterpret_cast<uint32_t *>(&r);
+    return bit_cast32<uint32_t>(__hadd2(__hmax2(hx, zero), bit_cast32<__half2>(ei)));
 }
 
 // Feature map elu+1 applied in place to row `row` of a 128-byte-swizzled tile
@@ -285,7 +293,9 @@ __device__ __forceinline__ void tmem_row64(uint32_t taddr, float (&v)[64]) {
     tmem_ld16(taddr + 16, b);
     tmem_ld16(taddr + 32, c);
     tmem_ld16(taddr + 48, d);
-    tmem_ld_wait();
+    tmem_ld_wait(a, b);
+    reg_keep(c);
+    reg_keep(d);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         v[i] = a[i];

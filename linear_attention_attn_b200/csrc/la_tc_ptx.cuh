@@ -186,7 +186,36 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// The first 16 TMEM lanes of the warp's quadrant (where an M = 64 accumulator keeps
+// its rows) spread over all 32 threads: thread l reads lane l % 16, 16 consecutive
+// fp32 columns from taddr's column + OFF * (l / 16).
+template <int OFF>
+__device__ __forceinline__ void tmem_ld16_halves(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16], %17;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr), "n"(OFF));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+// Registers that tcgen05.ld fills are valid only after tcgen05.wait::ld, but the
+// compiler sees a load's outputs as ready at once and may schedule their uses
+// ahead of the wait.  So the wait takes the loaded registers as operands, and
+// further arrays loaded before the same wait pass through an empty asm after it
+// (volatile asm statements keep their order): every use comes after the wait.
+__device__ __forceinline__ void reg_keep(float (&a)[16]) {
+    asm volatile("" : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]), "+f"(a[4]), "+f"(a[5]), "+f"(a[6]), "+f"(a[7]), "+f"(a[8]), "+f"(a[9]), "+f"(a[10]), "+f"(a[11]), "+f"(a[12]), "+f"(a[13]), "+f"(a[14]), "+f"(a[15]));
+}
+__device__ __forceinline__ void tmem_ld_wait(float (&a)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3]), "+f"(a[4]), "+f"(a[5]), "+f"(a[6]), "+f"(a[7]), "+f"(a[8]), "+f"(a[9]), "+f"(a[10]), "+f"(a[11]), "+f"(a[12]), "+f"(a[13]), "+f"(a[14]), "+f"(a[15]) :: "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait(float (&a)[16], float (&b)[16]) {
+    tmem_ld_wait(a);
+    reg_keep(b);
+}
 
 // ------------------------------------------------------------ descriptors --
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100

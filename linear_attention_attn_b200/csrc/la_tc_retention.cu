@@ -12,14 +12,16 @@
 //
 // One CTA per (b, h) walks the chunks in order.  Warp 0 streams q/k/v chunks
 // with TMA (two 64-column boxes per 64-row chunk, 128-byte swizzle); warp 1
-// issues the UMMAs in the order P, dS, O_intra, O_inter, so that dS (which does
-// not depend on the state) and O_intra run while the state of the previous
-// chunk is being carried; warps 2..5 form gamma^(C-1-j) k and the masked
-// P~ = P o M (hi + lo bf16 each); warps 6..9 combine the two output
-// accumulators and store o; warps 10..13 carry the fp32 state
-// S <- gamma^C S + dS, kept in shared memory as a bf16 hi + lo pair that is
-// also the B operand of Q S.  The chain from one chunk to the next is only
-// O_inter (reads S_c) -> state update -> O_inter of the next chunk.
+// issues the UMMAs of chunk c in the order dS, O_intra, P of chunk c + 1,
+// O_inter, so that dS (which does not depend on the state), O_intra and the
+// next P run while the state is being carried; warps 2..5 form the masked
+// P~ = P o M (hi + lo bf16; the M = 64 accumulator rows spread over all 32
+// lanes of a warp); warps 6..9 combine the two output accumulators and store
+// o; warps 10..17 hold the fp32 state S <- gamma^C S + dS in registers, write
+// it to shared memory as the bf16 hi + lo B operand of Q S, and form
+// K^ = diag(gamma^(C-1-j)) K of the next chunk (hi + lo) while Q S runs.  The
+// chain from one chunk to the next is O_inter (reads S_c) -> state operand
+// write -> O_inter of the next chunk.
 //   P       M=64  N=64  K=128  A = Q (K-major)        B = K (K-major)
 //   O_intra M=64  N=128 K=64   A = P~ hi, lo (K-major) B = V (MN-major)
 //   O_inter M=64  N=128 K=128  A = Q (K-major)        B = S hi, lo (MN-major)
@@ -55,13 +57,38 @@ __device__ __forceinline__ uint8_t *align1024r(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// Four 8-element chunks (4 part .. 4 part + 3 of the row's 16, across the two boxes)
+// of row `row` of a [64 x 128] tile, scaled by f, as the bf16 hi tile and (if lo_too)
+// the lo tile, lo = round(x f - hi), kTile128 bytes further.
+static __device__ __noinline__ void scale_split_row(const uint8_t *src, uint8_t *dst, int row, int part, float f,
+                                                    bool lo_too) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int ch = part * 4 + i;
+        const int off = (ch >> 3) * kBox + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+        const uint4 u = *reinterpret_cast<const uint4 *>(src + off);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 x = h2<true>::to_f2(w[k]);
+            const float a = x.x * f, b = x.y * f;
+            hi[k] = h2<true>::from_f2(a, b);
+            const float2 hv = h2<true>::to_f2(hi[k]);
+            lo[k] = h2<true>::from_f2(a - hv.x, b - hv.y);
+        }
+        *reinterpret_cast<uint4 *>(dst + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        if (lo_too) *reinterpret_cast<uint4 *>(dst + kTile128 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+}
+
 // Stores 16 columns (16*c16 .. +15, c16 in 0..7) of row `row` of a 128-column tile
 // kept as boxes of 64 columns, `box_bytes` apart.
 __device__ __forceinline__ void st16_wide(uint8_t *t, int box_bytes, int row, int c16, const float (&v)[16]) {
     store_chunk16<true>(t + (c16 >> 2) * box_bytes, row, c16 & 3, v);
 }
 
-// Warp roles: 0 TMA, 1 UMMA, 2..5 K^ and decay mask, 6..9 output, 10..17 state
+// Warp roles: 0 TMA, 1 UMMA, 2..5 decay mask, 6..9 output, 10..17 state and K^
 // (two warps per TMEM lane quadrant, 64 state columns each).
 constexpr int kRXw0 = 2, kRXWarps = 4, kROw0 = 6, kROWarps = 4, kRSw0 = 10, kRSWarps = 8;
 constexpr int kRThreads = (kRSw0 + kRSWarps) * 32;
@@ -94,7 +121,12 @@ struct RetJobs {
     const float *sin[3];
     float *sout[3];
     int sin_t[3];
+    // Per pass, which operands carry a bf16 lo part besides the hi part (fp32 = hi + lo):
+    // kLoK (K^ of dS), kLoP (P~ of O_intra), kLoS (S of O_inter).  The launches set all
+    // three: each lo left out adds about 6e-4 to the relative L2 error of the output.
+    int lo[3];
 };
+constexpr int kLoK = 1, kLoP = 2, kLoS = 4;
 
 // Grid: one CTA per (pass, b, h), pass = blockIdx.x / BH.  decay[h] = gamma_h.
 __global__ void __launch_bounds__(kRThreads, 1)
@@ -133,6 +165,8 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
     const int pass = blockIdx.x / BH;
     const int bh = blockIdx.x % BH;
     const bool rev = jobs.rev[pass] != 0;
+    const int lo_mask = jobs.lo[pass];
+    const int nlk = (lo_mask & kLoK) ? 2 : 1, nlp = (lo_mask & kLoP) ? 2 : 1, nls = (lo_mask & kLoS) ? 2 : 1;
     const CUtensorMap *tmQ = &jobs.q[pass], *tmK = &jobs.k[pass], *tmV = &jobs.v[pass], *tmO = &jobs.o[pass];
     const float gamma = dec.gamma[bh % H];
     const int nchunks = (T + kC - 1) / kC;
@@ -144,7 +178,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         }
         mbar_init(pfull, 1);
         mbar_init(ptready, kRXWarps);
-        mbar_init(khready, kRXWarps);
+        mbar_init(khready, kRSWarps);
         mbar_init(dsfull, 1);
         mbar_init(dsread, kRSWarps);
         mbar_init(sready, kRSWarps);
@@ -245,7 +279,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
-                    for (int op = 0; op < 2; ++op)
+                    for (int op = 0; op < nlk; ++op)
                         umma_f16_ss(tmem + cDS, desc_at(dkh, op * kTile128 + kk * 2048), desc_at(dv, kk * 2048), ID_DS,
                                     (kk | op) ? 1u : 0u);
                 }
@@ -258,7 +292,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
-                    for (int op = 0; op < 2; ++op)
+                    for (int op = 0; op < nlp; ++op)
                         umma_f16_ss(tmem + cOI, desc_at(dpt, op * kBox + kk * 32), desc_at(dv, kk * 2048), ID_OI,
                                     (kk | op) ? 1u : 0u);
                 }
@@ -276,7 +310,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
 #pragma unroll
-                    for (int op = 0; op < 2; ++op)
+                    for (int op = 0; op < nls; ++op)
                         umma_f16_ss(tmem + cOX, desc_at(dq, off), desc_at(ds, op * 32768 + kk * 2048), ID_OI,
                                     (kk | op) ? 1u : 0u);
                 }
@@ -290,75 +324,40 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_ret_fault, 0x400u);
         }
     } else if (warp < kROw0) {
-        // Feature-map warps: K^ = diag(gamma^(C-1-j)) K as hi + lo (thread xt: row xt % 64,
-        // 8-element chunks 8 (xt / 64) .. + 7), then the decay mask P~ = P o M as hi + lo
-        // (warp w reads TMEM lane quadrant w % 4; lanes 0..15 hold chunk rows 16 (w % 4) + l).
-        const int xt = threadIdx.x - kRXw0 * 32;
-        const int krow = xt & 63, part = xt >> 6;
+        // Decay-mask warps: P~ = P o M as hi + lo (warp w reads TMEM lane quadrant w % 4,
+        // where chunk rows 16 (w % 4) + l sit in lanes l = 0..15).
         const int sub = warp & 3;
         const uint32_t lanes = (uint32_t)(32 * sub) << 16;
-        const int ri = 16 * sub + lane;
-        int s = 0;
-        uint32_t ph = 0;
+        const int ri = 16 * sub + (lane & 15), hcol = lane >> 4;   // row; column half (M = 64 rows in lanes 0..15)
         for (int it = 0; it < nchunks; ++it) {
             const uint32_t pc = (uint32_t)(it & 1);
-            bool got = LA_RWAIT(&full[s], ph, 0x100u);
-            if (got && it > 0) got = LA_RWAIT(dsfull, pc ^ 1u, 0x200u);   // K^ buffer free
-            got = __all_sync(0xffffffffu, got);
+            // P~ of the previous chunk: its O_intra completed before this chunk's P, which pfull tracks
+            const bool got = __all_sync(0xffffffffu, LA_RWAIT(pfull, pc, 0x400u));
             if (!got) break;
-            // forwards in time the weights count back from the chunk's last valid row, so
-            // that the state after a partial last chunk is the state after token T - 1
-            const int rows = min(kC, T - (rev ? nchunks - 1 - it : it) * kC);
-            const float f = rev ? gpow[krow] : (krow < rows ? gpow[rows - 1 - krow] : 0.f);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int ch = part * 8 + i;               // 0..15 across the two boxes
-                const int off = (ch >> 3) * kBox + krow * 128 + (((ch & 7) ^ (krow & 7)) << 4);
-                const uint4 u = *reinterpret_cast<const uint4 *>(sK + s * kTile128 + off);
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float2 x = h2<true>::to_f2(w[k]);
-                    const float a = x.x * f, b = x.y * f;
-                    hi[k] = h2<true>::from_f2(a, b);
-                    const float2 hv = h2<true>::to_f2(hi[k]);
-                    lo[k] = h2<true>::from_f2(a - hv.x, b - hv.y);
-                }
-                *reinterpret_cast<uint4 *>(sKh + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(sKh + kTile128 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(khready);
-            // ---- P~ = (Q K^T) o M, hi + lo (P~ of the previous chunk: its O_intra
-            //      completed before this chunk's P, which pfull tracks)
-            got = __all_sync(0xffffffffu, LA_RWAIT(pfull, pc, 0x400u));
-            if (!got) break;
+            __syncwarp();   // converged for the .sync.aligned TMEM loads
             tc_fence_after();
+            // lanes 0..15 take columns 0..31 of their row, lanes 16..31 columns 32..63
 #pragma unroll
-            for (int c16 = 0; c16 < 4; ++c16) {
+            for (int h16 = 0; h16 < 2; ++h16) {
+                const int c16 = 2 * hcol + h16;
                 float x[16];
-                tmem_ld16(tmem + cP + lanes + 16 * c16, x);
-                tmem_ld_wait();
-                if (lane < 16) {
+                tmem_ld16_halves<32>(tmem + cP + lanes + 16 * h16, x);
+                tmem_ld_wait(x);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int j = 16 * c16 + e;
-                        const int dlt = rev ? j - ri : ri - j;     // causal: i >= j; backwards: j >= i
-                        x[e] = dlt >= 0 ? x[e] * gpow[dlt] : 0.f;
-                    }
-                    uint32_t hw[8], lw[8];
-                    split_hi_lo16_packed(x, hw, lw);
-                    store_chunk16_packed(sPt, ri, c16, hw);
-                    store_chunk16_packed(sPt + kBox, ri, c16, lw);
+                for (int e = 0; e < 16; ++e) {
+                    const int j = 16 * c16 + e;
+                    const int dlt = rev ? j - ri : ri - j;     // causal: i >= j; backwards: j >= i
+                    x[e] = dlt >= 0 ? x[e] * gpow[dlt] : 0.f;
                 }
+                uint32_t hw[8], lw[8];
+                split_hi_lo16_packed(x, hw, lw);
+                store_chunk16_packed(sPt, ri, c16, hw);
+                if (nlp == 2) store_chunk16_packed(sPt + kBox, ri, c16, lw);
             }
             tc_fence_before();
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(ptready);
-            if (++s == NST) { s = 0; ph ^= 1; }
         }
     } else if (warp < kRSw0) {
         // Output warps: o = O_intra + diag(gamma^(i+1)) O_inter (backwards: gamma^(C-i)),
@@ -367,7 +366,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         const int ot = threadIdx.x - kROw0 * 32;
         const int sub = warp & 3;
         const uint32_t lanes = (uint32_t)(32 * sub) << 16;
-        const int ri = 16 * sub + lane;
+        const int ri = 16 * sub + (lane & 15), hcol = lane >> 4;   // row; column half (M = 64 rows in lanes 0..15)
         bool live = true;
         for (int it = 0; it < nchunks; ++it) {
             const int c = rev ? nchunks - 1 - it : it;
@@ -378,19 +377,21 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             got = __all_sync(0xffffffffu, got);
             live = live && got;
             if (got) {
+                __syncwarp();   // converged for the .sync.aligned TMEM loads
                 tc_fence_after();
                 // backwards the entering state sits one past the chunk's last valid row
                 const int rows = min(kC, T - c * kC);
                 const float g1 = rev ? (ri < rows ? gpow[rows - ri] : 0.f) : gpow[ri + 1];
+                // lanes 0..15 take columns 0..63 of their row, lanes 16..31 columns 64..127
 #pragma unroll
-                for (int c16 = 0; c16 < 8; ++c16) {
+                for (int h16 = 0; h16 < 4; ++h16) {
                     float a[16], b[16];
-                    tmem_ld16(tmem + cOI + lanes + 16 * c16, a);
-                    tmem_ld16(tmem + cOX + lanes + 16 * c16, b);
-                    tmem_ld_wait();
+                    tmem_ld16_halves<64>(tmem + cOI + lanes + 16 * h16, a);
+                    tmem_ld16_halves<64>(tmem + cOX + lanes + 16 * h16, b);
+                    tmem_ld_wait(a, b);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) a[i] = fmaf(g1, b[i], a[i]);
-                    if (lane < 16) st16_wide(sO, kBox, ri, c16, a);
+                    st16_wide(sO, kBox, ri, 4 * hcol + h16, a);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -440,7 +441,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                 uint32_t hw[8], lw[8];
                 split_hi_lo16_packed(*reinterpret_cast<const float(*)[16]>(&st[16 * c4]), hw, lw);
                 store_chunk16_packed(sS + half * 16384, d, c4, hw);
-                store_chunk16_packed(sS + 32768 + half * 16384, d, c4, lw);
+                if (nls == 2) store_chunk16_packed(sS + 32768 + half * 16384, d, c4, lw);
             }
             fence_async_smem();
         } else {
@@ -449,10 +450,30 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(sready);                // S_0
-        for (int it = 0; it < nchunks; ++it) {
+        // K^ = diag(gamma^(C-1-j)) K of chunk iteration itk as hi + lo, written while Q S of
+        // the previous chunk runs: thread kt takes row kt % 64 and the 8-element chunks
+        // 4 (kt / 64) .. + 3 of the row's 16.  Forwards in time the weights count back from
+        // the chunk's last valid row, so that the state after a partial last chunk is the
+        // state after token T - 1.
+        const int kt = threadIdx.x - kRSw0 * 32;
+        const int krow = kt & 63, kpart = kt >> 6;
+        auto build_khat = [&](int itk) -> bool {
+            const int sk = itk % NST;
+            if (!__all_sync(0xffffffffu, LA_RWAIT(&full[sk], (uint32_t)((itk / NST) & 1), 0x100u))) return false;
+            const int rows = min(kC, T - (rev ? nchunks - 1 - itk : itk) * kC);
+            const float f = rev ? gpow[krow] : (krow < rows ? gpow[rows - 1 - krow] : 0.f);
+            scale_split_row(sK + sk * kTile128, sKh, krow, kpart, f, nlk == 2);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(khready);
+            return true;
+        };
+        const bool k0 = nchunks > 0 && build_khat(0);
+        for (int it = 0; it < nchunks && k0; ++it) {
             const uint32_t pc = (uint32_t)(it & 1);
             bool got = __all_sync(0xffffffffu, LA_RWAIT(dsfull, pc, 0x1000u));
             if (!got) break;
+            __syncwarp();   // converged for the .sync.aligned TMEM loads
             tc_fence_after();
             const uint32_t base = tmem + cDS + lanes + 64u * half;
             const float g = (it == (rev ? 0 : nchunks - 1)) ? gLast : gC;
@@ -460,13 +481,15 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             for (int c4 = 0; c4 < 4; ++c4) {
                 float a[16];
                 tmem_ld16(base + 16 * c4, a);
-                tmem_ld_wait();
+                tmem_ld_wait(a);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) st[16 * c4 + i] = fmaf(g, st[16 * c4 + i], a[i]);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(dsread);
+            // dS_c is complete, so it has read K^_c: the buffer takes K^ of the next chunk
+            if (it + 1 < nchunks && !build_khat(it + 1)) break;
             got = __all_sync(0xffffffffu, LA_RWAIT(sfree, pc, 0x2000u));   // Q S_c has read the operand
             if (!got) break;
             // the 64 columns are columns 0..63 of box `half` (each box holds 64 state columns)
@@ -475,7 +498,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                 uint32_t hw[8], lw[8];
                 split_hi_lo16_packed(*reinterpret_cast<const float(*)[16]>(&st[16 * c4]), hw, lw);
                 store_chunk16_packed(sS + half * 16384, d, c4, hw);
-                store_chunk16_packed(sS + 32768 + half * 16384, d, c4, lw);
+                if (nls == 2) store_chunk16_packed(sS + 32768 + half * 16384, d, c4, lw);
             }
             fence_async_smem();
             __syncwarp();
@@ -512,6 +535,7 @@ la_status retention_fwd(const void *q, const void *k, const void *v, void *o, co
     memset(&jobs, 0, sizeof jobs);
     jobs.sin[0] = sin;
     jobs.sout[0] = sout;
+    jobs.lo[0] = kLoK | kLoP | kLoS;
     LA_TRY(retention_map(&jobs.q[0], q, s));
     LA_TRY(retention_map(&jobs.k[0], k, s));
     LA_TRY(retention_map(&jobs.v[0], v, s));
@@ -549,6 +573,7 @@ la_status retention_bwd(const void *q, const void *k, const void *v, const void 
         jobs.sin[np] = all[p].sin;
         jobs.sin_t[np] = all[p].sin_t;
         jobs.sout[np] = all[p].sout;
+        jobs.lo[np] = kLoK | kLoP | kLoS;
     }
     return launch_pdl("tc_retention_bwd", retention_kernel, dim3((unsigned)(np * s.BH())), dim3(kRThreads),
                   (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
@@ -563,3 +588,4 @@ unsigned int read_and_clear_retention_fault() {
 
 }  // namespace tc
 }  // namespace la
+

@@ -242,7 +242,7 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             if (BIDIR) {
                 float t16[16];
                 tmem_ld16(base + 64, t16);
-                tmem_ld_wait();
+                tmem_ld_wait(t16);
                 zz = t16[0];
             }
             tc_fence_before();
@@ -477,7 +477,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 if (BIDIR) {
                     float t16[16];
                     tmem_ld16(base + 64, t16);
-                    tmem_ld_wait();
+                    tmem_ld_wait(t16);
                     inv = 1.f / (t16[0] + eps * sc);
                 }
                 float v[64];
@@ -804,7 +804,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                     float a0[16], a1[16];
                     tmem_ld16(d2 + 32 * hf, a0);
                     tmem_ld16(d2 + 32 * hf + 16, a1);
-                    tmem_ld_wait();
+                    tmem_ld_wait(a0, a1);
                     if (hf == 1) {   // every TMEM read of this accumulator pair is complete
                         tc_fence_before();
                         __syncwarp();
@@ -917,7 +917,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 if (BIDIR) {
                     float t16[16];
                     tmem_ld16(base + 64, t16);
-                    tmem_ld_wait();
+                    tmem_ld_wait(t16);
                     zz = t16[0];
                 }
                 tc_fence_before();
@@ -961,6 +961,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 float u[64], t16[16];   // u = f(q) S, t16[0] = f(q).z (one wait for all five loads)
                 tmem_ld16(d1 + 64, t16);
                 tmem_row64(d1, u);
+                reg_keep(t16);   // loaded before the wait inside tmem_row64
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc12empty[b]);
@@ -1218,11 +1219,11 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                     if (BIDIR) {
                         float kf[16];
                         load_chunk16<BF16>(sK + s * kTileBytes, row, c16, kf);
-                        tmem_ld_wait();
+                        tmem_ld_wait(aa, bb);
 #pragma unroll
                         for (int i = 0; i < 16; ++i) out[i] = fmaf(aa[i], cur_isd, dz[16 * c16 + i]) * fminf(kf[i], 1.f);
                     } else {
-                        tmem_ld_wait();
+                        tmem_ld_wait(aa, bb);
 #pragma unroll
                         for (int i = 0; i < 16; ++i) out[i] = aa[i] * cur_isd;
                     }
