@@ -47,10 +47,9 @@ __host__ __device__ inline int max_slots(int BH) { return (kGrid + BH - 1) / BH 
 
 // ------------------------------------------------------------ 16-bit I/O --
 // Packed pairs travel as uint32_t.  Reinterpreting a local through a pointer of
-// another type breaks C++'s aliasing rules, and the optimiser is then free to
-// read a value that was never stored (a bf16 pair read back as zero after it was
-// packed made a hi + lo split return lo = x); memcpy is the defined bit copy and
-// compiles to a register move.
+// another type breaks C++'s aliasing rules (the optimiser may then assume the
+// two never alias); memcpy is the defined bit copy and compiles to a register
+// move.
 template <typename To, typename From>
 __device__ __forceinline__ To bit_cast32(const From &x) {
     static_assert(sizeof(To) == 4 && sizeof(From) == 4, "32-bit values only");

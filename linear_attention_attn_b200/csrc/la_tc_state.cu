@@ -549,6 +549,7 @@ struct BwdQLayout {
     static constexpr int misc = baroff + nbars * 8;
     static constexpr int bytes = misc + 32 + 1024;
     static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
+    static_assert(kStateElems * 4 <= 2 * OPB, "the operand block stages a [dS | dz] partial");
 };
 
 template <bool BIDIR, bool BF16>
@@ -587,7 +588,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     uint64_t *opready = accSfree + 1;
     uint64_t *drain = opready + 1;
     uint64_t *drain2 = drain + 1;
-    uint64_t *stfull = drain2 + 1;       // the first head's state copied into the staging block
+    uint64_t *stfull = drain2 + 1;       // a head's state copied into the staging block ahead of its build
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc);
     int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
 
@@ -871,12 +872,17 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 
         float *isc3 = reinterpret_cast<float *>(smem + L::iscoff);
         int hidx = -1;
+        int copies = src_single ? 1 : 0;   // bulk copies of a head's state into the staging block so far
+        int landed = 0;                    // ... seen complete
         auto build = [&](long long h, int zb) {
             const float *srch = src + h * (long long)src_per_head;
             const int ns = src_single ? 1 : (P.last_cta((int)h) - P.first_cta((int)h) + 1);
             float m;
-            if (src_single && hidx == 0) {   // copied by the TMA thread at the start
-                if (!LA_WAIT(stfull, 0, 0x800u)) live = false;
+            if (src_single) {   // copied ahead: the first head by the TMA thread, the next ones below
+                if (LA_WAIT(stfull, (uint32_t)(hidx & 1), 0x800u))
+                    ++landed;
+                else
+                    live = false;
                 m = stage_absmax(stage, tid);
             } else {
                 m = gather_state(srch, ns, stage, tid);
@@ -900,9 +906,21 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             cur_sc = sc;
             cur_scn = scn;
             if (tid == 0) mbar_arrive(opready);
+            // the staging block is read: the next head of this CTA's range comes in behind
+            // the current head's tiles instead of at the switch
+            if (src_single && tid == 0 && live && (h + 1) * nt < x1) {
+                mbar_arrive_expect_tx(stfull, kStateElems * 4);
+                bulk_load(stage, src + (h + 1) * (long long)src_per_head, kStateElems * 4, stfull);
+                ++copies;
+            }
         };
 
-        // [dS | dz] partial of the segment of head hs that just ended
+        // [dS | dz] partial of the segment of head hs that just ended.  It is staged in the
+        // state operand block: its last readers, MMA1 and MMA2 of the segment's last tile,
+        // completed before acc12full, which these warps waited for in that tile's epilogue,
+        // and the next head's operand is built only after the copy (the staging block holds
+        // that head's state, copied in ahead).
+        float *accst = reinterpret_cast<float *>(sOp);
         auto read_accS = [&](int hs, float scn) {
             bool got = live && LA_WAIT(accSfull, sfull_ph, 0x100u);
             got = __all_sync(0xffffffffu, got);
@@ -923,22 +941,22 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(accSfree);
-                if (lane < 16) {   // row i of [dS | dz] into the staging block (stride 65: no bank conflicts)
+                if (lane < 16) {   // row i of [dS | dz] into the operand block (stride 65: no bank conflicts)
                     const int i = 16 * sub + lane;
                     const float is = 1.f / scn;
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) stage[i * 65 + c] = v[c] * is;
-                    stage[i * 65 + 64] = zz * is;
+                    for (int c = 0; c < 64; ++c) accst[i * 65 + c] = v[c] * is;
+                    accst[i * 65 + 64] = zz * is;
                 }
             }
             named_bar(1, kWorkers);
             if (live) {            // the slot as one contiguous, coalesced 16.6 KB copy
                 float4 *dst = reinterpret_cast<float4 *>(dpart + ((long long)hs * maxslots + (cta - P.first_cta(hs))) *
                                                                      kStateElems);
-                const float4 *src4 = reinterpret_cast<const float4 *>(stage);
+                const float4 *src4 = reinterpret_cast<const float4 *>(accst);
                 for (int e = tid; e < kStateElems / 4; e += kWorkers) dst[e] = src4[e];
             }
-            named_bar(1, kWorkers);   // the staging block is free for the next head's gather
+            named_bar(1, kWorkers);   // the operand block is free for the next head's operand
         };
 
         float2 *rinfo = reinterpret_cast<float2 *>(smem + L::rioff);
@@ -997,6 +1015,10 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             b ^= 1;
             if (b == 0) bph ^= 1;
         }
+        // a copy issued after the last wait that gave up lands before the CTA exits (only the
+        // last one can be unseen: no copy is issued once a wait has failed)
+        if (tid == 0 && copies > landed)
+            mbar_wait_slow(smem_u32(stfull), (uint32_t)((copies - 1) & 1), nullptr, &g_tc_fault, 0x800u);
     }
     tc_fence_before();
     __syncthreads();
