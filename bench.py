@@ -56,6 +56,20 @@ KERNEL_TENSORS = {
     "tc_retention_fwd": 4, "tc_retention_bwd": 7,
 }
 
+# CUDA-core (FMA) work of the recurrent causal-norm kernels per token-head, in flops (2 per FMA):
+# the forward's D+1 state columns each take D FMAs to update and D to form the output; the dq
+# pass adds the D rows (update and row sum); the dk, dv pass holds D rows and D columns.
+CAUSAL_FLOPS = {
+    "simt_causal_norm_fwd": lambda D: 4 * D * (D + 1),
+    "simt_causal_norm_bwd_q": lambda D: 4 * D * (D + 1) + 4 * D * D,
+    "simt_causal_norm_bwd_kv": lambda D: 8 * D * D,
+}
+
+
+def fp32_fma_peak_tflops(sm_mhz):
+    """FP32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops per clock."""
+    return 148 * 128 * 2 * (sm_mhz or 1965.0) * 1e6 / 1e12
+
 
 # ------------------------------------------------------------------ ranks --
 
@@ -197,6 +211,9 @@ def _oracle_step(w, q, k, v, g, gamma, nthreads):
     elif w.op == "simple":
         oracle.simple_fwd(q, k, v, nthreads=nthreads)
         oracle.simple_bwd(q, k, v, g, nthreads=nthreads)
+    elif w.op == "causal_norm":
+        oracle.causal_norm_fwd(q, k, v, None, "elu1", w.eps, nthreads=nthreads)
+        oracle.causal_norm_bwd(q, k, v, g, None, "elu1", w.eps, nthreads=nthreads)
     else:
         oracle.retention_fwd(q, k, v, gamma, nthreads=nthreads)
         oracle.retention_bwd(q, k, v, g, gamma, nthreads=nthreads)
@@ -278,6 +295,9 @@ WORKLOAD_TEXT = {
               "q,k ~ N(0,1) D^-1/2, v, dO ~ N(0,1)",
     "retention": "chunked causal decay (retention) fwd+bwd, bf16 storage / fp32 accumulate, B=%d H=%d T=%d D=%d, "
                  "gamma_h = 1 - 2^(-5-7h/(H-1)), q ~ N(0,1) D^-1/2, k, v, dO ~ N(0,1)",
+    "causal_norm": "causal linear attention with the norm term fwd+bwd (recurrent form on CUDA cores), fp16 storage / "
+                   "fp32 accumulate, B=%d H=%d T=%d D=%d, phi=elu+1, no decay, eps=1e-06, Q,K,V ~ 0.5 N(0,1), "
+                   "dO ~ N(0,1)",
 }
 
 
@@ -328,7 +348,7 @@ def run_ours(args, w):
     if seqpar:
         # the workload's T is the whole sequence; this rank holds a shard of T / world tokens
         from linear_attention_attn_b200 import seqpar as sp
-        if w.op == "retention" or w.T % world:
+        if w.op in ("retention", "causal_norm") or w.T % world:
             raise SystemExit("--seqpar needs the bidir or simple workload and T divisible by the GPU count")
         host = synth.make_inputs(w.with_T(w.T // world), seed=rank)
     else:
@@ -340,7 +360,8 @@ def run_ours(args, w):
     state = torch.empty((B, H, D, D + 1), dtype=torch.float32, device=dev)
     dstate = torch.empty_like(state)
     names = {"bidir": ("bidir_fwd", "bidir_bwd"), "simple": ("simple_fwd", "simple_bwd"),
-             "retention": ("chunk_decay_fwd", "chunk_decay_bwd")}[w.op]
+             "retention": ("chunk_decay_fwd", "chunk_decay_bwd"),
+             "causal_norm": ("causal_norm_fwd", "causal_norm_bwd")}[w.op]
     if seqpar:
         names = ("state_reduce", "state_bwd_q")
     ws_bytes = max(la.la_workspace_size(n, B, H, T, D, q.dtype) for n in names)
@@ -358,6 +379,9 @@ def run_ours(args, w):
         elif w.op == "simple":
             la.la_simple_fwd(q, k, v, o, state, workspace=ws)
             la.la_simple_bwd(q, k, v, g, dq, dk, dv, state, workspace=ws)
+        elif w.op == "causal_norm":
+            la.la_causal_norm_fwd(q, k, v, o, None, "elu1", w.eps)
+            la.la_causal_norm_bwd(q, k, v, g, dq, dk, dv, None, "elu1", w.eps, workspace=ws)
         else:
             la.la_chunk_decay_fwd(q, k, v, o, gamma, workspace=ws)
             la.la_chunk_decay_bwd(q, k, v, g, gamma, dq, dk, dv, workspace=ws)
@@ -444,6 +468,9 @@ def run_ours(args, w):
         elif w.op == "simple":
             la.la_simple_fwd(xq, xk, xv, xo, xst, workspace=ws, stream=s_cmp)
             la.la_simple_bwd(xq, xk, xv, xg, xdq, xdk, xdv, xst, workspace=ws, stream=s_cmp)
+        elif w.op == "causal_norm":
+            la.la_causal_norm_fwd(xq, xk, xv, xo, None, "elu1", w.eps, stream=s_cmp)
+            la.la_causal_norm_bwd(xq, xk, xv, xg, xdq, xdk, xdv, None, "elu1", w.eps, workspace=ws, stream=s_cmp)
         else:
             la.la_chunk_decay_fwd(xq, xk, xv, xo, gamma, workspace=ws, stream=s_cmp)
             la.la_chunk_decay_bwd(xq, xk, xv, xg, gamma, xdq, xdk, xdv, workspace=ws, stream=s_cmp)
@@ -494,6 +521,15 @@ def run_ours(args, w):
             roof = {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak, "peak_source": peak_kind, "traffic": traffic,
                     "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_ms": tot_ms / n_launch,
+                    "share_of_step": tot_ms / max(1e-9, sum(r[2] for r in per_kernel))}
+        elif name in CAUSAL_FLOPS and n_launch > 0:
+            flops = CAUSAL_FLOPS[name](D) * B * H * T
+            avg_s = tot_ms / n_launch / 1e3
+            fpeak = fp32_fma_peak_tflops((clocks or {}).get("sm_mhz"))
+            roof = {"bound": "alu", "kernel": name, "achieved": flops / avg_s / 1e12, "peak": fpeak,
+                    "unit": "TFLOP/s", "frac": flops / avg_s / 1e12 / fpeak,
+                    "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 flops x the sampled SM clock",
+                    "traffic": None, "algorithmic_flops_per_launch": flops, "avg_launch_ms": tot_ms / n_launch,
                     "share_of_step": tot_ms / max(1e-9, sum(r[2] for r in per_kernel))}
     step_bytes = 11 * tensor_bytes
     peak, peak_kind = measured_peaks()
@@ -703,9 +739,10 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--T", type=int, default=None, help="sequence length (default: the workload's)")
-    ap.add_argument("--workload", choices=["bidir", "simple", "retention", "decode"], default="bidir",
+    ap.add_argument("--workload", choices=["bidir", "simple", "retention", "decode", "causal_norm"], default="bidir",
                     help="bidir (the benchmark metric, B8 H16 D64 fp16), simple (B8 H16 D64 bf16), "
-                         "retention (B8 H32 D128 bf16) or decode (recurrent decay step, B64 H32 D128)")
+                         "retention (B8 H32 D128 bf16), decode (recurrent decay step, B64 H32 D128) or "
+                         "causal_norm (causal linear attention with the norm term, B8 H16 D64 fp16)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seqpar", action="store_true",
                     help="bidir/simple: split the workload's sequence along T across the GPUs (one all-reduce of "
@@ -723,7 +760,8 @@ def main(argv=None):
         if args.impl == "reference":
             return run_decode_reference(args)
         return run_decode(args)
-    base = {"bidir": "bidir_f16", "simple": "simple_bf16", "retention": "retention_bf16"}[args.workload]
+    base = {"bidir": "bidir_f16", "simple": "simple_bf16", "retention": "retention_bf16",
+            "causal_norm": "causal_norm_f16"}[args.workload]
     w = synth.WORKLOADS[base]
     w = w.with_T(args.T if args.T is not None else (4096 if args.workload != "retention" else 8192))
     if args.impl == "reference":

@@ -74,7 +74,9 @@ typedef enum {
     LA_OP_STATE_REDUCE = 6,
     LA_OP_STATE_APPLY = 7,
     LA_OP_STATE_BWD_Q = 8,
-    LA_OP_STATE_BWD_KV = 9
+    LA_OP_STATE_BWD_KV = 9,
+    LA_OP_CAUSAL_NORM_FWD = 10,
+    LA_OP_CAUSAL_NORM_BWD = 11
 } la_op;
 
 /* Feature map of the sequence-parallel stages: elu+1 with the norm term (the
@@ -225,6 +227,37 @@ la_status la_chunk_decay_bwd_state(const void *q, const void *k, const void *v, 
  * 1 <= n <= LA_MAX_SCAN_SEGMENTS (else LA_ERR_UNSUPPORTED). */
 la_status la_chunk_decay_scan(const float *states, const long long *gaps, int n, const float *decay,
                               float *out, int B, int H, int D, void *stream);
+
+/* ---- causal linear attention with the norm term ---------------------------
+ * The causal counterpart of la_bidir_*: every token sees only the tokens up to
+ * itself, with an optional per-head decay:
+ *   S_t = gamma_h S_{t-1} + f(k_t)^T v_t,  z_t = gamma_h z_{t-1} + f(k_t)
+ *   o_t = f(q_t) S_t / (f(q_t) . z_t + eps)
+ * f = elu + 1 (LA_FEATURE_ELU1) or the identity (LA_FEATURE_IDENTITY; then
+ * f(q_t) . z_t may come near -eps, which the caller must rule out).  decay is a
+ * HOST array of H values in (0, 1], read during the call, or NULL for gamma = 1:
+ * plain causal linear attention with the norm term.  Without the norm term the
+ * op is la_chunk_decay_* (identity f, gamma = 1 for plain causal linear
+ * attention).  Sources: "flash-linear-attention" README, "Different forms of
+ * linear attention" (FusedRecurrent: the recurrent form these calls compute);
+ * the norm term and f as in la_bidir_*.  Computed on CUDA cores, fp32, one CTA
+ * per (b, h) walking the sequence; all dtypes, D in {64, 128}. */
+la_status la_causal_norm_fwd(const void *q, const void *k, const void *v, void *o, const float *decay,
+                             la_feature feature, float eps, int B, int H, int T, int D, la_dtype dtype,
+                             void *stream);
+
+/* Gradients of sum(o * dout) for la_causal_norm_fwd.  With u_t = f(q_t) S_t,
+ * n_t = f(q_t) . z_t + eps, o_t = u_t / n_t, du_t = dout_t / n_t and
+ * dn_t = -(dout_t . o_t) / n_t:
+ *   dq_t = (S_t du_t + z_t dn_t) f'(q_t)
+ *   R_s = sum_{t>=s} gamma^(t-s) f(q_t)^T du_t,  r_s = sum_{t>=s} gamma^(t-s) f(q_t) dn_t
+ *   dk_s = (R_s v_s + r_s) f'(k_s),  dv_s = f(k_s) R_s.
+ * Workspace: la_workspace_size(LA_OP_CAUSAL_NORM_BWD, ...) bytes ((n_t, dn_t)
+ * of every row, 8 B per token-head). */
+la_status la_causal_norm_bwd(const void *q, const void *k, const void *v, const void *dout, const float *decay,
+                             la_feature feature, float eps, void *dq, void *dk, void *dv,
+                             int B, int H, int T, int D, la_dtype dtype,
+                             void *workspace, size_t workspace_bytes, void *stream);
 
 /* ---- the state form in stages, for a sequence split along T -------------
  * A sequence cut into shards along T (one per rank or per call) gives each

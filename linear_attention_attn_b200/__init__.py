@@ -28,7 +28,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 LA_F32, LA_F16, LA_BF16 = 0, 1, 2
 OPS = {"bidir_fwd": 0, "bidir_bwd": 1, "simple_fwd": 2, "simple_bwd": 3,
        "chunk_decay_fwd": 4, "chunk_decay_bwd": 5, "state_reduce": 6, "state_apply": 7,
-       "state_bwd_q": 8, "state_bwd_kv": 9}
+       "state_bwd_q": 8, "state_bwd_kv": 9, "causal_norm_fwd": 10, "causal_norm_bwd": 11}
 FEATURES = {"identity": 0, "elu1": 1}
 STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_ALIGNMENT",
           4: "LA_ERR_WORKSPACE", 5: "LA_ERR_CUDA", 6: "LA_ERR_TIMEOUT"}
@@ -57,13 +57,16 @@ _lib.la_chunk_decay_fwd_state.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I
 _lib.la_chunk_decay_bwd_state.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z,
                                           _P]
 _lib.la_chunk_decay_scan.argtypes = [_P, _P, _I, _P, _P, _I, _I, _I, _P]
+_lib.la_causal_norm_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _F, _I, _I, _I, _I, _I, _P]
+_lib.la_causal_norm_bwd.argtypes = [_P, _P, _P, _P, _P, _I, _F, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_state_reduce.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_state_apply.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
 _lib.la_state_bwd_q.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]
 _lib.la_state_bwd_kv.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]
 for _n in ("la_bidir_fwd", "la_simple_fwd", "la_bidir_bwd", "la_simple_bwd", "la_chunk_decay_fwd",
            "la_chunk_decay_bwd", "la_chunk_decay_step", "la_chunk_decay_fwd_state", "la_chunk_decay_bwd_state",
-           "la_chunk_decay_scan", "la_state_reduce", "la_state_apply", "la_state_bwd_q", "la_state_bwd_kv"):
+           "la_chunk_decay_scan", "la_state_reduce", "la_state_apply", "la_state_bwd_q", "la_state_bwd_kv",
+           "la_causal_norm_fwd", "la_causal_norm_bwd"):
     getattr(_lib, _n).restype = _I
 _lib.la_bidir_fwd_static.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.la_bidir_fwd_static.restype = _I
@@ -300,6 +303,33 @@ def la_chunk_decay_scan(states, gaps, decay, out, stream=None):
     dec = _decay(decay, H)
     _check(_lib.la_chunk_decay_scan(_ptr(states), ctypes.cast(garr, _P), n, ctypes.cast(dec, _P), _ptr(out), B, H,
                                     D, _stream(stream, states.device)), "la_chunk_decay_scan")
+
+
+def _decay_or_null(decay, H):
+    return (None, None) if decay is None else (lambda a: (ctypes.cast(a, _P), a))(_decay(decay, H))
+
+
+def la_causal_norm_fwd(q, k, v, o, decay=None, feature="elu1", eps: float = 1e-6, stream=None):
+    """Causal linear attention with the norm term: o_t <- f(q_t) S_t / (f(q_t) . z_t + eps), S_t and
+    z_t the decay[h]-weighted sums over s <= t of f(k_s)^T v_s and f(k_s) (decay None: 1)."""
+    B, H, T, D = _shape(q, k, v, o)
+    dp, _keep = _decay_or_null(decay, H)
+    _check(_lib.la_causal_norm_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), dp, _feature(feature),
+                                   ctypes.c_float(eps), B, H, T, D, _dtype_code(q), _stream(stream, q.device)),
+           "la_causal_norm_fwd")
+
+
+def la_causal_norm_bwd(q, k, v, dout, dq, dk, dv, decay=None, feature="elu1", eps: float = 1e-6, workspace=None,
+                       stream=None):
+    """dq, dk, dv <- gradients of sum(o * dout) for la_causal_norm_fwd."""
+    B, H, T, D = _shape(q, k, v, dout, dq, dk, dv)
+    dp, _keep = _decay_or_null(decay, H)
+    dt = _dtype_code(q)
+    wp, wn, _wkeep = _workspace("causal_norm_bwd", (B, H, T, D), dt, workspace, q.device, stream)
+    _check(_lib.la_causal_norm_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), dp, _feature(feature),
+                                   ctypes.c_float(eps), _ptr(dq), _ptr(dk), _ptr(dv), B, H, T, D, dt, wp, wn,
+                                   _stream(stream, q.device)),
+           "la_causal_norm_bwd")
 
 
 def la_chunk_decay_step(q, k, v, o, state, decay, stream=None):

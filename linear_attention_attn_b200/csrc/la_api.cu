@@ -273,7 +273,7 @@ size_t la_workspace_size(la_op op, int B, int H, int T, int D, la_dtype dtype) {
     const Shape s{B, H, T, D};
     if (s.B < 1 || s.H < 1 || s.T < 0 || (s.D != 64 && s.D != 128)) return 0;
     if (dtype != LA_F32 && dtype != LA_F16 && dtype != LA_BF16) return 0;
-    if ((int)op < 0 || (int)op > (int)LA_OP_STATE_BWD_KV) return 0;
+    if ((int)op < 0 || (int)op > (int)LA_OP_CAUSAL_NORM_BWD) return 0;
     return ws_size(op, s, dtype);
 }
 
@@ -394,6 +394,52 @@ la_status la_chunk_decay_bwd_state(const void *q, const void *k, const void *v, 
                                    la_dtype dtype, void *workspace, size_t workspace_bytes, void *stream) {
     return decay_bwd_entry(q, k, v, dout, state_in, dstate_in, dstate_out, decay, dq, dk, dv, B, H, T, D, dtype,
                            workspace, workspace_bytes, stream, true);
+}
+
+// Common front half of the causal-norm entry points.
+static la_status causal_entry(const Shape &s, la_dtype dt, const float *decay, la_feature f, float eps,
+                              DecayArgs *dec, int *has_decay) {
+    LA_TRY(validate(s, dt));
+    if (f != LA_FEATURE_IDENTITY && f != LA_FEATURE_ELU1) return fail(LA_ERR_UNSUPPORTED, "unknown feature map %d", (int)f);
+    if (!(eps >= 0.f) || !isfinite(eps)) return fail(LA_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    *has_decay = decay != nullptr;
+    if (decay) LA_TRY(decay_args(decay, s.H, dec));
+    return LA_OK;
+}
+
+la_status la_causal_norm_fwd(const void *q, const void *k, const void *v, void *o, const float *decay,
+                             la_feature feature, float eps, int B, int H, int T, int D, la_dtype dtype, void *stream) {
+    const Shape s{B, H, T, D};
+    DecayArgs dec;
+    int has_decay = 0;
+    LA_TRY(causal_entry(s, dtype, decay, feature, eps, &dec, &has_decay));
+    LA_TRY(check_ptr(q, "q"));
+    LA_TRY(check_ptr(k, "k"));
+    LA_TRY(check_ptr(v, "v"));
+    LA_TRY(check_ptr(o, "o"));
+    if (T == 0) return LA_OK;
+    return simt::causal_norm_fwd(q, k, v, o, dec, has_decay, feature == LA_FEATURE_ELU1, s, dtype, eps,
+                                 (cudaStream_t)stream);
+}
+
+la_status la_causal_norm_bwd(const void *q, const void *k, const void *v, const void *dout, const float *decay,
+                             la_feature feature, float eps, void *dq, void *dk, void *dv, int B, int H, int T, int D,
+                             la_dtype dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    const Shape s{B, H, T, D};
+    DecayArgs dec;
+    int has_decay = 0;
+    LA_TRY(causal_entry(s, dtype, decay, feature, eps, &dec, &has_decay));
+    LA_TRY(check_ptr(q, "q"));
+    LA_TRY(check_ptr(k, "k"));
+    LA_TRY(check_ptr(v, "v"));
+    LA_TRY(check_ptr(dout, "dout"));
+    LA_TRY(check_ptr(dq, "dq"));
+    LA_TRY(check_ptr(dk, "dk"));
+    LA_TRY(check_ptr(dv, "dv"));
+    LA_TRY(check_ws(LA_OP_CAUSAL_NORM_BWD, s, dtype, workspace, workspace_bytes));
+    if (T == 0) return LA_OK;
+    return simt::causal_norm_bwd(q, k, v, dout, dq, dk, dv, dec, has_decay, feature == LA_FEATURE_ELU1, s, dtype, eps,
+                                 workspace, (cudaStream_t)stream);
 }
 
 la_status la_chunk_decay_scan(const float *states, const long long *gaps, int n, const float *decay, float *out,

@@ -448,6 +448,212 @@ ret_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
     }
 }
 
+// ----------------------------------------------- causal with the norm term ---
+// Causal linear attention with the norm term and a per-head decay (gamma = 1 for
+// plain causal linear attention), the recurrent form:
+//   S_t = gamma S_{t-1} + f(k_t)^T v_t,  z_t = gamma z_{t-1} + f(k_t)
+//   o_t = f(q_t) S_t / (f(q_t) . z_t + eps),  f = elu + 1 (PHI) or the identity.
+// z is the state's column for a value that is always 1.
+
+// f applied in place to the first `n` tiles of a tile stack (rows past the sequence
+// are never read).
+template <int D, bool PHI>
+__device__ __forceinline__ void feature_tiles(float (*tiles)[kRetTile][D], int n) {
+    if (!PHI) return;
+    for (int e = threadIdx.x; e < n * kRetTile * D; e += blockDim.x) {
+        float *x = &tiles[e / (kRetTile * D)][(e / D) % kRetTile][e % D];
+        *x = feature(*x);
+    }
+}
+// f'(x) from f(x): elu + 1 is x + 1 > 1 for x > 0 (slope 1) and exp(x) <= 1 otherwise.
+template <bool PHI>
+__device__ __forceinline__ float feature_grad_of(float fx) { return PHI ? (fx > 1.f ? 1.f : fx) : 1.f; }
+
+// Forward: threads 0..D-1 hold column j of S, thread D holds z.
+template <typename T, int D, bool PHI>
+__global__ void __launch_bounds__(D + 1)
+causal_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, T *__restrict__ o,
+           DecayArgs dec, int has_decay, int T_len, int H, float eps) {
+    __shared__ float tiles[3][kRetTile][D];
+    __shared__ float acc[kRetTile][D + 1];
+    const int bh = blockIdx.x;
+    const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
+    const long long base = (long long)bh * T_len * D;
+    const int j = threadIdx.x;
+    float S[D];
+#pragma unroll
+    for (int i = 0; i < D; ++i) S[i] = 0.f;
+    const T *const src[3] = {q, k, v};
+    for (int ts = 0; ts < T_len; ts += kRetTile) {
+        __syncthreads();
+        load_rows<T, D, 3>(src, tiles, base, ts, T_len, blockDim.x);
+        __syncthreads();
+        feature_tiles<D, PHI>(tiles, 2);
+        __syncthreads();
+        const int nr = min(kRetTile, T_len - ts);
+        for (int r = 0; r < nr; ++r) {
+            const float vj = j < D ? tiles[2][r][j] : 1.f;
+            float a = 0.f;
+#pragma unroll
+            for (int i = 0; i < D; ++i) {
+                S[i] = fmaf(gamma, S[i], tiles[1][r][i] * vj);
+                a = fmaf(tiles[0][r][i], S[i], a);
+            }
+            acc[r][j] = a;
+        }
+        __syncthreads();
+        if (j < D)
+            for (int r = 0; r < nr; ++r)
+                io<T>::st(o + base + (long long)(ts + r) * D + j, acc[r][j] / (acc[r][D] + eps));
+    }
+}
+
+// Backward, forward sweep: dq, and per row (n_t, dn_t) for the reverse sweep, with
+// u_t = f(q_t) S_t, n_t = f(q_t) . z_t + eps, dn_t = -(dout_t . u_t) / n_t^2:
+//   df(q)_t[i] = (sum_j S_t[i][j] dout_t[j]) / n_t + z_t[i] dn_t,  dq = df(q) f'(q).
+// Threads 0..D hold the columns of [S | z] (u_t and n_t), threads D+1..2D the rows of S
+// and z[i] (the row sums of dq); a tile's rows meet in shared memory.
+template <typename T, int D, bool PHI>
+__global__ void __launch_bounds__(2 * D + 1)
+causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
+             T *__restrict__ dq, float2 *__restrict__ nd, DecayArgs dec, int has_decay, int T_len, int H, float eps) {
+    extern __shared__ float dsm[];               // causal_bwd_q_smem<D>() bytes
+    float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // f(q), f(k), v, dout
+    float(*U)[D + 1] = reinterpret_cast<float(*)[D + 1]>(dsm + 4 * kRetTile * D);  // dout_t[j] u_t[j], n_t - eps
+    float(*A)[D] = reinterpret_cast<float(*)[D]>(dsm + 4 * kRetTile * D + kRetTile * (D + 1));
+    float(*Z)[D] = A + kRetTile;
+    float2 *info = reinterpret_cast<float2 *>(dsm + 6 * kRetTile * D + kRetTile * (D + 1));   // (1 / n_t, dn_t)
+    const int bh = blockIdx.x;
+    const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
+    const long long base = (long long)bh * T_len * D;
+    const bool col_side = threadIdx.x <= D;
+    const int idx = col_side ? threadIdx.x : threadIdx.x - (D + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;   // full warps
+    float Sx[D];
+    float zi = 0.f;
+#pragma unroll
+    for (int i = 0; i < D; ++i) Sx[i] = 0.f;
+    const T *const src[4] = {q, k, v, g};
+    for (int ts = 0; ts < T_len; ts += kRetTile) {
+        __syncthreads();
+        load_rows<T, D, 4>(src, tiles, base, ts, T_len, blockDim.x);
+        __syncthreads();
+        feature_tiles<D, PHI>(tiles, 2);
+        __syncthreads();
+        const int nr = min(kRetTile, T_len - ts);
+        for (int r = 0; r < nr; ++r) {
+            if (col_side) {
+                const float vj = idx < D ? tiles[2][r][idx] : 1.f;
+                float a = 0.f;
+#pragma unroll
+                for (int i = 0; i < D; ++i) {
+                    Sx[i] = fmaf(gamma, Sx[i], tiles[1][r][i] * vj);
+                    a = fmaf(tiles[0][r][i], Sx[i], a);
+                }
+                U[r][idx] = idx < D ? a * tiles[3][r][idx] : a;
+            } else {
+                const float ki = tiles[1][r][idx];
+                float a = 0.f;
+#pragma unroll
+                for (int j = 0; j < D; ++j) {
+                    Sx[j] = fmaf(gamma, Sx[j], ki * tiles[2][r][j]);
+                    a = fmaf(Sx[j], tiles[3][r][j], a);
+                }
+                zi = fmaf(gamma, zi, ki);
+                A[r][idx] = a;
+                Z[r][idx] = zi;
+            }
+        }
+        __syncthreads();
+        for (int r = warp; warp < nwarps && r < nr; r += nwarps) {   // dout_t . u_t, a warp per row, fixed order
+            float p = 0.f;
+            for (int j = lane; j < D; j += 32) p += U[r][j];
+#pragma unroll
+            for (int m = 16; m > 0; m >>= 1) p += __shfl_xor_sync(0xffffffffu, p, m);
+            if (lane == 0) {
+                const float n = U[r][D] + eps, inv = 1.f / n;
+                const float dn = -p * inv * inv;
+                info[r] = make_float2(inv, dn);
+                nd[(long long)bh * T_len + ts + r] = make_float2(n, dn);
+            }
+        }
+        __syncthreads();
+        if (!col_side)
+            for (int r = 0; r < nr; ++r) {
+                const float2 in = info[r];
+                const float d = fmaf(A[r][idx], in.x, Z[r][idx] * in.y);
+                io<T>::st(dq + base + (long long)(ts + r) * D + idx, d * feature_grad_of<PHI>(tiles[0][r][idx]));
+            }
+    }
+}
+
+template <int D>
+constexpr size_t causal_bwd_q_smem() {
+    return (size_t)(6 * kRetTile * D + kRetTile * (D + 1)) * sizeof(float) + kRetTile * sizeof(float2);
+}
+static_assert((6 * kRetTile * 64 + kRetTile * 65) % 2 == 0 && (6 * kRetTile * 128 + kRetTile * 129) % 2 == 0,
+              "the float2 block of causal_bwd_q starts 8-byte aligned");
+
+// Backward, reverse sweep over R_s = gamma R_{s+1} + f(q_s)^T du_s and r_s = gamma r_{s+1} +
+// f(q_s) dn_s with du_s = dout_s / n_s: threads 0..D-1 hold row i of R and r[i]
+// (dk_s[i] = (sum_j R[i][j] v_s[j] + r[i]) f'(k_s[i])), threads D..2D-1 column j of R
+// (dv_s[j] = sum_i f(k_s)[i] R[i][j]).
+template <typename T, int D, bool PHI>
+__global__ void __launch_bounds__(2 * D)
+causal_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
+              const float2 *__restrict__ nd, T *__restrict__ dk, T *__restrict__ dv, DecayArgs dec, int has_decay,
+              int T_len, int H) {
+    __shared__ float tiles[4][kRetTile][D];
+    __shared__ float2 info[kRetTile];
+    const int bh = blockIdx.x;
+    const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
+    const long long base = (long long)bh * T_len * D;
+    const bool row_side = threadIdx.x < D;
+    const int idx = row_side ? threadIdx.x : threadIdx.x - D;
+    float Rx[D];
+    float ri = 0.f;
+#pragma unroll
+    for (int m = 0; m < D; ++m) Rx[m] = 0.f;
+    const T *const src[4] = {q, k, v, g};
+    const int ntiles = (T_len + kRetTile - 1) / kRetTile;
+    for (int tile = ntiles - 1; tile >= 0; --tile) {
+        const int ts = tile * kRetTile;
+        __syncthreads();
+        load_rows<T, D, 4>(src, tiles, base, ts, T_len, blockDim.x);
+        const int nr = min(kRetTile, T_len - ts);
+        if (threadIdx.x < nr) {
+            const float2 x = nd[(long long)bh * T_len + ts + threadIdx.x];
+            info[threadIdx.x] = make_float2(1.f / x.x, x.y);
+        }
+        __syncthreads();
+        feature_tiles<D, PHI>(tiles, 2);
+        __syncthreads();
+        for (int r = nr - 1; r >= 0; --r) {
+            const float2 in = info[r];
+            float acc = 0.f;
+            if (row_side) {
+                const float qi = tiles[0][r][idx];
+#pragma unroll
+                for (int j = 0; j < D; ++j) {
+                    Rx[j] = fmaf(gamma, Rx[j], qi * (tiles[3][r][j] * in.x));
+                    acc = fmaf(Rx[j], tiles[2][r][j], acc);
+                }
+                ri = fmaf(gamma, ri, qi * in.y);
+                const float fk = tiles[1][r][idx];
+                io<T>::st(dk + base + (long long)(ts + r) * D + idx, (acc + ri) * feature_grad_of<PHI>(fk));
+            } else {
+                const float duj = tiles[3][r][idx] * in.x;
+#pragma unroll
+                for (int i = 0; i < D; ++i) {
+                    Rx[i] = fmaf(gamma, Rx[i], tiles[0][r][i] * duj);
+                    acc = fmaf(tiles[1][r][i], Rx[i], acc);
+                }
+                io<T>::st(dv + base + (long long)(ts + r) * D + idx, acc);
+            }
+        }
+    }
+}
+
 // -------------------------------------------------------------- drivers ---
 
 namespace {
@@ -619,6 +825,8 @@ size_t workspace_size(la_op op, const Shape &s) {
     case LA_OP_STATE_REDUCE:
     case LA_OP_STATE_BWD_Q:
         return state_bytes(s, simt_splits(s));
+    case LA_OP_CAUSAL_NORM_BWD:   // (n_t, dn_t) of every row
+        return ((size_t)s.BH() * s.T * sizeof(float2) + 255) / 256 * 256;
     default:
         return 0;
     }
@@ -679,6 +887,58 @@ la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, 
     }
 #undef LA_RET_BWD
 }
+
+namespace {
+
+template <typename T, int D, bool PHI>
+la_status causal_fwd_t(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, int has_decay,
+                       const Shape &s, float eps, cudaStream_t st) {
+    return launch("simt_causal_norm_fwd", causal_fwd<T, D, PHI>, dim3((unsigned)s.BH()), dim3(D + 1), 0, st,
+                  (const T *)q, (const T *)k, (const T *)v, (T *)o, dec, has_decay, s.T, s.H, eps);
+}
+
+template <typename T, int D, bool PHI>
+la_status causal_bwd_t(const void *q, const void *k, const void *v, const void *g, void *dq, void *dk, void *dv,
+                       const DecayArgs &dec, int has_decay, const Shape &s, float eps, void *ws, cudaStream_t st) {
+    float2 *nd = (float2 *)ws;
+    la_status rc = launch("simt_causal_norm_bwd_q", causal_bwd_q<T, D, PHI>, dim3((unsigned)s.BH()),
+                          dim3(2 * D + 1), causal_bwd_q_smem<D>(), st, (const T *)q, (const T *)k, (const T *)v,
+                          (const T *)g, (T *)dq, nd, dec, has_decay, s.T, s.H, eps);
+    if (rc) return rc;
+    return launch("simt_causal_norm_bwd_kv", causal_bwd_kv<T, D, PHI>, dim3((unsigned)s.BH()), dim3(2 * D), 0, st,
+                  (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const float2 *)nd, (T *)dk, (T *)dv, dec,
+                  has_decay, s.T, s.H);
+}
+
+// dtype x D x feature map dispatch of F<T, D, PHI>(args...)
+#define LA_CAUSAL_DISPATCH(F, ...)                                                                  \
+    do {                                                                                           \
+        if (dt == LA_F32) {                                                                        \
+            if (s.D == 64) return phi ? F<float, 64, true>(__VA_ARGS__) : F<float, 64, false>(__VA_ARGS__); \
+            return phi ? F<float, 128, true>(__VA_ARGS__) : F<float, 128, false>(__VA_ARGS__);     \
+        }                                                                                          \
+        if (dt == LA_F16) {                                                                        \
+            if (s.D == 64) return phi ? F<__half, 64, true>(__VA_ARGS__) : F<__half, 64, false>(__VA_ARGS__); \
+            return phi ? F<__half, 128, true>(__VA_ARGS__) : F<__half, 128, false>(__VA_ARGS__);   \
+        }                                                                                          \
+        if (s.D == 64)                                                                             \
+            return phi ? F<__nv_bfloat16, 64, true>(__VA_ARGS__) : F<__nv_bfloat16, 64, false>(__VA_ARGS__); \
+        return phi ? F<__nv_bfloat16, 128, true>(__VA_ARGS__) : F<__nv_bfloat16, 128, false>(__VA_ARGS__); \
+    } while (0)
+
+}  // namespace
+
+la_status causal_norm_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, int has_decay,
+                          bool phi, const Shape &s, la_dtype dt, float eps, cudaStream_t st) {
+    LA_CAUSAL_DISPATCH(causal_fwd_t, q, k, v, o, dec, has_decay, s, eps, st);
+}
+
+la_status causal_norm_bwd(const void *q, const void *k, const void *v, const void *g, void *dq, void *dk, void *dv,
+                          const DecayArgs &dec, int has_decay, bool phi, const Shape &s, la_dtype dt, float eps,
+                          void *ws, cudaStream_t st) {
+    LA_CAUSAL_DISPATCH(causal_bwd_t, q, k, v, g, dq, dk, dv, dec, has_decay, s, eps, ws, st);
+}
+#undef LA_CAUSAL_DISPATCH
 
 }  // namespace simt
 }  // namespace la

@@ -62,9 +62,12 @@ def _bind(lib):
     lib.oracle_retention_step.argtypes = [P, P, P, P, P, P, L, L, L]
     lib.oracle_retention_fwd_state.argtypes = [P, P, P, P, P, P, P, L, L, L, L, I]
     lib.oracle_retention_bwd_state.argtypes = [P, P, P, P, P, P, P, P, P, P, P, L, L, L, L, I]
+    lib.oracle_causal_norm_fwd.argtypes = [P, P, P, P, I, Dbl, P, L, L, L, L, I]
+    lib.oracle_causal_norm_bwd.argtypes = [P, P, P, P, P, I, Dbl, P, P, P, L, L, L, L, I]
     for name in ("oracle_bidir_fwd", "oracle_simple_fwd", "oracle_bidir_bwd",
                  "oracle_simple_bwd", "oracle_retention_fwd", "oracle_retention_bwd",
-                 "oracle_retention_step", "oracle_retention_fwd_state", "oracle_retention_bwd_state"):
+                 "oracle_retention_step", "oracle_retention_fwd_state", "oracle_retention_bwd_state",
+                 "oracle_causal_norm_fwd", "oracle_causal_norm_bwd"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -223,6 +226,38 @@ class Oracle:
         _check(rc, "oracle_retention_bwd_state")
         return dq, dk, dv, rout
 
+    def _causal_args(self, q, gamma, feature):
+        B, H, T, D = _shape4(q)
+        gm = None if gamma is None else _f64(gamma).reshape(-1)
+        if gm is not None and gm.shape[0] != H:
+            raise ValueError("gamma must have H=%d entries" % H)
+        if feature not in ("elu1", "identity"):
+            raise ValueError("feature must be 'elu1' or 'identity'")
+        return (B, H, T, D), gm, 1 if feature == "elu1" else 0
+
+    def causal_norm_fwd(self, q, k, v, gamma=None, feature="elu1", eps: float = 1e-6, nthreads: int | None = None):
+        """Causal linear attention with the norm term: o_t = f(q_t) S_t / (f(q_t) . z_t + eps) with
+        S_t, z_t the gamma-decayed sums over s <= t of f(k_s)^T v_s and f(k_s) (gamma None: 1)."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        (B, H, T, D), gm, up = self._causal_args(q, gamma, feature)
+        o = np.empty_like(q)
+        rc = self._lib.oracle_causal_norm_fwd(_p(q), _p(k), _p(v), None if gm is None else _p(gm), up, float(eps),
+                                              _p(o), B, H, T, D, nthreads or default_threads())
+        _check(rc, "oracle_causal_norm_fwd")
+        return o
+
+    def causal_norm_bwd(self, q, k, v, dout, gamma=None, feature="elu1", eps: float = 1e-6,
+                        nthreads: int | None = None):
+        """Gradients (dq, dk, dv) of sum(o * dout) for causal_norm_fwd."""
+        q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(dout)
+        (B, H, T, D), gm, up = self._causal_args(q, gamma, feature)
+        dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+        rc = self._lib.oracle_causal_norm_bwd(_p(q), _p(k), _p(v), _p(g), None if gm is None else _p(gm), up,
+                                              float(eps), _p(dq), _p(dk), _p(dv), B, H, T, D,
+                                              nthreads or default_threads())
+        _check(rc, "oracle_causal_norm_bwd")
+        return dq, dk, dv
+
     def retention_step(self, q, k, v, gamma, state):
         """One decode step: returns (o, new_state) with new_state = gamma_h state + k^T v and
         o = q new_state; q, k, v are [B, H, D], state is [B, H, D, D] (not modified)."""
@@ -291,3 +326,11 @@ def retention_fwd_state(*a, **kw):
 
 def retention_bwd_state(*a, **kw):
     return _instance().retention_bwd_state(*a, **kw)
+
+
+def causal_norm_fwd(*a, **kw):
+    return _instance().causal_norm_fwd(*a, **kw)
+
+
+def causal_norm_bwd(*a, **kw):
+    return _instance().causal_norm_bwd(*a, **kw)

@@ -26,6 +26,9 @@
  *            o_t = sum_{s<=t} gamma^(t-s) (q_t . k_s) v_s
  *            computed in the recurrent ("FusedRecurrent") form
  *            S_t = gamma S_{t-1} + k_t^T v_t,  o_t = q_t S_t.
+ *   causal with the norm term (plain causal linear attention at gamma = 1):
+ *            S_t = gamma S_{t-1} + f(k_t)^T v_t,  z_t = gamma z_{t-1} + f(k_t)
+ *            o_t = f(q_t) S_t / (f(q_t) . z_t + eps),  f = phi or the identity.
  *
  * The backward formulas are derived by hand from those definitions (chain
  * rule, written out next to each function).  Every function works on one
@@ -420,3 +423,124 @@ int oracle_retention_bwd_state(const double *q, const double *k, const double *v
     jb.B = B; jb.H = H; jb.T = T; jb.D = D;
     return for_each_head(&jb, retention_bwd_head, (size_t)(2 * D * D), nthreads);
 }
+
+/* ------------------------------------- causal with the norm term (recurrent) -- */
+
+static double feat(const job_t *jb, double x) { return jb->use_phi ? phi(x) : x; }
+static double dfeat(const job_t *jb, double x) { return jb->use_phi ? dphi(x) : 1.0; }
+static double head_gamma(const job_t *jb, long bh) { return jb->gamma ? jb->gamma[bh % jb->H] : 1.0; }
+
+/* Forward, one head:
+ *   S_t = gamma S_{t-1} + f(k_t)^T v_t,  z_t = gamma z_{t-1} + f(k_t)   (S_{-1} = 0, z_{-1} = 0)
+ *   o_t = f(q_t) S_t / (f(q_t) . z_t + eps). */
+static void causal_fwd_head(job_t *jb, long bh, double *scratch) {
+    const long T = jb->T, D = jb->D;
+    const double gamma = head_gamma(jb, bh);
+    const long off = bh * T * D;
+    const double *q = jb->q + off, *k = jb->k + off, *v = jb->v + off;
+    double *o = jb->o + off;
+    double *S = scratch, *z = S + D * D, *fq = z + D, *fk = fq + D;
+    memset(S, 0, (size_t)(D * D + D) * sizeof(double));
+    for (long t = 0; t < T; ++t) {
+        for (long i = 0; i < D; ++i) {
+            fq[i] = feat(jb, q[t * D + i]);
+            fk[i] = feat(jb, k[t * D + i]);
+        }
+        for (long i = 0; i < D; ++i) {
+            z[i] = gamma * z[i] + fk[i];
+            for (long j = 0; j < D; ++j) S[i * D + j] = gamma * S[i * D + j] + fk[i] * v[t * D + j];
+        }
+        double n = jb->eps;
+        for (long i = 0; i < D; ++i) n += fq[i] * z[i];
+        for (long j = 0; j < D; ++j) {
+            double u = 0.0;
+            for (long i = 0; i < D; ++i) u += fq[i] * S[i * D + j];
+            o[t * D + j] = u / n;
+        }
+    }
+}
+
+/* Backward, one head.  With u_t = f(q_t) S_t, n_t = f(q_t) . z_t + eps, o_t = u_t / n_t:
+ *   du_t = dout_t / n_t,   dn_t = -(dout_t . o_t) / n_t
+ *   df(q)_t[i] = sum_j S_t[i][j] du_t[j] + z_t[i] dn_t                     (forward sweep)
+ *   R_s = gamma R_{s+1} + f(q_s)^T du_s,   r_s = gamma r_{s+1} + f(q_s) dn_s  (reverse sweep)
+ *   df(k)_s[i] = sum_j R_s[i][j] v_s[j] + r_s[i],   dv_s[j] = sum_i f(k_s)[i] R_s[i][j]
+ *   dq = df(q) f'(q),  dk = df(k) f'(k). */
+static void causal_bwd_head(job_t *jb, long bh, double *scratch) {
+    const long T = jb->T, D = jb->D;
+    const double gamma = head_gamma(jb, bh);
+    const long off = bh * T * D;
+    const double *q = jb->q + off, *k = jb->k + off, *v = jb->v + off, *g = jb->g + off;
+    double *dq = jb->dq + off, *dk = jb->dk + off, *dv = jb->dv + off;
+    double *S = scratch, *z = S + D * D, *R = z + D, *r = R + D * D, *fq = r + D, *fk = fq + D;
+    double *nt = fk + D, *dnt = nt + T;            /* n_t and dn_t of every row */
+    memset(S, 0, (size_t)(2 * D * D + 2 * D) * sizeof(double));
+    for (long t = 0; t < T; ++t) {
+        for (long i = 0; i < D; ++i) {
+            fq[i] = feat(jb, q[t * D + i]);
+            fk[i] = feat(jb, k[t * D + i]);
+        }
+        for (long i = 0; i < D; ++i) {
+            z[i] = gamma * z[i] + fk[i];
+            for (long j = 0; j < D; ++j) S[i * D + j] = gamma * S[i * D + j] + fk[i] * v[t * D + j];
+        }
+        double n = jb->eps;
+        for (long i = 0; i < D; ++i) n += fq[i] * z[i];
+        double go = 0.0;                          /* dout_t . o_t */
+        for (long j = 0; j < D; ++j) {
+            double u = 0.0;
+            for (long i = 0; i < D; ++i) u += fq[i] * S[i * D + j];
+            go += g[t * D + j] * (u / n);
+        }
+        const double dn = -go / n;
+        nt[t] = n;
+        dnt[t] = dn;
+        for (long i = 0; i < D; ++i) {
+            double a = z[i] * dn;
+            for (long j = 0; j < D; ++j) a += S[i * D + j] * (g[t * D + j] / n);
+            dq[t * D + i] = a * dfeat(jb, q[t * D + i]);
+        }
+    }
+    for (long s = T - 1; s >= 0; --s) {
+        for (long i = 0; i < D; ++i) {
+            fq[i] = feat(jb, q[s * D + i]);
+            fk[i] = feat(jb, k[s * D + i]);
+        }
+        for (long i = 0; i < D; ++i) {
+            r[i] = gamma * r[i] + fq[i] * dnt[s];
+            for (long j = 0; j < D; ++j) R[i * D + j] = gamma * R[i * D + j] + fq[i] * (g[s * D + j] / nt[s]);
+        }
+        for (long i = 0; i < D; ++i) {
+            double a = r[i];
+            for (long j = 0; j < D; ++j) a += R[i * D + j] * v[s * D + j];
+            dk[s * D + i] = a * dfeat(jb, k[s * D + i]);
+        }
+        for (long j = 0; j < D; ++j) {
+            double a = 0.0;
+            for (long i = 0; i < D; ++i) a += fk[i] * R[i * D + j];
+            dv[s * D + j] = a;
+        }
+    }
+}
+
+/* gamma: [H] decays in (0, 1], or NULL for gamma = 1.  use_phi: 1 = elu + 1, 0 = identity. */
+int oracle_causal_norm_fwd(const double *q, const double *k, const double *v, const double *gamma, int use_phi,
+                           double eps, double *o, long B, long H, long T, long D, int nthreads) {
+    if (check_dims(B, H, T, D) || (T > 0 && (!q || !k || !v || !o))) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.gamma = gamma; jb.o = o; jb.use_phi = use_phi; jb.use_norm = 1; jb.eps = eps;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D;
+    return for_each_head(&jb, causal_fwd_head, (size_t)(D * D + 3 * D), nthreads);
+}
+
+int oracle_causal_norm_bwd(const double *q, const double *k, const double *v, const double *dout,
+                           const double *gamma, int use_phi, double eps, double *dq, double *dk, double *dv,
+                           long B, long H, long T, long D, int nthreads) {
+    if (check_dims(B, H, T, D) || (T > 0 && (!q || !k || !v || !dout || !dq || !dk || !dv))) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.g = dout; jb.gamma = gamma; jb.dq = dq; jb.dk = dk; jb.dv = dv;
+    jb.use_phi = use_phi; jb.use_norm = 1; jb.eps = eps;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D;
+    return for_each_head(&jb, causal_bwd_head, (size_t)(2 * D * D + 4 * D + 2 * T), nthreads);
+}
+

@@ -25,7 +25,7 @@ DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 class Workload:
     """One named synthetic workload (shapes, dtype and the input recipe)."""
     name: str
-    op: str                      # "bidir" | "simple" | "retention"
+    op: str                      # "bidir" | "simple" | "retention" | "causal_norm"
     B: int
     H: int
     T: int
@@ -62,6 +62,9 @@ WORKLOADS = {
     # retention, bf16, q scaled by D^-1/2 (T swept 128 .. 8192)
     "retention_bf16": Workload("retention_bf16", "retention", 8, 32, 2048, 128, "bf16",
                                q_scale=128 ** -0.5),
+    # causal linear attention with the norm term (phi = elu+1, no decay), the bidir recipe and shape
+    "causal_norm_f16": Workload("causal_norm_f16", "causal_norm", 8, 16, 4096, 64, "f16",
+                                q_scale=0.5, k_scale=0.5, v_scale=0.5),
     # vision-style long sequence, forward only, 256x256 token grid
     "vision_f16": Workload("vision_f16", "bidir", 2, 10, 65536, 64, "f16",
                            q_scale=0.5, k_scale=0.5, v_scale=0.5, vision_offset=True, bwd=False),

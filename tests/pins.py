@@ -398,6 +398,54 @@ def check_segment_backward(orc):
         _close(np.concatenate([a, b], axis=2), c, rtol=1e-12, atol=1e-12, what="segments vs whole %s" % n)
 
 
+def brute_causal_norm(q, k, v, gamma, eps, use_phi=True):
+    """Pairwise causal form: o_t = sum_{s<=t} a_ts v_s / (sum_{s<=t} a_ts + eps) with
+    a_ts = gamma^(t-s) f(q_t).f(k_s), f = phi or the identity (gamma None: 1)."""
+    f = _feature if use_phi else (lambda x: np.asarray(x, dtype=np.float64))
+    T = q.shape[2]
+    gm = np.ones(q.shape[1]) if gamma is None else np.asarray(gamma, dtype=np.float64)
+    dt = np.arange(T)[:, None] - np.arange(T)[None, :]
+    mask = np.where(dt[None] >= 0, gm[:, None, None] ** np.maximum(dt, 0)[None], 0.0)    # [H, T, T]
+    a = np.einsum("bhti,bhsi->bhts", f(q), f(k)) * mask[None]
+    return np.einsum("bhts,bhsj->bhtj", a, v) / (a.sum(-1, keepdims=True) + eps)
+
+
+def check_causal_norm(orc):
+    """Causal linear attention with the norm term: the pairwise form for both feature maps and
+    several decays; at gamma = 1 its last row is the bidirectional output's last row (the prefix
+    is the whole sequence there); v = 1 gives (n - eps) / n in every column; gradients of both
+    feature maps by finite differences."""
+    B, H, T, D = 2, 3, 9, 4
+    q, k, v = _rand((B, H, T, D), 81), _rand((B, H, T, D), 82), _rand((B, H, T, D), 83)
+    for gamma in (None, [0.5, 0.9, 1.0]):
+        for feature, up in (("elu1", True), ("identity", False)):
+            eps = 1e-3 if up else 50.0      # identity: keep the denominator away from 0
+            got = orc.causal_norm_fwd(q, k, v, gamma, feature, eps)
+            _close(got, brute_causal_norm(q, k, v, gamma, eps, up), rtol=1e-11, atol=1e-12,
+                   what="causal norm %s gamma=%s vs the pairwise form" % (feature, gamma))
+    last = orc.causal_norm_fwd(q, k, v, None, "elu1", 1e-3)[:, :, -1]
+    _close(last, orc.bidir_fwd(q, k, v, eps=1e-3)[:, :, -1], rtol=1e-12, atol=1e-13,
+           what="causal norm last row vs bidirectional")
+    ones = np.ones_like(v)
+    o1 = orc.causal_norm_fwd(q, k, ones, [0.5, 0.9, 1.0], "elu1", 0.25)
+    gm = np.array([0.5, 0.9, 1.0])
+    n = np.zeros((B, H, T))
+    for t in range(T):
+        w = gm[:, None] ** (t - np.arange(t + 1))[None, :]                                     # [H, t+1]
+        n[:, :, t] = np.einsum("bhi,bhsi,hs->bh", _feature(q[:, :, t]), _feature(k[:, :, :t + 1]), w) + 0.25
+    _close(o1, np.broadcast_to(((n - 0.25) / n)[..., None], o1.shape), rtol=1e-12, atol=1e-13, what="v = 1")
+    Bs, Hs, Ts, Ds = 1, 2, 5, 3
+    qs = _keep_off_zero(_rand((Bs, Hs, Ts, Ds), 84))
+    ks = _keep_off_zero(_rand((Bs, Hs, Ts, Ds), 85))
+    vs, gs = _rand((Bs, Hs, Ts, Ds), 86), _rand((Bs, Hs, Ts, Ds), 87)
+    for gamma, feature, eps in (([0.6, 0.95], "elu1", 0.05), (None, "identity", 20.0)):
+        fwd = lambda a, b, c: orc.causal_norm_fwd(a, b, c, gamma, feature, eps)
+        fd = _fd_grads(fwd, qs, ks, vs, gs)
+        got = orc.causal_norm_bwd(qs, ks, vs, gs, gamma, feature, eps)
+        for name, a, b in zip(("dq", "dk", "dv"), got, fd):
+            _close(a, b, rtol=1e-6, atol=1e-7, what="causal norm %s %s vs finite differences" % (feature, name))
+
+
 ALL_CHECKS = (check_golden, check_brute, check_closed_forms, check_invariances,
               check_fd_gradients, check_autograd, check_decode_step, check_state_segments,
-              check_segment_backward)
+              check_segment_backward, check_causal_norm)

@@ -27,6 +27,7 @@ def test_header_declares_the_api():
     names = declared_functions()
     for n in ("la_bidir_fwd", "la_bidir_bwd", "la_simple_fwd", "la_simple_bwd", "la_chunk_decay_fwd",
               "la_chunk_decay_bwd", "la_chunk_decay_step", "la_chunk_decay_fwd_state", "la_chunk_decay_bwd_state",
+              "la_chunk_decay_scan", "la_causal_norm_fwd", "la_causal_norm_bwd",
               "la_workspace_size", "la_status_string", "la_last_error"):
         assert n in names
 
@@ -132,6 +133,28 @@ def test_decay_scan_validation(lib):
     assert call(out=0x400004) == 3
     bad = (ctypes.c_float * 2)(0.5, 0.0)
     assert call(dec=bad) == 1
+
+
+def test_causal_norm_validation(lib):
+    P = ctypes.c_void_p
+    f = lib.la_causal_norm_fwd
+    f.restype = ctypes.c_int
+    b = lib.la_causal_norm_bwd
+    b.restype = ctypes.c_int
+
+    def fwd(feature=1, eps=1e-6, q=0x1000, dec=None, D=64):
+        return f(P(q), P(0x1000), P(0x1000), P(0x1000), dec, feature, ctypes.c_float(eps), 1, 2, 16, D, 1, P(0))
+    assert fwd(feature=5) == 2
+    assert fwd(eps=-1.0) == 1
+    assert fwd(q=0) == 1
+    assert fwd(q=0x1008) == 3
+    assert fwd(D=32) == 2
+    bad = (ctypes.c_float * 2)(0.5, 2.0)
+    assert fwd(dec=ctypes.cast(bad, P)) == 1
+    need = lib.la_workspace_size(11, 1, 2, 16, 64, 1)
+    assert need == 256            # 2 x 16 rows x 8 bytes, rounded up to 256
+    assert b(P(0x1000), P(0x1000), P(0x1000), P(0x1000), None, 1, ctypes.c_float(1e-6), P(0x1000), P(0x1000),
+             P(0x1000), 1, 2, 16, 64, 1, P(0), ctypes.c_size_t(0), P(0)) == 4
 
 
 def test_status_strings(lib):

@@ -44,6 +44,13 @@ MUTATIONS = [
     ("bwd_state_in_ignored", "    if (jb->state_in) memcpy(S,", "    if (0) memcpy(S,", 0),
     ("bwd_dstate_in_ignored", "    if (jb->dstate_in) memcpy(R,", "    if (0) memcpy(R,", 0),
     ("bwd_dstate_out_is_state", "memcpy(jb->dstate_out + bh * D * D, R,", "memcpy(jb->dstate_out + bh * D * D, S,", 0),
+    ("causal_drops_eps", "double n = jb->eps;\n        for (long i = 0; i < D; ++i) n += fq[i] * z[i];\n        for (long j",
+     "double n = 0.0;\n        for (long i = 0; i < D; ++i) n += fq[i] * z[i];\n        for (long j", 0),
+    ("causal_z_not_decayed", "z[i] = gamma * z[i] + fk[i];", "z[i] = z[i] + fk[i];", 0),
+    ("causal_bwd_dn_sign", "const double dn = -go / n;", "const double dn = go / n;", 0),
+    ("causal_bwd_drops_r", "double a = r[i];", "double a = 0.0;", 0),
+    ("causal_bwd_dk_uses_f", "dk[s * D + i] = a * dfeat(jb, k[s * D + i]);", "dk[s * D + i] = a * feat(jb, k[s * D + i]);", 0),
+    ("causal_bwd_dq_drops_z", "double a = z[i] * dn;", "double a = 0.0;", 0),
     ("fwd_state_out_before_last_token", "    if (jb->state_out) memcpy(jb->state_out + bh * D * D, S,",
      "    if (jb->state_out) memcpy(jb->state_out + bh * D * D, jb->state_in ? jb->state_in + bh * D * D : S,", 0),
 ]
