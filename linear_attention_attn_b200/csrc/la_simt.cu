@@ -469,20 +469,39 @@ __device__ __forceinline__ void feature_tiles(float (*tiles)[kRetTile][D], int n
 template <bool PHI>
 __device__ __forceinline__ float feature_grad_of(float fx) { return PHI ? (fx > 1.f ? 1.f : fx) : 1.f; }
 
-// Forward: threads 0..D-1 hold column j of S, thread D holds z.
+// Each state line (a column or a row of S, or z) is split over P threads: thread p of a
+// line takes the D / P entries p D / P .. (p + 1) D / P - 1 of it, and the line's P partial
+// dot products meet through xor shuffles among P adjacent lanes (fixed order).  Blocks are
+// whole warps; the threads past the last line compute on zeros and store nothing.
+template <int D> constexpr int causal_split() { return D == 64 ? 4 : 2; }
+template <int N> constexpr int round_warps(int n) { return (n + 31) / 32 * 32; }
+template <int D> constexpr int causal_fwd_threads() { return round_warps<0>(causal_split<D>() * (D + 1)); }
+template <int D> constexpr int causal_bwd_q_threads() { return round_warps<0>(causal_split<D>() * (2 * D + 1)); }
+template <int D> constexpr int causal_bwd_kv_threads() { return 2 * causal_split<D>() * D; }
+
+template <int P>
+__device__ __forceinline__ float line_sum(float s) {
+#pragma unroll
+    for (int m = 1; m < P; m <<= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+    return s;
+}
+
+// Forward: the D + 1 columns of [S | z] (z: the column of a value that is always 1).
 template <typename T, int D, bool PHI>
-__global__ void __launch_bounds__(D + 1)
+__global__ void __launch_bounds__(causal_fwd_threads<D>())
 causal_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, T *__restrict__ o,
            DecayArgs dec, int has_decay, int T_len, int H, float eps) {
+    constexpr int P = causal_split<D>(), DP = D / P;
     __shared__ float tiles[3][kRetTile][D];
     __shared__ float acc[kRetTile][D + 1];
     const int bh = blockIdx.x;
     const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
     const long long base = (long long)bh * T_len * D;
-    const int j = threadIdx.x;
-    float S[D];
+    const int j = threadIdx.x / P, i0 = (threadIdx.x % P) * DP;
+    const bool lead = threadIdx.x % P == 0 && j <= D;
+    float S[DP];
 #pragma unroll
-    for (int i = 0; i < D; ++i) S[i] = 0.f;
+    for (int i = 0; i < DP; ++i) S[i] = 0.f;
     const T *const src[3] = {q, k, v};
     for (int ts = 0; ts < T_len; ts += kRetTile) {
         __syncthreads();
@@ -493,30 +512,33 @@ causal_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict
         const int nr = min(kRetTile, T_len - ts);
         for (int r = 0; r < nr; ++r) {
             const float vj = j < D ? tiles[2][r][j] : 1.f;
-            float a = 0.f;
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < D; ++i) {
-                S[i] = fmaf(gamma, S[i], tiles[1][r][i] * vj);
-                a = fmaf(tiles[0][r][i], S[i], a);
+            for (int i = 0; i < DP; ++i) {
+                S[i] = fmaf(gamma, S[i], tiles[1][r][i0 + i] * vj);
+                a[i & 3] = fmaf(tiles[0][r][i0 + i], S[i], a[i & 3]);
             }
-            acc[r][j] = a;
+            const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
+            if (lead) acc[r][j] = s;
         }
         __syncthreads();
-        if (j < D)
-            for (int r = 0; r < nr; ++r)
-                io<T>::st(o + base + (long long)(ts + r) * D + j, acc[r][j] / (acc[r][D] + eps));
+        for (int e = threadIdx.x; e < nr * D; e += blockDim.x) {
+            const int r = e / D, c = e % D;
+            io<T>::st(o + base + (long long)(ts + r) * D + c, acc[r][c] / (acc[r][D] + eps));
+        }
     }
 }
 
 // Backward, forward sweep: dq, and per row (n_t, dn_t) for the reverse sweep, with
 // u_t = f(q_t) S_t, n_t = f(q_t) . z_t + eps, dn_t = -(dout_t . u_t) / n_t^2:
 //   df(q)_t[i] = (sum_j S_t[i][j] dout_t[j]) / n_t + z_t[i] dn_t,  dq = df(q) f'(q).
-// Threads 0..D hold the columns of [S | z] (u_t and n_t), threads D+1..2D the rows of S
-// and z[i] (the row sums of dq); a tile's rows meet in shared memory.
+// The first P (D + 1) threads hold the columns of [S | z] (u_t and n_t), the next P D the
+// rows of S and z[i] (the row sums of dq); a tile's rows meet in shared memory.
 template <typename T, int D, bool PHI>
-__global__ void __launch_bounds__(2 * D + 1)
+__global__ void __launch_bounds__(causal_bwd_q_threads<D>())
 causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
              T *__restrict__ dq, float2 *__restrict__ nd, DecayArgs dec, int has_decay, int T_len, int H, float eps) {
+    constexpr int P = causal_split<D>(), DP = D / P, NCOL = P * (D + 1);
     extern __shared__ float dsm[];               // causal_bwd_q_smem<D>() bytes
     float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // f(q), f(k), v, dout
     float(*U)[D + 1] = reinterpret_cast<float(*)[D + 1]>(dsm + 4 * kRetTile * D);  // dout_t[j] u_t[j], n_t - eps
@@ -526,13 +548,16 @@ causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
     const int bh = blockIdx.x;
     const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
     const long long base = (long long)bh * T_len * D;
-    const bool col_side = threadIdx.x <= D;
-    const int idx = col_side ? threadIdx.x : threadIdx.x - (D + 1);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;   // full warps
-    float Sx[D];
+    const bool col_side = threadIdx.x < NCOL;
+    const int t2 = col_side ? threadIdx.x : threadIdx.x - NCOL;
+    const int line = t2 / P, x0 = (t2 % P) * DP;       // column (col side) or row (row side); entry range
+    const bool row_live = !col_side && line < D;
+    const bool lead = t2 % P == 0 && (col_side || row_live);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    float Sx[DP];
     float zi = 0.f;
 #pragma unroll
-    for (int i = 0; i < D; ++i) Sx[i] = 0.f;
+    for (int i = 0; i < DP; ++i) Sx[i] = 0.f;
     const T *const src[4] = {q, k, v, g};
     for (int ts = 0; ts < T_len; ts += kRetTile) {
         __syncthreads();
@@ -542,32 +567,37 @@ causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
         __syncthreads();
         const int nr = min(kRetTile, T_len - ts);
         for (int r = 0; r < nr; ++r) {
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
             if (col_side) {
-                const float vj = idx < D ? tiles[2][r][idx] : 1.f;
-                float a = 0.f;
+                const float vj = line < D ? tiles[2][r][line] : 1.f;
 #pragma unroll
-                for (int i = 0; i < D; ++i) {
-                    Sx[i] = fmaf(gamma, Sx[i], tiles[1][r][i] * vj);
-                    a = fmaf(tiles[0][r][i], Sx[i], a);
+                for (int i = 0; i < DP; ++i) {
+                    Sx[i] = fmaf(gamma, Sx[i], tiles[1][r][x0 + i] * vj);
+                    a[i & 3] = fmaf(tiles[0][r][x0 + i], Sx[i], a[i & 3]);
                 }
-                U[r][idx] = idx < D ? a * tiles[3][r][idx] : a;
-            } else {
-                const float ki = tiles[1][r][idx];
-                float a = 0.f;
+            } else if (row_live) {
+                const float ki = tiles[1][r][line];
 #pragma unroll
-                for (int j = 0; j < D; ++j) {
-                    Sx[j] = fmaf(gamma, Sx[j], ki * tiles[2][r][j]);
-                    a = fmaf(Sx[j], tiles[3][r][j], a);
+                for (int jj = 0; jj < DP; ++jj) {
+                    Sx[jj] = fmaf(gamma, Sx[jj], ki * tiles[2][r][x0 + jj]);
+                    a[jj & 3] = fmaf(Sx[jj], tiles[3][r][x0 + jj], a[jj & 3]);
                 }
                 zi = fmaf(gamma, zi, ki);
-                A[r][idx] = a;
-                Z[r][idx] = zi;
+            }
+            const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
+            if (lead) {
+                if (col_side) {
+                    U[r][line] = line < D ? s * tiles[3][r][line] : s;
+                } else {
+                    A[r][line] = s;
+                    Z[r][line] = zi;
+                }
             }
         }
         __syncthreads();
-        for (int r = warp; warp < nwarps && r < nr; r += nwarps) {   // dout_t . u_t, a warp per row, fixed order
+        for (int r = warp; r < nr; r += nwarps) {   // dout_t . u_t, a warp per row, fixed order
             float p = 0.f;
-            for (int j = lane; j < D; j += 32) p += U[r][j];
+            for (int jj = lane; jj < D; jj += 32) p += U[r][jj];
 #pragma unroll
             for (int m = 16; m > 0; m >>= 1) p += __shfl_xor_sync(0xffffffffu, p, m);
             if (lane == 0) {
@@ -578,12 +608,12 @@ causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
             }
         }
         __syncthreads();
-        if (!col_side)
-            for (int r = 0; r < nr; ++r) {
-                const float2 in = info[r];
-                const float d = fmaf(A[r][idx], in.x, Z[r][idx] * in.y);
-                io<T>::st(dq + base + (long long)(ts + r) * D + idx, d * feature_grad_of<PHI>(tiles[0][r][idx]));
-            }
+        for (int e = threadIdx.x; e < nr * D; e += blockDim.x) {
+            const int r = e / D, c = e % D;
+            const float2 in = info[r];
+            const float d = fmaf(A[r][c], in.x, Z[r][c] * in.y);
+            io<T>::st(dq + base + (long long)(ts + r) * D + c, d * feature_grad_of<PHI>(tiles[0][r][c]));
+        }
     }
 }
 
@@ -595,25 +625,30 @@ static_assert((6 * kRetTile * 64 + kRetTile * 65) % 2 == 0 && (6 * kRetTile * 12
               "the float2 block of causal_bwd_q starts 8-byte aligned");
 
 // Backward, reverse sweep over R_s = gamma R_{s+1} + f(q_s)^T du_s and r_s = gamma r_{s+1} +
-// f(q_s) dn_s with du_s = dout_s / n_s: threads 0..D-1 hold row i of R and r[i]
-// (dk_s[i] = (sum_j R[i][j] v_s[j] + r[i]) f'(k_s[i])), threads D..2D-1 column j of R
+// f(q_s) dn_s with du_s = dout_s / n_s: the first P D threads hold the rows of R and r[i]
+// (dk_s[i] = (sum_j R[i][j] v_s[j] + r[i]) f'(k_s[i])), the next P D the columns of R
 // (dv_s[j] = sum_i f(k_s)[i] R[i][j]).
 template <typename T, int D, bool PHI>
-__global__ void __launch_bounds__(2 * D)
+__global__ void __launch_bounds__(causal_bwd_kv_threads<D>())
 causal_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
               const float2 *__restrict__ nd, T *__restrict__ dk, T *__restrict__ dv, DecayArgs dec, int has_decay,
               int T_len, int H) {
-    __shared__ float tiles[4][kRetTile][D];
-    __shared__ float2 info[kRetTile];
+    constexpr int P = causal_split<D>(), DP = D / P;
+    extern __shared__ float dsm[];               // causal_bwd_kv_smem<D>() bytes
+    float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // f(q), f(k), v, dout
+    float(*res)[kRetTile][D] = tiles + 4;        // dk before f' (rows), dv (columns)
+    float2 *info = reinterpret_cast<float2 *>(dsm + 6 * kRetTile * D);
     const int bh = blockIdx.x;
     const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
     const long long base = (long long)bh * T_len * D;
-    const bool row_side = threadIdx.x < D;
-    const int idx = row_side ? threadIdx.x : threadIdx.x - D;
-    float Rx[D];
+    const bool row_side = threadIdx.x < P * D;
+    const int t2 = row_side ? threadIdx.x : threadIdx.x - P * D;
+    const int line = t2 / P, x0 = (t2 % P) * DP;
+    const bool lead = t2 % P == 0;
+    float Rx[DP];
     float ri = 0.f;
 #pragma unroll
-    for (int m = 0; m < D; ++m) Rx[m] = 0.f;
+    for (int m = 0; m < DP; ++m) Rx[m] = 0.f;
     const T *const src[4] = {q, k, v, g};
     const int ntiles = (T_len + kRetTile - 1) / kRetTile;
     for (int tile = ntiles - 1; tile >= 0; --tile) {
@@ -630,28 +665,39 @@ causal_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
         __syncthreads();
         for (int r = nr - 1; r >= 0; --r) {
             const float2 in = info[r];
-            float acc = 0.f;
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
             if (row_side) {
-                const float qi = tiles[0][r][idx];
+                const float qi = tiles[0][r][line];
 #pragma unroll
-                for (int j = 0; j < D; ++j) {
-                    Rx[j] = fmaf(gamma, Rx[j], qi * (tiles[3][r][j] * in.x));
-                    acc = fmaf(Rx[j], tiles[2][r][j], acc);
+                for (int jj = 0; jj < DP; ++jj) {
+                    Rx[jj] = fmaf(gamma, Rx[jj], qi * (tiles[3][r][x0 + jj] * in.x));
+                    a[jj & 3] = fmaf(Rx[jj], tiles[2][r][x0 + jj], a[jj & 3]);
                 }
                 ri = fmaf(gamma, ri, qi * in.y);
-                const float fk = tiles[1][r][idx];
-                io<T>::st(dk + base + (long long)(ts + r) * D + idx, (acc + ri) * feature_grad_of<PHI>(fk));
             } else {
-                const float duj = tiles[3][r][idx] * in.x;
+                const float duj = tiles[3][r][line] * in.x;
 #pragma unroll
-                for (int i = 0; i < D; ++i) {
-                    Rx[i] = fmaf(gamma, Rx[i], tiles[0][r][i] * duj);
-                    acc = fmaf(tiles[1][r][i], Rx[i], acc);
+                for (int i = 0; i < DP; ++i) {
+                    Rx[i] = fmaf(gamma, Rx[i], tiles[0][r][x0 + i] * duj);
+                    a[i & 3] = fmaf(tiles[1][r][x0 + i], Rx[i], a[i & 3]);
                 }
-                io<T>::st(dv + base + (long long)(ts + r) * D + idx, acc);
             }
+            const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
+            if (lead) res[row_side ? 0 : 1][r][line] = row_side ? s + ri : s;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < nr * D; e += blockDim.x) {   // the tile's rows, coalesced
+            const int r = e / D, c = e % D;
+            const long long at = base + (long long)(ts + r) * D + c;
+            io<T>::st(dk + at, res[0][r][c] * feature_grad_of<PHI>(tiles[1][r][c]));
+            io<T>::st(dv + at, res[1][r][c]);
         }
     }
+}
+
+template <int D>
+constexpr size_t causal_bwd_kv_smem() {
+    return (size_t)(6 * kRetTile * D) * sizeof(float) + kRetTile * sizeof(float2);
 }
 
 // -------------------------------------------------------------- drivers ---
@@ -893,7 +939,7 @@ namespace {
 template <typename T, int D, bool PHI>
 la_status causal_fwd_t(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, int has_decay,
                        const Shape &s, float eps, cudaStream_t st) {
-    return launch("simt_causal_norm_fwd", causal_fwd<T, D, PHI>, dim3((unsigned)s.BH()), dim3(D + 1), 0, st,
+    return launch("simt_causal_norm_fwd", causal_fwd<T, D, PHI>, dim3((unsigned)s.BH()), dim3(causal_fwd_threads<D>()), 0, st,
                   (const T *)q, (const T *)k, (const T *)v, (T *)o, dec, has_decay, s.T, s.H, eps);
 }
 
@@ -902,10 +948,11 @@ la_status causal_bwd_t(const void *q, const void *k, const void *v, const void *
                        const DecayArgs &dec, int has_decay, const Shape &s, float eps, void *ws, cudaStream_t st) {
     float2 *nd = (float2 *)ws;
     la_status rc = launch("simt_causal_norm_bwd_q", causal_bwd_q<T, D, PHI>, dim3((unsigned)s.BH()),
-                          dim3(2 * D + 1), causal_bwd_q_smem<D>(), st, (const T *)q, (const T *)k, (const T *)v,
+                          dim3(causal_bwd_q_threads<D>()), causal_bwd_q_smem<D>(), st, (const T *)q, (const T *)k, (const T *)v,
                           (const T *)g, (T *)dq, nd, dec, has_decay, s.T, s.H, eps);
     if (rc) return rc;
-    return launch("simt_causal_norm_bwd_kv", causal_bwd_kv<T, D, PHI>, dim3((unsigned)s.BH()), dim3(2 * D), 0, st,
+    return launch("simt_causal_norm_bwd_kv", causal_bwd_kv<T, D, PHI>, dim3((unsigned)s.BH()),
+                  dim3(causal_bwd_kv_threads<D>()), causal_bwd_kv_smem<D>(), st,
                   (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const float2 *)nd, (T *)dk, (T *)dv, dec,
                   has_decay, s.T, s.H);
 }
