@@ -79,9 +79,14 @@ typedef enum {
     LA_OP_CAUSAL_NORM_BWD = 11
 } la_op;
 
-/* Feature map of the sequence-parallel stages: elu+1 with the norm term (the
- * la_bidir_* op) or the identity without it (the la_simple_* op). */
-typedef enum { LA_FEATURE_IDENTITY = 0, LA_FEATURE_ELU1 = 1 } la_feature;
+/* Feature map of the state-form stages and of la_causal_norm_*: elu+1 with the
+ * norm term (the la_bidir_* op), the identity without it (the la_simple_* op), or
+ * the identity with the norm term (LA_FEATURE_NORM: features f(q), f(k) computed
+ * by the caller, e.g. the focusing function or the polarity split of
+ * la_feature_map_fwd, then attended with the norm term; dq, dk are then the
+ * gradients with respect to those features).  la_causal_norm_* take
+ * LA_FEATURE_ELU1 or LA_FEATURE_IDENTITY (the norm term is always on there). */
+typedef enum { LA_FEATURE_IDENTITY = 0, LA_FEATURE_ELU1 = 1, LA_FEATURE_NORM = 2 } la_feature;
 
 /* Largest H accepted by la_chunk_decay_* (the decays travel as kernel arguments). */
 #define LA_MAX_DECAY_HEADS 512
@@ -259,6 +264,30 @@ la_status la_causal_norm_bwd(const void *q, const void *k, const void *v, const 
                              int B, int H, int T, int D, la_dtype dtype,
                              void *workspace, size_t workspace_bytes, void *stream);
 
+/* ---- feature maps formed by the caller ------------------------------------
+ * Row-wise maps of [B,H,T,D] tensors, D in {32, 64, 128}, for the state-form
+ * stages with LA_FEATURE_NORM (the bidirectional op with the norm term on the
+ * features), as used by two of the models the "Flash Bi-directional Linear
+ * Attention" README lists (Focused-LA, PolaFormer); the maps are those models'
+ * feature maps, written from their definitions (|.| the 2-norm of a row, powers
+ * elementwise):
+ *  LA_FMAP_FOCUSED        y = relu(x), f = (|y| / |y^p|) y^p (0 for a row without a
+ *                         positive entry): the focusing function; width D.
+ *  LA_FMAP_POLARITY       f = [relu(x)^p, relu(-x)^p]; width 2 D (the query side and
+ *                         the same-sign key side of the polarity split).
+ *  LA_FMAP_POLARITY_SWAP  f = [relu(-x)^p, relu(x)^p]; width 2 D (the opposite-sign
+ *                         key side).
+ * p >= 1 (finite).  fp32 arithmetic, one warp per row; HBM bound. */
+typedef enum { LA_FMAP_FOCUSED = 0, LA_FMAP_POLARITY = 1, LA_FMAP_POLARITY_SWAP = 2 } la_fmap;
+
+/* y <- f(x): x [B,H,T,D], y [B,H,T,W] (W = D or 2 D as above), both dtype. */
+la_status la_feature_map_fwd(la_fmap kind, float p, const void *x, void *y, int B, int H, int T, int D,
+                             la_dtype dtype, void *stream);
+
+/* dx <- J(x)^T dy, the gradient through f: x, dx [B,H,T,D], dy [B,H,T,W]. */
+la_status la_feature_map_bwd(la_fmap kind, float p, const void *x, const void *dy, void *dx, int B, int H, int T,
+                             int D, la_dtype dtype, void *stream);
+
 /* ---- the state form in stages, for a sequence split along T -------------
  * A sequence cut into shards along T (one per rank or per call) gives each
  * shard's partial state; their sum over the shards is the state of the whole
@@ -267,12 +296,17 @@ la_status la_causal_norm_bwd(const void *q, const void *k, const void *v, const 
  * on every shard.  The backward likewise: la_state_bwd_q on every shard with
  * the whole sequence's state, a sum of the shards' [dS | dz], la_state_bwd_kv
  * on every shard.  With one shard the stages compute exactly la_bidir_* /
- * la_simple_* (feature = LA_FEATURE_ELU1 / LA_FEATURE_IDENTITY).  The library's
+ * la_simple_* (feature = LA_FEATURE_ELU1 / LA_FEATURE_IDENTITY); with
+ * LA_FEATURE_NORM they are la_bidir_* with f the identity, on features the
+ * caller formed (one shard covering the whole sequence is the single-GPU use:
+ * reduce then apply, bwd_q then bwd_kv).  The library's
  * addition: the pages only motivate long sequences ("Flash Bi-directional
  * Linear Attention" README: intro), the split is the state form's own.
  * Shapes, dtypes and alignment as for la_bidir_fwd; T is the shard's length
  * (0 allowed: a reduce then writes zeros).  States are [B,H,D,D+1] fp32 device
  * arrays as in la_bidir_fwd (column D holds z, 0 for LA_FEATURE_IDENTITY).
+ * f(x) below is elu(x)+1 for LA_FEATURE_ELU1 and x otherwise; the norm term
+ * (z, n_t, eps) is present for LA_FEATURE_ELU1 and LA_FEATURE_NORM.
  * Workspace: la_workspace_size(LA_OP_STATE_REDUCE / LA_OP_STATE_BWD_Q, ...);
  * the apply and bwd_kv stages take none. */
 
@@ -281,8 +315,8 @@ la_status la_state_reduce(const void *k, const void *v, float *state, int B, int
                           la_dtype dtype, la_feature feature, void *workspace, size_t workspace_bytes,
                           void *stream);
 
-/* o <- f(q_t) S / (f(q_t) . z + eps) (elu+1), or q_t S (identity), with the
- * whole sequence's state. */
+/* o <- f(q_t) S / (f(q_t) . z + eps) (elu+1 or norm), or q_t S (identity), with
+ * the whole sequence's state. */
 la_status la_state_apply(const void *q, const float *state, void *o, int B, int H, int T, int D,
                          la_dtype dtype, la_feature feature, float eps, void *stream);
 

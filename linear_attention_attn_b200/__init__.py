@@ -29,7 +29,7 @@ LA_F32, LA_F16, LA_BF16 = 0, 1, 2
 OPS = {"bidir_fwd": 0, "bidir_bwd": 1, "simple_fwd": 2, "simple_bwd": 3,
        "chunk_decay_fwd": 4, "chunk_decay_bwd": 5, "state_reduce": 6, "state_apply": 7,
        "state_bwd_q": 8, "state_bwd_kv": 9, "causal_norm_fwd": 10, "causal_norm_bwd": 11}
-FEATURES = {"identity": 0, "elu1": 1}
+FEATURES = {"identity": 0, "elu1": 1, "norm": 2}
 STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_ALIGNMENT",
           4: "LA_ERR_WORKSPACE", 5: "LA_ERR_CUDA", 6: "LA_ERR_TIMEOUT"}
 MAX_DECAY_HEADS = 512
@@ -57,6 +57,8 @@ _lib.la_chunk_decay_fwd_state.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I
 _lib.la_chunk_decay_bwd_state.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z,
                                           _P]
 _lib.la_chunk_decay_scan.argtypes = [_P, _P, _I, _P, _P, _I, _I, _I, _P]
+_lib.la_feature_map_fwd.argtypes = [_I, _F, _P, _P, _I, _I, _I, _I, _I, _P]
+_lib.la_feature_map_bwd.argtypes = [_I, _F, _P, _P, _P, _I, _I, _I, _I, _I, _P]
 _lib.la_causal_norm_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _F, _I, _I, _I, _I, _I, _P]
 _lib.la_causal_norm_bwd.argtypes = [_P, _P, _P, _P, _P, _I, _F, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_state_reduce.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P]
@@ -66,7 +68,7 @@ _lib.la_state_bwd_kv.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]
 for _n in ("la_bidir_fwd", "la_simple_fwd", "la_bidir_bwd", "la_simple_bwd", "la_chunk_decay_fwd",
            "la_chunk_decay_bwd", "la_chunk_decay_step", "la_chunk_decay_fwd_state", "la_chunk_decay_bwd_state",
            "la_chunk_decay_scan", "la_state_reduce", "la_state_apply", "la_state_bwd_q", "la_state_bwd_kv",
-           "la_causal_norm_fwd", "la_causal_norm_bwd"):
+           "la_causal_norm_fwd", "la_causal_norm_bwd", "la_feature_map_fwd", "la_feature_map_bwd"):
     getattr(_lib, _n).restype = _I
 _lib.la_bidir_fwd_static.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.la_bidir_fwd_static.restype = _I
@@ -307,6 +309,42 @@ def la_chunk_decay_scan(states, gaps, decay, out, stream=None):
 
 def _decay_or_null(decay, H):
     return (None, None) if decay is None else (lambda a: (ctypes.cast(a, _P), a))(_decay(decay, H))
+
+
+FMAPS = {"focused": 0, "polarity": 1, "polarity_swap": 2}
+
+
+def _fmap_args(kind, x, out, out_width):
+    if kind not in FMAPS:
+        raise ValueError("kind must be one of %s" % sorted(FMAPS))
+    if x.dim() != 4 or out.dim() != 4:
+        raise ValueError("expected [B, H, T, D] tensors")
+    B, H, T, D = (int(n) for n in x.shape)
+    if tuple(out.shape) != (B, H, T, out_width(D)) or out.dtype != x.dtype or out.device != x.device:
+        raise ValueError("output must be [B, H, T, %s] of the input's dtype and device" % ("D" if kind == "focused" else "2D"))
+    for t in (x, out):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    return B, H, T, D
+
+
+def la_feature_map_fwd(kind, x, y, p: float = 1.0, stream=None):
+    """y <- f(x) row by row: kind 'focused' (y = relu(x), (|y| / |y^p|) y^p; y [B,H,T,D]), 'polarity'
+    ([relu(x)^p, relu(-x)^p]; y [B,H,T,2D]) or 'polarity_swap' (the halves swapped)."""
+    width = (lambda D: D) if kind == "focused" else (lambda D: 2 * D)
+    B, H, T, D = _fmap_args(kind, x, y, width)
+    _check(_lib.la_feature_map_fwd(FMAPS[kind], ctypes.c_float(p), _ptr(x), _ptr(y), B, H, T, D, _dtype_code(x),
+                                   _stream(stream, x.device)), "la_feature_map_fwd")
+
+
+def la_feature_map_bwd(kind, x, dy, dx, p: float = 1.0, stream=None):
+    """dx <- J(x)^T dy, the gradient through la_feature_map_fwd."""
+    width = (lambda D: D) if kind == "focused" else (lambda D: 2 * D)
+    B, H, T, D = _fmap_args(kind, x, dy, width)
+    if tuple(dx.shape) != tuple(x.shape) or dx.dtype != x.dtype or not dx.is_cuda or not dx.is_contiguous():
+        raise ValueError("dx must be a contiguous CUDA tensor like x")
+    _check(_lib.la_feature_map_bwd(FMAPS[kind], ctypes.c_float(p), _ptr(x), _ptr(dy), _ptr(dx), B, H, T, D,
+                                   _dtype_code(x), _stream(stream, x.device)), "la_feature_map_bwd")
 
 
 def la_causal_norm_fwd(q, k, v, o, decay=None, feature="elu1", eps: float = 1e-6, stream=None):

@@ -239,7 +239,8 @@ static la_status stage_entry(Stage stage, la_op op, la_feature f, const void *x,
                              void *ws, size_t ws_bytes, void *stream) {
     const Shape s{B, H, T, D};
     LA_TRY(validate(s, dt));
-    if (f != LA_FEATURE_IDENTITY && f != LA_FEATURE_ELU1) return fail(LA_ERR_UNSUPPORTED, "unknown feature map %d", (int)f);
+    if (f != LA_FEATURE_IDENTITY && f != LA_FEATURE_ELU1 && f != LA_FEATURE_NORM)
+        return fail(LA_ERR_UNSUPPORTED, "unknown feature map %d", (int)f);
     if (!(eps >= 0.f) || !isfinite(eps)) return fail(LA_ERR_INVALID_ARG, "eps must be finite and >= 0");
     const char *xn = stage == Stage::Reduce || stage == Stage::BwdKV ? "k" : "q";
     LA_TRY(check_ptr(x, xn));
@@ -258,9 +259,8 @@ static la_status stage_entry(Stage stage, la_op op, la_feature f, const void *x,
         }
         return LA_OK;
     }
-    const bool bidir = f == LA_FEATURE_ELU1;
-    if (path_tc(op, s, dt)) return tc::state_stage(stage, bidir, x, y, sin, sout, out1, out2, s, dt, eps, ws, st);
-    return simt::state_stage(stage, bidir, x, y, sin, sout, out1, out2, s, dt, eps, ws, st);
+    if (path_tc(op, s, dt)) return tc::state_stage(stage, f, x, y, sin, sout, out1, out2, s, dt, eps, ws, st);
+    return simt::state_stage(stage, f, x, y, sin, sout, out1, out2, s, dt, eps, ws, st);
 }
 
 }  // namespace la
@@ -400,7 +400,9 @@ la_status la_chunk_decay_bwd_state(const void *q, const void *k, const void *v, 
 static la_status causal_entry(const Shape &s, la_dtype dt, const float *decay, la_feature f, float eps,
                               DecayArgs *dec, int *has_decay) {
     LA_TRY(validate(s, dt));
-    if (f != LA_FEATURE_IDENTITY && f != LA_FEATURE_ELU1) return fail(LA_ERR_UNSUPPORTED, "unknown feature map %d", (int)f);
+    // the norm term is always on here: LA_FEATURE_NORM is the identity feature map as well
+    if (f != LA_FEATURE_IDENTITY && f != LA_FEATURE_ELU1 && f != LA_FEATURE_NORM)
+        return fail(LA_ERR_UNSUPPORTED, "unknown feature map %d", (int)f);
     if (!(eps >= 0.f) || !isfinite(eps)) return fail(LA_ERR_INVALID_ARG, "eps must be finite and >= 0");
     *has_decay = decay != nullptr;
     if (decay) LA_TRY(decay_args(decay, s.H, dec));
@@ -440,6 +442,34 @@ la_status la_causal_norm_bwd(const void *q, const void *k, const void *v, const 
     if (T == 0) return LA_OK;
     return simt::causal_norm_bwd(q, k, v, dout, dq, dk, dv, dec, has_decay, feature == LA_FEATURE_ELU1, s, dtype, eps,
                                  workspace, (cudaStream_t)stream);
+}
+
+static la_status fmap_entry(bool bwd, la_fmap kind, float p, const void *x, const void *dy, void *out, int B,
+                            int H, int T, int D, la_dtype dt, void *stream) {
+    t_allow_null = (T == 0);
+    if (B < 1 || H < 1 || T < 0) return fail(LA_ERR_INVALID_ARG, "B, H must be >= 1 and T >= 0");
+    if (dt != LA_F32 && dt != LA_F16 && dt != LA_BF16) return fail(LA_ERR_UNSUPPORTED, "unknown dtype %d", (int)dt);
+    if (D != 32 && D != 64 && D != 128) return fail(LA_ERR_UNSUPPORTED, "D must be 32, 64 or 128 (got %d)", D);
+    if (kind != LA_FMAP_FOCUSED && kind != LA_FMAP_POLARITY && kind != LA_FMAP_POLARITY_SWAP)
+        return fail(LA_ERR_UNSUPPORTED, "unknown feature map kind %d", (int)kind);
+    if (!(p >= 1.f) || !isfinite(p)) return fail(LA_ERR_INVALID_ARG, "p must be finite and >= 1");
+    const long long rows = (long long)B * H * T;
+    if ((double)rows * D * 2 >= 2147483648.0) return fail(LA_ERR_UNSUPPORTED, "tensor too large");
+    LA_TRY(check_ptr(x, "x"));
+    if (bwd) LA_TRY(check_ptr(dy, "dy"));
+    LA_TRY(check_ptr(out, bwd ? "dx" : "y"));
+    if (rows == 0) return LA_OK;
+    return feature_map(bwd, (int)kind, p, x, dy, out, rows, D, dt, (cudaStream_t)stream);
+}
+
+la_status la_feature_map_fwd(la_fmap kind, float p, const void *x, void *y, int B, int H, int T, int D, la_dtype dtype,
+                             void *stream) {
+    return fmap_entry(false, kind, p, x, nullptr, y, B, H, T, D, dtype, stream);
+}
+
+la_status la_feature_map_bwd(la_fmap kind, float p, const void *x, const void *dy, void *dx, int B, int H, int T,
+                             int D, la_dtype dtype, void *stream) {
+    return fmap_entry(true, kind, p, x, dy, dx, B, H, T, D, dtype, stream);
 }
 
 la_status la_chunk_decay_scan(const float *states, const long long *gaps, int n, const float *decay, float *out,

@@ -124,6 +124,11 @@ size_t state_bytes(const Shape &s, long long copies);
 la_status decay_scan(const float *states, const long long *gaps, int n, const DecayArgs &dec, float *out, int B,
                      int H, int D, cudaStream_t st);
 
+// Row-wise feature map (kind 0 focusing, 1 polarity split, 2 swapped split) of `rows`
+// rows of D in {32, 64, 128}, or its backward (dx = J^T dy) when bwd.
+la_status feature_map(bool bwd, int kind, float p, const void *x, const void *dy, void *out, long long rows, int D,
+                      la_dtype dt, cudaStream_t st);
+
 // One recurrent (decode) step of the decay op: S <- gamma S + k^T v, o = q S,
 // with q, k, v, o [B,H,D] and the fp32 state [B,H,D,D] updated in place.
 la_status decay_step(const void *q, const void *k, const void *v, void *o, float *state, const DecayArgs &dec, int B,
@@ -145,7 +150,7 @@ la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const 
 la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin,
                     const float *rin, float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv,
                     const Shape &s, la_dtype dt, cudaStream_t st);
-la_status state_stage(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout,
+la_status state_stage(Stage stage, la_feature f, const void *x, const void *y, const float *sin, float *sout,
                       void *out1, void *out2, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
 // Causal linear attention with the norm term (has_decay = 0: gamma = 1; phi: elu + 1,
 // else the identity).  The backward's workspace holds (n_t, dn_t) of every row.

@@ -29,7 +29,7 @@ constexpr int kThreads = 256;
 
 // Partial S (and z for bidir) over rows [split*rps, min(T, (split+1)*rps)) of
 // head blockIdx.y.  Thread (ti, tj) owns the R x R block S[ti*R.., tj*R..].
-template <typename T, int D, bool BIDIR>
+template <typename T, int D, bool BIDIR, bool PHI = BIDIR>
 __global__ void __launch_bounds__(kThreads)
 state_partial(const T *__restrict__ k, const T *__restrict__ v, float *__restrict__ part,
               int T_len, int nsplit, int rps) {
@@ -55,7 +55,7 @@ state_partial(const T *__restrict__ k, const T *__restrict__ v, float *__restric
             float kk = 0.f, vv = 0.f;
             if (t < t1) {
                 kk = io<T>::ld(k + base + (long long)t * D + c);
-                if (BIDIR) kk = feature(kk);
+                if (PHI) kk = feature(kk);
                 vv = io<T>::ld(v + base + (long long)t * D + c);
             }
             ks[r][c] = kk;
@@ -103,7 +103,7 @@ combine(const float *__restrict__ part, float *__restrict__ out, int nsplit, int
 
 // o_t = f(q_t) S / (f(q_t).z + eps)  (bidir)  or  q_t S  (simple).
 // 32 rows per CTA, 8 threads per row, thread cg owns columns cg + 8c.
-template <typename T, int D, bool BIDIR>
+template <typename T, int D, bool BIDIR, bool PHI = BIDIR>
 __global__ void __launch_bounds__(kThreads)
 output(const T *__restrict__ q, const float *__restrict__ state, T *__restrict__ o, int T_len, float eps) {
     constexpr int TPR = kThreads / kTile;
@@ -122,7 +122,7 @@ output(const T *__restrict__ q, const float *__restrict__ state, T *__restrict__
     for (int e = threadIdx.x; e < kTile * D; e += kThreads) {
         const int r = e / D, c = e % D, t = row0 + r;
         float x = t < T_len ? io<T>::ld(q + base + (long long)t * D + c) : 0.f;
-        qs[r * LD + c] = (BIDIR && t < T_len) ? feature(x) : x;
+        qs[r * LD + c] = (PHI && t < T_len) ? feature(x) : x;
     }
     __syncthreads();
     const int r = threadIdx.x / TPR, cg = threadIdx.x % TPR, t = row0 + r;
@@ -147,7 +147,7 @@ output(const T *__restrict__ q, const float *__restrict__ state, T *__restrict__
 
 // Query side of the backward pass over rows [split*rps, ...) of one head:
 // writes dq and the split's partial (dS | dz) into part.
-template <typename T, int D, bool BIDIR>
+template <typename T, int D, bool BIDIR, bool PHI = BIDIR>
 __global__ void __launch_bounds__(kThreads)
 bwd_q(const T *__restrict__ q, const T *__restrict__ g, const float *__restrict__ state,
       T *__restrict__ dq, float *__restrict__ part, int T_len, int nsplit, int rps, float eps) {
@@ -189,7 +189,7 @@ bwd_q(const T *__restrict__ q, const T *__restrict__ g, const float *__restrict_
                 gg = io<T>::ld(g + base + (long long)t * D + c);
             }
             qraw[rr * LD + c] = x;
-            qf[rr * LD + c] = (BIDIR && t < t1) ? feature(x) : x;
+            qf[rr * LD + c] = (PHI && t < t1) ? feature(x) : x;
             gs[rr * LD + c] = gg;
         }
         __syncthreads();
@@ -218,7 +218,7 @@ bwd_q(const T *__restrict__ q, const T *__restrict__ g, const float *__restrict_
             const int i = cg + TPR * c;
             float a = 0.f;
             for (int j = 0; j < D; ++j) a = fmaf(gs[r * LD + j], S[i * LD + j], a);
-            if (BIDIR) a = (a - gdot * z[i]) / n * feature_grad(qraw[r * LD + i]);
+            if (BIDIR) a = (a - gdot * z[i]) / n * (PHI ? feature_grad(qraw[r * LD + i]) : 1.f);
             if (t < t1) io<T>::st(dq + base + (long long)t * D + i, a);
         }
         __syncthreads();
@@ -256,7 +256,7 @@ bwd_q(const T *__restrict__ q, const T *__restrict__ g, const float *__restrict_
 }
 
 // Key/value side: dk = (v dS^T + dz) f'(k),  dv = f(k) dS.
-template <typename T, int D, bool BIDIR>
+template <typename T, int D, bool BIDIR, bool PHI = BIDIR>
 __global__ void __launch_bounds__(kThreads)
 bwd_k(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ dstate,
       T *__restrict__ dk, T *__restrict__ dv, int T_len) {
@@ -283,7 +283,7 @@ bwd_k(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict_
             y = io<T>::ld(v + base + (long long)t * D + c);
         }
         kraw[r * LD + c] = x;
-        kf[r * LD + c] = BIDIR ? feature(x) : x;
+        kf[r * LD + c] = PHI ? feature(x) : x;
         vs[r * LD + c] = y;
     }
     __syncthreads();
@@ -294,7 +294,7 @@ bwd_k(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict_
         const int i = cg + TPR * c;
         float a = dz[i];
         for (int j = 0; j < D; ++j) a = fmaf(dS[i * LD + j], vs[r * LD + j], a);
-        if (BIDIR) a *= feature_grad(kraw[r * LD + i]);
+        if (PHI) a *= feature_grad(kraw[r * LD + i]);
         io<T>::st(dk + base + (long long)t * D + i, a);
     }
     float acc[CPT];
@@ -771,9 +771,9 @@ la_status state_bwd_t(bool bidir, const T *q, const T *k, const T *v, const T *g
 
 // One stage of the state form (see Stage): the same kernels as state_fwd_t /
 // state_bwd_t, with the state passed in or handed out instead of kept inside.
-template <typename T, int D>
-la_status stage_t(Stage stage, bool bidir, const T *x, const T *y, const float *sin, float *sout, T *out1, T *out2,
-                  const Shape &s, float eps, void *ws, cudaStream_t st) {
+template <typename T, int D, bool BIDIR, bool PHI>
+la_status stage_tt(Stage stage, const T *x, const T *y, const float *sin, float *sout, T *out1, T *out2,
+                   const Shape &s, float eps, void *ws, cudaStream_t st) {
     const int nsplit = simt_splits(s);
     const int rps = (s.T + nsplit - 1) / nsplit;
     float *part = (float *)ws;
@@ -782,43 +782,44 @@ la_status stage_t(Stage stage, bool bidir, const T *x, const T *y, const float *
     la_status rc;
     switch (stage) {
     case Stage::Reduce:
-        rc = bidir ? launch("simt_state_partial", state_partial<T, D, true>, g1, dim3(kThreads), 0, st, x, y, part,
-                            s.T, nsplit, rps)
-                   : launch("simt_state_partial", state_partial<T, D, false>, g1, dim3(kThreads), 0, st, x, y, part,
-                            s.T, nsplit, rps);
+        rc = launch("simt_state_partial", state_partial<T, D, BIDIR, PHI>, g1, dim3(kThreads), 0, st, x, y, part,
+                    s.T, nsplit, rps);
         if (rc) return rc;
         return launch("simt_combine", combine, dim3((unsigned)s.BH()), dim3(kThreads), 0, st, (const float *)part, sout,
                       nsplit, D * (D + 1));
     case Stage::Apply: {
         const size_t smem = (size_t)(D * D + D + kTile * (D + 1)) * sizeof(float);
-        return bidir ? launch("simt_output", output<T, D, true>, g2, dim3(kThreads), smem, st, x, sin, out1, s.T, eps)
-                     : launch("simt_output", output<T, D, false>, g2, dim3(kThreads), smem, st, x, sin, out1, s.T, eps);
+        return launch("simt_output", output<T, D, BIDIR, PHI>, g2, dim3(kThreads), smem, st, x, sin, out1, s.T, eps);
     }
     case Stage::BwdQ: {
         const size_t smemq = (size_t)(D * (D + 1) + D + 3 * kTile * (D + 1) + kTile) * sizeof(float);
-        rc = bidir ? launch("simt_bwd_q", bwd_q<T, D, true>, g1, dim3(kThreads), smemq, st, x, y, sin, out1, part, s.T,
-                            nsplit, rps, eps)
-                   : launch("simt_bwd_q", bwd_q<T, D, false>, g1, dim3(kThreads), smemq, st, x, y, sin, out1, part, s.T,
-                            nsplit, rps, eps);
+        rc = launch("simt_bwd_q", bwd_q<T, D, BIDIR, PHI>, g1, dim3(kThreads), smemq, st, x, y, sin, out1, part, s.T,
+                    nsplit, rps, eps);
         if (rc) return rc;
         return launch("simt_combine", combine, dim3((unsigned)s.BH()), dim3(kThreads), 0, st, (const float *)part, sout,
                       nsplit, D * (D + 1));
     }
     default: {
         const size_t smemk = (size_t)(D * (D + 1) + D + 3 * kTile * (D + 1)) * sizeof(float);
-        return bidir ? launch("simt_bwd_k", bwd_k<T, D, true>, g2, dim3(kThreads), smemk, st, x, y, sin, out1, out2, s.T)
-                     : launch("simt_bwd_k", bwd_k<T, D, false>, g2, dim3(kThreads), smemk, st, x, y, sin, out1, out2,
-                              s.T);
+        return launch("simt_bwd_k", bwd_k<T, D, BIDIR, PHI>, g2, dim3(kThreads), smemk, st, x, y, sin, out1, out2, s.T);
     }
     }
 }
 
+template <typename T, int D>
+la_status stage_t(Stage stage, la_feature f, const T *x, const T *y, const float *sin, float *sout, T *out1, T *out2,
+                  const Shape &s, float eps, void *ws, cudaStream_t st) {
+    if (f == LA_FEATURE_ELU1) return stage_tt<T, D, true, true>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st);
+    if (f == LA_FEATURE_NORM) return stage_tt<T, D, true, false>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st);
+    return stage_tt<T, D, false, false>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st);
+}
+
 template <typename T>
-la_status stage_d(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout, void *out1,
+la_status stage_d(Stage stage, la_feature f, const void *x, const void *y, const float *sin, float *sout, void *out1,
                   void *out2, const Shape &s, float eps, void *ws, cudaStream_t st) {
     if (s.D == 64)
-        return stage_t<T, 64>(stage, bidir, (const T *)x, (const T *)y, sin, sout, (T *)out1, (T *)out2, s, eps, ws, st);
-    return stage_t<T, 128>(stage, bidir, (const T *)x, (const T *)y, sin, sout, (T *)out1, (T *)out2, s, eps, ws, st);
+        return stage_t<T, 64>(stage, f, (const T *)x, (const T *)y, sin, sout, (T *)out1, (T *)out2, s, eps, ws, st);
+    return stage_t<T, 128>(stage, f, (const T *)x, (const T *)y, sin, sout, (T *)out1, (T *)out2, s, eps, ws, st);
 }
 
 template <typename T>
@@ -878,12 +879,12 @@ size_t workspace_size(la_op op, const Shape &s) {
     }
 }
 
-la_status state_stage(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout,
+la_status state_stage(Stage stage, la_feature f, const void *x, const void *y, const float *sin, float *sout,
                       void *out1, void *out2, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st) {
     switch (dt) {
-    case LA_F32: return stage_d<float>(stage, bidir, x, y, sin, sout, out1, out2, s, eps, ws, st);
-    case LA_F16: return stage_d<__half>(stage, bidir, x, y, sin, sout, out1, out2, s, eps, ws, st);
-    default: return stage_d<__nv_bfloat16>(stage, bidir, x, y, sin, sout, out1, out2, s, eps, ws, st);
+    case LA_F32: return stage_d<float>(stage, f, x, y, sin, sout, out1, out2, s, eps, ws, st);
+    case LA_F16: return stage_d<__half>(stage, f, x, y, sin, sout, out1, out2, s, eps, ws, st);
+    default: return stage_d<__nv_bfloat16>(stage, f, x, y, sin, sout, out1, out2, s, eps, ws, st);
     }
 }
 

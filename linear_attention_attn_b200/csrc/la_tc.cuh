@@ -36,7 +36,7 @@ la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, con
 la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
                     const DecayArgs &dec, const Shape &s, la_dtype dt, void *ws, cudaStream_t st);
 // One stage of the state form (Stage in la_internal.cuh).
-la_status state_stage(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout,
+la_status state_stage(Stage stage, la_feature f, const void *x, const void *y, const float *sin, float *sout,
                       void *out1, void *out2, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
 la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin,
                     const float *rin, float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv,

@@ -94,11 +94,17 @@ __device__ __forceinline__ uint32_t phi_h2(uint32_t x) {
     return bit_cast32<uint32_t>(__hadd2(__hmax2(hx, zero), bit_cast32<__half2>(ei)));
 }
 
+// The tile transforms below apply elu+1 when PHI is set and leave the values as
+// they are otherwise (features computed by the caller): then only the zeroing of
+// rows past the sequence end remains, and every lo part is zero (a 16-bit value
+// is its own 16-bit rounding).
+
 // Feature map elu+1 applied in place to row `row` of a 128-byte-swizzled tile
 // (the row's 8 chunks are visited in an order that spreads banks); rows that
 // lie past the sequence end are zeroed when `zero` is set.
-template <bool BF16>
+template <bool BF16, bool PHI = true>
 __device__ __forceinline__ void phi_row_inplace(uint8_t *tile, int row, bool zero) {
+    if (!PHI && !zero) return;
     uint8_t *p = tile + row * 128;
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
@@ -122,8 +128,16 @@ __device__ __forceinline__ void phi_row_inplace(uint8_t *tile, int row, bool zer
 // Feature map of one whole row of a 128-byte-swizzled tile in place, all eight
 // 16-byte chunks loaded before any is transformed (one shared-memory round trip
 // per row).  SPLIT keeps lo = round(phi(x) - hi) at the same position of lo_tile.
-template <bool BF16, bool SPLIT>
+template <bool BF16, bool SPLIT, bool PHI = true>
 __device__ __forceinline__ void phi_row_batched(uint8_t *tile, uint8_t *lo_tile, int row) {
+    if (!PHI) {
+        if (SPLIT) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4 *>(lo_tile + row * 128 + ((c ^ (row & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        return;
+    }
     uint8_t *p = tile + row * 128;
     uint4 u[8];
 #pragma unroll
@@ -153,10 +167,15 @@ __device__ __forceinline__ void phi_row_batched(uint8_t *tile, uint8_t *lo_tile,
 
 // Feature map with a two-term result: hi = round(phi(x)) replaces x in place,
 // lo = round(phi(x) - hi) goes to the same position of `lo_tile`.
-template <bool BF16>
+template <bool BF16, bool PHI = true>
 __device__ __forceinline__ void phi_row_split(uint8_t *tile, uint8_t *lo_tile, int row) {
     uint8_t *p = tile + row * 128;
     uint8_t *q = lo_tile + row * 128;
+    if (!PHI) {
+#pragma unroll
+        for (int it = 0; it < 8; ++it) *reinterpret_cast<uint4 *>(q + ((it ^ (row & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        return;
+    }
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
         const int off = (it ^ (row & 7)) << 4;
@@ -177,8 +196,9 @@ __device__ __forceinline__ void phi_row_split(uint8_t *tile, uint8_t *lo_tile, i
 
 // The transform warps split a tile into 256 half rows: thread xi handles row
 // xi % 128, logical chunks 4 * (xi / 128) .. + 3 (chunk order spreads banks).
-template <bool BF16>
+template <bool BF16, bool PHI = true>
 __device__ __forceinline__ void phi_half_row(uint8_t *tile, int xi, bool zero) {
+    if (!PHI && !zero) return;
     const int row = xi & 127, c0 = (xi >> 7) * 4;
     uint8_t *p = tile + row * 128;
 #pragma unroll
@@ -203,7 +223,7 @@ __device__ __forceinline__ void phi_half_row(uint8_t *tile, int xi, bool zero) {
 }
 
 // As phi_half_row, keeping lo = round(phi(x) - hi) in lo_tile (zeroing both when `zero`).
-template <bool BF16>
+template <bool BF16, bool PHI = true>
 __device__ __forceinline__ void phi_half_row_split(uint8_t *tile, uint8_t *lo_tile, int xi, bool zero) {
     const int row = xi & 127, c0 = (xi >> 7) * 4;
 #pragma unroll
@@ -213,7 +233,7 @@ __device__ __forceinline__ void phi_half_row_split(uint8_t *tile, uint8_t *lo_ti
         uint32_t w[4] = {u.x, u.y, u.z, u.w}, l[4] = {0u, 0u, 0u, 0u};
         if (zero) {
             w[0] = w[1] = w[2] = w[3] = 0u;
-        } else {
+        } else if (PHI) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const float2 f = h2<BF16>::to_f2(w[k]);

@@ -75,7 +75,7 @@ struct ReduceLayout {
     static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
 };
 
-template <bool BIDIR, bool BF16>
+template <bool BIDIR, bool BF16, bool PHI>
 __global__ void __launch_bounds__(kThreads, 1)
 state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     float *__restrict__ part, int T, int BH, int nt, int maxslots) {
@@ -213,9 +213,9 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 if (!got) break;
                 const bool pad = j * kRows + (xi & 127) >= T;   // rows past the end: f(0) = 1 must not count
                 if (KLO)
-                    phi_half_row_split<BF16>(sK + s * kTileBytes, sKlo + s * kTileBytes, xi, pad);
+                    phi_half_row_split<BF16, PHI>(sK + s * kTileBytes, sKlo + s * kTileBytes, xi, pad);
                 else
-                    phi_half_row<BF16>(sK + s * kTileBytes, xi, pad);
+                    phi_half_row<BF16, PHI>(sK + s * kTileBytes, xi, pad);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&xf[s]);
@@ -289,7 +289,7 @@ struct OutputLayout {
     static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
 };
 
-template <bool BIDIR, bool BF16>
+template <bool BIDIR, bool BF16, bool PHI>
 __global__ void __launch_bounds__(kThreads, 1)
 output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
               const float *__restrict__ src, int src_per_head, int src_single, float *__restrict__ state_out, int T,
@@ -418,7 +418,7 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
                 const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
                 if (!got) break;
-                phi_half_row<BF16>(sQ + s * kTileBytes, xi, false);   // rows past T are never stored
+                phi_half_row<BF16, PHI>(sQ + s * kTileBytes, xi, false);   // rows past T are never stored
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&xf[s]);
@@ -552,7 +552,7 @@ struct BwdQLayout {
     static_assert(kStateElems * 4 <= 2 * OPB, "the operand block stages a [dS | dz] partial");
 };
 
-template <bool BIDIR, bool BF16>
+template <bool BIDIR, bool BF16, bool PHI>
 __global__ void __launch_bounds__(kQThreads, 1)
 bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
              const __grid_constant__ CUtensorMap tmDQ, const float *__restrict__ src, int src_per_head,
@@ -756,7 +756,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
                 const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
                 if (!got) break;
-                phi_row_batched<BF16, QLO>(sQ + s * kTileBytes, sQlo + s * kTileBytes, r);
+                phi_row_batched<BF16, QLO, PHI>(sQ + s * kTileBytes, sQlo + s * kTileBytes, r);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&xf[s]);
@@ -833,7 +833,7 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                                 for (int e = 0; e < 4; ++e) {
                                     const int i = 4 * i4 + e;
                                     const float acc = cc ? a1[i] : a0[i];
-                                    dq[i] = (acc - gdot * zv[e]) * inv * fminf(qf[i], 1.f);
+                                    dq[i] = (acc - gdot * zv[e]) * inv * (PHI ? fminf(qf[i], 1.f) : 1.f);
                                 }
                             }
                         } else {
@@ -1049,7 +1049,7 @@ struct BwdKvLayout {
     static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
 };
 
-template <bool BIDIR, bool BF16>
+template <bool BIDIR, bool BF16, bool PHI>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
               const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
@@ -1189,7 +1189,7 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             for (TileCursor t(x0, nt); t.x < x1; t.next()) {
                 const bool got = __all_sync(0xffffffffu, LA_WAIT(&full[s], ph, 0x8u));
                 if (!got) break;
-                phi_half_row<BF16>(sK + s * kTileBytes, xi, false);
+                phi_half_row<BF16, PHI>(sK + s * kTileBytes, xi, false);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&xf[s]);
@@ -1243,7 +1243,7 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                         load_chunk16<BF16>(sK + s * kTileBytes, row, c16, kf);
                         tmem_ld_wait(aa, bb);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) out[i] = fmaf(aa[i], cur_isd, dz[16 * c16 + i]) * fminf(kf[i], 1.f);
+                        for (int i = 0; i < 16; ++i) out[i] = fmaf(aa[i], cur_isd, dz[16 * c16 + i]) * (PHI ? fminf(kf[i], 1.f) : 1.f);
                     } else {
                         tmem_ld_wait(aa, bb);
 #pragma unroll
@@ -1362,15 +1362,20 @@ static size_t partial_bytes(const Shape &s) {
     return (b + 255) & ~(size_t)255;
 }
 
-template <bool BIDIR, bool BF16>
+// Launch names (string literals: the profiler keeps the pointers): "<base>" for elu+1 with
+// the norm term, "<base>_norm" for the norm term on features the caller computed,
+// "<base>_simple" for neither.
+#define LA_KNAME(base) (!BIDIR ? base "_simple" : (PHI ? base : base "_norm"))
+
+template <bool BIDIR, bool BF16, bool PHI>
 static la_status launch_reduce(const CUtensorMap &mk, const CUtensorMap &mv, float *part, const Shape &s, int nt,
                                cudaStream_t st) {
-    return launch_pdl(BIDIR ? "tc_state_reduce" : "tc_state_reduce_simple", state_reduce_kernel<BIDIR, BF16>,
+    return launch_pdl(LA_KNAME("tc_state_reduce"), state_reduce_kernel<BIDIR, BF16, PHI>,
                   dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads), (size_t)ReduceLayout<BIDIR, BF16>::bytes, st, mk, mv, part, s.T, (int)s.BH(), nt,
                   max_slots((int)s.BH()));
 }
 
-template <bool BIDIR, bool BF16>
+template <bool BIDIR, bool BF16, bool PHI>
 static la_status fwd_t(const void *q, const void *k, const void *v, void *o, float *state, const Shape &s,
                        float eps, void *ws, cudaStream_t st) {
     CUtensorMap mq, mk, mv, mo;
@@ -1381,13 +1386,13 @@ static la_status fwd_t(const void *q, const void *k, const void *v, void *o, flo
     const int nt = (s.T + kRows - 1) / kRows;
     const int ms = max_slots((int)s.BH());
     float *part = (float *)ws;
-    LA_TRY((launch_reduce<BIDIR, BF16>(mk, mv, part, s, nt, st)));
-    return launch_pdl(BIDIR ? "tc_output" : "tc_output_simple", output_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
+    LA_TRY((launch_reduce<BIDIR, BF16, PHI>(mk, mv, part, s, nt, st)));
+    return launch_pdl(LA_KNAME("tc_output"), output_kernel<BIDIR, BF16, PHI>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
                   (size_t)OutputLayout::bytes, st, mq, mo, (const float *)part, ms * kStateElems, 0, state, s.T, (int)s.BH(), nt,
                   eps, 1);
 }
 
-template <bool BIDIR, bool BF16>
+template <bool BIDIR, bool BF16, bool PHI>
 static la_status bwd_t(const void *q, const void *k, const void *v, const void *g, const float *state, void *dq,
                        void *dk, void *dv, const Shape &s, float eps, void *ws, cudaStream_t st) {
     CUtensorMap mq, mk, mv, mg, mdq, mdk, mdv;
@@ -1405,15 +1410,15 @@ static la_status bwd_t(const void *q, const void *k, const void *v, const void *
     const float *src = state;
     int per_head = kStateElems, single = 1;
     if (!state) {
-        LA_TRY((launch_reduce<BIDIR, BF16>(mk, mv, spart, s, nt, st)));
+        LA_TRY((launch_reduce<BIDIR, BF16, PHI>(mk, mv, spart, s, nt, st)));
         src = spart;
         per_head = ms * kStateElems;
         single = 0;
     }
-    LA_TRY(launch_pdl(BIDIR ? "tc_bwd_q" : "tc_bwd_q_simple", bwd_q_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kQThreads),
+    LA_TRY(launch_pdl(LA_KNAME("tc_bwd_q"), bwd_q_kernel<BIDIR, BF16, PHI>, dim3(grid_for((long long)s.BH() * nt)), dim3(kQThreads),
                   (size_t)BwdQLayout<BIDIR, BF16>::bytes, st, mq, mg, mdq, src, per_head, single, dpart, s.T, (int)s.BH(),
                   nt, ms, eps, state ? 0 : 1));
-    return launch_pdl(BIDIR ? "tc_bwd_kv" : "tc_bwd_kv_simple", bwd_kv_kernel<BIDIR, BF16>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
+    return launch_pdl(LA_KNAME("tc_bwd_kv"), bwd_kv_kernel<BIDIR, BF16, PHI>, dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads),
                   (size_t)BwdKvLayout::bytes, st, mk, mv, mdk, mdv, (const float *)dpart, ms * kStateElems, 0, s.T,
                   (int)s.BH(), nt, 1);
 }
@@ -1421,7 +1426,7 @@ static la_status bwd_t(const void *q, const void *k, const void *v, const void *
 // The state form in separate stages, for a sequence split along T (see the
 // sequence-parallel entry points): the caller sums the stages' states across
 // the shards between them.
-template <bool BIDIR, bool BF16>
+template <bool BIDIR, bool BF16, bool PHI>
 static la_status stage_t(Stage stage, const void *x, const void *y, const float *sin, float *sout, void *out1,
                          void *out2, const Shape &s, float eps, void *ws, cudaStream_t st) {
     const int nt = (s.T + kRows - 1) / kRows;
@@ -1432,7 +1437,7 @@ static la_status stage_t(Stage stage, const void *x, const void *y, const float 
         CUtensorMap mk, mv;
         LA_TRY(tensor_map(&mk, x, s, BF16));
         LA_TRY(tensor_map(&mv, y, s, BF16));
-        LA_TRY((launch_reduce<BIDIR, BF16>(mk, mv, part, s, nt, st)));
+        LA_TRY((launch_reduce<BIDIR, BF16, PHI>(mk, mv, part, s, nt, st)));
         return launch("tc_combine", combine_partials_kernel, dim3((unsigned)s.BH()), dim3(256), 0, st,
                       (const float *)part, sout, (int)s.BH(), nt, ms);
     }
@@ -1440,7 +1445,7 @@ static la_status stage_t(Stage stage, const void *x, const void *y, const float 
         CUtensorMap mq, mo;
         LA_TRY(tensor_map(&mq, x, s, BF16));
         LA_TRY(tensor_map(&mo, out1, s, BF16));
-        return launch_pdl(BIDIR ? "tc_output" : "tc_output_simple", output_kernel<BIDIR, BF16>,
+        return launch_pdl(LA_KNAME("tc_output"), output_kernel<BIDIR, BF16, PHI>,
                           dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads), (size_t)OutputLayout::bytes, st, mq,
                           mo, sin, kStateElems, 1, (float *)nullptr, s.T, (int)s.BH(), nt, eps, 0);
     }
@@ -1449,7 +1454,7 @@ static la_status stage_t(Stage stage, const void *x, const void *y, const float 
         LA_TRY(tensor_map(&mq, x, s, BF16));
         LA_TRY(tensor_map(&mg, y, s, BF16));
         LA_TRY(tensor_map(&mdq, out1, s, BF16));
-        LA_TRY(launch_pdl(BIDIR ? "tc_bwd_q" : "tc_bwd_q_simple", bwd_q_kernel<BIDIR, BF16>,
+        LA_TRY(launch_pdl(LA_KNAME("tc_bwd_q"), bwd_q_kernel<BIDIR, BF16, PHI>,
                           dim3(grid_for((long long)s.BH() * nt)), dim3(kQThreads), (size_t)BwdQLayout<BIDIR, BF16>::bytes,
                           st, mq, mg, mdq, sin, kStateElems, 1, part, s.T, (int)s.BH(), nt, ms, eps, 0));
         return launch("tc_combine", combine_partials_kernel, dim3((unsigned)s.BH()), dim3(256), 0, st,
@@ -1461,7 +1466,7 @@ static la_status stage_t(Stage stage, const void *x, const void *y, const float 
         LA_TRY(tensor_map(&mv, y, s, BF16));
         LA_TRY(tensor_map(&mdk, out1, s, BF16));
         LA_TRY(tensor_map(&mdv, out2, s, BF16));
-        return launch_pdl(BIDIR ? "tc_bwd_kv" : "tc_bwd_kv_simple", bwd_kv_kernel<BIDIR, BF16>,
+        return launch_pdl(LA_KNAME("tc_bwd_kv"), bwd_kv_kernel<BIDIR, BF16, PHI>,
                           dim3(grid_for((long long)s.BH() * nt)), dim3(kThreads), (size_t)BwdKvLayout::bytes, st, mk,
                           mv, mdk, mdv, sin, kStateElems, 1, s.T, (int)s.BH(), nt, 0);
     }
@@ -1482,31 +1487,35 @@ size_t state_workspace_size(la_op op, const Shape &s) {
     }
 }
 
-la_status state_stage(Stage stage, bool bidir, const void *x, const void *y, const float *sin, float *sout,
+la_status state_stage(Stage stage, la_feature f, const void *x, const void *y, const float *sin, float *sout,
                       void *out1, void *out2, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st) {
     const bool bf = dt == LA_BF16;
-    if (bidir) return bf ? stage_t<true, true>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st)
-                         : stage_t<true, false>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st);
-    return bf ? stage_t<false, true>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st)
-              : stage_t<false, false>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st);
+    if (f == LA_FEATURE_ELU1)
+        return bf ? stage_t<true, true, true>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st)
+                  : stage_t<true, false, true>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st);
+    if (f == LA_FEATURE_NORM)
+        return bf ? stage_t<true, true, false>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st)
+                  : stage_t<true, false, false>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st);
+    return bf ? stage_t<false, true, false>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st)
+              : stage_t<false, false, false>(stage, x, y, sin, sout, out1, out2, s, eps, ws, st);
 }
 
 la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, void *o, float *state, const Shape &s,
                     la_dtype dt, float eps, void *ws, cudaStream_t st) {
     const bool bf = dt == LA_BF16;
-    if (bidir) return bf ? fwd_t<true, true>(q, k, v, o, state, s, eps, ws, st)
-                         : fwd_t<true, false>(q, k, v, o, state, s, eps, ws, st);
-    return bf ? fwd_t<false, true>(q, k, v, o, state, s, eps, ws, st)
-              : fwd_t<false, false>(q, k, v, o, state, s, eps, ws, st);
+    if (bidir) return bf ? fwd_t<true, true, true>(q, k, v, o, state, s, eps, ws, st)
+                         : fwd_t<true, false, true>(q, k, v, o, state, s, eps, ws, st);
+    return bf ? fwd_t<false, true, false>(q, k, v, o, state, s, eps, ws, st)
+              : fwd_t<false, false, false>(q, k, v, o, state, s, eps, ws, st);
 }
 
 la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, const void *g, const float *state,
                     void *dq, void *dk, void *dv, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st) {
     const bool bf = dt == LA_BF16;
-    if (bidir) return bf ? bwd_t<true, true>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st)
-                         : bwd_t<true, false>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st);
-    return bf ? bwd_t<false, true>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st)
-              : bwd_t<false, false>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st);
+    if (bidir) return bf ? bwd_t<true, true, true>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st)
+                         : bwd_t<true, false, true>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st);
+    return bf ? bwd_t<false, true, false>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st)
+              : bwd_t<false, false, false>(q, k, v, g, state, dq, dk, dv, s, eps, ws, st);
 }
 
 unsigned int read_and_clear_state_fault() {

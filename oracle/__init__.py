@@ -63,11 +63,16 @@ def _bind(lib):
     lib.oracle_retention_fwd_state.argtypes = [P, P, P, P, P, P, P, L, L, L, L, I]
     lib.oracle_retention_bwd_state.argtypes = [P, P, P, P, P, P, P, P, P, P, P, L, L, L, L, I]
     lib.oracle_causal_norm_fwd.argtypes = [P, P, P, P, I, Dbl, P, L, L, L, L, I]
+    lib.oracle_normed_fwd.argtypes = [P, P, P, P, P, L, L, L, L, Dbl, I]
+    lib.oracle_normed_bwd.argtypes = [P, P, P, P, P, P, P, L, L, L, L, Dbl, I]
+    lib.oracle_feature_map_fwd.argtypes = [I, Dbl, P, P, L, L]
+    lib.oracle_feature_map_bwd.argtypes = [I, Dbl, P, P, P, L, L]
     lib.oracle_causal_norm_bwd.argtypes = [P, P, P, P, P, I, Dbl, P, P, P, L, L, L, L, I]
     for name in ("oracle_bidir_fwd", "oracle_simple_fwd", "oracle_bidir_bwd",
                  "oracle_simple_bwd", "oracle_retention_fwd", "oracle_retention_bwd",
                  "oracle_retention_step", "oracle_retention_fwd_state", "oracle_retention_bwd_state",
-                 "oracle_causal_norm_fwd", "oracle_causal_norm_bwd"):
+                 "oracle_causal_norm_fwd", "oracle_causal_norm_bwd", "oracle_normed_fwd", "oracle_normed_bwd",
+                 "oracle_feature_map_fwd", "oracle_feature_map_bwd"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -226,6 +231,52 @@ class Oracle:
         _check(rc, "oracle_retention_bwd_state")
         return dq, dk, dv, rout
 
+    def normed_fwd(self, q, k, v, eps: float = 1e-6, nthreads: int | None = None, want_state: bool = False):
+        """The bidirectional op with the identity feature map (q, k are features formed by the
+        caller): o = q S / (q . z + eps), S = sum_s k_s^T v_s, z = sum_s k_s."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, H, T, D = _shape4(q)
+        o = np.empty_like(q)
+        st = np.empty((B, H, D, D + 1)) if want_state else None
+        rc = self._lib.oracle_normed_fwd(_p(q), _p(k), _p(v), _p(o), _p(st) if st is not None else None,
+                                         B, H, T, D, float(eps), nthreads or default_threads())
+        _check(rc, "oracle_normed_fwd")
+        return (o, st) if want_state else o
+
+    def normed_bwd(self, q, k, v, dout, eps: float = 1e-6, nthreads: int | None = None):
+        """Gradients (dq, dk, dv) of sum(o * dout) for normed_fwd."""
+        q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(dout)
+        B, H, T, D = _shape4(q)
+        dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+        rc = self._lib.oracle_normed_bwd(_p(q), _p(k), _p(v), _p(g), _p(dq), _p(dk), _p(dv),
+                                         B, H, T, D, float(eps), nthreads or default_threads())
+        _check(rc, "oracle_normed_bwd")
+        return dq, dk, dv
+
+    FMAPS = {"focused": 0, "polarity": 1, "polarity_swap": 2}
+
+    def feature_map_fwd(self, kind, x, p: float = 1.0):
+        """Row-wise feature map of x [..., D]: 'focused' (width D) or 'polarity' / 'polarity_swap'
+        (width 2D)."""
+        x = np.ascontiguousarray(_f64(x))
+        D = x.shape[-1]
+        kd = self.FMAPS[kind]
+        w = D if kd == 0 else 2 * D
+        y = np.empty(x.shape[:-1] + (w,))
+        rc = self._lib.oracle_feature_map_fwd(kd, float(p), _p(x), _p(y), int(x.size // D), D)
+        _check(rc, "oracle_feature_map_fwd")
+        return y
+
+    def feature_map_bwd(self, kind, x, dy, p: float = 1.0):
+        """dx = J^T dy for feature_map_fwd."""
+        x = np.ascontiguousarray(_f64(x))
+        dy = np.ascontiguousarray(_f64(dy))
+        D = x.shape[-1]
+        dx = np.empty_like(x)
+        rc = self._lib.oracle_feature_map_bwd(self.FMAPS[kind], float(p), _p(x), _p(dy), _p(dx), int(x.size // D), D)
+        _check(rc, "oracle_feature_map_bwd")
+        return dx
+
     def _causal_args(self, q, gamma, feature):
         B, H, T, D = _shape4(q)
         gm = None if gamma is None else _f64(gamma).reshape(-1)
@@ -334,3 +385,19 @@ def causal_norm_fwd(*a, **kw):
 
 def causal_norm_bwd(*a, **kw):
     return _instance().causal_norm_bwd(*a, **kw)
+
+
+def normed_fwd(*a, **kw):
+    return _instance().normed_fwd(*a, **kw)
+
+
+def normed_bwd(*a, **kw):
+    return _instance().normed_bwd(*a, **kw)
+
+
+def feature_map_fwd(*a, **kw):
+    return _instance().feature_map_fwd(*a, **kw)
+
+
+def feature_map_bwd(*a, **kw):
+    return _instance().feature_map_bwd(*a, **kw)

@@ -544,3 +544,102 @@ int oracle_causal_norm_bwd(const double *q, const double *k, const double *v, co
     return for_each_head(&jb, causal_bwd_head, (size_t)(2 * D * D + 4 * D + 2 * T), nthreads);
 }
 
+/* --------------------- bidirectional with the norm term on given features -- */
+
+/* la_bidir's definition with f the identity: q, k are features the caller formed. */
+int oracle_normed_fwd(const double *q, const double *k, const double *v, double *o, double *state,
+                      long B, long H, long T, long D, double eps, int nthreads) {
+    if (check_dims(B, H, T, D) || !q || !k || !v || !o) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.o = o; jb.state = state;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D; jb.eps = eps; jb.use_phi = 0; jb.use_norm = 1;
+    return for_each_head(&jb, state_fwd_head, (size_t)(D * D + 2 * D), nthreads);
+}
+
+int oracle_normed_bwd(const double *q, const double *k, const double *v, const double *dout,
+                      double *dq, double *dk, double *dv,
+                      long B, long H, long T, long D, double eps, int nthreads) {
+    if (check_dims(B, H, T, D) || !q || !k || !v || !dout || !dq || !dk || !dv) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.g = dout; jb.dq = dq; jb.dk = dk; jb.dv = dv;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D; jb.eps = eps; jb.use_phi = 0; jb.use_norm = 1;
+    return for_each_head(&jb, state_bwd_head, (size_t)(2 * D * D + 4 * D), nthreads);
+}
+
+/* ----------------------------------------------------- feature maps, per row -- */
+
+/* kind 0, the focusing function of focused linear attention: with y = relu(x),
+ *   f(x) = (|y| / |y^p|) y^p      (|.| the 2-norm of the row, y^p elementwise; 0 if y = 0),
+ * so the row keeps the norm of relu(x) while its direction sharpens towards the
+ * largest entries.  Kinds 1 and 2, the polarity split: f(x) = [relu(x)^p, relu(-x)^p]
+ * (kind 1) or [relu(-x)^p, relu(x)^p] (kind 2), twice the width of x. */
+static int fmap_width(int kind, long D) { return kind == 0 ? (int)D : (int)(2 * D); }
+
+static void fmap_row_fwd(int kind, double p, const double *x, double *y, long D) {
+    if (kind == 0) {
+        double a = 0.0, b = 0.0;
+        for (long i = 0; i < D; ++i) {
+            const double r = x[i] > 0.0 ? x[i] : 0.0;
+            a += r * r;
+            b += pow(r, 2.0 * p);
+        }
+        a = sqrt(a);
+        b = sqrt(b);
+        for (long i = 0; i < D; ++i) {
+            const double r = x[i] > 0.0 ? x[i] : 0.0;
+            y[i] = b > 0.0 ? (a / b) * pow(r, p) : 0.0;
+        }
+        return;
+    }
+    for (long i = 0; i < D; ++i) {
+        const double pos = x[i] > 0.0 ? pow(x[i], p) : 0.0, neg = x[i] < 0.0 ? pow(-x[i], p) : 0.0;
+        y[i] = kind == 1 ? pos : neg;
+        y[D + i] = kind == 1 ? neg : pos;
+    }
+}
+
+/* dx = J^T dy, J the Jacobian of the row's map.  Focusing function, with a = |y|,
+ * b = |y^p|, u = y^p and s = dy . u (y = relu(x)):
+ *   dx_j = [x_j > 0] ((a / b) p y_j^(p-1) dy_j + s y_j / (a b) - s a p y_j^(2p-1) / b^3).
+ * Polarity split: d relu(x)^p / dx = p x^(p-1) [x > 0], d relu(-x)^p / dx = -p (-x)^(p-1) [x < 0]. */
+static void fmap_row_bwd(int kind, double p, const double *x, const double *dy, double *dx, long D) {
+    if (kind == 0) {
+        double a = 0.0, b = 0.0, s = 0.0;
+        for (long i = 0; i < D; ++i) {
+            const double r = x[i] > 0.0 ? x[i] : 0.0;
+            a += r * r;
+            b += pow(r, 2.0 * p);
+            s += dy[i] * pow(r, p);
+        }
+        a = sqrt(a);
+        b = sqrt(b);
+        for (long j = 0; j < D; ++j) {
+            if (!(x[j] > 0.0) || b <= 0.0) { dx[j] = 0.0; continue; }
+            const double r = x[j];
+            dx[j] = (a / b) * p * pow(r, p - 1.0) * dy[j] + s * r / (a * b) - s * a * p * pow(r, 2.0 * p - 1.0) / (b * b * b);
+        }
+        return;
+    }
+    for (long i = 0; i < D; ++i) {
+        const double dpos = x[i] > 0.0 ? p * pow(x[i], p - 1.0) : 0.0;
+        const double dneg = x[i] < 0.0 ? -p * pow(-x[i], p - 1.0) : 0.0;
+        const double gpos = kind == 1 ? dy[i] : dy[D + i], gneg = kind == 1 ? dy[D + i] : dy[i];
+        dx[i] = gpos * dpos + gneg * dneg;
+    }
+}
+
+/* x [rows, D] -> y [rows, width]; p > 0. */
+int oracle_feature_map_fwd(int kind, double p, const double *x, double *y, long rows, long D) {
+    if (kind < 0 || kind > 2 || !(p > 0.0) || rows < 0 || D < 1 || (rows > 0 && (!x || !y))) return -1;
+    const long w = fmap_width(kind, D);
+    for (long r = 0; r < rows; ++r) fmap_row_fwd(kind, p, x + r * D, y + r * w, D);
+    return 0;
+}
+
+int oracle_feature_map_bwd(int kind, double p, const double *x, const double *dy, double *dx, long rows, long D) {
+    if (kind < 0 || kind > 2 || !(p > 0.0) || rows < 0 || D < 1 || (rows > 0 && (!x || !dy || !dx))) return -1;
+    const long w = fmap_width(kind, D);
+    for (long r = 0; r < rows; ++r) fmap_row_bwd(kind, p, x + r * D, dy + r * w, dx + r * D, D);
+    return 0;
+}
+

@@ -446,6 +446,80 @@ def check_causal_norm(orc):
             _close(a, b, rtol=1e-6, atol=1e-7, what="causal norm %s %s vs finite differences" % (feature, name))
 
 
+def _focus_np(x, p):
+    """The focusing function written independently (numpy): y = relu(x), (|y| / |y^p|) y^p per row."""
+    y = np.maximum(np.asarray(x, dtype=np.float64), 0.0)
+    yp = y ** p
+    a = np.linalg.norm(y, axis=-1, keepdims=True)
+    b = np.linalg.norm(yp, axis=-1, keepdims=True)
+    return np.where(b > 0, a / np.where(b > 0, b, 1.0) * yp, 0.0)
+
+
+def _fd_rows(fn, x, dy, h=1e-6):
+    """Central differences of sum(fn(x) * dy) with respect to x."""
+    g = np.zeros_like(x)
+    for mi in np.ndindex(*x.shape):
+        a = x.copy()
+        a[mi] += h
+        lp = float((fn(a) * dy).sum())
+        a[mi] -= 2 * h
+        g[mi] = (lp - float((fn(a) * dy).sum())) / (2 * h)
+    return g
+
+
+def check_feature_maps(orc):
+    """The focusing function and the polarity split: a hand-worked row, the norm of relu(x) kept,
+    degree-1 homogeneity, p = 1 giving relu(x), the split recovering x, finite-difference gradients,
+    and agreement with an independent numpy restatement."""
+    # hand-worked: x = (1, 2, -1), p = 2: y = (1, 2, 0), |y| = sqrt 5, y^2 = (1, 4, 0), |y^2| = sqrt 17
+    _close(orc.feature_map_fwd("focused", np.array([[1.0, 2.0, -1.0]]), 2.0),
+           np.array([[1.0, 4.0, 0.0]]) * np.sqrt(5.0 / 17.0), rtol=1e-15, atol=0, what="focusing, hand-worked")
+    x = _rand((5, 7), 91)
+    x[2] = -np.abs(x[2])                                   # a row with no positive entry maps to 0
+    for p in (1.0, 2.0, 3.0):
+        f = orc.feature_map_fwd("focused", x, p)
+        _close(f, _focus_np(x, p), rtol=1e-13, atol=1e-15, what="focusing vs numpy, p=%g" % p)
+        _close(np.linalg.norm(f, axis=-1), np.linalg.norm(np.maximum(x, 0), axis=-1), rtol=1e-13, atol=1e-15,
+               what="focusing keeps |relu(x)|")
+        _close(orc.feature_map_fwd("focused", 2.5 * x, p), 2.5 * f, rtol=1e-13, atol=1e-15, what="degree 1")
+    _close(orc.feature_map_fwd("focused", x, 1.0), np.maximum(x, 0), rtol=1e-15, atol=0, what="p = 1 is relu")
+    s1, s2 = orc.feature_map_fwd("polarity", x, 1.0), orc.feature_map_fwd("polarity_swap", x, 1.0)
+    _close(s1[:, :7] - s1[:, 7:], x, rtol=0, atol=0, what="polarity split recovers x")
+    _close(s2, np.concatenate([s1[:, 7:], s1[:, :7]], axis=1), rtol=0, atol=0, what="swapped halves")
+    _close(orc.feature_map_fwd("polarity", x, 3.0)[:, :7], np.maximum(x, 0) ** 3, rtol=1e-15, atol=0,
+           what="polarity power")
+    xs = _keep_off_zero(_rand((3, 5), 92), 5e-2)
+    for kind, p, w in (("focused", 3.0, 5), ("focused", 1.5, 5), ("polarity", 2.0, 10), ("polarity_swap", 1.0, 10)):
+        dy = _rand((3, w), 93)
+        fd = _fd_rows(lambda a: orc.feature_map_fwd(kind, a, p), xs, dy)
+        _close(orc.feature_map_bwd(kind, xs, dy, p), fd, rtol=1e-6, atol=1e-8,
+               what="%s p=%g gradient vs finite differences" % (kind, p))
+
+
+def check_normed(orc):
+    """The bidirectional op on caller-formed features: the pairwise form; phi applied outside gives
+    the elu+1 op exactly; focused linear attention (the focusing function then this op) against an
+    independent numpy pairwise form; finite-difference gradients."""
+    B, H, T, D = 2, 2, 9, 4
+    q, k, v = np.abs(_rand((B, H, T, D), 94)), np.abs(_rand((B, H, T, D), 95)), _rand((B, H, T, D), 96)
+    a = np.einsum("bhti,bhsi->bhts", q, k)
+    _close(orc.normed_fwd(q, k, v, eps=1e-3), np.einsum("bhts,bhsj->bhtj", a, v) / (a.sum(-1, keepdims=True) + 1e-3),
+           rtol=1e-12, atol=1e-13, what="normed vs pairwise")
+    qr, kr = _rand((B, H, T, D), 97), _rand((B, H, T, D), 98)
+    _close(orc.normed_fwd(_feature(qr), _feature(kr), v, eps=1e-3), orc.bidir_fwd(qr, kr, v, eps=1e-3),
+           rtol=1e-12, atol=1e-13, what="normed on phi(q), phi(k) = bidir")
+    fq, fk = _focus_np(qr, 3.0), _focus_np(kr, 3.0)
+    a = np.einsum("bhti,bhsi->bhts", fq, fk)
+    want = np.einsum("bhts,bhsj->bhtj", a, v) / (a.sum(-1, keepdims=True) + 1e-2)
+    got = orc.normed_fwd(orc.feature_map_fwd("focused", qr, 3.0), orc.feature_map_fwd("focused", kr, 3.0), v, eps=1e-2)
+    _close(got, want, rtol=1e-11, atol=1e-12, what="focused linear attention")
+    qs, ks = np.abs(_rand((1, 2, 5, 3), 99)) + 0.1, np.abs(_rand((1, 2, 5, 3), 100)) + 0.1
+    vs, gs = _rand((1, 2, 5, 3), 101), _rand((1, 2, 5, 3), 102)
+    fd = _fd_grads(lambda x, y, z: orc.normed_fwd(x, y, z, eps=0.05), qs, ks, vs, gs)
+    for name, a, b in zip(("dq", "dk", "dv"), orc.normed_bwd(qs, ks, vs, gs, eps=0.05), fd):
+        _close(a, b, rtol=1e-6, atol=1e-7, what="normed %s vs finite differences" % name)
+
+
 ALL_CHECKS = (check_golden, check_brute, check_closed_forms, check_invariances,
               check_fd_gradients, check_autograd, check_decode_step, check_state_segments,
-              check_segment_backward, check_causal_norm)
+              check_segment_backward, check_causal_norm, check_feature_maps, check_normed)

@@ -51,6 +51,13 @@ MUTATIONS = [
     ("causal_bwd_drops_r", "double a = r[i];", "double a = 0.0;", 0),
     ("causal_bwd_dk_uses_f", "dk[s * D + i] = a * dfeat(jb, k[s * D + i]);", "dk[s * D + i] = a * feat(jb, k[s * D + i]);", 0),
     ("causal_bwd_dq_drops_z", "double a = z[i] * dn;", "double a = 0.0;", 0),
+    ("focus_drops_norm_ratio", "y[i] = b > 0.0 ? (a / b) * pow(r, p) : 0.0;", "y[i] = b > 0.0 ? pow(r, p) : 0.0;", 0),
+    ("focus_bwd_s_term_sign", "+ s * r / (a * b) - s * a * p", "- s * r / (a * b) - s * a * p", 0),
+    ("polarity_halves_swapped", "y[i] = kind == 1 ? pos : neg;", "y[i] = kind == 1 ? neg : pos;", 0),
+    ("polarity_bwd_neg_sign", "const double dneg = x[i] < 0.0 ? -p * pow(-x[i], p - 1.0) : 0.0;",
+     "const double dneg = x[i] < 0.0 ? p * pow(-x[i], p - 1.0) : 0.0;", 0),
+    ("normed_uses_phi", "jb.eps = eps; jb.use_phi = 0; jb.use_norm = 1;\n    return for_each_head(&jb, state_fwd_head",
+     "jb.eps = eps; jb.use_phi = 1; jb.use_norm = 1;\n    return for_each_head(&jb, state_fwd_head", 0),
     ("fwd_state_out_before_last_token", "    if (jb->state_out) memcpy(jb->state_out + bh * D * D, S,",
      "    if (jb->state_out) memcpy(jb->state_out + bh * D * D, jb->state_in ? jb->state_in + bh * D * D : S,", 0),
 ]
