@@ -63,6 +63,11 @@ CAUSAL_FLOPS = {
     "simt_causal_norm_fwd": lambda D: 4 * D * (D + 1),
     "simt_causal_norm_bwd_q": lambda D: 4 * D * (D + 1) + 4 * D * D,
     "simt_causal_norm_bwd_kv": lambda D: 8 * D * D,
+    # gated: the D columns (forward) or rows (dq) of S, each D FMAs to update and D to read out;
+    # the reverse sweep holds the rows and the columns of R
+    "simt_gated_fwd": lambda D: 4 * D * D,
+    "simt_gated_bwd_q": lambda D: 4 * D * D,
+    "simt_gated_bwd_kv": lambda D: 8 * D * D,
 }
 
 
@@ -214,6 +219,9 @@ def _oracle_step(w, q, k, v, g, gamma, nthreads):
     elif w.op == "causal_norm":
         oracle.causal_norm_fwd(q, k, v, None, "elu1", w.eps, nthreads=nthreads)
         oracle.causal_norm_bwd(q, k, v, g, None, "elu1", w.eps, nthreads=nthreads)
+    elif w.op == "gated":
+        oracle.gated_fwd(q, k, v, gamma, nthreads=nthreads)       # gamma carries the log gates here
+        oracle.gated_bwd(q, k, v, gamma, g, nthreads=nthreads)
     else:
         oracle.retention_fwd(q, k, v, gamma, nthreads=nthreads)
         oracle.retention_bwd(q, k, v, g, gamma, nthreads=nthreads)
@@ -228,9 +236,12 @@ def oracle_step_sample(w, inp, budget_s: float, threads: int):
     v = inp["v"].reshape(BH, w.T, w.D)
     g = inp["do"].reshape(BH, w.T, w.D)
     gam = inp.get("gamma")
+    lgate = inp["g"].reshape(BH, w.T, w.D) if "g" in inp else None
 
     def heads(n, Ts):
         x = [t[:n, :Ts].reshape(1, n, Ts, w.D) for t in (q, k, v, g)]
+        if lgate is not None:          # gated: the log gates of the same heads and tokens
+            return x + [lgate[:n, :Ts].reshape(1, n, Ts, w.D)]
         gm = None if gam is None else gam.reshape(-1)[[i % w.H for i in range(n)]]
         return x + [gm]
 
@@ -295,6 +306,9 @@ WORKLOAD_TEXT = {
               "q,k ~ N(0,1) D^-1/2, v, dO ~ N(0,1)",
     "retention": "chunked causal decay (retention) fwd+bwd, bf16 storage / fp32 accumulate, B=%d H=%d T=%d D=%d, "
                  "gamma_h = 1 - 2^(-5-7h/(H-1)), q ~ N(0,1) D^-1/2, k, v, dO ~ N(0,1)",
+    "gated": "gated linear attention fwd+bwd (recurrent form on CUDA cores), bf16 storage / fp32 accumulate, "
+             "B=%d H=%d T=%d D=%d, log gates log(sigmoid(N(0,1)))/16 per token and key dimension, "
+             "q ~ N(0,1) D^-1/2, k, v, dO ~ N(0,1)",
     "causal_norm": "causal linear attention with the norm term fwd+bwd (recurrent form on CUDA cores), fp16 storage / "
                    "fp32 accumulate, B=%d H=%d T=%d D=%d, phi=elu+1, no decay, eps=1e-06, Q,K,V ~ 0.5 N(0,1), "
                    "dO ~ N(0,1)",
@@ -348,7 +362,7 @@ def run_ours(args, w):
     if seqpar:
         # the workload's T is the whole sequence; this rank holds a shard of T / world tokens
         from linear_attention_attn_b200 import seqpar as sp
-        if w.op in ("retention", "causal_norm") or w.T % world:
+        if w.op in ("retention", "causal_norm", "gated") or w.T % world:
             raise SystemExit("--seqpar needs the bidir or simple workload and T divisible by the GPU count")
         host = synth.make_inputs(w.with_T(w.T // world), seed=rank)
     else:
@@ -361,12 +375,15 @@ def run_ours(args, w):
     dstate = torch.empty_like(state)
     names = {"bidir": ("bidir_fwd", "bidir_bwd"), "simple": ("simple_fwd", "simple_bwd"),
              "retention": ("chunk_decay_fwd", "chunk_decay_bwd"),
-             "causal_norm": ("causal_norm_fwd", "causal_norm_bwd")}[w.op]
+             "causal_norm": ("causal_norm_fwd", "causal_norm_bwd"), "gated": ("gated_fwd", "gated_bwd")}[w.op]
     if seqpar:
         names = ("state_reduce", "state_bwd_q")
     ws_bytes = max(la.la_workspace_size(n, B, H, T, D, q.dtype) for n in names)
     ws = torch.empty(max(256, ws_bytes), dtype=torch.uint8, device=dev)
     gamma = host.get("gamma")
+    gated = w.op == "gated"
+    lgate = host["g"].to(dev) if gated else None     # the log gates
+    dgate = torch.empty_like(q) if gated else None
     feature = "elu1" if w.op == "bidir" else "identity"
 
     def step():
@@ -382,6 +399,9 @@ def run_ours(args, w):
         elif w.op == "causal_norm":
             la.la_causal_norm_fwd(q, k, v, o, None, "elu1", w.eps)
             la.la_causal_norm_bwd(q, k, v, g, dq, dk, dv, None, "elu1", w.eps, workspace=ws)
+        elif gated:
+            la.la_gated_fwd(q, k, v, lgate, o)
+            la.la_gated_bwd(q, k, v, lgate, g, dq, dk, dv, dgate, workspace=ws)
         else:
             la.la_chunk_decay_fwd(q, k, v, o, gamma, workspace=ws)
             la.la_chunk_decay_bwd(q, k, v, g, gamma, dq, dk, dv, workspace=ws)
@@ -435,15 +455,18 @@ def run_ours(args, w):
     #      every step copies its inputs in and its outputs out; the copies of neighbouring steps
     #      overlap the compute (three streams, two device buffer sets), as a serving loop would run
     e2e = None
-    hq, hk, hv, hg = (host[n].pin_memory() for n in ("q", "k", "v", "do"))
-    hout = [[torch.empty_like(hq).pin_memory() for _ in range(4)] for _ in range(2)]
+    in_names = ["q", "k", "v", "do"] + (["g"] if gated else [])
+    hins = [host[n].pin_memory() for n in in_names]
+    n_out = 5 if gated else 4                    # o, dq, dk, dv (and the log gates' gradient)
+    hout = [[torch.empty_like(hins[0]).pin_memory() for _ in range(n_out)] for _ in range(2)]
     sets = []
     for si in range(2):
         if si == 0:
-            ins, outs = [q, k, v, g], [o, dq, dk, dv]
+            ins = [q, k, v, g] + ([lgate] if gated else [])
+            outs = [o, dq, dk, dv] + ([dgate] if gated else [])
         else:
-            ins = [torch.empty_like(q) for _ in range(4)]
-            outs = [torch.empty_like(q) for _ in range(4)]
+            ins = [torch.empty_like(q) for _ in in_names]
+            outs = [torch.empty_like(q) for _ in range(n_out)]
         sets.append((ins, outs, torch.empty_like(state)))
     s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     ev_in = [torch.cuda.Event() for _ in range(2)]
@@ -452,11 +475,13 @@ def run_ours(args, w):
 
     def e2e_step(i):
         si = i % 2
-        (xq, xk, xv, xg), (xo, xdq, xdk, xdv), xst = sets[si]
+        ins, outs, xst = sets[si]
+        xq, xk, xv, xg = ins[:4]
+        xo, xdq, xdk, xdv = outs[:4]
         with torch.cuda.stream(s_in):
             if i >= 2:
                 s_in.wait_event(ev_cmp[si])           # step i-2 is done with this input set
-            for d_, h_ in zip((xq, xk, xv, xg), (hq, hk, hv, hg)):
+            for d_, h_ in zip(ins, hins):
                 d_.copy_(h_, non_blocking=True)
             ev_in[si].record(s_in)
         s_cmp.wait_event(ev_in[si])
@@ -471,13 +496,16 @@ def run_ours(args, w):
         elif w.op == "causal_norm":
             la.la_causal_norm_fwd(xq, xk, xv, xo, None, "elu1", w.eps, stream=s_cmp)
             la.la_causal_norm_bwd(xq, xk, xv, xg, xdq, xdk, xdv, None, "elu1", w.eps, workspace=ws, stream=s_cmp)
+        elif gated:
+            la.la_gated_fwd(xq, xk, xv, ins[4], xo, stream=s_cmp)
+            la.la_gated_bwd(xq, xk, xv, ins[4], xg, xdq, xdk, xdv, outs[4], workspace=ws, stream=s_cmp)
         else:
             la.la_chunk_decay_fwd(xq, xk, xv, xo, gamma, workspace=ws, stream=s_cmp)
             la.la_chunk_decay_bwd(xq, xk, xv, xg, gamma, xdq, xdk, xdv, workspace=ws, stream=s_cmp)
         ev_cmp[si].record(s_cmp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_cmp[si])
-            for h_, d_ in zip(hout[si], (xo, xdq, xdk, xdv)):
+            for h_, d_ in zip(hout[si], outs):
                 h_.copy_(d_, non_blocking=True)
             ev_out[si].record(s_out)
 
@@ -502,7 +530,7 @@ def run_ours(args, w):
         e2e_ms = max_over_ranks(x0.elapsed_time(x1), dist, dev)
         tensor_bytes = B * H * T * D * q.element_size()
         e2e = {"value": aggregate_throughput(B * T * k_e2e, world, e2e_ms / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": 4 * tensor_bytes, "d2h_bytes_per_step": 4 * tensor_bytes,
+               "h2d_bytes_per_step": len(in_names) * tensor_bytes, "d2h_bytes_per_step": n_out * tensor_bytes,
                "steps": k_e2e, "note": "pinned host q, k, v, dO copied in and o, dq, dk, dv copied out every step "
                                        "through the C ABI; copies of neighbouring steps overlap the compute "
                                        "(three streams, two device buffer sets)"}
@@ -739,10 +767,12 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--T", type=int, default=None, help="sequence length (default: the workload's)")
-    ap.add_argument("--workload", choices=["bidir", "simple", "retention", "decode", "causal_norm"], default="bidir",
+    ap.add_argument("--workload", choices=["bidir", "simple", "retention", "decode", "causal_norm", "gated"],
+                    default="bidir",
                     help="bidir (the benchmark metric, B8 H16 D64 fp16), simple (B8 H16 D64 bf16), "
                          "retention (B8 H32 D128 bf16), decode (recurrent decay step, B64 H32 D128) or "
-                         "causal_norm (causal linear attention with the norm term, B8 H16 D64 fp16)")
+                         "causal_norm (causal linear attention with the norm term, B8 H16 D64 fp16) or "
+                         "gated (gated linear attention, B8 H16 D64 bf16)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seqpar", action="store_true",
                     help="bidir/simple: split the workload's sequence along T across the GPUs (one all-reduce of "
@@ -761,7 +791,7 @@ def main(argv=None):
             return run_decode_reference(args)
         return run_decode(args)
     base = {"bidir": "bidir_f16", "simple": "simple_bf16", "retention": "retention_bf16",
-            "causal_norm": "causal_norm_f16"}[args.workload]
+            "causal_norm": "causal_norm_f16", "gated": "gated_bf16"}[args.workload]
     w = synth.WORKLOADS[base]
     w = w.with_T(args.T if args.T is not None else (4096 if args.workload != "retention" else 8192))
     if args.impl == "reference":

@@ -76,7 +76,9 @@ typedef enum {
     LA_OP_STATE_BWD_Q = 8,
     LA_OP_STATE_BWD_KV = 9,
     LA_OP_CAUSAL_NORM_FWD = 10,
-    LA_OP_CAUSAL_NORM_BWD = 11
+    LA_OP_CAUSAL_NORM_BWD = 11,
+    LA_OP_GATED_FWD = 12,
+    LA_OP_GATED_BWD = 13
 } la_op;
 
 /* Feature map of the state-form stages and of la_causal_norm_*: elu+1 with the
@@ -263,6 +265,29 @@ la_status la_causal_norm_bwd(const void *q, const void *k, const void *v, const 
                              la_feature feature, float eps, void *dq, void *dk, void *dv,
                              int B, int H, int T, int D, la_dtype dtype,
                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---- gated linear attention ----------------------------------------------
+ * Causal linear attention whose decay is data dependent, per token and per key
+ * dimension (the GatedLinearAttention layer the "flash-linear-attention"
+ * README lists; its gates come from the model's projections, which stay the
+ * caller's):
+ *   S_t = diag(exp(g_t)) S_{t-1} + k_t^T v_t,  o_t = q_t S_t,
+ * g [B,H,T,D] the log gates (g <= 0 decays; dtype as q).  With g_t = log gamma_h
+ * for every t and dimension this is la_chunk_decay_*.  The recurrent form
+ * ("Different forms of linear attention": FusedRecurrent) on CUDA cores, fp32,
+ * one CTA per (b, h); every dtype, D in {64, 128}; no workspace. */
+la_status la_gated_fwd(const void *q, const void *k, const void *v, const void *g, void *o,
+                       int B, int H, int T, int D, la_dtype dtype, void *stream);
+
+/* Gradients of sum(o * dout): dq_t = S_t dout_t, and with
+ * R_t = q_t^T dout_t + diag(exp(g_{t+1})) R_{t+1}: dk_t = R_t v_t, dv_t = k_t R_t;
+ * dg_t = sum_{s>=t} (q_s dq_s - k_s dk_s) (elementwise, in fp32 from the unrounded
+ * dq and dk).  Workspace: la_workspace_size(LA_OP_GATED_BWD, ...) bytes (dq in
+ * fp32, 4 B per element). */
+la_status la_gated_bwd(const void *q, const void *k, const void *v, const void *g, const void *dout,
+                       void *dq, void *dk, void *dv, void *dg,
+                       int B, int H, int T, int D, la_dtype dtype,
+                       void *workspace, size_t workspace_bytes, void *stream);
 
 /* ---- feature maps formed by the caller ------------------------------------
  * Row-wise maps of [B,H,T,D] tensors, D in {32, 64, 128}, for the state-form

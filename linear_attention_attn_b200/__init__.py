@@ -28,7 +28,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 LA_F32, LA_F16, LA_BF16 = 0, 1, 2
 OPS = {"bidir_fwd": 0, "bidir_bwd": 1, "simple_fwd": 2, "simple_bwd": 3,
        "chunk_decay_fwd": 4, "chunk_decay_bwd": 5, "state_reduce": 6, "state_apply": 7,
-       "state_bwd_q": 8, "state_bwd_kv": 9, "causal_norm_fwd": 10, "causal_norm_bwd": 11}
+       "state_bwd_q": 8, "state_bwd_kv": 9, "causal_norm_fwd": 10, "causal_norm_bwd": 11, "gated_fwd": 12,
+       "gated_bwd": 13}
 FEATURES = {"identity": 0, "elu1": 1, "norm": 2}
 STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_ALIGNMENT",
           4: "LA_ERR_WORKSPACE", 5: "LA_ERR_CUDA", 6: "LA_ERR_TIMEOUT"}
@@ -57,6 +58,8 @@ _lib.la_chunk_decay_fwd_state.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I
 _lib.la_chunk_decay_bwd_state.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z,
                                           _P]
 _lib.la_chunk_decay_scan.argtypes = [_P, _P, _I, _P, _P, _I, _I, _I, _P]
+_lib.la_gated_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
+_lib.la_gated_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_feature_map_fwd.argtypes = [_I, _F, _P, _P, _I, _I, _I, _I, _I, _P]
 _lib.la_feature_map_bwd.argtypes = [_I, _F, _P, _P, _P, _I, _I, _I, _I, _I, _P]
 _lib.la_causal_norm_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _F, _I, _I, _I, _I, _I, _P]
@@ -68,7 +71,8 @@ _lib.la_state_bwd_kv.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]
 for _n in ("la_bidir_fwd", "la_simple_fwd", "la_bidir_bwd", "la_simple_bwd", "la_chunk_decay_fwd",
            "la_chunk_decay_bwd", "la_chunk_decay_step", "la_chunk_decay_fwd_state", "la_chunk_decay_bwd_state",
            "la_chunk_decay_scan", "la_state_reduce", "la_state_apply", "la_state_bwd_q", "la_state_bwd_kv",
-           "la_causal_norm_fwd", "la_causal_norm_bwd", "la_feature_map_fwd", "la_feature_map_bwd"):
+           "la_causal_norm_fwd", "la_causal_norm_bwd", "la_feature_map_fwd", "la_feature_map_bwd", "la_gated_fwd",
+           "la_gated_bwd"):
     getattr(_lib, _n).restype = _I
 _lib.la_bidir_fwd_static.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.la_bidir_fwd_static.restype = _I
@@ -309,6 +313,23 @@ def la_chunk_decay_scan(states, gaps, decay, out, stream=None):
 
 def _decay_or_null(decay, H):
     return (None, None) if decay is None else (lambda a: (ctypes.cast(a, _P), a))(_decay(decay, H))
+
+
+def la_gated_fwd(q, k, v, g, o, stream=None):
+    """Gated linear attention: S_t = diag(exp(g_t)) S_{t-1} + k_t^T v_t, o_t <- q_t S_t; g holds the
+    log gates, [B, H, T, D] like q."""
+    B, H, T, D = _shape(q, k, v, g, o)
+    _check(_lib.la_gated_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), B, H, T, D, _dtype_code(q),
+                             _stream(stream, q.device)), "la_gated_fwd")
+
+
+def la_gated_bwd(q, k, v, g, dout, dq, dk, dv, dg, workspace=None, stream=None):
+    """dq, dk, dv, dg <- gradients of sum(o * dout) for la_gated_fwd."""
+    B, H, T, D = _shape(q, k, v, g, dout, dq, dk, dv, dg)
+    dt = _dtype_code(q)
+    wp, wn, _keep = _workspace("gated_bwd", (B, H, T, D), dt, workspace, q.device, stream)
+    _check(_lib.la_gated_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+                             B, H, T, D, dt, wp, wn, _stream(stream, q.device)), "la_gated_bwd")
 
 
 FMAPS = {"focused": 0, "polarity": 1, "polarity_swap": 2}

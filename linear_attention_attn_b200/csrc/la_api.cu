@@ -273,7 +273,7 @@ size_t la_workspace_size(la_op op, int B, int H, int T, int D, la_dtype dtype) {
     const Shape s{B, H, T, D};
     if (s.B < 1 || s.H < 1 || s.T < 0 || (s.D != 64 && s.D != 128)) return 0;
     if (dtype != LA_F32 && dtype != LA_F16 && dtype != LA_BF16) return 0;
-    if ((int)op < 0 || (int)op > (int)LA_OP_CAUSAL_NORM_BWD) return 0;
+    if ((int)op < 0 || (int)op > (int)LA_OP_GATED_BWD) return 0;
     return ws_size(op, s, dtype);
 }
 
@@ -470,6 +470,38 @@ la_status la_feature_map_fwd(la_fmap kind, float p, const void *x, void *y, int 
 la_status la_feature_map_bwd(la_fmap kind, float p, const void *x, const void *dy, void *dx, int B, int H, int T,
                              int D, la_dtype dtype, void *stream) {
     return fmap_entry(true, kind, p, x, dy, dx, B, H, T, D, dtype, stream);
+}
+
+la_status la_gated_fwd(const void *q, const void *k, const void *v, const void *g, void *o, int B, int H, int T,
+                       int D, la_dtype dtype, void *stream) {
+    const Shape s{B, H, T, D};
+    LA_TRY(validate(s, dtype));
+    LA_TRY(check_ptr(q, "q"));
+    LA_TRY(check_ptr(k, "k"));
+    LA_TRY(check_ptr(v, "v"));
+    LA_TRY(check_ptr(g, "g"));
+    LA_TRY(check_ptr(o, "o"));
+    if (T == 0) return LA_OK;
+    return simt::gated_fwd(q, k, v, g, o, s, dtype, (cudaStream_t)stream);
+}
+
+la_status la_gated_bwd(const void *q, const void *k, const void *v, const void *g, const void *dout, void *dq,
+                       void *dk, void *dv, void *dg, int B, int H, int T, int D, la_dtype dtype, void *workspace,
+                       size_t workspace_bytes, void *stream) {
+    const Shape s{B, H, T, D};
+    LA_TRY(validate(s, dtype));
+    LA_TRY(check_ptr(q, "q"));
+    LA_TRY(check_ptr(k, "k"));
+    LA_TRY(check_ptr(v, "v"));
+    LA_TRY(check_ptr(g, "g"));
+    LA_TRY(check_ptr(dout, "dout"));
+    LA_TRY(check_ptr(dq, "dq"));
+    LA_TRY(check_ptr(dk, "dk"));
+    LA_TRY(check_ptr(dv, "dv"));
+    LA_TRY(check_ptr(dg, "dg"));
+    LA_TRY(check_ws(LA_OP_GATED_BWD, s, dtype, workspace, workspace_bytes));
+    if (T == 0) return LA_OK;
+    return simt::gated_bwd(q, k, v, g, dout, dq, dk, dv, dg, s, dtype, workspace, (cudaStream_t)stream);
 }
 
 la_status la_chunk_decay_scan(const float *states, const long long *gaps, int n, const float *decay, float *out,

@@ -159,6 +159,11 @@ la_status causal_norm_fwd(const void *q, const void *k, const void *v, void *o, 
 la_status causal_norm_bwd(const void *q, const void *k, const void *v, const void *g, void *dq, void *dk, void *dv,
                           const DecayArgs &dec, int has_decay, bool phi, const Shape &s, la_dtype dt, float eps,
                           void *ws, cudaStream_t st);
+// Gated linear attention (log gates g, the decay exp(g) per token and key dimension).
+la_status gated_fwd(const void *q, const void *k, const void *v, const void *g, void *o, const Shape &s, la_dtype dt,
+                    cudaStream_t st);
+la_status gated_bwd(const void *q, const void *k, const void *v, const void *g, const void *dout, void *dq, void *dk,
+                    void *dv, void *dg, const Shape &s, la_dtype dt, void *ws, cudaStream_t st);
 }  // namespace simt
 
 }  // namespace la

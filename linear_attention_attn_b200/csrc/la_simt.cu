@@ -700,6 +700,181 @@ constexpr size_t causal_bwd_kv_smem() {
     return (size_t)(6 * kRetTile * D) * sizeof(float) + kRetTile * sizeof(float2);
 }
 
+// ------------------------------------------------------ gated linear attention ---
+// Per-token, per-key-dimension decay, the recurrent form:
+//   S_t = diag(a_t) S_{t-1} + k_t^T v_t,  o_t = q_t S_t,  a_t = exp(g_t), g the log gates.
+// The state lines are split over P threads as in the causal-norm kernels.
+
+// exp of a gate tile in place (rows past the sequence are never read)
+template <int D>
+__device__ __forceinline__ void exp_tile(float (*tile)[D]) {
+    for (int e = threadIdx.x; e < kRetTile * D; e += blockDim.x) tile[e / D][e % D] = expf(tile[e / D][e % D]);
+}
+template <int D> constexpr int gated_fwd_threads() { return causal_split<D>() * D; }
+template <int D> constexpr int gated_kv_threads() { return 2 * causal_split<D>() * D; }
+
+// Forward: the D columns of S; thread p of column j holds S[i][j] for its D / P rows i.
+template <typename T, int D>
+__global__ void __launch_bounds__(gated_fwd_threads<D>())
+gated_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
+          T *__restrict__ o, int T_len) {
+    constexpr int P = causal_split<D>(), DP = D / P;
+    __shared__ float tiles[4][kRetTile][D];      // q, k, v, a = exp(g)
+    __shared__ float acc[kRetTile][D];
+    const long long base = (long long)blockIdx.x * T_len * D;
+    const int j = threadIdx.x / P, i0 = (threadIdx.x % P) * DP;
+    const bool lead = threadIdx.x % P == 0;
+    float S[DP];
+#pragma unroll
+    for (int i = 0; i < DP; ++i) S[i] = 0.f;
+    const T *const src[4] = {q, k, v, g};
+    for (int ts = 0; ts < T_len; ts += kRetTile) {
+        __syncthreads();
+        load_rows<T, D, 4>(src, tiles, base, ts, T_len, blockDim.x);
+        __syncthreads();
+        exp_tile<D>(tiles[3]);
+        __syncthreads();
+        const int nr = min(kRetTile, T_len - ts);
+        for (int r = 0; r < nr; ++r) {
+            const float vj = tiles[2][r][j];
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < DP; ++i) {
+                S[i] = fmaf(tiles[3][r][i0 + i], S[i], tiles[1][r][i0 + i] * vj);
+                a[i & 3] = fmaf(tiles[0][r][i0 + i], S[i], a[i & 3]);
+            }
+            const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
+            if (lead) acc[r][j] = s;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < nr * D; e += blockDim.x)
+            io<T>::st(o + base + (long long)(ts + e / D) * D + e % D, acc[e / D][e % D]);
+    }
+}
+
+// Backward, forward sweep: dq_t[i] = sum_j S_t[i][j] dout_t[j]; thread p of row i holds
+// S[i][j] for its D / P columns j.
+template <typename T, int D>
+__global__ void __launch_bounds__(gated_fwd_threads<D>())
+gated_bwd_q(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g, const T *__restrict__ dout,
+            T *__restrict__ dq, float *__restrict__ dq32, int T_len) {
+    constexpr int P = causal_split<D>(), DP = D / P;
+    __shared__ float tiles[4][kRetTile][D];      // k, v, a = exp(g), dout
+    __shared__ float acc[kRetTile][D];
+    const long long base = (long long)blockIdx.x * T_len * D;
+    const int i = threadIdx.x / P, j0 = (threadIdx.x % P) * DP;
+    const bool lead = threadIdx.x % P == 0;
+    float S[DP];
+#pragma unroll
+    for (int jj = 0; jj < DP; ++jj) S[jj] = 0.f;
+    const T *const src[4] = {k, v, g, dout};
+    for (int ts = 0; ts < T_len; ts += kRetTile) {
+        __syncthreads();
+        load_rows<T, D, 4>(src, tiles, base, ts, T_len, blockDim.x);
+        __syncthreads();
+        exp_tile<D>(tiles[2]);
+        __syncthreads();
+        const int nr = min(kRetTile, T_len - ts);
+        for (int r = 0; r < nr; ++r) {
+            const float ai = tiles[2][r][i], ki = tiles[0][r][i];
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int jj = 0; jj < DP; ++jj) {
+                S[jj] = fmaf(ai, S[jj], ki * tiles[1][r][j0 + jj]);
+                a[jj & 3] = fmaf(S[jj], tiles[3][r][j0 + jj], a[jj & 3]);
+            }
+            const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
+            if (lead) acc[r][i] = s;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < nr * D; e += blockDim.x) {
+            const long long at = base + (long long)(ts + e / D) * D + e % D;
+            io<T>::st(dq + at, acc[e / D][e % D]);
+            dq32[at] = acc[e / D][e % D];            // unrounded, for the log gates' gradient
+        }
+    }
+}
+
+// Backward, reverse sweep over R_t = q_t^T dout_t + diag(a_{t+1}) R_{t+1} (R_T = 0): the
+// first P D threads hold the rows of R (dk_t[i] = sum_j R[i][j] v_t[j]), the next P D its
+// columns (dv_t[j] = sum_i k_t[i] R[i][j]).  a_{t+1} of a tile's last row is the first row
+// of the tile after it (kept in `anext`).  The log gates' gradient comes out of the same
+// reverse walk: with G_t = sum_{s<=t} g_s, o_t = sum_{s<=t} (q_t e^{G_t}) . (k_s e^{-G_s}) v_s, so
+// dL/dG_t = q_t dq_t - k_t dk_t and dg_t = sum_{s>=t} (q_s dq_s - k_s dk_s), summed by thread i
+// of each key dimension in fp32 from the unrounded dq (dq32) and dk.
+template <typename T, int D>
+__global__ void __launch_bounds__(gated_kv_threads<D>())
+gated_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
+             const T *__restrict__ dout, const float *__restrict__ dq32, T *__restrict__ dk, T *__restrict__ dv,
+             T *__restrict__ dg, int T_len) {
+    constexpr int P = causal_split<D>(), DP = D / P;
+    extern __shared__ float dsm[];               // gated_bwd_kv_smem<D>() bytes
+    float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // q, k, v, dout, a = exp(g)
+    float(*res)[kRetTile][D] = tiles + 5;        // dk (rows), dv (columns)
+    float *anext = dsm + 7 * kRetTile * D;       // a of the row after the tile (0 past the sequence)
+    const long long base = (long long)blockIdx.x * T_len * D;
+    const bool row_side = threadIdx.x < P * D;
+    const int t2 = row_side ? threadIdx.x : threadIdx.x - P * D;
+    const int line = t2 / P, x0 = (t2 % P) * DP;
+    const bool lead = t2 % P == 0;
+    float Rx[DP];
+    float accg = 0.f;                            // thread i < D: sum over the rows after t of dL/dG[i]
+#pragma unroll
+    for (int m = 0; m < DP; ++m) Rx[m] = 0.f;
+    for (int e = threadIdx.x; e < D; e += blockDim.x) anext[e] = 0.f;
+    const T *const src[5] = {q, k, v, dout, g};
+    const int ntiles = (T_len + kRetTile - 1) / kRetTile;
+    for (int tile = ntiles - 1; tile >= 0; --tile) {
+        const int ts = tile * kRetTile;
+        __syncthreads();
+        load_rows<T, D, 5>(src, tiles, base, ts, T_len, blockDim.x);
+        __syncthreads();
+        exp_tile<D>(tiles[4]);
+        __syncthreads();
+        const int nr = min(kRetTile, T_len - ts);
+        for (int r = nr - 1; r >= 0; --r) {
+            const float *an = r + 1 < nr ? tiles[4][r + 1] : anext;    // a_{t+1}
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
+            if (row_side) {
+                const float qi = tiles[0][r][line], ai = an[line];
+#pragma unroll
+                for (int jj = 0; jj < DP; ++jj) {
+                    Rx[jj] = fmaf(ai, Rx[jj], qi * tiles[3][r][x0 + jj]);
+                    a[jj & 3] = fmaf(Rx[jj], tiles[2][r][x0 + jj], a[jj & 3]);
+                }
+            } else {
+                const float gj = tiles[3][r][line];
+#pragma unroll
+                for (int i = 0; i < DP; ++i) {
+                    Rx[i] = fmaf(an[x0 + i], Rx[i], tiles[0][r][x0 + i] * gj);
+                    a[i & 3] = fmaf(tiles[1][r][x0 + i], Rx[i], a[i & 3]);
+                }
+            }
+            const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
+            if (lead) res[row_side ? 0 : 1][r][line] = s;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < nr * D; e += blockDim.x) {
+            const long long at = base + (long long)(ts + e / D) * D + e % D;
+            io<T>::st(dk + at, res[0][e / D][e % D]);
+            io<T>::st(dv + at, res[1][e / D][e % D]);
+        }
+        if (threadIdx.x < D) {
+            const int i = threadIdx.x;
+            for (int r = nr - 1; r >= 0; --r) {
+                const long long at = base + (long long)(ts + r) * D + i;
+                accg = fmaf(tiles[0][r][i], dq32[at], accg);
+                accg = fmaf(-tiles[1][r][i], res[0][r][i], accg);
+                io<T>::st(dg + at, accg);
+            }
+        }
+        for (int e = threadIdx.x; e < D; e += blockDim.x) anext[e] = tiles[4][0][e];
+    }
+}
+
+template <int D>
+constexpr size_t gated_bwd_kv_smem() { return (size_t)(7 * kRetTile * D + D) * sizeof(float); }
+
 // -------------------------------------------------------------- drivers ---
 
 namespace {
@@ -874,6 +1049,8 @@ size_t workspace_size(la_op op, const Shape &s) {
         return state_bytes(s, simt_splits(s));
     case LA_OP_CAUSAL_NORM_BWD:   // (n_t, dn_t) of every row
         return ((size_t)s.BH() * s.T * sizeof(float2) + 255) / 256 * 256;
+    case LA_OP_GATED_BWD:         // dq in fp32, for the log gates' gradient
+        return ((size_t)s.BH() * s.T * s.D * sizeof(float) + 255) / 256 * 256;
     default:
         return 0;
     }
@@ -987,6 +1164,48 @@ la_status causal_norm_bwd(const void *q, const void *k, const void *v, const voi
     LA_CAUSAL_DISPATCH(causal_bwd_t, q, k, v, g, dq, dk, dv, dec, has_decay, s, eps, ws, st);
 }
 #undef LA_CAUSAL_DISPATCH
+
+namespace {
+
+template <typename T, int D>
+la_status gated_fwd_t(const void *q, const void *k, const void *v, const void *g, void *o, const Shape &s,
+                      cudaStream_t st) {
+    return launch("simt_gated_fwd", gated_fwd<T, D>, dim3((unsigned)s.BH()), dim3(gated_fwd_threads<D>()), 0, st,
+                  (const T *)q, (const T *)k, (const T *)v, (const T *)g, (T *)o, s.T);
+}
+
+template <typename T, int D>
+la_status gated_bwd_t(const void *q, const void *k, const void *v, const void *g, const void *dout, void *dq,
+                      void *dk, void *dv, void *dg, const Shape &s, void *ws, cudaStream_t st) {
+    const dim3 grid((unsigned)s.BH());
+    float *dq32 = (float *)ws;
+    la_status rc = launch("simt_gated_bwd_q", gated_bwd_q<T, D>, grid, dim3(gated_fwd_threads<D>()), 0, st,
+                          (const T *)k, (const T *)v, (const T *)g, (const T *)dout, (T *)dq, dq32, s.T);
+    if (rc) return rc;
+    return launch("simt_gated_bwd_kv", gated_bwd_kv<T, D>, grid, dim3(gated_kv_threads<D>()), gated_bwd_kv_smem<D>(),
+                  st, (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const T *)dout, (const float *)dq32,
+                  (T *)dk, (T *)dv, (T *)dg, s.T);
+}
+
+#define LA_GATED_DISPATCH(F, ...)                                                     \
+    do {                                                                              \
+        if (dt == LA_F32) return s.D == 64 ? F<float, 64>(__VA_ARGS__) : F<float, 128>(__VA_ARGS__); \
+        if (dt == LA_F16) return s.D == 64 ? F<__half, 64>(__VA_ARGS__) : F<__half, 128>(__VA_ARGS__); \
+        return s.D == 64 ? F<__nv_bfloat16, 64>(__VA_ARGS__) : F<__nv_bfloat16, 128>(__VA_ARGS__); \
+    } while (0)
+
+}  // namespace
+
+la_status gated_fwd(const void *q, const void *k, const void *v, const void *g, void *o, const Shape &s, la_dtype dt,
+                    cudaStream_t st) {
+    LA_GATED_DISPATCH(gated_fwd_t, q, k, v, g, o, s, st);
+}
+
+la_status gated_bwd(const void *q, const void *k, const void *v, const void *g, const void *dout, void *dq, void *dk,
+                    void *dv, void *dg, const Shape &s, la_dtype dt, void *ws, cudaStream_t st) {
+    LA_GATED_DISPATCH(gated_bwd_t, q, k, v, g, dout, dq, dk, dv, dg, s, ws, st);
+}
+#undef LA_GATED_DISPATCH
 
 }  // namespace simt
 }  // namespace la

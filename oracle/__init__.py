@@ -66,13 +66,15 @@ def _bind(lib):
     lib.oracle_normed_fwd.argtypes = [P, P, P, P, P, L, L, L, L, Dbl, I]
     lib.oracle_normed_bwd.argtypes = [P, P, P, P, P, P, P, L, L, L, L, Dbl, I]
     lib.oracle_feature_map_fwd.argtypes = [I, Dbl, P, P, L, L]
+    lib.oracle_gated_fwd.argtypes = [P, P, P, P, P, L, L, L, L, I]
+    lib.oracle_gated_bwd.argtypes = [P, P, P, P, P, P, P, P, P, L, L, L, L, I]
     lib.oracle_feature_map_bwd.argtypes = [I, Dbl, P, P, P, L, L]
     lib.oracle_causal_norm_bwd.argtypes = [P, P, P, P, P, I, Dbl, P, P, P, L, L, L, L, I]
     for name in ("oracle_bidir_fwd", "oracle_simple_fwd", "oracle_bidir_bwd",
                  "oracle_simple_bwd", "oracle_retention_fwd", "oracle_retention_bwd",
                  "oracle_retention_step", "oracle_retention_fwd_state", "oracle_retention_bwd_state",
                  "oracle_causal_norm_fwd", "oracle_causal_norm_bwd", "oracle_normed_fwd", "oracle_normed_bwd",
-                 "oracle_feature_map_fwd", "oracle_feature_map_bwd"):
+                 "oracle_feature_map_fwd", "oracle_feature_map_bwd", "oracle_gated_fwd", "oracle_gated_bwd"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -253,6 +255,25 @@ class Oracle:
         _check(rc, "oracle_normed_bwd")
         return dq, dk, dv
 
+    def gated_fwd(self, q, k, v, lg, nthreads: int | None = None):
+        """Gated linear attention: S_t = diag(exp(lg_t)) S_{t-1} + k_t^T v_t, o_t = q_t S_t."""
+        q, k, v, lg = _f64(q), _f64(k), _f64(v), _f64(lg)
+        B, H, T, D = _shape4(q)
+        o = np.empty_like(q)
+        rc = self._lib.oracle_gated_fwd(_p(q), _p(k), _p(v), _p(lg), _p(o), B, H, T, D, nthreads or default_threads())
+        _check(rc, "oracle_gated_fwd")
+        return o
+
+    def gated_bwd(self, q, k, v, lg, dout, nthreads: int | None = None):
+        """Gradients (dq, dk, dv, dlg) of sum(o * dout) for gated_fwd."""
+        q, k, v, lg, g = _f64(q), _f64(k), _f64(v), _f64(lg), _f64(dout)
+        B, H, T, D = _shape4(q)
+        dq, dk, dv, dg = (np.empty_like(q) for _ in range(4))
+        rc = self._lib.oracle_gated_bwd(_p(q), _p(k), _p(v), _p(lg), _p(g), _p(dq), _p(dk), _p(dv), _p(dg),
+                                        B, H, T, D, nthreads or default_threads())
+        _check(rc, "oracle_gated_bwd")
+        return dq, dk, dv, dg
+
     FMAPS = {"focused": 0, "polarity": 1, "polarity_swap": 2}
 
     def feature_map_fwd(self, kind, x, p: float = 1.0):
@@ -401,3 +422,11 @@ def feature_map_fwd(*a, **kw):
 
 def feature_map_bwd(*a, **kw):
     return _instance().feature_map_bwd(*a, **kw)
+
+
+def gated_fwd(*a, **kw):
+    return _instance().gated_fwd(*a, **kw)
+
+
+def gated_bwd(*a, **kw):
+    return _instance().gated_bwd(*a, **kw)

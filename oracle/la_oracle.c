@@ -26,6 +26,8 @@
  *            o_t = sum_{s<=t} gamma^(t-s) (q_t . k_s) v_s
  *            computed in the recurrent ("FusedRecurrent") form
  *            S_t = gamma S_{t-1} + k_t^T v_t,  o_t = q_t S_t.
+ *   gated (data-dependent decay per token and key dimension, g_t <= 0 the log gates):
+ *            S_t = diag(exp(g_t)) S_{t-1} + k_t^T v_t,  o_t = q_t S_t.
  *   causal with the norm term (plain causal linear attention at gamma = 1):
  *            S_t = gamma S_{t-1} + f(k_t)^T v_t,  z_t = gamma z_{t-1} + f(k_t)
  *            o_t = f(q_t) S_t / (f(q_t) . z_t + eps),  f = phi or the identity.
@@ -641,5 +643,94 @@ int oracle_feature_map_bwd(int kind, double p, const double *x, const double *dy
     const long w = fmap_width(kind, D);
     for (long r = 0; r < rows; ++r) fmap_row_bwd(kind, p, x + r * D, dy + r * w, dx + r * D, D);
     return 0;
+}
+
+/* ------------------------------------------ gated linear attention (recurrent) -- */
+
+/* Forward, one head: S_t[i][j] = exp(g_t[i]) S_{t-1}[i][j] + k_t[i] v_t[j], o_t = q_t S_t. */
+static void gated_fwd_head(job_t *jb, long bh, double *scratch) {
+    const long T = jb->T, D = jb->D;
+    const long off = bh * T * D;
+    const double *q = jb->q + off, *k = jb->k + off, *v = jb->v + off, *lg = jb->state_in + off;
+    double *o = jb->o + off;
+    double *S = scratch;
+    memset(S, 0, (size_t)(D * D) * sizeof(double));
+    for (long t = 0; t < T; ++t) {
+        for (long i = 0; i < D; ++i) {
+            const double a = exp(lg[t * D + i]);
+            for (long j = 0; j < D; ++j) S[i * D + j] = a * S[i * D + j] + k[t * D + i] * v[t * D + j];
+        }
+        for (long j = 0; j < D; ++j) {
+            double u = 0.0;
+            for (long i = 0; i < D; ++i) u += q[t * D + i] * S[i * D + j];
+            o[t * D + j] = u;
+        }
+    }
+}
+
+/* Backward, one head.
+ *   dq_t[i] = sum_j S_t[i][j] dout_t[j]                                   (forward sweep)
+ *   R_t = q_t^T dout_t + diag(exp(g_{t+1})) R_{t+1}  (R_T = 0)            (reverse sweep)
+ *   dk_t[i] = sum_j R_t[i][j] v_t[j],   dv_t[j] = sum_i k_t[i] R_t[i][j]
+ * and the log gates: with G_t = sum_{s<=t} g_s, o_t = sum_{s<=t} (q_t e^{G_t}) . (k_s e^{-G_s}) v_s,
+ * so dL/dG_t = q_t dq_t - k_t dk_t (elementwise) and dg_t = sum_{s>=t} (q_s dq_s - k_s dk_s). */
+static void gated_bwd_head(job_t *jb, long bh, double *scratch) {
+    const long T = jb->T, D = jb->D;
+    const long off = bh * T * D;
+    const double *q = jb->q + off, *k = jb->k + off, *v = jb->v + off, *g = jb->g + off, *lg = jb->state_in + off;
+    double *dq = jb->dq + off, *dk = jb->dk + off, *dv = jb->dv + off, *dg = jb->state_out + off;
+    double *S = scratch, *R = S + D * D, *acc = R + D * D;
+    memset(S, 0, (size_t)(2 * D * D + D) * sizeof(double));
+    for (long t = 0; t < T; ++t) {
+        for (long i = 0; i < D; ++i) {
+            const double a = exp(lg[t * D + i]);
+            for (long j = 0; j < D; ++j) S[i * D + j] = a * S[i * D + j] + k[t * D + i] * v[t * D + j];
+        }
+        for (long i = 0; i < D; ++i) {
+            double a = 0.0;
+            for (long j = 0; j < D; ++j) a += S[i * D + j] * g[t * D + j];
+            dq[t * D + i] = a;
+        }
+    }
+    for (long t = T - 1; t >= 0; --t) {
+        for (long i = 0; i < D; ++i) {
+            const double a = t + 1 < T ? exp(lg[(t + 1) * D + i]) : 0.0;
+            for (long j = 0; j < D; ++j) R[i * D + j] = a * R[i * D + j] + q[t * D + i] * g[t * D + j];
+        }
+        for (long i = 0; i < D; ++i) {
+            double a = 0.0;
+            for (long j = 0; j < D; ++j) a += R[i * D + j] * v[t * D + j];
+            dk[t * D + i] = a;
+        }
+        for (long j = 0; j < D; ++j) {
+            double a = 0.0;
+            for (long i = 0; i < D; ++i) a += k[t * D + i] * R[i * D + j];
+            dv[t * D + j] = a;
+        }
+    }
+    for (long t = T - 1; t >= 0; --t)
+        for (long i = 0; i < D; ++i) {
+            acc[i] += q[t * D + i] * dq[t * D + i] - k[t * D + i] * dk[t * D + i];
+            dg[t * D + i] = acc[i];
+        }
+}
+
+/* lg: [B, H, T, D] log gates (<= 0 for a decay); dg: their gradient. */
+int oracle_gated_fwd(const double *q, const double *k, const double *v, const double *lg, double *o,
+                     long B, long H, long T, long D, int nthreads) {
+    if (check_dims(B, H, T, D) || (T > 0 && (!q || !k || !v || !lg || !o))) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.state_in = lg; jb.o = o;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D;
+    return for_each_head(&jb, gated_fwd_head, (size_t)(D * D), nthreads);
+}
+
+int oracle_gated_bwd(const double *q, const double *k, const double *v, const double *lg, const double *dout,
+                     double *dq, double *dk, double *dv, double *dg, long B, long H, long T, long D, int nthreads) {
+    if (check_dims(B, H, T, D) || (T > 0 && (!q || !k || !v || !lg || !dout || !dq || !dk || !dv || !dg))) return -1;
+    job_t jb; memset(&jb, 0, sizeof jb);
+    jb.q = q; jb.k = k; jb.v = v; jb.state_in = lg; jb.g = dout; jb.dq = dq; jb.dk = dk; jb.dv = dv; jb.state_out = dg;
+    jb.B = B; jb.H = H; jb.T = T; jb.D = D;
+    return for_each_head(&jb, gated_bwd_head, (size_t)(2 * D * D + D), nthreads);
 }
 

@@ -25,7 +25,7 @@ DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 class Workload:
     """One named synthetic workload (shapes, dtype and the input recipe)."""
     name: str
-    op: str                      # "bidir" | "simple" | "retention" | "causal_norm"
+    op: str                      # "bidir" | "simple" | "retention" | "causal_norm" | "gated"
     B: int
     H: int
     T: int
@@ -65,6 +65,9 @@ WORKLOADS = {
     # causal linear attention with the norm term (phi = elu+1, no decay), the bidir recipe and shape
     "causal_norm_f16": Workload("causal_norm_f16", "causal_norm", 8, 16, 4096, 64, "f16",
                                 q_scale=0.5, k_scale=0.5, v_scale=0.5),
+    # gated linear attention, bf16: q scaled by D^-1/2, log gates log(sigmoid(N(0,1))) / 16 per token
+    # and key dimension (about -0.04: decays near 0.96)
+    "gated_bf16": Workload("gated_bf16", "gated", 8, 16, 4096, 64, "bf16", q_scale=64 ** -0.5),
     # vision-style long sequence, forward only, 256x256 token grid
     "vision_f16": Workload("vision_f16", "bidir", 2, 10, 65536, 64, "f16",
                            q_scale=0.5, k_scale=0.5, v_scale=0.5, vision_offset=True, bwd=False),
@@ -124,4 +127,6 @@ def make_inputs(w: Workload, seed: int = 0, with_grad: bool | None = None) -> di
         out[n] = x.to(dt).contiguous()
     if w.op == "retention":
         out["gamma"] = retention_gammas(w.H)
+    if w.op == "gated":
+        out["g"] = (torch.nn.functional.logsigmoid(normal(shape, seed, 4)) / 16.0).to(dt).contiguous()
     return out

@@ -520,6 +520,43 @@ def check_normed(orc):
         _close(a, b, rtol=1e-6, atol=1e-7, what="normed %s vs finite differences" % name)
 
 
+def brute_gated(q, k, v, lg):
+    """Pairwise form: o_t = sum_{s<=t} sum_i q_t[i] k_s[i] exp(sum_{s<r<=t} lg_r[i]) v_s."""
+    B, H, T, D = q.shape
+    G = np.cumsum(lg, axis=2)                                   # G_t = sum_{r<=t} lg_r
+    o = np.zeros_like(v, dtype=np.float64)
+    for t in range(T):
+        w = np.exp(G[:, :, t:t + 1, :] - G[:, :, :t + 1, :])     # [B, H, t+1, D]
+        a = np.einsum("bhi,bhsi->bhs", q[:, :, t], k[:, :, :t + 1] * w)
+        o[:, :, t] = np.einsum("bhs,bhsj->bhj", a, v[:, :, :t + 1])
+    return o
+
+
+def check_gated(orc):
+    """Gated linear attention: the pairwise form; constant gates log gamma_h give retention; zero
+    gates the causal prefix sums; finite differences of dq, dk, dv and of the log gates."""
+    B, H, T, D = 2, 3, 8, 4
+    q, k, v = _rand((B, H, T, D), 111), _rand((B, H, T, D), 112), _rand((B, H, T, D), 113)
+    lg = -np.abs(_rand((B, H, T, D), 114)) * 0.4
+    _close(orc.gated_fwd(q, k, v, lg), brute_gated(q, k, v, lg), rtol=1e-12, atol=1e-13, what="gated vs pairwise")
+    gam = np.array([0.5, 0.9, 1.0])
+    lgc = np.broadcast_to(np.log(gam)[None, :, None, None], q.shape).copy()
+    _close(orc.gated_fwd(q, k, v, lgc), orc.retention_fwd(q, k, v, gam), rtol=1e-12, atol=1e-13,
+           what="constant gates = retention")
+    a = np.tril(np.einsum("bhti,bhsi->bhts", q, k))
+    _close(orc.gated_fwd(q, k, v, np.zeros_like(q)), np.einsum("bhts,bhsj->bhtj", a, v), rtol=1e-12, atol=1e-13,
+           what="zero gates = causal prefix sums")
+    Bs, Hs, Ts, Ds = 1, 2, 5, 3
+    qs, ks, vs, gs = (_rand((Bs, Hs, Ts, Ds), 115 + i) for i in range(4))
+    ls = -np.abs(_rand((Bs, Hs, Ts, Ds), 119)) * 0.5
+    got = orc.gated_bwd(qs, ks, vs, ls, gs)
+    fd = _fd_grads(lambda x, y, z: orc.gated_fwd(x, y, z, ls), qs, ks, vs, gs)
+    for name, a, b in zip(("dq", "dk", "dv"), got[:3], fd):
+        _close(a, b, rtol=1e-6, atol=1e-7, what="gated %s vs finite differences" % name)
+    fdg = _fd_rows(lambda x: orc.gated_fwd(qs, ks, vs, x), ls, gs)
+    _close(got[3], fdg, rtol=1e-6, atol=1e-7, what="gated dlog-gate vs finite differences")
+
+
 ALL_CHECKS = (check_golden, check_brute, check_closed_forms, check_invariances,
               check_fd_gradients, check_autograd, check_decode_step, check_state_segments,
-              check_segment_backward, check_causal_norm, check_feature_maps, check_normed)
+              check_segment_backward, check_causal_norm, check_feature_maps, check_normed, check_gated)

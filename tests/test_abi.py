@@ -27,7 +27,8 @@ def test_header_declares_the_api():
     names = declared_functions()
     for n in ("la_bidir_fwd", "la_bidir_bwd", "la_simple_fwd", "la_simple_bwd", "la_chunk_decay_fwd",
               "la_chunk_decay_bwd", "la_chunk_decay_step", "la_chunk_decay_fwd_state", "la_chunk_decay_bwd_state",
-              "la_chunk_decay_scan", "la_causal_norm_fwd", "la_causal_norm_bwd",
+              "la_chunk_decay_scan", "la_causal_norm_fwd", "la_causal_norm_bwd", "la_gated_fwd", "la_gated_bwd",
+              "la_feature_map_fwd", "la_feature_map_bwd",
               "la_workspace_size", "la_status_string", "la_last_error"):
         assert n in names
 

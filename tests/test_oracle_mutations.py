@@ -58,6 +58,14 @@ MUTATIONS = [
      "const double dneg = x[i] < 0.0 ? p * pow(-x[i], p - 1.0) : 0.0;", 0),
     ("normed_uses_phi", "jb.eps = eps; jb.use_phi = 0; jb.use_norm = 1;\n    return for_each_head(&jb, state_fwd_head",
      "jb.eps = eps; jb.use_phi = 1; jb.use_norm = 1;\n    return for_each_head(&jb, state_fwd_head", 0),
+    ("gated_reverse_gate_of_t", "const double a = t + 1 < T ? exp(lg[(t + 1) * D + i]) : 0.0;",
+     "const double a = t + 1 < T ? exp(lg[t * D + i]) : 0.0;", 0),
+    ("gated_dg_forward_cumsum", "    for (long t = T - 1; t >= 0; --t)\n        for (long i = 0; i < D; ++i) {\n            acc[i] +=",
+     "    for (long t = 0; t < T; ++t)\n        for (long i = 0; i < D; ++i) {\n            acc[i] +=", 0),
+    ("gated_dg_k_sign", "acc[i] += q[t * D + i] * dq[t * D + i] - k[t * D + i] * dk[t * D + i];",
+     "acc[i] += q[t * D + i] * dq[t * D + i] + k[t * D + i] * dk[t * D + i];", 0),
+    ("gated_fwd_gate_not_exp", "            const double a = exp(lg[t * D + i]);\n            for (long j = 0; j < D; ++j) S[i * D + j] = a * S[i * D + j] + k[t * D + i] * v[t * D + j];\n        }\n        for (long j = 0; j < D; ++j) {\n            double u",
+     "            const double a = 1.0 + lg[t * D + i];\n            for (long j = 0; j < D; ++j) S[i * D + j] = a * S[i * D + j] + k[t * D + i] * v[t * D + j];\n        }\n        for (long j = 0; j < D; ++j) {\n            double u", 0),
     ("fwd_state_out_before_last_token", "    if (jb->state_out) memcpy(jb->state_out + bh * D * D, S,",
      "    if (jb->state_out) memcpy(jb->state_out + bh * D * D, jb->state_in ? jb->state_in + bh * D * D : S,", 0),
 ]
