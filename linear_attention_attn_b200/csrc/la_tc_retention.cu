@@ -90,7 +90,7 @@ __device__ __forceinline__ void st16_wide(uint8_t *t, int box_bytes, int row, in
 
 // Warp roles: 0 TMA, 1 UMMA, 2..5 decay mask, 6..9 output, 10..17 state and K^
 // (two warps per TMEM lane quadrant, 64 state columns each).
-constexpr int kRXw0 = 2, kRXWarps = 4, kROw0 = 6, kROWarps = 4, kRSw0 = 10, kRSWarps = 8;
+constexpr int kRXWarps = 4, kROw0 = 6, kROWarps = 4, kRSw0 = 10, kRSWarps = 8;   // mask warps 2..5
 constexpr int kRThreads = (kRSw0 + kRSWarps) * 32;
 
 struct RetLayout {
