@@ -102,6 +102,20 @@ def max_over_ranks(value: float, dist, device=None) -> float:
     return float(t.item())
 
 
+def auto_steps(step, stream, dev, dist, target_s: float = 1.5, least: int = 200, most: int = 200000) -> int:
+    """Number of timed steps for a timed region of about target_s seconds (at least `least`), so
+    that the clock sampler sees the GPU under load; every rank takes the same count."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = 10
+    e0.record(stream)
+    for i in range(n):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    per = max_over_ranks(e0.elapsed_time(e1) / n / 1e3, dist, dev)
+    return int(min(most, max(least, math.ceil(target_s / max(per, 1e-7)))))
+
+
 def aggregate_throughput(units_per_rank: float, world: int, seconds: float) -> float:
     """Whole-job throughput: units processed by all ranks / the slowest rank's time."""
     return units_per_rank * world / seconds
@@ -172,6 +186,13 @@ class ClockSampler:
                                          stdout=self.out, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        # the timed region starts only once nvidia-smi is writing samples (bounded wait)
+        t0 = time.time()
+        while time.time() - t0 < 5.0 and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.01)
 
     def stop(self):
         if self.proc is None:
@@ -409,6 +430,8 @@ def run_ours(args, w):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
+    if args.steps is None:
+        args.steps = 200 if args.profile_only else auto_steps(lambda i: step(), stream, dev, dist)
     if args.profile_only:
         for _ in range(args.steps):
             step()
@@ -680,6 +703,8 @@ def run_decode(args):
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize(dev)
+    if args.steps is None:
+        args.steps = auto_steps(step, stream, dev, dist)
     if dist is not None:
         dist.barrier()
     sampler = ClockSampler(gpu_selector(dev))
@@ -764,7 +789,9 @@ def run_decode(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: enough for a timed region of about 1.5 s, at least 200; "
+                         "the oracle arm: 200)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--T", type=int, default=None, help="sequence length (default: the workload's)")
     ap.add_argument("--workload", choices=["bidir", "simple", "retention", "decode", "causal_norm", "gated"],
@@ -788,6 +815,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.workload == "decode":
         if args.impl == "reference":
+            if args.steps is None:
+                args.steps = 200
             return run_decode_reference(args)
         return run_decode(args)
     base = {"bidir": "bidir_f16", "simple": "simple_bf16", "retention": "retention_bf16",
@@ -795,6 +824,8 @@ def main(argv=None):
     w = synth.WORKLOADS[base]
     w = w.with_T(args.T if args.T is not None else (4096 if args.workload != "retention" else 8192))
     if args.impl == "reference":
+        if args.steps is None:
+            args.steps = 200
         return run_reference(args, w)
     return run_ours(args, w)
 
