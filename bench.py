@@ -418,7 +418,7 @@ def run_ours(args, w):
             la.la_simple_fwd(q, k, v, o, state, workspace=ws)
             la.la_simple_bwd(q, k, v, g, dq, dk, dv, state, workspace=ws)
         elif w.op == "causal_norm":
-            la.la_causal_norm_fwd(q, k, v, o, None, "elu1", w.eps)
+            la.la_causal_norm_fwd(q, k, v, o, None, "elu1", w.eps, workspace=ws)
             la.la_causal_norm_bwd(q, k, v, g, dq, dk, dv, None, "elu1", w.eps, workspace=ws)
         elif gated:
             la.la_gated_fwd(q, k, v, lgate, o)
@@ -517,7 +517,7 @@ def run_ours(args, w):
             la.la_simple_fwd(xq, xk, xv, xo, xst, workspace=ws, stream=s_cmp)
             la.la_simple_bwd(xq, xk, xv, xg, xdq, xdk, xdv, xst, workspace=ws, stream=s_cmp)
         elif w.op == "causal_norm":
-            la.la_causal_norm_fwd(xq, xk, xv, xo, None, "elu1", w.eps, stream=s_cmp)
+            la.la_causal_norm_fwd(xq, xk, xv, xo, None, "elu1", w.eps, workspace=ws, stream=s_cmp)
             la.la_causal_norm_bwd(xq, xk, xv, xg, xdq, xdk, xdv, None, "elu1", w.eps, workspace=ws, stream=s_cmp)
         elif gated:
             la.la_gated_fwd(xq, xk, xv, ins[4], xo, stream=s_cmp)

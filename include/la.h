@@ -247,11 +247,16 @@ la_status la_chunk_decay_scan(const float *states, const long long *gaps, int n,
  * op is la_chunk_decay_* (identity f, gamma = 1 for plain causal linear
  * attention).  Sources: "flash-linear-attention" README, "Different forms of
  * linear attention" (FusedRecurrent: the recurrent form these calls compute);
- * the norm term and f as in la_bidir_*.  Computed on CUDA cores, fp32, one CTA
- * per (b, h) walking the sequence; all dtypes, D in {64, 128}. */
+ * the norm term and f as in la_bidir_*.  Computed on CUDA cores, fp32; all
+ * dtypes, D in {64, 128}.  The sequence is cut into chunks of 256 tokens, one
+ * CTA per (b, h, chunk) walking its chunk from the state the tokens before it
+ * leave; those states come from each chunk's own state (a sum of outer
+ * products) and a scan over the chunks.
+ * Workspace: la_workspace_size(LA_OP_CAUSAL_NORM_FWD, ...) bytes (the chunk
+ * states, B H ceil(T / 256) D (D + 1) fp32 values; 0, NULL allowed, for T <= 256). */
 la_status la_causal_norm_fwd(const void *q, const void *k, const void *v, void *o, const float *decay,
                              la_feature feature, float eps, int B, int H, int T, int D, la_dtype dtype,
-                             void *stream);
+                             void *workspace, size_t workspace_bytes, void *stream);
 
 /* Gradients of sum(o * dout) for la_causal_norm_fwd.  With u_t = f(q_t) S_t,
  * n_t = f(q_t) . z_t + eps, o_t = u_t / n_t, du_t = dout_t / n_t and
@@ -260,7 +265,8 @@ la_status la_causal_norm_fwd(const void *q, const void *k, const void *v, void *
  *   R_s = sum_{t>=s} gamma^(t-s) f(q_t)^T du_t,  r_s = sum_{t>=s} gamma^(t-s) f(q_t) dn_t
  *   dk_s = (R_s v_s + r_s) f'(k_s),  dv_s = f(k_s) R_s.
  * Workspace: la_workspace_size(LA_OP_CAUSAL_NORM_BWD, ...) bytes ((n_t, dn_t)
- * of every row, 8 B per token-head). */
+ * of every row, 8 B per token-head, then the chunk states of the forward and,
+ * reusing them, of the reverse sweep). */
 la_status la_causal_norm_bwd(const void *q, const void *k, const void *v, const void *dout, const float *decay,
                              la_feature feature, float eps, void *dq, void *dk, void *dv,
                              int B, int H, int T, int D, la_dtype dtype,

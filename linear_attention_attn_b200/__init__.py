@@ -62,7 +62,7 @@ _lib.la_gated_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
 _lib.la_gated_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_feature_map_fwd.argtypes = [_I, _F, _P, _P, _I, _I, _I, _I, _I, _P]
 _lib.la_feature_map_bwd.argtypes = [_I, _F, _P, _P, _P, _I, _I, _I, _I, _I, _P]
-_lib.la_causal_norm_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _F, _I, _I, _I, _I, _I, _P]
+_lib.la_causal_norm_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _F, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_causal_norm_bwd.argtypes = [_P, _P, _P, _P, _P, _I, _F, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_state_reduce.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_state_apply.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
@@ -368,13 +368,15 @@ def la_feature_map_bwd(kind, x, dy, dx, p: float = 1.0, stream=None):
                                    _dtype_code(x), _stream(stream, x.device)), "la_feature_map_bwd")
 
 
-def la_causal_norm_fwd(q, k, v, o, decay=None, feature="elu1", eps: float = 1e-6, stream=None):
+def la_causal_norm_fwd(q, k, v, o, decay=None, feature="elu1", eps: float = 1e-6, workspace=None, stream=None):
     """Causal linear attention with the norm term: o_t <- f(q_t) S_t / (f(q_t) . z_t + eps), S_t and
     z_t the decay[h]-weighted sums over s <= t of f(k_s)^T v_s and f(k_s) (decay None: 1)."""
     B, H, T, D = _shape(q, k, v, o)
     dp, _keep = _decay_or_null(decay, H)
+    dt = _dtype_code(q)
+    wp, wn, _wkeep = _workspace("causal_norm_fwd", (B, H, T, D), dt, workspace, q.device, stream)
     _check(_lib.la_causal_norm_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), dp, _feature(feature),
-                                   ctypes.c_float(eps), B, H, T, D, _dtype_code(q), _stream(stream, q.device)),
+                                   ctypes.c_float(eps), B, H, T, D, dt, wp, wn, _stream(stream, q.device)),
            "la_causal_norm_fwd")
 
 

@@ -410,7 +410,8 @@ static la_status causal_entry(const Shape &s, la_dtype dt, const float *decay, l
 }
 
 la_status la_causal_norm_fwd(const void *q, const void *k, const void *v, void *o, const float *decay,
-                             la_feature feature, float eps, int B, int H, int T, int D, la_dtype dtype, void *stream) {
+                             la_feature feature, float eps, int B, int H, int T, int D, la_dtype dtype,
+                             void *workspace, size_t workspace_bytes, void *stream) {
     const Shape s{B, H, T, D};
     DecayArgs dec;
     int has_decay = 0;
@@ -419,8 +420,9 @@ la_status la_causal_norm_fwd(const void *q, const void *k, const void *v, void *
     LA_TRY(check_ptr(k, "k"));
     LA_TRY(check_ptr(v, "v"));
     LA_TRY(check_ptr(o, "o"));
+    LA_TRY(check_ws(LA_OP_CAUSAL_NORM_FWD, s, dtype, workspace, workspace_bytes));
     if (T == 0) return LA_OK;
-    return simt::causal_norm_fwd(q, k, v, o, dec, has_decay, feature == LA_FEATURE_ELU1, s, dtype, eps,
+    return simt::causal_norm_fwd(q, k, v, o, dec, has_decay, feature == LA_FEATURE_ELU1, s, dtype, eps, workspace,
                                  (cudaStream_t)stream);
 }
 

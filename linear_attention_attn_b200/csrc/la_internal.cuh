@@ -153,9 +153,10 @@ la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, 
 la_status state_stage(Stage stage, la_feature f, const void *x, const void *y, const float *sin, float *sout,
                       void *out1, void *out2, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
 // Causal linear attention with the norm term (has_decay = 0: gamma = 1; phi: elu + 1,
-// else the identity).  The backward's workspace holds (n_t, dn_t) of every row.
+// else the identity).  The workspaces hold the chunk states (sequences of more than one
+// chunk) and, for the backward, (n_t, dn_t) of every row before them.
 la_status causal_norm_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, int has_decay,
-                          bool phi, const Shape &s, la_dtype dt, float eps, cudaStream_t st);
+                          bool phi, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
 la_status causal_norm_bwd(const void *q, const void *k, const void *v, const void *g, void *dq, void *dk, void *dv,
                           const DecayArgs &dec, int has_decay, bool phi, const Shape &s, la_dtype dt, float eps,
                           void *ws, cudaStream_t st);

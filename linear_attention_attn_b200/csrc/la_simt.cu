@@ -24,6 +24,18 @@ namespace simt {
 constexpr int kTile = 32;      // rows per shared-memory tile
 constexpr int kRetTile = 16;   // rows per tile in the recurrent (retention) kernels
 constexpr int kThreads = 256;
+constexpr int kCausalChunk = 256;   // tokens per chunk of the causal-norm kernels (a multiple of kRetTile)
+static_assert(kCausalChunk % kRetTile == 0, "chunks hold whole recurrent tiles");
+
+inline int causal_chunks(int T_len) { return T_len <= kCausalChunk ? 1 : (T_len + kCausalChunk - 1) / kCausalChunk; }
+inline size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+// (n_t, dn_t) of every row of the causal-norm backward
+inline size_t nd_bytes(const Shape &s) { return round256((size_t)s.BH() * s.T * sizeof(float2)); }
+// the [B H][chunk][D][D + 1] fp32 chunk states; none for a single chunk
+inline size_t causal_state_bytes(const Shape &s) {
+    const int nc = causal_chunks(s.T);
+    return nc > 1 ? round256((size_t)s.BH() * nc * s.D * (s.D + 1) * sizeof(float)) : 0;
+}
 
 // ------------------------------------------------------------ reductions --
 
@@ -470,7 +482,7 @@ template <bool PHI>
 __device__ __forceinline__ float feature_grad_of(float fx) { return PHI ? (fx > 1.f ? 1.f : fx) : 1.f; }
 
 // Each state line (a column or a row of S, or z) is split over P threads: thread p of a
-// line takes the D / P entries p D / P .. (p + 1) D / P - 1 of it, and the line's P partial
+// line takes the D / P entries part_entry(p, 0 .. D / P - 1) of it, and the line's P partial
 // dot products meet through xor shuffles among P adjacent lanes (fixed order).  Blocks are
 // whole warps; the threads past the last line compute on zeros and store nothing.
 template <int D> constexpr int causal_split() { return D == 64 ? 4 : 2; }
@@ -486,37 +498,161 @@ __device__ __forceinline__ float line_sum(float s) {
     return s;
 }
 
+// A line's D entries are dealt to its P parts in float4 groups, round robin: part p holds
+// group m = entries 4 p + 4 P m .. 4 p + 4 P m + 3, its i-th entry part_entry(p, i).  The P
+// parts of a line (adjacent lanes) then read one contiguous 16 P-byte span of a shared-memory
+// row per group, a single conflict-free 128-bit load each.
+template <int P>
+__device__ __forceinline__ int part_entry(int p, int i) { return 4 * p + 4 * P * (i >> 2) + (i & 3); }
+template <int P>
+__device__ __forceinline__ float4 part_group(const float *row, int p, int m) {
+    return *reinterpret_cast<const float4 *>(row + 4 * p + 4 * P * m);
+}
+__device__ __forceinline__ float f4(const float4 &x, int e) { return e == 0 ? x.x : e == 1 ? x.y : e == 2 ? x.z : x.w; }
+
+// ---- chunks along T.  One CTA per head runs the recurrence over too few threads to fill the
+// GPU (B H CTAs), so the sequence is cut into chunks of kCausalChunk tokens, one CTA per (head,
+// chunk), each starting from the state that the tokens before its chunk leave (the backward's
+// reverse sweep: after its chunk).  Those states come from two short passes: every chunk's own
+// state from a zero state (a sum of weighted outer products, no recurrence), then a scan over
+// the chunks of one head:  S_in[c] = gamma^L S_in[c-1] + E[c-1]  (reverse: from the last chunk).
+// States are [B H][chunk][D][D + 1] fp32, the last column z (forward) or r (reverse).
+template <int D>
+__device__ __forceinline__ const float *chunk_state(const float *st, int bh, int c) {
+    return st ? st + ((long long)bh * gridDim.y + c) * D * (D + 1) : nullptr;
+}
+
+constexpr int kChunkStateRows = 32;     // token rows per shared-memory tile of causal_chunk_state
+
+// E[c] = sum over the chunk's tokens t of w_t a_t^T [b_t | c_t]:
+//   forward (REV false): a = f(k), b = v, c = 1, w_t = gamma^(s1 - 1 - t)  (the state after the
+//     chunk's last token s1 - 1, from a zero state before its first);
+//   reverse (REV true):  a = f(q), b = dout / n, c = dn, w_t = gamma^(t - s0)  (R, r at the chunk's
+//     first token s0, from a zero state after its last).
+// 256 threads as 16 x 16; thread (ti, tj) accumulates rows 4 ti + 64 m + 0..3 by columns
+// 4 tj + 64 n + 0..3 (float4 reads of the staged rows), and rows' c column for tj = 0.
+template <typename T, int D, bool PHI, bool REV>
+__global__ void __launch_bounds__(256)
+causal_chunk_state(const T *__restrict__ a_src, const T *__restrict__ b_src, const float2 *__restrict__ nd,
+                   float *__restrict__ E, DecayArgs dec, int has_decay, int T_len, int H, int L) {
+    constexpr int G = D / 64;                  // float4 groups per thread and side
+    __shared__ __align__(16) float As[kChunkStateRows][D];
+    __shared__ __align__(16) float Bs[kChunkStateRows][D];
+    __shared__ float Cs[kChunkStateRows];
+    const int c = blockIdx.x, bh = blockIdx.y, nc = gridDim.x;
+    if (REV ? c == 0 : c == nc - 1) return;    // no other chunk starts from this one's state
+    const int s0 = c * L, s1 = min(T_len, s0 + L);
+    const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
+    const long long base = (long long)bh * T_len * D;
+    const int tj = threadIdx.x & 15, ti = threadIdx.x >> 4;
+    float acc[4 * G][4 * G], accc[4 * G];
+#pragma unroll
+    for (int m = 0; m < 4 * G; ++m) {
+        accc[m] = 0.f;
+#pragma unroll
+        for (int n = 0; n < 4 * G; ++n) acc[m][n] = 0.f;
+    }
+    for (int ts = s0; ts < s1; ts += kChunkStateRows) {
+        const int nr = min(kChunkStateRows, s1 - ts);
+        __syncthreads();
+        for (int e = threadIdx.x; e < kChunkStateRows * D; e += blockDim.x) {
+            const int r = e / D, x = e % D, t = ts + r;
+            float a = 0.f, b = 0.f;
+            if (r < nr) {
+                const float w = has_decay ? powf(gamma, (float)(REV ? t - s0 : s1 - 1 - t)) : 1.f;
+                a = io<T>::ld(a_src + base + (long long)t * D + x);
+                a = (PHI ? feature(a) : a) * w;
+                b = io<T>::ld(b_src + base + (long long)t * D + x);
+                if (REV) b *= 1.f / nd[(long long)bh * T_len + t].x;
+            }
+            As[r][x] = a;
+            Bs[r][x] = b;
+        }
+        if (threadIdx.x < kChunkStateRows)
+            Cs[threadIdx.x] = threadIdx.x < nr ? (REV ? nd[(long long)bh * T_len + ts + threadIdx.x].y : 1.f) : 0.f;
+        __syncthreads();
+        for (int r = 0; r < nr; ++r) {
+            float a[4 * G], b[4 * G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float4 x = *reinterpret_cast<const float4 *>(&As[r][64 * g + 4 * ti]);
+                const float4 y = *reinterpret_cast<const float4 *>(&Bs[r][64 * g + 4 * tj]);
+                a[4 * g] = x.x, a[4 * g + 1] = x.y, a[4 * g + 2] = x.z, a[4 * g + 3] = x.w;
+                b[4 * g] = y.x, b[4 * g + 1] = y.y, b[4 * g + 2] = y.z, b[4 * g + 3] = y.w;
+            }
+            const float cr = Cs[r];
+#pragma unroll
+            for (int m = 0; m < 4 * G; ++m) {
+#pragma unroll
+                for (int n = 0; n < 4 * G; ++n) acc[m][n] = fmaf(a[m], b[n], acc[m][n]);
+                accc[m] = fmaf(a[m], cr, accc[m]);
+            }
+        }
+    }
+    float *out = E + ((long long)bh * nc + c) * D * (D + 1);
+#pragma unroll
+    for (int m = 0; m < 4 * G; ++m) {
+        const int i = 64 * (m / 4) + 4 * ti + m % 4;
+#pragma unroll
+        for (int n = 0; n < 4 * G; ++n) out[i * (D + 1) + 64 * (n / 4) + 4 * tj + n % 4] = acc[m][n];
+        if (tj == 0) out[i * (D + 1) + D] = accc[m];
+    }
+}
+
+// In place over the nc chunk states of each head: the state entering chunk c (forward) or the
+// reverse state entering it from the chunks after it (REV).  Every chunk but the last (REV: the
+// first) has L tokens; the state of the last chunk visited is never read.
+__global__ void __launch_bounds__(256)
+causal_chunk_scan(float *__restrict__ E, DecayArgs dec, int has_decay, int H, int nc, int per_head, int L, int rev) {
+    const int bh = blockIdx.y, e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= per_head) return;
+    const float f = has_decay ? (float)pow((double)dec.gamma[bh % H], (double)L) : 1.f;
+    float *p = E + (long long)bh * nc * per_head + e;
+    float run = 0.f;
+    for (int i = 0; i < nc; ++i) {
+        const long long at = (long long)(rev ? nc - 1 - i : i) * per_head;
+        const float own = i == nc - 1 ? 0.f : p[at];
+        p[at] = run;
+        run = fmaf(f, run, own);
+    }
+}
+
 // Forward: the D + 1 columns of [S | z] (z: the column of a value that is always 1).
 template <typename T, int D, bool PHI>
 __global__ void __launch_bounds__(causal_fwd_threads<D>())
 causal_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, T *__restrict__ o,
-           DecayArgs dec, int has_decay, int T_len, int H, float eps) {
+           const float *__restrict__ st_in, DecayArgs dec, int has_decay, int T_len, int H, int L, float eps) {
     constexpr int P = causal_split<D>(), DP = D / P;
-    __shared__ float tiles[3][kRetTile][D];
+    __shared__ __align__(16) float tiles[3][kRetTile][D];
     __shared__ float acc[kRetTile][D + 1];
-    const int bh = blockIdx.x;
+    const int bh = blockIdx.x, s0 = blockIdx.y * L, s1 = min(T_len, s0 + L);
     const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
     const long long base = (long long)bh * T_len * D;
-    const int j = threadIdx.x / P, i0 = (threadIdx.x % P) * DP;
-    const bool lead = threadIdx.x % P == 0 && j <= D;
+    const int j = threadIdx.x / P, pp = threadIdx.x % P;
+    const bool lead = pp == 0 && j <= D;
+    const float *const S0 = chunk_state<D>(st_in, bh, blockIdx.y);
     float S[DP];
 #pragma unroll
-    for (int i = 0; i < DP; ++i) S[i] = 0.f;
+    for (int i = 0; i < DP; ++i) S[i] = S0 && j <= D ? S0[part_entry<P>(pp, i) * (D + 1) + j] : 0.f;
     const T *const src[3] = {q, k, v};
-    for (int ts = 0; ts < T_len; ts += kRetTile) {
+    for (int ts = s0; ts < s1; ts += kRetTile) {
         __syncthreads();
         load_rows<T, D, 3>(src, tiles, base, ts, T_len, blockDim.x);
         __syncthreads();
         feature_tiles<D, PHI>(tiles, 2);
         __syncthreads();
-        const int nr = min(kRetTile, T_len - ts);
+        const int nr = min(kRetTile, s1 - ts);
         for (int r = 0; r < nr; ++r) {
             const float vj = j < D ? tiles[2][r][j] : 1.f;
             float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < DP; ++i) {
-                S[i] = fmaf(gamma, S[i], tiles[1][r][i0 + i] * vj);
-                a[i & 3] = fmaf(tiles[0][r][i0 + i], S[i], a[i & 3]);
+            for (int m = 0; m < DP / 4; ++m) {
+                const float4 kk = part_group<P>(tiles[1][r], pp, m), qq = part_group<P>(tiles[0][r], pp, m);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    S[4 * m + e] = fmaf(gamma, S[4 * m + e], f4(kk, e) * vj);
+                    a[e] = fmaf(f4(qq, e), S[4 * m + e], a[e]);
+                }
             }
             const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
             if (lead) acc[r][j] = s;
@@ -537,50 +673,64 @@ causal_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict
 template <typename T, int D, bool PHI>
 __global__ void __launch_bounds__(causal_bwd_q_threads<D>())
 causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
-             T *__restrict__ dq, float2 *__restrict__ nd, DecayArgs dec, int has_decay, int T_len, int H, float eps) {
+             T *__restrict__ dq, float2 *__restrict__ nd, const float *__restrict__ st_in, DecayArgs dec, int has_decay,
+             int T_len, int H, int L, float eps) {
     constexpr int P = causal_split<D>(), DP = D / P, NCOL = P * (D + 1);
-    extern __shared__ float dsm[];               // causal_bwd_q_smem<D>() bytes
+    extern __shared__ __align__(16) float dsm[];   // causal_bwd_q_smem<D>() bytes
     float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // f(q), f(k), v, dout
     float(*U)[D + 1] = reinterpret_cast<float(*)[D + 1]>(dsm + 4 * kRetTile * D);  // dout_t[j] u_t[j], n_t - eps
     float(*A)[D] = reinterpret_cast<float(*)[D]>(dsm + 4 * kRetTile * D + kRetTile * (D + 1));
     float(*Z)[D] = A + kRetTile;
     float2 *info = reinterpret_cast<float2 *>(dsm + 6 * kRetTile * D + kRetTile * (D + 1));   // (1 / n_t, dn_t)
-    const int bh = blockIdx.x;
+    const int bh = blockIdx.x, s0 = blockIdx.y * L, s1 = min(T_len, s0 + L);
     const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
     const long long base = (long long)bh * T_len * D;
     const bool col_side = threadIdx.x < NCOL;
     const int t2 = col_side ? threadIdx.x : threadIdx.x - NCOL;
-    const int line = t2 / P, x0 = (t2 % P) * DP;       // column (col side) or row (row side); entry range
+    const int line = t2 / P, pp = t2 % P;              // column (col side) or row (row side); part
     const bool row_live = !col_side && line < D;
     const bool lead = t2 % P == 0 && (col_side || row_live);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    // the entering [S | z]: the col side takes column `line` (z for line = D), the row side row `line`
+    const float *const S0 = chunk_state<D>(st_in, bh, blockIdx.y);
     float Sx[DP];
-    float zi = 0.f;
+    float zi = S0 && row_live ? S0[line * (D + 1) + D] : 0.f;
 #pragma unroll
-    for (int i = 0; i < DP; ++i) Sx[i] = 0.f;
+    for (int i = 0; i < DP; ++i) {
+        const int x = part_entry<P>(pp, i);
+        Sx[i] = !S0 ? 0.f : col_side ? S0[x * (D + 1) + line] : row_live ? S0[line * (D + 1) + x] : 0.f;
+    }
     const T *const src[4] = {q, k, v, g};
-    for (int ts = 0; ts < T_len; ts += kRetTile) {
+    for (int ts = s0; ts < s1; ts += kRetTile) {
         __syncthreads();
         load_rows<T, D, 4>(src, tiles, base, ts, T_len, blockDim.x);
         __syncthreads();
         feature_tiles<D, PHI>(tiles, 2);
         __syncthreads();
-        const int nr = min(kRetTile, T_len - ts);
+        const int nr = min(kRetTile, s1 - ts);
         for (int r = 0; r < nr; ++r) {
             float a[4] = {0.f, 0.f, 0.f, 0.f};
             if (col_side) {
                 const float vj = line < D ? tiles[2][r][line] : 1.f;
 #pragma unroll
-                for (int i = 0; i < DP; ++i) {
-                    Sx[i] = fmaf(gamma, Sx[i], tiles[1][r][x0 + i] * vj);
-                    a[i & 3] = fmaf(tiles[0][r][x0 + i], Sx[i], a[i & 3]);
+                for (int m = 0; m < DP / 4; ++m) {
+                    const float4 kk = part_group<P>(tiles[1][r], pp, m), qq = part_group<P>(tiles[0][r], pp, m);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        Sx[4 * m + e] = fmaf(gamma, Sx[4 * m + e], f4(kk, e) * vj);
+                        a[e] = fmaf(f4(qq, e), Sx[4 * m + e], a[e]);
+                    }
                 }
             } else if (row_live) {
                 const float ki = tiles[1][r][line];
 #pragma unroll
-                for (int jj = 0; jj < DP; ++jj) {
-                    Sx[jj] = fmaf(gamma, Sx[jj], ki * tiles[2][r][x0 + jj]);
-                    a[jj & 3] = fmaf(Sx[jj], tiles[3][r][x0 + jj], a[jj & 3]);
+                for (int m = 0; m < DP / 4; ++m) {
+                    const float4 vv = part_group<P>(tiles[2][r], pp, m), gg = part_group<P>(tiles[3][r], pp, m);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        Sx[4 * m + e] = fmaf(gamma, Sx[4 * m + e], ki * f4(vv, e));
+                        a[e] = fmaf(Sx[4 * m + e], f4(gg, e), a[e]);
+                    }
                 }
                 zi = fmaf(gamma, zi, ki);
             }
@@ -631,31 +781,34 @@ static_assert((6 * kRetTile * 64 + kRetTile * 65) % 2 == 0 && (6 * kRetTile * 12
 template <typename T, int D, bool PHI>
 __global__ void __launch_bounds__(causal_bwd_kv_threads<D>())
 causal_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
-              const float2 *__restrict__ nd, T *__restrict__ dk, T *__restrict__ dv, DecayArgs dec, int has_decay,
-              int T_len, int H) {
+              const float2 *__restrict__ nd, T *__restrict__ dk, T *__restrict__ dv, const float *__restrict__ st_in,
+              DecayArgs dec, int has_decay, int T_len, int H, int L) {
     constexpr int P = causal_split<D>(), DP = D / P;
-    extern __shared__ float dsm[];               // causal_bwd_kv_smem<D>() bytes
+    extern __shared__ __align__(16) float dsm[];   // causal_bwd_kv_smem<D>() bytes
     float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // f(q), f(k), v, dout
     float(*res)[kRetTile][D] = tiles + 4;        // dk before f' (rows), dv (columns)
     float2 *info = reinterpret_cast<float2 *>(dsm + 6 * kRetTile * D);
-    const int bh = blockIdx.x;
+    const int bh = blockIdx.x, s0 = blockIdx.y * L, s1 = min(T_len, s0 + L);
     const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
     const long long base = (long long)bh * T_len * D;
     const bool row_side = threadIdx.x < P * D;
     const int t2 = row_side ? threadIdx.x : threadIdx.x - P * D;
-    const int line = t2 / P, x0 = (t2 % P) * DP;
-    const bool lead = t2 % P == 0;
+    const int line = t2 / P, pp = t2 % P;
+    const bool lead = pp == 0;
+    // the entering [R | r] (the tokens after this chunk): rows on the row side, columns on the other
+    const float *const R0 = chunk_state<D>(st_in, bh, blockIdx.y);
     float Rx[DP];
-    float ri = 0.f;
+    float ri = R0 && row_side ? R0[line * (D + 1) + D] : 0.f;
 #pragma unroll
-    for (int m = 0; m < DP; ++m) Rx[m] = 0.f;
+    for (int i = 0; i < DP; ++i) {
+        const int x = part_entry<P>(pp, i);
+        Rx[i] = !R0 ? 0.f : row_side ? R0[line * (D + 1) + x] : R0[x * (D + 1) + line];
+    }
     const T *const src[4] = {q, k, v, g};
-    const int ntiles = (T_len + kRetTile - 1) / kRetTile;
-    for (int tile = ntiles - 1; tile >= 0; --tile) {
-        const int ts = tile * kRetTile;
+    for (int ts = s0 + (s1 - s0 - 1) / kRetTile * kRetTile; ts >= s0; ts -= kRetTile) {
         __syncthreads();
         load_rows<T, D, 4>(src, tiles, base, ts, T_len, blockDim.x);
-        const int nr = min(kRetTile, T_len - ts);
+        const int nr = min(kRetTile, s1 - ts);
         if (threadIdx.x < nr) {
             const float2 x = nd[(long long)bh * T_len + ts + threadIdx.x];
             info[threadIdx.x] = make_float2(1.f / x.x, x.y);
@@ -669,17 +822,25 @@ causal_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
             if (row_side) {
                 const float qi = tiles[0][r][line];
 #pragma unroll
-                for (int jj = 0; jj < DP; ++jj) {
-                    Rx[jj] = fmaf(gamma, Rx[jj], qi * (tiles[3][r][x0 + jj] * in.x));
-                    a[jj & 3] = fmaf(Rx[jj], tiles[2][r][x0 + jj], a[jj & 3]);
+                for (int m = 0; m < DP / 4; ++m) {
+                    const float4 gg = part_group<P>(tiles[3][r], pp, m), vv = part_group<P>(tiles[2][r], pp, m);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        Rx[4 * m + e] = fmaf(gamma, Rx[4 * m + e], qi * (f4(gg, e) * in.x));
+                        a[e] = fmaf(Rx[4 * m + e], f4(vv, e), a[e]);
+                    }
                 }
                 ri = fmaf(gamma, ri, qi * in.y);
             } else {
                 const float duj = tiles[3][r][line] * in.x;
 #pragma unroll
-                for (int i = 0; i < DP; ++i) {
-                    Rx[i] = fmaf(gamma, Rx[i], tiles[0][r][x0 + i] * duj);
-                    a[i & 3] = fmaf(tiles[1][r][x0 + i], Rx[i], a[i & 3]);
+                for (int m = 0; m < DP / 4; ++m) {
+                    const float4 qq = part_group<P>(tiles[0][r], pp, m), kk = part_group<P>(tiles[1][r], pp, m);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        Rx[4 * m + e] = fmaf(gamma, Rx[4 * m + e], f4(qq, e) * duj);
+                        a[e] = fmaf(f4(kk, e), Rx[4 * m + e], a[e]);
+                    }
                 }
             }
             const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
@@ -713,17 +874,18 @@ __device__ __forceinline__ void exp_tile(float (*tile)[D]) {
 template <int D> constexpr int gated_fwd_threads() { return causal_split<D>() * D; }
 template <int D> constexpr int gated_kv_threads() { return 2 * causal_split<D>() * D; }
 
-// Forward: the D columns of S; thread p of column j holds S[i][j] for its D / P rows i.
+// Forward: the D columns of S; thread p of column j holds S[i][j] for its D / P rows
+// i = part_entry(p, .).
 template <typename T, int D>
 __global__ void __launch_bounds__(gated_fwd_threads<D>())
 gated_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
           T *__restrict__ o, int T_len) {
     constexpr int P = causal_split<D>(), DP = D / P;
-    __shared__ float tiles[4][kRetTile][D];      // q, k, v, a = exp(g)
+    __shared__ __align__(16) float tiles[4][kRetTile][D];      // q, k, v, a = exp(g)
     __shared__ float acc[kRetTile][D];
     const long long base = (long long)blockIdx.x * T_len * D;
-    const int j = threadIdx.x / P, i0 = (threadIdx.x % P) * DP;
-    const bool lead = threadIdx.x % P == 0;
+    const int j = threadIdx.x / P, pp = threadIdx.x % P;
+    const bool lead = pp == 0;
     float S[DP];
 #pragma unroll
     for (int i = 0; i < DP; ++i) S[i] = 0.f;
@@ -739,9 +901,14 @@ gated_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
             const float vj = tiles[2][r][j];
             float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < DP; ++i) {
-                S[i] = fmaf(tiles[3][r][i0 + i], S[i], tiles[1][r][i0 + i] * vj);
-                a[i & 3] = fmaf(tiles[0][r][i0 + i], S[i], a[i & 3]);
+            for (int m = 0; m < DP / 4; ++m) {
+                const float4 aa = part_group<P>(tiles[3][r], pp, m), kk = part_group<P>(tiles[1][r], pp, m),
+                             qq = part_group<P>(tiles[0][r], pp, m);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    S[4 * m + e] = fmaf(f4(aa, e), S[4 * m + e], f4(kk, e) * vj);
+                    a[e] = fmaf(f4(qq, e), S[4 * m + e], a[e]);
+                }
             }
             const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
             if (lead) acc[r][j] = s;
@@ -753,17 +920,17 @@ gated_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
 }
 
 // Backward, forward sweep: dq_t[i] = sum_j S_t[i][j] dout_t[j]; thread p of row i holds
-// S[i][j] for its D / P columns j.
+// S[i][j] for its D / P columns j = part_entry(p, .).
 template <typename T, int D>
 __global__ void __launch_bounds__(gated_fwd_threads<D>())
 gated_bwd_q(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g, const T *__restrict__ dout,
             T *__restrict__ dq, float *__restrict__ dq32, int T_len) {
     constexpr int P = causal_split<D>(), DP = D / P;
-    __shared__ float tiles[4][kRetTile][D];      // k, v, a = exp(g), dout
+    __shared__ __align__(16) float tiles[4][kRetTile][D];      // k, v, a = exp(g), dout
     __shared__ float acc[kRetTile][D];
     const long long base = (long long)blockIdx.x * T_len * D;
-    const int i = threadIdx.x / P, j0 = (threadIdx.x % P) * DP;
-    const bool lead = threadIdx.x % P == 0;
+    const int i = threadIdx.x / P, pp = threadIdx.x % P;
+    const bool lead = pp == 0;
     float S[DP];
 #pragma unroll
     for (int jj = 0; jj < DP; ++jj) S[jj] = 0.f;
@@ -779,9 +946,13 @@ gated_bwd_q(const T *__restrict__ k, const T *__restrict__ v, const T *__restric
             const float ai = tiles[2][r][i], ki = tiles[0][r][i];
             float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int jj = 0; jj < DP; ++jj) {
-                S[jj] = fmaf(ai, S[jj], ki * tiles[1][r][j0 + jj]);
-                a[jj & 3] = fmaf(S[jj], tiles[3][r][j0 + jj], a[jj & 3]);
+            for (int m = 0; m < DP / 4; ++m) {
+                const float4 vv = part_group<P>(tiles[1][r], pp, m), gg = part_group<P>(tiles[3][r], pp, m);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    S[4 * m + e] = fmaf(ai, S[4 * m + e], ki * f4(vv, e));
+                    a[e] = fmaf(S[4 * m + e], f4(gg, e), a[e]);
+                }
             }
             const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
             if (lead) acc[r][i] = s;
@@ -808,15 +979,15 @@ gated_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
              const T *__restrict__ dout, const float *__restrict__ dq32, T *__restrict__ dk, T *__restrict__ dv,
              T *__restrict__ dg, int T_len) {
     constexpr int P = causal_split<D>(), DP = D / P;
-    extern __shared__ float dsm[];               // gated_bwd_kv_smem<D>() bytes
+    extern __shared__ __align__(16) float dsm[];   // gated_bwd_kv_smem<D>() bytes
     float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // q, k, v, dout, a = exp(g)
     float(*res)[kRetTile][D] = tiles + 5;        // dk (rows), dv (columns)
     float *anext = dsm + 7 * kRetTile * D;       // a of the row after the tile (0 past the sequence)
     const long long base = (long long)blockIdx.x * T_len * D;
     const bool row_side = threadIdx.x < P * D;
     const int t2 = row_side ? threadIdx.x : threadIdx.x - P * D;
-    const int line = t2 / P, x0 = (t2 % P) * DP;
-    const bool lead = t2 % P == 0;
+    const int line = t2 / P, pp = t2 % P;
+    const bool lead = pp == 0;
     float Rx[DP];
     float accg = 0.f;                            // thread i < D: sum over the rows after t of dL/dG[i]
 #pragma unroll
@@ -838,16 +1009,25 @@ gated_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
             if (row_side) {
                 const float qi = tiles[0][r][line], ai = an[line];
 #pragma unroll
-                for (int jj = 0; jj < DP; ++jj) {
-                    Rx[jj] = fmaf(ai, Rx[jj], qi * tiles[3][r][x0 + jj]);
-                    a[jj & 3] = fmaf(Rx[jj], tiles[2][r][x0 + jj], a[jj & 3]);
+                for (int m = 0; m < DP / 4; ++m) {
+                    const float4 gg = part_group<P>(tiles[3][r], pp, m), vv = part_group<P>(tiles[2][r], pp, m);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        Rx[4 * m + e] = fmaf(ai, Rx[4 * m + e], qi * f4(gg, e));
+                        a[e] = fmaf(Rx[4 * m + e], f4(vv, e), a[e]);
+                    }
                 }
             } else {
                 const float gj = tiles[3][r][line];
 #pragma unroll
-                for (int i = 0; i < DP; ++i) {
-                    Rx[i] = fmaf(an[x0 + i], Rx[i], tiles[0][r][x0 + i] * gj);
-                    a[i & 3] = fmaf(tiles[1][r][x0 + i], Rx[i], a[i & 3]);
+                for (int m = 0; m < DP / 4; ++m) {
+                    const float4 aa = part_group<P>(an, pp, m), qq = part_group<P>(tiles[0][r], pp, m),
+                                 kk = part_group<P>(tiles[1][r], pp, m);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        Rx[4 * m + e] = fmaf(f4(aa, e), Rx[4 * m + e], f4(qq, e) * gj);
+                        a[e] = fmaf(f4(kk, e), Rx[4 * m + e], a[e]);
+                    }
                 }
             }
             const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
@@ -1047,8 +1227,10 @@ size_t workspace_size(la_op op, const Shape &s) {
     case LA_OP_STATE_REDUCE:
     case LA_OP_STATE_BWD_Q:
         return state_bytes(s, simt_splits(s));
-    case LA_OP_CAUSAL_NORM_BWD:   // (n_t, dn_t) of every row
-        return ((size_t)s.BH() * s.T * sizeof(float2) + 255) / 256 * 256;
+    case LA_OP_CAUSAL_NORM_FWD:   // the chunk states
+        return causal_state_bytes(s);
+    case LA_OP_CAUSAL_NORM_BWD:   // (n_t, dn_t) of every row, then the chunk states
+        return nd_bytes(s) + causal_state_bytes(s);
     case LA_OP_GATED_BWD:         // dq in fp32, for the log gates' gradient
         return ((size_t)s.BH() * s.T * s.D * sizeof(float) + 255) / 256 * 256;
     default:
@@ -1114,25 +1296,51 @@ la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, 
 
 namespace {
 
+// The chunk states (forward, then reverse for the backward) of every head, scanned in place.
+template <typename T, int D, bool PHI, bool REV>
+la_status causal_states(const void *a, const void *b, const float2 *nd, float *E, const DecayArgs &dec, int has_decay,
+                        const Shape &s, cudaStream_t st) {
+    const int nc = causal_chunks(s.T), per_head = D * (D + 1);
+    la_status rc = launch(REV ? "simt_causal_norm_state_rev" : "simt_causal_norm_state",
+                          causal_chunk_state<T, D, PHI, REV>, dim3((unsigned)nc, (unsigned)s.BH()), dim3(256), 0, st,
+                          (const T *)a, (const T *)b, nd, E, dec, has_decay, s.T, s.H, kCausalChunk);
+    if (rc) return rc;
+    return launch("simt_causal_norm_scan", causal_chunk_scan, dim3((unsigned)((per_head + 255) / 256), (unsigned)s.BH()),
+                  dim3(256), 0, st, E, dec, has_decay, s.H, nc, per_head, kCausalChunk, (int)REV);
+}
+
 template <typename T, int D, bool PHI>
 la_status causal_fwd_t(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, int has_decay,
-                       const Shape &s, float eps, cudaStream_t st) {
-    return launch("simt_causal_norm_fwd", causal_fwd<T, D, PHI>, dim3((unsigned)s.BH()), dim3(causal_fwd_threads<D>()), 0, st,
-                  (const T *)q, (const T *)k, (const T *)v, (T *)o, dec, has_decay, s.T, s.H, eps);
+                       const Shape &s, float eps, void *ws, cudaStream_t st) {
+    const int nc = causal_chunks(s.T);
+    float *E = nc > 1 ? (float *)ws : nullptr;
+    if (E) {
+        const la_status rc = causal_states<T, D, PHI, false>(k, v, nullptr, E, dec, has_decay, s, st);
+        if (rc) return rc;
+    }
+    return launch("simt_causal_norm_fwd", causal_fwd<T, D, PHI>, dim3((unsigned)s.BH(), (unsigned)nc),
+                  dim3(causal_fwd_threads<D>()), 0, st, (const T *)q, (const T *)k, (const T *)v, (T *)o,
+                  (const float *)E, dec, has_decay, s.T, s.H, kCausalChunk, eps);
 }
 
 template <typename T, int D, bool PHI>
 la_status causal_bwd_t(const void *q, const void *k, const void *v, const void *g, void *dq, void *dk, void *dv,
                        const DecayArgs &dec, int has_decay, const Shape &s, float eps, void *ws, cudaStream_t st) {
+    const int nc = causal_chunks(s.T);
     float2 *nd = (float2 *)ws;
-    la_status rc = launch("simt_causal_norm_bwd_q", causal_bwd_q<T, D, PHI>, dim3((unsigned)s.BH()),
-                          dim3(causal_bwd_q_threads<D>()), causal_bwd_q_smem<D>(), st, (const T *)q, (const T *)k, (const T *)v,
-                          (const T *)g, (T *)dq, nd, dec, has_decay, s.T, s.H, eps);
+    float *E = nc > 1 ? (float *)((char *)ws + nd_bytes(s)) : nullptr;
+    const dim3 grid((unsigned)s.BH(), (unsigned)nc);
+    la_status rc;
+    if (E && (rc = causal_states<T, D, PHI, false>(k, v, nullptr, E, dec, has_decay, s, st))) return rc;
+    rc = launch("simt_causal_norm_bwd_q", causal_bwd_q<T, D, PHI>, grid, dim3(causal_bwd_q_threads<D>()),
+                causal_bwd_q_smem<D>(), st, (const T *)q, (const T *)k, (const T *)v, (const T *)g, (T *)dq, nd,
+                (const float *)E, dec, has_decay, s.T, s.H, kCausalChunk, eps);
     if (rc) return rc;
-    return launch("simt_causal_norm_bwd_kv", causal_bwd_kv<T, D, PHI>, dim3((unsigned)s.BH()),
-                  dim3(causal_bwd_kv_threads<D>()), causal_bwd_kv_smem<D>(), st,
-                  (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const float2 *)nd, (T *)dk, (T *)dv, dec,
-                  has_decay, s.T, s.H);
+    // the reverse states need every row's (n, dn) from the dq pass; they reuse the forward's buffer
+    if (E && (rc = causal_states<T, D, PHI, true>(q, g, nd, E, dec, has_decay, s, st))) return rc;
+    return launch("simt_causal_norm_bwd_kv", causal_bwd_kv<T, D, PHI>, grid, dim3(causal_bwd_kv_threads<D>()),
+                  causal_bwd_kv_smem<D>(), st, (const T *)q, (const T *)k, (const T *)v, (const T *)g,
+                  (const float2 *)nd, (T *)dk, (T *)dv, (const float *)E, dec, has_decay, s.T, s.H, kCausalChunk);
 }
 
 // dtype x D x feature map dispatch of F<T, D, PHI>(args...)
@@ -1154,8 +1362,8 @@ la_status causal_bwd_t(const void *q, const void *k, const void *v, const void *
 }  // namespace
 
 la_status causal_norm_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, int has_decay,
-                          bool phi, const Shape &s, la_dtype dt, float eps, cudaStream_t st) {
-    LA_CAUSAL_DISPATCH(causal_fwd_t, q, k, v, o, dec, has_decay, s, eps, st);
+                          bool phi, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st) {
+    LA_CAUSAL_DISPATCH(causal_fwd_t, q, k, v, o, dec, has_decay, s, eps, ws, st);
 }
 
 la_status causal_norm_bwd(const void *q, const void *k, const void *v, const void *g, void *dq, void *dk, void *dv,

@@ -143,8 +143,9 @@ def test_causal_norm_validation(lib):
     b = lib.la_causal_norm_bwd
     b.restype = ctypes.c_int
 
-    def fwd(feature=1, eps=1e-6, q=0x1000, dec=None, D=64):
-        return f(P(q), P(0x1000), P(0x1000), P(0x1000), dec, feature, ctypes.c_float(eps), 1, 2, 16, D, 1, P(0))
+    def fwd(feature=1, eps=1e-6, q=0x1000, dec=None, D=64, T=16, ws=0, ws_bytes=0):
+        return f(P(q), P(0x1000), P(0x1000), P(0x1000), dec, feature, ctypes.c_float(eps), 1, 2, T, D, 1, P(ws),
+                 ctypes.c_size_t(ws_bytes), P(0))
     assert fwd(feature=5) == 2
     assert fwd(eps=-1.0) == 1
     assert fwd(q=0) == 1
@@ -154,6 +155,13 @@ def test_causal_norm_validation(lib):
     assert fwd(dec=ctypes.cast(bad, P)) == 1
     need = lib.la_workspace_size(11, 1, 2, 16, 64, 1)
     assert need == 256            # 2 x 16 rows x 8 bytes, rounded up to 256
+    # one chunk of 256 tokens needs no chunk states; 257 tokens make two chunks of [64][65] fp32 states
+    assert lib.la_workspace_size(10, 1, 2, 256, 64, 1) == 0
+    assert lib.la_workspace_size(10, 1, 2, 257, 64, 1) == 2 * 2 * 64 * 65 * 4
+    assert lib.la_workspace_size(11, 1, 2, 257, 64, 1) == 4352 + 2 * 2 * 64 * 65 * 4
+    assert fwd(T=257) == 4        # no workspace for two chunks
+    assert fwd(T=257, ws=0x1080, ws_bytes=1 << 20) == 3     # not 256-byte aligned
+    assert fwd(T=257, ws=0x1000, ws_bytes=100) == 4
     assert b(P(0x1000), P(0x1000), P(0x1000), P(0x1000), None, 1, ctypes.c_float(1e-6), P(0x1000), P(0x1000),
              P(0x1000), 1, 2, 16, 64, 1, P(0), ctypes.c_size_t(0), P(0)) == 4
 
