@@ -325,14 +325,26 @@ bwd_k(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict_
 
 // Loads rows [ts, ts+kRetTile) of up to four [T, D] tensors of one head into
 // fp32 shared tiles (zero past T).
-template <typename T, int D, int N>
+template <typename T, int D, int N, int NT>
 __device__ __forceinline__ void load_rows(const T *const (&src)[N], float (*dst)[kRetTile][D], long long base,
-                                          int ts, int T_len, int nthreads) {
-    for (int e = threadIdx.x; e < kRetTile * D; e += nthreads) {
-        const int r = e / D, c = e % D, t = ts + r;
+                                          int ts, int T_len) {
+    // NT threads; every load of the tile is issued before the first shared-memory store
+    constexpr int PER = (kRetTile * D + NT - 1) / NT;
+    float x[N][PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int e = threadIdx.x + u * NT, t = ts + e / D;
 #pragma unroll
         for (int m = 0; m < N; ++m)
-            dst[m][r][c] = t < T_len ? io<T>::ld(src[m] + base + (long long)t * D + c) : 0.f;
+            x[m][u] = e < kRetTile * D && t < T_len ? io<T>::ld(src[m] + base + (long long)t * D + e % D) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int e = threadIdx.x + u * NT;
+        if (e < kRetTile * D) {
+#pragma unroll
+            for (int m = 0; m < N; ++m) dst[m][e / D][e % D] = x[m][u];
+        }
     }
 }
 
@@ -353,7 +365,7 @@ ret_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ 
     const T *const src[3] = {q, k, v};
     for (int ts = 0; ts < T_len; ts += kRetTile) {
         __syncthreads();
-        load_rows<T, D, 3>(src, tiles, base, ts, T_len, D);
+        load_rows<T, D, 3, D>(src, tiles, base, ts, T_len);
         __syncthreads();
         const int nr = min(kRetTile, T_len - ts);
         for (int r = 0; r < nr; ++r) {
@@ -390,7 +402,7 @@ ret_bwd_dq(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict
     const T *const src[3] = {k, v, g};
     for (int ts = 0; ts < T_len; ts += kRetTile) {
         __syncthreads();
-        load_rows<T, D, 3>(src, tiles, base, ts, T_len, D);
+        load_rows<T, D, 3, D>(src, tiles, base, ts, T_len);
         __syncthreads();
         const int nr = min(kRetTile, T_len - ts);
         for (int r = 0; r < nr; ++r) {
@@ -430,7 +442,7 @@ ret_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
     for (int tile = ntiles - 1; tile >= 0; --tile) {
         const int ts = tile * kRetTile;
         __syncthreads();
-        load_rows<T, D, 4>(src, tiles, base, ts, T_len, 2 * D);
+        load_rows<T, D, 4, 2 * D>(src, tiles, base, ts, T_len);
         __syncthreads();
         const int nr = min(kRetTile, T_len - ts);
         for (int r = nr - 1; r >= 0; --r) {
@@ -509,6 +521,11 @@ __device__ __forceinline__ float4 part_group(const float *row, int p, int m) {
     return *reinterpret_cast<const float4 *>(row + 4 * p + 4 * P * m);
 }
 __device__ __forceinline__ float f4(const float4 &x, int e) { return e == 0 ? x.x : e == 1 ? x.y : e == 2 ? x.z : x.w; }
+// s <- gamma s + x y, or s + x y without a decay (one FMA)
+template <bool DECAY>
+__device__ __forceinline__ float decay_fma(float gamma, float s, float x, float y) {
+    return DECAY ? fmaf(gamma, s, x * y) : fmaf(x, y, s);
+}
 
 // ---- chunks along T.  One CTA per head runs the recurrence over too few threads to fill the
 // GPU (B H CTAs), so the sequence is cut into chunks of kCausalChunk tokens, one CTA per (head,
@@ -522,7 +539,29 @@ __device__ __forceinline__ const float *chunk_state(const float *st, int bh, int
     return st ? st + ((long long)bh * gridDim.y + c) * D * (D + 1) : nullptr;
 }
 
-constexpr int kChunkStateRows = 32;     // token rows per shared-memory tile of causal_chunk_state
+// token rows per shared-memory tile of causal_chunk_state (two buffers of a and b rows: 32 KB)
+template <int D> constexpr int chunk_state_rows() { return 2048 / D; }
+
+// One tile of causal_chunk_state's inputs into registers: thread x holds entries x + 256 u of
+// the tile's rows (rows at or past s1 are not read); rc: the c value of row x (x < the tile's rows).
+template <typename T, int D, bool REV, int EPT>
+__device__ __forceinline__ void chunk_fetch(const T *__restrict__ a, const T *__restrict__ b,
+                                            const float2 *__restrict__ ndh, int ts, int s1, float (&ra)[EPT],
+                                            float (&rb)[EPT], float (&rn)[EPT], float &rc) {
+#pragma unroll
+    for (int u = 0; u < EPT; ++u) {
+        const int e = threadIdx.x + 256 * u, t = ts + e / D;
+        if (t < s1) {
+            ra[u] = io<T>::ld(a + (long long)t * D + e % D);
+            rb[u] = io<T>::ld(b + (long long)t * D + e % D);
+            if (REV) rn[u] = ndh[t].x;
+        }
+    }
+    if (threadIdx.x < chunk_state_rows<D>()) {
+        const int t = ts + threadIdx.x;
+        rc = t < s1 ? (REV ? ndh[t].y : 1.f) : 0.f;
+    }
+}
 
 // E[c] = sum over the chunk's tokens t of w_t a_t^T [b_t | c_t]:
 //   forward (REV false): a = f(k), b = v, c = 1, w_t = gamma^(s1 - 1 - t)  (the state after the
@@ -530,20 +569,24 @@ constexpr int kChunkStateRows = 32;     // token rows per shared-memory tile of 
 //   reverse (REV true):  a = f(q), b = dout / n, c = dn, w_t = gamma^(t - s0)  (R, r at the chunk's
 //     first token s0, from a zero state after its last).
 // 256 threads as 16 x 16; thread (ti, tj) accumulates rows 4 ti + 64 m + 0..3 by columns
-// 4 tj + 64 n + 0..3 (float4 reads of the staged rows), and rows' c column for tj = 0.
+// 4 tj + 64 n + 0..3 (float4 reads of the staged rows), and rows' c column for tj = 0.  Tiles
+// are double buffered: the next tile's loads are in flight while the current one is summed.
 template <typename T, int D, bool PHI, bool REV>
 __global__ void __launch_bounds__(256)
 causal_chunk_state(const T *__restrict__ a_src, const T *__restrict__ b_src, const float2 *__restrict__ nd,
                    float *__restrict__ E, DecayArgs dec, int has_decay, int T_len, int H, int L) {
     constexpr int G = D / 64;                  // float4 groups per thread and side
-    __shared__ __align__(16) float As[kChunkStateRows][D];
-    __shared__ __align__(16) float Bs[kChunkStateRows][D];
-    __shared__ float Cs[kChunkStateRows];
+    constexpr int R = chunk_state_rows<D>(), EPT = R * D / 256;
+    __shared__ __align__(16) float As[2][R][D];
+    __shared__ __align__(16) float Bs[2][R][D];
+    __shared__ float Cs[2][R];
     const int c = blockIdx.x, bh = blockIdx.y, nc = gridDim.x;
     if (REV ? c == 0 : c == nc - 1) return;    // no other chunk starts from this one's state
     const int s0 = c * L, s1 = min(T_len, s0 + L);
     const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
     const long long base = (long long)bh * T_len * D;
+    const T *const a_h = a_src + base, *const b_h = b_src + base;
+    const float2 *const ndh = REV ? nd + (long long)bh * T_len : nullptr;
     const int tj = threadIdx.x & 15, ti = threadIdx.x >> 4;
     float acc[4 * G][4 * G], accc[4 * G];
 #pragma unroll
@@ -552,35 +595,40 @@ causal_chunk_state(const T *__restrict__ a_src, const T *__restrict__ b_src, con
 #pragma unroll
         for (int n = 0; n < 4 * G; ++n) acc[m][n] = 0.f;
     }
-    for (int ts = s0; ts < s1; ts += kChunkStateRows) {
-        const int nr = min(kChunkStateRows, s1 - ts);
-        __syncthreads();
-        for (int e = threadIdx.x; e < kChunkStateRows * D; e += blockDim.x) {
-            const int r = e / D, x = e % D, t = ts + r;
-            float a = 0.f, b = 0.f;
+    float ra[EPT], rb[EPT], rn[EPT], rc = 0.f;
+#pragma unroll
+    for (int u = 0; u < EPT; ++u) ra[u] = rb[u] = rn[u] = 0.f;
+    chunk_fetch<T, D, REV, EPT>(a_h, b_h, ndh, s0, s1, ra, rb, rn, rc);
+    int buf = 0;
+    for (int ts = s0; ts < s1; ts += R, buf ^= 1) {
+        const int nr = min(R, s1 - ts);
+        // the registers of this tile into buffer `buf` (last read two tiles ago, before the
+        // barrier of the previous tile)
+#pragma unroll
+        for (int u = 0; u < EPT; ++u) {
+            const int e = threadIdx.x + 256 * u, r = e / D, t = ts + r;
+            float av = 0.f, bv = 0.f;
             if (r < nr) {
                 const float w = has_decay ? powf(gamma, (float)(REV ? t - s0 : s1 - 1 - t)) : 1.f;
-                a = io<T>::ld(a_src + base + (long long)t * D + x);
-                a = (PHI ? feature(a) : a) * w;
-                b = io<T>::ld(b_src + base + (long long)t * D + x);
-                if (REV) b *= 1.f / nd[(long long)bh * T_len + t].x;
+                av = (PHI ? feature(ra[u]) : ra[u]) * w;
+                bv = REV ? rb[u] * (1.f / rn[u]) : rb[u];
             }
-            As[r][x] = a;
-            Bs[r][x] = b;
+            As[buf][r][e % D] = av;
+            Bs[buf][r][e % D] = bv;
         }
-        if (threadIdx.x < kChunkStateRows)
-            Cs[threadIdx.x] = threadIdx.x < nr ? (REV ? nd[(long long)bh * T_len + ts + threadIdx.x].y : 1.f) : 0.f;
+        if (threadIdx.x < R) Cs[buf][threadIdx.x] = rc;
         __syncthreads();
+        if (ts + R < s1) chunk_fetch<T, D, REV, EPT>(a_h, b_h, ndh, ts + R, s1, ra, rb, rn, rc);
         for (int r = 0; r < nr; ++r) {
             float a[4 * G], b[4 * G];
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const float4 x = *reinterpret_cast<const float4 *>(&As[r][64 * g + 4 * ti]);
-                const float4 y = *reinterpret_cast<const float4 *>(&Bs[r][64 * g + 4 * tj]);
+                const float4 x = *reinterpret_cast<const float4 *>(&As[buf][r][64 * g + 4 * ti]);
+                const float4 y = *reinterpret_cast<const float4 *>(&Bs[buf][r][64 * g + 4 * tj]);
                 a[4 * g] = x.x, a[4 * g + 1] = x.y, a[4 * g + 2] = x.z, a[4 * g + 3] = x.w;
                 b[4 * g] = y.x, b[4 * g + 1] = y.y, b[4 * g + 2] = y.z, b[4 * g + 3] = y.w;
             }
-            const float cr = Cs[r];
+            const float cr = Cs[buf][r];
 #pragma unroll
             for (int m = 0; m < 4 * G; ++m) {
 #pragma unroll
@@ -618,7 +666,7 @@ causal_chunk_scan(float *__restrict__ E, DecayArgs dec, int has_decay, int H, in
 }
 
 // Forward: the D + 1 columns of [S | z] (z: the column of a value that is always 1).
-template <typename T, int D, bool PHI>
+template <typename T, int D, bool PHI, bool DECAY>
 __global__ void __launch_bounds__(causal_fwd_threads<D>())
 causal_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, T *__restrict__ o,
            const float *__restrict__ st_in, DecayArgs dec, int has_decay, int T_len, int H, int L, float eps) {
@@ -637,11 +685,12 @@ causal_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict
     const T *const src[3] = {q, k, v};
     for (int ts = s0; ts < s1; ts += kRetTile) {
         __syncthreads();
-        load_rows<T, D, 3>(src, tiles, base, ts, T_len, blockDim.x);
+        load_rows<T, D, 3, causal_fwd_threads<D>()>(src, tiles, base, ts, T_len);
         __syncthreads();
         feature_tiles<D, PHI>(tiles, 2);
         __syncthreads();
         const int nr = min(kRetTile, s1 - ts);
+#pragma unroll 2
         for (int r = 0; r < nr; ++r) {
             const float vj = j < D ? tiles[2][r][j] : 1.f;
             float a[4] = {0.f, 0.f, 0.f, 0.f};
@@ -650,7 +699,7 @@ causal_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict
                 const float4 kk = part_group<P>(tiles[1][r], pp, m), qq = part_group<P>(tiles[0][r], pp, m);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    S[4 * m + e] = fmaf(gamma, S[4 * m + e], f4(kk, e) * vj);
+                    S[4 * m + e] = decay_fma<DECAY>(gamma, S[4 * m + e], f4(kk, e), vj);
                     a[e] = fmaf(f4(qq, e), S[4 * m + e], a[e]);
                 }
             }
@@ -670,7 +719,7 @@ causal_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict
 //   df(q)_t[i] = (sum_j S_t[i][j] dout_t[j]) / n_t + z_t[i] dn_t,  dq = df(q) f'(q).
 // The first P (D + 1) threads hold the columns of [S | z] (u_t and n_t), the next P D the
 // rows of S and z[i] (the row sums of dq); a tile's rows meet in shared memory.
-template <typename T, int D, bool PHI>
+template <typename T, int D, bool PHI, bool DECAY>
 __global__ void __launch_bounds__(causal_bwd_q_threads<D>())
 causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
              T *__restrict__ dq, float2 *__restrict__ nd, const float *__restrict__ st_in, DecayArgs dec, int has_decay,
@@ -703,11 +752,12 @@ causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
     const T *const src[4] = {q, k, v, g};
     for (int ts = s0; ts < s1; ts += kRetTile) {
         __syncthreads();
-        load_rows<T, D, 4>(src, tiles, base, ts, T_len, blockDim.x);
+        load_rows<T, D, 4, causal_bwd_q_threads<D>()>(src, tiles, base, ts, T_len);
         __syncthreads();
         feature_tiles<D, PHI>(tiles, 2);
         __syncthreads();
         const int nr = min(kRetTile, s1 - ts);
+#pragma unroll 2
         for (int r = 0; r < nr; ++r) {
             float a[4] = {0.f, 0.f, 0.f, 0.f};
             if (col_side) {
@@ -717,7 +767,7 @@ causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
                     const float4 kk = part_group<P>(tiles[1][r], pp, m), qq = part_group<P>(tiles[0][r], pp, m);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        Sx[4 * m + e] = fmaf(gamma, Sx[4 * m + e], f4(kk, e) * vj);
+                        Sx[4 * m + e] = decay_fma<DECAY>(gamma, Sx[4 * m + e], f4(kk, e), vj);
                         a[e] = fmaf(f4(qq, e), Sx[4 * m + e], a[e]);
                     }
                 }
@@ -728,11 +778,11 @@ causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
                     const float4 vv = part_group<P>(tiles[2][r], pp, m), gg = part_group<P>(tiles[3][r], pp, m);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        Sx[4 * m + e] = fmaf(gamma, Sx[4 * m + e], ki * f4(vv, e));
+                        Sx[4 * m + e] = decay_fma<DECAY>(gamma, Sx[4 * m + e], ki, f4(vv, e));
                         a[e] = fmaf(Sx[4 * m + e], f4(gg, e), a[e]);
                     }
                 }
-                zi = fmaf(gamma, zi, ki);
+                zi = DECAY ? fmaf(gamma, zi, ki) : zi + ki;
             }
             const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
             if (lead) {
@@ -778,7 +828,7 @@ static_assert((6 * kRetTile * 64 + kRetTile * 65) % 2 == 0 && (6 * kRetTile * 12
 // f(q_s) dn_s with du_s = dout_s / n_s: the first P D threads hold the rows of R and r[i]
 // (dk_s[i] = (sum_j R[i][j] v_s[j] + r[i]) f'(k_s[i])), the next P D the columns of R
 // (dv_s[j] = sum_i f(k_s)[i] R[i][j]).
-template <typename T, int D, bool PHI>
+template <typename T, int D, bool PHI, bool DECAY>
 __global__ void __launch_bounds__(causal_bwd_kv_threads<D>())
 causal_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
               const float2 *__restrict__ nd, T *__restrict__ dk, T *__restrict__ dv, const float *__restrict__ st_in,
@@ -807,7 +857,7 @@ causal_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
     const T *const src[4] = {q, k, v, g};
     for (int ts = s0 + (s1 - s0 - 1) / kRetTile * kRetTile; ts >= s0; ts -= kRetTile) {
         __syncthreads();
-        load_rows<T, D, 4>(src, tiles, base, ts, T_len, blockDim.x);
+        load_rows<T, D, 4, causal_bwd_kv_threads<D>()>(src, tiles, base, ts, T_len);
         const int nr = min(kRetTile, s1 - ts);
         if (threadIdx.x < nr) {
             const float2 x = nd[(long long)bh * T_len + ts + threadIdx.x];
@@ -815,7 +865,9 @@ causal_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
         }
         __syncthreads();
         feature_tiles<D, PHI>(tiles, 2);
+        for (int e = threadIdx.x; e < nr * D; e += blockDim.x) tiles[3][e / D][e % D] *= info[e / D].x;   // du
         __syncthreads();
+#pragma unroll 2
         for (int r = nr - 1; r >= 0; --r) {
             const float2 in = info[r];
             float a[4] = {0.f, 0.f, 0.f, 0.f};
@@ -826,19 +878,19 @@ causal_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
                     const float4 gg = part_group<P>(tiles[3][r], pp, m), vv = part_group<P>(tiles[2][r], pp, m);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        Rx[4 * m + e] = fmaf(gamma, Rx[4 * m + e], qi * (f4(gg, e) * in.x));
+                        Rx[4 * m + e] = decay_fma<DECAY>(gamma, Rx[4 * m + e], qi, f4(gg, e));
                         a[e] = fmaf(Rx[4 * m + e], f4(vv, e), a[e]);
                     }
                 }
-                ri = fmaf(gamma, ri, qi * in.y);
+                ri = DECAY ? fmaf(gamma, ri, qi * in.y) : fmaf(qi, in.y, ri);
             } else {
-                const float duj = tiles[3][r][line] * in.x;
+                const float duj = tiles[3][r][line];
 #pragma unroll
                 for (int m = 0; m < DP / 4; ++m) {
                     const float4 qq = part_group<P>(tiles[0][r], pp, m), kk = part_group<P>(tiles[1][r], pp, m);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        Rx[4 * m + e] = fmaf(gamma, Rx[4 * m + e], f4(qq, e) * duj);
+                        Rx[4 * m + e] = decay_fma<DECAY>(gamma, Rx[4 * m + e], f4(qq, e), duj);
                         a[e] = fmaf(f4(kk, e), Rx[4 * m + e], a[e]);
                     }
                 }
@@ -892,11 +944,12 @@ gated_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
     const T *const src[4] = {q, k, v, g};
     for (int ts = 0; ts < T_len; ts += kRetTile) {
         __syncthreads();
-        load_rows<T, D, 4>(src, tiles, base, ts, T_len, blockDim.x);
+        load_rows<T, D, 4, gated_fwd_threads<D>()>(src, tiles, base, ts, T_len);
         __syncthreads();
         exp_tile<D>(tiles[3]);
         __syncthreads();
         const int nr = min(kRetTile, T_len - ts);
+#pragma unroll 2
         for (int r = 0; r < nr; ++r) {
             const float vj = tiles[2][r][j];
             float a[4] = {0.f, 0.f, 0.f, 0.f};
@@ -937,11 +990,12 @@ gated_bwd_q(const T *__restrict__ k, const T *__restrict__ v, const T *__restric
     const T *const src[4] = {k, v, g, dout};
     for (int ts = 0; ts < T_len; ts += kRetTile) {
         __syncthreads();
-        load_rows<T, D, 4>(src, tiles, base, ts, T_len, blockDim.x);
+        load_rows<T, D, 4, gated_fwd_threads<D>()>(src, tiles, base, ts, T_len);
         __syncthreads();
         exp_tile<D>(tiles[2]);
         __syncthreads();
         const int nr = min(kRetTile, T_len - ts);
+#pragma unroll 2
         for (int r = 0; r < nr; ++r) {
             const float ai = tiles[2][r][i], ki = tiles[0][r][i];
             float a[4] = {0.f, 0.f, 0.f, 0.f};
@@ -998,11 +1052,12 @@ gated_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
     for (int tile = ntiles - 1; tile >= 0; --tile) {
         const int ts = tile * kRetTile;
         __syncthreads();
-        load_rows<T, D, 5>(src, tiles, base, ts, T_len, blockDim.x);
+        load_rows<T, D, 5, gated_kv_threads<D>()>(src, tiles, base, ts, T_len);
         __syncthreads();
         exp_tile<D>(tiles[4]);
         __syncthreads();
         const int nr = min(kRetTile, T_len - ts);
+#pragma unroll 2
         for (int r = nr - 1; r >= 0; --r) {
             const float *an = r + 1 < nr ? tiles[4][r + 1] : anext;    // a_{t+1}
             float a[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1318,9 +1373,10 @@ la_status causal_fwd_t(const void *q, const void *k, const void *v, void *o, con
         const la_status rc = causal_states<T, D, PHI, false>(k, v, nullptr, E, dec, has_decay, s, st);
         if (rc) return rc;
     }
-    return launch("simt_causal_norm_fwd", causal_fwd<T, D, PHI>, dim3((unsigned)s.BH(), (unsigned)nc),
-                  dim3(causal_fwd_threads<D>()), 0, st, (const T *)q, (const T *)k, (const T *)v, (T *)o,
-                  (const float *)E, dec, has_decay, s.T, s.H, kCausalChunk, eps);
+    const auto kern = has_decay ? causal_fwd<T, D, PHI, true> : causal_fwd<T, D, PHI, false>;
+    return launch("simt_causal_norm_fwd", kern, dim3((unsigned)s.BH(), (unsigned)nc), dim3(causal_fwd_threads<D>()), 0,
+                  st, (const T *)q, (const T *)k, (const T *)v, (T *)o, (const float *)E, dec, has_decay, s.T, s.H,
+                  kCausalChunk, eps);
 }
 
 template <typename T, int D, bool PHI>
@@ -1332,15 +1388,17 @@ la_status causal_bwd_t(const void *q, const void *k, const void *v, const void *
     const dim3 grid((unsigned)s.BH(), (unsigned)nc);
     la_status rc;
     if (E && (rc = causal_states<T, D, PHI, false>(k, v, nullptr, E, dec, has_decay, s, st))) return rc;
-    rc = launch("simt_causal_norm_bwd_q", causal_bwd_q<T, D, PHI>, grid, dim3(causal_bwd_q_threads<D>()),
-                causal_bwd_q_smem<D>(), st, (const T *)q, (const T *)k, (const T *)v, (const T *)g, (T *)dq, nd,
-                (const float *)E, dec, has_decay, s.T, s.H, kCausalChunk, eps);
+    const auto kq = has_decay ? causal_bwd_q<T, D, PHI, true> : causal_bwd_q<T, D, PHI, false>;
+    const auto kkv = has_decay ? causal_bwd_kv<T, D, PHI, true> : causal_bwd_kv<T, D, PHI, false>;
+    rc = launch("simt_causal_norm_bwd_q", kq, grid, dim3(causal_bwd_q_threads<D>()), causal_bwd_q_smem<D>(), st,
+                (const T *)q, (const T *)k, (const T *)v, (const T *)g, (T *)dq, nd, (const float *)E, dec, has_decay,
+                s.T, s.H, kCausalChunk, eps);
     if (rc) return rc;
     // the reverse states need every row's (n, dn) from the dq pass; they reuse the forward's buffer
     if (E && (rc = causal_states<T, D, PHI, true>(q, g, nd, E, dec, has_decay, s, st))) return rc;
-    return launch("simt_causal_norm_bwd_kv", causal_bwd_kv<T, D, PHI>, grid, dim3(causal_bwd_kv_threads<D>()),
-                  causal_bwd_kv_smem<D>(), st, (const T *)q, (const T *)k, (const T *)v, (const T *)g,
-                  (const float2 *)nd, (T *)dk, (T *)dv, (const float *)E, dec, has_decay, s.T, s.H, kCausalChunk);
+    return launch("simt_causal_norm_bwd_kv", kkv, grid, dim3(causal_bwd_kv_threads<D>()), causal_bwd_kv_smem<D>(), st,
+                  (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const float2 *)nd, (T *)dk, (T *)dv,
+                  (const float *)E, dec, has_decay, s.T, s.H, kCausalChunk);
 }
 
 // dtype x D x feature map dispatch of F<T, D, PHI>(args...)
