@@ -421,7 +421,7 @@ def run_ours(args, w):
             la.la_causal_norm_fwd(q, k, v, o, None, "elu1", w.eps, workspace=ws)
             la.la_causal_norm_bwd(q, k, v, g, dq, dk, dv, None, "elu1", w.eps, workspace=ws)
         elif gated:
-            la.la_gated_fwd(q, k, v, lgate, o)
+            la.la_gated_fwd(q, k, v, lgate, o, workspace=ws)
             la.la_gated_bwd(q, k, v, lgate, g, dq, dk, dv, dgate, workspace=ws)
         else:
             la.la_chunk_decay_fwd(q, k, v, o, gamma, workspace=ws)
@@ -520,7 +520,7 @@ def run_ours(args, w):
             la.la_causal_norm_fwd(xq, xk, xv, xo, None, "elu1", w.eps, workspace=ws, stream=s_cmp)
             la.la_causal_norm_bwd(xq, xk, xv, xg, xdq, xdk, xdv, None, "elu1", w.eps, workspace=ws, stream=s_cmp)
         elif gated:
-            la.la_gated_fwd(xq, xk, xv, ins[4], xo, stream=s_cmp)
+            la.la_gated_fwd(xq, xk, xv, ins[4], xo, workspace=ws, stream=s_cmp)
             la.la_gated_bwd(xq, xk, xv, ins[4], xg, xdq, xdk, xdv, outs[4], workspace=ws, stream=s_cmp)
         else:
             la.la_chunk_decay_fwd(xq, xk, xv, xo, gamma, workspace=ws, stream=s_cmp)

@@ -280,16 +280,23 @@ la_status la_causal_norm_bwd(const void *q, const void *k, const void *v, const 
  *   S_t = diag(exp(g_t)) S_{t-1} + k_t^T v_t,  o_t = q_t S_t,
  * g [B,H,T,D] the log gates (g <= 0 decays; dtype as q).  With g_t = log gamma_h
  * for every t and dimension this is la_chunk_decay_*.  The recurrent form
- * ("Different forms of linear attention": FusedRecurrent) on CUDA cores, fp32,
- * one CTA per (b, h); every dtype, D in {64, 128}; no workspace. */
+ * ("Different forms of linear attention": FusedRecurrent) on CUDA cores, fp32;
+ * every dtype, D in {64, 128}.  As la_causal_norm_*, the sequence is cut into
+ * chunks of 256 tokens, each walked by its own CTA from the state the chunks
+ * before it leave (a chunk's own state and its gate product per key dimension,
+ * then a scan over the chunks).
+ * Workspace: la_workspace_size(LA_OP_GATED_FWD, ...) bytes (the chunk states and
+ * gate products; 0, NULL allowed, for T <= 256). */
 la_status la_gated_fwd(const void *q, const void *k, const void *v, const void *g, void *o,
-                       int B, int H, int T, int D, la_dtype dtype, void *stream);
+                       int B, int H, int T, int D, la_dtype dtype,
+                       void *workspace, size_t workspace_bytes, void *stream);
 
 /* Gradients of sum(o * dout): dq_t = S_t dout_t, and with
  * R_t = q_t^T dout_t + diag(exp(g_{t+1})) R_{t+1}: dk_t = R_t v_t, dv_t = k_t R_t;
  * dg_t = sum_{s>=t} (q_s dq_s - k_s dk_s) (elementwise, in fp32 from the unrounded
  * dq and dk).  Workspace: la_workspace_size(LA_OP_GATED_BWD, ...) bytes (dq in
- * fp32, 4 B per element). */
+ * fp32, 4 B per element, in which the reverse sweep leaves each chunk's part of
+ * dg; then the chunk states, gate products and per-chunk dg totals). */
 la_status la_gated_bwd(const void *q, const void *k, const void *v, const void *g, const void *dout,
                        void *dq, void *dk, void *dv, void *dg,
                        int B, int H, int T, int D, la_dtype dtype,

@@ -58,7 +58,7 @@ _lib.la_chunk_decay_fwd_state.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I
 _lib.la_chunk_decay_bwd_state.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z,
                                           _P]
 _lib.la_chunk_decay_scan.argtypes = [_P, _P, _I, _P, _P, _I, _I, _I, _P]
-_lib.la_gated_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
+_lib.la_gated_fwd.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_gated_bwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]
 _lib.la_feature_map_fwd.argtypes = [_I, _F, _P, _P, _I, _I, _I, _I, _I, _P]
 _lib.la_feature_map_bwd.argtypes = [_I, _F, _P, _P, _P, _I, _I, _I, _I, _I, _P]
@@ -315,11 +315,13 @@ def _decay_or_null(decay, H):
     return (None, None) if decay is None else (lambda a: (ctypes.cast(a, _P), a))(_decay(decay, H))
 
 
-def la_gated_fwd(q, k, v, g, o, stream=None):
+def la_gated_fwd(q, k, v, g, o, workspace=None, stream=None):
     """Gated linear attention: S_t = diag(exp(g_t)) S_{t-1} + k_t^T v_t, o_t <- q_t S_t; g holds the
     log gates, [B, H, T, D] like q."""
     B, H, T, D = _shape(q, k, v, g, o)
-    _check(_lib.la_gated_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), B, H, T, D, _dtype_code(q),
+    dt = _dtype_code(q)
+    wp, wn, _keep = _workspace("gated_fwd", (B, H, T, D), dt, workspace, q.device, stream)
+    _check(_lib.la_gated_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), B, H, T, D, dt, wp, wn,
                              _stream(stream, q.device)), "la_gated_fwd")
 
 

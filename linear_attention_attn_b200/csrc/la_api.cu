@@ -475,7 +475,7 @@ la_status la_feature_map_bwd(la_fmap kind, float p, const void *x, const void *d
 }
 
 la_status la_gated_fwd(const void *q, const void *k, const void *v, const void *g, void *o, int B, int H, int T,
-                       int D, la_dtype dtype, void *stream) {
+                       int D, la_dtype dtype, void *workspace, size_t workspace_bytes, void *stream) {
     const Shape s{B, H, T, D};
     LA_TRY(validate(s, dtype));
     LA_TRY(check_ptr(q, "q"));
@@ -483,8 +483,9 @@ la_status la_gated_fwd(const void *q, const void *k, const void *v, const void *
     LA_TRY(check_ptr(v, "v"));
     LA_TRY(check_ptr(g, "g"));
     LA_TRY(check_ptr(o, "o"));
+    LA_TRY(check_ws(LA_OP_GATED_FWD, s, dtype, workspace, workspace_bytes));
     if (T == 0) return LA_OK;
-    return simt::gated_fwd(q, k, v, g, o, s, dtype, (cudaStream_t)stream);
+    return simt::gated_fwd(q, k, v, g, o, s, dtype, workspace, (cudaStream_t)stream);
 }
 
 la_status la_gated_bwd(const void *q, const void *k, const void *v, const void *g, const void *dout, void *dq,

@@ -162,7 +162,7 @@ la_status causal_norm_bwd(const void *q, const void *k, const void *v, const voi
                           void *ws, cudaStream_t st);
 // Gated linear attention (log gates g, the decay exp(g) per token and key dimension).
 la_status gated_fwd(const void *q, const void *k, const void *v, const void *g, void *o, const Shape &s, la_dtype dt,
-                    cudaStream_t st);
+                    void *ws, cudaStream_t st);
 la_status gated_bwd(const void *q, const void *k, const void *v, const void *g, const void *dout, void *dq, void *dk,
                     void *dv, void *dg, const Shape &s, la_dtype dt, void *ws, cudaStream_t st);
 }  // namespace simt

@@ -24,7 +24,7 @@ namespace simt {
 constexpr int kTile = 32;      // rows per shared-memory tile
 constexpr int kRetTile = 16;   // rows per tile in the recurrent (retention) kernels
 constexpr int kThreads = 256;
-constexpr int kCausalChunk = 256;   // tokens per chunk of the causal-norm kernels (a multiple of kRetTile)
+constexpr int kCausalChunk = 256;   // tokens per chunk of the causal-norm and gated kernels (whole tiles)
 static_assert(kCausalChunk % kRetTile == 0, "chunks hold whole recurrent tiles");
 
 inline int causal_chunks(int T_len) { return T_len <= kCausalChunk ? 1 : (T_len + kCausalChunk - 1) / kCausalChunk; }
@@ -35,6 +35,15 @@ inline size_t nd_bytes(const Shape &s) { return round256((size_t)s.BH() * s.T * 
 inline size_t causal_state_bytes(const Shape &s) {
     const int nc = causal_chunks(s.T);
     return nc > 1 ? round256((size_t)s.BH() * nc * s.D * (s.D + 1) * sizeof(float)) : 0;
+}
+// gated: dq in fp32; the [B H][chunk][D][D] states and the [B H][chunk][D] factors (or totals)
+inline size_t dq32_bytes(const Shape &s) { return round256((size_t)s.BH() * s.T * s.D * sizeof(float)); }
+inline size_t gated_e_bytes(const Shape &s) {
+    return round256((size_t)s.BH() * causal_chunks(s.T) * s.D * s.D * sizeof(float));
+}
+inline size_t gated_a_bytes(const Shape &s) { return round256((size_t)s.BH() * causal_chunks(s.T) * s.D * sizeof(float)); }
+inline size_t gated_state_bytes(const Shape &s) {
+    return causal_chunks(s.T) > 1 ? gated_e_bytes(s) + gated_a_bytes(s) : 0;
 }
 
 // ------------------------------------------------------------ reductions --
@@ -483,10 +492,11 @@ ret_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
 // are never read).
 template <int D, bool PHI>
 __device__ __forceinline__ void feature_tiles(float (*tiles)[kRetTile][D], int n) {
-    if (!PHI) return;
-    for (int e = threadIdx.x; e < n * kRetTile * D; e += blockDim.x) {
-        float *x = &tiles[e / (kRetTile * D)][(e / D) % kRetTile][e % D];
-        *x = feature(*x);
+    if (PHI) {
+        for (int e = threadIdx.x; e < n * kRetTile * D; e += blockDim.x) {
+            float *x = &tiles[e / (kRetTile * D)][(e / D) % kRetTile][e % D];
+            *x = feature(*x);
+        }
     }
 }
 // f'(x) from f(x): elu + 1 is x + 1 > 1 for x > 0 (slope 1) and exp(x) <= 1 otherwise.
@@ -534,9 +544,9 @@ __device__ __forceinline__ float decay_fma(float gamma, float s, float x, float 
 // state from a zero state (a sum of weighted outer products, no recurrence), then a scan over
 // the chunks of one head:  S_in[c] = gamma^L S_in[c-1] + E[c-1]  (reverse: from the last chunk).
 // States are [B H][chunk][D][D + 1] fp32, the last column z (forward) or r (reverse).
-template <int D>
+template <int D, int W = D + 1>
 __device__ __forceinline__ const float *chunk_state(const float *st, int bh, int c) {
-    return st ? st + ((long long)bh * gridDim.y + c) * D * (D + 1) : nullptr;
+    return st ? st + ((long long)bh * gridDim.y + c) * D * W : nullptr;
 }
 
 // token rows per shared-memory tile of causal_chunk_state (two buffers of a and b rows: 32 KB)
@@ -648,20 +658,36 @@ causal_chunk_state(const T *__restrict__ a_src, const T *__restrict__ b_src, con
 }
 
 // In place over the nc chunk states of each head: the state entering chunk c (forward) or the
-// reverse state entering it from the chunks after it (REV).  Every chunk but the last (REV: the
-// first) has L tokens; the state of the last chunk visited is never read.
+// reverse state entering it from the chunks after it (rev), in chunk order:
+//   run <- f_c run + own_c,  f_c = A[c][i] for a state row i (gated), else gamma^L.
+// Every chunk but the last (rev: the first) has L tokens; the state of the last chunk visited
+// is never read.  States hold per_head values, rows of row_len.
 __global__ void __launch_bounds__(256)
-causal_chunk_scan(float *__restrict__ E, DecayArgs dec, int has_decay, int H, int nc, int per_head, int L, int rev) {
+chunk_scan(float *__restrict__ E, const float *__restrict__ A, DecayArgs dec, int has_decay, int H, int nc,
+           int per_head, int row_len, int L, int rev) {
     const int bh = blockIdx.y, e = blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= per_head) return;
-    const float f = has_decay ? (float)pow((double)dec.gamma[bh % H], (double)L) : 1.f;
+    const int rows = per_head / row_len, i = e / row_len;
+    const float fl = has_decay ? (float)pow((double)dec.gamma[bh % H], (double)L) : 1.f;
     float *p = E + (long long)bh * nc * per_head + e;
     float run = 0.f;
-    for (int i = 0; i < nc; ++i) {
-        const long long at = (long long)(rev ? nc - 1 - i : i) * per_head;
-        const float own = i == nc - 1 ? 0.f : p[at];
-        p[at] = run;
-        run = fmaf(f, run, own);
+    constexpr int kBatch = 8;                  // chunks whose loads are in flight together
+    for (int n0 = 0; n0 < nc; n0 += kBatch) {
+        float own[kBatch], f[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int n = n0 + u, c = rev ? nc - 1 - n : n;
+            own[u] = n < nc - 1 ? p[(long long)c * per_head] : 0.f;
+            f[u] = !A || n >= nc ? fl : A[((long long)bh * nc + c) * rows + i];
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int n = n0 + u, c = rev ? nc - 1 - n : n;
+            if (n < nc) {
+                p[(long long)c * per_head] = run;
+                run = fmaf(f[u], run, own[u]);
+            }
+        }
     }
 }
 
@@ -926,29 +952,152 @@ __device__ __forceinline__ void exp_tile(float (*tile)[D]) {
 template <int D> constexpr int gated_fwd_threads() { return causal_split<D>() * D; }
 template <int D> constexpr int gated_kv_threads() { return 2 * causal_split<D>() * D; }
 
+// ---- chunks along T, as for the causal-norm kernels.  A chunk's own state from a zero state
+// weights each token by the product of the gates between it and the chunk's end (forward) or
+// start (reverse), exp of a running sum of log gates per key dimension i:
+//   forward (REV false): E[c][i][j] = sum_t exp(sum_{u=t+1}^{s1-1} g_u[i]) k_t[i] v_t[j],
+//     A[c][i] = exp(sum_{u=s0}^{s1-1} g_u[i])   (S after the chunk = diag(A) S before + E);
+//   reverse (REV true):  E[c][i][j] = sum_t exp(sum_{u=s0+1}^{t} g_u[i]) q_t[i] dout_t[j],
+//     A[c][i] = exp(sum_{u=s0+1}^{s1} g_u[i])   (R at s0 = E + diag(A) R at s1; no g past T).
+// E is [B H][chunk][D][D], A [B H][chunk][D]; threads < D form the weights of column i, all
+// 256 accumulate rows 4 ti + 64 m + 0..3 by columns 4 tj + 64 n + 0..3 as causal_chunk_state.
+template <typename T, int D, bool REV>
+__global__ void __launch_bounds__(256)
+gated_chunk_state(const T *__restrict__ a_src, const T *__restrict__ b_src, const T *__restrict__ g,
+                  float *__restrict__ E, float *__restrict__ A, int T_len, int L) {
+    constexpr int G = D / 64, R = chunk_state_rows<D>();
+    __shared__ __align__(16) float As[R][D];
+    __shared__ __align__(16) float Bs[R][D];
+    __shared__ float Gs[R][D];
+    const int c = blockIdx.x, bh = blockIdx.y, nc = gridDim.x;
+    if (REV ? c == 0 : c == nc - 1) return;    // no other chunk starts from this one's state
+    const int s0 = c * L, s1 = min(T_len, s0 + L), ntiles = (s1 - s0 + R - 1) / R;
+    const long long base = (long long)bh * T_len * D;
+    const int tj = threadIdx.x & 15, ti = threadIdx.x >> 4;
+    float acc[4 * G][4 * G];
+#pragma unroll
+    for (int m = 0; m < 4 * G; ++m)
+#pragma unroll
+        for (int n = 0; n < 4 * G; ++n) acc[m][n] = 0.f;
+    float run = 0.f;                           // thread i < D: the running sum of log gates
+    // the tiles in the order they are summed (forward: from the chunk's end), each fetched into
+    // registers while the one before it is weighted and summed
+    constexpr int EPT = R * D / 256;
+    float ra[EPT], rb[EPT], rg[EPT];
+    const T *const a_h = a_src + base, *const b_h = b_src + base, *const g_h = g + base;
+#define LA_GATED_FETCH(N_)                                                              \
+    do {                                                                                \
+        const int ts_ = s0 + (REV ? (N_) : ntiles - 1 - (N_)) * R, nr_ = min(R, s1 - ts_); \
+        _Pragma("unroll") for (int u = 0; u < EPT; ++u) {                               \
+            const int e = threadIdx.x + 256 * u, r = e / D;                             \
+            const long long at = (long long)(ts_ + r) * D + e % D;                      \
+            ra[u] = r < nr_ ? io<T>::ld(a_h + at) : 0.f;                                \
+            rb[u] = r < nr_ ? io<T>::ld(b_h + at) : 0.f;                                \
+            rg[u] = r < nr_ ? io<T>::ld(g_h + at) : 0.f;                                \
+        }                                                                               \
+    } while (0)
+    LA_GATED_FETCH(0);
+    for (int n = 0; n < ntiles; ++n) {
+        const int ts = s0 + (REV ? n : ntiles - 1 - n) * R, nr = min(R, s1 - ts);
+        __syncthreads();                       // the previous tile is summed
+#pragma unroll
+        for (int u = 0; u < EPT; ++u) {
+            const int e = threadIdx.x + 256 * u;
+            As[e / D][e % D] = ra[u];
+            Bs[e / D][e % D] = rb[u];
+            Gs[e / D][e % D] = rg[u];
+        }
+        __syncthreads();
+        if (n + 1 < ntiles) LA_GATED_FETCH(n + 1);
+        if (threadIdx.x < D) {
+            const int i = threadIdx.x;
+            if (REV) {
+                for (int r = 0; r < nr; ++r) {
+                    if (ts + r > s0) run += Gs[r][i];
+                    As[r][i] *= expf(run);
+                }
+            } else {
+                for (int r = nr - 1; r >= 0; --r) {
+                    As[r][i] *= expf(run);
+                    run += Gs[r][i];
+                }
+            }
+        }
+        __syncthreads();
+        for (int r = 0; r < nr; ++r) {
+            float a[4 * G], b[4 * G];
+#pragma unroll
+            for (int gq = 0; gq < G; ++gq) {
+                const float4 x = *reinterpret_cast<const float4 *>(&As[r][64 * gq + 4 * ti]);
+                const float4 y = *reinterpret_cast<const float4 *>(&Bs[r][64 * gq + 4 * tj]);
+                a[4 * gq] = x.x, a[4 * gq + 1] = x.y, a[4 * gq + 2] = x.z, a[4 * gq + 3] = x.w;
+                b[4 * gq] = y.x, b[4 * gq + 1] = y.y, b[4 * gq + 2] = y.z, b[4 * gq + 3] = y.w;
+            }
+#pragma unroll
+            for (int m = 0; m < 4 * G; ++m)
+#pragma unroll
+                for (int n2 = 0; n2 < 4 * G; ++n2) acc[m][n2] = fmaf(a[m], b[n2], acc[m][n2]);
+        }
+    }
+#undef LA_GATED_FETCH
+    float *out = E + ((long long)bh * nc + c) * D * D;
+#pragma unroll
+    for (int m = 0; m < 4 * G; ++m) {
+        const int i = 64 * (m / 4) + 4 * ti + m % 4;
+#pragma unroll
+        for (int n = 0; n < 4 * G; ++n) out[i * D + 64 * (n / 4) + 4 * tj + n % 4] = acc[m][n];
+    }
+    if (threadIdx.x < D) {
+        const float next = REV && s1 < T_len ? io<T>::ld(g + base + (long long)s1 * D + threadIdx.x) : 0.f;
+        A[((long long)bh * nc + c) * D + threadIdx.x] = expf(run + next);
+    }
+}
+
+// dg of a sequence cut into chunks: each chunk's part (fp32, summed over its own rows from the
+// end) plus the totals of the chunks after it.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+gated_dg_carry(const float *__restrict__ part, const float *__restrict__ totals, T *__restrict__ dg, int T_len,
+               int L) {
+    __shared__ float carry[D];
+    const int c = blockIdx.x, bh = blockIdx.y, nc = gridDim.x;
+    if (threadIdx.x < D) {
+        float sum = 0.f;
+        for (int c2 = nc - 1; c2 > c; --c2) sum += totals[((long long)bh * nc + c2) * D + threadIdx.x];
+        carry[threadIdx.x] = sum;
+    }
+    __syncthreads();
+    const int s0 = c * L, s1 = min(T_len, s0 + L);
+    const long long base = (long long)bh * T_len * D;
+    for (long long e = (long long)s0 * D + threadIdx.x; e < (long long)s1 * D; e += blockDim.x)
+        io<T>::st(dg + base + e, part[base + e] + carry[e % D]);
+}
+
 // Forward: the D columns of S; thread p of column j holds S[i][j] for its D / P rows
 // i = part_entry(p, .).
 template <typename T, int D>
 __global__ void __launch_bounds__(gated_fwd_threads<D>())
 gated_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
-          T *__restrict__ o, int T_len) {
+          T *__restrict__ o, const float *__restrict__ st_in, int T_len, int L) {
     constexpr int P = causal_split<D>(), DP = D / P;
     __shared__ __align__(16) float tiles[4][kRetTile][D];      // q, k, v, a = exp(g)
     __shared__ float acc[kRetTile][D];
+    const int s0 = blockIdx.y * L, s1 = min(T_len, s0 + L);
     const long long base = (long long)blockIdx.x * T_len * D;
     const int j = threadIdx.x / P, pp = threadIdx.x % P;
     const bool lead = pp == 0;
+    const float *const S0 = chunk_state<D, D>(st_in, blockIdx.x, blockIdx.y);
     float S[DP];
 #pragma unroll
-    for (int i = 0; i < DP; ++i) S[i] = 0.f;
+    for (int i = 0; i < DP; ++i) S[i] = S0 ? S0[part_entry<P>(pp, i) * D + j] : 0.f;
     const T *const src[4] = {q, k, v, g};
-    for (int ts = 0; ts < T_len; ts += kRetTile) {
+    for (int ts = s0; ts < s1; ts += kRetTile) {
         __syncthreads();
         load_rows<T, D, 4, gated_fwd_threads<D>()>(src, tiles, base, ts, T_len);
         __syncthreads();
         exp_tile<D>(tiles[3]);
         __syncthreads();
-        const int nr = min(kRetTile, T_len - ts);
+        const int nr = min(kRetTile, s1 - ts);
 #pragma unroll 2
         for (int r = 0; r < nr; ++r) {
             const float vj = tiles[2][r][j];
@@ -977,24 +1126,26 @@ gated_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict_
 template <typename T, int D>
 __global__ void __launch_bounds__(gated_fwd_threads<D>())
 gated_bwd_q(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g, const T *__restrict__ dout,
-            T *__restrict__ dq, float *__restrict__ dq32, int T_len) {
+            T *__restrict__ dq, float *__restrict__ dq32, const float *__restrict__ st_in, int T_len, int L) {
     constexpr int P = causal_split<D>(), DP = D / P;
     __shared__ __align__(16) float tiles[4][kRetTile][D];      // k, v, a = exp(g), dout
     __shared__ float acc[kRetTile][D];
+    const int s0 = blockIdx.y * L, s1 = min(T_len, s0 + L);
     const long long base = (long long)blockIdx.x * T_len * D;
     const int i = threadIdx.x / P, pp = threadIdx.x % P;
     const bool lead = pp == 0;
+    const float *const S0 = chunk_state<D, D>(st_in, blockIdx.x, blockIdx.y);
     float S[DP];
 #pragma unroll
-    for (int jj = 0; jj < DP; ++jj) S[jj] = 0.f;
+    for (int jj = 0; jj < DP; ++jj) S[jj] = S0 ? S0[i * D + part_entry<P>(pp, jj)] : 0.f;
     const T *const src[4] = {k, v, g, dout};
-    for (int ts = 0; ts < T_len; ts += kRetTile) {
+    for (int ts = s0; ts < s1; ts += kRetTile) {
         __syncthreads();
         load_rows<T, D, 4, gated_fwd_threads<D>()>(src, tiles, base, ts, T_len);
         __syncthreads();
         exp_tile<D>(tiles[2]);
         __syncthreads();
-        const int nr = min(kRetTile, T_len - ts);
+        const int nr = min(kRetTile, s1 - ts);
 #pragma unroll 2
         for (int r = 0; r < nr; ++r) {
             const float ai = tiles[2][r][i], ki = tiles[0][r][i];
@@ -1030,33 +1181,44 @@ gated_bwd_q(const T *__restrict__ k, const T *__restrict__ v, const T *__restric
 template <typename T, int D>
 __global__ void __launch_bounds__(gated_kv_threads<D>())
 gated_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
-             const T *__restrict__ dout, const float *__restrict__ dq32, T *__restrict__ dk, T *__restrict__ dv,
-             T *__restrict__ dg, int T_len) {
+             const T *__restrict__ dout, float *__restrict__ dq32, T *__restrict__ dk, T *__restrict__ dv,
+             T *__restrict__ dg, const float *__restrict__ st_in, float *__restrict__ totals, int T_len, int L) {
     constexpr int P = causal_split<D>(), DP = D / P;
     extern __shared__ __align__(16) float dsm[];   // gated_bwd_kv_smem<D>() bytes
     float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // q, k, v, dout, a = exp(g)
     float(*res)[kRetTile][D] = tiles + 5;        // dk (rows), dv (columns)
     float *anext = dsm + 7 * kRetTile * D;       // a of the row after the tile (0 past the sequence)
+    const int s0 = blockIdx.y * L, s1 = min(T_len, s0 + L);
     const long long base = (long long)blockIdx.x * T_len * D;
     const bool row_side = threadIdx.x < P * D;
     const int t2 = row_side ? threadIdx.x : threadIdx.x - P * D;
     const int line = t2 / P, pp = t2 % P;
     const bool lead = pp == 0;
+    // the entering R (the tokens after this chunk): rows on the row side, columns on the other
+    const float *const R0 = chunk_state<D, D>(st_in, blockIdx.x, blockIdx.y);
     float Rx[DP];
-    float accg = 0.f;                            // thread i < D: sum over the rows after t of dL/dG[i]
+    float accg = 0.f;                            // thread i < D: sum over the chunk's rows after t of dL/dG[i]
 #pragma unroll
-    for (int m = 0; m < DP; ++m) Rx[m] = 0.f;
-    for (int e = threadIdx.x; e < D; e += blockDim.x) anext[e] = 0.f;
+    for (int m = 0; m < DP; ++m) {
+        const int x = part_entry<P>(pp, m);
+        Rx[m] = !R0 ? 0.f : row_side ? R0[line * D + x] : R0[x * D + line];
+    }
+    for (int e = threadIdx.x; e < D; e += blockDim.x)     // the first gate after the chunk
+        anext[e] = s1 < T_len ? expf(io<T>::ld(g + base + (long long)s1 * D + e)) : 0.f;
     const T *const src[5] = {q, k, v, dout, g};
-    const int ntiles = (T_len + kRetTile - 1) / kRetTile;
-    for (int tile = ntiles - 1; tile >= 0; --tile) {
-        const int ts = tile * kRetTile;
+    for (int ts = s0 + (s1 - s0 - 1) / kRetTile * kRetTile; ts >= s0; ts -= kRetTile) {
         __syncthreads();
         load_rows<T, D, 5, gated_kv_threads<D>()>(src, tiles, base, ts, T_len);
         __syncthreads();
         exp_tile<D>(tiles[4]);
         __syncthreads();
-        const int nr = min(kRetTile, T_len - ts);
+        const int nr = min(kRetTile, s1 - ts);
+        float dqv[kRetTile];                     // thread i < D: this tile's dq32[., i], loaded during the sweep
+        if (threadIdx.x < D) {
+#pragma unroll
+            for (int r = 0; r < kRetTile; ++r)
+                dqv[r] = r < nr ? dq32[base + (long long)(ts + r) * D + threadIdx.x] : 0.f;
+        }
 #pragma unroll 2
         for (int r = nr - 1; r >= 0; --r) {
             const float *an = r + 1 < nr ? tiles[4][r + 1] : anext;    // a_{t+1}
@@ -1096,15 +1258,21 @@ gated_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
         }
         if (threadIdx.x < D) {
             const int i = threadIdx.x;
-            for (int r = nr - 1; r >= 0; --r) {
+#pragma unroll
+            for (int r = kRetTile - 1; r >= 0; --r) {
+                if (r >= nr) continue;
                 const long long at = base + (long long)(ts + r) * D + i;
-                accg = fmaf(tiles[0][r][i], dq32[at], accg);
+                accg = fmaf(tiles[0][r][i], dqv[r], accg);
                 accg = fmaf(-tiles[1][r][i], res[0][r][i], accg);
-                io<T>::st(dg + at, accg);
+                // one chunk: dg itself; several: the chunk's part in fp32, in place of dq32
+                // (this thread's own element, read just above), completed by gated_dg_carry
+                if (totals) dq32[at] = accg;
+                else io<T>::st(dg + at, accg);
             }
         }
         for (int e = threadIdx.x; e < D; e += blockDim.x) anext[e] = tiles[4][0][e];
     }
+    if (totals && threadIdx.x < D) totals[((long long)blockIdx.x * gridDim.y + blockIdx.y) * D + threadIdx.x] = accg;
 }
 
 template <int D>
@@ -1286,8 +1454,10 @@ size_t workspace_size(la_op op, const Shape &s) {
         return causal_state_bytes(s);
     case LA_OP_CAUSAL_NORM_BWD:   // (n_t, dn_t) of every row, then the chunk states
         return nd_bytes(s) + causal_state_bytes(s);
-    case LA_OP_GATED_BWD:         // dq in fp32, for the log gates' gradient
-        return ((size_t)s.BH() * s.T * s.D * sizeof(float) + 255) / 256 * 256;
+    case LA_OP_GATED_FWD:         // the chunk states and factors
+        return gated_state_bytes(s);
+    case LA_OP_GATED_BWD:         // dq in fp32 for the log gates' gradient, the chunk states, factors, totals
+        return dq32_bytes(s) + gated_state_bytes(s) + (causal_chunks(s.T) > 1 ? gated_a_bytes(s) : 0);
     default:
         return 0;
     }
@@ -1360,8 +1530,8 @@ la_status causal_states(const void *a, const void *b, const float2 *nd, float *E
                           causal_chunk_state<T, D, PHI, REV>, dim3((unsigned)nc, (unsigned)s.BH()), dim3(256), 0, st,
                           (const T *)a, (const T *)b, nd, E, dec, has_decay, s.T, s.H, kCausalChunk);
     if (rc) return rc;
-    return launch("simt_causal_norm_scan", causal_chunk_scan, dim3((unsigned)((per_head + 255) / 256), (unsigned)s.BH()),
-                  dim3(256), 0, st, E, dec, has_decay, s.H, nc, per_head, kCausalChunk, (int)REV);
+    return launch("simt_chunk_scan", chunk_scan, dim3((unsigned)((per_head + 255) / 256), (unsigned)s.BH()), dim3(256),
+                  0, st, E, (const float *)nullptr, dec, has_decay, s.H, nc, per_head, D + 1, kCausalChunk, (int)REV);
 }
 
 template <typename T, int D, bool PHI>
@@ -1433,24 +1603,56 @@ la_status causal_norm_bwd(const void *q, const void *k, const void *v, const voi
 
 namespace {
 
+// The gated chunk states and factors of every head, scanned in place.
+template <typename T, int D, bool REV>
+la_status gated_states(const void *a, const void *b, const void *g, float *E, float *A, const Shape &s,
+                       cudaStream_t st) {
+    const int nc = causal_chunks(s.T);
+    la_status rc = launch(REV ? "simt_gated_state_rev" : "simt_gated_state", gated_chunk_state<T, D, REV>,
+                          dim3((unsigned)nc, (unsigned)s.BH()), dim3(256), 0, st, (const T *)a, (const T *)b,
+                          (const T *)g, E, A, s.T, kCausalChunk);
+    if (rc) return rc;
+    return launch("simt_chunk_scan", chunk_scan, dim3((unsigned)((D * D + 255) / 256), (unsigned)s.BH()), dim3(256), 0,
+                  st, E, (const float *)A, DecayArgs{}, 0, s.H, nc, D * D, D, kCausalChunk, (int)REV);
+}
+
 template <typename T, int D>
-la_status gated_fwd_t(const void *q, const void *k, const void *v, const void *g, void *o, const Shape &s,
+la_status gated_fwd_t(const void *q, const void *k, const void *v, const void *g, void *o, const Shape &s, void *ws,
                       cudaStream_t st) {
-    return launch("simt_gated_fwd", gated_fwd<T, D>, dim3((unsigned)s.BH()), dim3(gated_fwd_threads<D>()), 0, st,
-                  (const T *)q, (const T *)k, (const T *)v, (const T *)g, (T *)o, s.T);
+    const int nc = causal_chunks(s.T);
+    float *E = nc > 1 ? (float *)ws : nullptr;
+    float *A = E ? (float *)((char *)ws + gated_e_bytes(s)) : nullptr;
+    if (E) {
+        const la_status rc = gated_states<T, D, false>(k, v, g, E, A, s, st);
+        if (rc) return rc;
+    }
+    return launch("simt_gated_fwd", gated_fwd<T, D>, dim3((unsigned)s.BH(), (unsigned)nc), dim3(gated_fwd_threads<D>()),
+                  0, st, (const T *)q, (const T *)k, (const T *)v, (const T *)g, (T *)o, (const float *)E, s.T,
+                  kCausalChunk);
 }
 
 template <typename T, int D>
 la_status gated_bwd_t(const void *q, const void *k, const void *v, const void *g, const void *dout, void *dq,
                       void *dk, void *dv, void *dg, const Shape &s, void *ws, cudaStream_t st) {
-    const dim3 grid((unsigned)s.BH());
+    const int nc = causal_chunks(s.T);
+    const dim3 grid((unsigned)s.BH(), (unsigned)nc);
     float *dq32 = (float *)ws;
-    la_status rc = launch("simt_gated_bwd_q", gated_bwd_q<T, D>, grid, dim3(gated_fwd_threads<D>()), 0, st,
-                          (const T *)k, (const T *)v, (const T *)g, (const T *)dout, (T *)dq, dq32, s.T);
+    char *rest = (char *)ws + dq32_bytes(s);
+    float *E = nc > 1 ? (float *)rest : nullptr;
+    float *A = E ? (float *)(rest + gated_e_bytes(s)) : nullptr;
+    float *totals = E ? (float *)(rest + gated_e_bytes(s) + gated_a_bytes(s)) : nullptr;
+    la_status rc;
+    if (E && (rc = gated_states<T, D, false>(k, v, g, E, A, s, st))) return rc;
+    rc = launch("simt_gated_bwd_q", gated_bwd_q<T, D>, grid, dim3(gated_fwd_threads<D>()), 0, st, (const T *)k,
+                (const T *)v, (const T *)g, (const T *)dout, (T *)dq, dq32, (const float *)E, s.T, kCausalChunk);
     if (rc) return rc;
-    return launch("simt_gated_bwd_kv", gated_bwd_kv<T, D>, grid, dim3(gated_kv_threads<D>()), gated_bwd_kv_smem<D>(),
-                  st, (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const T *)dout, (const float *)dq32,
-                  (T *)dk, (T *)dv, (T *)dg, s.T);
+    if (E && (rc = gated_states<T, D, true>(q, dout, g, E, A, s, st))) return rc;
+    rc = launch("simt_gated_bwd_kv", gated_bwd_kv<T, D>, grid, dim3(gated_kv_threads<D>()), gated_bwd_kv_smem<D>(), st,
+                (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const T *)dout, dq32, (T *)dk, (T *)dv,
+                (T *)dg, (const float *)E, totals, s.T, kCausalChunk);
+    if (rc || !E) return rc;
+    return launch("simt_gated_dg_carry", gated_dg_carry<T, D>, dim3((unsigned)nc, (unsigned)s.BH()), dim3(256), 0, st,
+                  (const float *)dq32, (const float *)totals, (T *)dg, s.T, kCausalChunk);
 }
 
 #define LA_GATED_DISPATCH(F, ...)                                                     \
@@ -1463,8 +1665,8 @@ la_status gated_bwd_t(const void *q, const void *k, const void *v, const void *g
 }  // namespace
 
 la_status gated_fwd(const void *q, const void *k, const void *v, const void *g, void *o, const Shape &s, la_dtype dt,
-                    cudaStream_t st) {
-    LA_GATED_DISPATCH(gated_fwd_t, q, k, v, g, o, s, st);
+                    void *ws, cudaStream_t st) {
+    LA_GATED_DISPATCH(gated_fwd_t, q, k, v, g, o, s, ws, st);
 }
 
 la_status gated_bwd(const void *q, const void *k, const void *v, const void *g, const void *dout, void *dq, void *dk,

@@ -166,6 +166,27 @@ def test_causal_norm_validation(lib):
              P(0x1000), 1, 2, 16, 64, 1, P(0), ctypes.c_size_t(0), P(0)) == 4
 
 
+def test_gated_workspace(lib):
+    P = ctypes.c_void_p
+    f = lib.la_gated_fwd
+    f.restype = ctypes.c_int
+    lib.la_workspace_size.restype = ctypes.c_size_t
+    # one chunk (T <= 256): no forward workspace, the backward holds dq in fp32
+    assert lib.la_workspace_size(12, 1, 2, 256, 64, 1) == 0
+    assert lib.la_workspace_size(13, 1, 2, 256, 64, 1) == 2 * 256 * 64 * 4
+    # two chunks: [2 heads][2 chunks][64][64] states and [2][2][64] gate products (and dg totals)
+    states, per_dim = 2 * 2 * 64 * 64 * 4, 2 * 2 * 64 * 4
+    assert lib.la_workspace_size(12, 1, 2, 257, 64, 1) == states + per_dim
+    assert lib.la_workspace_size(13, 1, 2, 257, 64, 1) == 2 * 257 * 64 * 4 + states + 2 * per_dim
+
+    def fwd(T, ws=0, ws_bytes=0):
+        return f(P(0x1000), P(0x1000), P(0x1000), P(0x1000), P(0x1000), 1, 2, T, 64, 1, P(ws),
+                 ctypes.c_size_t(ws_bytes), P(0))
+    assert fwd(257) == 4
+    assert fwd(257, ws=0x1010, ws_bytes=1 << 20) == 3
+    assert fwd(257, ws=0x1000, ws_bytes=states) == 4
+
+
 def test_status_strings(lib):
     lib.la_status_string.restype = ctypes.c_char_p
     assert lib.la_status_string(0) == b"LA_OK"

@@ -1,6 +1,6 @@
 """GPU parity of gated linear attention (la_gated_*), through the C ABI, against the fp64 oracle:
-every dtype, D = 64 and 128, ragged lengths; constant gates against the decay op; sampled heads
-at the benchmark size."""
+every dtype, D = 64 and 128, lengths of one chunk (256 tokens) and of several, whole or ragged;
+constant gates against the decay op; sampled heads at the benchmark size."""
 import numpy as np
 import pytest
 import torch
@@ -42,7 +42,7 @@ def _ref(inp):
 
 
 @pytest.mark.parametrize("dtype,D,T", [("bf16", 64, 300), ("f16", 128, 300), ("f32", 64, 37), ("f32", 128, 129),
-                                       ("bf16", 128, 2)])
+                                       ("bf16", 128, 2), ("bf16", 64, 1024), ("f16", 64, 517), ("f32", 128, 512)])
 def test_matches_oracle(dtype, D, T):
     inp = _inputs(dtype, 2, 3, T, D, seed=61)
     got, want = _run(inp), _ref(inp)
@@ -54,7 +54,7 @@ def test_matches_oracle(dtype, D, T):
 def test_constant_gates_are_the_decay_op():
     """g_t = log gamma_h everywhere: la_gated_fwd equals la_chunk_decay_fwd (CUDA-core path, f32)."""
     import linear_attention_attn_b200 as la
-    B, H, T, D = 2, 3, 200, 64
+    B, H, T, D = 2, 3, 600, 64
     inp = _inputs("f32", B, H, T, D, seed=62)
     gam = [0.5, 0.9, 0.999]
     g = torch.log(torch.tensor(gam, dtype=torch.float32))[None, :, None, None].expand(B, H, T, D).contiguous()
