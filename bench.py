@@ -327,10 +327,12 @@ WORKLOAD_TEXT = {
               "q,k ~ N(0,1) D^-1/2, v, dO ~ N(0,1)",
     "retention": "chunked causal decay (retention) fwd+bwd, bf16 storage / fp32 accumulate, B=%d H=%d T=%d D=%d, "
                  "gamma_h = 1 - 2^(-5-7h/(H-1)), q ~ N(0,1) D^-1/2, k, v, dO ~ N(0,1)",
-    "gated": "gated linear attention fwd+bwd (recurrent form on CUDA cores), bf16 storage / fp32 accumulate, "
+    "gated": "gated linear attention fwd+bwd (recurrent form in 256-token chunks on CUDA cores), bf16 storage / "
+             "fp32 accumulate, "
              "B=%d H=%d T=%d D=%d, log gates log(sigmoid(N(0,1)))/16 per token and key dimension, "
              "q ~ N(0,1) D^-1/2, k, v, dO ~ N(0,1)",
-    "causal_norm": "causal linear attention with the norm term fwd+bwd (recurrent form on CUDA cores), fp16 storage / "
+    "causal_norm": "causal linear attention with the norm term fwd+bwd (recurrent form in 256-token chunks on CUDA "
+                   "cores), fp16 storage / "
                    "fp32 accumulate, B=%d H=%d T=%d D=%d, phi=elu+1, no decay, eps=1e-06, Q,K,V ~ 0.5 N(0,1), "
                    "dO ~ N(0,1)",
 }
