@@ -18,6 +18,8 @@
 // thread.
 #include "la_internal.cuh"
 
+#include <string.h>
+
 namespace la {
 namespace simt {
 
@@ -357,6 +359,82 @@ __device__ __forceinline__ void load_rows(const T *const (&src)[N], float (*dst)
     }
 }
 
+// 16 bytes of T as floats
+template <typename T> struct vec16;
+template <> struct vec16<float> {
+    static constexpr int n = 4;
+    static __device__ __forceinline__ void unpack(const uint4 &u, float *f) {
+        f[0] = __uint_as_float(u.x), f[1] = __uint_as_float(u.y), f[2] = __uint_as_float(u.z), f[3] = __uint_as_float(u.w);
+    }
+};
+template <> struct vec16<__half> {
+    static constexpr int n = 8;
+    static __device__ __forceinline__ void unpack(const uint4 &u, float *f) {
+        const unsigned w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __half2 h;
+            memcpy(&h, &w[i], 4);
+            const float2 x = __half22float2(h);
+            f[2 * i] = x.x, f[2 * i + 1] = x.y;
+        }
+    }
+};
+template <> struct vec16<__nv_bfloat16> {
+    static constexpr int n = 8;
+    static __device__ __forceinline__ void unpack(const uint4 &u, float *f) {
+        const unsigned w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 h;
+            memcpy(&h, &w[i], 4);
+            const float2 x = __bfloat1622float2(h);
+            f[2 * i] = x.x, f[2 * i + 1] = x.y;
+        }
+    }
+};
+
+// A tile of N row blocks by 16-byte loads into registers (rows are contiguous and 16-byte aligned:
+// D e is a multiple of 16 and the tensors start 16-byte aligned; rows at or past T_len read as 0),
+// then into shared memory as floats; NT threads, every load issued before the first store.
+template <typename T, int D, int NT>
+struct TileVec {
+    static constexpr int VE = vec16<T>::n, NV = kRetTile * D / VE, PER = (NV + NT - 1) / NT;
+};
+template <typename T, int D, int N, int NT>
+__device__ __forceinline__ void fetch_rows(const T *const (&src)[N], uint4 (&x)[N][TileVec<T, D, NT>::PER],
+                                           long long base, int ts, int T_len) {
+    using V = TileVec<T, D, NT>;
+#pragma unroll
+    for (int u = 0; u < V::PER; ++u) {
+        const int vi = threadIdx.x + u * NT, t = ts + vi * V::VE / D;
+#pragma unroll
+        for (int m = 0; m < N; ++m)
+            x[m][u] = vi < V::NV && t < T_len
+                          ? __ldg(reinterpret_cast<const uint4 *>(src[m] + base + (long long)ts * D + (long long)vi * V::VE))
+                          : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+template <typename T, int D, int N, int NT>
+__device__ __forceinline__ void stash_rows(const uint4 (&x)[N][TileVec<T, D, NT>::PER], float (*dst)[kRetTile][D]) {
+    using V = TileVec<T, D, NT>;
+#pragma unroll
+    for (int u = 0; u < V::PER; ++u) {
+        const int vi = threadIdx.x + u * NT;
+        if (vi < V::NV) {
+#pragma unroll
+            for (int m = 0; m < N; ++m) {
+                float f[V::VE];
+                vec16<T>::unpack(x[m][u], f);
+                float *d = &dst[m][0][0] + vi * V::VE;
+#pragma unroll
+                for (int w = 0; w < V::VE; w += 4)
+                    *reinterpret_cast<float4 *>(d + w) = make_float4(f[w], f[w + 1], f[w + 2], f[w + 3]);
+            }
+        }
+    }
+}
+
 // Forward recurrence, thread j holds column j of S:
 //   S_t = gamma S_{t-1} + k_t^T v_t,   o_t[j] = sum_i q_t[i] S_t[i][j].
 template <typename T, int D>
@@ -509,8 +587,11 @@ __device__ __forceinline__ float feature_grad_of(float fx) { return PHI ? (fx > 
 // whole warps; the threads past the last line compute on zeros and store nothing.
 template <int D> constexpr int causal_split() { return D == 64 ? 4 : 2; }
 template <int N> constexpr int round_warps(int n) { return (n + 31) / 32 * 32; }
-template <int D> constexpr int causal_fwd_threads() { return round_warps<0>(causal_split<D>() * (D + 1)); }
-template <int D> constexpr int causal_bwd_q_threads() { return round_warps<0>(causal_split<D>() * (2 * D + 1)); }
+// forward: column groups of four, each over D / 8 threads of 8 rows (part_entry)
+template <int D> constexpr int causal_fwd_parts() { return D / 8; }
+template <int D> constexpr int causal_fwd_threads() { return D / 4 * causal_fwd_parts<D>(); }
+// dq sweep: column groups of four, each over 8 threads of D / 8 rows
+template <int D> constexpr int causal_bwd_q_threads() { return D / 4 * 8; }
 template <int D> constexpr int causal_bwd_kv_threads() { return 2 * causal_split<D>() * D; }
 
 template <int P>
@@ -531,6 +612,28 @@ __device__ __forceinline__ float4 part_group(const float *row, int p, int m) {
     return *reinterpret_cast<const float4 *>(row + 4 * p + 4 * P * m);
 }
 __device__ __forceinline__ float f4(const float4 &x, int e) { return e == 0 ? x.x : e == 1 ? x.y : e == 2 ? x.z : x.w; }
+// The P parts (adjacent lanes, P a power of two >= 4) of a group of four lines each hold partial
+// sums col[0..3] of the four lines; returns the whole sum of line (p & 3) in part p.  Fixed order:
+// halves above the first four lanes first, then two exchange rounds (3 shuffles for P = 4).
+template <int P>
+__device__ __forceinline__ float group_reduce_scatter(const float (&col)[4], int p) {
+    float c0 = col[0], c1 = col[1], c2 = col[2], c3 = col[3];
+#pragma unroll
+    for (int m = P / 2; m >= 4; m >>= 1) {
+        c0 += __shfl_xor_sync(0xffffffffu, c0, m);
+        c1 += __shfl_xor_sync(0xffffffffu, c1, m);
+        c2 += __shfl_xor_sync(0xffffffffu, c2, m);
+        c3 += __shfl_xor_sync(0xffffffffu, c3, m);
+    }
+    const bool hi = p & 2, odd = p & 1;
+    float k0 = hi ? c2 : c0, k1 = hi ? c3 : c1;           // lines kept: 2 hi + 0, 2 hi + 1
+    k0 += __shfl_xor_sync(0xffffffffu, hi ? c0 : c2, 2);
+    k1 += __shfl_xor_sync(0xffffffffu, hi ? c1 : c3, 2);
+    float kk = odd ? k1 : k0;                             // line 2 hi + odd
+    kk += __shfl_xor_sync(0xffffffffu, odd ? k0 : k1, 1);
+    return kk;
+}
+
 // s <- gamma s + x y, or s + x y without a decay (one FMA)
 template <bool DECAY>
 __device__ __forceinline__ float decay_fma(float gamma, float s, float x, float y) {
@@ -691,46 +794,79 @@ chunk_scan(float *__restrict__ E, const float *__restrict__ A, DecayArgs dec, in
     }
 }
 
-// Forward: the D + 1 columns of [S | z] (z: the column of a value that is always 1).
+// Forward: the columns of S in groups of four; thread p of group g holds S[i][4 g + c] (c < 4)
+// for its eight rows i = part_entry(p, .), so each k and q entry it reads serves four columns;
+// group 0 also holds z (the column of a value that is always 1) for its rows.
 template <typename T, int D, bool PHI, bool DECAY>
 __global__ void __launch_bounds__(causal_fwd_threads<D>())
 causal_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, T *__restrict__ o,
            const float *__restrict__ st_in, DecayArgs dec, int has_decay, int T_len, int H, int L, float eps) {
-    constexpr int P = causal_split<D>(), DP = D / P;
+    constexpr int P = causal_fwd_parts<D>(), DP = 8, C = 4;
     __shared__ __align__(16) float tiles[3][kRetTile][D];
     __shared__ float acc[kRetTile][D + 1];
     const int bh = blockIdx.x, s0 = blockIdx.y * L, s1 = min(T_len, s0 + L);
     const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
     const long long base = (long long)bh * T_len * D;
-    const int j = threadIdx.x / P, pp = threadIdx.x % P;
-    const bool lead = pp == 0 && j <= D;
+    const int grp = threadIdx.x / P, pp = threadIdx.x % P, j0 = C * grp;
+    const bool zgrp = grp == 0, warp0 = threadIdx.x < 32;
     const float *const S0 = chunk_state<D>(st_in, bh, blockIdx.y);
-    float S[DP];
+    float S[C][DP], Sz[DP];
 #pragma unroll
-    for (int i = 0; i < DP; ++i) S[i] = S0 && j <= D ? S0[part_entry<P>(pp, i) * (D + 1) + j] : 0.f;
+    for (int i = 0; i < DP; ++i) {
+        const int x = part_entry<P>(pp, i);
+#pragma unroll
+        for (int c = 0; c < C; ++c) S[c][i] = S0 ? S0[x * (D + 1) + j0 + c] : 0.f;
+        Sz[i] = S0 && zgrp ? S0[x * (D + 1) + D] : 0.f;
+    }
     const T *const src[3] = {q, k, v};
+    constexpr int NT = causal_fwd_threads<D>();
     for (int ts = s0; ts < s1; ts += kRetTile) {
         __syncthreads();
-        load_rows<T, D, 3, causal_fwd_threads<D>()>(src, tiles, base, ts, T_len);
+        {
+            uint4 x[3][TileVec<T, D, NT>::PER];
+            fetch_rows<T, D, 3, NT>(src, x, base, ts, T_len);
+            stash_rows<T, D, 3, NT>(x, tiles);
+        }
         __syncthreads();
         feature_tiles<D, PHI>(tiles, 2);
         __syncthreads();
         const int nr = min(kRetTile, s1 - ts);
 #pragma unroll 2
         for (int r = 0; r < nr; ++r) {
-            const float vj = j < D ? tiles[2][r][j] : 1.f;
-            float a[4] = {0.f, 0.f, 0.f, 0.f};
+            const float4 vv = *reinterpret_cast<const float4 *>(&tiles[2][r][j0]);
+            float a[C][4], az[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                az[e] = 0.f;
+#pragma unroll
+                for (int c = 0; c < C; ++c) a[c][e] = 0.f;
+            }
 #pragma unroll
             for (int m = 0; m < DP / 4; ++m) {
                 const float4 kk = part_group<P>(tiles[1][r], pp, m), qq = part_group<P>(tiles[0][r], pp, m);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    S[4 * m + e] = decay_fma<DECAY>(gamma, S[4 * m + e], f4(kk, e), vj);
-                    a[e] = fmaf(f4(qq, e), S[4 * m + e], a[e]);
+                    const float ke = f4(kk, e), qe = f4(qq, e);
+#pragma unroll
+                    for (int c = 0; c < C; ++c) {
+                        S[c][4 * m + e] = decay_fma<DECAY>(gamma, S[c][4 * m + e], ke, f4(vv, c));
+                        a[c][e] = fmaf(qe, S[c][4 * m + e], a[c][e]);
+                    }
+                    if (zgrp) {
+                        Sz[4 * m + e] = DECAY ? fmaf(gamma, Sz[4 * m + e], ke) : Sz[4 * m + e] + ke;
+                        az[e] = fmaf(qe, Sz[4 * m + e], az[e]);
+                    }
                 }
             }
-            const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
-            if (lead) acc[r][j] = s;
+            float col[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) col[c] = (a[c][0] + a[c][1]) + (a[c][2] + a[c][3]);
+            const float mine = group_reduce_scatter<P>(col, pp);
+            if (pp < C) acc[r][j0 + pp] = mine;
+            if (warp0) {                          // group 0 (lanes 0 .. P - 1 of warp 0): n_t - eps
+                const float zs = line_sum<P>((az[0] + az[1]) + (az[2] + az[3]));
+                if (threadIdx.x == 0) acc[r][D] = zs;
+            }
         }
         __syncthreads();
         for (int e = threadIdx.x; e < nr * D; e += blockDim.x) {
@@ -740,88 +876,121 @@ causal_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict
     }
 }
 
+// Row sums over the four column groups of a warp (lane bits 3 and 4), scattered: each lane
+// enters partial sums v[0 .. N) of N rows and leaves with the whole sums of N / 4 of them,
+// rows (lane & 16 ? N / 2 : 0) + (lane & 8 ? N / 4 : 0) + x for x < N / 4.  Fixed order.
+template <int N>
+__device__ __forceinline__ void rows_reduce_scatter(const float (&v)[N], float (&out)[N / 4], int lane) {
+    const bool b4 = lane & 16, b3 = lane & 8;
+    float h[N / 2];
+#pragma unroll
+    for (int x = 0; x < N / 2; ++x)
+        h[x] = (b4 ? v[N / 2 + x] : v[x]) + __shfl_xor_sync(0xffffffffu, b4 ? v[x] : v[N / 2 + x], 16);
+#pragma unroll
+    for (int x = 0; x < N / 4; ++x)
+        out[x] = (b3 ? h[N / 4 + x] : h[x]) + __shfl_xor_sync(0xffffffffu, b3 ? h[x] : h[N / 4 + x], 8);
+}
+
 // Backward, forward sweep: dq, and per row (n_t, dn_t) for the reverse sweep, with
 // u_t = f(q_t) S_t, n_t = f(q_t) . z_t + eps, dn_t = -(dout_t . u_t) / n_t^2:
 //   df(q)_t[i] = (sum_j S_t[i][j] dout_t[j]) / n_t + z_t[i] dn_t,  dq = df(q) f'(q).
-// The first P (D + 1) threads hold the columns of [S | z] (u_t and n_t), the next P D the
-// rows of S and z[i] (the row sums of dq); a tile's rows meet in shared memory.
+// S is held once, in blocks: thread p of column group g holds S[i][4 g + c] (c < 4) for the D / 8
+// rows i = part_entry(p, .), and forms from them both the column sums u_t (over the 8 threads of
+// the group) and the row sums of dq (over the column groups: the four of a warp by shuffles, the
+// warps through shared memory); group 0 also holds z.  Each k, q entry read serves four columns
+// and each v, dO entry D / 8 rows.
 template <typename T, int D, bool PHI, bool DECAY>
 __global__ void __launch_bounds__(causal_bwd_q_threads<D>())
 causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
              T *__restrict__ dq, float2 *__restrict__ nd, const float *__restrict__ st_in, DecayArgs dec, int has_decay,
              int T_len, int H, int L, float eps) {
-    constexpr int P = causal_split<D>(), DP = D / P, NCOL = P * (D + 1);
+    constexpr int P = 8, DP = D / P, C = 4, NT = causal_bwd_q_threads<D>(), W = NT / 32;
     extern __shared__ __align__(16) float dsm[];   // causal_bwd_q_smem<D>() bytes
     float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // f(q), f(k), v, dout
     float(*U)[D + 1] = reinterpret_cast<float(*)[D + 1]>(dsm + 4 * kRetTile * D);  // dout_t[j] u_t[j], n_t - eps
-    float(*A)[D] = reinterpret_cast<float(*)[D]>(dsm + 4 * kRetTile * D + kRetTile * (D + 1));
-    float(*Z)[D] = A + kRetTile;
-    float2 *info = reinterpret_cast<float2 *>(dsm + 6 * kRetTile * D + kRetTile * (D + 1));   // (1 / n_t, dn_t)
+    float(*Z)[D] = reinterpret_cast<float(*)[D]>(dsm + 4 * kRetTile * D + kRetTile * (D + 1));   // z_t
+    float(*A)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm + 5 * kRetTile * D + kRetTile * (D + 1));
+    float2 *info = reinterpret_cast<float2 *>(dsm + (5 + W) * kRetTile * D + kRetTile * (D + 1));   // (1 / n_t, dn_t)
     const int bh = blockIdx.x, s0 = blockIdx.y * L, s1 = min(T_len, s0 + L);
     const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
     const long long base = (long long)bh * T_len * D;
-    const bool col_side = threadIdx.x < NCOL;
-    const int t2 = col_side ? threadIdx.x : threadIdx.x - NCOL;
-    const int line = t2 / P, pp = t2 % P;              // column (col side) or row (row side); part
-    const bool row_live = !col_side && line < D;
-    const bool lead = t2 % P == 0 && (col_side || row_live);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-    // the entering [S | z]: the col side takes column `line` (z for line = D), the row side row `line`
+    const int grp = threadIdx.x / P, pp = threadIdx.x % P, j0 = C * grp;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool zgrp = grp == 0;
+    const int rbase = (lane & 16 ? DP / 2 : 0) + (lane & 8 ? DP / 4 : 0);   // rows this lane's dq sums cover
     const float *const S0 = chunk_state<D>(st_in, bh, blockIdx.y);
-    float Sx[DP];
-    float zi = S0 && row_live ? S0[line * (D + 1) + D] : 0.f;
+    float S[C][DP], Sz[DP];
 #pragma unroll
     for (int i = 0; i < DP; ++i) {
         const int x = part_entry<P>(pp, i);
-        Sx[i] = !S0 ? 0.f : col_side ? S0[x * (D + 1) + line] : row_live ? S0[line * (D + 1) + x] : 0.f;
+#pragma unroll
+        for (int c = 0; c < C; ++c) S[c][i] = S0 ? S0[x * (D + 1) + j0 + c] : 0.f;
+        Sz[i] = S0 && zgrp ? S0[x * (D + 1) + D] : 0.f;
     }
     const T *const src[4] = {q, k, v, g};
     for (int ts = s0; ts < s1; ts += kRetTile) {
         __syncthreads();
-        load_rows<T, D, 4, causal_bwd_q_threads<D>()>(src, tiles, base, ts, T_len);
+        {
+            uint4 x[4][TileVec<T, D, NT>::PER];
+            fetch_rows<T, D, 4, NT>(src, x, base, ts, T_len);
+            stash_rows<T, D, 4, NT>(x, tiles);
+        }
         __syncthreads();
         feature_tiles<D, PHI>(tiles, 2);
         __syncthreads();
         const int nr = min(kRetTile, s1 - ts);
 #pragma unroll 2
         for (int r = 0; r < nr; ++r) {
-            float a[4] = {0.f, 0.f, 0.f, 0.f};
-            if (col_side) {
-                const float vj = line < D ? tiles[2][r][line] : 1.f;
+            const float4 vv = *reinterpret_cast<const float4 *>(&tiles[2][r][j0]);
+            const float4 gv = *reinterpret_cast<const float4 *>(&tiles[3][r][j0]);
+            float au[C][4], ad[DP], az[4];
 #pragma unroll
-                for (int m = 0; m < DP / 4; ++m) {
-                    const float4 kk = part_group<P>(tiles[1][r], pp, m), qq = part_group<P>(tiles[0][r], pp, m);
+            for (int e = 0; e < 4; ++e) {
+                az[e] = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        Sx[4 * m + e] = decay_fma<DECAY>(gamma, Sx[4 * m + e], f4(kk, e), vj);
-                        a[e] = fmaf(f4(qq, e), Sx[4 * m + e], a[e]);
+                for (int c = 0; c < C; ++c) au[c][e] = 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < DP; ++i) ad[i] = 0.f;
+#pragma unroll
+            for (int m = 0; m < DP / 4; ++m) {
+                const float4 kk = part_group<P>(tiles[1][r], pp, m), qq = part_group<P>(tiles[0][r], pp, m);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 4 * m + e;
+                    const float ke = f4(kk, e), qe = f4(qq, e);
+#pragma unroll
+                    for (int c = 0; c < C; ++c) {
+                        S[c][i] = decay_fma<DECAY>(gamma, S[c][i], ke, f4(vv, c));
+                        au[c][e] = fmaf(qe, S[c][i], au[c][e]);
+                        ad[i] = fmaf(S[c][i], f4(gv, c), ad[i]);
+                    }
+                    if (zgrp) {
+                        Sz[i] = DECAY ? fmaf(gamma, Sz[i], ke) : Sz[i] + ke;
+                        az[e] = fmaf(qe, Sz[i], az[e]);
                     }
                 }
-            } else if (row_live) {
-                const float ki = tiles[1][r][line];
-#pragma unroll
-                for (int m = 0; m < DP / 4; ++m) {
-                    const float4 vv = part_group<P>(tiles[2][r], pp, m), gg = part_group<P>(tiles[3][r], pp, m);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        Sx[4 * m + e] = decay_fma<DECAY>(gamma, Sx[4 * m + e], ki, f4(vv, e));
-                        a[e] = fmaf(Sx[4 * m + e], f4(gg, e), a[e]);
-                    }
-                }
-                zi = DECAY ? fmaf(gamma, zi, ki) : zi + ki;
             }
-            const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
-            if (lead) {
-                if (col_side) {
-                    U[r][line] = line < D ? s * tiles[3][r][line] : s;
-                } else {
-                    A[r][line] = s;
-                    Z[r][line] = zi;
-                }
+            float col[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) col[c] = (au[c][0] + au[c][1]) + (au[c][2] + au[c][3]);
+            const float u = group_reduce_scatter<P>(col, pp);
+            if (pp < C) U[r][j0 + pp] = u * f4(gv, pp);
+            if (warp == 0) {                      // group 0 (lanes 0 .. 7 of warp 0): n_t - eps
+                const float zs = line_sum<P>((az[0] + az[1]) + (az[2] + az[3]));
+                if (lane == 0) U[r][D] = zs;
             }
+            if (zgrp) {
+#pragma unroll
+                for (int i = 0; i < DP; ++i) Z[r][part_entry<P>(pp, i)] = Sz[i];
+            }
+            float rs[DP / 4];
+            rows_reduce_scatter<DP>(ad, rs, lane);
+#pragma unroll
+            for (int x = 0; x < DP / 4; ++x) A[warp][r][part_entry<P>(pp, rbase + x)] = rs[x];
         }
         __syncthreads();
-        for (int r = warp; r < nr; r += nwarps) {   // dout_t . u_t, a warp per row, fixed order
+        for (int r = warp; r < nr; r += W) {      // dout_t . u_t, a warp per row, fixed order
             float p = 0.f;
             for (int jj = lane; jj < D; jj += 32) p += U[r][jj];
 #pragma unroll
@@ -834,10 +1003,13 @@ causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
             }
         }
         __syncthreads();
-        for (int e = threadIdx.x; e < nr * D; e += blockDim.x) {
+        for (int e = threadIdx.x; e < nr * D; e += NT) {
             const int r = e / D, c = e % D;
             const float2 in = info[r];
-            const float d = fmaf(A[r][c], in.x, Z[r][c] * in.y);
+            float a = 0.f;
+#pragma unroll
+            for (int w = 0; w < W; ++w) a += A[w][r][c];
+            const float d = fmaf(a, in.x, Z[r][c] * in.y);
             io<T>::st(dq + base + (long long)(ts + r) * D + c, d * feature_grad_of<PHI>(tiles[0][r][c]));
         }
     }
@@ -845,9 +1017,10 @@ causal_bwd_q(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
 
 template <int D>
 constexpr size_t causal_bwd_q_smem() {
-    return (size_t)(6 * kRetTile * D + kRetTile * (D + 1)) * sizeof(float) + kRetTile * sizeof(float2);
+    constexpr int W = causal_bwd_q_threads<D>() / 32;
+    return (size_t)((5 + W) * kRetTile * D + kRetTile * (D + 1)) * sizeof(float) + kRetTile * sizeof(float2);
 }
-static_assert((6 * kRetTile * 64 + kRetTile * 65) % 2 == 0 && (6 * kRetTile * 128 + kRetTile * 129) % 2 == 0,
+static_assert(((5 + 4) * kRetTile * 64 + kRetTile * 65) % 2 == 0 && ((5 + 8) * kRetTile * 128 + kRetTile * 129) % 2 == 0,
               "the float2 block of causal_bwd_q starts 8-byte aligned");
 
 // Backward, reverse sweep over R_s = gamma R_{s+1} + f(q_s)^T du_s and r_s = gamma r_{s+1} +
