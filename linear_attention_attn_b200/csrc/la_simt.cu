@@ -592,7 +592,7 @@ template <int D> constexpr int causal_fwd_parts() { return D / 8; }
 template <int D> constexpr int causal_fwd_threads() { return D / 4 * causal_fwd_parts<D>(); }
 // dq sweep: column groups of four, each over 8 threads of D / 8 rows
 template <int D> constexpr int causal_bwd_q_threads() { return D / 4 * 8; }
-template <int D> constexpr int causal_bwd_kv_threads() { return 2 * causal_split<D>() * D; }
+template <int D> constexpr int causal_bwd_kv_threads() { return D / 4 * 8; }   // as the dq sweep
 
 template <int P>
 __device__ __forceinline__ float line_sum(float s) {
@@ -1024,39 +1024,49 @@ static_assert(((5 + 4) * kRetTile * 64 + kRetTile * 65) % 2 == 0 && ((5 + 8) * k
               "the float2 block of causal_bwd_q starts 8-byte aligned");
 
 // Backward, reverse sweep over R_s = gamma R_{s+1} + f(q_s)^T du_s and r_s = gamma r_{s+1} +
-// f(q_s) dn_s with du_s = dout_s / n_s: the first P D threads hold the rows of R and r[i]
-// (dk_s[i] = (sum_j R[i][j] v_s[j] + r[i]) f'(k_s[i])), the next P D the columns of R
-// (dv_s[j] = sum_i f(k_s)[i] R[i][j]).
+// f(q_s) dn_s with du_s = dout_s / n_s:
+//   dk_s[i] = (sum_j R[i][j] v_s[j] + r[i]) f'(k_s[i]),  dv_s[j] = sum_i f(k_s)[i] R[i][j].
+// R is held in blocks as S in the dq sweep: thread p of column group g holds R[i][4 g + c] for the
+// D / 8 rows i = part_entry(p, .); the column sums (dv) meet over the group's 8 threads, the row
+// sums (dk) over the column groups (shuffles within a warp, shared memory across warps); group 0
+// also holds r.
 template <typename T, int D, bool PHI, bool DECAY>
 __global__ void __launch_bounds__(causal_bwd_kv_threads<D>())
 causal_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
               const float2 *__restrict__ nd, T *__restrict__ dk, T *__restrict__ dv, const float *__restrict__ st_in,
               DecayArgs dec, int has_decay, int T_len, int H, int L) {
-    constexpr int P = causal_split<D>(), DP = D / P;
+    constexpr int P = 8, DP = D / P, C = 4, NT = causal_bwd_kv_threads<D>(), W = NT / 32;
     extern __shared__ __align__(16) float dsm[];   // causal_bwd_kv_smem<D>() bytes
-    float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // f(q), f(k), v, dout
-    float(*res)[kRetTile][D] = tiles + 4;        // dk before f' (rows), dv (columns)
-    float2 *info = reinterpret_cast<float2 *>(dsm + 6 * kRetTile * D);
+    float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // f(q), f(k), v, dout (then du)
+    float(*A)[kRetTile][D] = tiles + 4;                                          // per warp: row sums of dk
+    float(*DV)[D] = reinterpret_cast<float(*)[D]>(dsm + (4 + W) * kRetTile * D);  // dv
+    float(*Rr)[D] = DV + kRetTile;                                               // r_s
+    float2 *info = reinterpret_cast<float2 *>(dsm + (6 + W) * kRetTile * D);    // (1 / n_s, dn_s)
     const int bh = blockIdx.x, s0 = blockIdx.y * L, s1 = min(T_len, s0 + L);
     const float gamma = has_decay ? dec.gamma[bh % H] : 1.f;
     const long long base = (long long)bh * T_len * D;
-    const bool row_side = threadIdx.x < P * D;
-    const int t2 = row_side ? threadIdx.x : threadIdx.x - P * D;
-    const int line = t2 / P, pp = t2 % P;
-    const bool lead = pp == 0;
-    // the entering [R | r] (the tokens after this chunk): rows on the row side, columns on the other
+    const int grp = threadIdx.x / P, pp = threadIdx.x % P, j0 = C * grp;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool zgrp = grp == 0;
+    const int rbase = (lane & 16 ? DP / 2 : 0) + (lane & 8 ? DP / 4 : 0);
+    // the entering [R | r] (the tokens after this chunk)
     const float *const R0 = chunk_state<D>(st_in, bh, blockIdx.y);
-    float Rx[DP];
-    float ri = R0 && row_side ? R0[line * (D + 1) + D] : 0.f;
+    float R[C][DP], ri[DP];
 #pragma unroll
     for (int i = 0; i < DP; ++i) {
         const int x = part_entry<P>(pp, i);
-        Rx[i] = !R0 ? 0.f : row_side ? R0[line * (D + 1) + x] : R0[x * (D + 1) + line];
+#pragma unroll
+        for (int c = 0; c < C; ++c) R[c][i] = R0 ? R0[x * (D + 1) + j0 + c] : 0.f;
+        ri[i] = R0 && zgrp ? R0[x * (D + 1) + D] : 0.f;
     }
     const T *const src[4] = {q, k, v, g};
     for (int ts = s0 + (s1 - s0 - 1) / kRetTile * kRetTile; ts >= s0; ts -= kRetTile) {
         __syncthreads();
-        load_rows<T, D, 4, causal_bwd_kv_threads<D>()>(src, tiles, base, ts, T_len);
+        {
+            uint4 x[4][TileVec<T, D, NT>::PER];
+            fetch_rows<T, D, 4, NT>(src, x, base, ts, T_len);
+            stash_rows<T, D, 4, NT>(x, tiles);
+        }
         const int nr = min(kRetTile, s1 - ts);
         if (threadIdx.x < nr) {
             const float2 x = nd[(long long)bh * T_len + ts + threadIdx.x];
@@ -1064,52 +1074,67 @@ causal_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
         }
         __syncthreads();
         feature_tiles<D, PHI>(tiles, 2);
-        for (int e = threadIdx.x; e < nr * D; e += blockDim.x) tiles[3][e / D][e % D] *= info[e / D].x;   // du
+        for (int e = threadIdx.x; e < nr * D; e += NT) tiles[3][e / D][e % D] *= info[e / D].x;   // du
         __syncthreads();
 #pragma unroll 2
         for (int r = nr - 1; r >= 0; --r) {
-            const float2 in = info[r];
-            float a[4] = {0.f, 0.f, 0.f, 0.f};
-            if (row_side) {
-                const float qi = tiles[0][r][line];
+            const float4 du = *reinterpret_cast<const float4 *>(&tiles[3][r][j0]);
+            const float4 vv = *reinterpret_cast<const float4 *>(&tiles[2][r][j0]);
+            const float dn = info[r].y;
+            float av[C][4], ak[DP];
 #pragma unroll
-                for (int m = 0; m < DP / 4; ++m) {
-                    const float4 gg = part_group<P>(tiles[3][r], pp, m), vv = part_group<P>(tiles[2][r], pp, m);
+            for (int e = 0; e < 4; ++e)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        Rx[4 * m + e] = decay_fma<DECAY>(gamma, Rx[4 * m + e], qi, f4(gg, e));
-                        a[e] = fmaf(Rx[4 * m + e], f4(vv, e), a[e]);
+                for (int c = 0; c < C; ++c) av[c][e] = 0.f;
+#pragma unroll
+            for (int i = 0; i < DP; ++i) ak[i] = 0.f;
+#pragma unroll
+            for (int m = 0; m < DP / 4; ++m) {
+                const float4 qq = part_group<P>(tiles[0][r], pp, m), kk = part_group<P>(tiles[1][r], pp, m);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 4 * m + e;
+                    const float qe = f4(qq, e), ke = f4(kk, e);
+#pragma unroll
+                    for (int c = 0; c < C; ++c) {
+                        R[c][i] = decay_fma<DECAY>(gamma, R[c][i], qe, f4(du, c));
+                        ak[i] = fmaf(R[c][i], f4(vv, c), ak[i]);
+                        av[c][e] = fmaf(ke, R[c][i], av[c][e]);
                     }
-                }
-                ri = DECAY ? fmaf(gamma, ri, qi * in.y) : fmaf(qi, in.y, ri);
-            } else {
-                const float duj = tiles[3][r][line];
-#pragma unroll
-                for (int m = 0; m < DP / 4; ++m) {
-                    const float4 qq = part_group<P>(tiles[0][r], pp, m), kk = part_group<P>(tiles[1][r], pp, m);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        Rx[4 * m + e] = decay_fma<DECAY>(gamma, Rx[4 * m + e], f4(qq, e), duj);
-                        a[e] = fmaf(f4(kk, e), Rx[4 * m + e], a[e]);
-                    }
+                    if (zgrp) ri[i] = DECAY ? fmaf(gamma, ri[i], qe * dn) : fmaf(qe, dn, ri[i]);
                 }
             }
-            const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
-            if (lead) res[row_side ? 0 : 1][r][line] = row_side ? s + ri : s;
+            float col[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) col[c] = (av[c][0] + av[c][1]) + (av[c][2] + av[c][3]);
+            const float dvj = group_reduce_scatter<P>(col, pp);
+            if (pp < C) DV[r][j0 + pp] = dvj;
+            if (zgrp) {
+#pragma unroll
+                for (int i = 0; i < DP; ++i) Rr[r][part_entry<P>(pp, i)] = ri[i];
+            }
+            float rs[DP / 4];
+            rows_reduce_scatter<DP>(ak, rs, lane);
+#pragma unroll
+            for (int x = 0; x < DP / 4; ++x) A[warp][r][part_entry<P>(pp, rbase + x)] = rs[x];
         }
         __syncthreads();
-        for (int e = threadIdx.x; e < nr * D; e += blockDim.x) {   // the tile's rows, coalesced
+        for (int e = threadIdx.x; e < nr * D; e += NT) {   // the tile's rows, coalesced
             const int r = e / D, c = e % D;
             const long long at = base + (long long)(ts + r) * D + c;
-            io<T>::st(dk + at, res[0][r][c] * feature_grad_of<PHI>(tiles[1][r][c]));
-            io<T>::st(dv + at, res[1][r][c]);
+            float a = Rr[r][c];
+#pragma unroll
+            for (int w = 0; w < W; ++w) a += A[w][r][c];
+            io<T>::st(dk + at, a * feature_grad_of<PHI>(tiles[1][r][c]));
+            io<T>::st(dv + at, DV[r][c]);
         }
     }
 }
 
 template <int D>
 constexpr size_t causal_bwd_kv_smem() {
-    return (size_t)(6 * kRetTile * D) * sizeof(float) + kRetTile * sizeof(float2);
+    constexpr int W = causal_bwd_kv_threads<D>() / 32;
+    return (size_t)((6 + W) * kRetTile * D) * sizeof(float) + kRetTile * sizeof(float2);
 }
 
 // ------------------------------------------------------ gated linear attention ---
