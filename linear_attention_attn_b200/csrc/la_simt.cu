@@ -43,7 +43,9 @@ inline size_t dq32_bytes(const Shape &s) { return round256((size_t)s.BH() * s.T 
 inline size_t gated_e_bytes(const Shape &s) {
     return round256((size_t)s.BH() * causal_chunks(s.T) * s.D * s.D * sizeof(float));
 }
-inline size_t gated_a_bytes(const Shape &s) { return round256((size_t)s.BH() * causal_chunks(s.T) * s.D * sizeof(float)); }
+inline size_t gated_a_bytes(const Shape &s) {
+    return round256((size_t)s.BH() * causal_chunks(s.T) * s.D * sizeof(float));
+}
 inline size_t gated_state_bytes(const Shape &s) {
     return causal_chunks(s.T) > 1 ? gated_e_bytes(s) + gated_a_bytes(s) : 0;
 }
@@ -364,7 +366,8 @@ template <typename T> struct vec16;
 template <> struct vec16<float> {
     static constexpr int n = 4;
     static __device__ __forceinline__ void unpack(const uint4 &u, float *f) {
-        f[0] = __uint_as_float(u.x), f[1] = __uint_as_float(u.y), f[2] = __uint_as_float(u.z), f[3] = __uint_as_float(u.w);
+        f[0] = __uint_as_float(u.x), f[1] = __uint_as_float(u.y);
+        f[2] = __uint_as_float(u.z), f[3] = __uint_as_float(u.w);
     }
 };
 template <> struct vec16<__half> {
@@ -409,10 +412,10 @@ __device__ __forceinline__ void fetch_rows(const T *const (&src)[N], uint4 (&x)[
     for (int u = 0; u < V::PER; ++u) {
         const int vi = threadIdx.x + u * NT, t = ts + vi * V::VE / D;
 #pragma unroll
-        for (int m = 0; m < N; ++m)
-            x[m][u] = vi < V::NV && t < T_len
-                          ? __ldg(reinterpret_cast<const uint4 *>(src[m] + base + (long long)ts * D + (long long)vi * V::VE))
-                          : make_uint4(0u, 0u, 0u, 0u);
+        for (int m = 0; m < N; ++m) {
+            const T *at = src[m] + base + (long long)ts * D + (long long)vi * V::VE;
+            x[m][u] = vi < V::NV && t < T_len ? __ldg(reinterpret_cast<const uint4 *>(at)) : make_uint4(0u, 0u, 0u, 0u);
+        }
     }
 }
 template <typename T, int D, int N, int NT>
@@ -1020,7 +1023,8 @@ constexpr size_t causal_bwd_q_smem() {
     constexpr int W = causal_bwd_q_threads<D>() / 32;
     return (size_t)((5 + W) * kRetTile * D + kRetTile * (D + 1)) * sizeof(float) + kRetTile * sizeof(float2);
 }
-static_assert(((5 + 4) * kRetTile * 64 + kRetTile * 65) % 2 == 0 && ((5 + 8) * kRetTile * 128 + kRetTile * 129) % 2 == 0,
+static_assert(((5 + 4) * kRetTile * 64 + kRetTile * 65) % 2 == 0 &&
+                  ((5 + 8) * kRetTile * 128 + kRetTile * 129) % 2 == 0,
               "the float2 block of causal_bwd_q starts 8-byte aligned");
 
 // Backward, reverse sweep over R_s = gamma R_{s+1} + f(q_s)^T du_s and r_s = gamma r_{s+1} +
@@ -1147,8 +1151,8 @@ template <int D>
 __device__ __forceinline__ void exp_tile(float (*tile)[D]) {
     for (int e = threadIdx.x; e < kRetTile * D; e += blockDim.x) tile[e / D][e % D] = expf(tile[e / D][e % D]);
 }
-template <int D> constexpr int gated_fwd_threads() { return causal_split<D>() * D; }
-template <int D> constexpr int gated_kv_threads() { return 2 * causal_split<D>() * D; }
+// the state in blocks of four columns by D / 8 rows per thread, as the causal-norm sweeps
+template <int D> constexpr int gated_threads() { return D / 4 * 8; }
 
 // ---- chunks along T, as for the causal-norm kernels.  A chunk's own state from a zero state
 // weights each token by the product of the gates between it and the chunk's end (forward) or
@@ -1271,142 +1275,186 @@ gated_dg_carry(const float *__restrict__ part, const float *__restrict__ totals,
         io<T>::st(dg + base + e, part[base + e] + carry[e % D]);
 }
 
-// Forward: the D columns of S; thread p of column j holds S[i][j] for its D / P rows
-// i = part_entry(p, .).
+// Forward: thread p of column group g holds S[i][4 g + c] (c < 4) for the D / 8 rows
+// i = part_entry(p, .); o_t[j] is a column sum over the group's 8 threads.
 template <typename T, int D>
-__global__ void __launch_bounds__(gated_fwd_threads<D>())
+__global__ void __launch_bounds__(gated_threads<D>())
 gated_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
           T *__restrict__ o, const float *__restrict__ st_in, int T_len, int L) {
-    constexpr int P = causal_split<D>(), DP = D / P;
+    constexpr int P = 8, DP = D / P, C = 4, NT = gated_threads<D>();
     __shared__ __align__(16) float tiles[4][kRetTile][D];      // q, k, v, a = exp(g)
     __shared__ float acc[kRetTile][D];
     const int s0 = blockIdx.y * L, s1 = min(T_len, s0 + L);
     const long long base = (long long)blockIdx.x * T_len * D;
-    const int j = threadIdx.x / P, pp = threadIdx.x % P;
-    const bool lead = pp == 0;
+    const int grp = threadIdx.x / P, pp = threadIdx.x % P, j0 = C * grp;
     const float *const S0 = chunk_state<D, D>(st_in, blockIdx.x, blockIdx.y);
-    float S[DP];
+    float S[C][DP];
 #pragma unroll
-    for (int i = 0; i < DP; ++i) S[i] = S0 ? S0[part_entry<P>(pp, i) * D + j] : 0.f;
+    for (int i = 0; i < DP; ++i)
+#pragma unroll
+        for (int c = 0; c < C; ++c) S[c][i] = S0 ? S0[part_entry<P>(pp, i) * D + j0 + c] : 0.f;
     const T *const src[4] = {q, k, v, g};
     for (int ts = s0; ts < s1; ts += kRetTile) {
         __syncthreads();
-        load_rows<T, D, 4, gated_fwd_threads<D>()>(src, tiles, base, ts, T_len);
+        {
+            uint4 x[4][TileVec<T, D, NT>::PER];
+            fetch_rows<T, D, 4, NT>(src, x, base, ts, T_len);
+            stash_rows<T, D, 4, NT>(x, tiles);
+        }
         __syncthreads();
         exp_tile<D>(tiles[3]);
         __syncthreads();
         const int nr = min(kRetTile, s1 - ts);
 #pragma unroll 2
         for (int r = 0; r < nr; ++r) {
-            const float vj = tiles[2][r][j];
-            float a[4] = {0.f, 0.f, 0.f, 0.f};
+            const float4 vv = *reinterpret_cast<const float4 *>(&tiles[2][r][j0]);
+            float a[C][4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+                for (int c = 0; c < C; ++c) a[c][e] = 0.f;
 #pragma unroll
             for (int m = 0; m < DP / 4; ++m) {
                 const float4 aa = part_group<P>(tiles[3][r], pp, m), kk = part_group<P>(tiles[1][r], pp, m),
                              qq = part_group<P>(tiles[0][r], pp, m);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    S[4 * m + e] = fmaf(f4(aa, e), S[4 * m + e], f4(kk, e) * vj);
-                    a[e] = fmaf(f4(qq, e), S[4 * m + e], a[e]);
+                    const int i = 4 * m + e;
+#pragma unroll
+                    for (int c = 0; c < C; ++c) {
+                        S[c][i] = fmaf(f4(aa, e), S[c][i], f4(kk, e) * f4(vv, c));
+                        a[c][e] = fmaf(f4(qq, e), S[c][i], a[c][e]);
+                    }
                 }
             }
-            const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
-            if (lead) acc[r][j] = s;
+            float col[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) col[c] = (a[c][0] + a[c][1]) + (a[c][2] + a[c][3]);
+            const float oj = group_reduce_scatter<P>(col, pp);
+            if (pp < C) acc[r][j0 + pp] = oj;
         }
         __syncthreads();
-        for (int e = threadIdx.x; e < nr * D; e += blockDim.x)
+        for (int e = threadIdx.x; e < nr * D; e += NT)
             io<T>::st(o + base + (long long)(ts + e / D) * D + e % D, acc[e / D][e % D]);
     }
 }
 
-// Backward, forward sweep: dq_t[i] = sum_j S_t[i][j] dout_t[j]; thread p of row i holds
-// S[i][j] for its D / P columns j = part_entry(p, .).
+// Backward, forward sweep: dq_t[i] = sum_j S_t[i][j] dout_t[j], row sums over the column groups
+// (the four of a warp by shuffles, the warps through shared memory).
 template <typename T, int D>
-__global__ void __launch_bounds__(gated_fwd_threads<D>())
+__global__ void __launch_bounds__(gated_threads<D>())
 gated_bwd_q(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g, const T *__restrict__ dout,
             T *__restrict__ dq, float *__restrict__ dq32, const float *__restrict__ st_in, int T_len, int L) {
-    constexpr int P = causal_split<D>(), DP = D / P;
-    __shared__ __align__(16) float tiles[4][kRetTile][D];      // k, v, a = exp(g), dout
-    __shared__ float acc[kRetTile][D];
+    constexpr int P = 8, DP = D / P, C = 4, NT = gated_threads<D>(), W = NT / 32;
+    extern __shared__ __align__(16) float dsm[];   // gated_bwd_q_smem<D>() bytes
+    float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // k, v, a = exp(g), dout
+    float(*A)[kRetTile][D] = tiles + 4;                                          // per warp: row sums of dq
     const int s0 = blockIdx.y * L, s1 = min(T_len, s0 + L);
     const long long base = (long long)blockIdx.x * T_len * D;
-    const int i = threadIdx.x / P, pp = threadIdx.x % P;
-    const bool lead = pp == 0;
+    const int grp = threadIdx.x / P, pp = threadIdx.x % P, j0 = C * grp;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rbase = (lane & 16 ? DP / 2 : 0) + (lane & 8 ? DP / 4 : 0);
     const float *const S0 = chunk_state<D, D>(st_in, blockIdx.x, blockIdx.y);
-    float S[DP];
+    float S[C][DP];
 #pragma unroll
-    for (int jj = 0; jj < DP; ++jj) S[jj] = S0 ? S0[i * D + part_entry<P>(pp, jj)] : 0.f;
+    for (int i = 0; i < DP; ++i)
+#pragma unroll
+        for (int c = 0; c < C; ++c) S[c][i] = S0 ? S0[part_entry<P>(pp, i) * D + j0 + c] : 0.f;
     const T *const src[4] = {k, v, g, dout};
     for (int ts = s0; ts < s1; ts += kRetTile) {
         __syncthreads();
-        load_rows<T, D, 4, gated_fwd_threads<D>()>(src, tiles, base, ts, T_len);
+        {
+            uint4 x[4][TileVec<T, D, NT>::PER];
+            fetch_rows<T, D, 4, NT>(src, x, base, ts, T_len);
+            stash_rows<T, D, 4, NT>(x, tiles);
+        }
         __syncthreads();
         exp_tile<D>(tiles[2]);
         __syncthreads();
         const int nr = min(kRetTile, s1 - ts);
 #pragma unroll 2
         for (int r = 0; r < nr; ++r) {
-            const float ai = tiles[2][r][i], ki = tiles[0][r][i];
-            float a[4] = {0.f, 0.f, 0.f, 0.f};
+            const float4 vv = *reinterpret_cast<const float4 *>(&tiles[1][r][j0]);
+            const float4 gv = *reinterpret_cast<const float4 *>(&tiles[3][r][j0]);
+            float ad[DP];
+#pragma unroll
+            for (int i = 0; i < DP; ++i) ad[i] = 0.f;
 #pragma unroll
             for (int m = 0; m < DP / 4; ++m) {
-                const float4 vv = part_group<P>(tiles[1][r], pp, m), gg = part_group<P>(tiles[3][r], pp, m);
+                const float4 aa = part_group<P>(tiles[2][r], pp, m), kk = part_group<P>(tiles[0][r], pp, m);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    S[4 * m + e] = fmaf(ai, S[4 * m + e], ki * f4(vv, e));
-                    a[e] = fmaf(S[4 * m + e], f4(gg, e), a[e]);
+                    const int i = 4 * m + e;
+#pragma unroll
+                    for (int c = 0; c < C; ++c) {
+                        S[c][i] = fmaf(f4(aa, e), S[c][i], f4(kk, e) * f4(vv, c));
+                        ad[i] = fmaf(S[c][i], f4(gv, c), ad[i]);
+                    }
                 }
             }
-            const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
-            if (lead) acc[r][i] = s;
+            float rs[DP / 4];
+            rows_reduce_scatter<DP>(ad, rs, lane);
+#pragma unroll
+            for (int x = 0; x < DP / 4; ++x) A[warp][r][part_entry<P>(pp, rbase + x)] = rs[x];
         }
         __syncthreads();
-        for (int e = threadIdx.x; e < nr * D; e += blockDim.x) {
-            const long long at = base + (long long)(ts + e / D) * D + e % D;
-            io<T>::st(dq + at, acc[e / D][e % D]);
-            dq32[at] = acc[e / D][e % D];            // unrounded, for the log gates' gradient
+        for (int e = threadIdx.x; e < nr * D; e += NT) {
+            const int r = e / D, c = e % D;
+            float d = 0.f;
+#pragma unroll
+            for (int w = 0; w < W; ++w) d += A[w][r][c];
+            const long long at = base + (long long)(ts + r) * D + c;
+            io<T>::st(dq + at, d);
+            dq32[at] = d;                            // unrounded, for the log gates' gradient
         }
     }
 }
 
-// Backward, reverse sweep over R_t = q_t^T dout_t + diag(a_{t+1}) R_{t+1} (R_T = 0): the
-// first P D threads hold the rows of R (dk_t[i] = sum_j R[i][j] v_t[j]), the next P D its
-// columns (dv_t[j] = sum_i k_t[i] R[i][j]).  a_{t+1} of a tile's last row is the first row
-// of the tile after it (kept in `anext`).  The log gates' gradient comes out of the same
-// reverse walk: with G_t = sum_{s<=t} g_s, o_t = sum_{s<=t} (q_t e^{G_t}) . (k_s e^{-G_s}) v_s, so
-// dL/dG_t = q_t dq_t - k_t dk_t and dg_t = sum_{s>=t} (q_s dq_s - k_s dk_s), summed by thread i
-// of each key dimension in fp32 from the unrounded dq (dq32) and dk.
+template <int D>
+constexpr size_t gated_bwd_q_smem() { return (size_t)(4 + gated_threads<D>() / 32) * kRetTile * D * sizeof(float); }
+
+// Backward, reverse sweep over R_t = q_t^T dout_t + diag(a_{t+1}) R_{t+1} (R after the sequence
+// is 0): dk_t[i] = sum_j R[i][j] v_t[j] (row sums over the column groups), dv_t[j] = sum_i k_t[i]
+// R[i][j] (column sums over a group's 8 threads), R held in blocks as S in the forward.  a_{t+1}
+// of a tile's last row is the first row of the tile after it (kept in `anext`).  The log gates'
+// gradient comes out of the same reverse walk: with G_t = sum_{s<=t} g_s,
+// o_t = sum_{s<=t} (q_t e^{G_t}) . (k_s e^{-G_s}) v_s, so dL/dG_t = q_t dq_t - k_t dk_t and
+// dg_t = sum_{s>=t} (q_s dq_s - k_s dk_s), summed by thread i of each key dimension in fp32 from
+// the unrounded dq (dq32) and dk.
 template <typename T, int D>
-__global__ void __launch_bounds__(gated_kv_threads<D>())
+__global__ void __launch_bounds__(gated_threads<D>())
 gated_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ g,
              const T *__restrict__ dout, float *__restrict__ dq32, T *__restrict__ dk, T *__restrict__ dv,
              T *__restrict__ dg, const float *__restrict__ st_in, float *__restrict__ totals, int T_len, int L) {
-    constexpr int P = causal_split<D>(), DP = D / P;
+    constexpr int P = 8, DP = D / P, C = 4, NT = gated_threads<D>(), W = NT / 32;
     extern __shared__ __align__(16) float dsm[];   // gated_bwd_kv_smem<D>() bytes
     float(*tiles)[kRetTile][D] = reinterpret_cast<float(*)[kRetTile][D]>(dsm);   // q, k, v, dout, a = exp(g)
-    float(*res)[kRetTile][D] = tiles + 5;        // dk (rows), dv (columns)
-    float *anext = dsm + 7 * kRetTile * D;       // a of the row after the tile (0 past the sequence)
+    float(*A)[kRetTile][D] = tiles + 5;                                          // per warp: row sums of dk
+    float(*DV)[D] = reinterpret_cast<float(*)[D]>(dsm + (5 + W) * kRetTile * D);  // dv
+    float *anext = dsm + (6 + W) * kRetTile * D;     // a of the row after the tile (0 past the sequence)
     const int s0 = blockIdx.y * L, s1 = min(T_len, s0 + L);
     const long long base = (long long)blockIdx.x * T_len * D;
-    const bool row_side = threadIdx.x < P * D;
-    const int t2 = row_side ? threadIdx.x : threadIdx.x - P * D;
-    const int line = t2 / P, pp = t2 % P;
-    const bool lead = pp == 0;
-    // the entering R (the tokens after this chunk): rows on the row side, columns on the other
+    const int grp = threadIdx.x / P, pp = threadIdx.x % P, j0 = C * grp;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rbase = (lane & 16 ? DP / 2 : 0) + (lane & 8 ? DP / 4 : 0);
+    // the entering R (the tokens after this chunk)
     const float *const R0 = chunk_state<D, D>(st_in, blockIdx.x, blockIdx.y);
-    float Rx[DP];
-    float accg = 0.f;                            // thread i < D: sum over the chunk's rows after t of dL/dG[i]
+    float R[C][DP];
 #pragma unroll
-    for (int m = 0; m < DP; ++m) {
-        const int x = part_entry<P>(pp, m);
-        Rx[m] = !R0 ? 0.f : row_side ? R0[line * D + x] : R0[x * D + line];
-    }
-    for (int e = threadIdx.x; e < D; e += blockDim.x)     // the first gate after the chunk
+    for (int i = 0; i < DP; ++i)
+#pragma unroll
+        for (int c = 0; c < C; ++c) R[c][i] = R0 ? R0[part_entry<P>(pp, i) * D + j0 + c] : 0.f;
+    float accg = 0.f;                            // thread i < D: sum over the chunk's rows after t of dL/dG[i]
+    for (int e = threadIdx.x; e < D; e += NT)    // the first gate after the chunk
         anext[e] = s1 < T_len ? expf(io<T>::ld(g + base + (long long)s1 * D + e)) : 0.f;
     const T *const src[5] = {q, k, v, dout, g};
     for (int ts = s0 + (s1 - s0 - 1) / kRetTile * kRetTile; ts >= s0; ts -= kRetTile) {
         __syncthreads();
-        load_rows<T, D, 5, gated_kv_threads<D>()>(src, tiles, base, ts, T_len);
+        {
+            uint4 x[5][TileVec<T, D, NT>::PER];
+            fetch_rows<T, D, 5, NT>(src, x, base, ts, T_len);
+            stash_rows<T, D, 5, NT>(x, tiles);
+        }
         __syncthreads();
         exp_tile<D>(tiles[4]);
         __syncthreads();
@@ -1420,39 +1468,49 @@ gated_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
 #pragma unroll 2
         for (int r = nr - 1; r >= 0; --r) {
             const float *an = r + 1 < nr ? tiles[4][r + 1] : anext;    // a_{t+1}
-            float a[4] = {0.f, 0.f, 0.f, 0.f};
-            if (row_side) {
-                const float qi = tiles[0][r][line], ai = an[line];
+            const float4 gv = *reinterpret_cast<const float4 *>(&tiles[3][r][j0]);
+            const float4 vv = *reinterpret_cast<const float4 *>(&tiles[2][r][j0]);
+            float ak[DP], av[C][4];
 #pragma unroll
-                for (int m = 0; m < DP / 4; ++m) {
-                    const float4 gg = part_group<P>(tiles[3][r], pp, m), vv = part_group<P>(tiles[2][r], pp, m);
+            for (int i = 0; i < DP; ++i) ak[i] = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        Rx[4 * m + e] = fmaf(ai, Rx[4 * m + e], qi * f4(gg, e));
-                        a[e] = fmaf(Rx[4 * m + e], f4(vv, e), a[e]);
-                    }
-                }
-            } else {
-                const float gj = tiles[3][r][line];
+            for (int e = 0; e < 4; ++e)
 #pragma unroll
-                for (int m = 0; m < DP / 4; ++m) {
-                    const float4 aa = part_group<P>(an, pp, m), qq = part_group<P>(tiles[0][r], pp, m),
-                                 kk = part_group<P>(tiles[1][r], pp, m);
+                for (int c = 0; c < C; ++c) av[c][e] = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        Rx[4 * m + e] = fmaf(f4(aa, e), Rx[4 * m + e], f4(qq, e) * gj);
-                        a[e] = fmaf(f4(kk, e), Rx[4 * m + e], a[e]);
+            for (int m = 0; m < DP / 4; ++m) {
+                const float4 aa = part_group<P>(an, pp, m), qq = part_group<P>(tiles[0][r], pp, m),
+                             kk = part_group<P>(tiles[1][r], pp, m);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 4 * m + e;
+#pragma unroll
+                    for (int c = 0; c < C; ++c) {
+                        R[c][i] = fmaf(f4(aa, e), R[c][i], f4(qq, e) * f4(gv, c));
+                        ak[i] = fmaf(R[c][i], f4(vv, c), ak[i]);
+                        av[c][e] = fmaf(f4(kk, e), R[c][i], av[c][e]);
                     }
                 }
             }
-            const float s = line_sum<P>((a[0] + a[1]) + (a[2] + a[3]));
-            if (lead) res[row_side ? 0 : 1][r][line] = s;
+            float col[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) col[c] = (av[c][0] + av[c][1]) + (av[c][2] + av[c][3]);
+            const float dvj = group_reduce_scatter<P>(col, pp);
+            if (pp < C) DV[r][j0 + pp] = dvj;
+            float rs[DP / 4];
+            rows_reduce_scatter<DP>(ak, rs, lane);
+#pragma unroll
+            for (int x = 0; x < DP / 4; ++x) A[warp][r][part_entry<P>(pp, rbase + x)] = rs[x];
         }
         __syncthreads();
-        for (int e = threadIdx.x; e < nr * D; e += blockDim.x) {
-            const long long at = base + (long long)(ts + e / D) * D + e % D;
-            io<T>::st(dk + at, res[0][e / D][e % D]);
-            io<T>::st(dv + at, res[1][e / D][e % D]);
+        for (int e = threadIdx.x; e < nr * D; e += NT) {
+            const int r = e / D, c = e % D;
+            float a = 0.f;
+#pragma unroll
+            for (int w = 0; w < W; ++w) a += A[w][r][c];
+            const long long at = base + (long long)(ts + r) * D + c;
+            io<T>::st(dk + at, a);
+            io<T>::st(dv + at, DV[r][c]);
         }
         if (threadIdx.x < D) {
             const int i = threadIdx.x;
@@ -1460,21 +1518,26 @@ gated_bwd_kv(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
             for (int r = kRetTile - 1; r >= 0; --r) {
                 if (r >= nr) continue;
                 const long long at = base + (long long)(ts + r) * D + i;
+                float dki = 0.f;
+#pragma unroll
+                for (int w = 0; w < W; ++w) dki += A[w][r][i];
                 accg = fmaf(tiles[0][r][i], dqv[r], accg);
-                accg = fmaf(-tiles[1][r][i], res[0][r][i], accg);
+                accg = fmaf(-tiles[1][r][i], dki, accg);
                 // one chunk: dg itself; several: the chunk's part in fp32, in place of dq32
-                // (this thread's own element, read just above), completed by gated_dg_carry
+                // (this thread's own element, read above), completed by gated_dg_carry
                 if (totals) dq32[at] = accg;
                 else io<T>::st(dg + at, accg);
             }
         }
-        for (int e = threadIdx.x; e < D; e += blockDim.x) anext[e] = tiles[4][0][e];
+        for (int e = threadIdx.x; e < D; e += NT) anext[e] = tiles[4][0][e];
     }
     if (totals && threadIdx.x < D) totals[((long long)blockIdx.x * gridDim.y + blockIdx.y) * D + threadIdx.x] = accg;
 }
 
 template <int D>
-constexpr size_t gated_bwd_kv_smem() { return (size_t)(7 * kRetTile * D + D) * sizeof(float); }
+constexpr size_t gated_bwd_kv_smem() {
+    return (size_t)((6 + gated_threads<D>() / 32) * kRetTile * D + D) * sizeof(float);
+}
 
 // -------------------------------------------------------------- drivers ---
 
@@ -1824,7 +1887,7 @@ la_status gated_fwd_t(const void *q, const void *k, const void *v, const void *g
         const la_status rc = gated_states<T, D, false>(k, v, g, E, A, s, st);
         if (rc) return rc;
     }
-    return launch("simt_gated_fwd", gated_fwd<T, D>, dim3((unsigned)s.BH(), (unsigned)nc), dim3(gated_fwd_threads<D>()),
+    return launch("simt_gated_fwd", gated_fwd<T, D>, dim3((unsigned)s.BH(), (unsigned)nc), dim3(gated_threads<D>()),
                   0, st, (const T *)q, (const T *)k, (const T *)v, (const T *)g, (T *)o, (const float *)E, s.T,
                   kCausalChunk);
 }
@@ -1841,11 +1904,12 @@ la_status gated_bwd_t(const void *q, const void *k, const void *v, const void *g
     float *totals = E ? (float *)(rest + gated_e_bytes(s) + gated_a_bytes(s)) : nullptr;
     la_status rc;
     if (E && (rc = gated_states<T, D, false>(k, v, g, E, A, s, st))) return rc;
-    rc = launch("simt_gated_bwd_q", gated_bwd_q<T, D>, grid, dim3(gated_fwd_threads<D>()), 0, st, (const T *)k,
-                (const T *)v, (const T *)g, (const T *)dout, (T *)dq, dq32, (const float *)E, s.T, kCausalChunk);
+    rc = launch("simt_gated_bwd_q", gated_bwd_q<T, D>, grid, dim3(gated_threads<D>()), gated_bwd_q_smem<D>(), st,
+                (const T *)k, (const T *)v, (const T *)g, (const T *)dout, (T *)dq, dq32, (const float *)E, s.T,
+                kCausalChunk);
     if (rc) return rc;
     if (E && (rc = gated_states<T, D, true>(q, dout, g, E, A, s, st))) return rc;
-    rc = launch("simt_gated_bwd_kv", gated_bwd_kv<T, D>, grid, dim3(gated_kv_threads<D>()), gated_bwd_kv_smem<D>(), st,
+    rc = launch("simt_gated_bwd_kv", gated_bwd_kv<T, D>, grid, dim3(gated_threads<D>()), gated_bwd_kv_smem<D>(), st,
                 (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const T *)dout, dq32, (T *)dk, (T *)dv,
                 (T *)dg, (const float *)E, totals, s.T, kCausalChunk);
     if (rc || !E) return rc;
