@@ -56,18 +56,18 @@ KERNEL_TENSORS = {
     "tc_retention_fwd": 4, "tc_retention_bwd": 7,
 }
 
-# CUDA-core (FMA) work of the recurrent causal-norm kernels per token-head, in flops (2 per FMA):
-# the forward's D+1 state columns each take D FMAs to update and D to form the output; the dq
-# pass adds the D rows (update and row sum); the dk, dv pass holds D rows and D columns.
+# CUDA-core work of the recurrent kernels per token-head, in flops (2 per multiply-add, 1 per
+# other product), counting the state once (the arithmetic the recurrence needs, not a layout's):
+# causal-norm forward: the D + 1 columns of [S | z] updated and read out, D FMAs each; dq sweep:
+# those plus the D row sums of S.dO; reverse sweep: R and r updated, the row sums (dk) and the
+# column sums (dv).  Gated: a state entry's update a_i S_ij + k_i v_j is 3 flops, a read-out 2.
 CAUSAL_FLOPS = {
     "simt_causal_norm_fwd": lambda D: 4 * D * (D + 1),
-    "simt_causal_norm_bwd_q": lambda D: 4 * D * (D + 1) + 4 * D * D,
-    "simt_causal_norm_bwd_kv": lambda D: 8 * D * D,
-    # gated: the D columns (forward) or rows (dq) of S, each D FMAs to update and D to read out;
-    # the reverse sweep holds the rows and the columns of R
-    "simt_gated_fwd": lambda D: 4 * D * D,
-    "simt_gated_bwd_q": lambda D: 4 * D * D,
-    "simt_gated_bwd_kv": lambda D: 8 * D * D,
+    "simt_causal_norm_bwd_q": lambda D: 4 * D * (D + 1) + 2 * D * D,
+    "simt_causal_norm_bwd_kv": lambda D: 6 * D * D + 2 * D,
+    "simt_gated_fwd": lambda D: 5 * D * D,
+    "simt_gated_bwd_q": lambda D: 5 * D * D,
+    "simt_gated_bwd_kv": lambda D: 7 * D * D + 4 * D,
 }
 
 
