@@ -16,6 +16,12 @@
 // forms of linear attention", FusedRecurrent): one CTA per (b,h) walks T
 // with the D x D state held in registers, one state column (or row) per
 // thread.
+// Causal linear attention with the norm term and gated linear attention (the
+// same recurrent form, with the norm term of the bidirectional op, resp. gates
+// per token and key dimension): the sequence in chunks of 256 tokens, each
+// chunk's own state from a zero state (causal_chunk_state / gated_chunk_state),
+// a scan over the chunks (chunk_scan), and one CTA per (b,h, chunk) walking its
+// chunk with the state held once in register blocks of four columns.
 #include "la_internal.cuh"
 
 #include <string.h>
@@ -584,13 +590,10 @@ __device__ __forceinline__ void feature_tiles(float (*tiles)[kRetTile][D], int n
 template <bool PHI>
 __device__ __forceinline__ float feature_grad_of(float fx) { return PHI ? (fx > 1.f ? 1.f : fx) : 1.f; }
 
-// Each state line (a column or a row of S, or z) is split over P threads: thread p of a
-// line takes the D / P entries part_entry(p, 0 .. D / P - 1) of it, and the line's P partial
-// dot products meet through xor shuffles among P adjacent lanes (fixed order).  Blocks are
-// whole warps; the threads past the last line compute on zeros and store nothing.
-template <int D> constexpr int causal_split() { return D == 64 ? 4 : 2; }
-template <int N> constexpr int round_warps(int n) { return (n + 31) / 32 * 32; }
-// forward: column groups of four, each over D / 8 threads of 8 rows (part_entry)
+// The state is held in register blocks: the threads of a column group (P adjacent lanes) hold
+// four columns of it, thread p the rows part_entry(p, 0 ..), and partial sums meet through xor
+// shuffles among those lanes (fixed order).
+// forward: column groups of four, each over D / 8 threads of 8 rows
 template <int D> constexpr int causal_fwd_parts() { return D / 8; }
 template <int D> constexpr int causal_fwd_threads() { return D / 4 * causal_fwd_parts<D>(); }
 // dq sweep: column groups of four, each over 8 threads of D / 8 rows
@@ -1144,7 +1147,7 @@ constexpr size_t causal_bwd_kv_smem() {
 // ------------------------------------------------------ gated linear attention ---
 // Per-token, per-key-dimension decay, the recurrent form:
 //   S_t = diag(a_t) S_{t-1} + k_t^T v_t,  o_t = q_t S_t,  a_t = exp(g_t), g the log gates.
-// The state lines are split over P threads as in the causal-norm kernels.
+// The state is held in register blocks as in the causal-norm kernels.
 
 // exp of a gate tile in place (rows past the sequence are never read)
 template <int D>
