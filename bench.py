@@ -133,9 +133,20 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def source_hash() -> str:
+# The files the tensor-core kernels are compiled from (their launch code included): a change
+# anywhere else in the library leaves those kernels, and their DRAM traffic, as they were.
+TC_SOURCES = ("la_tc.cu", "la_tc.cuh", "la_tc_state.cu", "la_tc_retention.cu", "la_tc_common.cuh", "la_tc_ptx.cuh",
+              "la_internal.cuh")
+
+
+def source_hash(names=None) -> str:
+    """sha256 prefix of the library's kernel sources (every csrc file, or those in `names`) and
+    of include/la.h."""
+    csrc = os.path.join(ROOT, "linear_attention_attn_b200", "csrc")
+    paths = sorted(glob.glob(os.path.join(csrc, "*"))) if names is None else \
+        sorted(os.path.join(csrc, n) for n in names)
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "linear_attention_attn_b200", "csrc", "*"))):
+    for p in paths + [os.path.join(ROOT, "include", "la.h")]:
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode())
             h.update(f.read())
@@ -152,7 +163,7 @@ def ncu_traffic(kernel: str, T: int):
     except Exception:
         return None
     e = rec.get(kernel)
-    if not e or e.get("source_sha") != source_hash():
+    if not e or e.get("source_sha") != source_hash(TC_SOURCES):
         return None
     return float(e["dram_bytes_per_launch"]) * (T / float(e["T"]))
 
