@@ -1164,16 +1164,18 @@ template <int D> constexpr int gated_threads() { return D / 4 * 8; }
 //     A[c][i] = exp(sum_{u=s0}^{s1-1} g_u[i])   (S after the chunk = diag(A) S before + E);
 //   reverse (REV true):  E[c][i][j] = sum_t exp(sum_{u=s0+1}^{t} g_u[i]) q_t[i] dout_t[j],
 //     A[c][i] = exp(sum_{u=s0+1}^{s1} g_u[i])   (R at s0 = E + diag(A) R at s1; no g past T).
-// E is [B H][chunk][D][D], A [B H][chunk][D]; threads < D form the weights of column i, all
-// 256 accumulate rows 4 ti + 64 m + 0..3 by columns 4 tj + 64 n + 0..3 as causal_chunk_state.
+// E is [B H][chunk][D][D], A [B H][chunk][D]; the 256 threads form the weights (256 / D per key
+// dimension) and accumulate rows 4 ti + 64 m + 0..3 by columns 4 tj + 64 n + 0..3 as
+// causal_chunk_state.
 template <typename T, int D, bool REV>
 __global__ void __launch_bounds__(256)
 gated_chunk_state(const T *__restrict__ a_src, const T *__restrict__ b_src, const T *__restrict__ g,
                   float *__restrict__ E, float *__restrict__ A, int T_len, int L) {
-    constexpr int G = D / 64, R = chunk_state_rows<D>();
+    constexpr int G = D / 64, R = chunk_state_rows<D>(), TPC = 256 / D, RPT = R / TPC;
     __shared__ __align__(16) float As[R][D];
     __shared__ __align__(16) float Bs[R][D];
     __shared__ float Gs[R][D];
+    __shared__ float Part[TPC][D];
     const int c = blockIdx.x, bh = blockIdx.y, nc = gridDim.x;
     if (REV ? c == 0 : c == nc - 1) return;    // no other chunk starts from this one's state
     const int s0 = c * L, s1 = min(T_len, s0 + L), ntiles = (s1 - s0 + R - 1) / R;
@@ -1184,7 +1186,7 @@ gated_chunk_state(const T *__restrict__ a_src, const T *__restrict__ b_src, cons
     for (int m = 0; m < 4 * G; ++m)
 #pragma unroll
         for (int n = 0; n < 4 * G; ++n) acc[m][n] = 0.f;
-    float run = 0.f;                           // thread i < D: the running sum of log gates
+    float run = 0.f;                           // the running sum of log gates of dimension threadIdx.x % D
     // the tiles in the order they are summed (forward: from the chunk's end), each fetched into
     // registers while the one before it is weighted and summed
     constexpr int EPT = R * D / 256;
@@ -1210,24 +1212,41 @@ gated_chunk_state(const T *__restrict__ a_src, const T *__restrict__ b_src, cons
             const int e = threadIdx.x + 256 * u;
             As[e / D][e % D] = ra[u];
             Bs[e / D][e % D] = rb[u];
-            Gs[e / D][e % D] = rg[u];
+            Gs[e / D][e % D] = REV && ts + e / D == s0 ? 0.f : rg[u];   // the reverse sums start after s0
         }
         __syncthreads();
         if (n + 1 < ntiles) LA_GATED_FETCH(n + 1);
-        if (threadIdx.x < D) {
-            const int i = threadIdx.x;
-            if (REV) {
-                for (int r = 0; r < nr; ++r) {
-                    if (ts + r > s0) run += Gs[r][i];
-                    As[r][i] *= expf(run);
-                }
-            } else {
-                for (int r = nr - 1; r >= 0; --r) {
-                    As[r][i] *= expf(run);
-                    run += Gs[r][i];
-                }
+        // the weights: running sums of the log gates of key dimension i over the tile, its rows
+        // split over TPC threads of RPT rows each (thread part qd; parts meet in shared memory)
+        const int i = threadIdx.x % D, qd = threadIdx.x / D;
+        float loc = 0.f;
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) loc += Gs[qd * RPT + j][i];
+        Part[qd][i] = loc;
+        __syncthreads();
+        float before = 0.f, after = 0.f;        // the parts of the rows before and after this part's
+#pragma unroll
+        for (int q2 = 0; q2 < TPC; ++q2) {
+            if (q2 < qd) before += Part[q2][i];
+            if (q2 > qd) after += Part[q2][i];
+        }
+        if (REV) {                              // exp of the sum up to and including the row
+            float sum = run + before;
+#pragma unroll
+            for (int j = 0; j < RPT; ++j) {
+                sum += Gs[qd * RPT + j][i];
+                As[qd * RPT + j][i] *= expf(sum);
+            }
+        } else {                                // exp of the sum of the rows after it
+            float sum = run + after;
+#pragma unroll
+            for (int j = RPT - 1; j >= 0; --j) {
+                As[qd * RPT + j][i] *= expf(sum);
+                sum += Gs[qd * RPT + j][i];
             }
         }
+#pragma unroll
+        for (int q2 = 0; q2 < TPC; ++q2) run += Part[q2][i];
         __syncthreads();
         for (int r = 0; r < nr; ++r) {
             float a[4 * G], b[4 * G];
