@@ -154,17 +154,23 @@ def source_hash(names=None) -> str:
 
 
 def ncu_traffic(kernel: str, T: int):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
-    current kernel sources (else None)."""
+    """DRAM bytes per launch of `kernel` at sequence length T from the committed ncu summaries:
+    of the captures taken on the current kernel sources, the one whose T is nearest, scaled by T
+    (None when no capture matches the sources)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
     except Exception:
         return None
-    e = rec.get(kernel)
-    if not e or e.get("source_sha") != source_hash(TC_SOURCES):
+    entries = rec.get(kernel) or []
+    if isinstance(entries, dict):
+        entries = [entries]
+    sha = source_hash(TC_SOURCES)
+    ok = [e for e in entries if e.get("source_sha") == sha]
+    if not ok:
         return None
+    e = min(ok, key=lambda e: abs(math.log(float(e["T"]) / T)))
     return float(e["dram_bytes_per_launch"]) * (T / float(e["T"]))
 
 
@@ -342,6 +348,9 @@ WORKLOAD_TEXT = {
              "fp32 accumulate, "
              "B=%d H=%d T=%d D=%d, log gates log(sigmoid(N(0,1)))/16 per token and key dimension, "
              "q ~ N(0,1) D^-1/2, k, v, dO ~ N(0,1)",
+    "vision": "long-sequence vision-style bidirectional linear attention fwd only, fp16 storage / fp32 accumulate, "
+              "B=%d H=%d T=%d D=%d (256x256 token grid), phi=elu+1, eps=1e-06, Q,K,V ~ 0.5 N(0,1) plus a smooth 2-D "
+              "sinusoidal offset of amplitude 0.1",
     "causal_norm": "causal linear attention with the norm term fwd+bwd (recurrent form in 256-token chunks on CUDA "
                    "cores), fp16 storage / "
                    "fp32 accumulate, B=%d H=%d T=%d D=%d, phi=elu+1, no decay, eps=1e-06, Q,K,V ~ 0.5 N(0,1), "
@@ -382,6 +391,120 @@ def time_step_at(la, w, dev, stream, steps, warmup):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     return e0.elapsed_time(e1) / steps
+
+
+class L2Flush:
+    """Writes a buffer twice the size of L2 (between timed steps whose data fits in L2)."""
+
+    def __init__(self, dev):
+        self.buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1.0)
+
+
+def time_each(fn, steps, warmup, stream, flush=None):
+    """Mean device time (ms) of fn() over `steps` calls, each bracketed by its own events on
+    `stream`; with `flush`, L2 is overwritten before every call, outside the events."""
+    for _ in range(warmup):
+        fn()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        if flush is not None:
+            flush()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / steps
+
+
+# Sub-records of the default line: every workload of the specification besides the headline,
+# at the sizes it names (simple_la and retention T sweeps, the vision forward), plus the causal
+# norm and gated ops at the headline shape.  (workload, T values, forward only)
+CONFIG_RECORDS = (("simple_bf16", (128, 1024, 4096, 16384), False),
+                  ("retention_bf16", (2048, 8192), False),
+                  ("vision_f16", (65536,), True),
+                  ("causal_norm_f16", (4096,), False),
+                  ("gated_bf16", (4096,), False))
+
+
+def config_records(la, dev, stream):
+    """Device-timed fwd+bwd (or fwd) of the other workloads: ms per step, tokens/s, GB/s at the
+    algorithmic bytes (4 tensors forward, 7 backward, of [B,H,T,D] in the storage dtype) and the
+    fraction of the measured copy bandwidth.  Each call timed on its own, L2 flushed in between
+    when a step's data fits in L2."""
+    peak, peak_kind = measured_peaks()
+    flush = L2Flush(dev)
+    out = {}
+    for base, Ts, fwd_only in CONFIG_RECORDS:
+        recs = []
+        for T in Ts:
+            w = synth.WORKLOADS[base].with_T(T)
+            host = synth.make_inputs(w, seed=0, with_grad=not fwd_only)
+            q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
+            g = host["do"].to(dev) if not fwd_only else None
+            o = torch.empty_like(q)
+            dq, dk, dv = ((torch.empty_like(q) for _ in range(3)) if not fwd_only else (None, None, None))
+            B, H, D = w.B, w.H, w.D
+            st = torch.empty((B, H, D, D + 1), dtype=torch.float32, device=dev)
+            ops = {"bidir": ("bidir_fwd", "bidir_bwd"), "simple": ("simple_fwd", "simple_bwd"),
+                   "retention": ("chunk_decay_fwd", "chunk_decay_bwd"),
+                   "causal_norm": ("causal_norm_fwd", "causal_norm_bwd"), "gated": ("gated_fwd", "gated_bwd")}[w.op]
+            nws = max(la.la_workspace_size(n, B, H, T, D, q.dtype) for n in ops)
+            ws = torch.empty(max(256, nws), dtype=torch.uint8, device=dev)
+            lg = host["g"].to(dev) if w.op == "gated" else None
+            dg = torch.empty_like(q) if w.op == "gated" else None
+            gam = host.get("gamma")
+
+            def fwd():
+                if w.op == "bidir":
+                    la.la_bidir_fwd(q, k, v, o, st, eps=w.eps, workspace=ws)
+                elif w.op == "simple":
+                    la.la_simple_fwd(q, k, v, o, st, workspace=ws)
+                elif w.op == "retention":
+                    la.la_chunk_decay_fwd(q, k, v, o, gam, workspace=ws)
+                elif w.op == "causal_norm":
+                    la.la_causal_norm_fwd(q, k, v, o, None, "elu1", w.eps, workspace=ws)
+                else:
+                    la.la_gated_fwd(q, k, v, lg, o, workspace=ws)
+
+            def bwd():
+                if w.op == "bidir":
+                    la.la_bidir_bwd(q, k, v, g, dq, dk, dv, st, eps=w.eps, workspace=ws)
+                elif w.op == "simple":
+                    la.la_simple_bwd(q, k, v, g, dq, dk, dv, st, workspace=ws)
+                elif w.op == "retention":
+                    la.la_chunk_decay_bwd(q, k, v, g, gam, dq, dk, dv, workspace=ws)
+                elif w.op == "causal_norm":
+                    la.la_causal_norm_bwd(q, k, v, g, dq, dk, dv, None, "elu1", w.eps, workspace=ws)
+                else:
+                    la.la_gated_bwd(q, k, v, lg, g, dq, dk, dv, dg, workspace=ws)
+
+            tb = B * H * T * D * q.element_size()
+            step_bytes = (4 if fwd_only else 11) * tb
+            fl = flush if step_bytes < 2 * L2_BYTES else None
+            n = 100 if step_bytes < 64e6 else 20
+            ms_f = time_each(fwd, n, 3, stream, fl)
+            rec = {"T": T, "B": B, "H": H, "D": D, "dtype": w.dtype, "fwd_ms": ms_f,
+                   "fwd_frac": 4 * tb / (ms_f / 1e3) / 1e9 / peak}
+            ms = ms_f
+            if not fwd_only:
+                ms_b = time_each(bwd, n, 3, stream, fl)
+                ms_s = time_each(lambda: (fwd(), bwd()), n, 3, stream, fl)
+                rec.update(bwd_ms=ms_b, bwd_frac=7 * tb / (ms_b / 1e3) / 1e9 / peak)
+                ms = ms_s
+            rec.update(ms_per_step=ms, tokens_per_s=B * T / (ms / 1e3),
+                       achieved_gbs=step_bytes / (ms / 1e3) / 1e9, frac=step_bytes / (ms / 1e3) / 1e9 / peak,
+                       l2_flushed=fl is not None)
+            recs.append(rec)
+            del q, k, v, g, o, dq, dk, dv, st, ws, lg, dg
+            torch.cuda.empty_cache()
+        out[base] = {"workload": WORKLOAD_TEXT[synth.WORKLOADS[base].op if base != "vision_f16" else "vision"]
+                     % (synth.WORKLOADS[base].B, synth.WORKLOADS[base].H, Ts[-1], synth.WORKLOADS[base].D),
+                     "step": "fwd" if fwd_only else "fwd+bwd", "peak_gbs": peak, "peak_source": peak_kind,
+                     "records": recs}
+    return out
 
 
 def run_ours(args, w):
@@ -614,6 +737,12 @@ def run_ours(args, w):
                           "achieved_gbs": b_s / (ms_s / 1e3) / 1e9,
                           "frac": b_s / (ms_s / 1e3) / 1e9 / measured_peaks()[0]})
 
+    # ---- the other workloads of the specification, device-timed (rank 0's GPU, N = 1 only)
+    configs = None
+    if world == 1 and args.sweep and w.op == "bidir" and not seqpar:   # the headline's tensors went with the sweep
+        torch.cuda.empty_cache()
+        configs = config_records(la, dev, stream)
+
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
@@ -637,7 +766,7 @@ def run_ours(args, w):
         "scaling": "strong" if seqpar else "weak",
         "vs_baseline": vs, "dtype": w.dtype, "data": "synthetic", "config": config_of(w, args),
         "roofline": roof, "step_roofline": step_roof, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": launches, "clocks": clocks, "t_sweep": sweep,
+        "gpu_launches": launches, "clocks": clocks, "t_sweep": sweep, "configs": configs,
         "kernels": [{"name": n, "launches": c, "total_ms": t} for n, c, t in per_kernel],
         "kernel_timing": "per-kernel CUDA events on the launch stream over %d further steps after the timed region" % k_prof,
     }

@@ -113,6 +113,10 @@ la_status la_bidir_fwd(const void *q, const void *k, const void *v, void *o, flo
 /* Size of the scratch array built into the library for la_bidir_fwd_static (32 MiB). */
 #define LA_STATIC_SCRATCH_BYTES (32u << 20)
 
+/* LA_STATIC_SCRATCH_BYTES as the built library has it (for bindings that do not
+ * read this header). */
+size_t la_static_scratch_bytes(void);
+
 /* la_bidir_fwd without a workspace argument, for callers that cannot allocate
  * device memory: code inside a host framework that owns the CUDA allocator and
  * only hands out the tensors it manages, plugins in a serving process, or
@@ -125,7 +129,12 @@ la_status la_bidir_fwd(const void *q, const void *k, const void *v, void *o, flo
  *  - Shapes whose la_workspace_size(LA_OP_BIDIR_FWD, ...) exceeds
  *    LA_STATIC_SCRATCH_BYTES return LA_ERR_WORKSPACE (see la_last_error()).
  *  - The first call on each device looks up the array's device address on that
- *    device (the current one); make that first call before any stream capture.
+ *    device (the current one), and so does the first call after the current
+ *    CUDA context changed (cudaDeviceReset, a re-created primary context, a
+ *    driver-API context made current): the address is kept per device with the
+ *    id of the context it belongs to.  Make that first call before any stream
+ *    capture: during a capture it returns LA_ERR_INVALID_ARG.  Calls whose
+ *    shape or dtype is invalid look nothing up (la_bidir_fwd reports them).
  *  - All calls share the array and it keeps the last call's contents; calls
  *    that overlap on the GPU (unordered streams or host threads) race on it.
  *    Nothing needs clearing between calls.                                    */

@@ -76,6 +76,8 @@ for _n in ("la_bidir_fwd", "la_simple_fwd", "la_bidir_bwd", "la_simple_bwd", "la
     getattr(_lib, _n).restype = _I
 _lib.la_bidir_fwd_static.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.la_bidir_fwd_static.restype = _I
+_lib.la_static_scratch_bytes.argtypes = []
+_lib.la_static_scratch_bytes.restype = _Z
 _lib.la_status_string.argtypes = [_I]
 _lib.la_status_string.restype = ctypes.c_char_p
 _lib.la_last_error.argtypes = []
@@ -191,7 +193,12 @@ def la_bidir_fwd_static(q, k, v, o, state=None, eps: float = 1e-6, stream=None):
                                     _stream(stream, q.device)), "la_bidir_fwd_static")
 
 
-STATIC_SCRATCH_BYTES = 32 << 20
+def la_static_scratch_bytes() -> int:
+    """Bytes of the scratch array built into the library for la_bidir_fwd_static."""
+    return int(_lib.la_static_scratch_bytes())
+
+
+STATIC_SCRATCH_BYTES = la_static_scratch_bytes()
 
 
 def la_simple_fwd(q, k, v, o, state=None, workspace=None, stream=None):

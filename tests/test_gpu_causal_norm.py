@@ -51,7 +51,7 @@ def test_matches_oracle(dtype, D, T, feature, decayed):
     o, dq, dk, dv = _run(inp, decay, feature, eps)
     want_o = oracle.causal_norm_fwd(inp["q"], inp["k"], inp["v"], decay, feature, eps)
     want = oracle.causal_norm_bwd(inp["q"], inp["k"], inp["v"], inp["do"], decay, feature, eps)
-    pu.assert_fwd(o, want_o, "o")
+    pu.assert_fwd(o, want_o, "o", dtype=inp["q"].dtype)
     for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
         pu.assert_grad(got, ref, name)
 
@@ -65,7 +65,7 @@ def test_single_token(dtype):
     o, dq, dk, dv = _run(inp, None, "elu1", 1e-6)
     want_o = oracle.causal_norm_fwd(inp["q"], inp["k"], inp["v"], None, "elu1", 1e-6)
     want = oracle.causal_norm_bwd(inp["q"], inp["k"], inp["v"], inp["do"], None, "elu1", 1e-6)
-    pu.assert_fwd(o, want_o, "o")
+    pu.assert_fwd(o, want_o, "o", dtype=inp["q"].dtype)
     pu.assert_grad(dv, want[2], "dv")
     assert pu.max_abs(dq, want[0]) < 1e-3 and pu.max_abs(dk, want[1]) < 1e-3
 
@@ -79,7 +79,7 @@ def test_benchmark_size_sampled_heads():
         sel = {n: inp[n][b:b + 1, h:h + 1] for n in ("q", "k", "v", "do")}
         want_o = oracle.causal_norm_fwd(sel["q"], sel["k"], sel["v"], None, "elu1", w.eps)
         want = oracle.causal_norm_bwd(sel["q"], sel["k"], sel["v"], sel["do"], None, "elu1", w.eps)
-        pu.assert_fwd(o[b:b + 1, h:h + 1], want_o, "o (%d,%d)" % (b, h))
+        pu.assert_fwd(o[b:b + 1, h:h + 1], want_o, "o (%d,%d)" % (b, h), dtype=inp["q"].dtype)
         for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
             pu.assert_grad(got[b:b + 1, h:h + 1], ref, "%s (%d,%d)" % (name, b, h))
 

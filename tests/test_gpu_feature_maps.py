@@ -38,7 +38,7 @@ def test_feature_map_matches_oracle(dtype, D, kind, p):
     torch.cuda.synchronize()
     want_y = oracle.feature_map_fwd(kind, x.double().numpy(), p)
     want_dx = oracle.feature_map_bwd(kind, x.double().numpy(), dy.double().numpy(), p)
-    pu.assert_fwd(y.cpu().double().numpy(), want_y, "%s y" % kind)
+    pu.assert_fwd(y, want_y, "%s y" % kind)
     pu.assert_grad(dx.cpu().double().numpy(), want_dx, "%s dx" % kind)
 
 
@@ -73,7 +73,7 @@ def test_normed_stages_match_oracle(dtype, D):
     got = _stages(la, *(t.to(dev) for t in (q, k, v, g)), 1e-6)
     torch.cuda.synchronize()
     qn, kn, vn, gn = (t.double().numpy() for t in (q, k, v, g))
-    pu.assert_fwd(got[0].cpu().double().numpy(), oracle.normed_fwd(qn, kn, vn, eps=1e-6), "o")
+    pu.assert_fwd(got[0], oracle.normed_fwd(qn, kn, vn, eps=1e-6), "o")
     for name, t, r in zip(("dq", "dk", "dv"), got[1:], oracle.normed_bwd(qn, kn, vn, gn, eps=1e-6)):
         pu.assert_grad(t.cpu().double().numpy(), r, name)
 
@@ -98,7 +98,7 @@ def test_focused_linear_attention_end_to_end(dtype):
     qn, kn, vn, gn = (t.double().numpy() for t in (q, k, v, g))
     fqn = _stored(oracle.feature_map_fwd("focused", qn, p), dtype)
     fkn = _stored(oracle.feature_map_fwd("focused", kn, p), dtype)
-    pu.assert_fwd(o.cpu().double().numpy(), oracle.normed_fwd(fqn, fkn, vn, eps=eps), "o")
+    pu.assert_fwd(o, oracle.normed_fwd(fqn, fkn, vn, eps=eps), "o")
     wdfq, wdfk, wdv = oracle.normed_bwd(fqn, fkn, vn, gn, eps=eps)
     pu.assert_grad(dv.cpu().double().numpy(), wdv, "dv")
     pu.assert_grad(dq.cpu().double().numpy(), oracle.feature_map_bwd("focused", qn, wdfq, p), "dq")
@@ -126,7 +126,7 @@ def test_polarity_split_attention_end_to_end():
     qn, kn, vn, gn = (t.double().numpy() for t in (q, k, v, g))
     fqn = _stored(oracle.feature_map_fwd("polarity", qn), "bf16")          # exact: relu of bf16 values
     fkn = _stored(oracle.feature_map_fwd("polarity_swap", kn), "bf16")
-    pu.assert_fwd(o.cpu().double().numpy(), oracle.normed_fwd(fqn, fkn, vn, eps=eps), "o")
+    pu.assert_fwd(o, oracle.normed_fwd(fqn, fkn, vn, eps=eps), "o")
     wdfq, wdfk, wdv = oracle.normed_bwd(fqn, fkn, vn, gn, eps=eps)
     pu.assert_grad(dv.cpu().double().numpy(), wdv, "dv")
     pu.assert_grad(dq.cpu().double().numpy(), oracle.feature_map_bwd("polarity", qn, wdfq), "dq")

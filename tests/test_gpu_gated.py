@@ -46,7 +46,7 @@ def _ref(inp):
 def test_matches_oracle(dtype, D, T):
     inp = _inputs(dtype, 2, 3, T, D, seed=61)
     got, want = _run(inp), _ref(inp)
-    pu.assert_fwd(got[0], want[0], "o")
+    pu.assert_fwd(got[0], want[0], "o", dtype=inp["q"].dtype)
     for name, a, b in zip(("dq", "dk", "dv", "dg"), got[1:], want[1:]):
         pu.assert_grad(a, b, name)
 
@@ -75,7 +75,7 @@ def test_benchmark_size_sampled_heads():
     for b, h in ((0, 0), (4, 9), (7, 15)):
         sel = {n: inp[n][b:b + 1, h:h + 1] for n in inp}
         want = _ref(sel)
-        pu.assert_fwd(got[0][b:b + 1, h:h + 1], want[0], "o (%d,%d)" % (b, h))
+        pu.assert_fwd(got[0][b:b + 1, h:h + 1], want[0], "o (%d,%d)" % (b, h), dtype=inp["q"].dtype)
         for name, a, r in zip(("dq", "dk", "dv", "dg"), got[1:], want[1:]):
             pu.assert_grad(a[b:b + 1, h:h + 1], r, "%s (%d,%d)" % (name, b, h))
 
