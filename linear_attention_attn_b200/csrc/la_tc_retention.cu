@@ -11,22 +11,18 @@
 // which is o_t = sum_{s<=t} gamma^(t-s) (q_t . k_s) v_s regrouped by chunk.
 //
 // One CTA per (b, h) walks the chunks in order.  Warp 0 streams q/k/v chunks
-// with TMA (two 64-column boxes per 64-row chunk, 128-byte swizzle); warp 1
-// issues the UMMAs of chunk c in the order dS, O_intra, P of chunk c + 1,
-// O_inter, so that dS (which does not depend on the state), O_intra and the
-// next P run while the state is being carried; warps 2..5 form the masked
-// P~ = P o M (hi + lo bf16; the M = 64 accumulator rows spread over all 32
-// lanes of a warp); warps 6..9 combine the two output accumulators and store
-// o; warps 10..17 hold the fp32 state S <- gamma^C S + dS in registers, write
-// it to shared memory as the bf16 hi + lo B operand of Q S, and form
-// K^ = diag(gamma^(C-1-j)) K of the next chunk (hi + lo) while Q S runs.  The
-// chain from one chunk to the next is O_inter (reads S_c) -> state operand
-// write -> O_inter of the next chunk.
-//   P       M=64  N=64  K=128  A = Q (K-major)        B = K (K-major)
-//   O_intra M=64  N=128 K=64   A = P~ hi, lo (K-major) B = V (MN-major)
-//   O_inter M=64  N=128 K=128  A = Q (K-major)        B = S hi, lo (MN-major)
-//   dS      M=128 N=128 K=64   A = K^ hi, lo (MN-major) B = V (MN-major)
-//
+// with TMA (two 64-column boxes per 64-row chunk, 128-byte swizzle) into three
+// stages, so the loads of the next two chunks are in flight while one is
+// computed; warp 1 issues the UMMAs; warps 2..5 form the masked P~ = P o M (hi +
+// lo bf16; the M = 64 accumulator rows spread over all 32 lanes of a warp); warps
+// 6..9 combine the two output parts and store o; warps 10..17 hold the fp32 state
+// in registers and form K^ = diag(gamma^(C-1-j)) K of the next chunk (hi + lo).
+// The outputs are computed transposed, O^T = V^T P~^T + S^T Q^T (M = 128, the
+// value dimension), so that the state, kept by the state warps as S^T, is the
+// A operand of O_inter^T straight from tensor memory (bf16 hi + lo, written with
+// tcgen05.st): it needs no shared memory, which goes to the third stage.  The
+// chain from one chunk to the next is O_inter^T (reads S_c) -> state operand
+// write -> O_inter^T of the next chunk.
 // The backward reuses the same kernel: with R_s = sum_{t>=s} gamma^(t-s) q_t^T dO_t,
 //   dq_t = sum_{s<=t} gamma^(t-s) (dO_t . v_s) k_s   = retention(dO, V, K)
 //   dv_s = sum_{t>=s} gamma^(t-s) (k_s . q_t) dO_t   = retention run backwards in time on (K, Q, dO)
@@ -82,33 +78,40 @@ static __device__ __noinline__ void scale_split_row(const uint8_t *src, uint8_t 
     }
 }
 
-// Stores 16 columns (16*c16 .. +15, c16 in 0..7) of row `row` of a 128-column tile
-// kept as boxes of 64 columns, `box_bytes` apart.
-__device__ __forceinline__ void st16_wide(uint8_t *t, int box_bytes, int row, int c16, const float (&v)[16]) {
-    store_chunk16<true>(t + (c16 >> 2) * box_bytes, row, c16 & 3, v);
-}
-
 // Warp roles: 0 TMA, 1 UMMA, 2..5 decay mask, 6..9 output, 10..17 state and K^
 // (two warps per TMEM lane quadrant, 64 state columns each).
 constexpr int kRXWarps = 4, kROw0 = 6, kROWarps = 4, kRSw0 = 10, kRSWarps = 8;   // mask warps 2..5
 constexpr int kRThreads = (kRSw0 + kRSWarps) * 32;
 
+// Shared memory: three stages of q/k/v chunks (so that the loads of the next two
+// chunks are in flight while one is computed), K^ and P~ (hi + lo each), the output
+// staging chunk, the decay powers and the barriers.  The state lives in tensor memory.
 struct RetLayout {
-    static constexpr int NST = 2;
+    static constexpr int NST = 3;
     static constexpr int qoff = 0;                              // [NST] q chunk (2 boxes)
     static constexpr int koff = qoff + NST * kTile128;
     static constexpr int voff = koff + NST * kTile128;
-    static constexpr int khoff = voff + NST * kTile128;         // k^ hi, lo
+    static constexpr int khoff = voff + NST * kTile128;         // K^ hi, lo
     static constexpr int ptoff = khoff + 2 * kTile128;          // P~ hi, lo: [64 x 64] each
-    static constexpr int soff = ptoff + 2 * kBox;               // S hi, lo: [128 x 128] each (2 x 16 KB)
-    static constexpr int ooff = soff + 2 * 2 * 16384;           // output staging chunk
-    static constexpr int gpoff = ooff + kTile128;               // gamma^k, k = 0..128
-    static constexpr int baroff = gpoff + 132 * 4;
-    static constexpr int nbars = 2 * NST + 10;
+    static constexpr int ooff = ptoff + 2 * kBox;               // output staging chunk
+    static constexpr int gpoff = ooff + kTile128;               // gamma^k, k = -64..128
+    static constexpr int baroff = gpoff + 196 * 4;
+    static constexpr int nbars = 2 * NST + 16;
     static constexpr int misc = baroff + nbars * 8;
     static constexpr int bytes = misc + 32 + 1024;
     static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
 };
+
+// Tensor memory (512 columns): P of two consecutive chunks (M = 64, 64 columns each),
+// the transposed output (M = 128: lane d, column = row of the chunk), dS^T, and the
+// state S^T as the A operand of O_inter^T, bf16 hi then lo (lane d, 64 columns each
+// holding 128 16-bit K values).  The output takes columns 128..255 in one of two ways
+// (see retention_kernel): two accumulators of consecutive chunks (cO, cO + 64), or
+// O_intra^T and O_inter^T of one chunk (cOI, cOX).
+constexpr uint32_t cP = 0, cO = 128, cOI = 128, cOX = 192, cDS = 256, cSA = 384;
+
+// Reference row of the folded output (see retention_kernel).
+constexpr int kM = 32;
 
 // Up to three retention passes in one launch: pass p reads (q, k, v) through
 // maps q[p], k[p], v[p], writes o[p], forwards (rev = 0) or backwards in time.
@@ -121,21 +124,40 @@ struct RetJobs {
     const float *sin[3];
     float *sout[3];
     int sin_t[3];
-    // Per pass, which operands carry a bf16 lo part besides the hi part (fp32 = hi + lo):
-    // kLoK (K^ of dS), kLoP (P~ of O_intra), kLoS (S of O_inter).  The launches set all
-    // three: each lo left out adds about 6e-4 to the relative L2 error of the output.
-    int lo[3];
 };
-constexpr int kLoK = 1, kLoP = 2, kLoS = 4;
 
 // Grid: one CTA per (pass, b, h), pass = blockIdx.x / BH.  decay[h] = gamma_h.
+//
+// FOLD: the two output parts share one accumulator, so that consecutive chunks can
+// use two of them and the epilogue of one chunk overlaps the products of the next.
+// With g_i the row scale of the inter-chunk part (gamma^(i+1); backwards
+// gamma^(rows-i)) and a reference row m = 32,
+//   o_i = f_i (sum_j w'_ij P_ij v_j + q_i (gamma^m S)),  f_i = g_i / gamma^m,
+//   w'_ij = w_ij gamma^m / g_i = gamma^(m-1-j) (j <= i)   [backwards gamma^(j+m-rows), j >= i],
+// so the state operand is written as gamma^m S and the epilogue multiplies row i by
+// f_i.  Every factor lies within gamma^(+-64) of 1, which stays far inside the fp32 and
+// bf16 ranges for gamma >= 1/8; smaller decays use FOLD = false, where O_intra^T and
+// O_inter^T keep accumulators of their own and the epilogue forms O_intra + g_i O_inter.
+//
+// Per chunk c the UMMAs are issued in the order P(c + 1), dS^T(c), O_intra^T(c),
+// O_inter^T(c): P of the next chunk goes to the other P buffer as soon as its data has
+// arrived, so the decay mask of chunk c + 1 overlaps the rest of chunk c, and every
+// product whose operands are ready is queued ahead of O_inter^T, the one that waits
+// for the state.  Every operand of the 16-bit products is exact or split hi + lo
+// (K^, P~, S), so the products carry fp32 accuracy into the fp32 accumulators.
+//   P           M=64  N=64  K=128  A = Q (K-major)            B = K (K-major)
+//   dS^T        M=128 N=128 K=64   A = V^T (MN-major)         B = K^ hi, lo (MN-major)
+//   O_intra^T   M=128 N=64  K=64   A = V^T (MN-major)         B = P~ hi, lo (K-major)
+//   O_inter^T   M=128 N=64  K=128  A = S^T hi, lo (tensor mem) B = Q (K-major)
+template <bool FOLD>
 __global__ void __launch_bounds__(kRThreads, 1)
 retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int H, int BH) {
     using L = RetLayout;
     constexpr int NST = L::NST;
     constexpr uint32_t ID_P = idesc_f16(64, 64, true, false, false);
-    constexpr uint32_t ID_OI = idesc_f16(64, 128, true, false, true);
-    constexpr uint32_t ID_DS = idesc_f16(128, 128, true, true, true);
+    constexpr uint32_t ID_OIT = idesc_f16(128, 64, true, true, false);
+    constexpr uint32_t ID_OXT = idesc_f16(128, 64, true, false, false);
+    constexpr uint32_t ID_DST = idesc_f16(128, 128, true, true, true);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024r(smem_raw);
     uint8_t *sQ = smem + L::qoff;
@@ -143,21 +165,22 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
     uint8_t *sV = smem + L::voff;
     uint8_t *sKh = smem + L::khoff;      // hi at +0, lo at +kTile128
     uint8_t *sPt = smem + L::ptoff;      // hi at +0, lo at +kBox
-    uint8_t *sS = smem + L::soff;        // hi at +0 (2 atoms of 16 KB), lo at +32 KB
     uint8_t *sO = smem + L::ooff;
-    float *gpow = reinterpret_cast<float *>(smem + L::gpoff);
+    float *gexp = reinterpret_cast<float *>(smem + L::gpoff);   // gexp[k + 64] = gamma^k
+#define GP(k) gexp[(k) + 64]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::baroff);
     uint64_t *empty = full + NST;
-    uint64_t *pfull = empty + NST;       // P = Q K^T in TMEM
-    uint64_t *ptready = pfull + 1;       // P read, P~ written (feature-map warps)
-    uint64_t *khready = ptready + 1;     // K^ written
-    uint64_t *dsfull = khready + 1;      // dS = K^^T V in TMEM
-    uint64_t *dsread = dsfull + 1;       // dS read (state warps)
+    uint64_t *pfull = empty + NST;       // [2] P of a chunk in TMEM buffer (chunk & 1)
+    uint64_t *ptready = pfull + 2;       // P read, P~ written (mask warps)
+    uint64_t *ptfree = ptready + 1;      // O_intra^T done reading P~
+    uint64_t *khready = ptfree + 1;      // K^ written
+    uint64_t *dsfull = khready + 1;      // dS^T = V^T K^ in TMEM
+    uint64_t *dsread = dsfull + 1;       // dS^T read (state warps)
     uint64_t *sready = dsread + 1;       // state operand holds S_c (phase c)
-    uint64_t *sfree = sready + 1;        // Q S of the chunk done reading the state operand
-    uint64_t *ofull = sfree + 1;         // O_intra and O_inter in TMEM
-    uint64_t *oread = ofull + 1;         // ... read (output warps)
-    uint64_t *drain = oread + 1;
+    uint64_t *sfree = sready + 1;        // O_inter^T of the chunk done reading the state operand
+    uint64_t *ofull = sfree + 1;         // [2] the output of a chunk in TMEM (FOLD: per buffer)
+    uint64_t *oread = ofull + 2;         // [2] ... read (output warps)
+    uint64_t *drain = oread + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc);
     int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
 
@@ -165,8 +188,6 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
     const int pass = blockIdx.x / BH;
     const int bh = blockIdx.x % BH;
     const bool rev = jobs.rev[pass] != 0;
-    const int lo_mask = jobs.lo[pass];
-    const int nlk = (lo_mask & kLoK) ? 2 : 1, nlp = (lo_mask & kLoP) ? 2 : 1, nls = (lo_mask & kLoS) ? 2 : 1;
     const CUtensorMap *tmQ = &jobs.q[pass], *tmK = &jobs.k[pass], *tmV = &jobs.v[pass], *tmO = &jobs.o[pass];
     const float gamma = dec.gamma[bh % H];
     const int nchunks = (T + kC - 1) / kC;
@@ -176,29 +197,29 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(pfull, 1);
+        mbar_init(&pfull[0], 1);
+        mbar_init(&pfull[1], 1);
         mbar_init(ptready, kRXWarps);
+        mbar_init(ptfree, 1);
         mbar_init(khready, kRSWarps);
         mbar_init(dsfull, 1);
         mbar_init(dsread, kRSWarps);
         mbar_init(sready, kRSWarps);
         mbar_init(sfree, 1);
-        mbar_init(ofull, 1);
-        mbar_init(oread, kROWarps);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ofull[b], 1);
+            mbar_init(&oread[b], kROWarps);
+        }
         mbar_init(drain, 1);
         *s_abort = 0;
         fence_mbar_init();
     }
-    if (threadIdx.x < 129) {
-        // gamma^k in fp32 as exp2(k log2 gamma): k = 0..C for the masks and row scales
+    if (threadIdx.x < 193) {
+        // gamma^k in fp32 as exp2(k log2 gamma), k = -64..128: the masks, row scales and
+        // the folded output's factors
         const float l2g = log2f(gamma);
-        gpow[threadIdx.x] = threadIdx.x == 0 ? 1.f : exp2f((float)threadIdx.x * l2g);
-    }
-    if (warp >= kRSw0) {
-        // S_0 = 0: the state operand (hi and lo, 4 x 16 KB), 16 bytes per thread per step
-        for (int i = threadIdx.x - kRSw0 * 32; i < 4 * 16384 / 16; i += kRSWarps * 32)
-            reinterpret_cast<uint4 *>(sS)[i] = make_uint4(0u, 0u, 0u, 0u);
-        fence_async_smem();
+        const int k = (int)threadIdx.x - 64;
+        gexp[threadIdx.x] = k == 0 ? 1.f : exp2f((float)k * l2g);
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch(tmQ);
@@ -219,7 +240,6 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
     // dependents are released only once this kernel is past its own wait.
     grid_dependency_wait();
     if (threadIdx.x == 0) grid_launch_dependents();
-    constexpr uint32_t cP = 0, cOI = 64, cOX = 192, cDS = 320;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -244,85 +264,89 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             }
         }
     } else if (warp == 1) {
-        // UMMA issue, per chunk c: dS (independent of the state), O_intra, P of
-        // chunk c + 1 (so that its decay mask overlaps the rest of chunk c), then
-        // Q S once the state warps have written S_c.
-        if (lane == 0) {
-            auto issue_p = [&](int sp) {
-                const uint64_t dq = sdesc_sw128(smem_u32(sQ + sp * kTile128), 16, 1024);
-                const uint64_t dk = sdesc_sw128(smem_u32(sK + sp * kTile128), 16, 1024);
+        // The whole warp runs the issue loop in step (waits included); one elected lane
+        // issues each UMMA and commit, so the descriptors stay warp-uniform.
+#define LA_WWAIT(bar, par, code) __all_sync(0xffffffffu, LA_RWAIT((bar), (par), (code)))
+        auto issue_p = [&](int c) {   // P = Q K^T of chunk iteration c into buffer c & 1
+            const int sp = c % NST;
+            const uint64_t dq = sdesc_sw128(smem_u32(sQ + sp * kTile128), 16, 1024);
+            const uint64_t dk = sdesc_sw128(smem_u32(sK + sp * kTile128), 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                    umma_f16_ss(tmem + cP, desc_at(dq, off), desc_at(dk, off), ID_P, kk ? 1u : 0u);
-                }
-                umma_commit(pfull);
-            };
-            int s = 0;
-            uint32_t ph = 0;
-            bool ok = nchunks > 0 && LA_RWAIT(&full[0], 0, 0x4u);
-            if (ok) {
-                tc_fence_after();
-                issue_p(0);
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+                umma_f16_ss_warp(tmem + cP + 64u * (uint32_t)(c & 1), desc_at(dq, off), desc_at(dk, off), ID_P,
+                                 kk ? 1u : 0u);
             }
-            for (int it = 0; it < nchunks && ok; ++it) {
-                const uint32_t pc = (uint32_t)(it & 1), pp = pc ^ 1u;
-                const int sn = s + 1 == NST ? 0 : s + 1;
-                const uint32_t phn = s + 1 == NST ? ph ^ 1u : ph;
-                const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTile128), 16, 1024);
-                const uint64_t dv = sdesc_sw128(smem_u32(sV + s * kTile128), kBox, 1024);
-                // dS = K^^T V
-                if (!LA_RWAIT(khready, pc, 0x80u)) break;
-                if (it > 0 && !LA_RWAIT(dsread, pp, 0x40u)) break;
-                tc_fence_after();
-                const uint64_t dkh = sdesc_sw128(smem_u32(sKh), kBox, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-                    for (int op = 0; op < nlk; ++op)
-                        umma_f16_ss(tmem + cDS, desc_at(dkh, op * kTile128 + kk * 2048), desc_at(dv, kk * 2048), ID_DS,
-                                    (kk | op) ? 1u : 0u);
-                }
-                umma_commit(dsfull);
-                // O_intra = P~ V (the mask has read P: its accumulator is free)
-                if (!LA_RWAIT(ptready, pc, 0x10u)) break;
-                if (it > 0 && !LA_RWAIT(oread, pp, 0x20u)) break;
-                tc_fence_after();
-                const uint64_t dpt = sdesc_sw128(smem_u32(sPt), 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-                    for (int op = 0; op < nlp; ++op)
-                        umma_f16_ss(tmem + cOI, desc_at(dpt, op * kBox + kk * 32), desc_at(dv, kk * 2048), ID_OI,
-                                    (kk | op) ? 1u : 0u);
-                }
-                // P of the next chunk
-                if (it + 1 < nchunks) {
-                    if (!LA_RWAIT(&full[sn], phn, 0x4u)) break;
-                    tc_fence_after();
-                    issue_p(sn);
-                }
-                // O_inter = Q S_c
-                if (!LA_RWAIT(sready, pc, 0x1000u)) break;
-                tc_fence_after();
-                const uint64_t ds = sdesc_sw128(smem_u32(sS), 16384, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-#pragma unroll
-                    for (int op = 0; op < nls; ++op)
-                        umma_f16_ss(tmem + cOX, desc_at(dq, off), desc_at(ds, op * 32768 + kk * 2048), ID_OI,
-                                    (kk | op) ? 1u : 0u);
-                }
-                umma_commit(ofull);
-                umma_commit(sfree);
-                umma_commit(&empty[s]);
-                s = sn;
-                ph = phn;
-            }
-            umma_commit(drain);
-            mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_ret_fault, 0x400u);
+            umma_commit_warp(&pfull[c & 1]);
+        };
+        bool ok = nchunks > 0 && LA_WWAIT(&full[0], 0, 0x4u);
+        if (ok) {
+            tc_fence_after();
+            issue_p(0);
         }
+        const uint64_t dkh = sdesc_sw128(smem_u32(sKh), kBox, 1024);
+        const uint64_t dpt = sdesc_sw128(smem_u32(sPt), 16, 1024);
+        for (int it = 0; it < nchunks && ok; ++it) {
+            const uint32_t pc = (uint32_t)(it & 1), pp = pc ^ 1u;
+            const int s = it % NST;
+            // P of the next chunk: its buffer was last read by the mask of chunk it - 1,
+            // which finished before O_intra^T(it - 1) was issued
+            if (it + 1 < nchunks) {
+                if (!LA_WWAIT(&full[(it + 1) % NST], (uint32_t)(((it + 1) / NST) & 1), 0x4u)) break;
+                tc_fence_after();
+                issue_p(it + 1);
+            }
+            const uint64_t dv = sdesc_sw128(smem_u32(sV + s * kTile128), kBox, 1024);
+            // dS^T = V^T K^
+            if (!LA_WWAIT(khready, pc, 0x80u)) break;
+            if (it > 0 && !LA_WWAIT(dsread, pp, 0x40u)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                for (int op = 0; op < 2; ++op)
+                    umma_f16_ss_warp(tmem + cDS, desc_at(dv, kk * 2048), desc_at(dkh, op * kTile128 + kk * 2048),
+                                     ID_DST, (kk | op) ? 1u : 0u);
+            }
+            umma_commit_warp(dsfull);
+            // O_intra^T = V^T P~^T, once the output warps have read what its accumulator
+            // held (FOLD: the chunk before the previous one; else the previous chunk)
+            const int ob = FOLD ? (it & 1) : 0;
+            const uint32_t cIn = FOLD ? cO + 64u * (uint32_t)ob : cOI;
+            const uint32_t cEx = FOLD ? cIn : cOX;
+            if (!LA_WWAIT(ptready, pc, 0x10u)) break;
+            if (FOLD ? it >= 2 && !LA_WWAIT(&oread[ob], (uint32_t)(((it >> 1) & 1) ^ 1), 0x20u)
+                     : it > 0 && !LA_WWAIT(&oread[0], pp, 0x20u))
+                break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                for (int op = 0; op < 2; ++op)
+                    umma_f16_ss_warp(tmem + cIn, desc_at(dv, kk * 2048), desc_at(dpt, op * kBox + kk * 32), ID_OIT,
+                                     (kk | op) ? 1u : 0u);
+            }
+            umma_commit_warp(ptfree);
+            // O_inter^T = S^T Q^T once the state warps have written S_c
+            if (!LA_WWAIT(sready, pc, 0x1000u)) break;
+            tc_fence_after();
+            const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTile128), 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+#pragma unroll
+                for (int op = 0; op < 2; ++op)
+                    umma_f16_ts_warp(tmem + cEx, tmem + cSA + 64u * op + 8u * kk, desc_at(dq, off), ID_OXT,
+                                     (FOLD || (kk | op)) ? 1u : 0u);
+            }
+            umma_commit_warp(&ofull[ob]);
+            umma_commit_warp(sfree);
+            umma_commit_warp(&empty[s]);
+        }
+        umma_commit_warp(drain);
+        mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_ret_fault, 0x400u);
+        __syncwarp();
+#undef LA_WWAIT
     } else if (warp < kROw0) {
         // Decay-mask warps: P~ = P o M as hi + lo (warp w reads TMEM lane quadrant w % 4,
         // where chunk rows 16 (w % 4) + l sit in lanes l = 0..15).
@@ -331,9 +355,10 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         const int ri = 16 * sub + (lane & 15), hcol = lane >> 4;   // row; column half (M = 64 rows in lanes 0..15)
         for (int it = 0; it < nchunks; ++it) {
             const uint32_t pc = (uint32_t)(it & 1);
-            // P~ of the previous chunk: its O_intra completed before this chunk's P, which pfull tracks
-            const bool got = __all_sync(0xffffffffu, LA_RWAIT(pfull, pc, 0x400u));
-            if (!got) break;
+            const int rows = min(kC, T - (rev ? nchunks - 1 - it : it) * kC);
+            if (!__all_sync(0xffffffffu, LA_RWAIT(&pfull[it & 1], (uint32_t)((it >> 1) & 1), 0x400u))) break;
+            // P~ of the previous chunk has been read by its O_intra^T
+            if (it > 0 && !__all_sync(0xffffffffu, LA_RWAIT(ptfree, pc ^ 1u, 0x8u))) break;
             __syncwarp();   // converged for the .sync.aligned TMEM loads
             tc_fence_after();
             // lanes 0..15 take columns 0..31 of their row, lanes 16..31 columns 32..63
@@ -341,18 +366,18 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             for (int h16 = 0; h16 < 2; ++h16) {
                 const int c16 = 2 * hcol + h16;
                 float x[16];
-                tmem_ld16_halves<32>(tmem + cP + lanes + 16 * h16, x);
-                tmem_ld_wait(x);
+                tmem_ld16_halves_sync<32>(tmem + cP + 64u * (uint32_t)(it & 1) + lanes + 16 * h16, x);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int j = 16 * c16 + e;
                     const int dlt = rev ? j - ri : ri - j;     // causal: i >= j; backwards: j >= i
-                    x[e] = dlt >= 0 ? x[e] * gpow[dlt] : 0.f;
+                    const float wgt = FOLD ? (rev ? GP(j + kM - rows) : GP(kM - 1 - j)) : GP(dlt);
+                    x[e] = dlt >= 0 ? x[e] * wgt : 0.f;
                 }
                 uint32_t hw[8], lw[8];
                 split_hi_lo16_packed(x, hw, lw);
                 store_chunk16_packed(sPt, ri, c16, hw);
-                if (nlp == 2) store_chunk16_packed(sPt + kBox, ri, c16, lw);
+                store_chunk16_packed(sPt + kBox, ri, c16, lw);
             }
             tc_fence_before();
             fence_async_smem();
@@ -360,20 +385,25 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             if (lane == 0) mbar_arrive(ptready);
         }
     } else if (warp < kRSw0) {
-        // Output warps: o = O_intra + diag(gamma^(i+1)) O_inter (backwards: gamma^(C-i)),
-        // staged and stored with TMA.  Named barrier 1 (these 128 threads) is
-        // reached by all of them whatever the waits return.
+        // Output warps: o = O_intra + diag(gamma^(i+1)) O_inter (backwards: gamma^(rows-i);
+        // folded: f_i times the one accumulator), from the transposed parts (TMEM lane d,
+        // column = row i of the chunk).  Each warp takes its 32 lanes as two groups of 16
+        // in rounds of 16 columns: a 16x256b TMEM load gives the MMA-fragment layout of a
+        // [16 d x 16 i] block, and stmatrix .trans writes its four 8x8 parts transposed, as
+        // 16-byte rows of the staging chunk (row i, 8 consecutive d).  Named barrier 1
+        // (these 128 threads) is reached by all of them whatever the waits return.
         const int ot = threadIdx.x - kROw0 * 32;
         const int sub = warp & 3;
-        const uint32_t lanes = (uint32_t)(32 * sub) << 16;
-        const int ri = 16 * sub + (lane & 15), hcol = lane >> 4;   // row; column half (M = 64 rows in lanes 0..15)
+        const int q4 = lane & 3;                            // fragment: columns 2 q4 (+1) of lanes lane / 4 (+8)
+        const int mk = lane >> 3, mj = lane & 7;            // stmatrix: matrix mk, stored row mj
         bool live = true;
         for (int it = 0; it < nchunks; ++it) {
             const int c = rev ? nchunks - 1 - it : it;
             const uint32_t pc = (uint32_t)(it & 1);
             if (ot == 0) tma_store_wait_read<0>();
             named_bar(1, kROWarps * 32);
-            bool got = live && LA_RWAIT(ofull, pc, 0x800u);
+            const int ob = FOLD ? (it & 1) : 0;
+            bool got = live && LA_RWAIT(&ofull[ob], FOLD ? (uint32_t)((it >> 1) & 1) : pc, 0x800u);
             got = __all_sync(0xffffffffu, got);
             live = live && got;
             if (got) {
@@ -381,21 +411,52 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                 tc_fence_after();
                 // backwards the entering state sits one past the chunk's last valid row
                 const int rows = min(kC, T - c * kC);
-                const float g1 = rev ? (ri < rows ? gpow[rows - ri] : 0.f) : gpow[ri + 1];
-                // lanes 0..15 take columns 0..63 of their row, lanes 16..31 columns 64..127
+                auto scale = [&](int i) -> float {   // FOLD: f_i; else g_i of the inter-chunk part
+                    if (FOLD) return rev ? (i < rows ? GP(rows - i - kM) : 0.f) : GP(i + 1 - kM);
+                    return rev ? (i < rows ? GP(rows - i) : 0.f) : GP(i + 1);
+                };
+#pragma unroll 1
+                for (int h = 0; h < 4; ++h) {
+                    const int i0 = 16 * h + 2 * q4;
+                    const float f0 = scale(i0), f1 = scale(i0 + 1), f8 = scale(i0 + 8), f9 = scale(i0 + 9);
 #pragma unroll
-                for (int h16 = 0; h16 < 4; ++h16) {
-                    float a[16], b[16];
-                    tmem_ld16_halves<64>(tmem + cOI + lanes + 16 * h16, a);
-                    tmem_ld16_halves<64>(tmem + cOX + lanes + 16 * h16, b);
-                    tmem_ld_wait(a, b);
+                    for (int half = 0; half < 2; ++half) {
+                        const int dbase = 32 * sub + 16 * half;
+                        const uint32_t tl = (uint32_t)dbase << 16;
+                        uint32_t r[8];
+                        float y[8];
+                        if (FOLD) {
+                            tmem_ld16x256b_x2_sync(tmem + cO + 64u * (uint32_t)ob + tl + 16 * h, r);
+                            y[0] = f0 * __uint_as_float(r[0]);
+                            y[1] = f1 * __uint_as_float(r[1]);
+                            y[2] = f0 * __uint_as_float(r[2]);
+                            y[3] = f1 * __uint_as_float(r[3]);
+                            y[4] = f8 * __uint_as_float(r[4]);
+                            y[5] = f9 * __uint_as_float(r[5]);
+                            y[6] = f8 * __uint_as_float(r[6]);
+                            y[7] = f9 * __uint_as_float(r[7]);
+                        } else {
+                            uint32_t x[8];
+                            tmem_ld16x256b_x2_sync(tmem + cOI + tl + 16 * h, r);
+                            tmem_ld16x256b_x2_sync(tmem + cOX + tl + 16 * h, x);
+                            const float fs[8] = {f0, f1, f0, f1, f8, f9, f8, f9};
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) a[i] = fmaf(g1, b[i], a[i]);
-                    st16_wide(sO, kBox, ri, 4 * hcol + h16, a);
+                            for (int e = 0; e < 8; ++e) y[e] = fmaf(fs[e], __uint_as_float(x[e]), __uint_as_float(r[e]));
+                        }
+                        if (h == 3 && half == 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&oread[ob]);
+                        }
+                        // matrices: (d 0..7, i 0..7), (d 8..15, i 0..7), (d 0..7, i 8..15), (d 8..15, i 8..15)
+                        const int row = 16 * h + mj + (mk >= 2 ? 8 : 0);
+                        const int dch = dbase + ((mk & 1) ? 8 : 0);
+                        const uint32_t sa = smem_u32(sO + (dch >> 6) * kBox + row * 128 +
+                                                     ((((dch & 63) >> 3) ^ (row & 7)) << 4));
+                        stmatrix_x4_trans(sa, h2<true>::from_f2(y[0], y[1]), h2<true>::from_f2(y[2], y[3]),
+                                          h2<true>::from_f2(y[4], y[5]), h2<true>::from_f2(y[6], y[7]));
+                    }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(oread);
             }
             fence_async_smem();
             named_bar(1, kROWarps * 32);
@@ -407,62 +468,73 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         }
         if (ot == 0) tma_store_wait_all<0>();
     } else {
-        // State warps: S_{c+1} = gamma^C S_c + dS_c in fp32 registers; thread (d, half)
-        // holds columns 64 half .. 64 half + 63 of state row d (its TMEM lane) and
-        // writes them as the bf16 hi + lo operand of Q S.
+        // State warps: S^T_{c+1} = gamma^C S^T_c + dS^T_c in fp32 registers; thread (d, half)
+        // holds row d of S^T (column d of S), entries 64 half .. 64 half + 63 (its TMEM lane
+        // of dS^T), and writes them as the bf16 hi + lo A operand of O_inter^T.
         const int sub = warp & 3, half = (warp - kRSw0) >> 2;
         const uint32_t lanes = (uint32_t)(32 * sub) << 16;
         const int d = 32 * sub + lane;
-        const float gC = gpow[kC];
+        const float gC = GP(kC);
+        const float gm = FOLD ? GP(kM) : 1.f;   // the state operand holds gamma^m S (FOLD)
         // decay over the partial chunk at the end of the sequence: the last chunk
         // forwards, the first one backwards
-        const float gLast = gpow[min(kC, T - (nchunks - 1) * kC)];
+        const float gLast = GP(min(kC, T - (nchunks - 1) * kC));
         float st[64];
         const float *sin = jobs.sin[pass];
         float *sout = jobs.sout[pass];
-        const long long srow = ((long long)bh * 128 + d) * 128 + 64 * half;   // this thread's 64 state entries
-        if (sin) {   // S_0 given: registers and the hi + lo operand of the first Q S
-            if (jobs.sin_t[pass]) {   // st[c] = sin[64 half + c][d]: lanes read consecutive d
-                const float *col = sin + (long long)bh * 128 * 128 + (long long)(64 * half) * 128 + d;
-#pragma unroll
-                for (int c = 0; c < 64; ++c) st[c] = col[(long long)c * 128];
-            } else {
+        const long long sbase = (long long)bh * 128 * 128;
+        if (sin) {
+            if (jobs.sin_t[pass]) {   // sin holds S^T: row d, entries 64 half ..
 #pragma unroll
                 for (int c4 = 0; c4 < 16; ++c4) {
-                    const float4 x = *reinterpret_cast<const float4 *>(sin + srow + 4 * c4);
+                    const float4 x = *reinterpret_cast<const float4 *>(sin + sbase + (long long)d * 128 + 64 * half + 4 * c4);
                     st[4 * c4] = x.x;
                     st[4 * c4 + 1] = x.y;
                     st[4 * c4 + 2] = x.z;
                     st[4 * c4 + 3] = x.w;
                 }
-            }
+            } else {                  // sin holds S: column d (lanes read consecutive d)
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t hw[8], lw[8];
-                split_hi_lo16_packed(*reinterpret_cast<const float(*)[16]>(&st[16 * c4]), hw, lw);
-                store_chunk16_packed(sS + half * 16384, d, c4, hw);
-                if (nls == 2) store_chunk16_packed(sS + 32768 + half * 16384, d, c4, lw);
+                for (int c = 0; c < 64; ++c) st[c] = sin[sbase + (long long)(64 * half + c) * 128 + d];
             }
-            fence_async_smem();
         } else {
 #pragma unroll
             for (int i = 0; i < 64; ++i) st[i] = 0.f;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sready);                // S_0
-        // K^ = diag(gamma^(C-1-j)) K of chunk iteration itk as hi + lo, written while Q S of
-        // the previous chunk runs: thread kt takes row kt % 64 and the 8-element chunks
-        // 4 (kt / 64) .. + 3 of the row's 16.  Forwards in time the weights count back from
-        // the chunk's last valid row, so that the state after a partial last chunk is the
-        // state after token T - 1.
+        // The state operand: this thread's 64 entries as 32 packed columns of its lane,
+        // hi at cSA + 32 half, lo 64 columns further, in four rounds of 8 columns.
+        auto write_state = [&]() {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                uint32_t hw[8], lw[8];
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const float a = gm * st[16 * r + 2 * m], b = gm * st[16 * r + 2 * m + 1];
+                    hw[m] = h2<true>::from_f2(a, b);
+                    const float2 hv = h2<true>::to_f2(hw[m]);
+                    lw[m] = h2<true>::from_f2(a - hv.x, b - hv.y);
+                }
+                tmem_st8(tmem + cSA + lanes + 32 * half + 8 * r, hw);
+                tmem_st8(tmem + cSA + 64 + lanes + 32 * half + 8 * r, lw);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sready);
+        };
+        write_state();                                     // S_0
+        // K^ = diag(gamma^(C-1-j)) K of chunk iteration itk as hi + lo: thread kt takes row
+        // kt % 64 and the 8-element chunks 4 (kt / 64) .. + 3 of the row's 16.  Forwards in
+        // time the weights count back from the chunk's last valid row, so that the state
+        // after a partial last chunk is the state after token T - 1.
         const int kt = threadIdx.x - kRSw0 * 32;
         const int krow = kt & 63, kpart = kt >> 6;
         auto build_khat = [&](int itk) -> bool {
             const int sk = itk % NST;
             if (!__all_sync(0xffffffffu, LA_RWAIT(&full[sk], (uint32_t)((itk / NST) & 1), 0x100u))) return false;
             const int rows = min(kC, T - (rev ? nchunks - 1 - itk : itk) * kC);
-            const float f = rev ? gpow[krow] : (krow < rows ? gpow[rows - 1 - krow] : 0.f);
-            scale_split_row(sK + sk * kTile128, sKh, krow, kpart, f, nlk == 2);
+            const float f = rev ? GP(krow) : (krow < rows ? GP(rows - 1 - krow) : 0.f);
+            scale_split_row(sK + sk * kTile128, sKh, krow, kpart, f, true);
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(khready);
@@ -471,8 +543,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         const bool k0 = nchunks > 0 && build_khat(0);
         for (int it = 0; it < nchunks && k0; ++it) {
             const uint32_t pc = (uint32_t)(it & 1);
-            bool got = __all_sync(0xffffffffu, LA_RWAIT(dsfull, pc, 0x1000u));
-            if (!got) break;
+            if (!__all_sync(0xffffffffu, LA_RWAIT(dsfull, pc, 0x1000u))) break;
             __syncwarp();   // converged for the .sync.aligned TMEM loads
             tc_fence_after();
             const uint32_t base = tmem + cDS + lanes + 64u * half;
@@ -480,35 +551,24 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
                 float a[16];
-                tmem_ld16(base + 16 * c4, a);
-                tmem_ld_wait(a);
+                tmem_ld16_sync(base + 16 * c4, a);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) st[16 * c4 + i] = fmaf(g, st[16 * c4 + i], a[i]);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(dsread);
-            // dS_c is complete, so it has read K^_c: the buffer takes K^ of the next chunk
-            if (it + 1 < nchunks && !build_khat(it + 1)) break;
-            got = __all_sync(0xffffffffu, LA_RWAIT(sfree, pc, 0x2000u));   // Q S_c has read the operand
-            if (!got) break;
-            // the 64 columns are columns 0..63 of box `half` (each box holds 64 state columns)
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                uint32_t hw[8], lw[8];
-                split_hi_lo16_packed(*reinterpret_cast<const float(*)[16]>(&st[16 * c4]), hw, lw);
-                store_chunk16_packed(sS + half * 16384, d, c4, hw);
-                if (nls == 2) store_chunk16_packed(sS + 32768 + half * 16384, d, c4, lw);
-            }
-            fence_async_smem();
+            if (it + 1 == nchunks) break;                  // st holds the state after the sequence
+            // dS^T_c is complete, so it has read K^_c: the buffer takes K^ of the next chunk
+            if (!build_khat(it + 1)) break;
+            if (!__all_sync(0xffffffffu, LA_RWAIT(sfree, pc, 0x2000u))) break;   // O_inter^T(c) read S_c
             __syncwarp();
-            if (lane == 0) mbar_arrive(sready);
+            tc_fence_after();
+            write_state();
         }
-        if (sout && !*s_abort) {   // S after the last chunk
+        if (sout && !*s_abort) {   // S after the last chunk: column d of S, lanes write consecutive d
 #pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4)
-                *reinterpret_cast<float4 *>(sout + srow + 4 * c4) =
-                    make_float4(st[4 * c4], st[4 * c4 + 1], st[4 * c4 + 2], st[4 * c4 + 3]);
+            for (int c = 0; c < 64; ++c) sout[sbase + (long long)(64 * half + c) * 128 + d] = st[c];
         }
     }
     tc_fence_before();
@@ -517,6 +577,14 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+#undef GP
+}
+
+// The folded output needs every factor gamma^k, |k| <= 64, well inside the fp32 range.
+static bool fold_ok(const DecayArgs &dec, int H) {
+    for (int h = 0; h < H; ++h)
+        if (!(dec.gamma[h] >= 0.125f)) return false;
+    return true;
 }
 
 #ifndef LA_TRY
@@ -535,13 +603,15 @@ la_status retention_fwd(const void *q, const void *k, const void *v, void *o, co
     memset(&jobs, 0, sizeof jobs);
     jobs.sin[0] = sin;
     jobs.sout[0] = sout;
-    jobs.lo[0] = kLoK | kLoP | kLoS;
     LA_TRY(retention_map(&jobs.q[0], q, s));
     LA_TRY(retention_map(&jobs.k[0], k, s));
     LA_TRY(retention_map(&jobs.v[0], v, s));
     LA_TRY(retention_map(&jobs.o[0], o, s));
-    return launch_pdl("tc_retention_fwd", retention_kernel, dim3((unsigned)s.BH()), dim3(kRThreads),
-                  (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
+    if (fold_ok(dec, s.H))
+        return launch_pdl("tc_retention_fwd", retention_kernel<true>, dim3((unsigned)s.BH()), dim3(kRThreads),
+                          (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
+    return launch_pdl("tc_retention_fwd_unfolded", retention_kernel<false>, dim3((unsigned)s.BH()), dim3(kRThreads),
+                      (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
 }
 
 la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin,
@@ -573,10 +643,12 @@ la_status retention_bwd(const void *q, const void *k, const void *v, const void 
         jobs.sin[np] = all[p].sin;
         jobs.sin_t[np] = all[p].sin_t;
         jobs.sout[np] = all[p].sout;
-        jobs.lo[np] = kLoK | kLoP | kLoS;
     }
-    return launch_pdl("tc_retention_bwd", retention_kernel, dim3((unsigned)(np * s.BH())), dim3(kRThreads),
-                  (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
+    if (fold_ok(dec, s.H))
+        return launch_pdl("tc_retention_bwd", retention_kernel<true>, dim3((unsigned)(np * s.BH())), dim3(kRThreads),
+                          (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
+    return launch_pdl("tc_retention_bwd_unfolded", retention_kernel<false>, dim3((unsigned)(np * s.BH())),
+                      dim3(kRThreads), (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
 }
 
 unsigned int read_and_clear_retention_fault() {

@@ -185,3 +185,17 @@ def test_other_stream():
     s = torch.cuda.Stream()
     got = pu.gpu_run("bidir", inp, eps=w.eps, stream=s)
     pu.compare("bidir", got, pu.oracle_run("bidir", inp, eps=w.eps))
+
+
+# Strong per-head decays on the tensor-core path: gamma >= 1/8 folds the two output parts of
+# a chunk into one accumulator (every factor gamma^k with |k| <= 64 in range); smaller decays
+# keep the two parts apart.  Heads of both kinds in one call, and each kind alone; several
+# chunks with a ragged tail, so the row scales and the state carried between chunks count.
+@pytest.mark.parametrize("gammas", [(0.05, 0.3, 0.9, 0.999), (0.125, 0.5, 0.75, 1.0), (0.06, 0.1, 0.11, 0.02)],
+                         ids=["mixed", "folded", "unfolded"])
+def test_retention_strong_decays(gammas):
+    w = _workload("retention", "bf16", 2, len(gammas), 300, 128)
+    inp = synth.make_inputs(w, seed=3)
+    inp["gamma"] = torch.tensor(gammas, dtype=torch.float32)
+    got = pu.gpu_run("retention", inp)
+    pu.compare("retention", got, pu.oracle_run("retention", inp))
