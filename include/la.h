@@ -404,6 +404,25 @@ la_status la_chunk_decay_step(const void *q, const void *k, const void *v, void 
  * LA_ERR_CUDA if the word could not be read. */
 la_status la_device_check(void);
 
+/* ---- test hooks (fault injection without a GPU fault) -------------------
+ * The library's own failure paths, made to run on demand by the tests.  The
+ * pages describe no such hooks; they exist to test this library.              */
+
+/* The launch that comes after `after` further kernel launches of this library
+ * fails before it reaches the GPU: its entry point returns LA_ERR_CUDA and
+ * la_last_error() names the kernel and "injected launch failure".  after = -1
+ * disarms; only one failure is armed at a time (process wide).  Returns
+ * LA_ERR_INVALID_ARG for after < -1. */
+la_status la_debug_fail_launch(int after);
+
+/* Enqueues on `stream` a one-CTA kernel whose single wait, on an mbarrier that
+ * nothing arrives on, gives up after limit_us microseconds (1 .. 1000000), the
+ * way every bounded wait of the tensor-core kernels does: it sets the fault
+ * word that la_device_check() reports as LA_ERR_TIMEOUT and returns.  With
+ * waited_out (a device int, or NULL) the kernel also writes 1 there when the
+ * wait ran out.  Nothing is left in flight, so the context stays usable. */
+la_status la_debug_wait_timeout(unsigned int limit_us, int *waited_out, void *stream);
+
 /* Static text for a status code. */
 const char *la_status_string(la_status status);
 

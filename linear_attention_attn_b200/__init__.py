@@ -76,6 +76,10 @@ for _n in ("la_bidir_fwd", "la_simple_fwd", "la_bidir_bwd", "la_simple_bwd", "la
     getattr(_lib, _n).restype = _I
 _lib.la_bidir_fwd_static.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.la_bidir_fwd_static.restype = _I
+_lib.la_debug_fail_launch.argtypes = [_I]
+_lib.la_debug_fail_launch.restype = _I
+_lib.la_debug_wait_timeout.argtypes = [ctypes.c_uint, _P, _P]
+_lib.la_debug_wait_timeout.restype = _I
 _lib.la_static_scratch_bytes.argtypes = []
 _lib.la_static_scratch_bytes.restype = _Z
 _lib.la_status_string.argtypes = [_I]
@@ -485,6 +489,18 @@ def la_last_error() -> str:
 def la_device_check() -> None:
     """Raise LAError if a tensor-core kernel gave up waiting since the last check."""
     _check(_lib.la_device_check(), "la_device_check")
+
+
+def la_debug_fail_launch(after: int) -> None:
+    """Test hook: the launch after `after` further launches of the library fails (-1 disarms)."""
+    _check(_lib.la_debug_fail_launch(int(after)), "la_debug_fail_launch")
+
+
+def la_debug_wait_timeout(limit_us: int, waited_out=None, stream=None) -> None:
+    """Test hook: a kernel whose bounded wait runs out after limit_us (see include/la.h)."""
+    dev = waited_out.device if waited_out is not None else None
+    _check(_lib.la_debug_wait_timeout(int(limit_us), _ptr(waited_out), _stream(stream, dev)),
+           "la_debug_wait_timeout")
 
 
 def la_launch_count() -> int:

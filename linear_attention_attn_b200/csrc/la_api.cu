@@ -86,6 +86,21 @@ static cudaEvent_t take_event() {
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+// Launches still to pass before the injected failure (-1: none armed).
+static std::atomic<long long> g_fail_after{-1};
+
+bool injected_launch_failure(const char *name) {
+    long long n = g_fail_after.load(std::memory_order_relaxed);
+    while (n >= 0) {
+        if (g_fail_after.compare_exchange_weak(n, n - 1, std::memory_order_relaxed)) {
+            if (n > 0) return false;
+            set_error("%s: injected launch failure (la_debug_fail_launch)", name);
+            return true;
+        }
+    }
+    return false;
+}
+
 void prof_before(const char *name, cudaStream_t s) {
     t_pending_name = nullptr;
     if (!g_prof_on.load(std::memory_order_relaxed)) return;
@@ -582,6 +597,12 @@ la_status la_device_check(void) {
 }
 
 long long la_launch_count(void) { return g_launches.load(); }
+
+la_status la_debug_fail_launch(int after) {
+    if (after < -1) return fail(LA_ERR_INVALID_ARG, "after must be >= -1 (got %d)", after);
+    g_fail_after.store(after);
+    return LA_OK;
+}
 
 int la_prof_enable(int enabled) { return g_prof_on.exchange(enabled ? 1 : 0); }
 

@@ -23,11 +23,15 @@ la_status launch_fail(cudaError_t e, const char *what, const void *kernel, dim3 
 void prof_before(const char *name, cudaStream_t s);
 void prof_after(cudaStream_t s);
 void count_launch();
+// Test hook (la_debug_fail_launch): true when this launch is to fail without running;
+// the error text is then set.  Checked before any CUDA call of the launch.
+bool injected_launch_failure(const char *name);
 
 template <typename Kernel, typename... Args>
 la_status launch(const char *name, Kernel kernel, dim3 grid, dim3 block, size_t smem,
                  cudaStream_t stream, Args... args) {
     if (grid.x == 0 || grid.y == 0 || grid.z == 0) return LA_OK;
+    if (injected_launch_failure(name)) return LA_ERR_CUDA;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -51,6 +55,7 @@ template <typename Kernel, typename... Args>
 la_status launch_pdl(const char *name, Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                      Args... args) {
     if (grid.x == 0 || grid.y == 0 || grid.z == 0) return LA_OK;
+    if (injected_launch_failure(name)) return LA_ERR_CUDA;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return cuda_fail(e, name);

@@ -22,9 +22,10 @@ bool supports(la_op op, const Shape &s, la_dtype dt) {
 }
 
 unsigned int read_and_clear_fault() {
-    const unsigned int a = read_and_clear_state_fault(), b = read_and_clear_retention_fault();
-    if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu) return 0xFFFFFFFFu;
-    return a | b;
+    const unsigned int a = read_and_clear_state_fault(), b = read_and_clear_retention_fault(),
+                       c = read_and_clear_debug_fault();
+    if (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu) return 0xFFFFFFFFu;
+    return a | b | c;
 }
 
 size_t workspace_size(la_op op, const Shape &s, la_dtype) {

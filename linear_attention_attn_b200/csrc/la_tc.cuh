@@ -16,6 +16,7 @@ size_t state_workspace_size(la_op op, const Shape &s);
 unsigned int read_and_clear_fault();
 unsigned int read_and_clear_state_fault();
 unsigned int read_and_clear_retention_fault();
+unsigned int read_and_clear_debug_fault();
 
 // [BH, T, D] 16-bit tensor map: boxes of box_rows x 64 columns, 128-byte swizzle.
 la_status make_tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16, int box_rows);

@@ -59,8 +59,8 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // it.  Only a wait that has lasted 20 us (a pipeline fill, a head change) backs
 // off with __nanosleep, to leave issue slots to the warps that share its
 // scheduler.
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                            unsigned int *fault_word, unsigned int code) {
+static __device__ __noinline__ bool mbar_wait_slow_for(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                                    unsigned int *fault_word, unsigned int code, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();
     while (true) {
 #pragma unroll 1
@@ -68,13 +68,19 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity
             if (mbar_try_wait(bar, parity)) return true;
         if (abort_flag && *abort_flag) return false;
         const uint64_t dt = globaltimer_ns() - t0;
-        if (dt > kWaitLimitNs) {
+        if (dt > limit_ns) {
             if (abort_flag) *abort_flag = 1;
             atomicOr(fault_word, code | 0x80000000u);
             return false;
         }
         if (dt > 20000) __nanosleep(256);
     }
+}
+
+// The wait of every kernel here: bounded by kWaitLimitNs.
+static __device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                                      unsigned int *fault_word, unsigned int code) {
+    return mbar_wait_slow_for(bar, parity, abort_flag, fault_word, code, kWaitLimitNs);
 }
 
 // Bounded wait for the phase with the given parity to complete.

@@ -191,3 +191,8 @@ def test_status_strings(lib):
     lib.la_status_string.restype = ctypes.c_char_p
     assert lib.la_status_string(0) == b"LA_OK"
     assert lib.la_status_string(5) == b"LA_ERR_CUDA"
+
+
+def test_fail_launch_hook_validates_without_a_gpu(lib):
+    assert lib.la_debug_fail_launch(-2) == 1           # LA_ERR_INVALID_ARG
+    assert lib.la_debug_fail_launch(-1) == 0           # disarm
