@@ -186,7 +186,10 @@ la_status la_chunk_decay_fwd(const void *q, const void *k, const void *v, void *
  * T = 0 state_out <- state_in.  The library's addition for chunked prefill and
  * for splitting a sequence into segments; source of the form as for
  * la_chunk_decay_fwd ("flash-linear-attention" README, FusedChunk: the
- * inter-chunk state carried from chunk to chunk). */
+ * inter-chunk state carried from chunk to chunk).
+ * o may be NULL: then only state_out is computed (q is not read and may be
+ * NULL), at about half the cost of the whole op: the first pass of a sequence
+ * split into segments needs only each segment's own end state. */
 la_status la_chunk_decay_fwd_state(const void *q, const void *k, const void *v, void *o,
                                    const float *state_in, float *state_out, const float *decay,
                                    int B, int H, int T, int D, la_dtype dtype,
@@ -213,7 +216,9 @@ la_status la_chunk_decay_bwd(const void *q, const void *k, const void *v, const 
  * three are [B,H,D,D] fp32 device arrays, 16-byte aligned, row i = the index
  * of q (R) or k (S); dstate_out must not overlap state_in or dstate_in
  * (LA_ERR_INVALID_ARG).  dq may be NULL: then only dk and dv are computed
- * (state_in is not read).  With T = 0, dstate_out <- dstate_in.  The library's
+ * (state_in is not read).  dq, dk and dv may all be NULL: then only
+ * dstate_out = R_0 is computed (k and v are not read and may be NULL), about a
+ * third of the cost of the whole backward.  With T = 0, dstate_out <- dstate_in.  The library's
  * addition for splitting a sequence into segments (the reverse-time
  * recurrence is the backward of the FusedChunk form, "flash-linear-attention"
  * README). */

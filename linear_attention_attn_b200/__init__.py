@@ -254,18 +254,19 @@ def la_chunk_decay_fwd(q, k, v, o, decay, workspace=None, stream=None):
 
 def la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=None, state_out=None, workspace=None, stream=None):
     """la_chunk_decay_fwd continuing from state_in ([B, H, D, D] float32, zero if None) and
-    writing the state after the last token to state_out (if given); they may be the same tensor."""
+    writing the state after the last token to state_out (if given); they may be the same tensor.
+    o may be None: then only state_out is computed (q is not read and may be None)."""
     import torch
-    B, H, T, D = _shape(q, k, v, o)
+    B, H, T, D = _shape(k, v, q, o)
     for st, name in ((state_in, "state_in"), (state_out, "state_out")):
         if st is not None and (tuple(st.shape) != (B, H, D, D) or st.dtype != torch.float32 or not st.is_cuda
-                               or not st.is_contiguous() or st.device != q.device):
+                               or not st.is_contiguous() or st.device != k.device):
             raise ValueError("%s must be a contiguous float32 CUDA tensor [B, H, D, D] on the inputs' device" % name)
-    dt = _dtype_code(q)
+    dt = _dtype_code(k)
     dec = _decay(decay, H)
-    wp, wn, _keep = _workspace("chunk_decay_fwd", (B, H, T, D), dt, workspace, q.device, stream)
+    wp, wn, _keep = _workspace("chunk_decay_fwd", (B, H, T, D), dt, workspace, k.device, stream)
     _check(_lib.la_chunk_decay_fwd_state(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state_in), _ptr(state_out),
-                                         ctypes.cast(dec, _P), B, H, T, D, dt, wp, wn, _stream(stream, q.device)),
+                                         ctypes.cast(dec, _P), B, H, T, D, dt, wp, wn, _stream(stream, k.device)),
            "la_chunk_decay_fwd_state")
 
 
@@ -274,9 +275,10 @@ def la_chunk_decay_bwd_state(q, k, v, dout, decay, dq, dk, dv, state_in=None, ds
     """la_chunk_decay_bwd of one segment: state_in is the state of the tokens before it,
     dstate_in R = sum gamma^(u-T) q_u^T dout_u of the tokens after it (both [B, H, D, D] float32,
     zero if None); dstate_out (if given, not overlapping either) receives R at the segment's
-    first row.  dq may be None: then only dk and dv are computed."""
+    first row.  dq may be None: then only dk and dv are computed; dq, dk and dv may all be
+    None: then only dstate_out is computed (k and v are not read and may be None)."""
     import torch
-    B, H, T, D = _shape(q, k, v, dout, dq, dk, dv)
+    B, H, T, D = _shape(q, dout, k, v, dq, dk, dv)
     for st, name in ((state_in, "state_in"), (dstate_in, "dstate_in"), (dstate_out, "dstate_out")):
         if st is not None and (tuple(st.shape) != (B, H, D, D) or st.dtype != torch.float32 or not st.is_cuda
                                or not st.is_contiguous() or st.device != q.device):

@@ -318,13 +318,16 @@ la_status la_simple_bwd(const void *q, const void *k, const void *v, const void 
 
 static la_status decay_fwd_entry(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
                                  const float *decay, int B, int H, int T, int D, la_dtype dtype, void *workspace,
-                                 size_t workspace_bytes, void *stream) {
+                                 size_t workspace_bytes, void *stream, bool state_entry) {
     const Shape s{B, H, T, D};
     LA_TRY(validate(s, dtype));
-    LA_TRY(check_ptr(q, "q"));
+    // o == NULL on the state entry point: the state only (q is then not read either)
+    const bool sonly = state_entry && !o;
+    if (sonly && !sout) return fail(LA_ERR_INVALID_ARG, "o and state_out are both NULL: nothing to compute");
+    if (!sonly) LA_TRY(check_ptr(q, "q"));
     LA_TRY(check_ptr(k, "k"));
     LA_TRY(check_ptr(v, "v"));
-    LA_TRY(check_ptr(o, "o"));
+    if (!sonly) LA_TRY(check_ptr(o, "o"));
     if (sin) LA_TRY(check_state(sin, "state_in"));
     if (sout) LA_TRY(check_state(sout, "state_out"));
     DecayArgs dec;
@@ -345,14 +348,15 @@ static la_status decay_fwd_entry(const void *q, const void *k, const void *v, vo
 
 la_status la_chunk_decay_fwd(const void *q, const void *k, const void *v, void *o, const float *decay, int B, int H,
                              int T, int D, la_dtype dtype, void *workspace, size_t workspace_bytes, void *stream) {
-    return decay_fwd_entry(q, k, v, o, nullptr, nullptr, decay, B, H, T, D, dtype, workspace, workspace_bytes, stream);
+    return decay_fwd_entry(q, k, v, o, nullptr, nullptr, decay, B, H, T, D, dtype, workspace, workspace_bytes, stream,
+                           false);
 }
 
 la_status la_chunk_decay_fwd_state(const void *q, const void *k, const void *v, void *o, const float *state_in,
                                    float *state_out, const float *decay, int B, int H, int T, int D, la_dtype dtype,
                                    void *workspace, size_t workspace_bytes, void *stream) {
     return decay_fwd_entry(q, k, v, o, state_in, state_out, decay, B, H, T, D, dtype, workspace, workspace_bytes,
-                           stream);
+                           stream, true);
 }
 
 static la_status decay_bwd_entry(const void *q, const void *k, const void *v, const void *dout, const float *sin,
@@ -361,13 +365,16 @@ static la_status decay_bwd_entry(const void *q, const void *k, const void *v, co
                                  void *stream, bool dq_optional) {
     const Shape s{B, H, T, D};
     LA_TRY(validate(s, dtype));
+    // dq, dk and dv all NULL on the state entry point: R at the first row only (k, v not read)
+    const bool sonly = dq_optional && !dq && !dk && !dv;
+    if (sonly && !rout) return fail(LA_ERR_INVALID_ARG, "dq, dk, dv and dstate_out are all NULL: nothing to compute");
     LA_TRY(check_ptr(q, "q"));
-    LA_TRY(check_ptr(k, "k"));
-    LA_TRY(check_ptr(v, "v"));
+    if (!sonly) LA_TRY(check_ptr(k, "k"));
+    if (!sonly) LA_TRY(check_ptr(v, "v"));
     LA_TRY(check_ptr(dout, "dout"));
     if (dq || !dq_optional) LA_TRY(check_ptr(dq, "dq"));
-    LA_TRY(check_ptr(dk, "dk"));
-    LA_TRY(check_ptr(dv, "dv"));
+    if (!sonly) LA_TRY(check_ptr(dk, "dk"));
+    if (!sonly) LA_TRY(check_ptr(dv, "dv"));
     if (sin) LA_TRY(check_state(sin, "state_in"));
     if (rin) LA_TRY(check_state(rin, "dstate_in"));
     if (rout) {

@@ -446,7 +446,9 @@ __device__ __forceinline__ void stash_rows(const uint4 (&x)[N][TileVec<T, D, NT>
 
 // Forward recurrence, thread j holds column j of S:
 //   S_t = gamma S_{t-1} + k_t^T v_t,   o_t[j] = sum_i q_t[i] S_t[i][j].
-template <typename T, int D>
+// OUT = false: the state only (q is not read, o not written; q must still point at a
+// readable tensor of the same shape, e.g. k).
+template <typename T, int D, bool OUT>
 __global__ void __launch_bounds__(D)
 ret_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v, T *__restrict__ o,
         DecayArgs dec, int T_len, int H, const float *__restrict__ sin, float *__restrict__ sout) {
@@ -470,9 +472,9 @@ ret_fwd(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ 
 #pragma unroll
             for (int i = 0; i < D; ++i) {
                 S[i] = fmaf(gamma, S[i], tiles[1][r][i] * vj);
-                acc = fmaf(tiles[0][r][i], S[i], acc);
+                if (OUT) acc = fmaf(tiles[0][r][i], S[i], acc);
             }
-            io<T>::st(o + base + (long long)(ts + r) * D + j, acc);
+            if (OUT) io<T>::st(o + base + (long long)(ts + r) * D + j, acc);
         }
     }
     if (sout) {
@@ -518,7 +520,9 @@ ret_bwd_dq(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict
 // 0..D-1 hold row i of R (dk_s[i] = sum_j R[i][j] v_s[j]); threads D..2D-1
 // hold column j of R (dv_s[j] = sum_i k_s[i] R[i][j]).  R starts from rin (R one
 // past the segment's last row) or zero; rout receives R at the segment's first row.
-template <typename T, int D>
+// OUT = false: R only (rout), no dk, dv: k and v are not read (they must still point at
+// readable tensors of the same shape, e.g. q and g).
+template <typename T, int D, bool OUT>
 __global__ void __launch_bounds__(2 * D)
 ret_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
              const T *__restrict__ g, T *__restrict__ dk, T *__restrict__ dv, DecayArgs dec, int T_len, int H,
@@ -548,10 +552,10 @@ ret_bwd_dkdv(const T *__restrict__ q, const T *__restrict__ k, const T *__restri
 #pragma unroll
                 for (int j = 0; j < D; ++j) {
                     Rr[j] = fmaf(gamma, Rr[j], qi * tiles[3][r][j]);
-                    acc = fmaf(Rr[j], tiles[2][r][j], acc);
+                    if (OUT) acc = fmaf(Rr[j], tiles[2][r][j], acc);
                 }
-                io<T>::st(dk + base + (long long)(ts + r) * D + idx, acc);
-            } else {
+                if (OUT) io<T>::st(dk + base + (long long)(ts + r) * D + idx, acc);
+            } else if (OUT) {
                 const float gj = tiles[3][r][idx];
 #pragma unroll
                 for (int i = 0; i < D; ++i) {
@@ -1704,20 +1708,26 @@ la_status state_bwd_d(bool bidir, const void *q, const void *k, const void *v, c
 template <typename T, int D>
 la_status decay_fwd_t(const T *q, const T *k, const T *v, T *o, const float *sin, float *sout, const DecayArgs &dec,
                       const Shape &s, cudaStream_t st) {
-    return launch("simt_ret_fwd", ret_fwd<T, D>, dim3((unsigned)s.BH()), dim3(D), 0, st, q, k, v, o, dec, s.T, s.H,
-                  sin, sout);
+    if (!o)   // the state only
+        return launch("simt_ret_state", ret_fwd<T, D, false>, dim3((unsigned)s.BH()), dim3(D), 0, st, k, k, v, o, dec,
+                      s.T, s.H, sin, sout);
+    return launch("simt_ret_fwd", ret_fwd<T, D, true>, dim3((unsigned)s.BH()), dim3(D), 0, st, q, k, v, o, dec, s.T,
+                  s.H, sin, sout);
 }
 
 template <typename T, int D>
 la_status decay_bwd_t(const T *q, const T *k, const T *v, const T *g, const float *sin, const float *rin, float *rout,
                       const DecayArgs &dec, T *dq, T *dk, T *dv, const Shape &s, cudaStream_t st) {
+    if (!dq && !dk && !dv)   // R at the first row only
+        return launch("simt_ret_bwd_state", ret_bwd_dkdv<T, D, false>, dim3((unsigned)s.BH()), dim3(2 * D), 0, st, q,
+                      q, g, g, dk, dv, dec, s.T, s.H, rin, rout);
     if (dq) {   // dq == null: dk, dv only
         la_status rc = launch("simt_ret_bwd_dq", ret_bwd_dq<T, D>, dim3((unsigned)s.BH()), dim3(D), 0, st, k, v, g,
                               dq, dec, s.T, s.H, sin);
         if (rc) return rc;
     }
-    return launch("simt_ret_bwd_dkdv", ret_bwd_dkdv<T, D>, dim3((unsigned)s.BH()), dim3(2 * D), 0, st, q, k, v, g,
-                  dk, dv, dec, s.T, s.H, rin, rout);
+    return launch("simt_ret_bwd_dkdv", ret_bwd_dkdv<T, D, true>, dim3((unsigned)s.BH()), dim3(2 * D), 0, st, q, k, v,
+                  g, dk, dv, dec, s.T, s.H, rin, rout);
 }
 
 }  // namespace

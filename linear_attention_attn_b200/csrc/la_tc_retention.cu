@@ -124,6 +124,9 @@ struct RetJobs {
     const float *sin[3];
     float *sout[3];
     int sin_t[3];
+    // sonly[p] != 0: the pass computes its state only (sout), no output: only k and v
+    // are loaded, and per chunk only K^ and dS^T are formed.
+    int sonly[3];
 };
 
 // Grid: one CTA per (pass, b, h), pass = blockIdx.x / BH.  decay[h] = gamma_h.
@@ -188,6 +191,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
     const int pass = blockIdx.x / BH;
     const int bh = blockIdx.x % BH;
     const bool rev = jobs.rev[pass] != 0;
+    const bool sonly = jobs.sonly[pass] != 0;
     const CUtensorMap *tmQ = &jobs.q[pass], *tmK = &jobs.k[pass], *tmV = &jobs.v[pass], *tmO = &jobs.o[pass];
     const float gamma = dec.gamma[bh % H];
     const int nchunks = (T + kC - 1) / kC;
@@ -249,9 +253,9 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             for (int it = 0; it < nchunks; ++it) {
                 const int c = rev ? nchunks - 1 - it : it;
                 if (!LA_RWAIT(&empty[s], ph ^ 1, 0x1u)) break;
-                mbar_arrive_expect_tx(&full[s], 3 * kTile128);
+                mbar_arrive_expect_tx(&full[s], (sonly ? 2 : 3) * kTile128);
                 for (int b = 0; b < 2; ++b) {
-                    tma_load_3d(sQ + s * kTile128 + b * kBox, tmQ, &full[s], 64 * b, c * kC, bh);
+                    if (!sonly) tma_load_3d(sQ + s * kTile128 + b * kBox, tmQ, &full[s], 64 * b, c * kC, bh);
                     tma_load_3d(sK + s * kTile128 + b * kBox, tmK, &full[s], 64 * b, c * kC, bh);
                     tma_load_3d(sV + s * kTile128 + b * kBox, tmV, &full[s], 64 * b, c * kC, bh);
                 }
@@ -279,7 +283,28 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             }
             umma_commit_warp(&pfull[c & 1]);
         };
-        bool ok = nchunks > 0 && LA_WWAIT(&full[0], 0, 0x4u);
+        if (sonly) {
+            // state only: dS^T of every chunk, released as soon as it has read the stage
+            const uint64_t dkh = sdesc_sw128(smem_u32(sKh), kBox, 1024);
+            for (int it = 0; it < nchunks; ++it) {
+                const uint32_t pc = (uint32_t)(it & 1), pp = pc ^ 1u;
+                const int s = it % NST;
+                if (!LA_WWAIT(khready, pc, 0x80u)) break;
+                if (it > 0 && !LA_WWAIT(dsread, pp, 0x40u)) break;
+                tc_fence_after();
+                const uint64_t dv = sdesc_sw128(smem_u32(sV + s * kTile128), kBox, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                    for (int op = 0; op < 2; ++op)
+                        umma_f16_ss_warp(tmem + cDS, desc_at(dv, kk * 2048), desc_at(dkh, op * kTile128 + kk * 2048),
+                                         ID_DST, (kk | op) ? 1u : 0u);
+                }
+                umma_commit_warp(dsfull);
+                umma_commit_warp(&empty[s]);
+            }
+        }
+        bool ok = !sonly && nchunks > 0 && LA_WWAIT(&full[0], 0, 0x4u);
         if (ok) {
             tc_fence_after();
             issue_p(0);
@@ -353,7 +378,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         const int sub = warp & 3;
         const uint32_t lanes = (uint32_t)(32 * sub) << 16;
         const int ri = 16 * sub + (lane & 15), hcol = lane >> 4;   // row; column half (M = 64 rows in lanes 0..15)
-        for (int it = 0; it < nchunks; ++it) {
+        for (int it = 0; it < (sonly ? 0 : nchunks); ++it) {
             const uint32_t pc = (uint32_t)(it & 1);
             const int rows = min(kC, T - (rev ? nchunks - 1 - it : it) * kC);
             if (!__all_sync(0xffffffffu, LA_RWAIT(&pfull[it & 1], (uint32_t)((it >> 1) & 1), 0x400u))) break;
@@ -397,7 +422,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         const int q4 = lane & 3;                            // fragment: columns 2 q4 (+1) of lanes lane / 4 (+8)
         const int mk = lane >> 3, mj = lane & 7;            // stmatrix: matrix mk, stored row mj
         bool live = true;
-        for (int it = 0; it < nchunks; ++it) {
+        for (int it = 0; it < (sonly ? 0 : nchunks); ++it) {
             const int c = rev ? nchunks - 1 - it : it;
             const uint32_t pc = (uint32_t)(it & 1);
             if (ot == 0) tma_store_wait_read<0>();
@@ -522,7 +547,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             __syncwarp();
             if (lane == 0) mbar_arrive(sready);
         };
-        write_state();                                     // S_0
+        if (!sonly) write_state();                         // S_0
         // K^ = diag(gamma^(C-1-j)) K of chunk iteration itk as hi + lo: thread kt takes row
         // kt % 64 and the 8-element chunks 4 (kt / 64) .. + 3 of the row's 16.  Forwards in
         // time the weights count back from the chunk's last valid row, so that the state
@@ -561,6 +586,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             if (it + 1 == nchunks) break;                  // st holds the state after the sequence
             // dS^T_c is complete, so it has read K^_c: the buffer takes K^ of the next chunk
             if (!build_khat(it + 1)) break;
+            if (sonly) continue;                           // nothing reads the state operand
             if (!__all_sync(0xffffffffu, LA_RWAIT(sfree, pc, 0x2000u))) break;   // O_inter^T(c) read S_c
             __syncwarp();
             tc_fence_after();
@@ -603,12 +629,14 @@ la_status retention_fwd(const void *q, const void *k, const void *v, void *o, co
     memset(&jobs, 0, sizeof jobs);
     jobs.sin[0] = sin;
     jobs.sout[0] = sout;
-    LA_TRY(retention_map(&jobs.q[0], q, s));
+    jobs.sonly[0] = o == nullptr;   // the state only: q and o are not touched (their maps stand in as k's)
+    LA_TRY(retention_map(&jobs.q[0], o ? q : k, s));
     LA_TRY(retention_map(&jobs.k[0], k, s));
     LA_TRY(retention_map(&jobs.v[0], v, s));
-    LA_TRY(retention_map(&jobs.o[0], o, s));
+    LA_TRY(retention_map(&jobs.o[0], o ? o : k, s));
+    const char *name = o ? "tc_retention_fwd" : "tc_retention_state";
     if (fold_ok(dec, s.H))
-        return launch_pdl("tc_retention_fwd", retention_kernel<true>, dim3((unsigned)s.BH()), dim3(kRThreads),
+        return launch_pdl(name, retention_kernel<true>, dim3((unsigned)s.BH()), dim3(kRThreads),
                           (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
     return launch_pdl("tc_retention_fwd_unfolded", retention_kernel<false>, dim3((unsigned)s.BH()), dim3(kRThreads),
                       (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
@@ -621,7 +649,24 @@ la_status retention_bwd(const void *q, const void *k, const void *v, const void 
     memset(&jobs, 0, sizeof jobs);
     // dq = retention(dO, V, K); dv = reverse retention(K, Q, dO); dk = reverse retention(V, dO, Q).
     // Their states are S^T (S = sum k^T v), R and R^T (R = sum gamma^(t-s) q_t^T dO_t).
-    // dq == null leaves out the first pass.
+    // dq == null leaves out the first pass; dq, dk and dv all null leave only the second, as a
+    // state-only pass (R at the first row, rout).
+    const bool sonly = !dq && !dk && !dv;
+    if (sonly) {
+        jobs.rev[0] = 1;
+        jobs.sin[0] = rin;
+        jobs.sout[0] = rout;
+        jobs.sonly[0] = 1;
+        LA_TRY(retention_map(&jobs.q[0], q, s));
+        LA_TRY(retention_map(&jobs.k[0], q, s));
+        LA_TRY(retention_map(&jobs.v[0], g, s));
+        LA_TRY(retention_map(&jobs.o[0], q, s));
+        if (fold_ok(dec, s.H))
+            return launch_pdl("tc_retention_state", retention_kernel<true>, dim3((unsigned)s.BH()), dim3(kRThreads),
+                              (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
+        return launch_pdl("tc_retention_state_unfolded", retention_kernel<false>, dim3((unsigned)s.BH()),
+                          dim3(kRThreads), (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
+    }
     struct Pass {
         const void *q, *k, *v;
         void *o;

@@ -93,26 +93,30 @@ def decay_forward(q, k, v, o, decay, state_out=None, entering=None, group=None, 
                   workspace=None):
     """The decay op (retention) forward for this rank's segment of a sequence split along T
     (rank r holds the r-th segment).  A segment's output needs the state of every token before
-    it: pass 1 gives each segment's own end state E_r (from a zero state) and, on rank 0, its
-    final output; an all-gather shares the E_r and the segment lengths; la_chunk_decay_scan forms
-    S_r = sum_{r' < r} gamma^(tokens between) E_r'; pass 2 recomputes the segment from S_r.
+    it: pass 1 gives each segment's own end state E_r from a zero state (a state-only pass, o
+    not computed; on rank 0, whose entering state is zero, the whole forward, which is final);
+    an all-gather shares the E_r and the segment lengths; la_chunk_decay_scan forms
+    S_r = sum_{r' < r} gamma^(tokens between) E_r'; the forward then runs once from S_r.
     state_out (optional, [B, H, D, D] fp32) receives the state after this rank's segment (on the
     last rank: after the whole sequence); entering (optional, same shape) receives S_r, which
     decay_backward needs."""
     import torch
     ops = _decay_ops(ops)
-    B, H, T, D = (int(x) for x in q.shape)
+    B, H, T, D = (int(x) for x in k.shape)
     kw = {} if workspace is None else {"workspace": workspace}
     world, rank = _world(group)
-    sdt = torch.float32 if q.is_cuda else torch.float64
-    end = state_out if state_out is not None else torch.empty((B, H, D, D), dtype=sdt, device=q.device)
+    sdt = torch.float32 if k.is_cuda else torch.float64
+    end = state_out if state_out is not None else torch.empty((B, H, D, D), dtype=sdt, device=k.device)
     if entering is not None:
         entering.zero_()
-    ops.la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=None, state_out=end, stream=stream, **kw)
+    if world == 1 or rank == 0:                    # nothing enters the first segment: this pass is final
+        ops.la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=None, state_out=end, stream=stream, **kw)
+    else:                                          # this segment's own end state only
+        ops.la_chunk_decay_fwd_state(None, k, v, None, decay, state_in=None, state_out=end, stream=stream, **kw)
     if world == 1:
         return state_out
     ends, lens = _gather_states(end, T, group)
-    if rank == 0:                                  # nothing enters the first segment: pass 1 is final
+    if rank == 0:
         return state_out
     sin = entering if entering is not None else torch.empty_like(end)
     ops.la_chunk_decay_scan(ends, entering_gaps(lens, rank), decay, sin, stream=stream)
@@ -123,24 +127,29 @@ def decay_forward(q, k, v, o, decay, state_out=None, entering=None, group=None, 
 def decay_backward(q, k, v, dout, decay, dq, dk, dv, entering=None, group=None, ops=None, stream=None,
                    workspace=None):
     """The decay op's backward for this rank's segment, with `entering` the state S_r entering it
-    (from decay_forward; None for zero).  dq needs only S_r, so pass 1 (the whole backward from
-    S_r and a zero R) gives the final dq and each segment's own reverse-sweep state F_r at its
-    first token; an all-gather shares the F_r; la_chunk_decay_scan forms the R arriving from the
-    segments to the right, R_r = sum_{r' > r} gamma^(tokens between) F_r'; pass 2 recomputes dk
-    and dv from R_r (the last rank has none and skips it)."""
+    (from decay_forward; None for zero).  dk and dv need R, which arrives from the segments to the
+    right: pass 1 gives each segment's own reverse-sweep state F_r at its first token from a zero
+    R (a state-only pass; on the last rank, where nothing arrives, the whole backward, which is
+    final); an all-gather shares the F_r; la_chunk_decay_scan forms
+    R_r = sum_{r' > r} gamma^(tokens between) F_r'; the backward then runs once from S_r and R_r."""
     import torch
     ops = _decay_ops(ops)
     B, H, T, D = (int(x) for x in q.shape)
     kw = {} if workspace is None else {"workspace": workspace}
     world, rank = _world(group)
     f = torch.empty((B, H, D, D), dtype=torch.float32 if q.is_cuda else torch.float64, device=q.device)
-    ops.la_chunk_decay_bwd_state(q, k, v, dout, decay, dq, dk, dv, state_in=entering, dstate_in=None,
-                                 dstate_out=f, stream=stream, **kw)
+    if rank == world - 1:                          # nothing arrives after the last segment: final
+        ops.la_chunk_decay_bwd_state(q, k, v, dout, decay, dq, dk, dv, state_in=entering, dstate_in=None,
+                                     dstate_out=f, stream=stream, **kw)
+    else:                                          # this segment's own R at its first token only
+        ops.la_chunk_decay_bwd_state(q, None, None, dout, decay, None, None, None, dstate_out=f, stream=stream,
+                                     **kw)
     if world == 1:
         return
     fs, lens = _gather_states(f, T, group)
-    if rank == world - 1:                          # nothing arrives from after the last segment
+    if rank == world - 1:
         return
     rin = torch.empty_like(f)
     ops.la_chunk_decay_scan(fs, leaving_gaps(lens, rank), decay, rin, stream=stream)
-    ops.la_chunk_decay_bwd_state(q, k, v, dout, decay, None, dk, dv, dstate_in=rin, stream=stream, **kw)
+    ops.la_chunk_decay_bwd_state(q, k, v, dout, decay, dq, dk, dv, state_in=entering, dstate_in=rin,
+                                 stream=stream, **kw)

@@ -198,3 +198,43 @@ def test_sequence_split_across_emulated_ranks(dtype, D):
     for j, name in enumerate(("dq", "dk", "dv")):
         got = torch.cat([gr[j] for gr in grads], dim=2).cpu().double().numpy()
         pu.assert_grad(got, whole[j], "emulated ranks %s" % name)
+
+
+@pytest.mark.parametrize("dtype,D,T", [("bf16", 128, 300), ("bf16", 128, 37), ("f32", 64, 300), ("f16", 128, 129)])
+def test_state_only_passes(dtype, D, T):
+    """The state-only forms (o None; dq, dk, dv None) give exactly the states of the whole passes
+    (the same arithmetic computes them) and the oracle's; q and o, resp. k, v, dq, dk and dv are
+    not needed.  bf16 D = 128 runs on the tensor cores, the rest on the CUDA cores."""
+    import linear_attention_attn_b200 as la
+    w = synth.Workload("case", "retention", 2, 3, T, D, dtype, q_scale=D ** -0.5)
+    inp = synth.make_inputs(w, seed=25, with_grad=True)
+    dev = _dev()
+    sin = (synth.normal((w.B, w.H, D, D), 26, 0) * 4.0).to(dev)
+    rin = (synth.normal((w.B, w.H, D, D), 26, 1) * 4.0 * D ** -0.5).to(dev)
+    q, k, v, g = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    gam = inp["gamma"]
+    st = lambda: torch.full((w.B, w.H, D, D), float("nan"), dtype=torch.float32, device=dev)
+    s_full, s_only, r_full, r_only = st(), st(), st(), st()
+    la.la_chunk_decay_fwd_state(q, k, v, torch.empty_like(q), gam, state_in=sin, state_out=s_full)
+    la.la_chunk_decay_fwd_state(None, k, v, None, gam, state_in=sin, state_out=s_only)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    la.la_chunk_decay_bwd_state(q, k, v, g, gam, dq, dk, dv, state_in=sin, dstate_in=rin, dstate_out=r_full)
+    la.la_chunk_decay_bwd_state(q, None, None, g, gam, None, None, None, dstate_in=rin, dstate_out=r_only)
+    torch.cuda.synchronize()
+    assert torch.equal(s_only, s_full)
+    assert torch.equal(r_only, r_full)
+    _, want_s = oracle.retention_fwd_state(inp["q"], inp["k"], inp["v"], gam, sin.double().cpu().numpy())
+    want_r = oracle.retention_bwd_state(inp["q"], inp["k"], inp["v"], inp["do"], gam, sin.double().cpu().numpy(),
+                                        rin.double().cpu().numpy())[3]
+    assert _rel_l2(s_only.cpu().numpy(), want_s) <= STATE_REL_L2
+    assert _rel_l2(r_only.cpu().numpy(), want_r) <= STATE_REL_L2
+
+
+def test_state_only_calls_need_an_output():
+    import linear_attention_attn_b200 as la
+    dev = _dev()
+    k = torch.zeros((1, 1, 64, 128), dtype=torch.bfloat16, device=dev)
+    with pytest.raises(la.LAError):
+        la.la_chunk_decay_fwd_state(None, k, k, None, [0.9])
+    with pytest.raises(la.LAError):
+        la.la_chunk_decay_bwd_state(k, None, None, k, [0.9], None, None, None)

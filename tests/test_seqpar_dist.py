@@ -125,24 +125,29 @@ def test_two_ranks_match_the_whole_sequence(feature):
         np.testing.assert_allclose(got, want[i], rtol=1e-10, atol=1e-12, err_msg=name)
 
 
-def _decay_ops():
+def _decay_ops(calls):
     """The decay op's segment calls on float64 CPU tensors, from their definitions in
-    include/la.h: the recurrent form forwards (S) and backwards (R), and the combine."""
+    include/la.h: the recurrent form forwards (S) and backwards (R), the state-only forms (o, or
+    dq, dk and dv, None), and the combine.  `calls` records which form each call took."""
     def gam4(decay):
         return torch.as_tensor(list(decay), dtype=torch.float64)[None, :, None, None]
 
     def la_chunk_decay_fwd_state(q, k, v, o, decay, state_in=None, state_out=None, stream=None):
-        B, H, T, D = q.shape
+        calls.append("fwd" if o is not None else "fwd_state")
+        B, H, T, D = k.shape
         g = gam4(decay)
         S = state_in.clone() if state_in is not None else torch.zeros(B, H, D, D, dtype=torch.float64)
         for t in range(T):
             S = g * S + torch.einsum("bhi,bhj->bhij", k[:, :, t], v[:, :, t])
-            o[:, :, t] = torch.einsum("bhi,bhij->bhj", q[:, :, t], S)
+            if o is not None:
+                o[:, :, t] = torch.einsum("bhi,bhij->bhj", q[:, :, t], S)
         if state_out is not None:
             state_out.copy_(S)
 
     def la_chunk_decay_bwd_state(q, k, v, dout, decay, dq, dk, dv, state_in=None, dstate_in=None,
                                  dstate_out=None, stream=None):
+        sonly = dq is None and dk is None and dv is None
+        calls.append("bwd_state" if sonly else "bwd")
         B, H, T, D = q.shape
         g = gam4(decay)
         if dq is not None:
@@ -153,8 +158,9 @@ def _decay_ops():
         R = dstate_in.clone() if dstate_in is not None else torch.zeros(B, H, D, D, dtype=torch.float64)
         for s in reversed(range(T)):
             R = g * R + torch.einsum("bhi,bhj->bhij", q[:, :, s], dout[:, :, s])
-            dk[:, :, s] = torch.einsum("bhij,bhj->bhi", R, v[:, :, s])
-            dv[:, :, s] = torch.einsum("bhi,bhij->bhj", k[:, :, s], R)
+            if not sonly:
+                dk[:, :, s] = torch.einsum("bhij,bhj->bhi", R, v[:, :, s])
+                dv[:, :, s] = torch.einsum("bhi,bhij->bhj", k[:, :, s], R)
         if dstate_out is not None:
             dstate_out.copy_(R)
 
@@ -184,11 +190,12 @@ def _decay_rank_main(rank, world, port, cuts, gam, out):
     o = torch.empty_like(qs)
     st = torch.empty(2, 3, 6, 6, dtype=torch.float64)
     ent = torch.empty_like(st)
-    ops = _decay_ops()
+    calls = []
+    ops = _decay_ops(calls)
     seqpar.decay_forward(qs, ks, vs, o, gam, state_out=st, entering=ent, ops=ops)
     dq, dk, dv = (torch.empty_like(qs) for _ in range(3))
     seqpar.decay_backward(qs, ks, vs, gs, gam, dq, dk, dv, entering=ent, ops=ops)
-    out[rank] = (o.numpy(), st.numpy(), dq.numpy(), dk.numpy(), dv.numpy())
+    out[rank] = (o.numpy(), st.numpy(), dq.numpy(), dk.numpy(), dv.numpy(), list(calls))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -224,3 +231,8 @@ def test_decay_forward_and_backward_over_three_ranks():
     for i, name in enumerate(("dq", "dk", "dv")):
         got = np.concatenate([out[r][2 + i] for r in range(3)], axis=2)
         np.testing.assert_allclose(got, want[i], rtol=1e-10, atol=1e-12, err_msg=name)
+    # each rank runs the whole forward and the whole backward once; a state-only pass
+    # precedes them where the neighbours' states are needed
+    assert out[0][5] == ["fwd", "bwd_state", "bwd"]
+    assert out[1][5] == ["fwd_state", "fwd", "bwd_state", "bwd"]
+    assert out[2][5] == ["fwd_state", "fwd", "bwd"]
