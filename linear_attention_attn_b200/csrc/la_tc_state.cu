@@ -53,6 +53,11 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 
 // Waits used by every role; codes identify the barrier in the fault word.
 #define LA_WAIT(bar, par, code) mbar_wait((bar), (par), s_abort, &g_tc_fault, (code))
+// The UMMA-issuing warps run their loops with all 32 lanes in step (every lane waits, one
+// elected lane issues each UMMA and commit), so the descriptors stay warp-uniform: issued
+// by one lane alone, each UMMA first moved its operands to uniform registers, and on a
+// scheduler shared with busy warps that cost ~140 cycles an instruction.
+#define LA_WWAIT(bar, par, code) __all_sync(0xffffffffu, LA_WAIT((bar), (par), (code)))
 
 // ============================================================ state_reduce ==
 // Partial (S | z) of every (CTA, head) segment.  UMMA M = 64 (the state row i),
@@ -166,42 +171,41 @@ state_reduce_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            int s = 0, a = 0;
-            uint32_t ph = 0, aph = 0;
-            bool seg_start = true;
-            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long x = t.x;
-                const bool seg_end = (x + 1 == x1) || t.last_of_head();
-                if (seg_start) {
-                    if (!LA_WAIT(&accfree[a], aph ^ 1, 0x2u)) break;
-                }
-                if (!LA_WAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
-                tc_fence_after();
-                const uint32_t d = tmem + (uint32_t)a * 128u;
-                const uint32_t aV = smem_u32(sV + s * kTileBytes);
-                const uint32_t lbo = BIDIR ? (smem_u32(sOnes) - aV) : (uint32_t)kTileBytes;
-                const uint64_t dk = sdesc_sw128(smem_u32(sK + s * kTileBytes), kTileBytes, 1024);
-                const uint64_t dkl = sdesc_sw128(smem_u32(sKlo + s * kTileBytes), kTileBytes, 1024);
-                const uint64_t dv = sdesc_sw128(aV, lbo, 1024);
-#pragma unroll
-                for (int kk = 0; kk < kRows / 16; ++kk) {
-                    umma_f16_ss(d, desc_at(dk, kk * 2048), desc_at(dv, kk * 2048), IDESC,
-                                (seg_start && kk == 0) ? 0u : 1u);
-                    if (KLO) umma_f16_ss(d, desc_at(dkl, kk * 2048), desc_at(dv, kk * 2048), IDESC, 1u);
-                }
-                umma_commit(&empty[s]);
-                if (seg_end) {
-                    umma_commit(&accfull[a]);
-                    a ^= 1;
-                    if (a == 0) aph ^= 1;
-                }
-                seg_start = seg_end;
-                if (++s == NST) { s = 0; ph ^= 1; }
+        int s = 0, a = 0;
+        uint32_t ph = 0, aph = 0;
+        bool seg_start = true;
+        for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+            const long long x = t.x;
+            const bool seg_end = (x + 1 == x1) || t.last_of_head();
+            if (seg_start) {
+                if (!LA_WWAIT(&accfree[a], aph ^ 1, 0x2u)) break;
             }
-            umma_commit(drain);
-            mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+            if (!LA_WWAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
+            tc_fence_after();
+            const uint32_t d = tmem + (uint32_t)a * 128u;
+            const uint32_t aV = smem_u32(sV + s * kTileBytes);
+            const uint32_t lbo = BIDIR ? (smem_u32(sOnes) - aV) : (uint32_t)kTileBytes;
+            const uint64_t dk = sdesc_sw128(smem_u32(sK + s * kTileBytes), kTileBytes, 1024);
+            const uint64_t dkl = sdesc_sw128(smem_u32(sKlo + s * kTileBytes), kTileBytes, 1024);
+            const uint64_t dv = sdesc_sw128(aV, lbo, 1024);
+#pragma unroll
+            for (int kk = 0; kk < kRows / 16; ++kk) {
+                umma_f16_ss_warp(d, desc_at(dk, kk * 2048), desc_at(dv, kk * 2048), IDESC,
+                                 (seg_start && kk == 0) ? 0u : 1u);
+                if (KLO) umma_f16_ss_warp(d, desc_at(dkl, kk * 2048), desc_at(dv, kk * 2048), IDESC, 1u);
+            }
+            umma_commit_warp(&empty[s]);
+            if (seg_end) {
+                umma_commit_warp(&accfull[a]);
+                a ^= 1;
+                if (a == 0) aph ^= 1;
+            }
+            seg_start = seg_end;
+            if (++s == NST) { s = 0; ph ^= 1; }
         }
+        umma_commit_warp(drain);
+        mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+        __syncwarp();
     } else if (warp < kEw0) {
         if (BIDIR) {
             const int xi = threadIdx.x - kXw0 * 32;
@@ -377,39 +381,38 @@ output_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            int s = 0, a = 0, hidx = -1;
-            uint32_t ph = 0, aph = 0;
-            long long prev_h = -1;
-            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long h = t.h;
-                if (h != prev_h) {
-                    ++hidx;
-                    prev_h = h;
-                    if (!LA_WAIT(&opready[hidx & 1], (uint32_t)((hidx >> 1) & 1), 0x20u)) break;
-                }
-                if (!LA_WAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
-                if (!LA_WAIT(&accempty[a], aph ^ 1, 0x2u)) break;
-                tc_fence_after();
-                const uint32_t d = tmem + (uint32_t)a * 128u;
-                const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTileBytes), 16, 1024);
-                const uint64_t dop = sdesc_sw128(smem_u32(sOp + (hidx & 1) * 2 * OPB), 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-                    for (int op = 0; op < NOPS; ++op)
-                        umma_f16_ss(d, desc_at(dq, kk * 32), desc_at(dop, op * OPB + kk * 32), IDESC,
-                                    (kk | op) ? 1u : 0u);
-                }
-                umma_commit(&empty[s]);
-                umma_commit(&accfull[a]);
-                a ^= 1;
-                if (a == 0) aph ^= 1;
-                if (++s == NST) { s = 0; ph ^= 1; }
+        int s = 0, a = 0, hidx = -1;
+        uint32_t ph = 0, aph = 0;
+        long long prev_h = -1;
+        for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+            const long long h = t.h;
+            if (h != prev_h) {
+                ++hidx;
+                prev_h = h;
+                if (!LA_WWAIT(&opready[hidx & 1], (uint32_t)((hidx >> 1) & 1), 0x20u)) break;
             }
-            umma_commit(drain);
-            mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+            if (!LA_WWAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
+            if (!LA_WWAIT(&accempty[a], aph ^ 1, 0x2u)) break;
+            tc_fence_after();
+            const uint32_t d = tmem + (uint32_t)a * 128u;
+            const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTileBytes), 16, 1024);
+            const uint64_t dop = sdesc_sw128(smem_u32(sOp + (hidx & 1) * 2 * OPB), 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                for (int op = 0; op < NOPS; ++op)
+                    umma_f16_ss_warp(d, desc_at(dq, kk * 32), desc_at(dop, op * OPB + kk * 32), IDESC,
+                                     (kk | op) ? 1u : 0u);
+            }
+            umma_commit_warp(&empty[s]);
+            umma_commit_warp(&accfull[a]);
+            a ^= 1;
+            if (a == 0) aph ^= 1;
+            if (++s == NST) { s = 0; ph ^= 1; }
         }
+        umma_commit_warp(drain);
+        mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+        __syncwarp();
     } else if (warp < kEw0) {
         if (BIDIR) {
             const int xi = threadIdx.x - kXw0 * 32;
@@ -672,81 +675,79 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            int s = 0, b = 0;
-            uint32_t ph = 0, bph = 0, oph = 0;
-            long long prev_h = -1;
-            bool dead = false;
-            for (TileCursor t(x0, nt); t.x < x1 && !dead; t.next()) {
-                const long long h = t.h;
-                if (h != prev_h) {
-                    if (!LA_WAIT(opready, oph, 0x20u)) break;
-                    oph ^= 1;
-                    prev_h = h;
-                }
-                if (!LA_WAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
-                if (!LA_WAIT(&acc12empty[b], bph ^ 1, 0x2u)) break;
-                tc_fence_after();
-                const uint32_t d1 = tmem + (uint32_t)b * 256u, d2 = d1 + 96u;
-                const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTileBytes), 16, 1024);
-                const uint64_t dg = sdesc_sw128(smem_u32(sG + s * kTileBytes), 16, 1024);
-                const uint64_t dql = sdesc_sw128(smem_u32(sQlo + s * kTileBytes), 16, 1024);
-                const uint64_t dok = sdesc_sw128(smem_u32(sOp), 16, 1024);     // state operand read K-major
-                const uint64_t dom = sdesc_sw128(smem_u32(sOp), OPB, 1024);    // ... and MN-major
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-                    for (int op = 0; op < NOPS; ++op) {
-                        if (BIDIR)
-                            umma_f16_ss(d1, desc_at(dq, kk * 32), desc_at(dok, op * OPB + kk * 32), IDESC1,
-                                        (kk | op) ? 1u : 0u);
-                        umma_f16_ss(d2, desc_at(dg, kk * 32), desc_at(dom, op * OPB + kk * 2048), IDESC2,
-                                    (kk | op) ? 1u : 0u);
-                    }
-                    if (QLO) umma_f16_ss(d1, desc_at(dql, kk * 32), desc_at(dok, kk * 32), IDESC1, 1u);
-                }
-                umma_commit(&acc12full[b]);
-                b ^= 1;
-                if (b == 0) bph ^= 1;
-                if (++s == NST) { s = 0; ph ^= 1; }
+        int s = 0, b = 0;
+        uint32_t ph = 0, bph = 0, oph = 0;
+        long long prev_h = -1;
+        bool dead = false;
+        for (TileCursor t(x0, nt); t.x < x1 && !dead; t.next()) {
+            const long long h = t.h;
+            if (h != prev_h) {
+                if (!LA_WWAIT(opready, oph, 0x20u)) break;
+                oph ^= 1;
+                prev_h = h;
             }
-            umma_commit(drain);
-            mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+            if (!LA_WWAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
+            if (!LA_WWAIT(&acc12empty[b], bph ^ 1, 0x2u)) break;
+            tc_fence_after();
+            const uint32_t d1 = tmem + (uint32_t)b * 256u, d2 = d1 + 96u;
+            const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTileBytes), 16, 1024);
+            const uint64_t dg = sdesc_sw128(smem_u32(sG + s * kTileBytes), 16, 1024);
+            const uint64_t dql = sdesc_sw128(smem_u32(sQlo + s * kTileBytes), 16, 1024);
+            const uint64_t dok = sdesc_sw128(smem_u32(sOp), 16, 1024);     // state operand read K-major
+            const uint64_t dom = sdesc_sw128(smem_u32(sOp), OPB, 1024);    // ... and MN-major
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                for (int op = 0; op < NOPS; ++op) {
+                    if (BIDIR)
+                        umma_f16_ss_warp(d1, desc_at(dq, kk * 32), desc_at(dok, op * OPB + kk * 32), IDESC1,
+                                         (kk | op) ? 1u : 0u);
+                    umma_f16_ss_warp(d2, desc_at(dg, kk * 32), desc_at(dom, op * OPB + kk * 2048), IDESC2,
+                                     (kk | op) ? 1u : 0u);
+                }
+                if (QLO) umma_f16_ss_warp(d1, desc_at(dql, kk * 32), desc_at(dok, kk * 32), IDESC1, 1u);
+            }
+            umma_commit_warp(&acc12full[b]);
+            b ^= 1;
+            if (b == 0) bph ^= 1;
+            if (++s == NST) { s = 0; ph ^= 1; }
         }
+        umma_commit_warp(drain);
+        mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+        __syncwarp();
     } else if (warp == kQU2) {
         // Second UMMA issuer: MMA3 of every tile, in tile order, once the epilogue
         // warps have written its g/n and w.  A thread's issue rate, not the tensor
         // pipe, bounds these small-N UMMAs while the other warps of its scheduler
         // are busy, so the two UMMA groups of a tile come from two schedulers.
-        if (lane == 0) {
-            int s = 0;
-            uint32_t ph = 0;
-            long long seg = 0;                     // segments started (accS free parity)
-            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const bool seg_start = (t.x == x0) || t.j == 0;
-                const bool seg_end = (t.x + 1 == x1) || t.last_of_head();
-                if (seg_start) {
-                    if (!LA_WAIT(accSfree, (uint32_t)((seg & 1) ^ 1), 0x40u)) break;
-                    ++seg;
-                }
-                if (!LA_WAIT(&gnready[s], ph, 0x80u)) break;
-                tc_fence_after();
-                const uint32_t aG = smem_u32(sG + s * kTileBytes);
-                // the second MN atom of [g/n | w] starts at column 16 s of the shared w tile
-                const uint32_t lbo = BIDIR ? smem_u32(sW) + 32u * (uint32_t)s - aG : (uint32_t)kTileBytes;
-                const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTileBytes), kTileBytes, 1024);
-                const uint64_t dg = sdesc_sw128(aG, lbo, 1024);
-#pragma unroll
-                for (int kk = 0; kk < kRows / 16; ++kk)
-                    umma_f16_ss(tmem + kAccS, desc_at(dq, kk * 2048), desc_at(dg, kk * 2048), IDESC3,
-                                (seg_start && kk == 0) ? 0u : 1u);
-                umma_commit(&empty[s]);
-                if (seg_end) umma_commit(accSfull);
-                if (++s == NST) { s = 0; ph ^= 1; }
+        int s = 0;
+        uint32_t ph = 0;
+        long long seg = 0;                     // segments started (accS free parity)
+        for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+            const bool seg_start = (t.x == x0) || t.j == 0;
+            const bool seg_end = (t.x + 1 == x1) || t.last_of_head();
+            if (seg_start) {
+                if (!LA_WWAIT(accSfree, (uint32_t)((seg & 1) ^ 1), 0x40u)) break;
+                ++seg;
             }
-            umma_commit(drain2);
-            mbar_wait_slow(smem_u32(drain2), 0, nullptr, &g_tc_fault, 0x400u);
+            if (!LA_WWAIT(&gnready[s], ph, 0x80u)) break;
+            tc_fence_after();
+            const uint32_t aG = smem_u32(sG + s * kTileBytes);
+            // the second MN atom of [g/n | w] starts at column 16 s of the shared w tile
+            const uint32_t lbo = BIDIR ? smem_u32(sW) + 32u * (uint32_t)s - aG : (uint32_t)kTileBytes;
+            const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTileBytes), kTileBytes, 1024);
+            const uint64_t dg = sdesc_sw128(aG, lbo, 1024);
+#pragma unroll
+            for (int kk = 0; kk < kRows / 16; ++kk)
+                umma_f16_ss_warp(tmem + kAccS, desc_at(dq, kk * 2048), desc_at(dg, kk * 2048), IDESC3,
+                                 (seg_start && kk == 0) ? 0u : 1u);
+            umma_commit_warp(&empty[s]);
+            if (seg_end) umma_commit_warp(accSfull);
+            if (++s == NST) { s = 0; ph ^= 1; }
         }
+        umma_commit_warp(drain2);
+        mbar_wait_slow(smem_u32(drain2), 0, nullptr, &g_tc_fault, 0x400u);
+        __syncwarp();
     } else if (warp < kQDw0) {
         // Feature-map warps (bidir): f(q) in place, one row per thread.
         if (BIDIR) {
@@ -1143,44 +1144,43 @@ bwd_kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            int s = 0, b = 0;
-            uint32_t ph = 0, bph = 0, oph = 0;
-            long long prev_h = -1;
-            for (TileCursor t(x0, nt); t.x < x1; t.next()) {
-                const long long h = t.h;
-                if (h != prev_h) {
-                    if (!LA_WAIT(opready, oph, 0x20u)) break;
-                    oph ^= 1;
-                    prev_h = h;
-                }
-                if (!LA_WAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
-                if (!LA_WAIT(&accempty[b], bph ^ 1, 0x2u)) break;
-                tc_fence_after();
-                const uint32_t da = tmem + (uint32_t)b * 128u, db = da + 64u;
-                const uint64_t dk = sdesc_sw128(smem_u32(sK + s * kTileBytes), 16, 1024);
-                const uint64_t dv = sdesc_sw128(smem_u32(sV + s * kTileBytes), 16, 1024);
-                const uint64_t dok = sdesc_sw128(smem_u32(sOp), 16, 1024);
-                const uint64_t dom = sdesc_sw128(smem_u32(sOp), OPB, 1024);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-                    for (int op = 0; op < NOPS; ++op) {
-                        umma_f16_ss(da, desc_at(dv, kk * 32), desc_at(dok, op * OPB + kk * 32), IDESC_A,
-                                    (kk | op) ? 1u : 0u);
-                        umma_f16_ss(db, desc_at(dk, kk * 32), desc_at(dom, op * OPB + kk * 2048), IDESC_B,
-                                    (kk | op) ? 1u : 0u);
-                    }
-                }
-                umma_commit(&empty[s]);
-                umma_commit(&accfull[b]);
-                b ^= 1;
-                if (b == 0) bph ^= 1;
-                if (++s == NST) { s = 0; ph ^= 1; }
+        int s = 0, b = 0;
+        uint32_t ph = 0, bph = 0, oph = 0;
+        long long prev_h = -1;
+        for (TileCursor t(x0, nt); t.x < x1; t.next()) {
+            const long long h = t.h;
+            if (h != prev_h) {
+                if (!LA_WWAIT(opready, oph, 0x20u)) break;
+                oph ^= 1;
+                prev_h = h;
             }
-            umma_commit(drain);
-            mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+            if (!LA_WWAIT(BIDIR ? &xf[s] : &full[s], ph, 0x4u)) break;
+            if (!LA_WWAIT(&accempty[b], bph ^ 1, 0x2u)) break;
+            tc_fence_after();
+            const uint32_t da = tmem + (uint32_t)b * 128u, db = da + 64u;
+            const uint64_t dk = sdesc_sw128(smem_u32(sK + s * kTileBytes), 16, 1024);
+            const uint64_t dv = sdesc_sw128(smem_u32(sV + s * kTileBytes), 16, 1024);
+            const uint64_t dok = sdesc_sw128(smem_u32(sOp), 16, 1024);
+            const uint64_t dom = sdesc_sw128(smem_u32(sOp), OPB, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                for (int op = 0; op < NOPS; ++op) {
+                    umma_f16_ss_warp(da, desc_at(dv, kk * 32), desc_at(dok, op * OPB + kk * 32), IDESC_A,
+                                     (kk | op) ? 1u : 0u);
+                    umma_f16_ss_warp(db, desc_at(dk, kk * 32), desc_at(dom, op * OPB + kk * 2048), IDESC_B,
+                                     (kk | op) ? 1u : 0u);
+                }
+            }
+            umma_commit_warp(&empty[s]);
+            umma_commit_warp(&accfull[b]);
+            b ^= 1;
+            if (b == 0) bph ^= 1;
+            if (++s == NST) { s = 0; ph ^= 1; }
         }
+        umma_commit_warp(drain);
+        mbar_wait_slow(smem_u32(drain), 0, nullptr, &g_tc_fault, 0x400u);
+        __syncwarp();
     } else if (warp < kEw0) {
         if (BIDIR) {
             const int xi = threadIdx.x - kXw0 * 32;
