@@ -16,7 +16,7 @@ bool supports(la_op op, const Shape &s, la_dtype dt) {
     case LA_OP_STATE_BWD_Q:
     case LA_OP_STATE_BWD_KV: return s.D == 64;
     case LA_OP_CHUNK_DECAY_FWD:
-    case LA_OP_CHUNK_DECAY_BWD: return dt == LA_BF16 && s.D == 128;
+    case LA_OP_CHUNK_DECAY_BWD: return dt == LA_BF16 && (s.D == 64 || s.D == 128);
     default: return false;
     }
 }

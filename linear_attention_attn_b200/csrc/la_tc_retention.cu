@@ -53,14 +53,15 @@ __device__ __forceinline__ uint8_t *align1024r(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Four 8-element chunks (4 part .. 4 part + 3 of the row's 16, across the two boxes)
-// of row `row` of a [64 x 128] tile, scaled by f, as the bf16 hi tile and (if lo_too)
-// the lo tile, lo = round(x f - hi), kTile128 bytes further.
+// NCH 8-element chunks (NCH part .. NCH part + NCH - 1 of the row's 16, across the two
+// boxes) of row `row` of a [64 x 128] tile, scaled by f, as the bf16 hi tile and (if
+// lo_too) the lo tile, lo = round(x f - hi), kTile128 bytes further.
+template <int NCH>
 static __device__ __noinline__ void scale_split_row(const uint8_t *src, uint8_t *dst, int row, int part, float f,
                                                     bool lo_too) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int ch = part * 4 + i;
+    for (int i = 0; i < NCH; ++i) {
+        const int ch = part * NCH + i;
         const int off = (ch >> 3) * kBox + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
         const uint4 u = *reinterpret_cast<const uint4 *>(src + off);
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -152,7 +153,7 @@ struct RetJobs {
 //   dS^T        M=128 N=128 K=64   A = V^T (MN-major)         B = K^ hi, lo (MN-major)
 //   O_intra^T   M=128 N=64  K=64   A = V^T (MN-major)         B = P~ hi, lo (K-major)
 //   O_inter^T   M=128 N=64  K=128  A = S^T hi, lo (tensor mem) B = Q (K-major)
-template <bool FOLD>
+template <bool FOLD, int NBOX>
 __global__ void __launch_bounds__(kRThreads, 1)
 retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int H, int BH) {
     using L = RetLayout;
@@ -160,7 +161,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
     constexpr uint32_t ID_P = idesc_f16(64, 64, true, false, false);
     constexpr uint32_t ID_OIT = idesc_f16(128, 64, true, true, false);
     constexpr uint32_t ID_OXT = idesc_f16(128, 64, true, false, false);
-    constexpr uint32_t ID_DST = idesc_f16(128, 128, true, true, true);
+    constexpr uint32_t ID_DST = idesc_f16(128, 64 * NBOX, true, true, true);   // N = the key dimensions
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024r(smem_raw);
     uint8_t *sQ = smem + L::qoff;
@@ -195,6 +196,14 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
     const CUtensorMap *tmQ = &jobs.q[pass], *tmK = &jobs.k[pass], *tmV = &jobs.v[pass], *tmO = &jobs.o[pass];
     const float gamma = dec.gamma[bh % H];
     const int nchunks = (T + kC - 1) / kC;
+    // NBOX = 1 (D = 64): one 64-column box of each tile is loaded and stored, the other is
+    // zero, so every product keeps its D = 128 shape (with K = 64 where the key dimensions
+    // are summed) and the extra dimensions contribute nothing.  q and k take the first box;
+    // v, and so the output, the second: the value dimensions (the TMEM lanes of dS^T, of the
+    // state operand and of the output) are then lanes 64..127, whose warps run on other
+    // schedulers than the TMA and UMMA-issuing warps.
+    constexpr int nbox = NBOX, D = 64 * NBOX;
+    constexpr int vbox = 2 - NBOX;             // box of v's (and o's) columns 0..63
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
@@ -235,6 +244,19 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
+    if (NBOX == 1) {
+        // the unused boxes: the second of q, k of every stage and of K^ hi, lo, the first of v
+        // (3 NST + 2 boxes of 8 KB)
+        constexpr int nz = 3 * NST + 2;
+        for (int i = threadIdx.x; i < nz * (kBox / 16); i += kRThreads) {
+            const int b = i / (kBox / 16), e = i % (kBox / 16);
+            uint8_t *base = b < 2 * NST ? smem + L::qoff + b * kTile128 + kBox
+                          : b < 3 * NST ? smem + L::qoff + b * kTile128
+                                        : sKh + (b - 3 * NST) * kTile128 + kBox;
+            *reinterpret_cast<uint4 *>(base + e * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -253,11 +275,11 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             for (int it = 0; it < nchunks; ++it) {
                 const int c = rev ? nchunks - 1 - it : it;
                 if (!LA_RWAIT(&empty[s], ph ^ 1, 0x1u)) break;
-                mbar_arrive_expect_tx(&full[s], (sonly ? 2 : 3) * kTile128);
-                for (int b = 0; b < 2; ++b) {
+                mbar_arrive_expect_tx(&full[s], (sonly ? 2 : 3) * nbox * kBox);
+                for (int b = 0; b < nbox; ++b) {
                     if (!sonly) tma_load_3d(sQ + s * kTile128 + b * kBox, tmQ, &full[s], 64 * b, c * kC, bh);
                     tma_load_3d(sK + s * kTile128 + b * kBox, tmK, &full[s], 64 * b, c * kC, bh);
-                    tma_load_3d(sV + s * kTile128 + b * kBox, tmV, &full[s], 64 * b, c * kC, bh);
+                    tma_load_3d(sV + s * kTile128 + (b + vbox) * kBox, tmV, &full[s], 64 * b, c * kC, bh);
                 }
                 ++issued;
                 if (++s == NST) { s = 0; ph ^= 1; }
@@ -276,7 +298,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             const uint64_t dq = sdesc_sw128(smem_u32(sQ + sp * kTile128), 16, 1024);
             const uint64_t dk = sdesc_sw128(smem_u32(sK + sp * kTile128), 16, 1024);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
+            for (int kk = 0; kk < 4 * NBOX; ++kk) {   // K = the key dimensions
                 const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
                 umma_f16_ss_warp(tmem + cP + 64u * (uint32_t)(c & 1), desc_at(dq, off), desc_at(dk, off), ID_P,
                                  kk ? 1u : 0u);
@@ -357,7 +379,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             tc_fence_after();
             const uint64_t dq = sdesc_sw128(smem_u32(sQ + s * kTile128), 16, 1024);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
+            for (int kk = 0; kk < 4 * NBOX; ++kk) {   // K = the key dimensions
                 const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
 #pragma unroll
                 for (int op = 0; op < 2; ++op)
@@ -486,33 +508,40 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             fence_async_smem();
             named_bar(1, kROWarps * 32);
             if (ot == 0 && live) {
-                tma_store_3d(tmO, sO, 0, c * kC, bh);
-                tma_store_3d(tmO, sO + kBox, 64, c * kC, bh);
+                tma_store_3d(tmO, sO + vbox * kBox, 0, c * kC, bh);
+                if (NBOX == 2) tma_store_3d(tmO, sO + kBox, 64, c * kC, bh);
                 tma_store_commit();
             }
         }
         if (ot == 0) tma_store_wait_all<0>();
     } else {
         // State warps: S^T_{c+1} = gamma^C S^T_c + dS^T_c in fp32 registers; thread (d, half)
-        // holds row d of S^T (column d of S), entries 64 half .. 64 half + 63 (its TMEM lane
-        // of dS^T), and writes them as the bf16 hi + lo A operand of O_inter^T.
+        // holds row d of S^T (column d of S), entries SC half .. SC half + SC - 1 (its TMEM
+        // lane of dS^T), and writes them as the bf16 hi + lo A operand of O_inter^T.  D = 128:
+        // SC = 64.  D = 64: the value dimensions sit in lanes 64..127 (d = 64 + value index),
+        // whose rows split their 64 entries (SC = 32); the warps of lanes 0..63, which would
+        // hold zeros, only keep the barriers' counts.
+        constexpr int SC = 64 / (3 - NBOX);
         const int sub = warp & 3, half = (warp - kRSw0) >> 2;
         const uint32_t lanes = (uint32_t)(32 * sub) << 16;
         const int d = 32 * sub + lane;
+        const bool sact = NBOX == 2 || sub >= 2;
+        const int dv = d - 64 * vbox;          // the value dimension of lane d
+        const int col0 = SC * half;
         const float gC = GP(kC);
         const float gm = FOLD ? GP(kM) : 1.f;   // the state operand holds gamma^m S (FOLD)
         // decay over the partial chunk at the end of the sequence: the last chunk
         // forwards, the first one backwards
         const float gLast = GP(min(kC, T - (nchunks - 1) * kC));
-        float st[64];
+        float st[SC];
         const float *sin = jobs.sin[pass];
         float *sout = jobs.sout[pass];
-        const long long sbase = (long long)bh * 128 * 128;
-        if (sin) {
-            if (jobs.sin_t[pass]) {   // sin holds S^T: row d, entries 64 half ..
+        const long long sbase = (long long)bh * D * D;
+        if (sin && sact) {
+            if (jobs.sin_t[pass]) {   // sin holds S^T: row d, entries col0 ..
 #pragma unroll
-                for (int c4 = 0; c4 < 16; ++c4) {
-                    const float4 x = *reinterpret_cast<const float4 *>(sin + sbase + (long long)d * 128 + 64 * half + 4 * c4);
+                for (int c4 = 0; c4 < SC / 4; ++c4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(sin + sbase + (long long)dv * D + col0 + 4 * c4);
                     st[4 * c4] = x.x;
                     st[4 * c4 + 1] = x.y;
                     st[4 * c4 + 2] = x.z;
@@ -520,17 +549,18 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                 }
             } else {                  // sin holds S: column d (lanes read consecutive d)
 #pragma unroll
-                for (int c = 0; c < 64; ++c) st[c] = sin[sbase + (long long)(64 * half + c) * 128 + d];
+                for (int c = 0; c < SC; ++c) st[c] = sin[sbase + (long long)(col0 + c) * D + dv];
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) st[i] = 0.f;
+            for (int i = 0; i < SC; ++i) st[i] = 0.f;
         }
-        // The state operand: this thread's 64 entries as 32 packed columns of its lane,
-        // hi at cSA + 32 half, lo 64 columns further, in four rounds of 8 columns.
+        // The state operand: this thread's SC entries as SC / 2 packed columns of its lane,
+        // hi at cSA + col0 / 2, lo 64 columns further, in rounds of 8 columns.
         auto write_state = [&]() {
+            if (sact) {
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
+            for (int r = 0; r < SC / 16; ++r) {
                 uint32_t hw[8], lw[8];
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {
@@ -539,19 +569,21 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                     const float2 hv = h2<true>::to_f2(hw[m]);
                     lw[m] = h2<true>::from_f2(a - hv.x, b - hv.y);
                 }
-                tmem_st8(tmem + cSA + lanes + 32 * half + 8 * r, hw);
-                tmem_st8(tmem + cSA + 64 + lanes + 32 * half + 8 * r, lw);
+                tmem_st8(tmem + cSA + lanes + col0 / 2 + 8 * r, hw);
+                tmem_st8(tmem + cSA + 64 + lanes + col0 / 2 + 8 * r, lw);
             }
             tmem_st_wait();
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sready);
         };
         if (!sonly) write_state();                         // S_0
         // K^ = diag(gamma^(C-1-j)) K of chunk iteration itk as hi + lo: thread kt takes row
-        // kt % 64 and the 8-element chunks 4 (kt / 64) .. + 3 of the row's 16.  Forwards in
-        // time the weights count back from the chunk's last valid row, so that the state
-        // after a partial last chunk is the state after token T - 1.
+        // kt % 64 and the 8-element chunks 2 NBOX (kt / 64) .. + 2 NBOX - 1 of the row's 16
+        // (with D = 64 the first box only).  Forwards in time the weights count back from the
+        // chunk's last valid row, so that the state after a partial last chunk is the state
+        // after token T - 1.
         const int kt = threadIdx.x - kRSw0 * 32;
         const int krow = kt & 63, kpart = kt >> 6;
         auto build_khat = [&](int itk) -> bool {
@@ -559,7 +591,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             if (!__all_sync(0xffffffffu, LA_RWAIT(&full[sk], (uint32_t)((itk / NST) & 1), 0x100u))) return false;
             const int rows = min(kC, T - (rev ? nchunks - 1 - itk : itk) * kC);
             const float f = rev ? GP(krow) : (krow < rows ? GP(rows - 1 - krow) : 0.f);
-            scale_split_row(sK + sk * kTile128, sKh, krow, kpart, f, true);
+            scale_split_row<2 * NBOX>(sK + sk * kTile128, sKh, krow, kpart, f, true);
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(khready);
@@ -571,14 +603,16 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             if (!__all_sync(0xffffffffu, LA_RWAIT(dsfull, pc, 0x1000u))) break;
             __syncwarp();   // converged for the .sync.aligned TMEM loads
             tc_fence_after();
-            const uint32_t base = tmem + cDS + lanes + 64u * half;
+            const uint32_t base = tmem + cDS + lanes + (uint32_t)col0;
             const float g = (it == (rev ? 0 : nchunks - 1)) ? gLast : gC;
+            if (sact) {
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c4 = 0; c4 < SC / 16; ++c4) {
                 float a[16];
                 tmem_ld16_sync(base + 16 * c4, a);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) st[16 * c4 + i] = fmaf(g, st[16 * c4 + i], a[i]);
+            }
             }
             tc_fence_before();
             __syncwarp();
@@ -592,9 +626,9 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             tc_fence_after();
             write_state();
         }
-        if (sout && !*s_abort) {   // S after the last chunk: column d of S, lanes write consecutive d
+        if (sout && sact && !*s_abort) {   // S after the last chunk: column d of S, lanes write consecutive d
 #pragma unroll
-            for (int c = 0; c < 64; ++c) sout[sbase + (long long)(64 * half + c) * 128 + d] = st[c];
+            for (int c = 0; c < SC; ++c) sout[sbase + (long long)(col0 + c) * D + dv] = st[c];
         }
     }
     tc_fence_before();
@@ -621,6 +655,22 @@ static bool fold_ok(const DecayArgs &dec, int H) {
     } while (0)
 #endif
 
+// One launch of `passes` x BH CTAs: the folded kernel when every decay allows it (launch
+// name `folded`), else the one with two output accumulators (`unfolded`); D = 64 or 128.
+static la_status launch_retention(const char *folded, const char *unfolded, int passes, const RetJobs &jobs,
+                                  const DecayArgs &dec, const Shape &s, cudaStream_t st) {
+    const dim3 grid((unsigned)(passes * s.BH())), block(kRThreads);
+    const size_t smem = (size_t)RetLayout::bytes;
+    const bool fold = fold_ok(dec, s.H);
+    if (s.D == 64)
+        return fold ? launch_pdl(folded, retention_kernel<true, 1>, grid, block, smem, st, jobs, dec, s.T, s.H, (int)s.BH())
+                    : launch_pdl(unfolded, retention_kernel<false, 1>, grid, block, smem, st, jobs, dec, s.T, s.H,
+                                 (int)s.BH());
+    return fold ? launch_pdl(folded, retention_kernel<true, 2>, grid, block, smem, st, jobs, dec, s.T, s.H, (int)s.BH())
+                : launch_pdl(unfolded, retention_kernel<false, 2>, grid, block, smem, st, jobs, dec, s.T, s.H,
+                             (int)s.BH());
+}
+
 }  // namespace
 
 la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
@@ -634,12 +684,8 @@ la_status retention_fwd(const void *q, const void *k, const void *v, void *o, co
     LA_TRY(retention_map(&jobs.k[0], k, s));
     LA_TRY(retention_map(&jobs.v[0], v, s));
     LA_TRY(retention_map(&jobs.o[0], o ? o : k, s));
-    const char *name = o ? "tc_retention_fwd" : "tc_retention_state";
-    if (fold_ok(dec, s.H))
-        return launch_pdl(name, retention_kernel<true>, dim3((unsigned)s.BH()), dim3(kRThreads),
-                          (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
-    return launch_pdl("tc_retention_fwd_unfolded", retention_kernel<false>, dim3((unsigned)s.BH()), dim3(kRThreads),
-                      (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
+    return o ? launch_retention("tc_retention_fwd", "tc_retention_fwd_unfolded", 1, jobs, dec, s, st)
+             : launch_retention("tc_retention_state", "tc_retention_state_unfolded", 1, jobs, dec, s, st);
 }
 
 la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin,
@@ -661,11 +707,7 @@ la_status retention_bwd(const void *q, const void *k, const void *v, const void 
         LA_TRY(retention_map(&jobs.k[0], q, s));
         LA_TRY(retention_map(&jobs.v[0], g, s));
         LA_TRY(retention_map(&jobs.o[0], q, s));
-        if (fold_ok(dec, s.H))
-            return launch_pdl("tc_retention_state", retention_kernel<true>, dim3((unsigned)s.BH()), dim3(kRThreads),
-                              (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
-        return launch_pdl("tc_retention_state_unfolded", retention_kernel<false>, dim3((unsigned)s.BH()),
-                          dim3(kRThreads), (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
+        return launch_retention("tc_retention_state", "tc_retention_state_unfolded", 1, jobs, dec, s, st);
     }
     struct Pass {
         const void *q, *k, *v;
@@ -689,11 +731,7 @@ la_status retention_bwd(const void *q, const void *k, const void *v, const void 
         jobs.sin_t[np] = all[p].sin_t;
         jobs.sout[np] = all[p].sout;
     }
-    if (fold_ok(dec, s.H))
-        return launch_pdl("tc_retention_bwd", retention_kernel<true>, dim3((unsigned)(np * s.BH())), dim3(kRThreads),
-                          (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
-    return launch_pdl("tc_retention_bwd_unfolded", retention_kernel<false>, dim3((unsigned)(np * s.BH())),
-                      dim3(kRThreads), (size_t)RetLayout::bytes, st, jobs, dec, s.T, s.H, (int)s.BH());
+    return launch_retention("tc_retention_bwd", "tc_retention_bwd_unfolded", np, jobs, dec, s, st);
 }
 
 unsigned int read_and_clear_retention_fault() {

@@ -49,7 +49,7 @@ def test_backward_of_a_segment(dtype, D, T):
     assert _rel_l2(rout.cpu().numpy(), ref[3]) <= STATE_REL_L2
 
 
-@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f32", 64)])
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("bf16", 64), ("f32", 64)])
 def test_segments_chained_forwards_and_backwards(dtype, D):
     """One sequence of 700 tokens cut at 257 and 513: the forward hands S from segment to segment,
     the backward runs last segment first and hands R back; the concatenated outputs and gradients
@@ -200,11 +200,12 @@ def test_sequence_split_across_emulated_ranks(dtype, D):
         pu.assert_grad(got, whole[j], "emulated ranks %s" % name)
 
 
-@pytest.mark.parametrize("dtype,D,T", [("bf16", 128, 300), ("bf16", 128, 37), ("f32", 64, 300), ("f16", 128, 129)])
+@pytest.mark.parametrize("dtype,D,T", [("bf16", 128, 300), ("bf16", 128, 37), ("bf16", 64, 300), ("f32", 64, 300),
+                                       ("f16", 128, 129)])
 def test_state_only_passes(dtype, D, T):
     """The state-only forms (o None; dq, dk, dv None) give exactly the states of the whole passes
     (the same arithmetic computes them) and the oracle's; q and o, resp. k, v, dq, dk and dv are
-    not needed.  bf16 D = 128 runs on the tensor cores, the rest on the CUDA cores."""
+    not needed.  bf16 (D = 64 and 128) runs on the tensor cores, the rest on the CUDA cores."""
     import linear_attention_attn_b200 as la
     w = synth.Workload("case", "retention", 2, 3, T, D, dtype, q_scale=D ** -0.5)
     inp = synth.make_inputs(w, seed=25, with_grad=True)
