@@ -135,8 +135,17 @@ def measured_peaks():
 
 # The files the tensor-core kernels are compiled from (their launch code included): a change
 # anywhere else in the library leaves those kernels, and their DRAM traffic, as they were.
-TC_SOURCES = ("la_tc.cu", "la_tc.cuh", "la_tc_state.cu", "la_tc_retention.cu", "la_tc_common.cuh", "la_tc_ptx.cuh",
-              "la_internal.cuh")
+# The files each family of tensor-core kernels is compiled from (with include/la.h): a
+# committed ncu capture stands for a kernel only while its family's files are unchanged.
+TC_SOURCES = {
+    "state": ("la_tc.cuh", "la_tc_state.cu", "la_tc_common.cuh", "la_tc_ptx.cuh", "la_internal.cuh"),
+    "retention": ("la_tc.cuh", "la_tc_retention.cu", "la_tc_common.cuh", "la_tc_ptx.cuh", "la_internal.cuh"),
+}
+
+
+def kernel_sources(kernel: str):
+    """The source files of the tensor-core kernel launched under `kernel`."""
+    return TC_SOURCES["retention" if kernel.startswith("tc_retention") else "state"]
 
 
 def source_hash(names=None) -> str:
@@ -153,10 +162,10 @@ def source_hash(names=None) -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str, T: int):
-    """DRAM bytes per launch of `kernel` at sequence length T from the committed ncu summaries:
-    of the captures taken on the current kernel sources, the one whose T is nearest, scaled by T
-    (None when no capture matches the sources)."""
+def ncu_traffic(kernel: str, T: int, B: int, H: int, D: int):
+    """DRAM bytes per launch of `kernel` at [B, H, T, D] from the committed ncu summaries: of the
+    captures taken on the current kernel sources at the same B, H and D, the one whose T is
+    nearest, scaled by T (None when no capture matches)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
@@ -166,8 +175,8 @@ def ncu_traffic(kernel: str, T: int):
     entries = rec.get(kernel) or []
     if isinstance(entries, dict):
         entries = [entries]
-    sha = source_hash(TC_SOURCES)
-    ok = [e for e in entries if e.get("source_sha") == sha]
+    sha = source_hash(kernel_sources(kernel))
+    ok = [e for e in entries if e.get("source_sha") == sha and (e.get("B"), e.get("H"), e.get("D")) == (B, H, D)]
     if not ok:
         return None
     e = min(ok, key=lambda e: abs(math.log(float(e["T"]) / T)))
@@ -344,6 +353,8 @@ WORKLOAD_TEXT = {
               "q,k ~ N(0,1) D^-1/2, v, dO ~ N(0,1)",
     "retention": "chunked causal decay (retention) fwd+bwd, bf16 storage / fp32 accumulate, B=%d H=%d T=%d D=%d, "
                  "gamma_h = 1 - 2^(-5-7h/(H-1)), q ~ N(0,1) D^-1/2, k, v, dO ~ N(0,1)",
+    "causal": "plain causal linear attention fwd+bwd (the decay op with gamma = 1 on every head: no feature map, "
+              "no norm term), bf16 storage / fp32 accumulate, B=%d H=%d T=%d D=%d, q ~ N(0,1) D^-1/2, k, v, dO ~ N(0,1)",
     "gated": "gated linear attention fwd+bwd (recurrent form in 256-token chunks on CUDA cores), bf16 storage / "
              "fp32 accumulate, "
              "B=%d H=%d T=%d D=%d, log gates log(sigmoid(N(0,1)))/16 per token and key dimension, "
@@ -360,7 +371,8 @@ WORKLOAD_TEXT = {
 
 def config_of(w, args):
     step_bytes = 11 * w.B * w.H * w.T * w.D * 2
-    return {"workload": WORKLOAD_TEXT[w.op] % (w.B, w.H, w.T, w.D),
+    kind = "causal" if w.name == "causal_bf16" else w.op
+    return {"workload": WORKLOAD_TEXT[kind] % (w.B, w.H, w.T, w.D),
             "B": w.B, "H": w.H, "T": w.T, "D": w.D, "global_batch": w.B * max(1, args.gpus), "seq_len": w.T,
             "parallelism": "dp%d (independent batches, no collective)" % max(1, args.gpus),
             "l2": "inputs larger than L2: %.0f MB of algorithmic traffic per step vs 126 MB L2, no flush"
@@ -424,6 +436,7 @@ def time_each(fn, steps, warmup, stream, flush=None):
 # norm and gated ops at the headline shape.  (workload, T values, forward only)
 CONFIG_RECORDS = (("simple_bf16", (128, 1024, 4096, 16384), False),
                   ("retention_bf16", (2048, 8192), False),
+                  ("causal_bf16", (4096,), False),
                   ("vision_f16", (65536,), True),
                   ("causal_norm_f16", (4096,), False),
                   ("gated_bf16", (4096,), False))
@@ -500,7 +513,8 @@ def config_records(la, dev, stream):
             recs.append(rec)
             del q, k, v, g, o, dq, dk, dv, st, ws, lg, dg
             torch.cuda.empty_cache()
-        out[base] = {"workload": WORKLOAD_TEXT[synth.WORKLOADS[base].op if base != "vision_f16" else "vision"]
+        kind = {"vision_f16": "vision", "causal_bf16": "causal"}.get(base, synth.WORKLOADS[base].op)
+        out[base] = {"workload": WORKLOAD_TEXT[kind]
                      % (synth.WORKLOADS[base].B, synth.WORKLOADS[base].H, Ts[-1], synth.WORKLOADS[base].D),
                      "step": "fwd" if fwd_only else "fwd+bwd", "peak_gbs": peak, "peak_source": peak_kind,
                      "records": recs}
@@ -709,7 +723,7 @@ def run_ours(args, w):
             alg_bytes = KERNEL_TENSORS[name] * tensor_bytes
             avg_s = tot_ms / n_launch / 1e3
             achieved = alg_bytes / avg_s / 1e9
-            traffic = ncu_traffic(name, T)
+            traffic = ncu_traffic(name, T, B, H, D)
             roof = {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak, "peak_source": peak_kind, "traffic": traffic,
                     "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_ms": tot_ms / n_launch,
@@ -765,7 +779,8 @@ def run_ours(args, w):
         vs = value / page_rate
 
     line = {
-        "metric": METRIC if w.op == "bidir" else "%s fwd+bwd tokens/s" % w.op, "value": value, "unit": UNIT,
+        "metric": METRIC if w.op == "bidir" else "%s fwd+bwd tokens/s" % ("causal" if w.name == "causal_bf16" else w.op),
+        "value": value, "unit": UNIT,
         "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "strong" if seqpar else "weak",
@@ -942,7 +957,7 @@ def main(argv=None):
                          "the oracle arm: 200)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--T", type=int, default=None, help="sequence length (default: the workload's)")
-    ap.add_argument("--workload", choices=["bidir", "simple", "retention", "decode", "causal_norm", "gated"],
+    ap.add_argument("--workload", choices=["bidir", "simple", "retention", "causal", "decode", "causal_norm", "gated"],
                     default="bidir",
                     help="bidir (the benchmark metric, B8 H16 D64 fp16), simple (B8 H16 D64 bf16), "
                          "retention (B8 H32 D128 bf16), decode (recurrent decay step, B64 H32 D128) or "
@@ -967,7 +982,7 @@ def main(argv=None):
                 args.steps = 200
             return run_decode_reference(args)
         return run_decode(args)
-    base = {"bidir": "bidir_f16", "simple": "simple_bf16", "retention": "retention_bf16",
+    base = {"bidir": "bidir_f16", "simple": "simple_bf16", "retention": "retention_bf16", "causal": "causal_bf16",
             "causal_norm": "causal_norm_f16", "gated": "gated_bf16"}[args.workload]
     w = synth.WORKLOADS[base]
     w = w.with_T(args.T if args.T is not None else (4096 if args.workload != "retention" else 8192))

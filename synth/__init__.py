@@ -41,12 +41,12 @@ class Workload:
 
     def with_T(self, T: int) -> "Workload":
         return Workload(self.name, self.op, self.B, self.H, T, self.D, self.dtype, self.eps,
-                        self.q_scale, self.k_scale, self.v_scale, self.vision_offset, self.bwd)
+                        self.q_scale, self.k_scale, self.v_scale, self.vision_offset, self.bwd, dict(self.extra))
 
     def with_shape(self, B=None, H=None, T=None, D=None) -> "Workload":
         return Workload(self.name, self.op, B or self.B, H or self.H, T if T is not None else self.T,
                         D or self.D, self.dtype, self.eps, self.q_scale, self.k_scale, self.v_scale,
-                        self.vision_offset, self.bwd)
+                        self.vision_offset, self.bwd, dict(self.extra))
 
 
 # The five workloads the library is specified against.
@@ -62,6 +62,10 @@ WORKLOADS = {
     # retention, bf16, q scaled by D^-1/2 (T swept 128 .. 8192)
     "retention_bf16": Workload("retention_bf16", "retention", 8, 32, 2048, 128, "bf16",
                                q_scale=128 ** -0.5),
+    # plain causal linear attention (the decay op with gamma = 1 on every head, no feature map,
+    # no norm term), bf16, q scaled by D^-1/2, at the shape of the other causal workloads
+    "causal_bf16": Workload("causal_bf16", "retention", 8, 16, 4096, 64, "bf16", q_scale=64 ** -0.5,
+                            extra={"gamma": 1.0}),
     # causal linear attention with the norm term (phi = elu+1, no decay), the bidir recipe and shape
     "causal_norm_f16": Workload("causal_norm_f16", "causal_norm", 8, 16, 4096, 64, "f16",
                                 q_scale=0.5, k_scale=0.5, v_scale=0.5),
@@ -126,7 +130,8 @@ def make_inputs(w: Workload, seed: int = 0, with_grad: bool | None = None) -> di
             x = x + off
         out[n] = x.to(dt).contiguous()
     if w.op == "retention":
-        out["gamma"] = retention_gammas(w.H)
+        g = w.extra.get("gamma")
+        out["gamma"] = retention_gammas(w.H) if g is None else torch.full((w.H,), float(g), dtype=torch.float32)
     if w.op == "gated":
         out["g"] = (torch.nn.functional.logsigmoid(normal(shape, seed, 4)) / 16.0).to(dt).contiguous()
     return out
