@@ -16,7 +16,7 @@ bool supports(la_op op, const Shape &s, la_dtype dt) {
     case LA_OP_STATE_BWD_Q:
     case LA_OP_STATE_BWD_KV: return s.D == 64;
     case LA_OP_CHUNK_DECAY_FWD:
-    case LA_OP_CHUNK_DECAY_BWD: return dt == LA_BF16 && (s.D == 64 || s.D == 128);
+    case LA_OP_CHUNK_DECAY_BWD: return s.D == 64 || s.D == 128;
     default: return false;
     }
 }
@@ -41,13 +41,13 @@ size_t workspace_size(la_op op, const Shape &s, la_dtype) {
 }
 
 la_status decay_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
-                    const DecayArgs &dec, const Shape &s, la_dtype, void *, cudaStream_t st) {
-    return retention_fwd(q, k, v, o, sin, sout, dec, s, st);
+                    const DecayArgs &dec, const Shape &s, la_dtype dt, void *, cudaStream_t st) {
+    return retention_fwd(q, k, v, o, sin, sout, dec, s, dt == LA_BF16, st);
 }
 la_status decay_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin, const float *rin,
-                    float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv, const Shape &s, la_dtype, void *,
-                    cudaStream_t st) {
-    return retention_bwd(q, k, v, g, sin, rin, rout, dec, dq, dk, dv, s, st);
+                    float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv, const Shape &s, la_dtype dt,
+                    void *, cudaStream_t st) {
+    return retention_bwd(q, k, v, g, sin, rin, rout, dec, dq, dk, dv, s, dt == LA_BF16, st);
 }
 
 }  // namespace tc

@@ -20,15 +20,15 @@ unsigned int read_and_clear_debug_fault();
 
 // [BH, T, D] 16-bit tensor map: boxes of box_rows x 64 columns, 128-byte swizzle.
 la_status make_tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16, int box_rows);
-la_status retention_map(CUtensorMap *m, const void *ptr, const Shape &s);
-// Chunked causal decay forward on tensor cores (bf16, D = 128).
+la_status retention_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16);
+// Chunked causal decay forward on tensor cores (bf16 or fp16 storage, D = 64 or 128).
 la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
-                        const DecayArgs &dec, const Shape &s, cudaStream_t st);
+                        const DecayArgs &dec, const Shape &s, bool bf16, cudaStream_t st);
 // sin: state S entering the segment (or null); rin: R = sum_{t >= end} gamma^(t-end) q_t^T dO_t
 // entering from the right (or null); rout: R at the segment's first row (or null).  [BH, D, D].
 la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin,
                         const float *rin, float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv,
-                        const Shape &s, cudaStream_t st);
+                        const Shape &s, bool bf16, cudaStream_t st);
 la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, void *o, float *state,
                     const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
 la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, const void *g,

@@ -401,14 +401,15 @@ __device__ __forceinline__ float stage_absmax(const float *stage, int tid) {
     return m;
 }
 
-// Two-term bf16 split of 16 fp32 values, packed in pairs: hi = round(x),
+// Two-term 16-bit split (bf16 or fp16) of 16 fp32 values, packed in pairs: hi = round(x),
 // lo = round(x - hi) (x - hi is exact in fp32).
+template <bool BF16 = true>
 __device__ __forceinline__ void split_hi_lo16_packed(const float (&x)[16], uint32_t (&hw)[8], uint32_t (&lw)[8]) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-        hw[k] = h2<true>::from_f2(x[2 * k], x[2 * k + 1]);
-        const float2 hv = h2<true>::to_f2(hw[k]);
-        lw[k] = h2<true>::from_f2(x[2 * k] - hv.x, x[2 * k + 1] - hv.y);
+        hw[k] = h2<BF16>::from_f2(x[2 * k], x[2 * k + 1]);
+        const float2 hv = h2<BF16>::to_f2(hw[k]);
+        lw[k] = h2<BF16>::from_f2(x[2 * k] - hv.x, x[2 * k + 1] - hv.y);
     }
 }
 

@@ -1,5 +1,6 @@
 // la_tc_retention.cu -- tensor-core kernel of causal linear attention with a per-head
-// scalar decay (retention), forward, bf16 storage, D = 128, fp32 accumulation.
+// scalar decay (retention), forward and backward, bf16 or fp16 storage, D = 64 or 128,
+// fp32 accumulation.
 //
 // "flash-linear-attention" README, "Benchmarks" (RetNet) and "Different forms of
 // linear attention" (FusedChunk: chunkwise, the inter-chunk state kept on chip,
@@ -56,7 +57,7 @@ __device__ __forceinline__ uint8_t *align1024r(uint8_t *p) {
 // NCH 8-element chunks (NCH part .. NCH part + NCH - 1 of the row's 16, across the two
 // boxes) of row `row` of a [64 x 128] tile, scaled by f, as the bf16 hi tile and (if
 // lo_too) the lo tile, lo = round(x f - hi), kTile128 bytes further.
-template <int NCH>
+template <int NCH, bool BF>
 static __device__ __noinline__ void scale_split_row(const uint8_t *src, uint8_t *dst, int row, int part, float f,
                                                     bool lo_too) {
 #pragma unroll
@@ -68,11 +69,11 @@ static __device__ __noinline__ void scale_split_row(const uint8_t *src, uint8_t 
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const float2 x = h2<true>::to_f2(w[k]);
+            const float2 x = h2<BF>::to_f2(w[k]);
             const float a = x.x * f, b = x.y * f;
-            hi[k] = h2<true>::from_f2(a, b);
-            const float2 hv = h2<true>::to_f2(hi[k]);
-            lo[k] = h2<true>::from_f2(a - hv.x, b - hv.y);
+            hi[k] = h2<BF>::from_f2(a, b);
+            const float2 hv = h2<BF>::to_f2(hi[k]);
+            lo[k] = h2<BF>::from_f2(a - hv.x, b - hv.y);
         }
         *reinterpret_cast<uint4 *>(dst + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         if (lo_too) *reinterpret_cast<uint4 *>(dst + kTile128 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
@@ -140,8 +141,9 @@ struct RetJobs {
 //   w'_ij = w_ij gamma^m / g_i = gamma^(m-1-j) (j <= i)   [backwards gamma^(j+m-rows), j >= i],
 // so the state operand is written as gamma^m S and the epilogue multiplies row i by
 // f_i.  Every factor lies within gamma^(+-64) of 1, which stays far inside the fp32 and
-// bf16 ranges for gamma >= 1/8; smaller decays use FOLD = false, where O_intra^T and
-// O_inter^T keep accumulators of their own and the epilogue forms O_intra + g_i O_inter.
+// bf16 ranges for gamma >= 1/8 (fp16: gamma >= 0.9, see fold_ok); smaller decays use
+// FOLD = false, where O_intra^T and O_inter^T keep accumulators of their own and the
+// epilogue forms O_intra + g_i O_inter.
 //
 // Per chunk c the UMMAs are issued in the order P(c + 1), dS^T(c), O_intra^T(c),
 // O_inter^T(c): P of the next chunk goes to the other P buffer as soon as its data has
@@ -153,15 +155,15 @@ struct RetJobs {
 //   dS^T        M=128 N=128 K=64   A = V^T (MN-major)         B = K^ hi, lo (MN-major)
 //   O_intra^T   M=128 N=64  K=64   A = V^T (MN-major)         B = P~ hi, lo (K-major)
 //   O_inter^T   M=128 N=64  K=128  A = S^T hi, lo (tensor mem) B = Q (K-major)
-template <bool FOLD, int NBOX>
+template <bool FOLD, int NBOX, bool BF>
 __global__ void __launch_bounds__(kRThreads, 1)
 retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int H, int BH) {
     using L = RetLayout;
     constexpr int NST = L::NST;
-    constexpr uint32_t ID_P = idesc_f16(64, 64, true, false, false);
-    constexpr uint32_t ID_OIT = idesc_f16(128, 64, true, true, false);
-    constexpr uint32_t ID_OXT = idesc_f16(128, 64, true, false, false);
-    constexpr uint32_t ID_DST = idesc_f16(128, 64 * NBOX, true, true, true);   // N = the key dimensions
+    constexpr uint32_t ID_P = idesc_f16(64, 64, BF, false, false);
+    constexpr uint32_t ID_OIT = idesc_f16(128, 64, BF, true, false);
+    constexpr uint32_t ID_OXT = idesc_f16(128, 64, BF, false, false);
+    constexpr uint32_t ID_DST = idesc_f16(128, 64 * NBOX, BF, true, true);   // N = the key dimensions
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024r(smem_raw);
     uint8_t *sQ = smem + L::qoff;
@@ -422,7 +424,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                     x[e] = dlt >= 0 ? x[e] * wgt : 0.f;
                 }
                 uint32_t hw[8], lw[8];
-                split_hi_lo16_packed(x, hw, lw);
+                split_hi_lo16_packed<BF>(x, hw, lw);
                 store_chunk16_packed(sPt, ri, c16, hw);
                 store_chunk16_packed(sPt + kBox, ri, c16, lw);
             }
@@ -500,8 +502,8 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                         const int dch = dbase + ((mk & 1) ? 8 : 0);
                         const uint32_t sa = smem_u32(sO + (dch >> 6) * kBox + row * 128 +
                                                      ((((dch & 63) >> 3) ^ (row & 7)) << 4));
-                        stmatrix_x4_trans(sa, h2<true>::from_f2(y[0], y[1]), h2<true>::from_f2(y[2], y[3]),
-                                          h2<true>::from_f2(y[4], y[5]), h2<true>::from_f2(y[6], y[7]));
+                        stmatrix_x4_trans(sa, h2<BF>::from_f2(y[0], y[1]), h2<BF>::from_f2(y[2], y[3]),
+                                          h2<BF>::from_f2(y[4], y[5]), h2<BF>::from_f2(y[6], y[7]));
                     }
                 }
             }
@@ -565,9 +567,9 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {
                     const float a = gm * st[16 * r + 2 * m], b = gm * st[16 * r + 2 * m + 1];
-                    hw[m] = h2<true>::from_f2(a, b);
-                    const float2 hv = h2<true>::to_f2(hw[m]);
-                    lw[m] = h2<true>::from_f2(a - hv.x, b - hv.y);
+                    hw[m] = h2<BF>::from_f2(a, b);
+                    const float2 hv = h2<BF>::to_f2(hw[m]);
+                    lw[m] = h2<BF>::from_f2(a - hv.x, b - hv.y);
                 }
                 tmem_st8(tmem + cSA + lanes + col0 / 2 + 8 * r, hw);
                 tmem_st8(tmem + cSA + 64 + lanes + col0 / 2 + 8 * r, lw);
@@ -591,7 +593,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             if (!__all_sync(0xffffffffu, LA_RWAIT(&full[sk], (uint32_t)((itk / NST) & 1), 0x100u))) return false;
             const int rows = min(kC, T - (rev ? nchunks - 1 - itk : itk) * kC);
             const float f = rev ? GP(krow) : (krow < rows ? GP(rows - 1 - krow) : 0.f);
-            scale_split_row<2 * NBOX>(sK + sk * kTile128, sKh, krow, kpart, f, true);
+            scale_split_row<2 * NBOX, BF>(sK + sk * kTile128, sKh, krow, kpart, f, true);
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(khready);
@@ -640,10 +642,14 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
 #undef GP
 }
 
-// The folded output needs every factor gamma^k, |k| <= 64, well inside the fp32 range.
-static bool fold_ok(const DecayArgs &dec, int H) {
+// The folded output stores the masked products scaled by gamma^(m-1-j) (up to gamma^-32) and the
+// state operand as gamma^m S (gamma^32) in the 16-bit type: bf16 has the fp32 exponent range,
+// which gamma >= 1/8 keeps them far inside; fp16 (largest value 65504, smallest normal 6.1e-5)
+// takes the fold only for gamma >= 0.9 (factors within 29 and 1/29 of 1).
+static bool fold_ok(const DecayArgs &dec, int H, bool bf16) {
+    const float lo = bf16 ? 0.125f : 0.9f;
     for (int h = 0; h < H; ++h)
-        if (!(dec.gamma[h] >= 0.125f)) return false;
+        if (!(dec.gamma[h] >= lo)) return false;
     return true;
 }
 
@@ -657,40 +663,47 @@ static bool fold_ok(const DecayArgs &dec, int H) {
 
 // One launch of `passes` x BH CTAs: the folded kernel when every decay allows it (launch
 // name `folded`), else the one with two output accumulators (`unfolded`); D = 64 or 128.
-static la_status launch_retention(const char *folded, const char *unfolded, int passes, const RetJobs &jobs,
-                                  const DecayArgs &dec, const Shape &s, cudaStream_t st) {
+template <int NBOX, bool BF>
+static la_status launch_retention_t(const char *folded, const char *unfolded, int passes, const RetJobs &jobs,
+                                    const DecayArgs &dec, const Shape &s, cudaStream_t st) {
     const dim3 grid((unsigned)(passes * s.BH())), block(kRThreads);
     const size_t smem = (size_t)RetLayout::bytes;
-    const bool fold = fold_ok(dec, s.H);
+    return fold_ok(dec, s.H, BF)
+               ? launch_pdl(folded, retention_kernel<true, NBOX, BF>, grid, block, smem, st, jobs, dec, s.T, s.H,
+                            (int)s.BH())
+               : launch_pdl(unfolded, retention_kernel<false, NBOX, BF>, grid, block, smem, st, jobs, dec, s.T, s.H,
+                            (int)s.BH());
+}
+
+static la_status launch_retention(const char *folded, const char *unfolded, int passes, const RetJobs &jobs,
+                                  const DecayArgs &dec, const Shape &s, bool bf16, cudaStream_t st) {
     if (s.D == 64)
-        return fold ? launch_pdl(folded, retention_kernel<true, 1>, grid, block, smem, st, jobs, dec, s.T, s.H, (int)s.BH())
-                    : launch_pdl(unfolded, retention_kernel<false, 1>, grid, block, smem, st, jobs, dec, s.T, s.H,
-                                 (int)s.BH());
-    return fold ? launch_pdl(folded, retention_kernel<true, 2>, grid, block, smem, st, jobs, dec, s.T, s.H, (int)s.BH())
-                : launch_pdl(unfolded, retention_kernel<false, 2>, grid, block, smem, st, jobs, dec, s.T, s.H,
-                             (int)s.BH());
+        return bf16 ? launch_retention_t<1, true>(folded, unfolded, passes, jobs, dec, s, st)
+                    : launch_retention_t<1, false>(folded, unfolded, passes, jobs, dec, s, st);
+    return bf16 ? launch_retention_t<2, true>(folded, unfolded, passes, jobs, dec, s, st)
+                : launch_retention_t<2, false>(folded, unfolded, passes, jobs, dec, s, st);
 }
 
 }  // namespace
 
 la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
-                        const DecayArgs &dec, const Shape &s, cudaStream_t st) {
+                        const DecayArgs &dec, const Shape &s, bool bf16, cudaStream_t st) {
     RetJobs jobs;
     memset(&jobs, 0, sizeof jobs);
     jobs.sin[0] = sin;
     jobs.sout[0] = sout;
     jobs.sonly[0] = o == nullptr;   // the state only: q and o are not touched (their maps stand in as k's)
-    LA_TRY(retention_map(&jobs.q[0], o ? q : k, s));
-    LA_TRY(retention_map(&jobs.k[0], k, s));
-    LA_TRY(retention_map(&jobs.v[0], v, s));
-    LA_TRY(retention_map(&jobs.o[0], o ? o : k, s));
-    return o ? launch_retention("tc_retention_fwd", "tc_retention_fwd_unfolded", 1, jobs, dec, s, st)
-             : launch_retention("tc_retention_state", "tc_retention_state_unfolded", 1, jobs, dec, s, st);
+    LA_TRY(retention_map(&jobs.q[0], o ? q : k, s, bf16));
+    LA_TRY(retention_map(&jobs.k[0], k, s, bf16));
+    LA_TRY(retention_map(&jobs.v[0], v, s, bf16));
+    LA_TRY(retention_map(&jobs.o[0], o ? o : k, s, bf16));
+    return o ? launch_retention("tc_retention_fwd", "tc_retention_fwd_unfolded", 1, jobs, dec, s, bf16, st)
+             : launch_retention("tc_retention_state", "tc_retention_state_unfolded", 1, jobs, dec, s, bf16, st);
 }
 
 la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin,
                         const float *rin, float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv,
-                        const Shape &s, cudaStream_t st) {
+                        const Shape &s, bool bf16, cudaStream_t st) {
     RetJobs jobs;
     memset(&jobs, 0, sizeof jobs);
     // dq = retention(dO, V, K); dv = reverse retention(K, Q, dO); dk = reverse retention(V, dO, Q).
@@ -703,11 +716,11 @@ la_status retention_bwd(const void *q, const void *k, const void *v, const void 
         jobs.sin[0] = rin;
         jobs.sout[0] = rout;
         jobs.sonly[0] = 1;
-        LA_TRY(retention_map(&jobs.q[0], q, s));
-        LA_TRY(retention_map(&jobs.k[0], q, s));
-        LA_TRY(retention_map(&jobs.v[0], g, s));
-        LA_TRY(retention_map(&jobs.o[0], q, s));
-        return launch_retention("tc_retention_state", "tc_retention_state_unfolded", 1, jobs, dec, s, st);
+        LA_TRY(retention_map(&jobs.q[0], q, s, bf16));
+        LA_TRY(retention_map(&jobs.k[0], q, s, bf16));
+        LA_TRY(retention_map(&jobs.v[0], g, s, bf16));
+        LA_TRY(retention_map(&jobs.o[0], q, s, bf16));
+        return launch_retention("tc_retention_state", "tc_retention_state_unfolded", 1, jobs, dec, s, bf16, st);
     }
     struct Pass {
         const void *q, *k, *v;
@@ -722,16 +735,16 @@ la_status retention_bwd(const void *q, const void *k, const void *v, const void 
                          {v, g, q, dk, 1, rin, 1, nullptr}};
     int np = 0;
     for (int p = dq ? 0 : 1; p < 3; ++p, ++np) {
-        LA_TRY(retention_map(&jobs.q[np], all[p].q, s));
-        LA_TRY(retention_map(&jobs.k[np], all[p].k, s));
-        LA_TRY(retention_map(&jobs.v[np], all[p].v, s));
-        LA_TRY(retention_map(&jobs.o[np], all[p].o, s));
+        LA_TRY(retention_map(&jobs.q[np], all[p].q, s, bf16));
+        LA_TRY(retention_map(&jobs.k[np], all[p].k, s, bf16));
+        LA_TRY(retention_map(&jobs.v[np], all[p].v, s, bf16));
+        LA_TRY(retention_map(&jobs.o[np], all[p].o, s, bf16));
         jobs.rev[np] = all[p].rev;
         jobs.sin[np] = all[p].sin;
         jobs.sin_t[np] = all[p].sin_t;
         jobs.sout[np] = all[p].sout;
     }
-    return launch_retention("tc_retention_bwd", "tc_retention_bwd_unfolded", np, jobs, dec, s, st);
+    return launch_retention("tc_retention_bwd", "tc_retention_bwd_unfolded", np, jobs, dec, s, bf16, st);
 }
 
 unsigned int read_and_clear_retention_fault() {

@@ -1347,8 +1347,8 @@ la_status make_tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, bool 
     return LA_OK;
 }
 
-la_status retention_map(CUtensorMap *m, const void *ptr, const Shape &s) {
-    return make_tensor_map(m, ptr, s, true, 64);
+la_status retention_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16) {
+    return make_tensor_map(m, ptr, s, bf16, 64);
 }
 
 namespace {

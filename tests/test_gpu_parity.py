@@ -191,11 +191,13 @@ def test_other_stream():
 # a chunk into one accumulator (every factor gamma^k with |k| <= 64 in range); smaller decays
 # keep the two parts apart.  Heads of both kinds in one call, and each kind alone; several
 # chunks with a ragged tail, so the row scales and the state carried between chunks count.
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("gammas", [(0.05, 0.3, 0.9, 0.999), (0.125, 0.5, 0.75, 1.0), (0.06, 0.1, 0.11, 0.02)],
-                         ids=["mixed", "folded", "unfolded"])
-def test_retention_strong_decays(gammas, D):
-    w = _workload("retention", "bf16", 2, len(gammas), 300, D)
+@pytest.mark.parametrize("gammas", [(0.05, 0.3, 0.9, 0.999), (0.125, 0.5, 0.75, 1.0), (0.06, 0.1, 0.11, 0.02),
+                                    (0.9, 0.95, 0.999, 1.0)],
+                         ids=["mixed", "folded", "unfolded", "folded_f16"])
+def test_retention_strong_decays(gammas, D, dtype):
+    w = _workload("retention", dtype, 2, len(gammas), 300, D)
     inp = synth.make_inputs(w, seed=3)
     inp["gamma"] = torch.tensor(gammas, dtype=torch.float32)
     got = pu.gpu_run("retention", inp)
@@ -206,9 +208,10 @@ def test_retention_strong_decays(gammas, D):
 # tile and keeps the second one zero.  Plain causal linear attention (gamma = 1 on every head)
 # and the retention decays, over several chunks with a ragged tail; then the B8 H16 T4096 D64
 # shape of the causal workloads on sampled heads.
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("gamma", [1.0, None], ids=["causal", "retention"])
-def test_decay_d64(gamma):
-    w = _workload("retention", "bf16", 2, 3, 1000, 64)
+def test_decay_d64(gamma, dtype):
+    w = _workload("retention", dtype, 2, 3, 1000, 64)
     inp = synth.make_inputs(w, seed=4)
     if gamma is not None:
         inp["gamma"] = torch.full((w.H,), gamma, dtype=torch.float32)
