@@ -54,6 +54,12 @@ KERNEL_TENSORS = {
     # retention backward: the op's minimum (q, k, v, dO in; dq, dk, dv out), not the 12 tensors the
     # three-pass kernel actually moves, so its fraction shows the cost of that design
     "tc_retention_fwd": 4, "tc_retention_bwd": 7,
+    # causal linear attention with the norm term on the tensor cores (fp16, D = 64): f(q), f(k)
+    # formed (q, k in, both out); the forward (f(q), f(k), v in, o out); the backward's first
+    # pass (those and dout in, du out); the dn terms (f(q), f(k), dq and dk in fp32 = two
+    # 16-bit tensors each, in; dq, dk out)
+    "tc_causal_norm_phi": 4, "tc_causal_norm_fwd": 4, "tc_causal_norm_prep": 5,
+    "tc_causal_norm_dn_parts": 2, "tc_causal_norm_dn_apply": 8,
 }
 
 # CUDA-core work of the recurrent kernels per token-head, in flops (2 per multiply-add, 1 per
@@ -362,8 +368,8 @@ WORKLOAD_TEXT = {
     "vision": "long-sequence vision-style bidirectional linear attention fwd only, fp16 storage / fp32 accumulate, "
               "B=%d H=%d T=%d D=%d (256x256 token grid), phi=elu+1, eps=1e-06, Q,K,V ~ 0.5 N(0,1) plus a smooth 2-D "
               "sinusoidal offset of amplitude 0.1",
-    "causal_norm": "causal linear attention with the norm term fwd+bwd (recurrent form in 256-token chunks on CUDA "
-                   "cores), fp16 storage / "
+    "causal_norm": "causal linear attention with the norm term fwd+bwd (fp16 at D=64: the chunked decay kernel "
+                   "on tensor cores with a column of ones carrying the normaliser), fp16 storage / "
                    "fp32 accumulate, B=%d H=%d T=%d D=%d, phi=elu+1, no decay, eps=1e-06, Q,K,V ~ 0.5 N(0,1), "
                    "dO ~ N(0,1)",
 }

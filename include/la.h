@@ -261,13 +261,16 @@ la_status la_chunk_decay_scan(const float *states, const long long *gaps, int n,
  * op is la_chunk_decay_* (identity f, gamma = 1 for plain causal linear
  * attention).  Sources: "flash-linear-attention" README, "Different forms of
  * linear attention" (FusedRecurrent: the recurrent form these calls compute);
- * the norm term and f as in la_bidir_*.  Computed on CUDA cores, fp32; all
- * dtypes, D in {64, 128}.  The sequence is cut into chunks of 256 tokens, one
- * CTA per (b, h, chunk) walking its chunk from the state the tokens before it
- * leave; those states come from each chunk's own state (a sum of outer
- * products) and a scan over the chunks.
- * Workspace: la_workspace_size(LA_OP_CAUSAL_NORM_FWD, ...) bytes (the chunk
- * states, B H ceil(T / 256) D (D + 1) fp32 values; 0, NULL allowed, for T <= 256). */
+ * the norm term and f as in la_bidir_*.  All dtypes, D in {64, 128}.
+ * fp16 with D = 64 runs on the tensor cores (the chunked decay kernel with a
+ * column of ones next to v, which carries z, and the division in its epilogue;
+ * f(q), f(k) formed first into the workspace); the rest on CUDA cores in fp32,
+ * the sequence cut into chunks of 256 tokens, one CTA per (b, h, chunk) walking
+ * its chunk from the state the tokens before it leave (each chunk's own state,
+ * a sum of outer products, and a scan over the chunks).
+ * Workspace: la_workspace_size(LA_OP_CAUSAL_NORM_FWD, ...) bytes (tensor cores:
+ * f(q), f(k); CUDA cores: the chunk states, B H ceil(T / 256) D (D + 1) fp32
+ * values, 0 and NULL allowed for T <= 256). */
 la_status la_causal_norm_fwd(const void *q, const void *k, const void *v, void *o, const float *decay,
                              la_feature feature, float eps, int B, int H, int T, int D, la_dtype dtype,
                              void *workspace, size_t workspace_bytes, void *stream);
@@ -278,9 +281,10 @@ la_status la_causal_norm_fwd(const void *q, const void *k, const void *v, void *
  *   dq_t = (S_t du_t + z_t dn_t) f'(q_t)
  *   R_s = sum_{t>=s} gamma^(t-s) f(q_t)^T du_t,  r_s = sum_{t>=s} gamma^(t-s) f(q_t) dn_t
  *   dk_s = (R_s v_s + r_s) f'(k_s),  dv_s = f(k_s) R_s.
- * Workspace: la_workspace_size(LA_OP_CAUSAL_NORM_BWD, ...) bytes ((n_t, dn_t)
- * of every row, 8 B per token-head, then the chunk states of the forward and,
- * reusing them, of the reverse sweep). */
+ * Workspace: la_workspace_size(LA_OP_CAUSAL_NORM_BWD, ...) bytes (tensor cores:
+ * f(q), f(k), du = dout / n, dn, per-chunk sums and the fp32 dq, dk before the
+ * dn terms; CUDA cores: (n_t, dn_t) of every row, 8 B per token-head, then the
+ * chunk states of the forward and, reusing them, of the reverse sweep). */
 la_status la_causal_norm_bwd(const void *q, const void *k, const void *v, const void *dout, const float *decay,
                              la_feature feature, float eps, void *dq, void *dk, void *dv,
                              int B, int H, int T, int D, la_dtype dtype,

@@ -444,6 +444,9 @@ la_status la_causal_norm_fwd(const void *q, const void *k, const void *v, void *
     LA_TRY(check_ptr(o, "o"));
     LA_TRY(check_ws(LA_OP_CAUSAL_NORM_FWD, s, dtype, workspace, workspace_bytes));
     if (T == 0) return LA_OK;
+    if (path_tc(LA_OP_CAUSAL_NORM_FWD, s, dtype))
+        return tc::causal_norm_fwd(q, k, v, o, dec, has_decay, feature == LA_FEATURE_ELU1, s, dtype, eps, workspace,
+                                   (cudaStream_t)stream);
     return simt::causal_norm_fwd(q, k, v, o, dec, has_decay, feature == LA_FEATURE_ELU1, s, dtype, eps, workspace,
                                  (cudaStream_t)stream);
 }
@@ -464,6 +467,9 @@ la_status la_causal_norm_bwd(const void *q, const void *k, const void *v, const 
     LA_TRY(check_ptr(dv, "dv"));
     LA_TRY(check_ws(LA_OP_CAUSAL_NORM_BWD, s, dtype, workspace, workspace_bytes));
     if (T == 0) return LA_OK;
+    if (path_tc(LA_OP_CAUSAL_NORM_BWD, s, dtype))
+        return tc::causal_norm_bwd(q, k, v, dout, dq, dk, dv, dec, has_decay, feature == LA_FEATURE_ELU1, s, dtype,
+                                   eps, workspace, (cudaStream_t)stream);
     return simt::causal_norm_bwd(q, k, v, dout, dq, dk, dv, dec, has_decay, feature == LA_FEATURE_ELU1, s, dtype, eps,
                                  workspace, (cudaStream_t)stream);
 }

@@ -17,6 +17,8 @@ bool supports(la_op op, const Shape &s, la_dtype dt) {
     case LA_OP_STATE_BWD_KV: return s.D == 64;
     case LA_OP_CHUNK_DECAY_FWD:
     case LA_OP_CHUNK_DECAY_BWD: return s.D == 64 || s.D == 128;
+    case LA_OP_CAUSAL_NORM_FWD:
+    case LA_OP_CAUSAL_NORM_BWD: return causal_norm_supported(s, dt);
     default: return false;
     }
 }
@@ -36,6 +38,8 @@ size_t workspace_size(la_op op, const Shape &s, la_dtype) {
     case LA_OP_SIMPLE_BWD:
     case LA_OP_STATE_REDUCE:
     case LA_OP_STATE_BWD_Q: return state_workspace_size(op, s);
+    case LA_OP_CAUSAL_NORM_FWD:
+    case LA_OP_CAUSAL_NORM_BWD: return causal_norm_workspace(op, s, true);   // the larger, with elu + 1
     default: return 0;
     }
 }

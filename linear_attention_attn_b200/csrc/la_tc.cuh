@@ -21,14 +21,30 @@ unsigned int read_and_clear_debug_fault();
 // [BH, T, D] 16-bit tensor map: boxes of box_rows x 64 columns, 128-byte swizzle.
 la_status make_tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16, int box_rows);
 la_status retention_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16);
+la_status retention_map_f32(CUtensorMap *m, void *ptr, const Shape &s);
 // Chunked causal decay forward on tensor cores (bf16 or fp16 storage, D = 64 or 128).
 la_status retention_fwd(const void *q, const void *k, const void *v, void *o, const float *sin, float *sout,
                         const DecayArgs &dec, const Shape &s, bool bf16, cudaStream_t st);
 // sin: state S entering the segment (or null); rin: R = sum_{t >= end} gamma^(t-end) q_t^T dO_t
 // entering from the right (or null); rout: R at the segment's first row (or null).  [BH, D, D].
+// dq32, dk32 (or null; D = 64 only): dq and dk written in fp32 there instead of dq, dk.
 la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin,
                         const float *rin, float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv,
-                        const Shape &s, bool bf16, cudaStream_t st);
+                        const Shape &s, bool bf16, cudaStream_t st, float *dq32 = nullptr, float *dk32 = nullptr);
+// Causal linear attention with the norm term on features q, k formed by the caller (D = 64):
+// o_t = q_t S_t / n_t with n_t = q_t . z_t + eps.  With dout not null, o receives
+// du = dout / n instead and dn (fp32 [BH, T]) -(dout . o) / n.
+la_status retention_norm_fwd(const void *q, const void *k, const void *v, void *o, const void *dout, float *dn,
+                             const DecayArgs &dec, float eps, const Shape &s, bool bf16, cudaStream_t st);
+// Causal linear attention with the norm term (D = 64, fp16; has_decay = 0: gamma = 1; phi:
+// f = elu + 1, else the identity); workspace causal_norm_workspace(op, s, phi) bytes.
+bool causal_norm_supported(const Shape &s, la_dtype dt);
+size_t causal_norm_workspace(la_op op, const Shape &s, bool phi);
+la_status causal_norm_fwd(const void *q, const void *k, const void *v, void *o, const DecayArgs &dec, int has_decay,
+                          bool phi, const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
+la_status causal_norm_bwd(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
+                          void *dv, const DecayArgs &dec, int has_decay, bool phi, const Shape &s, la_dtype dt,
+                          float eps, void *ws, cudaStream_t st);
 la_status state_fwd(bool bidir, const void *q, const void *k, const void *v, void *o, float *state,
                     const Shape &s, la_dtype dt, float eps, void *ws, cudaStream_t st);
 la_status state_bwd(bool bidir, const void *q, const void *k, const void *v, const void *g,

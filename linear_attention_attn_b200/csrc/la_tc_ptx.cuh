@@ -373,6 +373,16 @@ __device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t a, ui
                  : "memory");
 }
 
+// The load that stmatrix_x4_trans inverts: four 8x8 matrices read transposed, thread 8k + j
+// giving the address of row j of stored matrix k; register k of thread t receives elements
+// (t/4, 2(t%4)) and (t/4, 2(t%4)+1) of matrix k.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t saddr, uint32_t &a, uint32_t &b, uint32_t &c, uint32_t &d) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+                 : "r"(saddr)
+                 : "memory");
+}
+
 // ------------------------------------------------------------ descriptors --
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100
 // version field = 1.  lbo/sbo in bytes (multiples of 16).

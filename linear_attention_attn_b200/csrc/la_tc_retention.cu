@@ -97,8 +97,10 @@ struct RetLayout {
     static constexpr int ptoff = khoff + 2 * kTile128;          // P~ hi, lo: [64 x 64] each
     static constexpr int ooff = ptoff + 2 * kBox;               // output staging chunk
     static constexpr int gpoff = ooff + kTile128;               // gamma^k, k = -64..128
-    static constexpr int baroff = gpoff + 196 * 4;
-    static constexpr int nbars = 2 * NST + 16;
+    static constexpr int denoff = gpoff + 196 * 4;              // [2][64] 1 / denominators (norm term)
+    static constexpr int dotoff = denoff + 2 * 64 * 4;          // [2][64] dout . o partial sums (prep)
+    static constexpr int baroff = dotoff + 2 * 64 * 4;
+    static constexpr int nbars = 2 * NST + 22;
     static constexpr int misc = baroff + nbars * 8;
     static constexpr int bytes = misc + 32 + 1024;
     static_assert(bytes <= 227 * 1024, "shared memory of one CTA");
@@ -129,6 +131,17 @@ struct RetJobs {
     // sonly[p] != 0: the pass computes its state only (sout), no output: only k and v
     // are loaded, and per chunk only K^ and dS^T are formed.
     int sonly[3];
+    // D = 64 only: o32[p] != 0 writes the pass's output in fp32 (map o[p] of fp32 [BH, T, 64],
+    // boxes of 32 columns), for a caller that adds to it before rounding.
+    int o32[3];
+    // Kernels with the norm term (NORM): eps of the denominators.  prep != 0 turns the
+    // forward into the first step of the backward: with dout (map g) loaded chunk by chunk,
+    // the output written is du = dout / n (n = f(q) . z + eps) instead of o, and dn receives
+    // -(dout . o) / n of every row, [BH, T] fp32.
+    CUtensorMap g;
+    float eps;
+    int prep;
+    float *dn;
 };
 
 // Grid: one CTA per (pass, b, h), pass = blockIdx.x / BH.  decay[h] = gamma_h.
@@ -155,9 +168,16 @@ struct RetJobs {
 //   dS^T        M=128 N=128 K=64   A = V^T (MN-major)         B = K^ hi, lo (MN-major)
 //   O_intra^T   M=128 N=64  K=64   A = V^T (MN-major)         B = P~ hi, lo (K-major)
 //   O_inter^T   M=128 N=64  K=128  A = S^T hi, lo (tensor mem) B = Q (K-major)
-template <bool FOLD, int NBOX, bool BF>
+//
+// NORM (D = 64, forward in time): causal linear attention with the norm term,
+// o_t = f(q_t) S_t / (f(q_t) . z_t + eps) with z_t the decayed sum of f(k_s).  The unused
+// first box of every v stage holds a column of ones (value index -1, TMEM lane 0), so the
+// same products carry z through the state (lane 0 of S^T) and give each row's denominator
+// in lane 0 of the output accumulator; the epilogue divides by it.
+template <bool FOLD, int NBOX, bool BF, bool NORM>
 __global__ void __launch_bounds__(kRThreads, 1)
 retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int H, int BH) {
+    static_assert(!NORM || NBOX == 1, "the norm term needs the free first box of v (D = 64)");
     using L = RetLayout;
     constexpr int NST = L::NST;
     constexpr uint32_t ID_P = idesc_f16(64, 64, BF, false, false);
@@ -174,6 +194,8 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
     uint8_t *sO = smem + L::ooff;
     float *gexp = reinterpret_cast<float *>(smem + L::gpoff);   // gexp[k + 64] = gamma^k
 #define GP(k) gexp[(k) + 64]
+    float *sDen = reinterpret_cast<float *>(smem + L::denoff);   // NORM: 1 / (f(q) . z + eps) per row
+    float *sDot = reinterpret_cast<float *>(smem + L::dotoff);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::baroff);
     uint64_t *empty = full + NST;
     uint64_t *pfull = empty + NST;       // [2] P of a chunk in TMEM buffer (chunk & 1)
@@ -187,6 +209,9 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
     uint64_t *ofull = sfree + 1;         // [2] the output of a chunk in TMEM (FOLD: per buffer)
     uint64_t *oread = ofull + 2;         // [2] ... read (output warps)
     uint64_t *drain = oread + 2;
+    uint64_t *gfull = drain + 1;         // [2] prep: the dout chunk in its buffer (iteration & 1)
+    uint64_t *denready = gfull + 2;      // [2] NORM: sDen[iteration & 1] written
+    uint64_t *denfree = denready + 2;    // [2] NORM: ... read
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc);
     int *s_abort = reinterpret_cast<int *>(tmem_slot + 1);
 
@@ -226,6 +251,11 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             mbar_init(&oread[b], kROWarps);
         }
         mbar_init(drain, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&gfull[b], 1);
+            mbar_init(&denready[b], 1);
+            mbar_init(&denfree[b], 2);
+        }
         *s_abort = 0;
         fence_mbar_init();
     }
@@ -241,6 +271,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         tma_prefetch(tmK);
         tma_prefetch(tmV);
         tma_prefetch(tmO);
+        if (NORM && jobs.prep) tma_prefetch(&jobs.g);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -255,7 +286,10 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             uint8_t *base = b < 2 * NST ? smem + L::qoff + b * kTile128 + kBox
                           : b < 3 * NST ? smem + L::qoff + b * kTile128
                                         : sKh + (b - 3 * NST) * kTile128 + kBox;
-            *reinterpret_cast<uint4 *>(base + e * 16) = make_uint4(0u, 0u, 0u, 0u);
+            // NORM: column 0 of v's first box is one (the 16-byte chunk of row e / 8 that
+            // the swizzle puts column 0 in)
+            const bool one = NORM && b >= 2 * NST && b < 3 * NST && (e & 7) == ((e >> 3) & 7);
+            *reinterpret_cast<uint4 *>(base + e * 16) = make_uint4(one ? h2<BF>::one() : 0u, 0u, 0u, 0u);
         }
         fence_async_smem();
     }
@@ -440,34 +474,129 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         // in rounds of 16 columns: a 16x256b TMEM load gives the MMA-fragment layout of a
         // [16 d x 16 i] block, and stmatrix .trans writes its four 8x8 parts transposed, as
         // 16-byte rows of the staging chunk (row i, 8 consecutive d).  Named barrier 1
-        // (these 128 threads) is reached by all of them whatever the waits return.
+        // (the warps that write the staging chunk: all four, or with D = 64 the two of lanes
+        // 64..127) is reached by all of them whatever the waits return.  With D = 64 the other
+        // two warps hold no output: they run ahead, releasing each accumulator as soon as it is
+        // full, and (NORM) the first of them forms the chunk's reciprocal denominators from
+        // lane 0 (the column of ones) into sDen[it & 1] a chunk ahead of their use.
         const int ot = threadIdx.x - kROw0 * 32;
         const int sub = warp & 3;
         const int q4 = lane & 3;                            // fragment: columns 2 q4 (+1) of lanes lane / 4 (+8)
         const int mk = lane >> 3, mj = lane & 7;            // stmatrix: matrix mk, stored row mj
+        // prep (forward only): the dout chunk of iteration it in the unused second box of K^
+        // hi (it even) or lo (it odd), loaded one iteration ahead
+        const bool prep = NORM && jobs.prep;
+        const bool out32 = NBOX == 1 && jobs.o32[pass];
+        auto gbuf = [&](int it) -> uint8_t * { return sKh + (it & 1) * kTile128 + kBox; };
+        if (prep && ot == 0 && nchunks > 0) {
+            mbar_arrive_expect_tx(&gfull[0], kBox);
+            tma_load_3d(gbuf(0), &jobs.g, &gfull[0], 0, 0, bh);
+        }
+        auto scale_in = [&](int rows, int i) -> float {   // FOLD: f_i; else g_i of the inter-chunk part
+            if (FOLD) return rev ? (i < rows ? GP(rows - i - kM) : 0.f) : GP(i + 1 - kM);
+            return rev ? (i < rows ? GP(rows - i) : 0.f) : GP(i + 1);
+        };
+        constexpr int kStageThreads = (NBOX == 1 ? 2 : kROWarps) * 32;   // named barrier 1
         bool live = true;
+        if (NBOX == 1 && sub < 2) {
+            for (int it = 0; it < (sonly ? 0 : nchunks); ++it) {
+                const int c = rev ? nchunks - 1 - it : it;
+                const int rows = min(kC, T - c * kC);
+                const int ob = FOLD ? (it & 1) : 0;
+                if (!__all_sync(0xffffffffu, LA_RWAIT(&ofull[ob], FOLD ? (uint32_t)((it >> 1) & 1) : (uint32_t)(it & 1),
+                                                      0x800u)))
+                    break;
+                __syncwarp();   // converged for the .sync.aligned TMEM loads
+                tc_fence_after();
+                if (NORM && sub == 0) {
+                    // sDen[it & 1] was last read for iteration it - 2
+                    if (it >= 2 && !__all_sync(0xffffffffu, LA_RWAIT(&denfree[it & 1], (uint32_t)(((it >> 1) & 1) ^ 1),
+                                                                      0x20000u)))
+                        break;
+                    float *den = sDen + 64 * (it & 1);
+                    // threads 0..3 hold lane 0, columns 16 h + 2 t, +1, +8, +9 (16x256b layout)
+#pragma unroll 1
+                    for (int h = 0; h < 4; ++h) {
+                        uint32_t r[8];
+                        float x0, x1, x8, x9;
+                        const int c0 = 16 * h + 2 * q4;
+                        if (FOLD) {
+                            tmem_ld16x256b_x2_sync(tmem + cO + 64u * (uint32_t)ob + 16 * h, r);
+                            x0 = scale_in(rows, c0) * __uint_as_float(r[0]);
+                            x1 = scale_in(rows, c0 + 1) * __uint_as_float(r[1]);
+                            x8 = scale_in(rows, c0 + 8) * __uint_as_float(r[4]);
+                            x9 = scale_in(rows, c0 + 9) * __uint_as_float(r[5]);
+                        } else {
+                            uint32_t xi[8];
+                            tmem_ld16x256b_x2_sync(tmem + cOI + 16 * h, xi);
+                            tmem_ld16x256b_x2_sync(tmem + cOX + 16 * h, r);
+                            x0 = fmaf(scale_in(rows, c0), __uint_as_float(r[0]), __uint_as_float(xi[0]));
+                            x1 = fmaf(scale_in(rows, c0 + 1), __uint_as_float(r[1]), __uint_as_float(xi[1]));
+                            x8 = fmaf(scale_in(rows, c0 + 8), __uint_as_float(r[4]), __uint_as_float(xi[4]));
+                            x9 = fmaf(scale_in(rows, c0 + 9), __uint_as_float(r[5]), __uint_as_float(xi[5]));
+                        }
+                        // the reciprocals, once per row (approximate reciprocal: a few fp32 ulp)
+                        if (lane < 4) {
+                            *reinterpret_cast<float2 *>(den + c0) =
+                                make_float2(__fdividef(1.f, x0 + jobs.eps), __fdividef(1.f, x1 + jobs.eps));
+                            *reinterpret_cast<float2 *>(den + c0 + 8) =
+                                make_float2(__fdividef(1.f, x8 + jobs.eps), __fdividef(1.f, x9 + jobs.eps));
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&denready[it & 1]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&oread[ob]);
+            }
+        } else {
         for (int it = 0; it < (sonly ? 0 : nchunks); ++it) {
             const int c = rev ? nchunks - 1 - it : it;
             const uint32_t pc = (uint32_t)(it & 1);
             if (ot == 0) tma_store_wait_read<0>();
-            named_bar(1, kROWarps * 32);
+            named_bar(1, kStageThreads);
+            // the buffer of iteration it + 1 was last read in iteration it - 1, now complete
+            if (prep && ot == 0 && it + 1 < nchunks) {
+                mbar_arrive_expect_tx(&gfull[(it + 1) & 1], kBox);
+                tma_load_3d(gbuf(it + 1), &jobs.g, &gfull[(it + 1) & 1], 0, (it + 1) * kC, bh);
+            }
             const int ob = FOLD ? (it & 1) : 0;
             bool got = live && LA_RWAIT(&ofull[ob], FOLD ? (uint32_t)((it >> 1) & 1) : pc, 0x800u);
             got = __all_sync(0xffffffffu, got);
             live = live && got;
+            // backwards the entering state sits one past the chunk's last valid row
+            const int rows = min(kC, T - c * kC);
+            auto scale = [&](int i) -> float { return scale_in(rows, i); };
             if (got) {
                 __syncwarp();   // converged for the .sync.aligned TMEM loads
                 tc_fence_after();
-                // backwards the entering state sits one past the chunk's last valid row
-                const int rows = min(kC, T - c * kC);
-                auto scale = [&](int i) -> float {   // FOLD: f_i; else g_i of the inter-chunk part
-                    if (FOLD) return rev ? (i < rows ? GP(rows - i - kM) : 0.f) : GP(i + 1 - kM);
-                    return rev ? (i < rows ? GP(rows - i) : 0.f) : GP(i + 1);
-                };
+            }
+            const float *den = sDen + 64 * (it & 1);
+            if (NORM && got) {
+                got = __all_sync(0xffffffffu, LA_RWAIT(&denready[it & 1], (uint32_t)((it >> 1) & 1), 0x40000u));
+                live = live && got;
+            }
+            if (got) {
+                const uint8_t *gb = gbuf(it);
+                if (prep) {
+                    got = __all_sync(0xffffffffu, LA_RWAIT(&gfull[it & 1], (uint32_t)((it >> 1) & 1), 0x8000u));
+                    live = live && got;
+                }
 #pragma unroll 1
                 for (int h = 0; h < 4; ++h) {
                     const int i0 = 16 * h + 2 * q4;
-                    const float f0 = scale(i0), f1 = scale(i0 + 1), f8 = scale(i0 + 8), f9 = scale(i0 + 9);
+                    float pA = 0.f, pB = 0.f, pC = 0.f, pD = 0.f;   // prep: dout . o of rows i0, +1, +8, +9
+                    float f0 = scale(i0), f1 = scale(i0 + 1), f8 = scale(i0 + 8), f9 = scale(i0 + 9);
+                    // NORM: each row times the reciprocal of its denominator
+                    const float u0 = NORM ? den[i0] : 1.f, u1 = NORM ? den[i0 + 1] : 1.f;
+                    const float u8 = NORM ? den[i0 + 8] : 1.f, u9 = NORM ? den[i0 + 9] : 1.f;
+                    if (FOLD) {
+                        f0 *= u0;
+                        f1 *= u1;
+                        f8 *= u8;
+                        f9 *= u9;
+                    }
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         const int dbase = 32 * sub + 16 * half;
@@ -489,13 +618,57 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                             tmem_ld16x256b_x2_sync(tmem + cOI + tl + 16 * h, r);
                             tmem_ld16x256b_x2_sync(tmem + cOX + tl + 16 * h, x);
                             const float fs[8] = {f0, f1, f0, f1, f8, f9, f8, f9};
+                            const float us[8] = {u0, u1, u0, u1, u8, u9, u8, u9};
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) y[e] = fmaf(fs[e], __uint_as_float(x[e]), __uint_as_float(r[e]));
+                            for (int e = 0; e < 8; ++e)
+                                y[e] = us[e] * fmaf(fs[e], __uint_as_float(x[e]), __uint_as_float(r[e]));
                         }
                         if (h == 3 && half == 1) {
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(&oread[ob]);
+                        }
+                        if (prep && got) {
+                            // y holds o: the sums dout . o, and du = dout / n in its place.  The
+                            // dout tile is laid out as the staging chunk (row i, value index d =
+                            // lane - 64), so ldmatrix .trans gives it in y's fragment layout.
+                            const int grow = 16 * h + mj + (mk >= 2 ? 8 : 0);
+                            const int gd = dbase - 64 + ((mk & 1) ? 8 : 0);
+                            uint32_t w0, w1, w2, w3;
+                            ldmatrix_x4_trans(smem_u32(gb + grow * 128 + (((gd >> 3) ^ (grow & 7)) << 4)), w0, w1, w2, w3);
+                            const float2 e0 = h2<BF>::to_f2(w0), e1 = h2<BF>::to_f2(w1), e2 = h2<BF>::to_f2(w2),
+                                         e3 = h2<BF>::to_f2(w3);
+                            const float g0 = e0.x, g1 = e0.y, g2 = e1.x, g3 = e1.y, g4 = e2.x, g5 = e2.y, g6 = e3.x,
+                                        g7 = e3.y;
+                            pA += y[0] * g0 + y[2] * g2;
+                            pB += y[1] * g1 + y[3] * g3;
+                            pC += y[4] * g4 + y[6] * g6;
+                            pD += y[5] * g5 + y[7] * g7;
+                            y[0] = g0 * u0;
+                            y[1] = g1 * u1;
+                            y[2] = g2 * u0;
+                            y[3] = g3 * u1;
+                            y[4] = g4 * u8;
+                            y[5] = g5 * u9;
+                            y[6] = g6 * u8;
+                            y[7] = g7 * u9;
+                        }
+                        if (NBOX == 1 && out32) {
+                            // fp32 staging: two boxes of [64 rows x 32 columns], 128-byte swizzle
+                            const int d0 = dbase - 64 + (lane >> 2);
+                            auto put = [&](int i, int d, float x) {
+                                *reinterpret_cast<float *>(sO + (d >> 5) * kBox + i * 128 +
+                                                           ((((d & 31) >> 2) ^ (i & 7)) << 4) + (d & 3) * 4) = x;
+                            };
+                            put(i0, d0, y[0]);
+                            put(i0 + 1, d0, y[1]);
+                            put(i0, d0 + 8, y[2]);
+                            put(i0 + 1, d0 + 8, y[3]);
+                            put(i0 + 8, d0, y[4]);
+                            put(i0 + 9, d0, y[5]);
+                            put(i0 + 8, d0 + 8, y[6]);
+                            put(i0 + 9, d0 + 8, y[7]);
+                            continue;
                         }
                         // matrices: (d 0..7, i 0..7), (d 8..15, i 0..7), (d 0..7, i 8..15), (d 8..15, i 8..15)
                         const int row = 16 * h + mj + (mk >= 2 ? 8 : 0);
@@ -505,17 +678,64 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
                         stmatrix_x4_trans(sa, h2<BF>::from_f2(y[0], y[1]), h2<BF>::from_f2(y[2], y[3]),
                                           h2<BF>::from_f2(y[4], y[5]), h2<BF>::from_f2(y[6], y[7]));
                     }
+                    if (prep) {
+                        // over the 8 lane groups of the warp, then one part per warp in sDot
+#pragma unroll
+                        for (int m = 4; m < 32; m <<= 1) {
+                            pA += __shfl_xor_sync(0xffffffffu, pA, m);
+                            pB += __shfl_xor_sync(0xffffffffu, pB, m);
+                            pC += __shfl_xor_sync(0xffffffffu, pC, m);
+                            pD += __shfl_xor_sync(0xffffffffu, pD, m);
+                        }
+                        if (lane < 4) {
+                            float *dst = sDot + (sub - 2) * 64;
+                            dst[i0] = pA;
+                            dst[i0 + 1] = pB;
+                            dst[i0 + 8] = pC;
+                            dst[i0 + 9] = pD;
+                        }
+                    }
                 }
             }
+            if (prep && sub >= 2) {
+                // dn = -(dout . o) / n of the chunk's rows, from the two warps' parts
+                named_bar(3, 64);
+                if (sub == 2 && got) {
+#pragma unroll
+                    for (int r2 = 0; r2 < 2; ++r2) {
+                        const int i = lane + 32 * r2;
+                        if (i < rows)
+                            jobs.dn[(long long)bh * T + (long long)c * kC + i] = -(sDot[i] + sDot[64 + i]) * den[i];
+                    }
+                }
+            }
+            if (NORM) {   // den read for this chunk
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&denfree[it & 1]);
+            }
             fence_async_smem();
-            named_bar(1, kROWarps * 32);
+            named_bar(1, kStageThreads);
             if (ot == 0 && live) {
-                tma_store_3d(tmO, sO + vbox * kBox, 0, c * kC, bh);
-                if (NBOX == 2) tma_store_3d(tmO, sO + kBox, 64, c * kC, bh);
+                if (NBOX == 1 && out32) {
+                    tma_store_3d(tmO, sO, 0, c * kC, bh);
+                    tma_store_3d(tmO, sO + kBox, 32, c * kC, bh);
+                } else {
+                    tma_store_3d(tmO, sO + vbox * kBox, 0, c * kC, bh);
+                    if (NBOX == 2) tma_store_3d(tmO, sO + kBox, 64, c * kC, bh);
+                }
                 tma_store_commit();
             }
         }
         if (ot == 0) tma_store_wait_all<0>();
+        if (prep && ot == 0) {
+            // every dout load has landed before the shared memory goes (an early exit may
+            // leave the last ones unread): the last phase of each buffer
+            for (int b = 0; b < 2; ++b) {
+                const int nb = (nchunks + 1 - b) / 2;
+                if (nb > 0) mbar_wait_slow(smem_u32(&gfull[b]), (uint32_t)((nb - 1) & 1), nullptr, &g_ret_fault, 0x10000u);
+            }
+        }
+        }
     } else {
         // State warps: S^T_{c+1} = gamma^C S^T_c + dS^T_c in fp32 registers; thread (d, half)
         // holds row d of S^T (column d of S), entries SC half .. SC half + SC - 1 (its TMEM
@@ -527,7 +747,8 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         const int sub = warp & 3, half = (warp - kRSw0) >> 2;
         const uint32_t lanes = (uint32_t)(32 * sub) << 16;
         const int d = 32 * sub + lane;
-        const bool sact = NBOX == 2 || sub >= 2;
+        // (NORM: lane 0, the column of ones, carries z; its warps hold the rest of lanes 0..31 as zeros)
+        const bool sact = NBOX == 2 || sub >= 2 || (NORM && sub == 0);
         const int dv = d - 64 * vbox;          // the value dimension of lane d
         const int col0 = SC * half;
         const float gC = GP(kC);
@@ -539,7 +760,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
         const float *sin = jobs.sin[pass];
         float *sout = jobs.sout[pass];
         const long long sbase = (long long)bh * D * D;
-        if (sin && sact) {
+        if (sin && sact && dv >= 0) {
             if (jobs.sin_t[pass]) {   // sin holds S^T: row d, entries col0 ..
 #pragma unroll
                 for (int c4 = 0; c4 < SC / 4; ++c4) {
@@ -628,7 +849,7 @@ retention_kernel(const __grid_constant__ RetJobs jobs, DecayArgs dec, int T, int
             tc_fence_after();
             write_state();
         }
-        if (sout && sact && !*s_abort) {   // S after the last chunk: column d of S, lanes write consecutive d
+        if (sout && sact && dv >= 0 && !*s_abort) {   // S after the last chunk: column d of S, lanes write consecutive d
 #pragma unroll
             for (int c = 0; c < SC; ++c) sout[sbase + (long long)(col0 + c) * D + dv] = st[c];
         }
@@ -669,10 +890,10 @@ static la_status launch_retention_t(const char *folded, const char *unfolded, in
     const dim3 grid((unsigned)(passes * s.BH())), block(kRThreads);
     const size_t smem = (size_t)RetLayout::bytes;
     return fold_ok(dec, s.H, BF)
-               ? launch_pdl(folded, retention_kernel<true, NBOX, BF>, grid, block, smem, st, jobs, dec, s.T, s.H,
+               ? launch_pdl(folded, retention_kernel<true, NBOX, BF, false>, grid, block, smem, st, jobs, dec, s.T, s.H,
                             (int)s.BH())
-               : launch_pdl(unfolded, retention_kernel<false, NBOX, BF>, grid, block, smem, st, jobs, dec, s.T, s.H,
-                            (int)s.BH());
+               : launch_pdl(unfolded, retention_kernel<false, NBOX, BF, false>, grid, block, smem, st, jobs, dec, s.T,
+                            s.H, (int)s.BH());
 }
 
 static la_status launch_retention(const char *folded, const char *unfolded, int passes, const RetJobs &jobs,
@@ -701,9 +922,39 @@ la_status retention_fwd(const void *q, const void *k, const void *v, void *o, co
              : launch_retention("tc_retention_state", "tc_retention_state_unfolded", 1, jobs, dec, s, bf16, st);
 }
 
+la_status retention_norm_fwd(const void *q, const void *k, const void *v, void *o, const void *dout, float *dn,
+                             const DecayArgs &dec, float eps, const Shape &s, bool bf16, cudaStream_t st) {
+    if (s.D != 64) return LA_ERR_UNSUPPORTED;
+    RetJobs jobs;
+    memset(&jobs, 0, sizeof jobs);
+    LA_TRY(retention_map(&jobs.q[0], q, s, bf16));
+    LA_TRY(retention_map(&jobs.k[0], k, s, bf16));
+    LA_TRY(retention_map(&jobs.v[0], v, s, bf16));
+    LA_TRY(retention_map(&jobs.o[0], o, s, bf16));
+    jobs.eps = eps;
+    if (dout) {
+        LA_TRY(retention_map(&jobs.g, dout, s, bf16));
+        jobs.prep = 1;
+        jobs.dn = dn;
+    }
+    const char *name = dout ? (fold_ok(dec, s.H, bf16) ? "tc_causal_norm_prep" : "tc_causal_norm_prep_unfolded")
+                            : (fold_ok(dec, s.H, bf16) ? "tc_causal_norm_fwd" : "tc_causal_norm_fwd_unfolded");
+    const dim3 grid((unsigned)s.BH()), block(kRThreads);
+    const size_t smem = (size_t)RetLayout::bytes;
+    if (fold_ok(dec, s.H, bf16))
+        return bf16 ? launch_pdl(name, retention_kernel<true, 1, true, true>, grid, block, smem, st, jobs, dec, s.T,
+                                 s.H, (int)s.BH())
+                    : launch_pdl(name, retention_kernel<true, 1, false, true>, grid, block, smem, st, jobs, dec, s.T,
+                                 s.H, (int)s.BH());
+    return bf16 ? launch_pdl(name, retention_kernel<false, 1, true, true>, grid, block, smem, st, jobs, dec, s.T, s.H,
+                             (int)s.BH())
+                : launch_pdl(name, retention_kernel<false, 1, false, true>, grid, block, smem, st, jobs, dec, s.T, s.H,
+                             (int)s.BH());
+}
+
 la_status retention_bwd(const void *q, const void *k, const void *v, const void *g, const float *sin,
                         const float *rin, float *rout, const DecayArgs &dec, void *dq, void *dk, void *dv,
-                        const Shape &s, bool bf16, cudaStream_t st) {
+                        const Shape &s, bool bf16, cudaStream_t st, float *dq32, float *dk32) {
     RetJobs jobs;
     memset(&jobs, 0, sizeof jobs);
     // dq = retention(dO, V, K); dv = reverse retention(K, Q, dO); dk = reverse retention(V, dO, Q).
@@ -738,7 +989,13 @@ la_status retention_bwd(const void *q, const void *k, const void *v, const void 
         LA_TRY(retention_map(&jobs.q[np], all[p].q, s, bf16));
         LA_TRY(retention_map(&jobs.k[np], all[p].k, s, bf16));
         LA_TRY(retention_map(&jobs.v[np], all[p].v, s, bf16));
-        LA_TRY(retention_map(&jobs.o[np], all[p].o, s, bf16));
+        float *o32 = p == 0 ? dq32 : p == 2 ? dk32 : nullptr;
+        if (o32) {
+            LA_TRY(retention_map_f32(&jobs.o[np], o32, s));
+            jobs.o32[np] = 1;
+        } else {
+            LA_TRY(retention_map(&jobs.o[np], all[p].o, s, bf16));
+        }
         jobs.rev[np] = all[p].rev;
         jobs.sin[np] = all[p].sin;
         jobs.sin_t[np] = all[p].sin_t;

@@ -1351,6 +1351,26 @@ la_status retention_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf
     return make_tensor_map(m, ptr, s, bf16, 64);
 }
 
+// [BH, T, 64] fp32 tensor, boxes of 64 rows x 32 columns (128 bytes), 128-byte swizzle.
+la_status retention_map_f32(CUtensorMap *m, void *ptr, const Shape &s) {
+    EncodeFn enc = encode_fn();
+    if (!enc) {
+        set_error("cuTensorMapEncodeTiled is unavailable from the driver");
+        return LA_ERR_CUDA;
+    }
+    const cuuint64_t dims[3] = {(cuuint64_t)s.D, (cuuint64_t)s.T, (cuuint64_t)s.BH()};
+    const cuuint64_t strides[2] = {(cuuint64_t)s.D * 4, (cuuint64_t)s.T * s.D * 4};
+    const cuuint32_t box[3] = {32, 64, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return LA_ERR_CUDA;
+    }
+    return LA_OK;
+}
+
 namespace {
 
 static la_status tensor_map(CUtensorMap *m, const void *ptr, const Shape &s, bool bf16) {

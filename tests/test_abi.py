@@ -153,12 +153,19 @@ def test_causal_norm_validation(lib):
     assert fwd(D=32) == 2
     bad = (ctypes.c_float * 2)(0.5, 2.0)
     assert fwd(dec=ctypes.cast(bad, P)) == 1
-    need = lib.la_workspace_size(11, 1, 2, 16, 64, 1)
+    # CUDA-core path (bf16): (n, dn) per row, then the chunk states
+    need = lib.la_workspace_size(11, 1, 2, 16, 64, 2)
     assert need == 256            # 2 x 16 rows x 8 bytes, rounded up to 256
     # one chunk of 256 tokens needs no chunk states; 257 tokens make two chunks of [64][65] fp32 states
-    assert lib.la_workspace_size(10, 1, 2, 256, 64, 1) == 0
-    assert lib.la_workspace_size(10, 1, 2, 257, 64, 1) == 2 * 2 * 64 * 65 * 4
-    assert lib.la_workspace_size(11, 1, 2, 257, 64, 1) == 4352 + 2 * 2 * 64 * 65 * 4
+    assert lib.la_workspace_size(10, 1, 2, 256, 64, 2) == 0
+    assert lib.la_workspace_size(10, 1, 2, 257, 64, 2) == 2 * 2 * 64 * 65 * 4
+    assert lib.la_workspace_size(11, 1, 2, 257, 64, 2) == 4352 + 2 * 2 * 64 * 65 * 4
+    # tensor-core path (fp16, D = 64), each part rounded up to 256 bytes: f(q), f(k) for both;
+    # the backward adds du (16-bit), dn (fp32 per row), the per-chunk sums ([2 heads][1 chunk]
+    # [2][64] fp32) and dq, dk in fp32
+    t16, t32 = 2 * 16 * 64 * 2, 2 * 16 * 64 * 4
+    assert lib.la_workspace_size(10, 1, 2, 16, 64, 1) == 2 * t16
+    assert lib.la_workspace_size(11, 1, 2, 16, 64, 1) == 3 * t16 + 256 + 2 * 128 * 4 + 2 * t32
     assert fwd(T=257) == 4        # no workspace for two chunks
     assert fwd(T=257, ws=0x1080, ws_bytes=1 << 20) == 3     # not 256-byte aligned
     assert fwd(T=257, ws=0x1000, ws_bytes=100) == 4

@@ -1,7 +1,8 @@
 """GPU parity of causal linear attention with the norm term (la_causal_norm_*), through the C
 ABI, against the fp64 oracle: both feature maps, with and without a per-head decay, every
-dtype, D = 64 and 128, lengths of one chunk (256 tokens) and of several, whole or with ragged
-tails; sampled heads at the benchmark's size."""
+dtype, D = 64 and 128, lengths of one chunk and of several, whole or with ragged tails; sampled
+heads at the benchmark's size.  fp16 and bf16 at D = 64 run on the tensor cores, the rest on the
+CUDA cores."""
 import numpy as np
 import pytest
 import torch
@@ -40,7 +41,8 @@ def _run(inp, decay, feature, eps):
 
 
 @pytest.mark.parametrize("dtype,D,T", [("f16", 64, 300), ("bf16", 128, 300), ("f32", 64, 37), ("f32", 128, 130),
-                                       ("bf16", 64, 2), ("f16", 128, 517), ("f16", 64, 1024), ("bf16", 128, 512)])
+                                       ("bf16", 64, 2), ("f16", 128, 517), ("f16", 64, 1024), ("bf16", 128, 512),
+                                       ("bf16", 64, 700), ("f16", 64, 64), ("f16", 64, 3)])
 @pytest.mark.parametrize("feature", ["elu1", "identity"])
 @pytest.mark.parametrize("decayed", [False, True])
 def test_matches_oracle(dtype, D, T, feature, decayed):
