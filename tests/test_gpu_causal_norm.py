@@ -114,3 +114,19 @@ def test_empty_sequence_is_a_no_op():
     la.la_causal_norm_fwd(z, z, z, z)
     la.la_causal_norm_bwd(z, z, z, z, z, z, z)
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("T", [300, 1000])
+def test_strong_decays_fp16(T):
+    """fp16 at D = 64 with a decay below 0.9 takes the tensor-core kernel with two output
+    accumulators (the folded one needs gamma >= 0.9 in fp16): o and the gradients against the
+    oracle, both feature maps."""
+    for feature, eps in (("elu1", 1e-6), ("identity", 1e-3)):
+        inp = _inputs("f16", 2, 3, T, 64, seed=45, feature=feature)
+        decay = [0.5, 0.85, 0.95]
+        o, dq, dk, dv = _run(inp, decay, feature, eps)
+        want_o = oracle.causal_norm_fwd(inp["q"], inp["k"], inp["v"], decay, feature, eps)
+        want = oracle.causal_norm_bwd(inp["q"], inp["k"], inp["v"], inp["do"], decay, feature, eps)
+        pu.assert_fwd(o, want_o, "o " + feature, dtype=inp["q"].dtype)
+        for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
+            pu.assert_grad(got, ref, name + " " + feature)
