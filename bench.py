@@ -146,12 +146,16 @@ def measured_peaks():
 TC_SOURCES = {
     "state": ("la_tc.cuh", "la_tc_state.cu", "la_tc_common.cuh", "la_tc_ptx.cuh", "la_internal.cuh"),
     "retention": ("la_tc.cuh", "la_tc_retention.cu", "la_tc_common.cuh", "la_tc_ptx.cuh", "la_internal.cuh"),
+    "causal": ("la_tc.cuh", "la_tc_retention.cu", "la_tc_causal.cu", "la_tc_common.cuh", "la_tc_ptx.cuh",
+               "la_internal.cuh"),
 }
 
 
 def kernel_sources(kernel: str):
     """The source files of the tensor-core kernel launched under `kernel`."""
-    return TC_SOURCES["retention" if kernel.startswith("tc_retention") else "state"]
+    if kernel.startswith("tc_retention"):
+        return TC_SOURCES["retention"]
+    return TC_SOURCES["causal" if kernel.startswith("tc_causal_norm") else "state"]
 
 
 def source_hash(names=None) -> str:
@@ -168,10 +172,10 @@ def source_hash(names=None) -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str, T: int, B: int, H: int, D: int):
-    """DRAM bytes per launch of `kernel` at [B, H, T, D] from the committed ncu summaries: of the
-    captures taken on the current kernel sources at the same B, H and D, the one whose T is
-    nearest, scaled by T (None when no capture matches)."""
+def ncu_traffic(kernel: str, T: int, B: int, H: int, D: int, dtype: str):
+    """DRAM bytes per launch of `kernel` at [B, H, T, D] in `dtype` from the committed ncu
+    summaries: of the captures taken on the current kernel sources at the same B, H, D and dtype,
+    the one whose T is nearest, scaled by T (None when no capture matches)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
@@ -182,7 +186,8 @@ def ncu_traffic(kernel: str, T: int, B: int, H: int, D: int):
     if isinstance(entries, dict):
         entries = [entries]
     sha = source_hash(kernel_sources(kernel))
-    ok = [e for e in entries if e.get("source_sha") == sha and (e.get("B"), e.get("H"), e.get("D")) == (B, H, D)]
+    ok = [e for e in entries if e.get("source_sha") == sha and
+          (e.get("B"), e.get("H"), e.get("D"), e.get("dtype")) == (B, H, D, dtype)]
     if not ok:
         return None
     e = min(ok, key=lambda e: abs(math.log(float(e["T"]) / T)))
@@ -729,7 +734,7 @@ def run_ours(args, w):
             alg_bytes = KERNEL_TENSORS[name] * tensor_bytes
             avg_s = tot_ms / n_launch / 1e3
             achieved = alg_bytes / avg_s / 1e9
-            traffic = ncu_traffic(name, T, B, H, D)
+            traffic = ncu_traffic(name, T, B, H, D, w.dtype)
             roof = {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak, "peak_source": peak_kind, "traffic": traffic,
                     "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_ms": tot_ms / n_launch,
