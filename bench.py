@@ -158,9 +158,34 @@ def kernel_sources(kernel: str):
     return TC_SOURCES["causal" if kernel.startswith("tc_causal_norm") else "state"]
 
 
+def strip_comments(src: str) -> str:
+    """C/C++ source without its comments (// to the end of the line, /* ... */), string and
+    character literals kept, so that a change to comments alone leaves the hash alone."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
+
+
 def source_hash(names=None) -> str:
     """sha256 prefix of the library's kernel sources (every csrc file, or those in `names`) and
-    of include/la.h."""
+    of include/la.h, comments left out."""
     csrc = os.path.join(ROOT, "linear_attention_attn_b200", "csrc")
     paths = sorted(glob.glob(os.path.join(csrc, "*"))) if names is None else \
         sorted(os.path.join(csrc, n) for n in names)
@@ -168,7 +193,7 @@ def source_hash(names=None) -> str:
     for p in paths + [os.path.join(ROOT, "include", "la.h")]:
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode())
-            h.update(f.read())
+            h.update(strip_comments(f.read().decode("utf-8")).encode())
     return h.hexdigest()[:16]
 
 

@@ -170,7 +170,10 @@ la_status la_simple_bwd(const void *q, const void *k, const void *v, const void 
 
 /* Causal linear attention with per-head decay (retention), forward.
  *  decay    HOST pointer to H floats, gamma_h in (0, 1]; read during the call.
- *  o        out: o_t = sum_{s<=t} gamma_h^(t-s) (q_t . k_s) v_s               */
+ *  o        out: o_t = sum_{s<=t} gamma_h^(t-s) (q_t . k_s) v_s
+ * fp16 and bf16 run on the tensor cores (chunks of 64 rows, one CTA per (b, h)
+ * carrying the state from chunk to chunk), D = 64 and 128; fp32 on CUDA cores.
+ * With gamma_h = 1 for every head this is plain causal linear attention.      */
 la_status la_chunk_decay_fwd(const void *q, const void *k, const void *v, void *o,
                              const float *decay,
                              int B, int H, int T, int D, la_dtype dtype,
