@@ -27,3 +27,12 @@ def test_every_capture_names_a_kernel_family():
         assert bench.kernel_sources(kernel)
         for e in entries:
             assert {"source_sha", "T", "B", "H", "D", "dtype", "dram_bytes_per_launch"} <= set(e)
+
+
+def test_causal_workload_keeps_its_unit_decay_through_resizing():
+    import synth
+    w = synth.WORKLOADS["causal_bf16"].with_T(130)
+    inp = synth.make_inputs(w, seed=1)
+    assert w.extra == {"gamma": 1.0}
+    assert inp["gamma"].tolist() == [1.0] * w.H
+    assert tuple(inp["q"].shape) == (w.B, w.H, 130, 64)
