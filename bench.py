@@ -353,6 +353,12 @@ def host_cores() -> int:
         return os.cpu_count() or 1
 
 
+def metric_of(w) -> str:
+    """The line's metric: the specification's for the bidirectional workload, else the op's own
+    fwd+bwd tokens/s (the same on both arms)."""
+    return METRIC if w.op == "bidir" else "%s fwd+bwd tokens/s" % ("causal" if w.name == "causal_bf16" else w.op)
+
+
 def run_reference(args, w):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -369,7 +375,7 @@ def run_reference(args, w):
         secs += dt
     value = statistics.median(rates)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric_of(w), "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(w, args),
@@ -815,7 +821,7 @@ def run_ours(args, w):
         vs = value / page_rate
 
     line = {
-        "metric": METRIC if w.op == "bidir" else "%s fwd+bwd tokens/s" % ("causal" if w.name == "causal_bf16" else w.op),
+        "metric": metric_of(w),
         "value": value, "unit": UNIT,
         "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
