@@ -395,6 +395,11 @@ WORKLOAD_TEXT = {
               "q,k ~ N(0,1) D^-1/2, v, dO ~ N(0,1)",
     "retention": "chunked causal decay (retention) fwd+bwd, bf16 storage / fp32 accumulate, B=%d H=%d T=%d D=%d, "
                  "gamma_h = 1 - 2^(-5-7h/(H-1)), q ~ N(0,1) D^-1/2, k, v, dO ~ N(0,1)",
+    "bidir_d128": "bidirectional linear attention fwd+bwd on the CUDA-core kernels (no tensor-core kernel at D=128), "
+                  "fp16 storage / fp32 accumulate, B=%d H=%d T=%d D=%d, phi=elu+1, eps=1e-06, Q,K,V ~ 0.5 N(0,1), "
+                  "dO ~ N(0,1)",
+    "simple_d128": "simple_la fwd+bwd on the CUDA-core kernels (no tensor-core kernel at D=128), bf16 storage / fp32 "
+                   "accumulate, B=%d H=%d T=%d D=%d, q,k ~ N(0,1) D^-1/2, v, dO ~ N(0,1)",
     "causal": "plain causal linear attention fwd+bwd (the decay op with gamma = 1 on every head: no feature map, "
               "no norm term), bf16 storage / fp32 accumulate, B=%d H=%d T=%d D=%d, q ~ N(0,1) D^-1/2, k, v, dO ~ N(0,1)",
     "gated": "gated linear attention fwd+bwd (recurrent form in 256-token chunks on CUDA cores), bf16 storage / "
@@ -481,7 +486,9 @@ CONFIG_RECORDS = (("simple_bf16", (128, 1024, 4096, 16384), False),
                   ("causal_bf16", (4096,), False),
                   ("vision_f16", (65536,), True),
                   ("causal_norm_f16", (4096,), False),
-                  ("gated_bf16", (4096,), False))
+                  ("gated_bf16", (4096,), False),
+                  ("bidir_f16_d128", (4096,), False),
+                  ("simple_bf16_d128", (4096,), False))
 
 
 def config_records(la, dev, stream):
@@ -555,7 +562,8 @@ def config_records(la, dev, stream):
             recs.append(rec)
             del q, k, v, g, o, dq, dk, dv, st, ws, lg, dg
             torch.cuda.empty_cache()
-        kind = {"vision_f16": "vision", "causal_bf16": "causal"}.get(base, synth.WORKLOADS[base].op)
+        kind = {"vision_f16": "vision", "causal_bf16": "causal", "bidir_f16_d128": "bidir_d128",
+                "simple_bf16_d128": "simple_d128"}.get(base, synth.WORKLOADS[base].op)
         out[base] = {"workload": WORKLOAD_TEXT[kind]
                      % (synth.WORKLOADS[base].B, synth.WORKLOADS[base].H, Ts[-1], synth.WORKLOADS[base].D),
                      "step": "fwd" if fwd_only else "fwd+bwd", "peak_gbs": peak, "peak_source": peak_kind,

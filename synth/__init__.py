@@ -72,6 +72,11 @@ WORKLOADS = {
     # gated linear attention, bf16: q scaled by D^-1/2, log gates log(sigmoid(N(0,1))) / 16 per token
     # and key dimension (about -0.04: decays near 0.96)
     "gated_bf16": Workload("gated_bf16", "gated", 8, 16, 4096, 64, "bf16", q_scale=64 ** -0.5),
+    # the bidirectional and simple_la recipes at D = 128 (the head size the CUDA-core kernels cover)
+    "bidir_f16_d128": Workload("bidir_f16_d128", "bidir", 8, 16, 4096, 128, "f16",
+                               q_scale=0.5, k_scale=0.5, v_scale=0.5),
+    "simple_bf16_d128": Workload("simple_bf16_d128", "simple", 8, 16, 4096, 128, "bf16",
+                                 q_scale=128 ** -0.5, k_scale=128 ** -0.5),
     # vision-style long sequence, forward only, 256x256 token grid
     "vision_f16": Workload("vision_f16", "bidir", 2, 10, 65536, 64, "f16",
                            q_scale=0.5, k_scale=0.5, v_scale=0.5, vision_offset=True, bwd=False),
